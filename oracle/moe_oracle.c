@@ -1,0 +1,385 @@
+/*
+ * moe_oracle.c -- plain, slow, obviously-correct CPU oracle of the Step-3.5-Flash
+ * routed-expert MoE FFN layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls this
+ * file: only the test suite, the package's smoke check and the benchmark's CPU-baseline
+ * leg use it.  It shares no code, header, table or constant generator with the CUDA
+ * library; both sides read the same seeded inputs and nothing else.
+ *
+ * What the layer computes (sources, all on the llm-atlas page "Step-3.5-Flash",
+ * table "Champs bruts du config.json" unless noted):
+ *   - moe_num_experts = 288, moe_top_k = 8: every token is routed to 8 of 288 experts;
+ *   - norm_expert_weight = true: the weights of the chosen experts are renormalised so
+ *     that they sum to 1;
+ *   - need_fp32_gate = true: router scores are fp32 values;
+ *   - moe_intermediate_size = 1280, share_expert_dim = 1280: the routed experts and the
+ *     always-on shared expert are gated FFNs of width 1280 on hidden size 4096;
+ *   - the same page's "FFN / MoE" paragraph: a sparse mixture of 288 routed experts with
+ *     top-8 routing.
+ * The pages leave the score function and the activation open; this oracle takes a
+ * softmax router, ties broken toward the lower expert index, and SiLU(gate)*up.
+ *
+ * Precision:
+ *   - router score s[t,e] = the EXACT real value of sum_h x[t,h]*W_r[e,h], rounded
+ *     once to fp32, nearest-even (every product of two bf16 or two fp32 numbers is an
+ *     exact dyadic rational; they are summed without error in integer bins);
+ *   - key[t,e] = fp32(s[t,e] + b[e]) when a router bias is given, else s[t,e];
+ *   - selection by (key descending, expert index ascending), stored by ascending index;
+ *   - routing weights: softmax over the selected keys, in fp64;
+ *   - expert FFNs and the combine: fp64, sequential accumulation.
+ *
+ * Parity status: every function here is pinned by tests (exact rational sums,
+ * brute-force subset enumeration, closed forms and invariants); none is unpinned.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define OR_F32 0
+#define OR_BF16 1
+
+/* ------------------------------------------------------------------------------------
+ * Exact dot product.
+ *
+ * Every finite bf16 or fp32 value v is m * 2^q with an integer m (|m| < 2^24) and an
+ * integer q.  A product of two such values is (m1*m2) * 2^(q1+q2), exact.  We add each
+ * product's integer mantissa into a bin indexed by its exponent (int64 bins; a bf16
+ * product has |m1*m2| < 2^16, an fp32 product is split into two 24-bit halves), then
+ * turn the bins into one big binary integer by carry propagation and round it once to
+ * the nearest fp32 (ties to even), with subnormal results handled.
+ * ---------------------------------------------------------------------------------- */
+
+/* smallest product exponent: fp32 subnormal * subnormal = 2^-149 * 2^-149 */
+#define BIN_EMIN (-298)
+/* largest exponent a bin can receive: bf16 max 2^120*2^120 = 2^240, fp32 hi half 2^232 */
+#define BIN_EMAX 241
+#define NBINS (BIN_EMAX - BIN_EMIN + 1)
+/* room for the carries of up to 2^62 in magnitude above the top bin */
+#define NBITS (NBINS + 72)
+
+typedef struct {
+  int32_t m; /* signed integer mantissa */
+  int32_t q; /* exponent: value = m * 2^q */
+  int finite;
+} dyadic;
+
+static dyadic decode_f32(uint32_t bits) {
+  dyadic d;
+  uint32_t sign = bits >> 31, ex = (bits >> 23) & 0xFF, fr = bits & 0x7FFFFF;
+  d.finite = (ex != 0xFF);
+  if (ex == 0) {
+    d.m = (int32_t)fr;
+    d.q = -149;
+  } else {
+    d.m = (int32_t)(fr | 0x800000u);
+    d.q = (int32_t)ex - 150;
+  }
+  if (sign) d.m = -d.m;
+  return d;
+}
+
+static dyadic decode_bf16(uint16_t bits) {
+  dyadic d;
+  uint32_t sign = bits >> 15, ex = (bits >> 7) & 0xFF, fr = bits & 0x7F;
+  d.finite = (ex != 0xFF);
+  if (ex == 0) {
+    d.m = (int32_t)fr;
+    d.q = -133;
+  } else {
+    d.m = (int32_t)(fr | 0x80u);
+    d.q = (int32_t)ex - 134;
+  }
+  if (sign) d.m = -d.m;
+  return d;
+}
+
+/* Round the integer  sum_b bins[b] * 2^(b + BIN_EMIN)  to the nearest fp32. */
+static float round_bins_to_f32(const int64_t* bins) {
+  /* 1. two's-complement bit string of the sum by carry propagation (floor division) */
+  static __thread uint8_t bit[NBITS];
+  int64_t carry = 0;
+  int nb = 0;
+  for (int b = 0; b < NBINS; ++b) {
+    /* v = bins[b] + carry may overflow only if |bins| ~ 2^63: excluded by the
+       caller's length limit */
+    int64_t v = bins[b] + carry;
+    bit[nb++] = (uint8_t)(v & 1);
+    carry = (v - (v & 1)) / 2; /* exact floor(v/2) */
+  }
+  while (carry != 0 && carry != -1) {
+    bit[nb++] = (uint8_t)(carry & 1);
+    carry = (carry - (carry & 1)) / 2;
+  }
+  int negative = (carry == -1);
+  if (negative) { /* magnitude = two's complement of the bit string */
+    int c = 1;
+    for (int i = 0; i < nb; ++i) {
+      int v = (bit[i] ^ 1) + c;
+      bit[i] = (uint8_t)(v & 1);
+      c = v >> 1;
+    }
+    /* c == 1 here would mean the magnitude is 2^nb: append it */
+    if (c) bit[nb++] = 1;
+  }
+  /* 2. highest set bit */
+  int top = -1;
+  for (int i = nb - 1; i >= 0; --i)
+    if (bit[i]) { top = i; break; }
+  if (top < 0) return negative ? -0.0f : 0.0f; /* exact zero: +0 (carry 0) */
+  int e_top = top + BIN_EMIN; /* value of the top bit is 2^e_top */
+  /* 3. position of the last kept bit: 24 significant bits for normals, 2^-149 floor */
+  int keep_lsb_exp = e_top - 23;
+  if (keep_lsb_exp < -149) keep_lsb_exp = -149;
+  int lsb = keep_lsb_exp - BIN_EMIN; /* bit index of the last kept bit (>= 0) */
+  uint64_t mant = 0;
+  for (int i = top; i >= lsb; --i) mant = (mant << 1) | bit[i];
+  int round_bit = (lsb - 1 >= 0) ? bit[lsb - 1] : 0;
+  int sticky = 0;
+  for (int i = lsb - 2; i >= 0; --i)
+    if (bit[i]) { sticky = 1; break; }
+  if (round_bit && (sticky || (mant & 1))) mant += 1;
+  /* mant * 2^keep_lsb_exp is exact in fp32 unless it overflows the range */
+  double v = ldexp((double)mant, keep_lsb_exp);
+  if (v > 3.4028234663852886e38) v = INFINITY; /* beyond FLT_MAX after rounding */
+  float f = (float)v; /* exact: mant has <= 25 bits and the exponent is in range */
+  return negative ? -f : f;
+}
+
+/* Exact sum_h x[h]*w[h] rounded once to fp32.  Returns 0 on success, -1 on a
+   non-finite input, -2 if the length could overflow a bin. */
+static int exact_dot_f32(int dtype, int n, const void* x, const void* w, float* out) {
+  int64_t bins[NBINS];
+  memset(bins, 0, sizeof(bins));
+  if (n > (1 << 30)) return -2;
+  for (int h = 0; h < n; ++h) {
+    dyadic a, b;
+    if (dtype == OR_BF16) {
+      a = decode_bf16(((const uint16_t*)x)[h]);
+      b = decode_bf16(((const uint16_t*)w)[h]);
+    } else {
+      a = decode_f32(((const uint32_t*)x)[h]);
+      b = decode_f32(((const uint32_t*)w)[h]);
+    }
+    if (!a.finite || !b.finite) return -1;
+    if (a.m == 0 || b.m == 0) continue;
+    int64_t p = (int64_t)a.m * (int64_t)b.m; /* |p| < 2^48 */
+    int q = a.q + b.q;
+    int64_t mag = p < 0 ? -p : p;
+    int64_t sgn = p < 0 ? -1 : 1;
+    int64_t lo = mag & 0xFFFFFF, hi = mag >> 24; /* both < 2^24 */
+    bins[q - BIN_EMIN] += sgn * lo;
+    if (hi) bins[q + 24 - BIN_EMIN] += sgn * hi;
+  }
+  *out = round_bins_to_f32(bins);
+  return 0;
+}
+
+/* Exposed for the tests that pin the exact dot product on its own. */
+int oracle_exact_dot(int dtype, int n, const void* x, const void* w, float* out) {
+  return exact_dot_f32(dtype, n, x, w, out);
+}
+
+static size_t esize(int dtype) { return dtype == OR_BF16 ? 2 : 4; }
+
+static double to_f64(int dtype, const void* base, size_t i) {
+  if (dtype == OR_BF16) {
+    uint32_t b = (uint32_t)((const uint16_t*)base)[i] << 16;
+    float f;
+    memcpy(&f, &b, 4);
+    return (double)f;
+  }
+  return (double)((const float*)base)[i];
+}
+
+/* ------------------------------------------------------------------------------------
+ * Router scores: s[t,e] = RN32(exact sum_h x[t,h] W_r[e,h]) for every token and expert
+ * (router logits; fp32 scores per need_fp32_gate).
+ * ---------------------------------------------------------------------------------- */
+int oracle_router_scores(int dtype, int64_t T, int H, int E, const void* x, const void* Wr,
+                         float* s_out, int nthreads) {
+  int err = 0;
+  size_t es = esize(dtype);
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel for schedule(dynamic, 16) reduction(| : err)
+  for (int64_t te = 0; te < T * (int64_t)E; ++te) {
+    int64_t t = te / E;
+    int e = (int)(te % E);
+    const char* xr = (const char*)x + (size_t)t * H * es;
+    const char* wr = (const char*)Wr + (size_t)e * H * es;
+    float s;
+    if (exact_dot_f32(dtype, H, xr, wr, &s) != 0) err |= 1;
+    s_out[te] = s;
+  }
+  return err ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------------------
+ * Routing of one token (softmax router, top-k, renormalised weights).
+ *   key[e] = fp32(s[e] + b[e])   (b = 0 when no bias is given)
+ *   S = the k experts first in the order (key descending, index ascending)
+ *   stored by ascending expert index;
+ *   w_j = exp(key_j - m) / sum_{i in S} exp(key_i - m), m = max_{i in S} key_i, fp64.
+ * The full-softmax denominator over all E experts cancels under the renormalisation
+ * that norm_expert_weight asks for, so it is never formed.
+ * ---------------------------------------------------------------------------------- */
+static int beats(float ka, int a, float kb, int b) { /* a is ordered before b */
+  return (ka > kb) || (ka == kb && a < b);
+}
+
+int oracle_route(int64_t T, int E, int k, const float* s, const float* bias, int32_t* idx_out,
+                 float* w_out, double* w64_out) {
+  if (k < 1 || k > E) return -1;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    float* key = (float*)malloc(sizeof(float) * E);
+    int* chosen = (int*)calloc(E, sizeof(int));
+    for (int e = 0; e < E; ++e) {
+      float v = s[t * E + e];
+      key[e] = bias ? (float)(v + bias[e]) : v; /* fp32 + fp32 -> RN fp32 */
+    }
+    /* k passes of "pick the best not yet chosen" */
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      for (int e = 0; e < E; ++e) {
+        if (chosen[e]) continue;
+        if (best < 0 || beats(key[e], e, key[best], best)) best = e;
+      }
+      chosen[best] = 1;
+    }
+    /* ascending expert index */
+    int j = 0;
+    double m = -INFINITY;
+    for (int e = 0; e < E; ++e)
+      if (chosen[e]) {
+        idx_out[t * k + j++] = e;
+        if ((double)key[e] > m) m = (double)key[e];
+      }
+    double z = 0.0;
+    for (j = 0; j < k; ++j) z += exp((double)key[idx_out[t * k + j]] - m);
+    for (j = 0; j < k; ++j) {
+      double w = exp((double)key[idx_out[t * k + j]] - m) / z;
+      if (w64_out) w64_out[t * k + j] = w;
+      if (w_out) w_out[t * k + j] = (float)w;
+    }
+    free(key);
+    free(chosen);
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------------------
+ * Dispatch bookkeeping by plain counting:
+ *   counts[e]  = number of (token, slot) assignments routed to e;
+ *   offsets[0] = 0, offsets[e+1] = offsets[e] + counts[e];
+ *   perm[offsets[e] + r] = t*k + j for the r-th token (ascending t) routed to e;
+ *   inv_perm[t*k + j]    = position of that assignment in perm.
+ * ---------------------------------------------------------------------------------- */
+int oracle_dispatch(int64_t T, int E, int k, const int32_t* idx, int32_t* counts,
+                    int32_t* offsets, int32_t* perm, int32_t* inv_perm) {
+  for (int e = 0; e < E; ++e) counts[e] = 0;
+  for (int64_t a = 0; a < T * k; ++a) {
+    int e = idx[a];
+    if (e < 0 || e >= E) return -1;
+    counts[e]++;
+  }
+  offsets[0] = 0;
+  for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+  int32_t* fill = (int32_t*)calloc(E, sizeof(int32_t));
+  for (int64_t t = 0; t < T; ++t)  /* token order makes the pass stable */
+    for (int j = 0; j < k; ++j) {
+      int e = idx[t * k + j];
+      int32_t pos = offsets[e] + fill[e]++;
+      perm[pos] = (int32_t)(t * k + j);
+      if (inv_perm) inv_perm[t * k + j] = pos;
+    }
+  free(fill);
+  return 0;
+}
+
+/* ------------------------------------------------------------------------------------
+ * One gated FFN on one token, fp64:
+ *   g_i = sum_h x_h Wgu[i, h],  u_i = sum_h x_h Wgu[I + i, h]     (gate rows, then up rows)
+ *   a_i = SiLU(g_i) * u_i,      SiLU(z) = z / (1 + exp(-z))
+ *   out_h += scale * sum_i a_i Wd[h, i]
+ * ---------------------------------------------------------------------------------- */
+static void gated_ffn_acc(int dtype, int H, int I, const void* xrow, const void* Wgu,
+                          const void* Wd, double scale, double* out, double* a /*[I]*/) {
+  for (int i = 0; i < I; ++i) {
+    double g = 0.0, u = 0.0;
+    for (int h = 0; h < H; ++h) {
+      double xv = to_f64(dtype, xrow, h);
+      g += xv * to_f64(dtype, Wgu, (size_t)i * H + h);
+      u += xv * to_f64(dtype, Wgu, (size_t)(I + i) * H + h);
+    }
+    a[i] = g / (1.0 + exp(-g)) * u;
+  }
+  for (int h = 0; h < H; ++h) {
+    double o = 0.0;
+    for (int i = 0; i < I; ++i) o += a[i] * to_f64(dtype, Wd, (size_t)h * I + i);
+    out[h] += scale * o;
+  }
+}
+
+/* The intermediate activation of one token through one expert (exposed so that the
+   tests can pin the gate/up/SiLU step on its own). */
+int oracle_expert_act(int dtype, int H, int I, const void* xrow, const void* Wgu_e,
+                      double* act_out) {
+  for (int i = 0; i < I; ++i) {
+    double g = 0.0, u = 0.0;
+    for (int h = 0; h < H; ++h) {
+      double xv = to_f64(dtype, xrow, h);
+      g += xv * to_f64(dtype, Wgu_e, (size_t)i * H + h);
+      u += xv * to_f64(dtype, Wgu_e, (size_t)(I + i) * H + h);
+    }
+    act_out[i] = g / (1.0 + exp(-g)) * u;
+  }
+  return 0;
+}
+
+/* ------------------------------------------------------------------------------------
+ * Layer output for a list of tokens, given their routing:
+ *   y_t = sum_j w[t,j] * FFN_{idx[t,j]}(x_t) + FFN_shared(x_t)      (fp64)
+ * The shared expert (share_expert_dim) is always on with weight 1; pass NULL shared
+ * weights for a layer without one.  Weight layouts: Wgu [E, 2I, H], Wd [E, H, I],
+ * Wsgu [2Is, H], Wsd [H, Is].  tok[n] is the token whose output goes to y[n, :];
+ * idx/w are indexed by token.
+ * ---------------------------------------------------------------------------------- */
+int oracle_moe_tokens(int dtype, int64_t ntok, const int64_t* tok, int H, int E, int k, int I,
+                      int Is, const void* x, const int32_t* idx, const double* w,
+                      const void* Wgu, const void* Wd, const void* Wsgu, const void* Wsd,
+                      double* y, int nthreads) {
+  size_t es = esize(dtype);
+  int bad = 0;
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t n = 0; n < ntok; ++n) {
+    int64_t t = tok[n];
+    const char* xr = (const char*)x + (size_t)t * H * es;
+    double* out = y + (size_t)n * H;
+    int Imax = I > Is ? I : Is;
+    double* a = (double*)malloc(sizeof(double) * (Imax > 0 ? Imax : 1));
+    for (int h = 0; h < H; ++h) out[h] = 0.0;
+    for (int j = 0; j < k; ++j) {
+      int e = idx[t * k + j];
+      if (e < 0 || e >= E) {
+        bad |= 1;
+        continue;
+      }
+      const char* gu = (const char*)Wgu + (size_t)e * 2 * I * H * es;
+      const char* d = (const char*)Wd + (size_t)e * H * I * es;
+      gated_ffn_acc(dtype, H, I, xr, gu, d, w[t * k + j], out, a);
+    }
+    if (Wsgu && Wsd && Is > 0) gated_ffn_acc(dtype, H, Is, xr, Wsgu, Wsd, 1.0, out, a);
+    free(a);
+  }
+  return bad ? -1 : 0;
+}

@@ -1,0 +1,393 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix (CPU only).
+
+Each test checks the oracle against something other than itself: exact rational
+arithmetic, brute-force enumeration, closed forms, special cases that reduce to a library
+routine, or invariants that the definition implies.
+"""
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import to_oracle
+from sparse_mixture_experts_ffn_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# --------------------------------------------------------------------------------------
+# exact rational helpers (independent of the oracle's integer-bin algorithm)
+# --------------------------------------------------------------------------------------
+def frac_to_f32(q: Fraction) -> np.float32:
+    """Round a rational to the nearest fp32, ties to even, subnormals included."""
+    if q == 0:
+        return np.float32(0.0)
+    neg = q < 0
+    q = abs(q)
+    e = q.numerator.bit_length() - q.denominator.bit_length()
+    while Fraction(2) ** e > q:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= q:
+        e += 1
+    lsb = max(e - 23, -149)
+    scaled = q / Fraction(2) ** lsb
+    n = scaled.numerator // scaled.denominator
+    rem = scaled - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    v = math.ldexp(n, lsb)
+    if v > float(np.finfo(np.float32).max):
+        v = math.inf
+    f = np.float32(v)
+    return -f if neg else f
+
+
+def exact_value(bits_or_f32) -> Fraction:
+    a = np.asarray(bits_or_f32)
+    if a.dtype == np.uint16:
+        f = (a.astype(np.uint32) << 16).view(np.float32)
+    else:
+        f = a.astype(np.float32)
+    return Fraction(float(f))
+
+
+def bf16_bits(values) -> np.ndarray:
+    t = torch.tensor(np.asarray(values, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def brute_dot(x, w) -> np.float32:
+    return frac_to_f32(sum((exact_value(a) * exact_value(b) for a, b in zip(x, w)), Fraction(0)))
+
+
+def random_wide_vector(rng, n, dtype):
+    """Values spanning many binades, with subnormals of the dtype and some cancellation."""
+    mant = rng.standard_normal(n)
+    lo = -140 if dtype == "bf16" else -155
+    expo = rng.integers(lo, 60, size=n)
+    v = np.ldexp(mant, expo)
+    if n >= 4:  # exact cancelling pairs
+        v[: n // 4] = -v[n // 4: 2 * (n // 4)]
+    if dtype == "bf16":
+        return bf16_bits(v.astype(np.float32))
+    return v.astype(np.float32)
+
+
+# --------------------------------------------------------------------------------------
+# exact router dot product
+# --------------------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_exact_dot_matches_rational_sum(dtype):
+    rng = np.random.default_rng(1234)
+    for trial in range(300):
+        n = int(rng.integers(1, 80))
+        x = random_wide_vector(rng, n, dtype)
+        w = random_wide_vector(rng, n, dtype)
+        got = oracle.exact_dot(x, w)
+        want = brute_dot(x, w)
+        assert got.tobytes() == want.tobytes() or (got == 0 and want == 0), (trial, got, want)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_exact_dot_router_like_vectors(dtype):
+    rng = np.random.default_rng(99)
+    for _ in range(20):
+        xv = rng.standard_normal(512).astype(np.float32)
+        wv = (rng.standard_normal(512) * 0.02).astype(np.float32)
+        x = bf16_bits(xv) if dtype == "bf16" else xv
+        w = bf16_bits(wv) if dtype == "bf16" else wv
+        assert oracle.exact_dot(x, w).tobytes() == brute_dot(x, w).tobytes()
+
+
+def test_exact_dot_rounding_cases():
+    one = np.float32(1.0)
+    ones = np.ones(3, np.float32)
+    # 1 + 2^-24 is the midpoint between 1 and 1+2^-23: ties to even -> 1
+    assert oracle.exact_dot(np.array([1.0, 2.0 ** -24], np.float32), ones[:2]) == one
+    # 1 + 3*2^-24 lies between 1+2^-23 and 1+2^-22 at their midpoint -> even is 1+2^-22
+    assert oracle.exact_dot(np.array([1.0, 3 * 2.0 ** -24], np.float32), ones[:2]) == np.float32(1 + 2 ** -22)
+    # a sticky bit far below breaks the tie upward
+    got = oracle.exact_dot(np.array([1.0, 2.0 ** -24, 2.0 ** -60], np.float32), ones)
+    assert got == np.float32(1 + 2 ** -23)
+    # a sequential fp32 sum would lose the small terms; the exact sum keeps them
+    v = np.array([2.0 ** 24, 1.0, 1.0], np.float32)
+    assert oracle.exact_dot(v, ones) == np.float32(2 ** 24 + 2)
+    # exact cancellation gives +0
+    z = oracle.exact_dot(np.array([3.0, -3.0], np.float32), np.ones(2, np.float32))
+    assert z == 0 and not np.signbit(z)
+    # subnormal results: 2^-140 * 2^-10 = 2^-150 is half the smallest subnormal -> ties to 0
+    tiny = np.array([2.0 ** -140], np.float32)
+    assert oracle.exact_dot(tiny, np.array([2.0 ** -10], np.float32)) == 0
+    # 3 * 2^-150 = 1.5 * 2^-149 -> ties to even -> 2 * 2^-149
+    assert oracle.exact_dot(tiny, np.array([3 * 2.0 ** -10], np.float32)) == np.float32(2 * 2.0 ** -149)
+    # bf16 products are exact: (1+2^-7)^2 = 1 + 2^-6 + 2^-14, representable in fp32
+    b = bf16_bits([1 + 2 ** -7])
+    assert oracle.exact_dot(b, b) == np.float32(1 + 2 ** -6 + 2 ** -14)
+
+
+def test_router_scores_are_exact_dots():
+    rng = np.random.default_rng(5)
+    x = bf16_bits(rng.standard_normal((3, 40)))
+    Wr = bf16_bits(rng.standard_normal((5, 40)) * 0.02)
+    s = oracle.router_scores(x, Wr)
+    for t in range(3):
+        for e in range(5):
+            assert s[t, e].tobytes() == brute_dot(x[t], Wr[e]).tobytes()
+
+
+# --------------------------------------------------------------------------------------
+# top-k selection and renormalised softmax
+# --------------------------------------------------------------------------------------
+def brute_force_set(key, k, bias=None):
+    E = len(key)
+    kk = [np.float32(key[e] + bias[e]) if bias is not None else np.float32(key[e]) for e in range(E)]
+    found = []
+    for S in itertools.combinations(range(E), k):
+        Sset = set(S)
+        ok = all(kk[a] > kk[b] or (kk[a] == kk[b] and a < b)
+                 for a in S for b in range(E) if b not in Sset)
+        if ok:
+            found.append(S)
+    assert len(found) == 1  # the order (key desc, index asc) is total
+    return list(found[0])
+
+
+@pytest.mark.parametrize("E", [2, 3, 5, 8])
+def test_selection_brute_force_with_ties(E):
+    rng = np.random.default_rng(E)
+    T = 60
+    # few distinct values so that ties are frequent
+    levels = rng.standard_normal(3).astype(np.float32)
+    s = levels[rng.integers(0, 3, size=(T, E))]
+    bias = rng.choice(np.array([0.0, 0.5, -0.25], np.float32), size=E)
+    for k in range(1, E + 1):
+        for b in (None, bias):
+            idx, w, w64 = oracle.route(s, k, b)
+            for t in range(T):
+                assert list(idx[t]) == brute_force_set(s[t], k, b)
+                assert np.all(np.diff(idx[t]) > 0)
+
+
+def test_selection_prefers_lower_index_on_equal_keys():
+    s = np.zeros((1, 6), np.float32)
+    idx, w, _ = oracle.route(s, 3)
+    assert list(idx[0]) == [0, 1, 2]
+    assert np.allclose(w, 1 / 3, rtol=0, atol=1e-7)
+
+
+def test_weights_sum_to_one_and_k1():
+    rng = np.random.default_rng(3)
+    s = (rng.standard_normal((200, 288)) * 1.28).astype(np.float32)
+    idx, w, w64 = oracle.route(s, 8)
+    assert np.all(np.abs(w.astype(np.float64).sum(1) - 1) <= 8 * 2.0 ** -23)
+    assert np.all(np.abs(w64.sum(1) - 1) <= 1e-14)
+    # the selected experts are the 8 largest scores (no ties in continuous data)
+    ref = np.sort(np.argsort(-s, axis=1, kind="stable")[:, :8], axis=1)
+    assert np.array_equal(idx, ref)
+    idx1, w1, _ = oracle.route(s, 1)
+    assert np.all(w1 == 1.0)
+    assert np.array_equal(idx1[:, 0], np.argmax(s, axis=1))
+
+
+def test_softmax_closed_form():
+    # keys 0 and ln 3: renormalised weights 1/4 and 3/4; higher key gets more weight
+    ln3 = np.float32(math.log(3.0))
+    s = np.array([[0.0, ln3, -5.0]], np.float32)
+    idx, w, w64 = oracle.route(s, 2)
+    assert list(idx[0]) == [0, 1]
+    assert abs(w64[0, 0] - 0.25) < 1e-7 and abs(w64[0, 1] - 0.75) < 1e-7
+    # the third expert's key cancels out of the renormalised weights
+    s2 = np.array([[0.0, ln3, 4.0]], np.float32)
+    idx2, _, w2 = oracle.route(s2, 2)
+    assert list(idx2[0]) == [1, 2]
+    assert abs(w2[0, 0] - 1 / (1 + math.exp(4.0 - float(ln3)))) < 1e-12
+
+
+def test_bias_shifts_selection():
+    s = np.zeros((1, 4), np.float32)
+    bias = np.array([0.0, 0.0, 1.0, 0.5], np.float32)
+    idx, w, w64 = oracle.route(s, 2, bias)
+    assert list(idx[0]) == [2, 3]
+    assert abs(w64[0, 1] / w64[0, 0] - math.exp(-0.5)) < 1e-12
+
+
+# --------------------------------------------------------------------------------------
+# dispatch bookkeeping
+# --------------------------------------------------------------------------------------
+def test_dispatch_against_library_sort():
+    rng = np.random.default_rng(8)
+    T, E, k = 97, 12, 3
+    idx = np.stack([np.sort(rng.choice(E, size=k, replace=False)) for _ in range(T)]).astype(np.int32)
+    counts, offsets, perm, inv = oracle.dispatch(idx, E)
+    assert np.array_equal(counts, np.bincount(idx.ravel(), minlength=E))
+    assert offsets[0] == 0 and np.array_equal(offsets[1:], np.cumsum(counts))
+    order = sorted(range(T * k), key=lambda a: (idx.ravel()[a], a // k))
+    assert list(perm) == order
+    assert np.array_equal(inv[perm], np.arange(T * k))
+
+
+# --------------------------------------------------------------------------------------
+# expert FFNs and the combine
+# --------------------------------------------------------------------------------------
+def silu(z):
+    return z / (1.0 + np.exp(-z))
+
+
+def test_silu_gate_up_closed_form():
+    ln3 = np.float32(math.log(3.0))
+    x = np.array([1.0], np.float32)
+    for g, want_silu in ((ln3, 0.75 * float(ln3)), (-ln3, -0.25 * float(ln3)), (np.float32(0), 0.0)):
+        Wgu = np.array([[g], [2.0]], np.float32)  # gate row, then up row
+        act = oracle.expert_act(x, Wgu)
+        assert abs(act[0] - 2.0 * want_silu) < 1e-7
+    # gate and up are not interchangeable: SiLU(2)*ln3 != SiLU(ln3)*2
+    act = oracle.expert_act(x, np.array([[2.0], [ln3]], np.float32))
+    assert abs(act[0] - 2.0 / (1 + math.exp(-2.0)) * float(ln3)) < 1e-7
+    assert abs(act[0] - 1.5 * float(ln3)) > 0.1
+
+
+def _numpy_ffn(x, Wgu, Wd):
+    """Dense gated FFN with numpy fp64 matmuls (a library routine, not the oracle)."""
+    I = Wgu.shape[0] // 2
+    g = x @ Wgu[:I].T
+    u = x @ Wgu[I:].T
+    return (silu(g) * u) @ Wd.T
+
+
+def _f64(t):
+    return t.to(torch.float64).numpy()
+
+
+def _small(dtype="f32", **kw):
+    base = dict(T=24, H=64, E=6, top_k=2, I=32, I_shared=32, r_std=0.1, rms_norm=False)
+    base.update(kw)
+    return inputs.small_config(dtype=dtype, **base)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_identical_experts_reduce_to_one_dense_ffn(dtype):
+    cfg = _small(dtype)
+    d = inputs.make_inputs(cfg)
+    Wgu = d["W_gate_up"][:1].expand(cfg.E, -1, -1).contiguous()
+    Wd = d["W_down"][:1].expand(cfg.E, -1, -1).contiguous()
+    r = oracle.moe_forward(to_oracle(d["x"]), to_oracle(d["W_router"]), to_oracle(Wgu), to_oracle(Wd),
+                           to_oracle(d["Ws_gate_up"]), to_oracle(d["Ws_down"]), top_k=cfg.top_k)
+    x = _f64(d["x"])
+    want = _numpy_ffn(x, _f64(Wgu[0]), _f64(Wd[0])) + _numpy_ffn(x, _f64(d["Ws_gate_up"]), _f64(d["Ws_down"]))
+    assert np.allclose(r["y"], want, rtol=1e-10, atol=1e-12)
+
+
+def test_top_k_equal_E_is_the_full_softmax_mixture():
+    cfg = _small("f32", top_k=6)
+    d = inputs.make_inputs(cfg)
+    r = oracle.moe_forward(to_oracle(d["x"]), to_oracle(d["W_router"]), to_oracle(d["W_gate_up"]),
+                           to_oracle(d["W_down"]), to_oracle(d["Ws_gate_up"]), to_oracle(d["Ws_down"]),
+                           top_k=cfg.E)
+    x = _f64(d["x"])
+    logits = x @ _f64(d["W_router"]).T  # fp64 library matmul, rounding differences << 1e-6
+    p = np.exp(logits - logits.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    want = _numpy_ffn(x, _f64(d["Ws_gate_up"]), _f64(d["Ws_down"]))
+    for e in range(cfg.E):
+        want += p[:, e:e + 1] * _numpy_ffn(x, _f64(d["W_gate_up"][e]), _f64(d["W_down"][e]))
+    assert np.allclose(r["y"], want, rtol=1e-6, atol=1e-9)
+    assert np.array_equal(r["idx"], np.tile(np.arange(cfg.E, dtype=np.int32), (cfg.T, 1)))
+
+
+def test_zero_down_projection_leaves_the_shared_expert():
+    cfg = _small("bf16")
+    d = inputs.make_inputs(cfg)
+    Wd0 = torch.zeros_like(d["W_down"])
+    r = oracle.moe_forward(to_oracle(d["x"]), to_oracle(d["W_router"]), to_oracle(d["W_gate_up"]),
+                           to_oracle(Wd0), to_oracle(d["Ws_gate_up"]), to_oracle(d["Ws_down"]),
+                           top_k=cfg.top_k)
+    want = _numpy_ffn(_f64(d["x"]), _f64(d["Ws_gate_up"]), _f64(d["Ws_down"]))
+    assert np.allclose(r["y"], want, rtol=1e-10, atol=1e-12)
+    r2 = oracle.moe_forward(to_oracle(d["x"]), to_oracle(d["W_router"]), to_oracle(d["W_gate_up"]),
+                            to_oracle(Wd0), None, None, top_k=cfg.top_k)
+    assert np.all(r2["y"] == 0.0)
+
+
+def test_zero_input():
+    cfg = _small("bf16")
+    d = inputs.make_inputs(cfg)
+    x0 = torch.zeros_like(d["x"])
+    r = oracle.moe_forward(to_oracle(x0), to_oracle(d["W_router"]), to_oracle(d["W_gate_up"]),
+                           to_oracle(d["W_down"]), to_oracle(d["Ws_gate_up"]), to_oracle(d["Ws_down"]),
+                           top_k=cfg.top_k)
+    assert np.all(r["scores"] == 0)
+    assert np.array_equal(r["idx"], np.tile(np.arange(cfg.top_k, dtype=np.int32), (cfg.T, 1)))
+    assert np.all(r["w"] == np.float32(1.0 / cfg.top_k))
+    assert np.all(r["y"] == 0.0)
+
+
+def test_duplicated_router_rows_tie_toward_lower_index():
+    cfg = _small("bf16", E=8, top_k=3)
+    d = inputs.make_inputs(cfg)
+    Wr = d["W_router"].clone()
+    Wr[5] = Wr[2]  # experts 2 and 5 always tie exactly
+    r = oracle.moe_forward(to_oracle(d["x"]), to_oracle(Wr), to_oracle(d["W_gate_up"]),
+                           to_oracle(d["W_down"]), None, None, top_k=cfg.top_k)
+    assert np.array_equal(r["scores"][:, 2], r["scores"][:, 5])
+    for t in range(cfg.T):
+        chosen = set(r["idx"][t])
+        assert not (5 in chosen and 2 not in chosen)
+
+
+def test_token_permutation_equivariance():
+    cfg = _small("bf16", T=30)
+    d = inputs.make_inputs(cfg)
+    args = [to_oracle(d[k]) for k in ("W_router", "W_gate_up", "W_down", "Ws_gate_up", "Ws_down")]
+    r = oracle.moe_forward(to_oracle(d["x"]), *args, top_k=cfg.top_k)
+    p = np.random.default_rng(0).permutation(cfg.T)
+    rp = oracle.moe_forward(to_oracle(d["x"])[p], *args, top_k=cfg.top_k)
+    assert np.array_equal(rp["idx"], r["idx"][p])
+    assert np.array_equal(rp["w"], r["w"][p])
+    assert np.array_equal(rp["y"], r["y"][p])
+
+
+def test_token_subset_matches_full_output():
+    cfg = _small("f32", T=20)
+    d = inputs.make_inputs(cfg)
+    args = [to_oracle(d[k]) for k in ("W_router", "W_gate_up", "W_down", "Ws_gate_up", "Ws_down")]
+    r = oracle.moe_forward(to_oracle(d["x"]), *args, top_k=cfg.top_k)
+    sub = [3, 17, 0]
+    rs = oracle.moe_forward(to_oracle(d["x"]), *args, top_k=cfg.top_k, tokens=sub)
+    assert np.array_equal(rs["y"], r["y"][sub])
+
+
+# --------------------------------------------------------------------------------------
+# the pages' shape constants
+# --------------------------------------------------------------------------------------
+def test_page_shapes_give_the_published_parameter_totals():
+    c = json.load(open(os.path.join(GOLDEN, "step35_flash_shapes.json")))
+    H, E, I, Is = c["hidden_size"], c["moe_num_experts"], c["moe_intermediate_size"], c["share_expert_dim"]
+    n_moe = c["moe_layers_enum_last"] - c["moe_layers_enum_first"] + 1
+    assert n_moe == 42
+    per_expert = 3 * H * I  # gate, up and down matrices of H x I
+    per_layer = E * per_expert + 3 * H * Is + E * H
+    total_moe = n_moe * per_layer
+    embed = 2 * c["vocab_size"] * H  # untied input and output embeddings
+    dense = (c["moe_layers_enum_first"]) * 3 * H * c["intermediate_size"]
+    # the routed experts are most of the 196 B; attention and norms make up the rest
+    assert 0.9 * 196e9 < total_moe + embed + dense < 196e9
+    # active: top-8 routed + shared + router per MoE layer, plus the dense layers and embeddings
+    active = n_moe * ((c["moe_top_k"] + 1) * per_expert + E * H) + dense + embed
+    assert 0.6 * 11e9 < active < 11e9
+    # two-matrix experts would be inconsistent with the published total
+    assert n_moe * E * 2 * H * I < 0.7 * 196e9
+
+
+def test_workload_table_matches_the_pages():
+    c = json.load(open(os.path.join(GOLDEN, "step35_flash_shapes.json")))
+    for name in ("decode_t4", "decode_t128", "prefill_t4096", "prefill_t16384_skew"):
+        cfg = inputs.CONFIGS[name]
+        assert (cfg.H, cfg.E, cfg.top_k, cfg.I, cfg.I_shared) == (
+            c["hidden_size"], c["moe_num_experts"], c["moe_top_k"], c["moe_intermediate_size"],
+            c["share_expert_dim"])
