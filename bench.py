@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark of the Step-3.5-Flash routed-expert MoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
+
+One step = one full forward of the layer (routing, dispatch, both grouped expert GEMMs,
+combine) over one batch of synthetic tokens with all inputs resident in HBM.  The L2 is
+flushed (a 2x-L2 write) before every timed step, outside the timed events.  Each step is
+timed with CUDA events on the launching stream; the sum over K steps, max over ranks,
+gives ``value`` = tokens of all ranks / time.  ``e2e`` repeats the measurement through the
+public API with the step's tokens copied from pinned host memory and the output read
+back inside the timed region.  Under torchrun each rank runs an independent replica on its
+own tokens (the layer shards by tokens; no collective on the data path): weak scaling.
+
+``--impl reference`` times the CPU oracle (plain C, OpenMP) on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_mixture_experts_ffn_b200 import inputs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s at T=4…16384; % of HBM or bf16 tensor-core roofline"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "decode_t4"
+DEFAULT_STEPS = {"decode_t4": 2000, "decode_t128": 500, "prefill_t4096": 200,
+                 "prefill_t16384_skew": 60, "tiny_f32_t64": 2000}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", sel, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception as e:  # pragma: no cover - no nvidia-smi
+            log("clock sampler unavailable:", e)
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self._t.join(timeout=2)
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[4:]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------
+# algorithmic bytes / flops
+# ------------------------------------------------------------------------------------------
+def algorithmic(cfg, counts: np.ndarray):
+    """Bytes and FLOPs of the layer and of its gate/up GEMM for one step (no padding)."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    H, I, Is, E, T, k = cfg.H, cfg.I, cfg.I_shared, cfg.E, cfg.T, cfg.top_k
+    touched = int((counts > 0).sum())
+    P = T * k
+    layer_bytes = (touched * 3 * H * I + 3 * H * Is + E * H + 2 * T * H) * es
+    layer_flops = 2 * T * E * H + P * 6 * H * I + T * 6 * H * Is
+    gu_bytes = (touched * 2 * I * H + 2 * Is * H + P * H + T * H + P * I + T * Is) * es
+    gu_flops = P * 4 * H * I + T * 4 * H * Is
+    dn_bytes = (touched * H * I + H * Is + P * I + T * Is + P * H + T * H) * es
+    dn_flops = P * 2 * H * I + T * 2 * H * Is
+    return dict(touched=touched, layer_bytes=layer_bytes, layer_flops=layer_flops,
+                gate_up_bytes=gu_bytes, gate_up_flops=gu_flops, down_bytes=dn_bytes, down_flops=dn_flops)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it still matches the source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        ent = d[f"{kernel}@{workload}"]
+        import hashlib
+        src = os.path.join(ROOT, ent["source"])
+        if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != ent["source_sha"]:
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------------------------------
+# the oracle on the host (cpu baseline and the reference arm)
+# ------------------------------------------------------------------------------------------
+def host_arrays(d):
+    import numpy as _np
+
+    def cv(t):
+        if t is None:
+            return None
+        t = t.detach().cpu().contiguous()
+        return t.view(torch.int16).numpy().view(_np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+    return {k: cv(v) for k, v in d.items()}
+
+
+def oracle_step(h, cfg, tokens):
+    """The whole hot path for the listed tokens: exact router over all experts, top-k and
+    weights, then the expert FFNs and the combine."""
+    import oracle
+    x = h["x"][tokens]
+    s = oracle.router_scores(x, h["W_router"])
+    bias = None if h.get("bias") is None else h["bias"].astype(np.float32)
+    idx, w, w64 = oracle.route(s, cfg.top_k, bias)
+    return oracle.moe_tokens(x, idx, w64, h["W_gate_up"], h["W_down"], h["Ws_gate_up"], h["Ws_down"])
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    d = inputs.make_inputs(cfg, "cpu") if cfg.T * cfg.H * cfg.E < 5e7 else None
+    if d is None:
+        x, Wr, bias = inputs.make_routing_inputs(cfg)
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        Wgu, Wd, Wsgu, Wsd = inputs.make_expert_weights(cfg, dev)
+        d = dict(x=x, W_router=Wr, bias=bias, W_gate_up=Wgu, W_down=Wd, Ws_gate_up=Wsgu, Ws_down=Wsd)
+    h = host_arrays(d)
+    cores = len(os.sched_getaffinity(0))
+    per_step = 1  # tokens per step: one token's full pass through the layer
+    for i in range(args.warmup):
+        oracle_step(h, cfg, [i % cfg.T])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle_step(h, cfg, [i % cfg.T])
+    dt = time.perf_counter() - t0
+    value = per_step * args.steps / dt
+    sample = f"{per_step} token of {cfg.name} per step (exact router over {cfg.E} experts, top-{cfg.top_k}, {cfg.top_k} routed + 1 shared expert FFNs)"
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+            "data": "synthetic", "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E,
+                                             "top_k": cfg.top_k, "I": cfg.I, "I_shared": cfg.I_shared},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(h, cfg, budget_s=10.0):
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    tokens = list(range(min(cfg.T, 8)))
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(h, cfg, tokens)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": len(tokens) * n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{len(tokens)} tokens of {cfg.name} x {n} repetitions ({dt:.1f} s): exact router over "
+                      f"{cfg.E} experts, top-{cfg.top_k}, routed + shared expert FFNs in fp64"}
+
+
+# ------------------------------------------------------------------------------------------
+# the CUDA path
+# ------------------------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.CONFIGS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = inputs.CONFIGS[args.workload]
+    if args.steps is None:
+        args.steps = DEFAULT_STEPS.get(cfg.name, 100)
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    import sparse_mixture_experts_ffn_b200 as moe
+    from sparse_mixture_experts_ffn_b200 import build
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    if rank == 0 or world == 1:
+        build.build()
+    if pg:
+        pg.barrier()
+    moe.load_library()
+
+    # ---- inputs (resident in HBM); each rank is a replica with its own tokens -------------
+    rcfg = inputs.with_sizes(cfg, seed=cfg.seed + 1000 * rank) if rank else cfg
+    x, Wr, bias = inputs.make_routing_inputs(rcfg)
+    Wgu, Wd, Wsgu, Wsd = inputs.make_expert_weights(cfg, dev)
+    x, Wr = x.to(dev), Wr.to(dev)
+    bias = None if bias is None else bias.to(dev)
+    shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared, cfg.top_k, cfg.torch_dtype)
+    ws = moe.alloc_workspace(shape, dev)
+    y = torch.empty_like(x)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(xin, yout, routing=False):
+        return moe.moe_layer_forward(xin, Wr, Wgu, Wd, Wsgu, Wsd, top_k=cfg.top_k, router_bias=bias,
+                                     y=yout, workspace=ws, routing=routing, stream=stream)
+
+    _, r = step(x, y, routing=True)
+    torch.cuda.synchronize()
+    status = moe.check_status(ws)
+    if status != moe.MOE_OK:
+        raise RuntimeError(f"device status {moe.status_string(status)}")
+    counts = r.counts.cpu().numpy()
+    route_stats = moe.route_stats(ws)
+    alg = algorithmic(cfg, counts)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(x, y)
+    torch.cuda.synchronize()
+
+    # ---- kernel-only timed region --------------------------------------------------------
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    moe.profile_read()
+    moe.profile_enable(True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    launches0 = moe.launch_count()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step(x, y)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    launches = moe.launch_count() - launches0
+    moe.profile_enable(False)
+    calls, stage_ms = moe.profile_read()
+    elapsed_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    if pg:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    status = moe.check_status(ws)
+
+    # ---- end to end through the public API, host buffers ----------------------------------
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    x_dev = torch.empty_like(x)
+    e_steps = max(3, min(args.steps, 500))
+    es_, ee_ = ([torch.cuda.Event(enable_timing=True) for _ in range(e_steps)] for _ in range(2))
+    for _ in range(3):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev, y)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    for i in range(e_steps):
+        flush.zero_()
+        es_[i].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev, y)
+        y_host.copy_(y, non_blocking=True)
+        ee_[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(es_, ee_))
+    if pg:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        pg.barrier()
+
+    if rank == 0:
+        peaks = measured_peaks()
+        ms_per_step = elapsed_ms / args.steps
+        value = world * cfg.T * args.steps / (elapsed_ms / 1e3)
+        e2e_value = world * cfg.T * e_steps / (e2e_ms / 1e3)
+        gu_ms = stage_ms["gate_up"] / max(calls, 1)
+        dn_ms = stage_ms["down"] / max(calls, 1)
+        tensor_bound = alg["gate_up_flops"] / (peaks["bf16_tflops"] * 1e12) > alg["gate_up_bytes"] / (peaks["hbm_gbs"] * 1e9)
+        if tensor_bound:
+            achieved = alg["gate_up_flops"] / (gu_ms / 1e3) / 1e12
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_tflops"]}
+        else:
+            achieved = alg["gate_up_bytes"] / (gu_ms / 1e3) / 1e9
+            roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"]}
+        roof.update({"kernel": "expert_gemm_tc_kernel<gated> (gate/up GEMM + SiLU*up)",
+                     "traffic": ncu_traffic("gate_up", cfg.name), "peak_source": peaks["source"],
+                     "ms_per_launch": gu_ms, "algorithmic_bytes": alg["gate_up_bytes"],
+                     "algorithmic_flops": alg["gate_up_flops"]})
+        layer_s = ms_per_step / 1e3
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "top_k": cfg.top_k,
+                       "I": cfg.I, "I_shared": cfg.I_shared, "tokens_per_gpu": cfg.T,
+                       "l2": "flushed before every timed step (2x L2 write, outside the events)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": roof,
+            "layer": {"touched_experts": alg["touched"], "algorithmic_bytes": alg["layer_bytes"],
+                      "algorithmic_flops": alg["layer_flops"],
+                      "hbm_gbs": alg["layer_bytes"] / layer_s / 1e9,
+                      "hbm_frac": alg["layer_bytes"] / layer_s / 1e9 / peaks["hbm_gbs"],
+                      "tflops": alg["layer_flops"] / layer_s / 1e12,
+                      "stage_ms_per_step": {k: v / max(calls, 1) for k, v in stage_ms.items()},
+                      "route_stats": route_stats, "device_status": moe.status_string(status)},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x.numel() * x.element_size(),
+                    "d2h_bytes_per_step": y.numel() * y.element_size(), "steps": e_steps},
+            "gpu_launches": int(launches),
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            oracle.build()
+            h = host_arrays(dict(x=x, W_router=Wr, bias=bias, W_gate_up=Wgu, W_down=Wd, Ws_gate_up=Wsgu,
+                                 Ws_down=Wsd))
+            line["cpu_baseline"] = cpu_baseline(h, cfg)
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,164 @@
+/*
+ * moe_layer.h -- C ABI of the B200 (sm_100a) routed-expert MoE FFN layer of Step-3.5-Flash.
+ *
+ * The layer (llm-atlas page "Step-3.5-Flash", table "Champs bruts du config.json":
+ * moe_num_experts 288, moe_top_k 8, norm_expert_weight true, need_fp32_gate true,
+ * moe_intermediate_size 1280, share_expert_dim 1280, hidden_size 4096; and the page's
+ * "FFN / MoE" paragraph: a sparse mixture of 288 routed experts with top-8 routing):
+ *
+ *   s[t,e]   = sum_h x[t,h] * W_router[e,h]      exact sum, rounded once to fp32
+ *   key[t,e] = fp32(s[t,e] + router_bias[e])     (router_bias optional)
+ *   S_t      = the top_k experts by (key descending, expert index ascending)
+ *   w[t,j]   = softmax of the keys over S_t      (renormalised: sums to 1)
+ *   y_t      = sum_{e in S_t} w * (SiLU(x_t Wg_e^T) * (x_t Wu_e^T)) Wd_e^T
+ *            + (SiLU(x_t Wsg^T) * (x_t Wsu^T)) Wsd^T      (shared expert, weight 1)
+ *
+ * The pages leave the score function and the activation open: this library uses a
+ * softmax router and SiLU(gate)*up.  Routing is decided on the exact fp32 score, so the
+ * chosen experts do not depend on summation order.
+ *
+ * Conventions for every entry point:
+ *   - all tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *     contiguous, 16-byte aligned; the library never allocates or frees device memory;
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream);
+ *     work is enqueued asynchronously and the call returns without synchronising;
+ *   - the return value reports argument validation and launch errors only; errors found
+ *     on the device (a bounded wait that timed out) are written to a status word in the
+ *     workspace and read back by moe_layer_check_status();
+ *   - inputs must be finite; NaN/Inf give an unspecified result but never a hang;
+ *   - y must not alias any input; the workspace must not be shared by calls that may
+ *     run concurrently.
+ */
+#ifndef MOE_LAYER_H
+#define MOE_LAYER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,         /* null pointer, bad top_k, misaligned pointer, ... */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,   /* sizes outside what the kernels tile (see below) */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes < moe_layer_workspace_bytes() */
+  MOE_ERR_CUDA = 4,                /* a CUDA runtime/driver call or launch failed */
+  MOE_ERR_DEVICE_TIMEOUT = 5,      /* a bounded device-side wait gave up */
+  MOE_ERR_DEVICE_BOUNDS = 6        /* a device-side index check failed */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Layer sizes.  T tokens, hidden size H, E routed experts, expert width I, shared
+ * expert width I_shared (0 = no shared expert), top_k experts per token.
+ * Supported: T >= 0 (T = 0 is a no-op), 1 <= top_k <= E <= 1024, T*top_k < 2^31.
+ *   MOE_BF16: H, I and I_shared (if nonzero) multiples of 128.
+ *   MOE_F32 : H a multiple of 8; I, I_shared >= 1.                                  */
+typedef struct {
+  int64_t T;
+  int32_t H, E, I, I_shared, top_k;
+  int32_t dtype; /* moe_dtype */
+} moe_layer_shape;
+
+/* Optional routing outputs (any field may be NULL; the struct pointer may be NULL).
+ *   topk_idx [T, top_k] int32  chosen experts of each token, ascending expert index
+ *   topk_w   [T, top_k] fp32   their renormalised softmax weights (same order)
+ *   counts   [E]        int32  number of tokens routed to each expert
+ *   offsets  [E + 1]    int32  exclusive prefix sum of counts (offsets[E] = T*top_k)
+ *   perm     [T*top_k]  int32  assignments t*top_k + j sorted by (expert, token):
+ *                              perm[offsets[e] + r] is the r-th token routed to e     */
+typedef struct {
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+} moe_routing_out;
+
+/* Device workspace needed by moe_layer_forward for this shape, in bytes (0 on an
+ * invalid shape).  Pure host computation. */
+MOE_API size_t moe_layer_workspace_bytes(const moe_layer_shape* shape);
+
+/* Forward pass of the MoE layer.
+ *   x          [T, H]          dtype   input tokens
+ *   W_router   [E, H]          dtype   router matrix
+ *   router_bias[E]             fp32    added to the router scores, or NULL
+ *   W_gate_up  [E, 2*I, H]     dtype   per expert: I gate rows, then I up rows
+ *   W_down     [E, H, I]       dtype   per expert down projection
+ *   Ws_gate_up [2*I_shared, H] dtype   shared expert gate rows then up rows (NULL iff
+ *                                      I_shared == 0)
+ *   Ws_down    [H, I_shared]   dtype   shared expert down projection
+ *   y          [T, H]          dtype   output (written, never read)
+ *   routing    optional routing outputs (see moe_routing_out)
+ *   workspace  device scratch of at least moe_layer_workspace_bytes(shape) bytes,
+ *              256-byte aligned, owned by the caller; its contents need no
+ *              initialisation and are overwritten.
+ * T = 0 returns MOE_OK at once (pointers are not inspected).
+ * Errors: MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED_SHAPE / MOE_ERR_WORKSPACE_TOO_SMALL
+ * before anything is enqueued; MOE_ERR_CUDA if a launch fails. */
+MOE_API moe_status moe_layer_forward(const moe_layer_shape* shape, const void* x, const void* W_router,
+                             const float* router_bias, const void* W_gate_up, const void* W_down,
+                             const void* Ws_gate_up, const void* Ws_down, void* y,
+                             moe_routing_out* routing, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* Synchronises `stream`, then returns the device status word of the most recent
+ * moe_layer_forward() that used this workspace (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or
+ * MOE_ERR_DEVICE_BOUNDS), or MOE_ERR_CUDA if the stream itself reports an error. */
+MOE_API moe_status moe_layer_check_status(void* workspace, void* stream);
+
+/* Routing diagnostics of the most recent forward on this workspace (synchronises):
+ *   n_refined : (token, expert) scores recomputed in fp64 because their fp32 key was not
+ *               certain and could change the chosen set;
+ *   n_exact   : scores that needed the exact (integer) dot product after that;
+ *   n_tokens_refined : tokens that needed any recomputation.                         */
+typedef struct {
+  int64_t n_refined;
+  int64_t n_exact;
+  int64_t n_tokens_refined;
+} moe_route_stats;
+MOE_API moe_status moe_layer_route_stats(void* workspace, moe_route_stats* out, void* stream);
+
+/* Byte offsets of the intermediate buffers inside the workspace (for inspection by
+ * tests; layout is private and may change between versions).  Sizes in elements:
+ *   x_perm [T*top_k, H] dtype, h [T*top_k, I] dtype, h_shared [T, I_shared] dtype,
+ *   o [T*top_k, H] dtype, o_shared [T, H] dtype, row_w [T*top_k] fp32 (routing weight
+ *   of each row of x_perm/h/o in expert order).  Returns MOE_ERR_INVALID_ARG on a bad
+ *   shape. */
+typedef struct {
+  size_t x_perm, h, h_shared, o, o_shared, row_w;
+} moe_workspace_layout;
+MOE_API moe_status moe_layer_workspace_layout(const moe_layer_shape* shape, moe_workspace_layout* out);
+
+/* Stage timing for benchmarks.  While enabled, every moe_layer_forward() also records
+ * CUDA events on its stream at the boundaries of its five stages:
+ *   0 routing  (router scores, certified top-k, softmax weights)
+ *   1 dispatch (histogram, scan, stable permutation, row gather)
+ *   2 gate/up  (grouped GEMM with the SiLU(gate)*up epilogue)
+ *   3 down     (grouped GEMM with the routing-weight epilogue)
+ *   4 combine  (unpermute and sum)
+ * moe_layer_profile_read() waits for the recorded events, adds each stage's elapsed
+ * milliseconds since the previous read into ms[0..n_stages), forgets them and returns
+ * the number of forward calls covered (or -1 on a CUDA error).  Process-wide; not meant
+ * for concurrent forwards on several threads. */
+MOE_API moe_status moe_layer_profile_enable(int enable);
+MOE_API int moe_layer_profile_read(float* ms, int n_stages);
+
+/* Number of kernels this library has launched in this process so far. */
+MOE_API int64_t moe_layer_launch_count(void);
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char* moe_status_string(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_LAYER_H */

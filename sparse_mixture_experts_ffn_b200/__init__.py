@@ -1,0 +1,218 @@
+"""Python binding of the sm_100a MoE layer library (``libmoe_layer.so``, C ABI in
+``include/moe_layer.h``).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA kernels.
+PyTorch provides device memory and the current stream.  There is no fallback: if the
+library is missing the call raises.
+
+    from sparse_mixture_experts_ffn_b200 import moe_layer_forward
+    y, routing = moe_layer_forward(x, W_router, W_gate_up, W_down, Ws_gate_up, Ws_down, top_k=8)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_layer.so")
+
+MOE_OK = 0
+MOE_F32, MOE_BF16 = 0, 1
+STATUS_NAMES = {
+    0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
+    3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT",
+    6: "MOE_ERR_DEVICE_BOUNDS",
+}
+EXPORTED = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_layer_check_status",
+            "moe_layer_route_stats", "moe_layer_workspace_layout", "moe_layer_profile_enable",
+            "moe_layer_profile_read", "moe_layer_launch_count", "moe_status_string")
+STAGES = ("routing", "dispatch", "gate_up", "down", "combine")
+
+
+class MoEShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("I", ctypes.c_int32), ("I_shared", ctypes.c_int32), ("top_k", ctypes.c_int32),
+                ("dtype", ctypes.c_int32)]
+
+
+class MoERoutingOut(ctypes.Structure):
+    _fields_ = [("topk_idx", ctypes.c_void_p), ("topk_w", ctypes.c_void_p),
+                ("counts", ctypes.c_void_p), ("offsets", ctypes.c_void_p),
+                ("perm", ctypes.c_void_p)]
+
+
+class MoERouteStats(ctypes.Structure):
+    _fields_ = [("n_refined", ctypes.c_int64), ("n_exact", ctypes.c_int64),
+                ("n_tokens_refined", ctypes.c_int64)]
+
+
+class MoEWorkspaceLayout(ctypes.Structure):
+    _fields_ = [("x_perm", ctypes.c_size_t), ("h", ctypes.c_size_t), ("h_shared", ctypes.c_size_t),
+                ("o", ctypes.c_size_t), ("o_shared", ctypes.c_size_t), ("row_w", ctypes.c_size_t)]
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load the CUDA library (no fallback: raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} not found: build it with `python -m sparse_mixture_experts_ffn_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    lib.moe_layer_workspace_bytes.argtypes = [ctypes.POINTER(MoEShape)]
+    lib.moe_layer_workspace_bytes.restype = ctypes.c_size_t
+    lib.moe_layer_forward.argtypes = [ctypes.POINTER(MoEShape), P, P, P, P, P, P, P, P,
+                                      ctypes.POINTER(MoERoutingOut), P, ctypes.c_size_t, P]
+    lib.moe_layer_forward.restype = ctypes.c_int
+    lib.moe_layer_check_status.argtypes = [P, P]
+    lib.moe_layer_check_status.restype = ctypes.c_int
+    lib.moe_layer_route_stats.argtypes = [P, ctypes.POINTER(MoERouteStats), P]
+    lib.moe_layer_route_stats.restype = ctypes.c_int
+    lib.moe_layer_workspace_layout.argtypes = [ctypes.POINTER(MoEShape), ctypes.POINTER(MoEWorkspaceLayout)]
+    lib.moe_layer_workspace_layout.restype = ctypes.c_int
+    lib.moe_layer_profile_enable.argtypes = [ctypes.c_int]
+    lib.moe_layer_profile_enable.restype = ctypes.c_int
+    lib.moe_layer_profile_read.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_int]
+    lib.moe_layer_profile_read.restype = ctypes.c_int
+    lib.moe_layer_launch_count.argtypes = []
+    lib.moe_layer_launch_count.restype = ctypes.c_int64
+    lib.moe_status_string.argtypes = [ctypes.c_int]
+    lib.moe_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def make_shape(T, H, E, I, I_shared, top_k, dtype) -> MoEShape:
+    import torch
+    code = MOE_BF16 if dtype == torch.bfloat16 else MOE_F32 if dtype == torch.float32 else -1
+    if code < 0:
+        raise TypeError(f"unsupported dtype {dtype}")
+    return MoEShape(int(T), int(H), int(E), int(I), int(I_shared), int(top_k), code)
+
+
+def workspace_bytes(shape: MoEShape) -> int:
+    return int(load_library().moe_layer_workspace_bytes(ctypes.byref(shape)))
+
+
+def workspace_layout(shape: MoEShape) -> MoEWorkspaceLayout:
+    out = MoEWorkspaceLayout()
+    rc = load_library().moe_layer_workspace_layout(ctypes.byref(shape), ctypes.byref(out))
+    if rc != MOE_OK:
+        raise MoEError(rc, "moe_layer_workspace_layout")
+    return out
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+@dataclass
+class Routing:
+    topk_idx: "object"
+    topk_w: "object"
+    counts: "object"
+    offsets: "object"
+    perm: "object"
+
+
+def alloc_workspace(shape: MoEShape, device):
+    import torch
+    nbytes = workspace_bytes(shape)
+    if nbytes == 0:
+        raise MoEError(1, "moe_layer_workspace_bytes")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def moe_layer_forward(x, W_router, W_gate_up, W_down, Ws_gate_up=None, Ws_down=None, *, top_k,
+                      router_bias=None, y=None, workspace=None, routing=True, stream=None):
+    """Run the MoE layer on the device.  Returns (y, Routing or None).
+
+    Shapes: x [T,H], W_router [E,H], W_gate_up [E,2I,H], W_down [E,H,I], Ws_gate_up
+    [2Is,H], Ws_down [H,Is] (or both None), router_bias [E] fp32 or None.  All CUDA,
+    contiguous, same dtype (bf16 or fp32).
+    """
+    import torch
+    lib = load_library()
+    T, H = x.shape
+    E = W_router.shape[0]
+    I = W_gate_up.shape[1] // 2
+    Is = 0 if Ws_gate_up is None else Ws_gate_up.shape[0] // 2
+    shape = make_shape(T, H, E, I, Is, top_k, x.dtype)
+    for name, t in (("x", x), ("W_router", W_router), ("W_gate_up", W_gate_up), ("W_down", W_down),
+                    ("Ws_gate_up", Ws_gate_up), ("Ws_down", Ws_down), ("router_bias", router_bias)):
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if y is None:
+        y = torch.empty_like(x)
+    if workspace is None:
+        workspace = alloc_workspace(shape, x.device)
+    r = None
+    rout = None
+    if routing:
+        dev = x.device
+        r = Routing(torch.empty(T, top_k, dtype=torch.int32, device=dev),
+                    torch.empty(T, top_k, dtype=torch.float32, device=dev),
+                    torch.empty(E, dtype=torch.int32, device=dev),
+                    torch.empty(E + 1, dtype=torch.int32, device=dev),
+                    torch.empty(T * top_k, dtype=torch.int32, device=dev))
+        rout = MoERoutingOut(r.topk_idx.data_ptr(), r.topk_w.data_ptr(), r.counts.data_ptr(),
+                             r.offsets.data_ptr(), r.perm.data_ptr())
+    if stream is None:
+        stream = torch.cuda.current_stream(x.device)
+    rc = lib.moe_layer_forward(ctypes.byref(shape), _ptr(x), _ptr(W_router), _ptr(router_bias),
+                               _ptr(W_gate_up), _ptr(W_down), _ptr(Ws_gate_up), _ptr(Ws_down),
+                               _ptr(y), ctypes.byref(rout) if rout is not None else None,
+                               _ptr(workspace), workspace.numel(), ctypes.c_void_p(stream.cuda_stream))
+    if rc != MOE_OK:
+        raise MoEError(rc, "moe_layer_forward")
+    return y, r
+
+
+def check_status(workspace, stream=None) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(workspace.device)
+    return int(load_library().moe_layer_check_status(_ptr(workspace), ctypes.c_void_p(stream.cuda_stream)))
+
+
+def route_stats(workspace, stream=None) -> dict:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(workspace.device)
+    out = MoERouteStats()
+    rc = load_library().moe_layer_route_stats(_ptr(workspace), ctypes.byref(out), ctypes.c_void_p(stream.cuda_stream))
+    if rc != MOE_OK:
+        raise MoEError(rc, "moe_layer_route_stats")
+    return dict(n_refined=out.n_refined, n_exact=out.n_exact, n_tokens_refined=out.n_tokens_refined)
+
+
+def status_string(status: int) -> str:
+    return load_library().moe_status_string(int(status)).decode()
+
+
+def profile_enable(enable: bool = True) -> None:
+    load_library().moe_layer_profile_enable(1 if enable else 0)
+
+
+def profile_read() -> tuple[int, dict]:
+    """(forward calls covered, {stage: total ms}) since the previous read."""
+    ms = (ctypes.c_float * len(STAGES))()
+    calls = load_library().moe_layer_profile_read(ms, len(STAGES))
+    if calls < 0:
+        raise MoEError(4, "moe_layer_profile_read")
+    return calls, {name: float(ms[i]) for i, name in enumerate(STAGES)}
+
+
+def launch_count() -> int:
+    return int(load_library().moe_layer_launch_count())

@@ -1,0 +1,487 @@
+// experts.cu -- grouped expert GEMMs of the MoE layer.
+//
+// bf16: one persistent, warp-specialised tcgen05 kernel per projection.  Weights are the
+// A operand (128 rows per tile, "swap-AB"), the tokens routed to an expert the B operand
+// (up to 128 per tile), so an expert's few tokens never pad a 128-row tile:
+//   gate/up:  h[p, i]  = SiLU(x_p . Wg[e, i]) * (x_p . Wu[e, i])     (SiLU(gate) * up)
+//   down:     o[p, c]  = w_p * (h_p . Wd[e, c])                     (routing weight fused)
+// with fp32 accumulators in tensor memory and bf16 outputs.  The shared expert
+// (share_expert_dim, always on, weight 1) is one more group over all T tokens.
+// Sources: llm-atlas page "Step-3.5-Flash", "Champs bruts du config.json":
+// moe_intermediate_size 1280, share_expert_dim 1280, hidden_size 4096, norm_expert_weight.
+//
+// fp32: plain CUDA-core kernels (fp32 FMA), same data flow.
+#include <algorithm>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------------------
+// tcgen05 grouped GEMM
+// ---------------------------------------------------------------------------------------
+struct TcParams {
+  CUtensorMap tmA[2];  // weights: [0] routed (all experts stacked), [1] shared expert
+  CUtensorMap tmB[2];  // activations: [0] routed rows in expert order, [1] shared rows
+  const int32_t* offsets;      // [E + 1]
+  const int32_t* group_order;  // [G]
+  const int32_t* item_start;   // [G + 1]
+  const float* row_w;          // routing weight per routed row (down projection only)
+  __nv_bfloat16* out[2];       // [0] routed rows, [1] shared rows
+  int ld_out[2];               // row stride of out (elements), routed and shared
+  int E, G;
+  int64_t T;
+  int kblocks[2];              // reduction length / kTileK, routed and shared
+  int a_rows_per_group;        // rows of one routed expert's weight matrix
+  int a_up_offset[2];          // gate/up: row offset of the up block (I or Is)
+  int mt[2];                   // weight row tiles per group, routed and shared
+  int rows_out[2];             // rows of out[0] (T*k) and out[1] (T)
+  int max_items;               // upper bound of the schedule length (host-computed)
+  Ctrl* ctrl;
+};
+
+template <bool GATED>
+struct TcCfg {
+  static constexpr int kStages = GATED ? 4 : 6;
+  static constexpr int kABytes = kTileM * kTileK * 2;  // 16 KB
+  static constexpr int kBBytes = kTileN * kTileK * 2;  // 16 KB
+  static constexpr int kStageBytes = (GATED ? 2 : 1) * kABytes + kBBytes;
+  static constexpr int kAccCols = (GATED ? 2 : 1) * kTileN;  // TMEM columns per accumulator
+  static constexpr int kTmemCols = 2 * kAccCols;             // double-buffered
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+struct Item {
+  int valid;   // 0: the schedule entry is inconsistent (reported; skipped by every role)
+  int sh;      // 0 routed expert, 1 shared expert
+  int g;       // group (expert id, or E for the shared expert)
+  int m;       // weight row tile
+  int row0;    // first activation row of the tile (in the routed or the shared row space)
+  int nvalid;  // tokens in the tile
+};
+
+__device__ __forceinline__ Item decode_item(const TcParams& p, int it) {
+  int lo = 0, hi = p.G - 1;
+  while (lo < hi) {  // last group slot whose first item is <= it
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(p.item_start + mid) <= it) lo = mid; else hi = mid - 1;
+  }
+  Item r;
+  r.g = __ldg(p.group_order + lo);
+  r.sh = (r.g == p.E) ? 1 : 0;
+  const int local = it - __ldg(p.item_start + lo);
+  const int base = r.sh ? 0 : __ldg(p.offsets + r.g);
+  const int cnt = r.sh ? static_cast<int>(p.T) : __ldg(p.offsets + r.g + 1) - base;
+  const int ntile = (cnt + kTileN - 1) / kTileN;
+  r.m = local / ntile;
+  const int n = local - r.m * ntile;
+  r.row0 = base + n * kTileN;
+  r.nvalid = min(kTileN, cnt - n * kTileN);
+  r.valid = (r.g >= 0 && r.g < p.G && ntile > 0 && r.m >= 0 && r.m < p.mt[r.sh] && r.nvalid >= 1 &&
+             r.row0 >= 0 && r.row0 + r.nvalid <= p.rows_out[r.sh]) ? 1 : 0;
+  if (!r.valid) {
+    r.nvalid = 0;
+    r.sh = 0;
+  }
+  return r;
+}
+
+// schedule length, clamped to the host bound (a larger value is reported, not run)
+__device__ __forceinline__ int schedule_length(const TcParams& p) {
+  const int total = __ldg(p.item_start + p.G);
+  if (total < 0 || total > p.max_items) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
+    return 0;
+  }
+  return total;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return g / (1.0f + __expf(-g)) * u;
+}
+
+// Wait without looking at the abort flag (teardown: in-flight copies must land).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, Ctrl* ctrl) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      set_status(ctrl, MOE_ERR_DEVICE_TIMEOUT);
+      return;
+    }
+  }
+}
+
+template <bool GATED>
+__global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
+  using C = TcCfg<GATED>;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  unsigned char* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* tfull = empty + C::kStages;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4 * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmA[0]);
+    tma_prefetch_desc(&p.tmB[0]);
+    tma_prefetch_desc(&p.tmA[1]);
+    tma_prefetch_desc(&p.tmB[1]);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = schedule_length(p);
+
+  if (warp == 0) {
+    // ------------------------------- TMA producer -------------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t used = 0;  // stages that ever received a copy
+      bool ok = true;
+      for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+        const Item t = decode_item(p, it);
+        if (!t.valid) {
+          if (blockIdx.x == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
+          continue;
+        }
+        const int arow = t.sh ? t.m * kTileM : t.g * p.a_rows_per_group + t.m * kTileM;
+        const int kb_n = p.kblocks[t.sh];
+        for (int kb = 0; kb < kb_n; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, p.ctrl, abort_flag)) { ok = false; break; }
+          unsigned char* st = smem + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          tma_load_2d(st, &p.tmA[t.sh], kb * kTileK, arow, &full[stage]);
+          if (GATED)
+            tma_load_2d(st + C::kABytes, &p.tmA[t.sh], kb * kTileK, arow + p.a_up_offset[t.sh],
+                        &full[stage]);
+          tma_load_2d(st + (GATED ? 2 : 1) * C::kABytes, &p.tmB[t.sh], kb * kTileK, t.row0,
+                      &full[stage]);
+          used |= 1u << stage;
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // every copy issued must have landed before the block exits
+      for (int s = 0; s < C::kStages; ++s) {
+        if (!(used & (1u << s))) continue;
+        // the last phase issued on stage s: stages before `stage` were last issued in the
+        // current pass (parity phase), the others in the previous pass (phase ^ 1)
+        const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+        mbar_wait_drain(&full[s], par, p.ctrl);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------- MMA issuer ---------------------------------------
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+        const Item t = decode_item(p, it);
+        if (!t.valid) continue;
+        const int n_mma = (t.nvalid + 15) & ~15;
+        const uint32_t idesc = idesc_bf16_f32(kTileM, n_mma);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.ctrl, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + acc * C::kAccCols;
+        const int kb_n = p.kblocks[t.sh];
+        for (int kb = 0; kb < kb_n; ++kb) {
+          if (!mbar_wait(&full[stage], phase, p.ctrl, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t b0 = a0 + (GATED ? 2 : 1) * C::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kTileK / 16; ++kk) {
+            const uint32_t accum = (kb | kk) ? 1u : 0u;
+            const uint64_t bdesc = sw128_kmajor_desc(b0 + kk * 32);
+            mma_bf16(d0, sw128_kmajor_desc(a0 + kk * 32), bdesc, idesc, accum);
+            if (GATED)
+              mma_bf16(d0 + kTileN, sw128_kmajor_desc(a0 + C::kABytes + kk * 32), bdesc, idesc,
+                       accum);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      // all MMAs issued by this thread complete before the accumulators are freed
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0, p.ctrl);
+    }
+  } else {
+    // ------------------------------- epilogue (warps 2..5) ----------------------------
+    const int quarter = warp & 3;  // TMEM lanes this warp may access: 32*quarter ..
+    const int r = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int it = blockIdx.x; it < total; it += gridDim.x) {
+      const Item t = decode_item(p, it);
+      if (!t.valid) continue;
+      if (!mbar_wait(&tfull[acc], acc_phase, p.ctrl, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::kAccCols;
+      const int ld = p.ld_out[t.sh];
+      __nv_bfloat16* out = p.out[t.sh] + static_cast<int64_t>(t.row0) * ld + t.m * kTileM + r;
+      for (int c0 = 0; c0 < t.nvalid; c0 += 16) {
+        float v[16];
+        tmem_ld16(trow + c0, v);
+        if (GATED) {
+          float u[16];
+          tmem_ld16(trow + kTileN + c0, u);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = silu_mul(v[j], u[j]);
+        } else if (!t.sh) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < t.nvalid) v[j] *= __ldg(p.row_w + t.row0 + c0 + j);
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (c0 + j < t.nvalid) out[static_cast<int64_t>(c0 + j) * ld] = __float2bfloat16_rn(v[j]);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// ---------------------------------------------------------------------------------------
+// fp32 CUDA-core path
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ int group_of_row(const int32_t* offsets, int E, int p) {
+  int lo = 0, hi = E - 1;  // last expert e with offsets[e] <= p
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(offsets + mid) <= p) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__global__ void gate_up_f32_kernel(const float* __restrict__ x_perm, const float* __restrict__ x,
+                                   const int32_t* __restrict__ offsets,
+                                   const float* __restrict__ Wgu, const float* __restrict__ Wsgu,
+                                   int64_t P, int64_t T, int H, int E, int I, int Is,
+                                   float* __restrict__ h, float* __restrict__ hs) {
+  const int64_t n_routed = P * I, total = n_routed + T * Is;
+  for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < total;
+       q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float *xr, *wg, *wu;
+    float* dst;
+    if (q < n_routed) {
+      const int64_t p = q / I;
+      const int i = static_cast<int>(q - p * I);
+      const int e = group_of_row(offsets, E, static_cast<int>(p));
+      xr = x_perm + p * H;
+      wg = Wgu + (static_cast<int64_t>(e) * 2 * I + i) * H;
+      wu = wg + static_cast<int64_t>(I) * H;
+      dst = h + q;
+    } else {
+      const int64_t qs = q - n_routed;
+      const int64_t t = qs / Is;
+      const int i = static_cast<int>(qs - t * Is);
+      xr = x + t * H;
+      wg = Wsgu + static_cast<int64_t>(i) * H;
+      wu = wg + static_cast<int64_t>(Is) * H;
+      dst = hs + qs;
+    }
+    float g = 0.f, u = 0.f;
+    for (int k = 0; k < H; ++k) {
+      const float xv = __ldg(xr + k);
+      g = fmaf(xv, __ldg(wg + k), g);
+      u = fmaf(xv, __ldg(wu + k), u);
+    }
+    *dst = g / (1.0f + expf(-g)) * u;
+  }
+}
+
+__global__ void down_f32_kernel(const float* __restrict__ h, const float* __restrict__ hs,
+                                const int32_t* __restrict__ offsets, const float* __restrict__ row_w,
+                                const float* __restrict__ Wd, const float* __restrict__ Wsd,
+                                int64_t P, int64_t T, int H, int E, int I, int Is,
+                                float* __restrict__ o, float* __restrict__ os) {
+  const int64_t n_routed = P * H, total = n_routed + (Is > 0 ? T * H : 0);
+  for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < total;
+       q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float *hr, *wr;
+    float scale, *dst;
+    int n;
+    if (q < n_routed) {
+      const int64_t p = q / H;
+      const int c = static_cast<int>(q - p * H);
+      const int e = group_of_row(offsets, E, static_cast<int>(p));
+      hr = h + p * I;
+      wr = Wd + (static_cast<int64_t>(e) * H + c) * I;
+      scale = row_w[p];
+      dst = o + q;
+      n = I;
+    } else {
+      const int64_t qs = q - n_routed;
+      const int64_t t = qs / H;
+      const int c = static_cast<int>(qs - t * H);
+      hr = hs + t * Is;
+      wr = Wsd + static_cast<int64_t>(c) * Is;
+      scale = 1.0f;
+      dst = os + qs;
+      n = Is;
+    }
+    float acc = 0.f;
+    for (int i = 0; i < n; ++i) acc = fmaf(__ldg(hr + i), __ldg(wr + i), acc);
+    *dst = scale * acc;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------
+static bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                           uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool GATED>
+static cudaError_t launch_tc(const TcParams& prm, int num_sms, cudaStream_t st) {
+  using C = TcCfg<GATED>;
+  auto kern = expert_gemm_tc_kernel<GATED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<num_sms, 192, C::kSmemBytes, st>>>(prm);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  const int64_t P = a.T * a.k;
+  const bool has_shared = a.Is > 0;
+  if (!a.bf16) {
+    const int64_t n1 = P * a.I + (has_shared ? a.T * a.Is : 0);
+    gate_up_f32_kernel<<<static_cast<unsigned>(std::min<int64_t>((n1 + 255) / 256, 148 * 32)), 256, 0, st>>>(
+        static_cast<const float*>(a.x_perm), static_cast<const float*>(a.x), a.offsets,
+        static_cast<const float*>(a.Wgu), static_cast<const float*>(a.Wsgu), P,
+        has_shared ? a.T : 0, a.H, a.E, a.I, a.Is, static_cast<float*>(a.h),
+        static_cast<float*>(a.h_shared));
+    count_launches(2);
+    if (a.stage_mark) a.stage_mark(a.stage_mark_ctx, 3, st);
+    const int64_t n2 = P * a.H + (has_shared ? a.T * a.H : 0);
+    down_f32_kernel<<<static_cast<unsigned>(std::min<int64_t>((n2 + 255) / 256, 148 * 32)), 256, 0, st>>>(
+        static_cast<const float*>(a.h), static_cast<const float*>(a.h_shared), a.offsets, a.row_w,
+        static_cast<const float*>(a.Wd), static_cast<const float*>(a.Wsd), P,
+        has_shared ? a.T : 0, a.H, a.E, a.I, a.Is, static_cast<float*>(a.o),
+        static_cast<float*>(a.o_shared));
+    return cudaGetLastError();
+  }
+  const int G = a.E + (has_shared ? 1 : 0);
+  // gate/up: A = W_gate_up viewed as [E*2I, H]; B = x_perm [P, H] (shared: x [T, H])
+  TcParams g{};
+  bool ok = encode_2d_bf16(&g.tmA[0], a.Wgu, static_cast<uint64_t>(a.E) * 2 * a.I, a.H, kTileM) &&
+            encode_2d_bf16(&g.tmB[0], a.x_perm, P, a.H, kTileN);
+  if (has_shared)
+    ok = ok && encode_2d_bf16(&g.tmA[1], a.Wsgu, 2ull * a.Is, a.H, kTileM) &&
+         encode_2d_bf16(&g.tmB[1], a.x, a.T, a.H, kTileN);
+  else {
+    g.tmA[1] = g.tmA[0];
+    g.tmB[1] = g.tmB[0];
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  g.offsets = a.offsets;
+  g.group_order = a.group_order;
+  g.item_start = a.item_start_gu;
+  g.row_w = a.row_w;
+  g.out[0] = static_cast<__nv_bfloat16*>(a.h);
+  g.out[1] = static_cast<__nv_bfloat16*>(a.h_shared);
+  g.E = a.E;
+  g.G = G;
+  g.T = a.T;
+  g.kblocks[0] = g.kblocks[1] = a.H / kTileK;
+  g.a_rows_per_group = 2 * a.I;
+  g.a_up_offset[0] = a.I;
+  g.a_up_offset[1] = a.Is;
+  g.mt[0] = a.I / kTileM;
+  g.mt[1] = a.Is / kTileM;
+  g.rows_out[0] = static_cast<int>(P);
+  g.rows_out[1] = static_cast<int>(a.T);
+  g.max_items = static_cast<int>(g.mt[0] * (P / kTileN + a.E + 1) + g.mt[1] * (a.T / kTileN + 1) + 1);
+  g.ctrl = a.ctrl;
+  g.ld_out[0] = a.I;
+  g.ld_out[1] = a.Is;
+  cudaError_t e = launch_tc<true>(g, a.num_sms, st);
+  if (e != cudaSuccess) return e;
+  if (a.stage_mark) a.stage_mark(a.stage_mark_ctx, 3, st);
+  // down: A = W_down viewed as [E*H, I]; B = h [P, I] (shared: Ws_down [H, Is], h_shared)
+  TcParams d{};
+  ok = encode_2d_bf16(&d.tmA[0], a.Wd, static_cast<uint64_t>(a.E) * a.H, a.I, kTileM) &&
+       encode_2d_bf16(&d.tmB[0], a.h, P, a.I, kTileN);
+  if (has_shared)
+    ok = ok && encode_2d_bf16(&d.tmA[1], a.Wsd, a.H, a.Is, kTileM) &&
+         encode_2d_bf16(&d.tmB[1], a.h_shared, a.T, a.Is, kTileN);
+  else {
+    d.tmA[1] = d.tmA[0];
+    d.tmB[1] = d.tmB[0];
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  d.offsets = a.offsets;
+  d.group_order = a.group_order;
+  d.item_start = a.item_start_dn;
+  d.row_w = a.row_w;
+  d.out[0] = static_cast<__nv_bfloat16*>(a.o);
+  d.out[1] = static_cast<__nv_bfloat16*>(a.o_shared);
+  d.ld_out[0] = d.ld_out[1] = a.H;
+  d.E = a.E;
+  d.G = G;
+  d.T = a.T;
+  d.kblocks[0] = a.I / kTileK;
+  d.kblocks[1] = has_shared ? a.Is / kTileK : 0;
+  d.a_rows_per_group = a.H;
+  d.a_up_offset[0] = d.a_up_offset[1] = 0;
+  d.mt[0] = d.mt[1] = a.H / kTileM;
+  d.rows_out[0] = static_cast<int>(P);
+  d.rows_out[1] = static_cast<int>(a.T);
+  d.max_items = static_cast<int>(d.mt[0] * (P / kTileN + a.E + 1) + d.mt[1] * (a.T / kTileN + 1) + 1);
+  d.ctrl = a.ctrl;
+  return launch_tc<false>(d, a.num_sms, st);
+}
+
+}  // namespace moe

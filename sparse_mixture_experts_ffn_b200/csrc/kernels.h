@@ -1,0 +1,113 @@
+// kernels.h -- host-side launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+struct Ctrl;
+
+// tokens per block of the histogram / permutation kernels
+constexpr int kTokBlock = 256;
+// rows of weights per tcgen05 tile (MMA M) and reduction elements per pipeline stage
+constexpr int kTileM = 128;
+constexpr int kTileK = 64;
+// tokens per tcgen05 tile (MMA N upper bound)
+constexpr int kTileN = 128;
+
+struct RouterArgs {
+  bool bf16;
+  int64_t T;
+  int H, E, k;
+  const void* x;
+  const void* Wr;
+  const float* bias;
+  double* scores64;  // [T, E]
+  double* xnorm;     // [T]
+  double* wnorm;     // [E]
+  int32_t* idx_ws;   // [T, k]
+  float* w_ws;       // [T, k]
+  int32_t* idx_user;
+  float* w_user;
+  Ctrl* ctrl;
+};
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
+
+struct DispatchArgs {
+  bool bf16;
+  int64_t T;
+  int H, E, k;
+  int I, Is;        // expert widths (Is = 0: no shared expert)
+  const void* x;
+  const int32_t* idx;   // [T, k]
+  const float* w;       // [T, k]
+  int32_t* blk_hist;    // [nblk, E]
+  int32_t* counts;      // [E]
+  int32_t* offsets;     // [E + 1]
+  int32_t* group_order;     // [G]   groups sorted by row count, descending
+  int32_t* item_start_gu;   // [G+1] tcgen05 tiles of the gate/up GEMM per group (prefix)
+  int32_t* item_start_dn;   // [G+1] tiles of the down GEMM
+  int32_t* perm;        // [T*k]
+  int32_t* inv_perm;    // [T*k]
+  float* row_w;         // [T*k]
+  int32_t* row_tok;     // [T*k]
+  void* x_perm;         // [T*k, H]
+  int32_t* counts_user;
+  int32_t* offsets_user;
+  int32_t* perm_user;
+  Ctrl* ctrl;
+};
+cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st);
+
+struct ExpertArgs {
+  bool bf16;
+  int64_t T;
+  int H, E, k, I, Is;
+  const void* x;
+  const void* Wgu;   // [E, 2I, H]
+  const void* Wd;    // [E, H, I]
+  const void* Wsgu;  // [2Is, H] or null
+  const void* Wsd;   // [H, Is]
+  const int32_t* offsets;
+  const int32_t* group_order;
+  const int32_t* item_start_gu;
+  const int32_t* item_start_dn;
+  const float* row_w;
+  const void* x_perm;
+  void* h;          // [T*k, I]
+  void* h_shared;   // [T, Is]
+  void* o;          // [T*k, H]
+  void* o_shared;   // [T, H]
+  int num_sms;
+  Ctrl* ctrl;
+  void (*stage_mark)(void* ctx, int stage, cudaStream_t st) = nullptr;  // between the GEMMs
+  void* stage_mark_ctx = nullptr;
+};
+cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st);
+
+struct CombineArgs {
+  bool bf16;
+  int64_t T;
+  int H, k;
+  bool has_shared;
+  const int32_t* inv_perm;
+  const void* o;
+  const void* o_shared;
+  void* y;
+  Ctrl* ctrl;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
+
+// adds n to the process-wide count of kernels launched by this library
+void count_launches(int n);
+
+// resolves cuTensorMapEncodeTiled through the runtime's driver entry point
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+
+}  // namespace moe

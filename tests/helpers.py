@@ -1,0 +1,67 @@
+"""Shared helpers of the test suite: running the CUDA path and the oracle on the same
+seeded inputs, and the parity criteria."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from conftest import to_oracle
+
+# output tolerance of the layer: max|err| <= 2e-2 * max|y_ref| and relative L2 <= 1e-2
+Y_MAX_TOL = 2e-2
+Y_REL_L2_TOL = 1e-2
+# routing weights (fp32) against the oracle's fp64 softmax of the same keys
+W_REL_TOL = 1e-5
+
+
+def y_errors(y_gpu, y_ref: np.ndarray):
+    yg = y_gpu.detach().float().cpu().numpy().astype(np.float64)
+    d = yg - y_ref
+    max_err = float(np.abs(d).max()) if d.size else 0.0
+    scale = float(np.abs(y_ref).max()) if y_ref.size else 0.0
+    rel_l2 = float(np.linalg.norm(d) / max(np.linalg.norm(y_ref), 1e-300)) if d.size else 0.0
+    return max_err, scale, rel_l2
+
+
+def assert_y_close(y_gpu, y_ref: np.ndarray, what=""):
+    max_err, scale, rel_l2 = y_errors(y_gpu, y_ref)
+    assert max_err <= Y_MAX_TOL * scale + 1e-30, f"{what}: max|err| {max_err:.3e} > 2e-2 * {scale:.3e}"
+    assert rel_l2 <= Y_REL_L2_TOL, f"{what}: relative L2 {rel_l2:.3e} > 1e-2"
+    return max_err / max(scale, 1e-300), rel_l2
+
+
+def oracle_arrays(d: dict):
+    return {k: to_oracle(v) if v is not None else None for k, v in d.items()}
+
+
+def oracle_routing(d: dict, top_k: int):
+    """Exact routing of every token by the oracle."""
+    a = oracle_arrays({"x": d["x"], "W_router": d["W_router"]})
+    s = oracle.router_scores(a["x"], a["W_router"])
+    bias = None if d.get("bias") is None else d["bias"].detach().cpu().numpy().astype(np.float32)
+    idx, w, w64 = oracle.route(s, top_k, bias)
+    counts, offsets, perm, inv = oracle.dispatch(idx, d["W_router"].shape[0])
+    return dict(scores=s, idx=idx, w=w, w64=w64, counts=counts, offsets=offsets, perm=perm, inv_perm=inv)
+
+
+def oracle_y(d: dict, routing: dict, tokens=None):
+    a = oracle_arrays({k: d.get(k) for k in ("x", "W_gate_up", "W_down", "Ws_gate_up", "Ws_down")})
+    return oracle.moe_tokens(a["x"], routing["idx"], routing["w64"], a["W_gate_up"], a["W_down"],
+                             a["Ws_gate_up"], a["Ws_down"], tokens=tokens)
+
+
+def assert_routing_exact(r_gpu, r_ref: dict, E: int):
+    idx = r_gpu.topk_idx.cpu().numpy()
+    assert np.array_equal(idx, r_ref["idx"]), (
+        f"topk_idx differs on {int((idx != r_ref['idx']).any(1).sum())} tokens")
+    assert np.array_equal(r_gpu.counts.cpu().numpy(), r_ref["counts"])
+    assert np.array_equal(r_gpu.offsets.cpu().numpy(), r_ref["offsets"])
+    assert np.array_equal(r_gpu.perm.cpu().numpy(), r_ref["perm"])
+    w = r_gpu.topk_w.cpu().numpy().astype(np.float64)
+    rel = np.abs(w - r_ref["w64"]) / np.maximum(np.abs(r_ref["w64"]), 1e-30)
+    assert float(rel.max()) <= W_REL_TOL, f"topk_w relative error {float(rel.max()):.3e}"
+
+
+def to_device(d: dict, device="cuda"):
+    return {k: (v.to(device).contiguous() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}

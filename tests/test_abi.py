@@ -1,0 +1,99 @@
+"""The C-ABI library loads, exports every entry point its header declares, and validates
+its arguments on the host (no device work is enqueued for any of these calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_mixture_experts_ffn_b200 as moe
+from sparse_mixture_experts_ffn_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return moe.load_library()
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^MOE_API\s+[\w\s\*]+?\b(\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) >= set(moe.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def shape(**kw):
+    base = dict(T=4096, H=4096, E=288, I=1280, I_shared=1280, top_k=8, dtype=moe.MOE_BF16)
+    base.update(kw)
+    return moe.MoEShape(base["T"], base["H"], base["E"], base["I"], base["I_shared"], base["top_k"], base["dtype"])
+
+
+def test_workspace_bytes(lib):
+    s = shape()
+    n = moe.workspace_bytes(s)
+    T, H, E, k, I = 4096, 4096, 288, 8, 1280
+    P = T * k
+    # x_perm, h, o (bf16) dominate; everything else is small
+    assert n >= 2 * (P * H + P * I + P * H + T * I + T * H)
+    assert n < 2 * (P * H + P * I + P * H + T * I + T * H) + 64 * 1024 * 1024
+    assert moe.workspace_bytes(shape(T=0)) > 0
+    for bad in (shape(top_k=0), shape(top_k=289), shape(E=0), shape(H=4000), shape(I=1000),
+                shape(I_shared=100), shape(E=1025, top_k=8), shape(dtype=7), shape(T=-1)):
+        assert moe.workspace_bytes(bad) == 0
+    # fp32 accepts any H multiple of 8 and any widths
+    assert moe.workspace_bytes(shape(dtype=moe.MOE_F32, H=72, I=40, I_shared=24)) > 0
+
+
+def test_workspace_layout_is_inside_the_workspace(lib):
+    s = shape(T=100)
+    lay = moe.workspace_layout(s)
+    n = moe.workspace_bytes(s)
+    for off in (lay.x_perm, lay.h, lay.h_shared, lay.o, lay.o_shared, lay.row_w):
+        assert off % 256 == 0 and off < n
+
+
+def call_forward(lib, s, x=16, wr=16, bias=None, wgu=16, wd=16, wsgu=16, wsd=16, y=16, ws=256,
+                 ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = moe.workspace_bytes(s) if moe.workspace_bytes(s) else 1 << 40
+    P = ctypes.c_void_p
+    return lib.moe_layer_forward(ctypes.byref(s), P(x), P(wr), P(bias), P(wgu), P(wd), P(wsgu), P(wsd),
+                                 P(y), None, P(ws), ws_bytes, None)
+
+
+def test_forward_rejects_bad_arguments_before_any_launch(lib):
+    s = shape()
+    # fake, aligned, never dereferenced addresses: every call below fails validation first
+    assert call_forward(lib, s, x=None) == 1
+    assert call_forward(lib, s, y=None) == 1
+    assert call_forward(lib, s, ws=None) == 1
+    assert call_forward(lib, s, x=24) == 1            # misaligned
+    assert call_forward(lib, s, ws=512 + 16) == 1     # workspace not 256-byte aligned
+    assert call_forward(lib, s, bias=18) == 1         # misaligned bias
+    assert call_forward(lib, s, wsgu=None) == 1       # shared expert half given
+    assert call_forward(lib, shape(I_shared=0)) == 1  # shared weights given without width
+    assert call_forward(lib, shape(top_k=0)) == 1
+    assert call_forward(lib, shape(top_k=300)) == 1
+    assert call_forward(lib, shape(H=4000)) == 2
+    assert call_forward(lib, shape(E=2000)) == 2
+    assert call_forward(lib, s, ws_bytes=moe.workspace_bytes(s) - 1) == 3
+    assert call_forward(lib, shape(T=0)) == 0         # empty batch: nothing to do
+    assert call_forward(lib, None if False else shape(dtype=5)) == 1
+
+
+def test_status_strings(lib):
+    for code, name in moe.STATUS_NAMES.items():
+        assert moe.status_string(code).startswith(name)
+    assert moe.status_string(99) == "unknown moe_status"

@@ -1,0 +1,182 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs.  Expert indices, counts, offsets and the permutation must match bit for bit;
+outputs within max|err| <= 2e-2 * max|y_ref| and relative L2 <= 1e-2."""
+import numpy as np
+import pytest
+import torch
+
+import sparse_mixture_experts_ffn_b200 as moe
+from helpers import (assert_routing_exact, assert_y_close, oracle_routing, oracle_y, to_device)
+from sparse_mixture_experts_ffn_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _library():
+    from sparse_mixture_experts_ffn_b200 import build
+    build.build()
+    moe.load_library()
+
+
+def run(d, top_k, **kw):
+    y, r = moe.moe_layer_forward(d["x"], d["W_router"], d["W_gate_up"], d["W_down"], d.get("Ws_gate_up"),
+                                 d.get("Ws_down"), top_k=top_k, router_bias=d.get("bias"), **kw)
+    return y, r
+
+
+def check_full(d, top_k, what):
+    ws = moe.alloc_workspace(moe.make_shape(d["x"].shape[0], d["x"].shape[1], d["W_router"].shape[0],
+                                            d["W_gate_up"].shape[1] // 2,
+                                            0 if d.get("Ws_gate_up") is None else d["Ws_gate_up"].shape[0] // 2,
+                                            top_k, d["x"].dtype), d["x"].device)
+    y, r = run(d, top_k, workspace=ws)
+    assert moe.check_status(ws) == moe.MOE_OK
+    ref = oracle_routing(d, top_k)
+    assert_routing_exact(r, ref, d["W_router"].shape[0])
+    y_ref = oracle_y(d, ref)
+    return assert_y_close(y, y_ref, what), moe.route_stats(ws)
+
+
+SMALL = [
+    dict(T=300, H=256, E=16, top_k=4, I=256, I_shared=256),
+    dict(T=1, H=256, E=16, top_k=4, I=128, I_shared=128),
+    dict(T=129, H=384, E=12, top_k=1, I=128, I_shared=256),
+    dict(T=77, H=256, E=8, top_k=8, I=128, I_shared=128),
+    dict(T=200, H=512, E=40, top_k=6, I=384, I_shared=0),
+    dict(T=1000, H=256, E=64, top_k=8, I=128, I_shared=128),
+]
+
+
+@pytest.mark.parametrize("sz", SMALL, ids=lambda s: "T{T}_H{H}_E{E}_k{top_k}_I{I}_Is{I_shared}".format(**s))
+def test_small_bf16_parity(sz):
+    cfg = inputs.small_config(**sz)
+    d = to_device(inputs.make_inputs(cfg, "cuda", shared=sz["I_shared"] > 0))
+    check_full(d, cfg.top_k, cfg.name)
+
+
+def test_small_bf16_with_router_bias():
+    cfg = inputs.small_config(T=257, H=256, E=32, top_k=4, I=128, I_shared=128)
+    d = inputs.make_inputs(cfg, "cuda")
+    d["bias"] = torch.linspace(-1.0, 1.0, cfg.E, dtype=torch.float32)
+    check_full(to_device(d), cfg.top_k, "bias")
+
+
+def test_tiny_fp32_workload():
+    cfg = inputs.CONFIGS["tiny_f32_t64"]
+    d = to_device(inputs.make_inputs(cfg, "cuda"))
+    check_full(d, cfg.top_k, cfg.name)
+
+
+def test_fp32_ragged_sizes():
+    cfg = inputs.small_config(T=45, H=72, E=10, top_k=3, I=40, I_shared=24, dtype="f32", r_std=0.1)
+    d = to_device(inputs.make_inputs(cfg, "cuda"))
+    check_full(d, cfg.top_k, "fp32 ragged")
+
+
+def test_group_sizes_at_tile_edges():
+    """Top-1 routing forced through the router: expert e gets exactly sizes[e] tokens."""
+    sizes = [0, 1, 15, 16, 17, 127, 128, 129, 255, 257, 2, 0]
+    E, H, I = len(sizes), 256, 128
+    T = sum(sizes)
+    owner = np.concatenate([np.full(n, e) for e, n in enumerate(sizes)])
+    rng = np.random.default_rng(0)
+    owner = owner[rng.permutation(T)]
+    x = torch.randn(T, H) * 0.01
+    x[torch.arange(T), torch.tensor(owner)] += 4.0  # token t points along axis owner[t]
+    Wr = torch.zeros(E, H)
+    Wr[torch.arange(E), torch.arange(E)] = 1.0
+    cfg = inputs.small_config(T=T, H=H, E=E, top_k=1, I=I, I_shared=I)
+    d = inputs.make_inputs(cfg, "cuda")
+    d["x"] = x.to(torch.bfloat16)
+    d["W_router"] = Wr.to(torch.bfloat16)
+    d = to_device(d)
+    y, r = run(d, 1)
+    assert np.array_equal(r.counts.cpu().numpy(), np.array(sizes))
+    ref = oracle_routing(d, 1)
+    assert_routing_exact(r, ref, E)
+    assert_y_close(y, oracle_y(d, ref), "tile edges")
+
+
+def test_ties_and_zero_input():
+    cfg = inputs.small_config(T=64, H=256, E=16, top_k=4, I=128, I_shared=128)
+    d = inputs.make_inputs(cfg, "cuda")
+    d["W_router"][7] = d["W_router"][3]   # exact ties between experts 3 and 7
+    d["W_router"][12] = d["W_router"][3]
+    d["x"][:8] = 0                          # all keys 0: experts 0..3 with weight 1/4
+    d = to_device(d)
+    y, r = run(d, 4)
+    ref = oracle_routing(d, 4)
+    assert_routing_exact(r, ref, cfg.E)
+    assert np.array_equal(r.topk_idx[:8].cpu().numpy(), np.tile(np.arange(4), (8, 1)))
+    assert torch.all(r.topk_w[:8] == 0.25)
+    assert torch.all(y[:8] == 0)
+    assert_y_close(y, oracle_y(d, ref), "ties")
+
+
+def test_empty_batch_is_a_no_op():
+    cfg = inputs.small_config(T=0, H=256, E=16, top_k=4, I=128, I_shared=128)
+    d = to_device(inputs.make_inputs(cfg, "cuda"))
+    y, r = run(d, 4)
+    assert y.shape == (0, 256)
+
+
+def test_repeat_runs_are_bitwise_identical():
+    cfg = inputs.small_config(T=500, H=256, E=32, top_k=8, I=256, I_shared=256)
+    d = to_device(inputs.make_inputs(cfg, "cuda"))
+    y1, r1 = run(d, 8)
+    y2, r2 = run(d, 8)
+    assert torch.equal(y1, y2)
+    assert torch.equal(r1.perm, r2.perm) and torch.equal(r1.topk_w, r2.topk_w)
+
+
+def test_intermediate_activation_matches_oracle():
+    """Per-kernel check of the gate/up GEMM + SiLU*up epilogue on the rows of x_perm."""
+    import oracle
+    from conftest import to_oracle
+    cfg = inputs.small_config(T=150, H=256, E=8, top_k=2, I=256, I_shared=128)
+    d = to_device(inputs.make_inputs(cfg, "cuda"))
+    shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared, cfg.top_k, torch.bfloat16)
+    ws = moe.alloc_workspace(shape, "cuda")
+    y, r = run(d, cfg.top_k, workspace=ws)
+    torch.cuda.synchronize()
+    lay = moe.workspace_layout(shape)
+    P = cfg.T * cfg.top_k
+    h = ws[lay.h:lay.h + P * cfg.I * 2].view(torch.bfloat16).view(P, cfg.I).float().cpu().numpy()
+    perm = r.perm.cpu().numpy()
+    idx = r.topk_idx.cpu().numpy()
+    xo = to_oracle(d["x"])
+    for pos in [0, 1, P // 3, P // 2, P - 1]:
+        a = perm[pos]
+        t, j = a // cfg.top_k, a % cfg.top_k
+        e = idx[t, j]
+        ref = oracle.expert_act(xo[t], to_oracle(d["W_gate_up"][e]))
+        err = np.abs(h[pos] - ref).max() / np.abs(ref).max()
+        assert err < 2e-2, (pos, err)
+
+
+# ------------------------------------------------------------------------------------
+# the full-size workloads
+# ------------------------------------------------------------------------------------
+FULL = ["decode_t4", "decode_t128", "prefill_t4096", "prefill_t16384_skew"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_workload(name):
+    cfg = inputs.CONFIGS[name]
+    d = to_device(inputs.make_inputs(cfg, "cuda"))
+    shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared, cfg.top_k, torch.bfloat16)
+    ws = moe.alloc_workspace(shape, "cuda")
+    y, r = run(d, cfg.top_k, workspace=ws)
+    assert moe.check_status(ws) == moe.MOE_OK
+    stats = moe.route_stats(ws)
+    ref = oracle_routing(d, cfg.top_k)
+    assert_routing_exact(r, ref, cfg.E)
+    if cfg.T <= 128:
+        tokens = np.arange(cfg.T)
+    else:
+        rng = np.random.default_rng(cfg.seed)
+        tokens = np.unique(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 46, replace=False)]))
+    y_ref = oracle_y(d, ref, tokens=tokens)
+    assert_y_close(y[torch.as_tensor(tokens, device=y.device)], y_ref, name)
+    print(name, "route stats", stats)
