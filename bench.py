@@ -239,8 +239,14 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.CONFIGS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--T", type=int, default=None, help="profiling variant: override the token count")
+    ap.add_argument("--E", type=int, default=None, help="profiling variant: override the expert count")
     args = ap.parse_args()
     cfg = inputs.CONFIGS[args.workload]
+    if args.T is not None or args.E is not None:
+        T = cfg.T if args.T is None else args.T
+        E = cfg.E if args.E is None else args.E
+        cfg = inputs.with_sizes(cfg, T=T, E=E, name=f"{cfg.name}[T={T},E={E}]")
     if args.steps is None:
         args.steps = DEFAULT_STEPS.get(cfg.name, 100)
     args.warmup = max(args.warmup, 3)

@@ -119,11 +119,14 @@ MOE_API moe_status moe_layer_check_status(void* workspace, void* stream);
  *   n_refined : (token, expert) scores recomputed in fp64 because their fp32 key was not
  *               certain and could change the chosen set;
  *   n_exact   : scores that needed the exact (integer) dot product after that;
- *   n_tokens_refined : tokens that needed any recomputation.                         */
+ *   n_tokens_refined : tokens that needed any recomputation;
+ *   n_weight_keys : keys of chosen experts recomputed in fp64 so that the routing
+ *               weights are computed from exact (or 1-ulp) keys.                        */
 typedef struct {
   int64_t n_refined;
   int64_t n_exact;
   int64_t n_tokens_refined;
+  int64_t n_weight_keys;
 } moe_route_stats;
 MOE_API moe_status moe_layer_route_stats(void* workspace, moe_route_stats* out, void* stream);
 
@@ -131,10 +134,14 @@ MOE_API moe_status moe_layer_route_stats(void* workspace, moe_route_stats* out, 
  * tests; layout is private and may change between versions).  Sizes in elements:
  *   x_perm [T*top_k, H] dtype, h [T*top_k, I] dtype, h_shared [T, I_shared] dtype,
  *   o [T*top_k, H] dtype, o_shared [T, H] dtype, row_w [T*top_k] fp32 (routing weight
- *   of each row of x_perm/h/o in expert order).  Returns MOE_ERR_INVALID_ARG on a bad
- *   shape. */
+ *   of each row of x_perm/h/o in expert order), scores: the fp64 router score estimates
+ *   before selection.  scores_slice > 0 for tensor-core scoring (bf16): the H products
+ *   are accumulated in fp32 over consecutive slices of scores_slice products and the
+ *   slices added in fp64; scores_slice = 0 means fp64 accumulation.  Token-major [T, E].
+ *   Returns MOE_ERR_INVALID_ARG on a bad shape. */
 typedef struct {
-  size_t x_perm, h, h_shared, o, o_shared, row_w;
+  size_t x_perm, h, h_shared, o, o_shared, row_w, scores;
+  int32_t scores_slice;
 } moe_workspace_layout;
 MOE_API moe_status moe_layer_workspace_layout(const moe_layer_shape* shape, moe_workspace_layout* out);
 

@@ -44,12 +44,13 @@ class MoERoutingOut(ctypes.Structure):
 
 class MoERouteStats(ctypes.Structure):
     _fields_ = [("n_refined", ctypes.c_int64), ("n_exact", ctypes.c_int64),
-                ("n_tokens_refined", ctypes.c_int64)]
+                ("n_tokens_refined", ctypes.c_int64), ("n_weight_keys", ctypes.c_int64)]
 
 
 class MoEWorkspaceLayout(ctypes.Structure):
     _fields_ = [("x_perm", ctypes.c_size_t), ("h", ctypes.c_size_t), ("h_shared", ctypes.c_size_t),
-                ("o", ctypes.c_size_t), ("o_shared", ctypes.c_size_t), ("row_w", ctypes.c_size_t)]
+                ("o", ctypes.c_size_t), ("o_shared", ctypes.c_size_t), ("row_w", ctypes.c_size_t),
+                ("scores", ctypes.c_size_t), ("scores_slice", ctypes.c_int32)]
 
 
 class MoEError(RuntimeError):
@@ -194,7 +195,8 @@ def route_stats(workspace, stream=None) -> dict:
     rc = load_library().moe_layer_route_stats(_ptr(workspace), ctypes.byref(out), ctypes.c_void_p(stream.cuda_stream))
     if rc != MOE_OK:
         raise MoEError(rc, "moe_layer_route_stats")
-    return dict(n_refined=out.n_refined, n_exact=out.n_exact, n_tokens_refined=out.n_tokens_refined)
+    return dict(n_refined=out.n_refined, n_exact=out.n_exact, n_tokens_refined=out.n_tokens_refined,
+                n_weight_keys=out.n_weight_keys)
 
 
 def status_string(status: int) -> str:

@@ -95,9 +95,11 @@ static int num_sms_current_device() {
 static size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
-  size_t ctrl, scores, xnorm, wnorm, idx, w, blk_hist, counts, offsets, group_order,
-      item_start_gu, item_start_dn, perm, inv_perm, row_w, row_tok, x_perm, h, h_shared, o,
-      o_shared, total;
+  size_t ctrl, group_done, tile_done, wss, zero_end, scores, xnorm, wnorm, idx, w, blk_hist, counts,
+      offsets, group_order, item_start_gu, item_start_dn, perm, inv_perm, row_w, row_tok, partial, spill,
+      x_perm, h, h_shared, o, o_shared, total;
+  int bn, ksplit;
+  int64_t max_tiles;
 };
 
 static bool make_layout(const moe_layer_shape* s, Layout& L) {
@@ -112,8 +114,20 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
     off = align256(off + bytes);
     return at;
   };
+  L.bn = choose_tile_n(s->T, s->top_k, s->E);
+  L.ksplit = s->dtype == MOE_BF16 ? choose_ksplit(s->T, s->top_k, s->E, s->I, s->I_shared, L.bn) : 1;
+  L.max_tiles = expert_tile_bound(s->T, s->top_k, s->E, s->I, s->I_shared, L.bn);
+  // control block and counters first: one memset per forward clears them
+  const bool tc_scores = router_scores_f32(*s);
+  const size_t groups = static_cast<size_t>(router_group_counters(s->T));
   L.ctrl = take(sizeof(Ctrl));
+  L.group_done = take(groups * 4);
+  L.tile_done = take(L.ksplit > 1 ? static_cast<size_t>(L.max_tiles) * 4 : 0);
+  // the small-batch router accumulates scores and row sums of squares atomically
+  L.wss = take(tc_scores ? 0 : groups * E * 8);
   L.scores = take(T * E * 8);
+  L.zero_end = tc_scores ? L.scores : off;
+  L.spill = take(T * E * 16);
   L.xnorm = take(T * 8);
   L.wnorm = take(E * 8);
   L.idx = take(P * 4);
@@ -128,6 +142,7 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.inv_perm = take(P * 4);
   L.row_w = take(P * 4);
   L.row_tok = take(P * 4);
+  L.partial = take(L.ksplit > 1 ? static_cast<size_t>(L.max_tiles) * L.ksplit * L.bn * 256 * 4 : 0);
   L.x_perm = take(P * H * es);
   L.h = take(P * I * es);
   L.h_shared = take(T * Is * es);
@@ -142,6 +157,7 @@ static moe_status validate_shape(const moe_layer_shape* s) {
   if (s->dtype != MOE_F32 && s->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (s->T < 0 || s->H < 1 || s->E < 1 || s->I < 1 || s->I_shared < 0) return MOE_ERR_INVALID_ARG;
   if (s->top_k < 1 || s->top_k > s->E) return MOE_ERR_INVALID_ARG;
+  if (s->H > (1 << 20)) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (s->E > 1024) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (s->T * static_cast<int64_t>(s->top_k) >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (static_cast<int64_t>(s->E) * 2 * s->I >= (int64_t(1) << 31) ||
@@ -179,6 +195,8 @@ extern "C" moe_status moe_layer_workspace_layout(const moe_layer_shape* shape,
   out->o = L.o;
   out->o_shared = L.o_shared;
   out->row_w = L.row_w;
+  out->scores = L.scores;
+  out->scores_slice = router_scores_f32(*shape) ? router_slice_len(shape->H) : 0;
   return MOE_OK;
 }
 
@@ -213,7 +231,7 @@ extern "C" moe_status moe_layer_forward(const moe_layer_shape* shape, const void
   const int64_t P = s.T * s.top_k;
   (void)P;
 
-  if (cudaMemsetAsync(ctrl, 0, sizeof(Ctrl), st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(ctrl, 0, L.zero_end, st) != cudaSuccess) return MOE_ERR_CUDA;
   StageMarks marks;
   begin_marks(marks);
   struct EndMarks {
@@ -232,8 +250,11 @@ extern "C" moe_status moe_layer_forward(const moe_layer_shape* shape, const void
   ra.Wr = W_router;
   ra.bias = router_bias;
   ra.scores64 = static_cast<double*>(at(L.scores));
+  ra.wss = static_cast<double*>(at(L.wss));
+  ra.spill = static_cast<float*>(at(L.spill));
   ra.xnorm = static_cast<double*>(at(L.xnorm));
   ra.wnorm = static_cast<double*>(at(L.wnorm));
+  ra.group_done = static_cast<unsigned int*>(at(L.group_done));
   ra.idx_ws = static_cast<int32_t*>(at(L.idx));
   ra.w_ws = static_cast<float*>(at(L.w));
   ra.idx_user = routing ? routing->topk_idx : nullptr;
@@ -250,6 +271,8 @@ extern "C" moe_status moe_layer_forward(const moe_layer_shape* shape, const void
   da.k = s.top_k;
   da.I = s.I;
   da.Is = s.I_shared;
+  da.bn = L.bn;
+  da.ksplit = L.ksplit;
   da.x = x;
   da.idx = ra.idx_ws;
   da.w = ra.w_ws;
@@ -290,6 +313,10 @@ extern "C" moe_status moe_layer_forward(const moe_layer_shape* shape, const void
   ea.item_start_dn = da.item_start_dn;
   ea.row_w = da.row_w;
   ea.x_perm = da.x_perm;
+  ea.bn = L.bn;
+  ea.ksplit = L.ksplit;
+  ea.partial = static_cast<float*>(at(L.partial));
+  ea.tile_done = static_cast<unsigned int*>(at(L.tile_done));
   ea.h = at(L.h);
   ea.h_shared = at(L.h_shared);
   ea.o = at(L.o);
@@ -338,6 +365,7 @@ extern "C" moe_status moe_layer_route_stats(void* workspace, moe_route_stats* ou
   out->n_refined = static_cast<int64_t>(c.n_refined);
   out->n_exact = static_cast<int64_t>(c.n_exact);
   out->n_tokens_refined = static_cast<int64_t>(c.n_tokens_refined);
+  out->n_weight_keys = static_cast<int64_t>(c.n_weight_keys);
   return MOE_OK;
 }
 

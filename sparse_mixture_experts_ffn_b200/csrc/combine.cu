@@ -17,6 +17,7 @@ template <typename T>
 __global__ void combine_kernel(const int32_t* __restrict__ inv_perm, const T* __restrict__ o,
                                const T* __restrict__ o_shared, int64_t Tn, int H, int k,
                                T* __restrict__ y, Ctrl* ctrl) {
+  pdl_wait();
   constexpr int V = Vec16<T>::N;
   const int vpr = H / V;
   const int64_t total = Tn * vpr;
@@ -47,24 +48,26 @@ __global__ void combine_kernel(const int32_t* __restrict__ inv_perm, const T* __
     for (int j = 0; j < V; ++j) out.v[j] = from_f32<T>(acc[j]);
     reinterpret_cast<uint4*>(y + t * H)[v] = *reinterpret_cast<const uint4*>(&out);
   }
+  pdl_trigger();
 }
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   const int64_t vec = a.T * (a.H / (a.bf16 ? 8 : 4));
   const int blocks = static_cast<int>(std::min<int64_t>((vec + 255) / 256, 148 * 16));
+  cudaError_t e;
   if (a.bf16)
-    combine_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
-        a.inv_perm, static_cast<const __nv_bfloat16*>(a.o),
-        a.has_shared ? static_cast<const __nv_bfloat16*>(a.o_shared) : nullptr, a.T, a.H, a.k,
-        static_cast<__nv_bfloat16*>(a.y), a.ctrl);
+    e = launch_pdl(combine_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st, a.inv_perm,
+                   static_cast<const __nv_bfloat16*>(a.o),
+                   a.has_shared ? static_cast<const __nv_bfloat16*>(a.o_shared) : nullptr, a.T, a.H,
+                   a.k, static_cast<__nv_bfloat16*>(a.y), a.ctrl);
   else
-    combine_kernel<float><<<blocks, 256, 0, st>>>(
-        a.inv_perm, static_cast<const float*>(a.o),
-        a.has_shared ? static_cast<const float*>(a.o_shared) : nullptr, a.T, a.H, a.k,
-        static_cast<float*>(a.y), a.ctrl);
+    e = launch_pdl(combine_kernel<float>, dim3(blocks), dim3(256), 0, st, a.inv_perm,
+                   static_cast<const float*>(a.o),
+                   a.has_shared ? static_cast<const float*>(a.o_shared) : nullptr, a.T, a.H, a.k,
+                   static_cast<float*>(a.y), a.ctrl);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace moe

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "moe_layer.h"
 
 namespace moe {
@@ -19,6 +21,7 @@ struct Ctrl {
   unsigned long long n_refined;      // scores recomputed in fp64
   unsigned long long n_exact;        // scores recomputed exactly
   unsigned long long n_tokens_refined;
+  unsigned long long n_weight_keys;  // chosen experts' keys recomputed in fp64 for weights
 };
 
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
@@ -54,6 +57,18 @@ __device__ __forceinline__ Vec16<T> ld16(const T* p) {
   Vec16<T> r;
   *reinterpret_cast<uint4*>(&r) = __ldg(reinterpret_cast<const uint4*>(p));
   return r;
+}
+
+// ---------------------------------------------------------------------------------------
+// programmatic dependent launch: kernels of one forward are launched so that the next
+// one may start its prologue while the previous one drains.  pdl_wait() blocks until every
+// preceding kernel of the stream has completed and its memory is visible; it must come
+// before the first read of anything an earlier kernel wrote.  pdl_trigger() lets the next
+// kernel launch early.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------------------
@@ -203,7 +218,26 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 
 // 32 lanes x 32 bits x 16 columns: thread i of the warp gets columns [col, col+16) of
-// TMEM lane (lane_base + i).
+// TMEM lane (lane_base + i).  The _nowait form needs a tmem_wait_ld() before its
+// registers are read.
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// named barrier among `count` threads (ids 1..15; 0 is __syncthreads)
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* out) {
   uint32_t r[16];
   asm volatile(
@@ -216,6 +250,25 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* out) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) out[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------------------------------
+// host: launch with programmatic stream serialisation (see pdl_wait / pdl_trigger)
+// ---------------------------------------------------------------------------------------
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 }  // namespace moe

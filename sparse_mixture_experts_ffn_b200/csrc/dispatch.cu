@@ -6,6 +6,10 @@
 // config.json": moe_num_experts, moe_top_k): counts[e] = #{(t,j): idx[t,j] = e};
 // offsets[0] = 0, offsets[e+1] = offsets[e] + counts[e]; perm[offsets[e] + r] = t*k + j for
 // the r-th token (ascending t) routed to e; inv_perm is its inverse.
+//
+// Small batches run one single-block kernel (histogram in shared memory, scans, stable
+// placement); large batches a block histogram, a scan kernel and a block-parallel
+// placement.  Both then gather the token rows into expert order.
 #include <algorithm>
 
 #include <cuda_bf16.h>
@@ -22,6 +26,7 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ i
                                                    int k, int E, int32_t* __restrict__ blk_hist,
                                                    Ctrl* ctrl) {
   extern __shared__ int sh_hist[];
+  pdl_wait();
   for (int e = threadIdx.x; e < E; e += blockDim.x) sh_hist[e] = 0;
   __syncthreads();
   const int64_t a0 = static_cast<int64_t>(blockIdx.x) * kTokBlock * k;
@@ -37,6 +42,7 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ i
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     blk_hist[static_cast<int64_t>(blockIdx.x) * E + e] = sh_hist[e];
+  pdl_trigger();
 }
 
 // exclusive scan of up to 2 * blockDim.x values held two per thread; blockDim.x = 1024
@@ -69,48 +75,36 @@ __device__ int block_scan_pair(int v0, int v1, int* warp_tot, int& total) {
   return excl;  // exclusive prefix of v0; v1's is excl + v0
 }
 
-// One block of 1024 threads: per-expert block prefixes, counts, offsets, LPT group
-// order and the tile schedules of both grouped GEMMs.  Group g < E is routed expert g;
-// group E (when present) is the shared expert with all T tokens.
-__global__ void __launch_bounds__(1024) scan_kernel(
-    int64_t T, int k, int E, int nblk, int has_shared, int mt_gu, int mt_gu_shared, int mt_dn,
-    int32_t* __restrict__ blk_hist, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-    int32_t* __restrict__ group_order, int32_t* __restrict__ item_start_gu,
-    int32_t* __restrict__ item_start_dn, int32_t* __restrict__ counts_user,
-    int32_t* __restrict__ offsets_user) {
-  __shared__ int cnt[2048];
-  __shared__ int order[2048];
-  __shared__ int warp_tot[33];
-  const int G = E + (has_shared ? 1 : 0);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = 0;
-    for (int b = 0; b < nblk; ++b) {
-      const int64_t i = static_cast<int64_t>(b) * E + e;
-      const int c = blk_hist[i];
-      blk_hist[i] = run;
-      run += c;
-    }
-    cnt[e] = run;
-    counts[e] = run;
-    if (counts_user) counts_user[e] = run;
-  }
-  if (has_shared && threadIdx.x == 0) cnt[E] = static_cast<int>(T);
-  __syncthreads();
-  // offsets over the routed experts
+struct ScheduleArgs {
+  int64_t T;
+  int E, has_shared, mt_gu, mt_gu_shared, mt_dn, bn, ksplit;
+  int32_t* offsets;
+  int32_t* group_order;
+  int32_t* item_start_gu;
+  int32_t* item_start_dn;
+  int32_t* offsets_user;
+};
+
+// From the group sizes cnt[0..G) (routed experts, then the shared expert with all T
+// tokens): offsets of the routed experts, the largest-first group order and the tile
+// prefix sums of both grouped GEMMs (gate/up tiles counted ksplit times, once per slice
+// of the reduction).  Block of 1024 threads; cnt/order in shared memory.
+__device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* order, int* warp_tot) {
+  const int E = a.E, G = E + (a.has_shared ? 1 : 0);
   {
     const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
     const int v0 = i0 < E ? cnt[i0] : 0, v1 = i1 < E ? cnt[i1] : 0;
     int total;
     const int ex = block_scan_pair(v0, v1, warp_tot, total);
-    if (i0 < E) offsets[i0] = ex;
-    if (i1 < E) offsets[i1] = ex + v0;
-    if (offsets_user) {
-      if (i0 < E) offsets_user[i0] = ex;
-      if (i1 < E) offsets_user[i1] = ex + v0;
+    if (i0 < E) a.offsets[i0] = ex;
+    if (i1 < E) a.offsets[i1] = ex + v0;
+    if (a.offsets_user) {
+      if (i0 < E) a.offsets_user[i0] = ex;
+      if (i1 < E) a.offsets_user[i1] = ex + v0;
     }
     if (threadIdx.x == 0) {
-      offsets[E] = total;
-      if (offsets_user) offsets_user[E] = total;
+      a.offsets[E] = total;
+      if (a.offsets_user) a.offsets_user[E] = total;
     }
   }
   // largest group first: rank by (count desc, index asc)
@@ -124,52 +118,42 @@ __global__ void __launch_bounds__(1024) scan_kernel(
     order[r] = g;
   }
   __syncthreads();
-  for (int r = threadIdx.x; r < G; r += blockDim.x) group_order[r] = order[r];
-  // tile counts per group in that order, then their prefix sums
-  {
-    const int r0 = 2 * threadIdx.x, r1 = r0 + 1;
-    auto tiles = [&](int r, bool gu) -> int {
-      if (r >= G) return 0;
-      const int g = order[r];
-      const int nt = (cnt[g] + kTileN - 1) / kTileN;
-      const int mt = gu ? (g < E ? mt_gu : mt_gu_shared) : mt_dn;
-      return nt * mt;
-    };
-    int total;
-    int a0 = tiles(r0, true), a1 = tiles(r1, true);
-    int ex = block_scan_pair(a0, a1, warp_tot, total);
-    if (r0 < G) item_start_gu[r0] = ex;
-    if (r1 < G) item_start_gu[r1] = ex + a0;
-    if (threadIdx.x == 0) item_start_gu[G] = total;
-    a0 = tiles(r0, false);
-    a1 = tiles(r1, false);
-    ex = block_scan_pair(a0, a1, warp_tot, total);
-    if (r0 < G) item_start_dn[r0] = ex;
-    if (r1 < G) item_start_dn[r1] = ex + a0;
-    if (threadIdx.x == 0) item_start_dn[G] = total;
-  }
+  for (int r = threadIdx.x; r < G; r += blockDim.x) a.group_order[r] = order[r];
+  const int r0 = 2 * threadIdx.x, r1 = r0 + 1;
+  auto tiles = [&](int r, bool gu) -> int {
+    if (r >= G) return 0;
+    const int g = order[r];
+    const int nt = (cnt[g] + a.bn - 1) / a.bn;
+    const int mt = gu ? (g < E ? a.mt_gu : a.mt_gu_shared) * a.ksplit : a.mt_dn;
+    return nt * mt;
+  };
+  int total;
+  int a0 = tiles(r0, true), a1 = tiles(r1, true);
+  int ex = block_scan_pair(a0, a1, warp_tot, total);
+  if (r0 < G) a.item_start_gu[r0] = ex;
+  if (r1 < G) a.item_start_gu[r1] = ex + a0;
+  if (threadIdx.x == 0) a.item_start_gu[G] = total;
+  a0 = tiles(r0, false);
+  a1 = tiles(r1, false);
+  ex = block_scan_pair(a0, a1, warp_tot, total);
+  if (r0 < G) a.item_start_dn[r0] = ex;
+  if (r1 < G) a.item_start_dn[r1] = ex + a0;
+  if (threadIdx.x == 0) a.item_start_dn[G] = total;
 }
 
-// Stable positions: one warp walks its block's assignments in (token, slot) order, 32 at
-// a time; equal experts inside a chunk get consecutive positions in lane order.
-__global__ void __launch_bounds__(256) permute_kernel(
-    const int32_t* __restrict__ idx, const float* __restrict__ w, int64_t T, int k, int E,
-    const int32_t* __restrict__ offsets, const int32_t* __restrict__ blk_hist,
-    int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm, float* __restrict__ row_w,
-    int32_t* __restrict__ row_tok, int32_t* __restrict__ perm_user) {
-  extern __shared__ int base[];
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    base[e] = offsets[e] + blk_hist[static_cast<int64_t>(blockIdx.x) * E + e];
-  __syncthreads();
-  if (threadIdx.x >= 32) return;
-  const int lane = threadIdx.x;
-  const int64_t a0 = static_cast<int64_t>(blockIdx.x) * kTokBlock * k;
-  const int64_t a1 = min64(a0 + static_cast<int64_t>(kTokBlock) * k, T * k);
+// Stable placement of the assignments [a0, a1) by one warp, 32 at a time, in (token,
+// slot) order: equal experts inside a chunk get consecutive positions in lane order.
+// base[e] holds the next free position of expert e and is advanced.
+__device__ void place_assignments(const int32_t* __restrict__ idx, const float* __restrict__ w,
+                                  int64_t a0, int64_t a1, int k, int E, int* base,
+                                  int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
+                                  float* __restrict__ row_w, int32_t* __restrict__ row_tok,
+                                  int32_t* __restrict__ perm_user) {
+  const int lane = threadIdx.x & 31;
   for (int64_t c = a0; c < a1; c += 32) {
     const int64_t a = c + lane;
-    const bool valid = a < a1;
-    int e = valid ? idx[a] : -1;
-    if (e >= E) e = -1;  // reported by hist_kernel
+    int e = (a < a1) ? idx[a] : -1;
+    if (e < 0 || e >= E) e = -1;  // reported by the histogram
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(peers & ((1u << lane) - 1u));
     int pos = 0;
@@ -187,11 +171,129 @@ __global__ void __launch_bounds__(256) permute_kernel(
   }
 }
 
+// One block of 1024 threads: per-expert block prefixes, counts and the schedule.
+__global__ void __launch_bounds__(1024) scan_kernel(ScheduleArgs sa, int k, int nblk,
+                                                    int32_t* __restrict__ blk_hist,
+                                                    int32_t* __restrict__ counts,
+                                                    int32_t* __restrict__ counts_user) {
+  __shared__ int cnt[2048];
+  __shared__ int order[2048];
+  __shared__ int warp_tot[33];
+  pdl_wait();
+  const int E = sa.E;
+  // each warp scans the block counts of one expert at a time (lanes over blocks)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = warp; e < E; e += blockDim.x / 32) {
+    int run = 0;
+    for (int b0 = 0; b0 < nblk; b0 += 32) {
+      const int b = b0 + lane;
+      const int64_t i = static_cast<int64_t>(b) * E + e;
+      const int c = (b < nblk) ? blk_hist[i] : 0;
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (b < nblk) blk_hist[i] = run + incl - c;
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+      cnt[e] = run;
+      counts[e] = run;
+      if (counts_user) counts_user[e] = run;
+    }
+  }
+  if (sa.has_shared && threadIdx.x == 0) cnt[E] = static_cast<int>(sa.T);
+  __syncthreads();
+  build_schedule(sa, cnt, order, warp_tot);
+  pdl_trigger();
+}
+
+// Placement for large batches: block b owns the assignments of tokens [256b, 256b+256);
+// its 8 warps split them into 8 consecutive ranges, count per warp, prefix the counts per
+// expert across warps, then place.
+constexpr int kPermWarps = 8;
+
+__global__ void __launch_bounds__(32 * kPermWarps) permute_kernel(
+    const int32_t* __restrict__ idx, const float* __restrict__ w, int64_t T, int k, int E,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ blk_hist,
+    int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm, float* __restrict__ row_w,
+    int32_t* __restrict__ row_tok, int32_t* __restrict__ perm_user) {
+  extern __shared__ int wcnt[];  // [kPermWarps][E]
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) wcnt[i] = 0;
+  __syncthreads();
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * kTokBlock * k;
+  const int64_t b1 = min64(b0 + static_cast<int64_t>(kTokBlock) * k, T * k);
+  const int64_t per = (((b1 - b0) + kPermWarps - 1) / kPermWarps + 31) / 32 * 32;
+  const int64_t a0 = min64(b0 + warp * per, b1), a1 = min64(a0 + per, b1);
+  int* mine = wcnt + warp * E;
+  for (int64_t a = a0 + lane; a < a1; a += 32) {
+    const int e = idx[a];
+    if (e >= 0 && e < E) atomicAdd(&mine[e], 1);
+  }
+  __syncthreads();
+  // per expert: exclusive prefix across warps, offset by the block's base position
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = offsets[e] + blk_hist[static_cast<int64_t>(blockIdx.x) * E + e];
+    for (int q = 0; q < kPermWarps; ++q) {
+      const int c = wcnt[q * E + e];
+      wcnt[q * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  place_assignments(idx, w, a0, a1, k, E, mine, perm, inv_perm, row_w, row_tok, perm_user);
+  pdl_trigger();
+}
+
+// Small batches: histogram, scans, schedule and placement in one block.
+__global__ void __launch_bounds__(1024) dispatch_small_kernel(
+    ScheduleArgs sa, const int32_t* __restrict__ idx, const float* __restrict__ w, int k,
+    int32_t* __restrict__ counts, int32_t* __restrict__ counts_user, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv_perm, float* __restrict__ row_w, int32_t* __restrict__ row_tok,
+    int32_t* __restrict__ perm_user, Ctrl* ctrl) {
+  __shared__ int cnt[2048];
+  __shared__ int order[2048];
+  __shared__ int base[1024];
+  __shared__ int warp_tot[33];
+  pdl_wait();
+  const int E = sa.E;
+  const int64_t P = sa.T * k;
+  for (int e = threadIdx.x; e < E + 1; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int64_t a = threadIdx.x; a < P; a += blockDim.x) {
+    const int e = idx[a];
+    if (e < 0 || e >= E) {
+      set_status(ctrl, MOE_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    counts[e] = cnt[e];
+    if (counts_user) counts_user[e] = cnt[e];
+  }
+  if (sa.has_shared && threadIdx.x == 0) cnt[E] = static_cast<int>(sa.T);
+  __syncthreads();
+  build_schedule(sa, cnt, order, warp_tot);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) base[e] = sa.offsets[e];
+  __syncthreads();
+  if (threadIdx.x < 32)
+    place_assignments(idx, w, 0, P, k, E, base, perm, inv_perm, row_w, row_tok, perm_user);
+  pdl_trigger();
+}
+
 // x_perm[pos, :] = x[row_tok[pos], :], 16-byte vectors
 template <typename T>
 __global__ void gather_rows_kernel(const T* __restrict__ x, const int32_t* __restrict__ row_tok,
                                    int64_t P, int64_t Tn, int H, T* __restrict__ x_perm,
                                    Ctrl* ctrl) {
+  pdl_wait();
   constexpr int V = Vec16<T>::N;
   const int vpr = H / V;
   const int64_t total = P * vpr;
@@ -207,34 +309,68 @@ __global__ void gather_rows_kernel(const T* __restrict__ x, const int32_t* __res
     const uint4 val = __ldg(reinterpret_cast<const uint4*>(x + t * H) + v);
     reinterpret_cast<uint4*>(x_perm + p * H)[v] = val;
   }
+  pdl_trigger();
 }
+
+// assignments up to which the single-block path is used
+constexpr int64_t kSmallDispatch = 4096;
 
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
-  const int nblk = static_cast<int>((a.T + kTokBlock - 1) / kTokBlock);
-  const size_t smem_e = sizeof(int) * static_cast<size_t>(a.E);
-  hist_kernel<<<nblk, 256, smem_e, st>>>(a.idx, a.T, a.k, a.E, a.blk_hist, a.ctrl);
-  const int mt_gu = a.I / kTileM;
-  const int mt_gu_sh = a.Is / kTileM;
-  const int mt_dn = a.H / kTileM;
-  scan_kernel<<<1, 1024, 0, st>>>(a.T, a.k, a.E, nblk, a.Is > 0 ? 1 : 0, mt_gu, mt_gu_sh, mt_dn,
-                                  a.blk_hist, a.counts, a.offsets, a.group_order, a.item_start_gu,
-                                  a.item_start_dn, a.counts_user, a.offsets_user);
-  permute_kernel<<<nblk, 256, smem_e, st>>>(a.idx, a.w, a.T, a.k, a.E, a.offsets, a.blk_hist,
-                                            a.perm, a.inv_perm, a.row_w, a.row_tok, a.perm_user);
   const int64_t P = a.T * a.k;
+  ScheduleArgs sa{};
+  sa.T = a.T;
+  sa.E = a.E;
+  sa.has_shared = a.Is > 0 ? 1 : 0;
+  sa.mt_gu = a.I / kTileM;
+  sa.mt_gu_shared = a.Is / kTileM;
+  sa.mt_dn = a.H / kTileM;
+  sa.bn = a.bn;
+  sa.ksplit = a.ksplit;
+  sa.offsets = a.offsets;
+  sa.group_order = a.group_order;
+  sa.item_start_gu = a.item_start_gu;
+  sa.item_start_dn = a.item_start_dn;
+  sa.offsets_user = a.offsets_user;
+  cudaError_t e;
+  int launches = 0;
+  if (P <= kSmallDispatch) {
+    e = launch_pdl(dispatch_small_kernel, dim3(1), dim3(1024), 0, st, sa, a.idx, a.w, a.k, a.counts,
+                   a.counts_user, a.perm, a.inv_perm, a.row_w, a.row_tok, a.perm_user, a.ctrl);
+    if (e != cudaSuccess) return e;
+    launches = 1;
+  } else {
+    const int nblk = static_cast<int>((a.T + kTokBlock - 1) / kTokBlock);
+    const size_t smem_e = sizeof(int) * static_cast<size_t>(a.E);
+    e = launch_pdl(hist_kernel, dim3(nblk), dim3(256), smem_e, st, a.idx, a.T, a.k, a.E, a.blk_hist, a.ctrl);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, sa, a.k, nblk, a.blk_hist, a.counts,
+                   a.counts_user);
+    if (e != cudaSuccess) return e;
+    const size_t smem_p = smem_e * kPermWarps;
+    if (smem_p > 48 * 1024) {
+      e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_p));
+      if (e != cudaSuccess) return e;
+    }
+    e = launch_pdl(permute_kernel, dim3(nblk), dim3(32 * kPermWarps), smem_p, st, a.idx, a.w, a.T, a.k,
+                   a.E, static_cast<const int32_t*>(a.offsets), static_cast<const int32_t*>(a.blk_hist),
+                   a.perm, a.inv_perm, a.row_w, a.row_tok, a.perm_user);
+    if (e != cudaSuccess) return e;
+    launches = 3;
+  }
   const int64_t vec = P * (a.H / (a.bf16 ? 8 : 4));
   const int blocks = static_cast<int>(std::min<int64_t>((vec + 255) / 256, 148 * 16));
   if (a.bf16)
-    gather_rows_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(a.x), a.row_tok, P, a.T, a.H,
-        static_cast<__nv_bfloat16*>(a.x_perm), a.ctrl);
+    e = launch_pdl(gather_rows_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st,
+                   static_cast<const __nv_bfloat16*>(a.x), static_cast<const int32_t*>(a.row_tok), P,
+                   a.T, a.H, static_cast<__nv_bfloat16*>(a.x_perm), a.ctrl);
   else
-    gather_rows_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(a.x), a.row_tok,
-                                                      P, a.T, a.H, static_cast<float*>(a.x_perm),
-                                                      a.ctrl);
-  count_launches(4);
-  return cudaGetLastError();
+    e = launch_pdl(gather_rows_kernel<float>, dim3(blocks), dim3(256), 0, st,
+                   static_cast<const float*>(a.x), static_cast<const int32_t*>(a.row_tok), P, a.T, a.H,
+                   static_cast<float*>(a.x_perm), a.ctrl);
+  count_launches(launches + 1);
+  return e;
 }
 
 }  // namespace moe

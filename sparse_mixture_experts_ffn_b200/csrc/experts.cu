@@ -42,22 +42,39 @@ struct TcParams {
   int mt[2];                   // weight row tiles per group, routed and shared
   int rows_out[2];             // rows of out[0] (T*k) and out[1] (T)
   int max_items;               // upper bound of the schedule length (host-computed)
+  int ksplit;                  // gate/up: slices of the reduction per tile (1 = no split)
+  int max_tiles;               // bound of tile ids (split partial buffers)
+  float* partial;              // [max_tiles][ksplit][BN][256] fp32 gate|up partial sums
+  unsigned int* tile_done;     // [max_tiles] slices finished per tile, zero before the launch
   Ctrl* ctrl;
 };
 
-template <bool GATED>
+constexpr int kMaxDynSmem = 232448;  // 227 KB per block on sm_100
+
+template <bool GATED, int BN>
 struct TcCfg {
-  static constexpr int kStages = GATED ? 4 : 6;
-  static constexpr int kABytes = kTileM * kTileK * 2;  // 16 KB
-  static constexpr int kBBytes = kTileN * kTileK * 2;  // 16 KB
+  static constexpr int kABytes = kTileM * kTileK * 2;  // 16 KB of weights per operand tile
+  static constexpr int kBBytes = BN * kTileK * 2;      // token rows
   static constexpr int kStageBytes = (GATED ? 2 : 1) * kABytes + kBBytes;
-  static constexpr int kAccCols = (GATED ? 2 : 1) * kTileN;  // TMEM columns per accumulator
-  static constexpr int kTmemCols = 2 * kAccCols;             // double-buffered
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kStagingBytes = BN * kTileM * 2;  // epilogue tile [BN][128] bf16
+  static constexpr int kAuxBytes = 1024;                 // barriers, TMEM slot, row weights
+  static constexpr int kFit = (kMaxDynSmem - kStagingBytes - 1024 - kAuxBytes) / kStageBytes;
+  static constexpr int kStages = kFit > 12 ? 12 : kFit;
+  static constexpr int kAccCols = (GATED ? 2 : 1) * BN;  // TMEM columns per accumulator
+  static constexpr int kTmemCols = (2 * kAccCols <= 32) ? 32 : (2 * kAccCols <= 64) ? 64
+                                 : (2 * kAccCols <= 128) ? 128 : (2 * kAccCols <= 256) ? 256 : 512;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + kAuxBytes;
+  static_assert(kStages >= 2, "pipeline too shallow");
+  static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(2 * kAccCols <= 512, "accumulators exceed tensor memory");
+  static_assert(kSmemBytes <= kMaxDynSmem, "shared memory budget");
+  static_assert(BN % 16 == 0 && BN <= 128, "tile width");
 };
 
 struct Item {
   int valid;   // 0: the schedule entry is inconsistent (reported; skipped by every role)
+  int ks;      // slice of the reduction (split gate/up tiles), else 0
+  int tile;    // tile id (items of one tile share it)
   int sh;      // 0 routed expert, 1 shared expert
   int g;       // group (expert id, or E for the shared expert)
   int m;       // weight row tile
@@ -65,6 +82,7 @@ struct Item {
   int nvalid;  // tokens in the tile
 };
 
+template <int BN>
 __device__ __forceinline__ Item decode_item(const TcParams& p, int it) {
   int lo = 0, hi = p.G - 1;
   while (lo < hi) {  // last group slot whose first item is <= it
@@ -74,16 +92,21 @@ __device__ __forceinline__ Item decode_item(const TcParams& p, int it) {
   Item r;
   r.g = __ldg(p.group_order + lo);
   r.sh = (r.g == p.E) ? 1 : 0;
-  const int local = it - __ldg(p.item_start + lo);
+  const int ks_n = p.ksplit;
+  const int local_item = it - __ldg(p.item_start + lo);
+  const int local = local_item / ks_n;  // slices of one tile are consecutive items
+  r.ks = local_item - local * ks_n;
+  r.tile = it / ks_n;                   // every group's item count is a multiple of ks_n
   const int base = r.sh ? 0 : __ldg(p.offsets + r.g);
   const int cnt = r.sh ? static_cast<int>(p.T) : __ldg(p.offsets + r.g + 1) - base;
-  const int ntile = (cnt + kTileN - 1) / kTileN;
-  r.m = local / ntile;
+  const int ntile = (cnt + BN - 1) / BN;
+  r.m = ntile > 0 ? local / ntile : 0;
   const int n = local - r.m * ntile;
-  r.row0 = base + n * kTileN;
-  r.nvalid = min(kTileN, cnt - n * kTileN);
+  r.row0 = base + n * BN;
+  r.nvalid = min(BN, cnt - n * BN);
   r.valid = (r.g >= 0 && r.g < p.G && ntile > 0 && r.m >= 0 && r.m < p.mt[r.sh] && r.nvalid >= 1 &&
-             r.row0 >= 0 && r.row0 + r.nvalid <= p.rows_out[r.sh]) ? 1 : 0;
+             r.row0 >= 0 && r.row0 + r.nvalid <= p.rows_out[r.sh] &&
+             (ks_n == 1 || (r.tile >= 0 && r.tile < p.max_tiles))) ? 1 : 0;
   if (!r.valid) {
     r.nvalid = 0;
     r.sh = 0;
@@ -116,19 +139,28 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   }
 }
 
-template <bool GATED>
+// Persistent grouped GEMM: 192 threads, one block per SM.
+//   warp 0      TMA producer (one lane): weight tiles (gate and up for GATED) and token rows
+//   warp 1      allocates tensor memory; one lane issues the tcgen05 MMAs
+//   warps 2..5  epilogue: tensor memory -> registers -> shared staging tile -> global
+// Accumulators are double-buffered in tensor memory, so the epilogue of one tile overlaps
+// the main loop of the next.
+template <bool GATED, int BN>
 __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
-  using C = TcCfg<GATED>;
+  using C = TcCfg<GATED, BN>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   unsigned char* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  __nv_bfloat16* staging = reinterpret_cast<__nv_bfloat16*>(smem + C::kStages * C::kStageBytes);
+  unsigned char* aux = smem + C::kStages * C::kStageBytes + C::kStagingBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(aux);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* sw = reinterpret_cast<float*>(aux + 512);  // [BN] routing weights of the tile rows
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -155,6 +187,7 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
   const int total = schedule_length(p);
 
   if (warp == 0) {
@@ -165,14 +198,15 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
       uint32_t used = 0;  // stages that ever received a copy
       bool ok = true;
       for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-        const Item t = decode_item(p, it);
+        const Item t = decode_item<BN>(p, it);
         if (!t.valid) {
           if (blockIdx.x == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
           continue;
         }
         const int arow = t.sh ? t.m * kTileM : t.g * p.a_rows_per_group + t.m * kTileM;
         const int kb_n = p.kblocks[t.sh];
-        for (int kb = 0; kb < kb_n; ++kb) {
+        const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, p.ctrl, abort_flag)) { ok = false; break; }
           unsigned char* st = smem + stage * C::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
@@ -202,7 +236,7 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-        const Item t = decode_item(p, it);
+        const Item t = decode_item<BN>(p, it);
         if (!t.valid) continue;
         const int n_mma = (t.nvalid + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(kTileM, n_mma);
@@ -210,19 +244,19 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
         tc_fence_after();
         const uint32_t d0 = tmem_base + acc * C::kAccCols;
         const int kb_n = p.kblocks[t.sh];
-        for (int kb = 0; kb < kb_n; ++kb) {
+        const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, p.ctrl, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
           const uint32_t b0 = a0 + (GATED ? 2 : 1) * C::kABytes;
 #pragma unroll
           for (int kk = 0; kk < kTileK / 16; ++kk) {
-            const uint32_t accum = (kb | kk) ? 1u : 0u;
+            const uint32_t accum = (kb != kb0 || kk) ? 1u : 0u;
             const uint64_t bdesc = sw128_kmajor_desc(b0 + kk * 32);
             mma_bf16(d0, sw128_kmajor_desc(a0 + kk * 32), bdesc, idesc, accum);
             if (GATED)
-              mma_bf16(d0 + kTileN, sw128_kmajor_desc(a0 + C::kABytes + kk * 32), bdesc, idesc,
-                       accum);
+              mma_bf16(d0 + BN, sw128_kmajor_desc(a0 + C::kABytes + kk * 32), bdesc, idesc, accum);
           }
           mma_commit(&empty[stage]);
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -238,39 +272,101 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
   } else {
     // ------------------------------- epilogue (warps 2..5) ----------------------------
     const int quarter = warp & 3;  // TMEM lanes this warp may access: 32*quarter ..
-    const int r = quarter * 32 + lane;
+    const int r = quarter * 32 + lane;  // weight row within the tile = output column
+    const int et = threadIdx.x - 64;    // 0..127
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int it = blockIdx.x; it < total; it += gridDim.x) {
-      const Item t = decode_item(p, it);
+      const Item t = decode_item<BN>(p, it);
       if (!t.valid) continue;
+      if (!GATED && et < BN)
+        sw[et] = (t.sh || et >= t.nvalid) ? 1.0f : __ldg(p.row_w + t.row0 + et);
       if (!mbar_wait(&tfull[acc], acc_phase, p.ctrl, abort_flag)) break;
       tc_fence_after();
+      named_bar_sync(1, 128);  // staging free (previous tile copied out), sw visible
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::kAccCols;
-      const int ld = p.ld_out[t.sh];
-      __nv_bfloat16* out = p.out[t.sh] + static_cast<int64_t>(t.row0) * ld + t.m * kTileM + r;
-      for (int c0 = 0; c0 < t.nvalid; c0 += 16) {
-        float v[16];
-        tmem_ld16(trow + c0, v);
-        if (GATED) {
-          float u[16];
-          tmem_ld16(trow + kTileN + c0, u);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = silu_mul(v[j], u[j]);
-        } else if (!t.sh) {
+      if (GATED && p.ksplit > 1) {
+        // this slice's gate|up partial sums -> its own fp32 slab; the last slice of the
+        // tile adds the slabs, applies SiLU(gate)*up and writes the tile
+        float* slab = p.partial + (static_cast<int64_t>(t.tile) * p.ksplit + t.ks) * BN * 256;
+        for (int c0 = 0; c0 < t.nvalid; c0 += 16) {
+          uint32_t a[16], u[16];
+          tmem_ld16_nowait(trow + c0, a);
+          tmem_ld16_nowait(trow + BN + c0, u);
+          tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (c0 + j < t.nvalid) v[j] *= __ldg(p.row_w + t.row0 + c0 + j);
+            if (c0 + j < t.nvalid) {
+              slab[(c0 + j) * 256 + r] = __uint_as_float(a[j]);
+              slab[(c0 + j) * 256 + 128 + r] = __uint_as_float(u[j]);
+            }
         }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (et == 0) sw[0] = (atomicAdd(p.tile_done + t.tile, 1u) == static_cast<unsigned>(p.ksplit - 1)) ? 1.f : 0.f;
+        named_bar_sync(1, 128);
+        const bool last_slice = sw[0] != 0.f;
+        named_bar_sync(1, 128);  // the flag is read by all before it can be rewritten
+        if (!last_slice) continue;  // another slice finishes this tile
+        __threadfence();
+        const float* tile_slabs = p.partial + static_cast<int64_t>(t.tile) * p.ksplit * BN * 256;
+        for (int n = 0; n < t.nvalid; ++n) {
+          float gs = 0.f, us = 0.f;
+          for (int q = 0; q < p.ksplit; ++q) {
+            gs += __ldcg(tile_slabs + (static_cast<int64_t>(q) * BN + n) * 256 + r);
+            us += __ldcg(tile_slabs + (static_cast<int64_t>(q) * BN + n) * 256 + 128 + r);
+          }
+          staging[n * kTileM + r] = __float2bfloat16_rn(silu_mul(gs, us));
+        }
+        named_bar_sync(1, 128);
+        const int ld = p.ld_out[t.sh];
+        __nv_bfloat16* out = p.out[t.sh] + static_cast<int64_t>(t.row0) * ld + t.m * kTileM;
+        const uint4* src = reinterpret_cast<const uint4*>(staging);
+        for (int i = et; i < t.nvalid * 16; i += 128) {
+          const int n = i >> 4, c = i & 15;
+          *reinterpret_cast<uint4*>(out + static_cast<int64_t>(n) * ld + c * 8) = src[n * 16 + c];
+        }
+        named_bar_sync(1, 128);  // staging and sw[0] free for the next tile
+        continue;
+      }
+      for (int c0 = 0; c0 < t.nvalid; c0 += 16) {
+        uint32_t a[16];
+        tmem_ld16_nowait(trow + c0, a);
+        if (GATED) {
+          uint32_t u[16];
+          tmem_ld16_nowait(trow + BN + c0, u);
+          tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (c0 + j < t.nvalid) out[static_cast<int64_t>(c0 + j) * ld] = __float2bfloat16_rn(v[j]);
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < t.nvalid)
+              staging[(c0 + j) * kTileM + r] =
+                  __float2bfloat16_rn(silu_mul(__uint_as_float(a[j]), __uint_as_float(u[j])));
+        } else {
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < t.nvalid)
+              staging[(c0 + j) * kTileM + r] = __float2bfloat16_rn(__uint_as_float(a[j]) * sw[c0 + j]);
+        }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      mbar_arrive(&tempty[acc]);  // the accumulator may be overwritten now
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      named_bar_sync(1, 128);  // staging tile complete
+      // rows of 128 bf16 (256 B) -> out[row0 + n][m*128 ...], 16-byte coalesced stores
+      const int ld = p.ld_out[t.sh];
+      __nv_bfloat16* out = p.out[t.sh] + static_cast<int64_t>(t.row0) * ld + t.m * kTileM;
+      const uint4* src = reinterpret_cast<const uint4*>(staging);
+      for (int i = et; i < t.nvalid * 16; i += 128) {
+        const int n = i >> 4, c = i & 15;
+        *reinterpret_cast<uint4*>(out + static_cast<int64_t>(n) * ld + c * 8) = src[n * 16 + c];
+      }
     }
   }
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -380,16 +476,32 @@ static bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, ui
   return r == CUDA_SUCCESS;
 }
 
-template <bool GATED>
+template <bool GATED, int BN>
 static cudaError_t launch_tc(const TcParams& prm, int num_sms, cudaStream_t st) {
-  using C = TcCfg<GATED>;
-  auto kern = expert_gemm_tc_kernel<GATED>;
+  using C = TcCfg<GATED, BN>;
+  auto kern = expert_gemm_tc_kernel<GATED, BN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<num_sms, 192, C::kSmemBytes, st>>>(prm);
+  e = launch_pdl(kern, dim3(num_sms), dim3(192), static_cast<size_t>(C::kSmemBytes), st, prm);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
+}
+
+template <bool GATED>
+static cudaError_t launch_tc_bn(const TcParams& prm, int bn, int num_sms, cudaStream_t st) {
+  if (bn == 16) return launch_tc<GATED, 16>(prm, num_sms, st);
+  return launch_tc<GATED, 128>(prm, num_sms, st);
+}
+
+// Upper bound of the tiles of one grouped GEMM whose weight matrices have `rows` rows per
+// routed expert and `rows_shared` for the shared one: every touched expert contributes
+// ceil(count / bn) token tiles, with at most min(T*k, E) partial ones.
+int64_t expert_tile_bound(int64_t T, int k, int E, int rows, int rows_shared, int bn) {
+  const int64_t P = T * k;
+  const int64_t routed = (P / bn + std::min<int64_t>(P, E) + 1) * (rows / kTileM);
+  const int64_t shared = rows_shared ? (T / bn + 1) * (rows_shared / kTileM) : 0;
+  return routed + shared + 1;
 }
 
 cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
@@ -417,10 +529,10 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   // gate/up: A = W_gate_up viewed as [E*2I, H]; B = x_perm [P, H] (shared: x [T, H])
   TcParams g{};
   bool ok = encode_2d_bf16(&g.tmA[0], a.Wgu, static_cast<uint64_t>(a.E) * 2 * a.I, a.H, kTileM) &&
-            encode_2d_bf16(&g.tmB[0], a.x_perm, P, a.H, kTileN);
+            encode_2d_bf16(&g.tmB[0], a.x_perm, P, a.H, a.bn);
   if (has_shared)
     ok = ok && encode_2d_bf16(&g.tmA[1], a.Wsgu, 2ull * a.Is, a.H, kTileM) &&
-         encode_2d_bf16(&g.tmB[1], a.x, a.T, a.H, kTileN);
+         encode_2d_bf16(&g.tmB[1], a.x, a.T, a.H, a.bn);
   else {
     g.tmA[1] = g.tmA[0];
     g.tmB[1] = g.tmB[0];
@@ -443,20 +555,24 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   g.mt[1] = a.Is / kTileM;
   g.rows_out[0] = static_cast<int>(P);
   g.rows_out[1] = static_cast<int>(a.T);
-  g.max_items = static_cast<int>(g.mt[0] * (P / kTileN + a.E + 1) + g.mt[1] * (a.T / kTileN + 1) + 1);
+  g.ksplit = a.ksplit;
+  g.max_tiles = static_cast<int>(expert_tile_bound(a.T, a.k, a.E, a.I, a.Is, a.bn));
+  g.max_items = g.max_tiles * a.ksplit;
+  g.partial = a.partial;
+  g.tile_done = a.tile_done;
   g.ctrl = a.ctrl;
   g.ld_out[0] = a.I;
   g.ld_out[1] = a.Is;
-  cudaError_t e = launch_tc<true>(g, a.num_sms, st);
+  cudaError_t e = launch_tc_bn<true>(g, a.bn, a.num_sms, st);
   if (e != cudaSuccess) return e;
   if (a.stage_mark) a.stage_mark(a.stage_mark_ctx, 3, st);
   // down: A = W_down viewed as [E*H, I]; B = h [P, I] (shared: Ws_down [H, Is], h_shared)
   TcParams d{};
   ok = encode_2d_bf16(&d.tmA[0], a.Wd, static_cast<uint64_t>(a.E) * a.H, a.I, kTileM) &&
-       encode_2d_bf16(&d.tmB[0], a.h, P, a.I, kTileN);
+       encode_2d_bf16(&d.tmB[0], a.h, P, a.I, a.bn);
   if (has_shared)
     ok = ok && encode_2d_bf16(&d.tmA[1], a.Wsd, a.H, a.Is, kTileM) &&
-         encode_2d_bf16(&d.tmB[1], a.h_shared, a.T, a.Is, kTileN);
+         encode_2d_bf16(&d.tmB[1], a.h_shared, a.T, a.Is, a.bn);
   else {
     d.tmA[1] = d.tmA[0];
     d.tmB[1] = d.tmB[0];
@@ -479,9 +595,11 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   d.mt[0] = d.mt[1] = a.H / kTileM;
   d.rows_out[0] = static_cast<int>(P);
   d.rows_out[1] = static_cast<int>(a.T);
-  d.max_items = static_cast<int>(d.mt[0] * (P / kTileN + a.E + 1) + d.mt[1] * (a.T / kTileN + 1) + 1);
+  d.ksplit = 1;
+  d.max_tiles = static_cast<int>(expert_tile_bound(a.T, a.k, a.E, a.H, a.Is > 0 ? a.H : 0, a.bn));
+  d.max_items = d.max_tiles;
   d.ctrl = a.ctrl;
-  return launch_tc<false>(d, a.num_sms, st);
+  return launch_tc_bn<false>(d, a.bn, a.num_sms, st);
 }
 
 }  // namespace moe

@@ -5,6 +5,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
+#include "moe_layer.h"
+
 namespace moe {
 
 struct Ctrl;
@@ -14,8 +18,11 @@ constexpr int kTokBlock = 256;
 // rows of weights per tcgen05 tile (MMA M) and reduction elements per pipeline stage
 constexpr int kTileM = 128;
 constexpr int kTileK = 64;
-// tokens per tcgen05 tile (MMA N upper bound)
-constexpr int kTileN = 128;
+// tokens per tcgen05 tile (MMA N upper bound): 16 when experts hold a few tokens each
+// (decode), 128 otherwise
+inline int choose_tile_n(int64_t T, int k, int E) {
+  return (T * k <= static_cast<int64_t>(6) * E) ? 16 : 128;
+}
 
 struct RouterArgs {
   bool bf16;
@@ -24,22 +31,32 @@ struct RouterArgs {
   const void* x;
   const void* Wr;
   const float* bias;
-  double* scores64;  // [T, E]
+  double* scores64;  // [T, E], zero before the forward on the small-batch path
+  double* wss;       // [router_group_counters(T), E] zero before the forward
   double* xnorm;     // [T]
   double* wnorm;     // [E]
+  unsigned int* group_done;  // [router_group_counters(T)], zero before the forward
   int32_t* idx_ws;   // [T, k]
   float* w_ws;       // [T, k]
   int32_t* idx_user;
   float* w_user;
+  float* spill;      // [4, T, E] key state of tokens that need exact dots
   Ctrl* ctrl;
 };
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
+int64_t router_group_counters(int64_t T);
+// whether the router scores of this shape come from the tensor cores (else fp64)
+bool router_scores_f32(const moe_layer_shape& s);
+// products per fp32-accumulated slice of the tensor-core router scores
+int router_slice_len(int H);
 
 struct DispatchArgs {
   bool bf16;
   int64_t T;
   int H, E, k;
   int I, Is;        // expert widths (Is = 0: no shared expert)
+  int bn;           // tokens per GEMM tile
+  int ksplit;       // gate/up reduction slices
   const void* x;
   const int32_t* idx;   // [T, k]
   const float* w;       // [T, k]
@@ -76,6 +93,10 @@ struct ExpertArgs {
   const int32_t* item_start_dn;
   const float* row_w;
   const void* x_perm;
+  int bn;           // tokens per GEMM tile (16 or 128)
+  int ksplit;       // gate/up reduction slices (1, 2 or 4)
+  float* partial;   // split partial sums (ksplit > 1)
+  unsigned int* tile_done;  // per-tile slice counters, zero before the forward
   void* h;          // [T*k, I]
   void* h_shared;   // [T, Is]
   void* o;          // [T*k, H]
@@ -86,6 +107,18 @@ struct ExpertArgs {
   void* stage_mark_ctx = nullptr;
 };
 cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st);
+int64_t expert_tile_bound(int64_t T, int k, int E, int rows, int rows_shared, int bn);
+
+// reduction slices of the gate/up GEMM: split when a 16-token tiling leaves fewer than
+// about six tiles per SM of a 148-SM B200 (small decode batches)
+inline int choose_ksplit(int64_t T, int k, int E, int I, int Is, int bn) {
+  if (bn != 16) return 1;
+  const int64_t touched = std::min<int64_t>(static_cast<int64_t>(T) * k, E);
+  const int64_t tiles = touched * (I / kTileM) + (Is ? ((T + 15) / 16) * (Is / kTileM) : 0);
+  for (int ks = 1; ks < 4; ks *= 2)
+    if (tiles * ks >= 6 * 148) return ks;
+  return 4;
+}
 
 struct CombineArgs {
   bool bf16;

@@ -3,15 +3,21 @@
 // The routing decision must equal the one made on the exact fp32 router score
 // s[t,e] = RN32(sum_h x[t,h] W_r[e,h]) (llm-atlas page "Step-3.5-Flash", table "Champs
 // bruts du config.json": need_fp32_gate true, moe_top_k 8, norm_expert_weight true).
-// A fast score s^ comes with a rigorous bound |s^ - s_real| <= delta; the fp32 key of an
-// expert is then known to lie in [key(s^-delta), key(s^+delta)].  Experts whose interval
-// can matter for the top-k set are recomputed in fp64 (delta ~ 2^-41 relative) and, if
-// that is still not conclusive, with an exact integer dot product.
+// A fast score s^ comes with a rigorous bound |s^ - s_real| <= delta, so the fp32 key of
+// an expert lies in [key(s^ - delta), key(s^ + delta)].  Each candidate is classified as
+// certainly chosen, certainly not chosen, or undecided; only undecided ones are
+// recomputed, in fp64 (delta ~ 2^-41 relative) and, if that is still not conclusive, with
+// an exact integer dot product.
+//
+//   small batches: one fused kernel computes fp64 scores of all experts; the last block
+//                  of each token group to finish selects for those tokens;
+//   large batches: a tcgen05 GEMM (fp32 accumulation) scores, then a selection kernel.
 #include <algorithm>
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <float.h>
+#include <limits.h>
 #include <stdint.h>
 
 #include "common.cuh"
@@ -19,104 +25,85 @@
 
 namespace moe {
 
+constexpr double kU53 = 1.1102230246251565e-16;  // 2^-53
+constexpr double kU23 = 1.1920928955078125e-07;  // 2^-23
+
 // ---------------------------------------------------------------------------------------
 // Upper bounds of row 2-norms, fp64: sqrt(sum v^2) rounded up, with the fp64 summation
 // error (at most n*2^-53 relative for n terms) covered by a factor (1 + 2 n 2^-53).
 // One warp per row.
 // ---------------------------------------------------------------------------------------
+__device__ __forceinline__ double norm_ub_from_sumsq(double ss, int H) {
+  const double infl = __dadd_ru(1.0, __dmul_ru(2.0 * H, kU53));
+  return __dsqrt_ru(__dmul_ru(ss, infl));
+}
+
 template <typename T>
-__global__ void row_norm_ub_kernel(const T* __restrict__ A, int64_t rows, int H,
-                                   double* __restrict__ out) {
-  int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  int lane = threadIdx.x & 31;
-  if (row >= rows) return;
+__device__ double warp_sumsq(const T* __restrict__ p, int H) {
+  const int lane = threadIdx.x & 31;
   constexpr int V = Vec16<T>::N;
-  const T* p = A + row * H;
   double ss = 0.0;
-  for (int v = lane; v < H / V; v += 32) {
-    Vec16<T> a = ld16(p + v * V);
+  const int nv = H / V;
+  for (int vb = lane; vb < nv; vb += 4 * 32) {
+    Vec16<T> a[4];
 #pragma unroll
-    for (int j = 0; j < V; ++j) {
-      double d = static_cast<double>(to_f32(a.v[j]));
-      ss = fma(d, d, ss);
+    for (int u = 0; u < 4; ++u)
+      if (vb + 32 * u < nv) a[u] = ld16(p + (vb + 32 * u) * V);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (vb + 32 * u >= nv) break;
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const double d = static_cast<double>(to_f32(a[u].v[j]));
+        ss = fma(d, d, ss);
+      }
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (lane == 0) {
-    double infl = __dadd_ru(1.0, __dmul_ru(2.0 * H, 1.1102230246251565e-16));  // 2^-53
-    out[row] = __dsqrt_ru(__dmul_ru(ss, infl));
-  }
+  return ss;
 }
 
-// ---------------------------------------------------------------------------------------
-// fp64 router scores: products exact in fp64, fp64 accumulation in any order.
-// One block (256 threads) per (expert, group of TT tokens).
-// ---------------------------------------------------------------------------------------
-template <typename T, int TT>
-__global__ void __launch_bounds__(256) router_scores_f64_kernel(
-    const T* __restrict__ x, const T* __restrict__ Wr, int64_t T_, int H, int E,
-    double* __restrict__ scores) {
-  const int e = blockIdx.x;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.y) * TT;
-  const int nt = static_cast<int>(min64(TT, T_ - t0));
-  constexpr int V = Vec16<T>::N;
-  double acc[TT];
-#pragma unroll
-  for (int t = 0; t < TT; ++t) acc[t] = 0.0;
-  const T* w = Wr + static_cast<size_t>(e) * H;
-  for (int v = threadIdx.x; v < H / V; v += blockDim.x) {
-    Vec16<T> wv = ld16(w + v * V);
-    double wd[V];
-#pragma unroll
-    for (int j = 0; j < V; ++j) wd[j] = static_cast<double>(to_f32(wv.v[j]));
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      if (t < nt) {
-        Vec16<T> xv = ld16(x + (t0 + t) * H + v * V);
-#pragma unroll
-        for (int j = 0; j < V; ++j) acc[t] = fma(static_cast<double>(to_f32(xv.v[j])), wd[j], acc[t]);
-      }
-    }
+// rows [0, rows_a) of A then [0, rows_b) of B, one warp per row
+template <typename T>
+__global__ void row_norm_ub_kernel(const T* __restrict__ A, int64_t rows_a, double* __restrict__ out_a,
+                                   const T* __restrict__ B, int64_t rows_b, double* __restrict__ out_b,
+                                   int H) {
+  pdl_wait();
+  const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (row < rows_a + rows_b) {
+    const bool first = row < rows_a;
+    const int64_t r = first ? row : row - rows_a;
+    const double ss = warp_sumsq((first ? A : B) + r * H, H);
+    if ((threadIdx.x & 31) == 0) (first ? out_a : out_b)[r] = norm_ub_from_sumsq(ss, H);
   }
-  __shared__ double red[8][TT];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int t = 0; t < TT; ++t) {
-    double v = acc[t];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) red[warp][t] = v;
-  }
-  __syncthreads();
-  if (threadIdx.x < nt) {
-    double v = 0.0;
-    for (int w8 = 0; w8 < (blockDim.x >> 5); ++w8) v += red[w8][threadIdx.x];
-    scores[(t0 + threadIdx.x) * E + e] = v;
-  }
+  pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------------------
 // Exact dot product of one (token, expert) pair by one warp, rounded once to fp32.
-// Every bf16/fp32 value is m * 2^q with integer m; each product's integer mantissa is
-// added into an int64 bin for its exponent (fp32 products are split in two 24-bit
-// halves).  Lane 0 then folds the bins into 32-bit limbs, resolves the sign and rounds
-// the integer to the nearest fp32 (ties to even, subnormals included).
+// Every bf16/fp32 value is m * 2^q with an integer m.  Each lane adds its products
+// exactly into a 128-bit fixed-point accumulator anchored 60 bits below its largest
+// product exponent; products further below go straight into int64 exponent bins in
+// shared memory.  The lane accumulators are then added into the bins (three 42-bit
+// pieces each), the bins are folded into 32-bit limbs, and the integer is rounded to the
+// nearest fp32 (ties to even, subnormals included).
 // ---------------------------------------------------------------------------------------
 constexpr int kQMin = -298;               // smallest product exponent (fp32 subnormal^2)
-constexpr int kNBins = 241 - kQMin + 1;   // up to 2^241 (bf16 max^2 / fp32 upper halves)
+constexpr int kQMax = 270;                // largest bin needed (anchor + 84 for bf16 max^2)
+constexpr int kNBins = kQMax - kQMin + 1;
 constexpr int kNLimbs = (kNBins + 31) / 32 + 4;
 
 __device__ __forceinline__ void decode(float v, int& m, int& q) {
-  uint32_t b = __float_as_uint(v);
-  uint32_t ex = (b >> 23) & 0xFF, fr = b & 0x7FFFFF;
+  const uint32_t b = __float_as_uint(v);
+  const uint32_t ex = (b >> 23) & 0xFF, fr = b & 0x7FFFFF;
   m = ex ? static_cast<int>(fr | 0x800000u) : static_cast<int>(fr);
   q = ex ? static_cast<int>(ex) - 150 : -149;
   if (b >> 31) m = -m;
 }
 __device__ __forceinline__ void decode(__nv_bfloat16 v, int& m, int& q) {
-  uint32_t b = __bfloat16_as_ushort(v);
-  uint32_t ex = (b >> 7) & 0xFF, fr = b & 0x7F;
+  const uint32_t b = __bfloat16_as_ushort(v);
+  const uint32_t ex = (b >> 7) & 0xFF, fr = b & 0x7F;
   m = ex ? static_cast<int>(fr | 0x80u) : static_cast<int>(fr);
   q = ex ? static_cast<int>(ex) - 134 : -133;
   if (b >> 15) m = -m;
@@ -135,59 +122,101 @@ __device__ float round_limbs_rn32(const uint32_t* d, int nl, bool negative) {
   auto bit = [&](int i) -> uint32_t { return (i < 0) ? 0u : (d[i >> 5] >> (i & 31)) & 1u; };
   uint32_t mant = 0;
   for (int i = P; i >= lsb; --i) mant = (mant << 1) | bit(i);
-  uint32_t rb = bit(lsb - 1);
+  const uint32_t rb = bit(lsb - 1);
   bool sticky = false;
   const int sb = lsb - 2;  // bits [0, sb] are sticky
   if (sb >= 0) {
     for (int j = 0; j < (sb >> 5); ++j) sticky |= (d[j] != 0);
-    uint32_t partial = d[sb >> 5] & (((sb & 31) == 31) ? 0xFFFFFFFFu : ((2u << (sb & 31)) - 1u));
+    const uint32_t partial =
+        d[sb >> 5] & (((sb & 31) == 31) ? 0xFFFFFFFFu : ((2u << (sb & 31)) - 1u));
     sticky |= (partial != 0);
   }
   if (rb && (sticky || (mant & 1u))) mant += 1;
-  double v = ldexp(static_cast<double>(mant), lsb_exp);
-  float f = (v > static_cast<double>(FLT_MAX)) ? __int_as_float(0x7f800000) : static_cast<float>(v);
+  const double v = ldexp(static_cast<double>(mant), lsb_exp);
+  const float f = (v > static_cast<double>(FLT_MAX)) ? __int_as_float(0x7f800000) : static_cast<float>(v);
   return negative ? -f : f;
 }
 
+__device__ __forceinline__ void bin_add(long long* bins, int q, long long v) {
+  atomicAdd(reinterpret_cast<unsigned long long*>(&bins[q - kQMin]), static_cast<unsigned long long>(v));
+}
+
 template <typename T>
-__device__ float warp_exact_dot_rn32(const T* __restrict__ a, const T* __restrict__ b, int H,
-                                     long long* bins /* kNBins, warp-private smem */) {
+__device__ __noinline__ float warp_exact_dot_rn32(const T* __restrict__ a, const T* __restrict__ b, int H,
+                                     long long* bins /* kNBins, warp-private smem */,
+                                     uint32_t* limbs /* kNLimbs, warp-private smem */) {
   const int lane = threadIdx.x & 31;
   for (int i = lane; i < kNBins; i += 32) bins[i] = 0;
   __syncwarp();
+  // pass 1: this lane's largest product exponent
+  int qmax = INT_MIN;
   for (int h = lane; h < H; h += 32) {
     int m1, q1, m2, q2;
     decode(a[h], m1, q1);
     decode(b[h], m2, q2);
-    long long p = static_cast<long long>(m1) * m2;
-    if (p == 0) continue;
-    const int q = q1 + q2;
-    const long long sg = p < 0 ? -1 : 1;
-    const long long mag = p < 0 ? -p : p;
-    atomicAdd(reinterpret_cast<unsigned long long*>(&bins[q - kQMin]),
-              static_cast<unsigned long long>(sg * (mag & 0xFFFFFF)));
-    if (mag >> 24)
-      atomicAdd(reinterpret_cast<unsigned long long*>(&bins[q + 24 - kQMin]),
-                static_cast<unsigned long long>(sg * (mag >> 24)));
+    if (m1 != 0 && m2 != 0) qmax = max(qmax, q1 + q2);
+  }
+  if (qmax != INT_MIN) {
+    const int anchor = max(qmax - 60, kQMin);
+    __int128 acc = 0;
+    for (int h = lane; h < H; h += 32) {
+      int m1, q1, m2, q2;
+      decode(a[h], m1, q1);
+      decode(b[h], m2, q2);
+      const long long p = static_cast<long long>(m1) * m2;  // |p| < 2^48
+      if (p == 0) continue;
+      const int q = q1 + q2;
+      if (q >= anchor) {
+        acc += static_cast<__int128>(p) << (q - anchor);  // < 2^108 per term, < 2^115 summed
+      } else {  // far below this lane's largest product: straight into the bins
+        const long long sg = p < 0 ? -1 : 1, mag = p < 0 ? -p : p;
+        bin_add(bins, q, sg * (mag & 0xFFFFFF));
+        if (mag >> 24) bin_add(bins, q + 24, sg * (mag >> 24));
+      }
+    }
+    // acc = p0 + p1 2^42 + p2 2^84 with 0 <= p0, p1 < 2^42 (floor semantics)
+    const long long mask42 = (1ll << 42) - 1;
+    const long long p0 = static_cast<long long>(acc & mask42);
+    const __int128 r1 = (acc - p0) >> 42;
+    const long long p1 = static_cast<long long>(r1 & mask42);
+    const long long p2 = static_cast<long long>((r1 - p1) >> 42);
+    if (p0) bin_add(bins, anchor, p0);
+    if (p1) bin_add(bins, anchor + 42, p1);
+    if (p2) bin_add(bins, anchor + 84, p2);
+  }
+  __syncwarp();
+  // limb j = sum of bins 32j .. 32j+31, each shifted into place (lane j computes limb j)
+  __int128 L = 0;
+  for (int j = lane; j < kNLimbs; j += 32) {
+    L = 0;
+    for (int i = 32 * j; i < 32 * j + 32 && i < kNBins; ++i)
+      L += static_cast<__int128>(bins[i]) << (i & 31);
+    // store as 4 x 32-bit two's-complement words next to each other (lane j: words 4j..4j+3)
+    const unsigned __int128 u = static_cast<unsigned __int128>(L);
+    limbs[4 * j + 0] = static_cast<uint32_t>(u);
+    limbs[4 * j + 1] = static_cast<uint32_t>(u >> 32);
+    limbs[4 * j + 2] = static_cast<uint32_t>(u >> 64);
+    limbs[4 * j + 3] = static_cast<uint32_t>(u >> 96);
   }
   __syncwarp();
   float result = 0.0f;
   if (lane == 0) {
-    __int128 L[kNLimbs];
-    for (int j = 0; j < kNLimbs; ++j) L[j] = 0;
-    for (int i = 0; i < kNBins; ++i) L[i >> 5] += static_cast<__int128>(bins[i]) << (i & 31);
     uint32_t d[kNLimbs];
     __int128 carry = 0;
     for (int j = 0; j < kNLimbs; ++j) {
-      __int128 v = L[j] + carry;
+      const unsigned __int128 u = static_cast<unsigned __int128>(limbs[4 * j]) |
+                                  (static_cast<unsigned __int128>(limbs[4 * j + 1]) << 32) |
+                                  (static_cast<unsigned __int128>(limbs[4 * j + 2]) << 64) |
+                                  (static_cast<unsigned __int128>(limbs[4 * j + 3]) << 96);
+      const __int128 v = static_cast<__int128>(u) + carry;
       d[j] = static_cast<uint32_t>(static_cast<unsigned __int128>(v) & 0xFFFFFFFFu);
       carry = v >> 32;  // arithmetic shift: floor division
     }
     const bool negative = (carry < 0);  // carry is 0 or -1: the limbs hold the full value
-    if (negative) {  // two's complement of the limb string
+    if (negative) {                     // two's complement of the limb string
       uint64_t c = 1;
       for (int j = 0; j < kNLimbs; ++j) {
-        uint64_t v = static_cast<uint64_t>(~d[j]) + c;
+        const uint64_t v = static_cast<uint64_t>(~d[j]) + c;
         d[j] = static_cast<uint32_t>(v);
         c = v >> 32;
       }
@@ -198,27 +227,18 @@ __device__ float warp_exact_dot_rn32(const T* __restrict__ a, const T* __restric
   return __shfl_sync(0xffffffffu, result, 0);
 }
 
-template <typename T>
-__device__ double warp_dot_f64(const T* __restrict__ a, const T* __restrict__ b, int H) {
-  const int lane = threadIdx.x & 31;
-  double acc = 0.0;
-  for (int h = lane; h < H; h += 32)
-    acc = fma(static_cast<double>(to_f32(a[h])), static_cast<double>(to_f32(b[h])), acc);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  return acc;
-}
-
 // ---------------------------------------------------------------------------------------
-// Certified selection.  One warp per token.
+// Certified selection of one token by one warp.  Lane l holds experts l, l+32, l+64, ...
+// (EPL of them) in registers: the two ends of each key interval, the best-estimate key
+// and a status.
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t ordered(float f) {
-  uint32_t b = __float_as_uint(f);
+  const uint32_t b = __float_as_uint(f);
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
 __device__ __forceinline__ float key_of(double s, const float* bias, int e) {
-  float s32 = __double2float_rn(s);
+  const float s32 = __double2float_rn(s);
   return bias ? __fadd_rn(s32, bias[e]) : s32;
 }
 
@@ -227,90 +247,374 @@ __device__ __forceinline__ bool better(float ka, int a, float kb, int b) {
   return (ka > kb) || (ka == kb && a < b);
 }
 
-constexpr int kSelectWarps = 4;
+enum : int { ST_OUT = 0, ST_CAND = 1, ST_IN = 2, ST_UNDECIDED = 3 };
 
-template <typename T, typename S>
-__global__ void __launch_bounds__(32 * kSelectWarps) route_select_kernel(
-    const S* __restrict__ scores, double delta_coef, double delta_abs,
-    const double* __restrict__ xnorm, const double* __restrict__ wnorm,
-    const float* __restrict__ bias, const T* __restrict__ x, const T* __restrict__ Wr,
-    int64_t T_, int H, int E, int k, int32_t* __restrict__ idx_ws, float* __restrict__ w_ws,
-    int32_t* __restrict__ idx_user, float* __restrict__ w_user, Ctrl* ctrl) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * kSelectWarps + warp;
-  // per warp: lo[E], hi[E] floats, flags[E] bytes, bins[kNBins] int64
-  const size_t per_warp = (static_cast<size_t>(E) * 9 + 15) / 16 * 16 + sizeof(long long) * kNBins;
-  unsigned char* mine = smem_raw + per_warp * warp;
-  long long* bins = reinterpret_cast<long long*>(mine);
-  float* lo = reinterpret_cast<float*>(mine + sizeof(long long) * kNBins);
-  float* hi = lo + E;
-  unsigned char* flag = reinterpret_cast<unsigned char*>(hi + E);  // 1 = candidate, 2 = chosen
-  if (t >= T_) return;
+// per-warp shared scratch of the exact dot product
+constexpr size_t kExactScratch =
+    ((sizeof(long long) * kNBins + sizeof(uint32_t) * 4 * kNLimbs + 15) / 16) * 16;
 
-  const T* xt = x + t * H;
-  const double nx = xnorm[t];
-  // 1. key intervals
-  for (int e = lane; e < E; e += 32) {
-    const double sh = static_cast<double>(scores[t * E + e]);
-    const double d = __dadd_ru(__dmul_ru(__dmul_ru(delta_coef, nx), wnorm[e]), delta_abs);
-    lo[e] = key_of(__dadd_rd(sh, -d), bias, e);
-    hi[e] = key_of(__dadd_ru(sh, d), bias, e);
+// experts per lane of the register-resident selection
+inline int select_epl(int E) { return E <= 128 ? 4 : (E <= 384 ? 12 : 32); }
+
+// register-array access with a run-time index, without spilling the array to memory
+template <int EPL, typename V>
+__device__ __forceinline__ V pick(const V (&a)[EPL], int i) {
+  V r = a[0];
+#pragma unroll
+  for (int j = 1; j < EPL; ++j)
+    if (j == i) r = a[j];
+  return r;
+}
+template <int EPL, typename V>
+__device__ __forceinline__ void put(V (&a)[EPL], int i, V v) {
+#pragma unroll
+  for (int j = 0; j < EPL; ++j)
+    if (j == i) a[j] = v;
+}
+
+// fp64 dot with four 16-byte loads per operand in flight per lane
+template <typename T>
+__device__ double warp_dot_f64_prefetch(const T* __restrict__ a, const T* __restrict__ b, int H) {
+  const int lane = threadIdx.x & 31;
+  constexpr int V = Vec16<T>::N;
+  const int nv = H / V;
+  double acc = 0.0;
+  int v = lane;
+  for (; v + 96 < nv; v += 128) {
+    Vec16<T> av[4], bv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      av[u] = ld16(a + (v + 32 * u) * V);
+      bv[u] = ld16(b + (v + 32 * u) * V);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int j = 0; j < V; ++j)
+        acc = fma(static_cast<double>(to_f32(av[u].v[j])), static_cast<double>(to_f32(bv[u].v[j])), acc);
   }
-  __syncwarp();
-  // 2. Lk = k-th largest lower bound: largest u with #{e : ordered(lo_e) >= u} >= k
-  uint32_t u = 0;
-  for (int bitpos = 31; bitpos >= 0; --bitpos) {
-    const uint32_t cand = u | (1u << bitpos);
-    int c = 0;
-    for (int e = lane; e < E; e += 32) c += (ordered(lo[e]) >= cand);
-    c = __reduce_add_sync(0xffffffffu, c);
-    if (c >= k) u = cand;
+  for (; v < nv; v += 32) {
+    const Vec16<T> av = ld16(a + v * V), bv = ld16(b + v * V);
+#pragma unroll
+    for (int j = 0; j < V; ++j)
+      acc = fma(static_cast<double>(to_f32(av.v[j])), static_cast<double>(to_f32(bv.v[j])), acc);
   }
-  // 3. candidates: hi_e >= Lk; everything else is beaten by >= k experts for certain
-  for (int e = lane; e < E; e += 32) flag[e] = (ordered(hi[e]) >= u) ? 1 : 0;
-  __syncwarp();
-  // 4. recompute the candidates whose key is not yet certain
-  int n_ref = 0, n_exact = 0;
-  for (int base = 0; base < E; base += 32) {
-    const int e = base + lane;
-    const bool need = (e < E) && flag[e] && (lo[e] != hi[e]);
-    unsigned mask = __ballot_sync(0xffffffffu, need);
-    while (mask) {
-      const int src = __ffs(mask) - 1;
-      mask &= mask - 1;
-      const int ee = base + src;
-      const T* we = Wr + static_cast<size_t>(ee) * H;
-      float klo, khi;
-      if constexpr (sizeof(S) == 4) {  // scores came from the fp32 pass: fp64 recompute first
-        const double s64 = warp_dot_f64(xt, we, H);
-        const double d = __dmul_ru(__dmul_ru(1.01 * H * 1.1102230246251565e-16, nx), wnorm[ee]);
-        klo = key_of(__dadd_rd(s64, -d), bias, ee);
-        khi = key_of(__dadd_ru(s64, d), bias, ee);
-        ++n_ref;
-      } else {
-        klo = lo[ee];
-        khi = hi[ee];
-      }
-      if (klo != khi) {
-        const float s32 = warp_exact_dot_rn32(xt, we, H, bins);
-        klo = khi = bias ? __fadd_rn(s32, bias[ee]) : s32;
-        ++n_exact;
-      }
-      if (lane == 0) {
-        lo[ee] = klo;
-        hi[ee] = khi;
-      }
-      __syncwarp();
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc;
+}
+
+// srow: score estimates of the token (fp64 values); |s^ - s| <= delta_coef ||x|| ||w_e||
+// + delta_abs.  refine_f64: recompute undecided candidates in fp64 before the exact pass
+// (the estimates are not fp64-accurate).  Norms ||w_e||: wnorm[e], or computed from the
+// sums of squares wss[e] when wss is given.
+// Fast path of the selection of one token by one warp.
+// srow: score estimates of the token (fp64 values), |s^ - s| <= delta_coef ||x|| ||w_e||
+// + delta_abs.  refine_f64: recompute undecided candidates in fp64 (the estimates are
+// not fp64 sums).  Norms ||w_e||: wnorm[e], or from the sums of squares wss[e].
+//   1. lower key bounds lo_e in registers (lane l holds experts l, l+32, ...);
+//   2. Lk, the k-th largest lower bound, by k rounds of warp max-extraction;
+//   3. candidates hi_e >= Lk compacted, in ascending expert order, into a 32-entry list
+//      in shared memory (only they can be chosen, and a candidate can only be beaten for
+//      certain by candidates);
+//   4. lane j classifies candidate j: chosen for certain if fewer than k candidates can be
+//      ranked before it, rejected for certain if k are ranked before it for certain;
+//   5. undecided ones are recomputed in fp64 by the whole warp, then classified again;
+//   6. open slots, renormalised softmax, outputs.
+// Returns false, writing nothing, if more than 32 candidates remain or a key is still
+// undecided; select_token_slow() then redoes the token.
+struct CandList {
+  int e[32];
+  float lo[32], hi[32], mid[32];
+};
+
+template <typename T, int EPL>
+__device__ __forceinline__ bool select_token(const double* __restrict__ srow, double delta_coef,
+                                             double delta_abs, bool refine_f64, double nx,
+                                             const double* __restrict__ wnorm,
+                                             const double* __restrict__ wss,
+                                             const float* __restrict__ bias, const T* __restrict__ xt,
+                                             const T* __restrict__ Wr, int H, int E, int k, int64_t t,
+                                             int32_t* __restrict__ idx_ws, float* __restrict__ w_ws,
+                                             int32_t* __restrict__ idx_user, float* __restrict__ w_user,
+                                             CandList& C, Ctrl* ctrl) {
+  const int lane = threadIdx.x & 31;
+  auto nw = [&](int e) -> double { return wss ? norm_ub_from_sumsq(wss[e], H) : wnorm[e]; };
+  const double cdx = __dmul_ru(delta_coef, nx);
+  // 1. lower bounds
+  uint32_t u[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    u[i] = 0;
+    if (e < E) {
+      const double d = __dadd_ru(__dmul_ru(cdx, nw(e)), delta_abs);
+      u[i] = ordered(key_of(__dadd_rd(srow[e], -d), bias, e));
     }
   }
-  // 5. pick the top k candidates by (key desc, index asc); all their keys are exact now
-  for (int j = 0; j < k; ++j) {
+  // 2. Lk
+  uint32_t lk = 0;
+  {
+    uint32_t taken = 0;
+    for (int r = 0; r < k; ++r) {
+      uint32_t best = 0;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i)
+        if (!(taken & (1u << i))) best = max(best, u[i]);
+      const uint32_t gbest = __reduce_max_sync(0xffffffffu, best);
+      const unsigned holders = __ballot_sync(0xffffffffu, best == gbest);
+      if (lane == __ffs(holders) - 1) {
+        bool done = false;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+          if (!done && !(taken & (1u << i)) && u[i] == gbest) {
+            taken |= 1u << i;
+            done = true;
+          }
+      }
+      lk = gbest;
+    }
+  }
+  // 3. candidates, compacted in ascending expert order
+  int cn = 0;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    float lo = 0.f, hi = 0.f, mid = 0.f;
+    bool cand = false;
+    if (e < E) {
+      const double sh = srow[e];
+      const double d = __dadd_ru(__dmul_ru(cdx, nw(e)), delta_abs);
+      hi = key_of(__dadd_ru(sh, d), bias, e);
+      cand = ordered(hi) >= lk;
+      if (cand) {
+        lo = key_of(__dadd_rd(sh, -d), bias, e);
+        mid = key_of(sh, bias, e);
+      }
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, cand);
+    const int pos = cn + __popc(m & ((1u << lane) - 1u));
+    if (cand && pos < 32) {
+      C.e[pos] = e;
+      C.lo[pos] = lo;
+      C.hi[pos] = hi;
+      C.mid[pos] = mid;
+    }
+    cn += __popc(m);
+  }
+  if (cn > 32) return false;
+  __syncwarp();
+  // 4. classification, lane j <-> candidate j
+  const bool mine = lane < cn;
+  const int my_e = mine ? C.e[lane] : 0;
+  float my_lo = mine ? C.lo[lane] : 0.f, my_hi = mine ? C.hi[lane] : 0.f, my_mid = mine ? C.mid[lane] : 0.f;
+  auto classify_mine = [&]() -> int {
+    int cp = 0, cc = 0;
+    for (int j = 0; j < cn; ++j) {
+      if (j == lane) continue;
+      const int f = C.e[j];
+      const float hf = C.hi[j], lf = C.lo[j];
+      cp += (hf > my_lo) || (hf == my_lo && f < my_e);
+      cc += (lf > my_hi) || (lf == my_hi && f < my_e);
+    }
+    return (cp < k) ? ST_IN : (cc >= k ? ST_OUT : ST_UNDECIDED);
+  };
+  int st = mine ? classify_mine() : ST_OUT;
+  // 5. fp64 recompute of the undecided candidates
+  int n_ref = 0;
+  if (refine_f64) {
+    unsigned need = __ballot_sync(0xffffffffu, st == ST_UNDECIDED && my_lo != my_hi);
+    if (need) {
+      while (need) {
+        const int src = __ffs(need) - 1;
+        need &= need - 1;
+        const int e = __shfl_sync(0xffffffffu, my_e, src);
+        const double s64 = warp_dot_f64_prefetch(xt, Wr + static_cast<size_t>(e) * H, H);
+        if (lane == src) {
+          const double d = __dmul_ru(__dmul_ru(1.01 * H * kU53, nx), nw(e));
+          my_lo = key_of(__dadd_rd(s64, -d), bias, e);
+          my_hi = key_of(__dadd_ru(s64, d), bias, e);
+          my_mid = key_of(s64, bias, e);
+          C.lo[lane] = my_lo;
+          C.hi[lane] = my_hi;
+          C.mid[lane] = my_mid;
+        }
+        ++n_ref;
+      }
+      __syncwarp();
+      st = mine ? classify_mine() : ST_OUT;
+    }
+  }
+  if (__any_sync(0xffffffffu, st == ST_UNDECIDED && my_lo != my_hi)) {
+    if (lane == 0 && n_ref) atomicAdd(&ctrl->n_refined, static_cast<unsigned long long>(n_ref));
+    return false;
+  }
+  // 6. open slots go to the best undecided candidates (their keys are exact)
+  int n_in = __popc(__ballot_sync(0xffffffffu, st == ST_IN));
+  for (int j = n_in; j < k; ++j) {
+    float bk = my_mid;
+    int be = (st == ST_UNDECIDED) ? my_e : -1;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (oe >= 0 && (be < 0 || better(ok, oe, bk, be))) {
+        bk = ok;
+        be = oe;
+      }
+    }
+    if (be < 0) {  // only with non-finite keys (outside the contract)
+      if (lane == 0) set_status(ctrl, MOE_ERR_DEVICE_BOUNDS);
+      break;
+    }
+    if (mine && my_e == be) st = ST_IN;
+  }
+  // 7. renormalised softmax over the chosen keys; outputs in ascending expert order
+  const bool in = st == ST_IN;
+  float m = in ? my_mid : -FLT_MAX;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const float ex = in ? expf(my_mid - m) : 0.0f;
+  float z = ex;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  const unsigned in_mask = __ballot_sync(0xffffffffu, in);
+  if (in) {
+    const int pos = __popc(in_mask & ((1u << lane) - 1u));
+    if (pos < k) {
+      const float w = ex / z;
+      idx_ws[t * k + pos] = my_e;
+      w_ws[t * k + pos] = w;
+      if (idx_user) idx_user[t * k + pos] = my_e;
+      if (w_user) w_user[t * k + pos] = w;
+    }
+  }
+  if (lane == 0) {
+    if (__popc(in_mask) != k) set_status(ctrl, MOE_ERR_DEVICE_BOUNDS);
+    if (n_ref) {
+      atomicAdd(&ctrl->n_refined, static_cast<unsigned long long>(n_ref));
+      atomicAdd(&ctrl->n_tokens_refined, 1ull);
+    }
+  }
+  return true;
+}
+
+// key state of one token in the workspace, for the rare path
+struct KeySpill {
+  float* lo;
+  float* hi;
+  float* mid;
+  int* st;
+};
+
+__device__ __forceinline__ KeySpill key_spill(float* base, int64_t T, int E, int64_t t) {
+  const int64_t n = T * E;
+  KeySpill s;
+  s.lo = base + t * E;
+  s.hi = base + n + t * E;
+  s.mid = base + 2 * n + t * E;
+  s.st = reinterpret_cast<int*>(base + 3 * n) + t * E;
+  return s;
+}
+
+// Rare path: the whole selection of one token with its key state in global memory (one
+// warp): intervals from the score estimates, fp64 recompute (when the estimates are not
+// fp64 sums) and exact dots for what stays undecided, classification, open slots,
+// weights and outputs.
+template <typename T>
+__device__ __noinline__ void select_token_slow(const double* __restrict__ srow, int64_t sstride,
+                                               double delta_coef,
+                                               double delta_abs, bool refine_f64, double nx,
+                                               const double* __restrict__ wnorm,
+                                               const double* __restrict__ wss, KeySpill sp,
+                                               const float* __restrict__ bias,
+                                               const T* __restrict__ xt, const T* __restrict__ Wr,
+                                               int H, int E, int k, int64_t t,
+                                               int32_t* __restrict__ idx_ws, float* __restrict__ w_ws,
+                                               int32_t* __restrict__ idx_user, float* __restrict__ w_user,
+                                               unsigned char* exact_scratch, Ctrl* ctrl) {
+  const int lane = threadIdx.x & 31;
+  auto nw = [&](int e) -> double { return wss ? norm_ub_from_sumsq(wss[e], H) : wnorm[e]; };
+  long long* bins = reinterpret_cast<long long*>(exact_scratch);
+  uint32_t* limbs = reinterpret_cast<uint32_t*>(exact_scratch + sizeof(long long) * kNBins);
+  for (int e = lane; e < E; e += 32) {
+    const double sh = srow[e * sstride];
+    const double d = __dadd_ru(__dmul_ru(__dmul_ru(delta_coef, nx), nw(e)), delta_abs);
+    sp.lo[e] = key_of(__dadd_rd(sh, -d), bias, e);
+    sp.hi[e] = key_of(__dadd_ru(sh, d), bias, e);
+    sp.mid[e] = key_of(sh, bias, e);
+    sp.st[e] = ST_CAND;
+  }
+  __syncwarp();
+  int n_ref = 0, n_exact = 0, n_in = 0;
+  for (int pass = refine_f64 ? 0 : 1; pass < 3; ++pass) {
+    // classify every remaining candidate
+    n_in = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e0 = base + lane;
+      unsigned mask = __ballot_sync(0xffffffffu, e0 < E && sp.st[e0] != ST_OUT);
+      while (mask) {
+        const int e = base + __ffs(mask) - 1;
+        mask &= mask - 1;
+        const float le = sp.lo[e], he = sp.hi[e];
+        int cp = 0, cc = 0;
+        for (int f = lane; f < E; f += 32) {
+          if (f == e) continue;
+          const float hf = sp.hi[f], lf = sp.lo[f];
+          cp += (hf > le) || (hf == le && f < e);
+          cc += (lf > he) || (lf == he && f < e);
+        }
+        cp = __reduce_add_sync(0xffffffffu, cp);
+        cc = __reduce_add_sync(0xffffffffu, cc);
+        const int st = (cp < k) ? ST_IN : (cc >= k ? ST_OUT : ST_UNDECIDED);
+        n_in += (st == ST_IN);
+        __syncwarp();
+        if (lane == 0) sp.st[e] = st;
+        __syncwarp();
+      }
+    }
+    if (pass == 2) break;  // keys of the undecided ones are exact now
+    // recompute the undecided ones whose key is not yet exact: fp64, then exactly
+    for (int base = 0; base < E; base += 32) {
+      const int e0 = base + lane;
+      unsigned mask = __ballot_sync(0xffffffffu, e0 < E && sp.st[e0] == ST_UNDECIDED && sp.lo[e0] != sp.hi[e0]);
+      while (mask) {
+        const int e = base + __ffs(mask) - 1;
+        mask &= mask - 1;
+        const T* we = Wr + static_cast<size_t>(e) * H;
+        float klo, khi, kmid;
+        if (pass == 0) {
+          const double s64 = warp_dot_f64_prefetch(xt, we, H);
+          const double d = __dmul_ru(__dmul_ru(1.01 * H * kU53, nx), nw(e));
+          klo = key_of(__dadd_rd(s64, -d), bias, e);
+          khi = key_of(__dadd_ru(s64, d), bias, e);
+          kmid = key_of(s64, bias, e);
+          ++n_ref;
+        } else {
+          const float s32 = warp_exact_dot_rn32(xt, we, H, bins, limbs);
+          klo = khi = kmid = bias ? __fadd_rn(s32, bias[e]) : s32;
+          ++n_exact;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          sp.lo[e] = klo;
+          sp.hi[e] = khi;
+          sp.mid[e] = kmid;
+        }
+        __syncwarp();
+      }
+    }
+    for (int e = lane; e < E; e += 32)
+      if (sp.st[e] == ST_UNDECIDED) sp.st[e] = ST_CAND;
+    __syncwarp();
+  }
+  // open slots: best undecided by (exact key desc, index asc)
+  for (int j = n_in; j < k; ++j) {
     float bk = 0.0f;
     int be = -1;
     for (int e = lane; e < E; e += 32)
-      if (flag[e] == 1 && (be < 0 || better(lo[e], e, bk, be))) {
-        bk = lo[e];
+      if (sp.st[e] == ST_UNDECIDED && (be < 0 || better(sp.mid[e], e, bk, be))) {
+        bk = sp.mid[e];
         be = e;
       }
 #pragma unroll
@@ -322,41 +626,43 @@ __global__ void __launch_bounds__(32 * kSelectWarps) route_select_kernel(
         be = oe;
       }
     }
-    if (be < 0) {  // only with non-finite keys (outside the contract): stay in bounds
+    if (be < 0) {
       if (lane == 0) set_status(ctrl, MOE_ERR_DEVICE_BOUNDS);
-      for (int e = 0; e < E; ++e)
-        if (flag[e] != 2) { be = e; break; }
+      break;
     }
-    if (lane == 0) flag[be] = 2;
+    __syncwarp();
+    if (lane == 0) sp.st[be] = ST_IN;
     __syncwarp();
   }
-  // 6. renormalised softmax over the chosen keys, fp64; write in ascending expert order
   float m = -FLT_MAX;
   for (int e = lane; e < E; e += 32)
-    if (flag[e] == 2) m = fmaxf(m, lo[e]);
+    if (sp.st[e] == ST_IN) m = fmaxf(m, sp.mid[e]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  double z = 0.0;
+  float z = 0.0f;
   for (int e = lane; e < E; e += 32)
-    if (flag[e] == 2) z += exp(static_cast<double>(lo[e]) - static_cast<double>(m));
+    if (sp.st[e] == ST_IN) z += expf(sp.mid[e] - m);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
   int written = 0;
   for (int base = 0; base < E; base += 32) {
     const int e = base + lane;
-    const bool ch = (e < E) && flag[e] == 2;
+    const bool ch = (e < E) && sp.st[e] == ST_IN;
     const unsigned mask = __ballot_sync(0xffffffffu, ch);
     if (ch) {
       const int pos = written + __popc(mask & ((1u << lane) - 1u));
-      const float w = static_cast<float>(exp(static_cast<double>(lo[e]) - static_cast<double>(m)) / z);
-      idx_ws[t * k + pos] = e;
-      w_ws[t * k + pos] = w;
-      if (idx_user) idx_user[t * k + pos] = e;
-      if (w_user) w_user[t * k + pos] = w;
+      if (pos < k) {
+        const float w = expf(sp.mid[e] - m) / z;
+        idx_ws[t * k + pos] = e;
+        w_ws[t * k + pos] = w;
+        if (idx_user) idx_user[t * k + pos] = e;
+        if (w_user) w_user[t * k + pos] = w;
+      }
     }
     written += __popc(mask);
   }
-  if (lane == 0 && (n_ref | n_exact)) {
+  if (lane == 0) {
+    if (written != k) set_status(ctrl, MOE_ERR_DEVICE_BOUNDS);
     if (n_ref) atomicAdd(&ctrl->n_refined, static_cast<unsigned long long>(n_ref));
     if (n_exact) atomicAdd(&ctrl->n_exact, static_cast<unsigned long long>(n_exact));
     atomicAdd(&ctrl->n_tokens_refined, 1ull);
@@ -364,41 +670,417 @@ __global__ void __launch_bounds__(32 * kSelectWarps) route_select_kernel(
 }
 
 // ---------------------------------------------------------------------------------------
+// Selection kernel for the tensor-core scores: one warp per token.
+// ---------------------------------------------------------------------------------------
+constexpr int kSelectWarps = 4;
+
+template <typename T, int EPL>
+__global__ void __launch_bounds__(32 * kSelectWarps) route_select_kernel(
+    const double* __restrict__ scores, double delta_coef, double delta_abs,
+    const double* __restrict__ xnorm, const double* __restrict__ wnorm,
+    const float* __restrict__ bias, const T* __restrict__ x, const T* __restrict__ Wr,
+    int64_t T_, int H, int E, int k, int32_t* __restrict__ idx_ws, float* __restrict__ w_ws,
+    int32_t* __restrict__ idx_user, float* __restrict__ w_user, float* __restrict__ spill,
+    Ctrl* ctrl) {
+  __shared__ __align__(16) unsigned char exact_scratch[kSelectWarps][kExactScratch];
+  __shared__ CandList cands[kSelectWarps];
+  pdl_wait();
+  const int warp = threadIdx.x >> 5;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kSelectWarps + warp;
+  if (t < T_) {
+    if (!select_token<T, EPL>(scores + t * E, delta_coef, delta_abs, true, xnorm[t], wnorm, nullptr,
+                              bias, x + t * H, Wr, H, E, k, t, idx_ws, w_ws, idx_user, w_user,
+                              cands[warp], ctrl))
+      select_token_slow<T>(scores + t * E, 1, delta_coef, delta_abs, true, xnorm[t], wnorm, nullptr,
+                           key_spill(spill, T_, E, t), bias, x + t * H, Wr, H, E, k, t, idx_ws, w_ws,
+                           idx_user, w_user, exact_scratch[warp], ctrl);
+  }
+  pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------------------
+// Small batches: fused fp64 scores, norms and selection.  Block (b, g, z) adds, for the
+// experts [16b, 16b+16), the tokens [16g, 16g+16) and the z-th quarter of the hidden
+// dimension, the fp64 partial scores into scores[t, e] and the partial sums of squares
+// of W_r rows into wss[g, e] (both zeroed before the launch; products exact in fp64, any
+// summation order).  Warp w owns experts 16b+2w and 16b+2w+1.  The last block of token
+// group g to finish (a counter in the workspace) then selects for the group's tokens, one
+// warp per token.
+// ---------------------------------------------------------------------------------------
+constexpr int kDecodeTok = 16;
+constexpr int kDecodeExp = 16;
+constexpr int kDecodeSplit = 4;
+constexpr int kDecodeThreads = 256;
+
+template <typename T, int EPL>
+__global__ void __launch_bounds__(kDecodeThreads, 1) router_decode_kernel(
+    const T* __restrict__ x, const T* __restrict__ Wr, const float* __restrict__ bias, int64_t T_,
+    int H, int E, int k, double* __restrict__ scores, double* __restrict__ wss,
+    unsigned int* __restrict__ group_done, int32_t* __restrict__ idx_ws, float* __restrict__ w_ws,
+    int32_t* __restrict__ idx_user, float* __restrict__ w_user, float* __restrict__ spill, Ctrl* ctrl) {
+  __shared__ __align__(16) unsigned char exact_scratch[kDecodeThreads / 32][kExactScratch];
+  __shared__ CandList cands[kDecodeThreads / 32];
+  __shared__ int is_last;
+  pdl_wait();
+  const int g = blockIdx.y;
+  const int64_t t0 = static_cast<int64_t>(g) * kDecodeTok;
+  const int nt = static_cast<int>(min64(kDecodeTok, T_ - t0));
+  constexpr int V = Vec16<T>::N;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int e0 = blockIdx.x * kDecodeExp + 2 * warp;
+  const bool has0 = e0 < E, has1 = e0 + 1 < E;
+  const int nv = H / V;
+  const int per = (nv + kDecodeSplit - 1) / kDecodeSplit;
+  const int v_begin = blockIdx.z * per, v_end = min(nv, v_begin + per);
+  double* wss_g = wss + static_cast<int64_t>(g) * E;
+  if (has0) {
+    double acc0[kDecodeTok], acc1[kDecodeTok];
+    double ss0 = 0.0, ss1 = 0.0;
+#pragma unroll
+    for (int j = 0; j < kDecodeTok; ++j) acc0[j] = acc1[j] = 0.0;
+    const T* w0 = Wr + static_cast<size_t>(e0) * H;
+    const T* w1 = Wr + static_cast<size_t>(has1 ? e0 + 1 : e0) * H;
+    for (int vb = v_begin + lane; vb < v_end; vb += 2 * 32) {
+      Vec16<T> a0[2], a1[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int v = vb + 32 * u;
+        if (v < v_end) {
+          a0[u] = ld16(w0 + v * V);
+          a1[u] = ld16(w1 + v * V);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int v = vb + 32 * u;
+        if (v >= v_end) break;
+        double d0[V], d1[V];
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+          d0[j] = static_cast<double>(to_f32(a0[u].v[j]));
+          d1[j] = static_cast<double>(to_f32(a1[u].v[j]));
+          ss0 = fma(d0[j], d0[j], ss0);
+          ss1 = fma(d1[j], d1[j], ss1);
+        }
+#pragma unroll
+        for (int tt = 0; tt < kDecodeTok; ++tt) {
+          if (tt < nt) {
+            const Vec16<T> xv = ld16(x + (t0 + tt) * H + v * V);
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+              const double xd = static_cast<double>(to_f32(xv.v[j]));
+              acc0[tt] = fma(xd, d0[j], acc0[tt]);
+              acc1[tt] = fma(xd, d1[j], acc1[tt]);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      ss0 += __shfl_xor_sync(0xffffffffu, ss0, o);
+      ss1 += __shfl_xor_sync(0xffffffffu, ss1, o);
+#pragma unroll
+      for (int tt = 0; tt < kDecodeTok; ++tt) {
+        acc0[tt] += __shfl_xor_sync(0xffffffffu, acc0[tt], o);
+        acc1[tt] += __shfl_xor_sync(0xffffffffu, acc1[tt], o);
+      }
+    }
+    if (lane == 0) {
+      atomicAdd(&wss_g[e0], ss0);
+      if (has1) atomicAdd(&wss_g[e0 + 1], ss1);
+#pragma unroll
+      for (int tt = 0; tt < kDecodeTok; ++tt) {
+        if (tt < nt) {
+          atomicAdd(&scores[(t0 + tt) * E + e0], acc0[tt]);
+          if (has1) atomicAdd(&scores[(t0 + tt) * E + e0 + 1], acc1[tt]);
+        }
+      }
+    }
+  }
+  // last block of the token group?
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned prev = atomicAdd(&group_done[g], 1u);
+    is_last = (prev == gridDim.x * gridDim.z - 1);
+  }
+  __syncthreads();
+  if (is_last) {
+    __threadfence();
+    for (int tt = warp; tt < nt; tt += kDecodeThreads / 32) {
+      const int64_t t = t0 + tt;
+      const T* xt = x + t * H;
+      const double nx = norm_ub_from_sumsq(warp_sumsq(xt, H), H);
+      // fp64 scores: |s^ - s| <= 1.01 * H * 2^-53 * ||x|| ||w|| (any summation order)
+      if (!select_token<T, EPL>(scores + t * E, 1.01 * H * kU53, 0.0, false, nx, nullptr, wss_g, bias,
+                                xt, Wr, H, E, k, t, idx_ws, w_ws, idx_user, w_user, cands[warp], ctrl))
+        select_token_slow<T>(scores + t * E, 1, 1.01 * H * kU53, 0.0, false, nx, nullptr, wss_g,
+                             key_spill(spill, T_, E, t), bias, xt, Wr, H, E, k, t, idx_ws, w_ws,
+                             idx_user, w_user, exact_scratch[warp], ctrl);
+    }
+  }
+  pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------------------
+// tcgen05 router GEMM.  Block (m, n) scores the tokens [128m, 128m+128) against the
+// experts [64n, 64n+64).  Every slice of kRtSliceSteps 64-product steps of the reduction
+// is accumulated in fp32 in one of two tensor-memory buffers and then drained by the
+// epilogue warps into fp64 registers, so the fp32 accumulation error of each partial is
+// bounded by the slice and the partials add up in fp64.  Only the token rows that exist
+// are loaded (16-row boxes); rows of the A tile beyond them are never read back.
+// Warp 0 issues TMA copies, warp 1 the MMAs, warps 2-5 (one thread per token) drain.
+// ---------------------------------------------------------------------------------------
+constexpr int kRtExperts = 64;
+constexpr int kRtStages = 8;
+constexpr int kRtSliceSteps = 4;                     // slice = 256 products
+constexpr int kRtABytes = kTileM * kTileK * 2;       // 16 KB of x (at most)
+constexpr int kRtBBytes = kRtExperts * kTileK * 2;   // 8 KB of W_router
+constexpr int kRtStageBytes = kRtABytes + kRtBBytes;
+constexpr int kRtSmem = kRtStages * kRtStageBytes + 1024 + 256;
+constexpr int kRtRowBox = 16;                        // token rows per TMA box
+
+struct RouterTcParams {
+  CUtensorMap tmX;   // x [T, H], box {64, 16}
+  CUtensorMap tmW;   // W_router [E, H], box {64, 64}
+  int64_t T;
+  int H, E;
+  double* scores;    // [T, E]
+  Ctrl* ctrl;
+};
+
+__global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_constant__ RouterTcParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  unsigned char* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kRtStages * kRtStageBytes);
+  uint64_t* empty = full + kRtStages;
+  uint64_t* tfull = empty + kRtStages;   // [2]
+  uint64_t* tempty = tfull + 2;          // [2]
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  constexpr uint32_t kCols = 128;  // two 64-column accumulators
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRtStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4 * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTileM;
+  const int e0 = blockIdx.y * kRtExperts;
+  const int ne = min(kRtExperts, p.E - e0);
+  const int kb_n = p.H / kTileK;
+  const int rows = static_cast<int>(min64(kTileM, p.T - t0));
+  const int nbox = (rows + kRtRowBox - 1) / kRtRowBox;
+  pdl_wait();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&p.tmX);
+      tma_prefetch_desc(&p.tmW);
+      const uint32_t bytes = nbox * kRtRowBox * kTileK * 2 + kRtBBytes;
+      int stage = 0;
+      uint32_t phase = 0, used = 0;
+      for (int kb = 0; kb < kb_n; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, p.ctrl, abort_flag)) break;
+        unsigned char* st = smem + stage * kRtStageBytes;
+        mbar_arrive_expect_tx(&full[stage], bytes);
+        for (int b = 0; b < nbox; ++b)
+          tma_load_2d(st + b * kRtRowBox * kTileK * 2, &p.tmX, kb * kTileK,
+                      static_cast<int32_t>(t0 + b * kRtRowBox), &full[stage]);
+        tma_load_2d(st + kRtABytes, &p.tmW, kb * kTileK, e0, &full[stage]);
+        used |= 1u << stage;
+        if (++stage == kRtStages) { stage = 0; phase ^= 1u; }
+      }
+      for (int s = 0; s < kRtStages; ++s)
+        if (used & (1u << s)) {
+          const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+          const uint64_t tw = globaltimer_ns();
+          while (!mbar_try_wait(&full[s], par))
+            if (globaltimer_ns() - tw > kWaitLimitNs) { set_status(p.ctrl, MOE_ERR_DEVICE_TIMEOUT); break; }
+        }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(kTileM, (ne + 15) & ~15);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kb = 0; kb < kb_n; ++kb) {
+        const int sl = kb / kRtSliceSteps;   // slice index
+        const bool first = (kb % kRtSliceSteps) == 0;
+        const bool last = (kb % kRtSliceSteps) == kRtSliceSteps - 1 || kb == kb_n - 1;
+        const int b = sl & 1;
+        if (first && !mbar_wait(&tempty[b], ((sl >> 1) & 1) ^ 1u, p.ctrl, abort_flag)) break;
+        if (!mbar_wait(&full[stage], phase, p.ctrl, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(smem + stage * kRtStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < kTileK / 16; ++kk)
+          mma_bf16(tmem_base + b * kRtExperts, sw128_kmajor_desc(a0 + kk * 32),
+                   sw128_kmajor_desc(a0 + kRtABytes + kk * 32), idesc, (first && kk == 0) ? 0u : 1u);
+        mma_commit(&empty[stage]);
+        if (last) mma_commit(&tfull[b]);
+        if (++stage == kRtStages) { stage = 0; phase ^= 1u; }
+      }
+      mma_commit(drain);
+      const uint64_t tw = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0))
+        if (globaltimer_ns() - tw > kWaitLimitNs) { set_status(p.ctrl, MOE_ERR_DEVICE_TIMEOUT); break; }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int64_t t = t0 + quarter * 32 + lane;
+    double acc[kRtExperts];
+#pragma unroll
+    for (int j = 0; j < kRtExperts; ++j) acc[j] = 0.0;
+    const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    bool ok = true;
+    const int n_sl = (kb_n + kRtSliceSteps - 1) / kRtSliceSteps;
+    for (int sl = 0; sl < n_sl && ok; ++sl) {
+      const int b = sl & 1;
+      if (!mbar_wait(&tfull[b], (sl >> 1) & 1, p.ctrl, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t r[kRtExperts];
+#pragma unroll
+      for (int j0 = 0; j0 < kRtExperts; j0 += 16) tmem_ld16_nowait(trow + b * kRtExperts + j0, r + j0);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < kRtExperts; ++j) acc[j] += static_cast<double>(__uint_as_float(r[j]));
+      tc_fence_before();
+      mbar_arrive(&tempty[b]);
+    }
+    if (ok && t < p.T) {
+      double* dst = p.scores + t * p.E + e0;
+#pragma unroll
+      for (int j = 0; j < kRtExperts; ++j)
+        if (j < ne) dst[j] = acc[j];
+    }
+  }
+  pdl_trigger();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, kCols);
+}
+
+// ---------------------------------------------------------------------------------------
 // host launchers
 // ---------------------------------------------------------------------------------------
-template <typename T>
-static cudaError_t launch_router_f64_t(const RouterArgs& a, cudaStream_t st) {
-  const T* x = static_cast<const T*>(a.x);
-  const T* Wr = static_cast<const T*>(a.Wr);
-  {
-    const int64_t rows = a.T;
-    row_norm_ub_kernel<T><<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, st>>>(x, rows, a.H, a.xnorm);
-    row_norm_ub_kernel<T><<<static_cast<unsigned>((a.E * 32 + 255) / 256), 256, 0, st>>>(Wr, a.E, a.H, a.wnorm);
-  }
-  constexpr int TT = 8;
-  dim3 grid(a.E, static_cast<unsigned>((a.T + TT - 1) / TT));
-  router_scores_f64_kernel<T, TT><<<grid, 256, 0, st>>>(x, Wr, a.T, a.H, a.E, a.scores64);
-  const size_t per_warp = (static_cast<size_t>(a.E) * 9 + 15) / 16 * 16 + sizeof(long long) * kNBins;
-  const size_t smem = per_warp * kSelectWarps;
-  auto kern = route_select_kernel<T, double>;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
-  // fp64 scores: |s^ - s| <= 1.01 * H * 2^-53 * ||x|| ||w|| (any summation order)
-  const double coef = 1.01 * a.H * 1.1102230246251565e-16;
-  kern<<<static_cast<unsigned>((a.T + kSelectWarps - 1) / kSelectWarps), 32 * kSelectWarps, smem, st>>>(
-      a.scores64, coef, 0.0, a.xnorm, a.wnorm, a.bias, x, Wr, a.T, a.H, a.E, a.k, a.idx_ws,
-      a.w_ws, a.idx_user, a.w_user, a.ctrl);
-  count_launches(4);
-  return cudaGetLastError();
+static bool encode_bf16_rows(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                             uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// bf16 batches score on the tensor cores (fp32 accumulation over slices, certified band,
+// fp64 / exact recompute near the top-k boundary); fp32 inputs, or more experts than one
+// tensor-memory row of accumulators allows, score in fp64 on the CUDA cores.
+constexpr int64_t kTcRouterMinTokens = 1;
+
+static bool router_tc_supported(bool bf16, int64_t T, int E, int H) {
+  return bf16 && T >= kTcRouterMinTokens && E <= 512 && H % kTileK == 0;
+}
+
+bool router_scores_f32(const moe_layer_shape& s) {
+  return router_tc_supported(s.dtype == MOE_BF16, s.T, s.E, s.H);
+}
+
+template <typename K>
+static cudaError_t allow_smem(K kern, size_t smem) {
+  if (smem <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+}
+
+int router_slice_len(int /*H*/) { return kRtSliceSteps * kTileK; }
+
+static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
+  using bf16 = __nv_bfloat16;
+  RouterTcParams p{};
+  p.T = a.T;
+  p.H = a.H;
+  p.E = a.E;
+  p.scores = a.scores64;
+  p.ctrl = a.ctrl;
+  if (!encode_bf16_rows(&p.tmX, a.x, a.T, a.H, kRtRowBox) ||
+      !encode_bf16_rows(&p.tmW, a.Wr, a.E, a.H, kRtExperts))
+    return cudaErrorInvalidValue;
+  cudaError_t e = allow_smem(router_gemm_tc_kernel, kRtSmem);
+  if (e != cudaSuccess) return e;
+  const bf16* x = static_cast<const bf16*>(a.x);
+  const bf16* Wr = static_cast<const bf16*>(a.Wr);
+  e = launch_pdl(row_norm_ub_kernel<bf16>, dim3(static_cast<unsigned>(((a.T + a.E) * 32 + 255) / 256)),
+                 dim3(256), 0, st, x, a.T, a.xnorm, Wr, static_cast<int64_t>(a.E), a.wnorm, a.H);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(router_gemm_tc_kernel,
+                 dim3(static_cast<unsigned>((a.T + kTileM - 1) / kTileM), (a.E + kRtExperts - 1) / kRtExperts),
+                 dim3(192), static_cast<size_t>(kRtSmem), st, p);
+  if (e != cudaSuccess) return e;
+  // Each slice of L = 256 products is accumulated in fp32 from exact products, at most
+  // 2^-23 relative per accumulation step (truncation included), so its error is
+  // <= 2 L 2^-23 * sum|x w| over the slice; adding the H/L partials in fp64 costs at most
+  // 2 (H/L) 2^-53 more; H 2^-125 covers partial sums flushed below the normal range.
+  const double slice = static_cast<double>(kRtSliceSteps) * kTileK;
+  const double coef = 2.0 * slice * kU23 + 2.0 * (a.H / slice + 1) * kU53;
+  const unsigned sgrid = static_cast<unsigned>((a.T + kSelectWarps - 1) / kSelectWarps);
+  auto sel = [&](auto kern) {
+    return launch_pdl(kern, dim3(sgrid), dim3(32 * kSelectWarps), 0, st, static_cast<const double*>(a.scores64),
+                      coef, a.H * 2.350988701644575e-38, static_cast<const double*>(a.xnorm),
+                      static_cast<const double*>(a.wnorm), a.bias, x, Wr, a.T, a.H, a.E, a.k, a.idx_ws,
+                      a.w_ws, a.idx_user, a.w_user, a.spill, a.ctrl);
+  };
+  const int epl = select_epl(a.E);
+  e = epl == 4 ? sel(route_select_kernel<bf16, 4>) : epl == 12 ? sel(route_select_kernel<bf16, 12>)
+                                                                : sel(route_select_kernel<bf16, 32>);
+  count_launches(3);
+  return e;
+}
+
+template <typename T>
+static cudaError_t launch_router_decode(const RouterArgs& a, cudaStream_t st) {
+  const dim3 grid((a.E + kDecodeExp - 1) / kDecodeExp, static_cast<unsigned>((a.T + kDecodeTok - 1) / kDecodeTok),
+                  kDecodeSplit);
+  auto go = [&](auto kern) {
+    return launch_pdl(kern, grid, dim3(kDecodeThreads), 0, st, static_cast<const T*>(a.x),
+                      static_cast<const T*>(a.Wr), a.bias, a.T, a.H, a.E, a.k, a.scores64, a.wss,
+                      a.group_done, a.idx_ws, a.w_ws, a.idx_user, a.w_user, a.spill, a.ctrl);
+  };
+  const int epl = select_epl(a.E);
+  const cudaError_t e = epl == 4 ? go(router_decode_kernel<T, 4>)
+                        : epl == 12 ? go(router_decode_kernel<T, 12>) : go(router_decode_kernel<T, 32>);
+  count_launches(1);
+  return e;
+}
+
+int64_t router_group_counters(int64_t T) { return (T + kDecodeTok - 1) / kDecodeTok; }
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
-  if (a.bf16) return launch_router_f64_t<__nv_bfloat16>(a, st);
-  return launch_router_f64_t<float>(a, st);
+  if (router_tc_supported(a.bf16, a.T, a.E, a.H)) return launch_router_tc(a, st);
+  if (a.bf16) return launch_router_decode<__nv_bfloat16>(a, st);
+  return launch_router_decode<float>(a, st);
 }
 
 }  // namespace moe

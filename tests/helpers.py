@@ -11,8 +11,11 @@ from conftest import to_oracle
 # output tolerance of the layer: max|err| <= 2e-2 * max|y_ref| and relative L2 <= 1e-2
 Y_MAX_TOL = 2e-2
 Y_REL_L2_TOL = 1e-2
-# routing weights (fp32) against the oracle's fp64 softmax of the same keys
-W_REL_TOL = 1e-5
+# routing weights (fp32 softmax of the chosen keys) against the oracle's fp64 softmax of
+# the exact keys.  Keys of experts chosen for certain come from the score estimate (fp64
+# accumulation, or fp32 slices of 256 products added in fp64 on the tensor-core path),
+# whose error on these workloads is a few 1e-6 of a logit.
+W_REL_TOL = 2e-5
 
 
 def y_errors(y_gpu, y_ref: np.ndarray):
@@ -51,7 +54,7 @@ def oracle_y(d: dict, routing: dict, tokens=None):
                              a["Ws_gate_up"], a["Ws_down"], tokens=tokens)
 
 
-def assert_routing_exact(r_gpu, r_ref: dict, E: int):
+def assert_routing_exact(r_gpu, r_ref: dict, E: int, w_tol: float = None):
     idx = r_gpu.topk_idx.cpu().numpy()
     assert np.array_equal(idx, r_ref["idx"]), (
         f"topk_idx differs on {int((idx != r_ref['idx']).any(1).sum())} tokens")
@@ -60,7 +63,8 @@ def assert_routing_exact(r_gpu, r_ref: dict, E: int):
     assert np.array_equal(r_gpu.perm.cpu().numpy(), r_ref["perm"])
     w = r_gpu.topk_w.cpu().numpy().astype(np.float64)
     rel = np.abs(w - r_ref["w64"]) / np.maximum(np.abs(r_ref["w64"]), 1e-30)
-    assert float(rel.max()) <= W_REL_TOL, f"topk_w relative error {float(rel.max()):.3e}"
+    tol = W_REL_TOL if w_tol is None else w_tol
+    assert float(rel.max()) <= tol, f"topk_w relative error {float(rel.max()):.3e}"
 
 
 def to_device(d: dict, device="cuda"):

@@ -180,3 +180,74 @@ def test_full_size_workload(name):
     y_ref = oracle_y(d, ref, tokens=tokens)
     assert_y_close(y[torch.as_tensor(tokens, device=y.device)], y_ref, name)
     print(name, "route stats", stats)
+
+
+# ------------------------------------------------------------------------------------
+# the tensor-core router's error bound
+# ------------------------------------------------------------------------------------
+def _tc_router_error_ratio(d, top_k):
+    """max |s^ - s| / (L 2^-23 ||x|| ||w||) of the tensor-core router score estimates kept in
+    the workspace (fp32 accumulation over slices of L products), against the oracle's exact
+    scores.  The certified selection assumes this ratio is at most 2."""
+    import oracle
+    from conftest import to_oracle
+    T, H = d["x"].shape
+    E = d["W_router"].shape[0]
+    shape = moe.make_shape(T, H, E, d["W_gate_up"].shape[1] // 2, d["Ws_gate_up"].shape[0] // 2, top_k,
+                           torch.bfloat16)
+    ws = moe.alloc_workspace(shape, "cuda")
+    y, r = run(d, top_k, workspace=ws)
+    assert moe.check_status(ws) == moe.MOE_OK
+    torch.cuda.synchronize()
+    lay = moe.workspace_layout(shape)
+    assert lay.scores_slice > 0
+    s_hat = ws[lay.scores:lay.scores + T * E * 8].view(torch.float64).view(T, E).cpu().numpy()
+    s = oracle.router_scores(to_oracle(d["x"]), to_oracle(d["W_router"])).astype(np.float64)
+    xf, wf = d["x"].double().cpu().numpy(), d["W_router"].double().cpu().numpy()
+    bound = lay.scores_slice * 2.0 ** -23 * np.outer(np.linalg.norm(xf, axis=1), np.linalg.norm(wf, axis=1))
+    ulp = np.spacing(np.abs(s).astype(np.float32)).astype(np.float64)  # s is already RN32(exact)
+    return float(((np.abs(s_hat - s) - 0.5 * ulp) / bound).max()), r, ws
+
+
+def test_tensor_core_router_error_is_far_inside_the_certified_band():
+    cfg = inputs.small_config(T=1024, H=4096, E=288, top_k=8, I=128, I_shared=128)
+    d = to_device(inputs.make_inputs(cfg, "cuda"))
+    ratio, r, ws = _tc_router_error_ratio(d, cfg.top_k)
+    print("tensor-core router error / (L 2^-23 |x||w|):", ratio, moe.route_stats(ws))
+    assert ratio < 0.25  # the selection assumes <= 2
+
+
+def test_tensor_core_router_wide_dynamic_range():
+    """Inputs spanning many binades with cancellation: the accumulation error is still
+    inside the band and the routing still matches the exact one."""
+    cfg = inputs.small_config(T=640, H=1024, E=96, top_k=8, I=128, I_shared=128)
+    d = inputs.make_inputs(cfg, "cuda")
+    g = torch.Generator().manual_seed(5)
+    scale = torch.pow(2.0, torch.randint(-20, 12, (cfg.T, cfg.H), generator=g).float())
+    x = (torch.randn(cfg.T, cfg.H, generator=g) * scale)
+    x[:, 1::2] = -x[:, 0::2] * (1 + 2.0 ** -7)  # near-cancelling pairs
+    d["x"] = x.to(torch.bfloat16)
+    d = to_device(d)
+    ratio, r, ws = _tc_router_error_ratio(d, cfg.top_k)
+    print("wide-range router error ratio:", ratio, moe.route_stats(ws))
+    assert ratio < 0.5
+    ref = oracle_routing(d, cfg.top_k)
+    # the keys of experts chosen for certain come from the fp32-accumulated estimate; with
+    # sum|x w| far above |s| their weights are checked at the looser 1e-3
+    assert_routing_exact(r, ref, cfg.E, w_tol=1e-3)
+
+
+def test_decode_tiles_with_popular_experts():
+    """16-token tiles (few tokens per expert) with a bias that sends most tokens to four
+    experts, so those experts and the shared expert span many tiles."""
+    cfg = inputs.small_config(T=90, H=256, E=64, top_k=4, I=256, I_shared=128)
+    d = inputs.make_inputs(cfg, "cuda")
+    b = torch.zeros(cfg.E, dtype=torch.float32)
+    b[:4] = 3.0
+    d["bias"] = b
+    d = to_device(d)
+    y, r = run(d, cfg.top_k)
+    assert int(r.counts.max()) > 40
+    ref = oracle_routing(d, cfg.top_k)
+    assert_routing_exact(r, ref, cfg.E)
+    assert_y_close(y, oracle_y(d, ref), "popular experts, 16-token tiles")
