@@ -154,6 +154,27 @@ def ncu_traffic(kernel: str, workload: str):
 
 
 # ------------------------------------------------------------------------------------------
+# ranks: every rank is an independent replica on its own tokens (weak scaling)
+# ------------------------------------------------------------------------------------------
+def rank_config(cfg, rank: int):
+    """Rank r processes its own batch: same shapes and weights, tokens from seed + 1000 r."""
+    return inputs.with_sizes(cfg, seed=cfg.seed + 1000 * rank) if rank else cfg
+
+
+def max_over_ranks(value: float, pg, device) -> float:
+    """The largest value over all ranks (the job's elapsed time is the slowest rank's)."""
+    if pg is None:
+        return value
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, steps: int, elapsed_ms: float) -> float:
+    return world * tokens_per_rank * steps / (elapsed_ms / 1e3)
+
+
+# ------------------------------------------------------------------------------------------
 # the oracle on the host (cpu baseline and the reference arm)
 # ------------------------------------------------------------------------------------------
 def host_arrays(d):
@@ -273,8 +294,7 @@ def main():
     moe.load_library()
 
     # ---- inputs (resident in HBM); each rank is a replica with its own tokens -------------
-    rcfg = inputs.with_sizes(cfg, seed=cfg.seed + 1000 * rank) if rank else cfg
-    x, Wr, bias = inputs.make_routing_inputs(rcfg)
+    x, Wr, bias = inputs.make_routing_inputs(rank_config(cfg, rank))
     Wgu, Wd, Wsgu, Wsd = inputs.make_expert_weights(cfg, dev)
     x, Wr = x.to(dev), Wr.to(dev)
     bias = None if bias is None else bias.to(dev)
@@ -324,11 +344,7 @@ def main():
     launches = moe.launch_count() - launches0
     moe.profile_enable(False)
     calls, stage_ms = moe.profile_read()
-    elapsed_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    if pg:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), pg, dev)
     status = moe.check_status(ws)
 
     # ---- end to end through the public API, host buffers ----------------------------------
@@ -352,18 +368,15 @@ def main():
         y_host.copy_(y, non_blocking=True)
         ee_[i].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(es_, ee_))
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(es_, ee_)), pg, dev)
     if pg:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         pg.barrier()
 
     if rank == 0:
         peaks = measured_peaks()
         ms_per_step = elapsed_ms / args.steps
-        value = world * cfg.T * args.steps / (elapsed_ms / 1e3)
-        e2e_value = world * cfg.T * e_steps / (e2e_ms / 1e3)
+        value = job_tokens_per_s(cfg.T, world, args.steps, elapsed_ms)
+        e2e_value = job_tokens_per_s(cfg.T, world, e_steps, e2e_ms)
         gu_ms = stage_ms["gate_up"] / max(calls, 1)
         dn_ms = stage_ms["down"] / max(calls, 1)
         tensor_bound = alg["gate_up_flops"] / (peaks["bf16_tflops"] * 1e12) > alg["gate_up_bytes"] / (peaks["hbm_gbs"] * 1e9)
