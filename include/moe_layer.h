@@ -162,6 +162,33 @@ MOE_API int moe_layer_profile_read(float* ms, int n_stages);
 /* Number of kernels this library has launched in this process so far. */
 MOE_API int64_t moe_layer_launch_count(void);
 
+/* Routing of a batch without a workspace argument, for callers that cannot allocate
+ * device memory (a runtime whose memory planner owns every buffer and hands a layer only
+ * its inputs and outputs; a host loop that must not call cudaMalloc, which can
+ * synchronise the device; a plugin called with tensors but no allocator).  This entry
+ * point has no counterpart on the source pages: it is a deployment convenience.
+ *
+ * Computes what moe_layer_forward() computes for routing -- router scores, the top_k
+ * experts of each token (ascending index, same certified selection) and their
+ * renormalised softmax weights -- and writes
+ *   topk_idx [T, top_k] int32 and topk_w [T, top_k] fp32 (device pointers, caller-owned).
+ * x, W_router and router_bias are as for moe_layer_forward(); the I and I_shared fields
+ * of the shape are not used.
+ *
+ * Scratch: a 16 MiB device array inside this library (present on every GPU that loads the
+ * library, until the process exits).  The call needs about T * (24 * E + 8) bytes of it
+ * (plus E / 2 per token for fp32 inputs), so batches of up to about 2400 tokens fit at
+ * E = 288.  Larger batches return MOE_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.
+ * The array is shared by all calls: calls that may overlap on the GPU (several streams or
+ * host threads) race and must be serialised by the caller.  Each call clears the part
+ * that must start at zero on its stream.
+ * The first call on a device looks up the array's device address (once per device, with
+ * that device current); make that first call before any stream capture.
+ * Returns validation and launch errors; device-side statuses are not reported. */
+MOE_API moe_status moe_layer_route_noalloc(const moe_layer_shape* shape, const void* x,
+                                           const void* W_router, const float* router_bias,
+                                           int32_t* topk_idx, float* topk_w, void* stream);
+
 /* Human-readable name of a status code (static string). */
 MOE_API const char* moe_status_string(moe_status status);
 
