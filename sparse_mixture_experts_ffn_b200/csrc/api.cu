@@ -96,7 +96,7 @@ static size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255);
 
 struct Layout {
   size_t ctrl, group_done, tile_done, wss, zero_end, scores, xnorm, wnorm, idx, w, blk_hist, counts,
-      offsets, group_order, item_start_gu, item_start_dn, perm, inv_perm, row_w, row_tok, partial, spill,
+      offsets, group_order, item_start_gu, item_start_dn, perm, inv_perm, row_w, row_tok, partial, spill, rsplit,
       x_perm, h, h_shared, o, o_shared, total;
   int bn, ksplit;
   int64_t max_tiles;
@@ -119,7 +119,7 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.max_tiles = expert_tile_bound(s->T, s->top_k, s->E, s->I, s->I_shared, L.bn);
   // control block and counters first: one memset per forward clears them
   const bool tc_scores = router_scores_f32(*s);
-  const size_t groups = static_cast<size_t>(router_group_counters(s->T));
+  const size_t groups = static_cast<size_t>(router_group_counters(s->T, s->E));
   L.ctrl = take(sizeof(Ctrl));
   L.group_done = take(groups * 4);
   L.tile_done = take(L.ksplit > 1 ? static_cast<size_t>(L.max_tiles) * 4 : 0);
@@ -128,6 +128,7 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.scores = take(T * E * 8);
   L.zero_end = tc_scores ? L.scores : off;
   L.spill = take(T * E * 16);
+  L.rsplit = take(router_split_bytes(*s));
   L.xnorm = take(T * 8);
   L.wnorm = take(E * 8);
   L.idx = take(P * 4);
@@ -143,7 +144,8 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.row_w = take(P * 4);
   L.row_tok = take(P * 4);
   L.partial = take(L.ksplit > 1 ? static_cast<size_t>(L.max_tiles) * L.ksplit * L.bn * 256 * 4 : 0);
-  L.x_perm = take(P * H * es);
+  // 16-token bf16 tiles gather their token rows from x; wider tiles and fp32 read a copy
+  L.x_perm = take(s->dtype == MOE_BF16 && L.bn == 16 ? 0 : P * H * es);
   L.h = take(P * I * es);
   L.h_shared = take(T * Is * es);
   L.o = take(P * H * es);
@@ -252,6 +254,7 @@ extern "C" moe_status moe_layer_forward(const moe_layer_shape* shape, const void
   ra.scores64 = static_cast<double*>(at(L.scores));
   ra.wss = static_cast<double*>(at(L.wss));
   ra.spill = static_cast<float*>(at(L.spill));
+  ra.rsplit = router_split_bytes(*shape) ? at(L.rsplit) : nullptr;
   ra.xnorm = static_cast<double*>(at(L.xnorm));
   ra.wnorm = static_cast<double*>(at(L.wnorm));
   ra.group_done = static_cast<unsigned int*>(at(L.group_done));
@@ -313,6 +316,7 @@ extern "C" moe_status moe_layer_forward(const moe_layer_shape* shape, const void
   ea.item_start_dn = da.item_start_dn;
   ea.row_w = da.row_w;
   ea.x_perm = da.x_perm;
+  ea.row_tok = da.row_tok;
   ea.bn = L.bn;
   ea.ksplit = L.ksplit;
   ea.partial = static_cast<float*>(at(L.partial));

@@ -107,17 +107,33 @@ __device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* order, int*
       if (a.offsets_user) a.offsets_user[E] = total;
     }
   }
-  // largest group first: rank by (count desc, index asc)
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
-    const int c = cnt[g];
-    int r = 0;
-    for (int h = 0; h < G; ++h) {
-      const int ch = cnt[h];
-      r += (ch > c) || (ch == c && h < g);
-    }
-    order[r] = g;
+  // largest group first: rank by (count desc, index asc).  Groups without tokens take the
+  // last places in index order; the others are first compacted (in index order) into the
+  // leading places of order[] and ranked among themselves only.
+  {
+    const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
+    const int z0 = (i0 < G && cnt[i0] > 0) ? 1 : 0, z1 = (i1 < G && cnt[i1] > 0) ? 1 : 0;
+    int nnz;
+    const int nz_ex = block_scan_pair(z0, z1, warp_tot, nnz);
+    if (i0 < G) order[z0 ? nz_ex : nnz + (i0 - nz_ex)] = i0;
+    if (i1 < G) order[z1 ? nz_ex + z0 : nnz + (i1 - nz_ex - z0)] = i1;
+    __syncthreads();
+    auto rank_of = [&](int g) {
+      const int c = cnt[g];
+      int r = 0;
+      for (int j = 0; j < nnz; ++j) {
+        const int h = order[j];
+        const int ch = cnt[h];
+        r += (ch > c) || (ch == c && h < g);
+      }
+      return r;
+    };
+    const int r0 = z0 ? rank_of(i0) : -1, r1 = z1 ? rank_of(i1) : -1;
+    __syncthreads();
+    if (r0 >= 0) order[r0] = i0;
+    if (r1 >= 0) order[r1] = i1;
+    __syncthreads();
   }
-  __syncthreads();
   for (int r = threadIdx.x; r < G; r += blockDim.x) a.group_order[r] = order[r];
   const int r0 = 2 * threadIdx.x, r1 = r0 + 1;
   auto tiles = [&](int r, bool gu) -> int {
@@ -358,6 +374,13 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st) {
                    a.perm, a.inv_perm, a.row_w, a.row_tok, a.perm_user);
     if (e != cudaSuccess) return e;
     launches = 3;
+  }
+  // 16-token bf16 tiles gather their token rows from x inside the GEMM (row-gather TMA,
+  // four rows per copy); wider tiles, whose copies would be too many, and the fp32 path
+  // read a permuted copy
+  if (a.bf16 && a.bn == 16) {
+    count_launches(launches);
+    return cudaSuccess;
   }
   const int64_t vec = P * (a.H / (a.bf16 ? 8 : 4));
   const int blocks = static_cast<int>(std::min<int64_t>((vec + 255) / 256, 148 * 16));

@@ -27,11 +27,14 @@ namespace moe {
 // ---------------------------------------------------------------------------------------
 struct TcParams {
   CUtensorMap tmA[2];  // weights: [0] routed (all experts stacked), [1] shared expert
-  CUtensorMap tmB[2];  // activations: [0] routed rows in expert order, [1] shared rows
+  CUtensorMap tmB[2];  // activations: [0] routed rows in expert order (gather: x rows,
+                       // one-row box), [1] shared rows
   const int32_t* offsets;      // [E + 1]
   const int32_t* group_order;  // [G]
   const int32_t* item_start;   // [G + 1]
   const float* row_w;          // routing weight per routed row (down projection only)
+  const int32_t* row_tok;      // token of each routed row (gather)
+  int gather;                  // routed token rows gathered from x by tmB[0] (gate/up)
   __nv_bfloat16* out[2];       // [0] routed rows, [1] shared rows
   int ld_out[2];               // row stride of out (elements), routed and shared
   int E, G;
@@ -192,35 +195,60 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
 
   if (warp == 0) {
     // ------------------------------- TMA producer -------------------------------------
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t used = 0;  // stages that ever received a copy
-      bool ok = true;
-      for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-        const Item t = decode_item<BN>(p, it);
-        if (!t.valid) {
-          if (blockIdx.x == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
-          continue;
-        }
-        const int arow = t.sh ? t.m * kTileM : t.g * p.a_rows_per_group + t.m * kTileM;
-        const int kb_n = p.kblocks[t.sh];
-        const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, p.ctrl, abort_flag)) { ok = false; break; }
-          unsigned char* st = smem + stage * C::kStageBytes;
-          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
-          tma_load_2d(st, &p.tmA[t.sh], kb * kTileK, arow, &full[stage]);
-          if (GATED)
-            tma_load_2d(st + C::kABytes, &p.tmA[t.sh], kb * kTileK, arow + p.a_up_offset[t.sh],
-                        &full[stage]);
-          tma_load_2d(st + (GATED ? 2 : 1) * C::kABytes, &p.tmB[t.sh], kb * kTileK, t.row0,
-                      &full[stage]);
-          used |= 1u << stage;
-          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+    // Lane 0 waits for free stages and loads the weight tiles; routed token rows of the
+    // gate/up GEMM come straight from x, four rows per lane and copy (row-gather TMA).
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t used = 0;  // stages that ever received a copy
+    bool ok = true;
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      const Item t = decode_item<BN>(p, it);
+      if (!t.valid) {
+        if (blockIdx.x == 0 && lane == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
+        continue;
+      }
+      const bool gath = GATED && p.gather && !t.sh;
+      int tok[4] = {0, 0, 0, 0};
+      if (gath && lane < BN / 4) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int n = lane * 4 + q;
+          const int v = __ldg(p.row_tok + t.row0 + (n < t.nvalid ? n : 0));
+          if (v < 0 || v >= p.T) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
+          tok[q] = (v < 0 || v >= p.T) ? 0 : v;  // padding rows repeat the first token
         }
       }
-      // every copy issued must have landed before the block exits
+      const int arow = t.sh ? t.m * kTileM : t.g * p.a_rows_per_group + t.m * kTileM;
+      const int kb_n = p.kblocks[t.sh];
+      const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        unsigned char* st = smem + stage * C::kStageBytes;
+        int good = 1;
+        if (lane == 0) {
+          good = mbar_wait(&empty[stage], phase ^ 1u, p.ctrl, abort_flag) ? 1 : 0;
+          if (good) {
+            mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+            tma_load_2d(st, &p.tmA[t.sh], kb * kTileK, arow, &full[stage]);
+            if (GATED)
+              tma_load_2d(st + C::kABytes, &p.tmA[t.sh], kb * kTileK, arow + p.a_up_offset[t.sh],
+                          &full[stage]);
+            if (!gath)
+              tma_load_2d(st + (GATED ? 2 : 1) * C::kABytes, &p.tmB[t.sh], kb * kTileK, t.row0,
+                          &full[stage]);
+          }
+        }
+        good = __shfl_sync(0xffffffffu, good, 0);
+        if (!good) { ok = false; break; }
+        if (gath && lane < BN / 4)
+          tma_gather4_2d(st + (GATED ? 2 : 1) * C::kABytes + lane * 4 * kTileK * 2, &p.tmB[0], kb * kTileK,
+                         tok[0], tok[1], tok[2], tok[3], &full[stage]);
+        used |= 1u << stage;
+        if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    __syncwarp();
+    // every copy issued must have landed before the block exits
+    if (lane == 0)
       for (int s = 0; s < C::kStages; ++s) {
         if (!(used & (1u << s))) continue;
         // the last phase issued on stage s: stages before `stage` were last issued in the
@@ -228,7 +256,6 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
         const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
         mbar_wait_drain(&full[s], par, p.ctrl);
       }
-    }
   } else if (warp == 1) {
     // ------------------------------- MMA issuer ---------------------------------------
     if (lane == 0) {
@@ -526,10 +553,13 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
     return cudaGetLastError();
   }
   const int G = a.E + (has_shared ? 1 : 0);
-  // gate/up: A = W_gate_up viewed as [E*2I, H]; B = x_perm [P, H] (shared: x [T, H])
+  // gate/up: A = W_gate_up viewed as [E*2I, H]; B = rows of x [T, H] gathered by token
+  // (16-token tiles) or x_perm [P, H] (shared: x [T, H] in order)
   TcParams g{};
+  const bool gather = a.bn == 16;
   bool ok = encode_2d_bf16(&g.tmA[0], a.Wgu, static_cast<uint64_t>(a.E) * 2 * a.I, a.H, kTileM) &&
-            encode_2d_bf16(&g.tmB[0], a.x_perm, P, a.H, a.bn);
+            (gather ? encode_2d_bf16(&g.tmB[0], a.x, a.T, a.H, 1)
+                    : encode_2d_bf16(&g.tmB[0], a.x_perm, P, a.H, a.bn));
   if (has_shared)
     ok = ok && encode_2d_bf16(&g.tmA[1], a.Wsgu, 2ull * a.Is, a.H, kTileM) &&
          encode_2d_bf16(&g.tmB[1], a.x, a.T, a.H, a.bn);
@@ -542,6 +572,8 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   g.group_order = a.group_order;
   g.item_start = a.item_start_gu;
   g.row_w = a.row_w;
+  g.row_tok = a.row_tok;
+  g.gather = gather ? 1 : 0;
   g.out[0] = static_cast<__nv_bfloat16*>(a.h);
   g.out[1] = static_cast<__nv_bfloat16*>(a.h_shared);
   g.E = a.E;

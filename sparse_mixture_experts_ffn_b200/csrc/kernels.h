@@ -41,10 +41,14 @@ struct RouterArgs {
   int32_t* idx_user;
   float* w_user;
   float* spill;      // [4, T, E] key state of tokens that need exact dots
+  void* rsplit;      // router_split_bytes(shape) bytes, or null: the reduction is not split
   Ctrl* ctrl;
 };
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
-int64_t router_group_counters(int64_t T);
+// counters of the router kernels, zero before the forward
+int64_t router_group_counters(int64_t T, int E);
+// scratch of the reduction-split tensor-core router (0 when a batch fills the GPU unsplit)
+size_t router_split_bytes(const moe_layer_shape& s);
 // whether the router scores of this shape come from the tensor cores (else fp64)
 bool router_scores_f32(const moe_layer_shape& s);
 // products per fp32-accumulated slice of the tensor-core router scores
@@ -92,7 +96,8 @@ struct ExpertArgs {
   const int32_t* item_start_gu;
   const int32_t* item_start_dn;
   const float* row_w;
-  const void* x_perm;
+  const int32_t* row_tok;  // [T*k] token of each routed row (bf16: gathered from x)
+  const void* x_perm;      // fp32 path: routed rows of x in expert order
   int bn;           // tokens per GEMM tile (16 or 128)
   int ksplit;       // gate/up reduction slices (1, 2 or 4)
   float* partial;   // split partial sums (ksplit > 1)

@@ -76,7 +76,7 @@ extern "C" moe_status moe_layer_route_noalloc(const moe_layer_shape* shape, cons
   // norms and the key spill of the rare exact path
   const size_t T = static_cast<size_t>(s.T), E = static_cast<size_t>(s.E);
   const bool tc = router_scores_f32(s);
-  const size_t groups = static_cast<size_t>(router_group_counters(s.T));
+  const size_t groups = static_cast<size_t>(router_group_counters(s.T, s.E));
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -118,6 +118,7 @@ extern "C" moe_status moe_layer_route_noalloc(const moe_layer_shape* shape, cons
   ra.idx_user = nullptr;
   ra.w_user = nullptr;
   ra.spill = reinterpret_cast<float*>(ws + o_spill);
+  ra.rsplit = nullptr;  // the scratch holds no reduction-split partials
   ra.ctrl = reinterpret_cast<Ctrl*>(ws + o_ctrl);
   return launch_router(ra, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

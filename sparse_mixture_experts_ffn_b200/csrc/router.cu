@@ -824,13 +824,21 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) router_decode_kernel(
 }
 
 // ---------------------------------------------------------------------------------------
-// tcgen05 router GEMM.  Block (m, n) scores the tokens [128m, 128m+128) against the
-// experts [64n, 64n+64).  Every slice of kRtSliceSteps 64-product steps of the reduction
-// is accumulated in fp32 in one of two tensor-memory buffers and then drained by the
-// epilogue warps into fp64 registers, so the fp32 accumulation error of each partial is
-// bounded by the slice and the partials add up in fp64.  Only the token rows that exist
-// are loaded (16-row boxes); rows of the A tile beyond them are never read back.
-// Warp 0 issues TMA copies, warp 1 the MMAs, warps 2-5 (one thread per token) drain.
+// tcgen05 router GEMM.  Block (m, n, z) scores the tokens [128m, 128m+128) against the
+// experts [64n, 64n+64) over chunk z of the reduction.  Every slice of kRtSliceSteps
+// 64-product steps is accumulated in fp32 in one of two tensor-memory buffers and then
+// drained by the epilogue warps, so the fp32 accumulation error of each partial is
+// bounded by the slice; the partials add up in fp64, in slice order.  Only the token
+// rows that exist are loaded (16-row boxes); rows of the A tile beyond them are never
+// read back.  Warp 0 issues TMA copies, warp 1 the MMAs, warps 2-5 (one thread per
+// token) drain.
+//
+// Unsplit (one chunk): the epilogue adds the slices in fp64 registers and writes the
+// scores.  Split (a batch whose tiles do not fill the GPU): each block writes its slices'
+// fp32 partials and the sums of squares of its x / W_router columns (for the norm bounds
+// of the selection); the last block of each (m, n) tile, found by a counter, adds the
+// partials in the same slice order -- the scores are bit-identical to the unsplit ones --
+// and finishes the norms of its rows.
 // ---------------------------------------------------------------------------------------
 constexpr int kRtExperts = 64;
 constexpr int kRtStages = 8;
@@ -840,6 +848,8 @@ constexpr int kRtBBytes = kRtExperts * kTileK * 2;   // 8 KB of W_router
 constexpr int kRtStageBytes = kRtABytes + kRtBBytes;
 constexpr int kRtSmem = kRtStages * kRtStageBytes + 1024 + 256;
 constexpr int kRtRowBox = 16;                        // token rows per TMA box
+constexpr int kRtMaxChunks = 8;
+constexpr int kRtSmTarget = 148;                     // blocks that fill the GPU
 
 struct RouterTcParams {
   CUtensorMap tmX;   // x [T, H], box {64, 16}
@@ -847,8 +857,52 @@ struct RouterTcParams {
   int64_t T;
   int H, E;
   double* scores;    // [T, E]
+  // split only
+  int chunks, chunk_slices;
+  const __nv_bfloat16* x;
+  const __nv_bfloat16* Wr;
+  float* part;       // [slices, T, E] fp32 slice partials
+  double* xss;       // [chunks, T] partial sums of squares
+  double* wss;       // [chunks, E]
+  unsigned int* tile_done;   // [tiles m x n], zero before the launch
+  double* xnorm;     // [T]
+  double* wnorm;     // [E]
   Ctrl* ctrl;
 };
+
+// Sum of squares of rows [0, nrows) of a bf16 matrix over columns [c0, c1) (multiples of
+// 8), by the four epilogue warps (w = 0..3), eight rows per warp at a time; out[r].
+__device__ void sumsq_rows_bf16(const __nv_bfloat16* __restrict__ base, int64_t ld, int nrows, int c0,
+                                int c1, double* __restrict__ out, int w, int lane) {
+  const int nv = (c1 - c0) / 8;
+  for (int r0 = w; r0 < nrows; r0 += 4 * 8) {
+    double ss[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) ss[u] = 0.0;
+#pragma unroll 2
+    for (int v = lane; v < nv; v += 32) {
+      Vec16<__nv_bfloat16> a[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (r0 + 4 * u < nrows) a[u] = ld16(base + (r0 + 4 * u) * ld + c0 + v * 8);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (r0 + 4 * u >= nrows) break;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const double d = static_cast<double>(__bfloat162float(a[u].v[j]));
+          ss[u] = fma(d, d, ss[u]);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss[u] += __shfl_xor_sync(0xffffffffu, ss[u], o);
+      if (lane == 0 && r0 + 4 * u < nrows) out[r0 + 4 * u] = ss[u];
+    }
+  }
+}
 
 __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_constant__ RouterTcParams p) {
   extern __shared__ unsigned char smem_raw[];
@@ -861,6 +915,7 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = abort_flag + 1;
   constexpr uint32_t kCols = 128;  // two 64-column accumulators
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -875,6 +930,7 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
+    *last_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, kCols);
@@ -885,7 +941,14 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTileM;
   const int e0 = blockIdx.y * kRtExperts;
   const int ne = min(kRtExperts, p.E - e0);
-  const int kb_n = p.H / kTileK;
+  const int kb_all = p.H / kTileK;
+  const int n_sl_all = (kb_all + kRtSliceSteps - 1) / kRtSliceSteps;
+  const bool split = p.chunks > 1;
+  const int sl_begin = blockIdx.z * p.chunk_slices;
+  const int sl_end = min(n_sl_all, sl_begin + p.chunk_slices);
+  const int kb_begin = sl_begin * kRtSliceSteps;
+  const int kb_end = min(kb_all, sl_end * kRtSliceSteps);
+  const int n_sl = sl_end - sl_begin;
   const int rows = static_cast<int>(min64(kTileM, p.T - t0));
   const int nbox = (rows + kRtRowBox - 1) / kRtRowBox;
   pdl_wait();
@@ -897,7 +960,7 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
       const uint32_t bytes = nbox * kRtRowBox * kTileK * 2 + kRtBBytes;
       int stage = 0;
       uint32_t phase = 0, used = 0;
-      for (int kb = 0; kb < kb_n; ++kb) {
+      for (int kb = kb_begin; kb < kb_end; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, p.ctrl, abort_flag)) break;
         unsigned char* st = smem + stage * kRtStageBytes;
         mbar_arrive_expect_tx(&full[stage], bytes);
@@ -921,10 +984,10 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
       const uint32_t idesc = idesc_bf16_f32(kTileM, (ne + 15) & ~15);
       int stage = 0;
       uint32_t phase = 0;
-      for (int kb = 0; kb < kb_n; ++kb) {
-        const int sl = kb / kRtSliceSteps;   // slice index
+      for (int kb = kb_begin; kb < kb_end; ++kb) {
+        const int sl = (kb - kb_begin) / kRtSliceSteps;   // slice within the chunk
         const bool first = (kb % kRtSliceSteps) == 0;
-        const bool last = (kb % kRtSliceSteps) == kRtSliceSteps - 1 || kb == kb_n - 1;
+        const bool last = (kb % kRtSliceSteps) == kRtSliceSteps - 1 || kb == kb_end - 1;
         const int b = sl & 1;
         if (first && !mbar_wait(&tempty[b], ((sl >> 1) & 1) ^ 1u, p.ctrl, abort_flag)) break;
         if (!mbar_wait(&full[stage], phase, p.ctrl, abort_flag)) break;
@@ -946,30 +1009,90 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
   } else {
     const int quarter = warp & 3;
     const int64_t t = t0 + quarter * 32 + lane;
-    double acc[kRtExperts];
-#pragma unroll
-    for (int j = 0; j < kRtExperts; ++j) acc[j] = 0.0;
     const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     bool ok = true;
-    const int n_sl = (kb_n + kRtSliceSteps - 1) / kRtSliceSteps;
-    for (int sl = 0; sl < n_sl && ok; ++sl) {
-      const int b = sl & 1;
-      if (!mbar_wait(&tfull[b], (sl >> 1) & 1, p.ctrl, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t r[kRtExperts];
+    if (!split) {
+      double acc[kRtExperts];
 #pragma unroll
-      for (int j0 = 0; j0 < kRtExperts; j0 += 16) tmem_ld16_nowait(trow + b * kRtExperts + j0, r + j0);
-      tmem_wait_ld();
+      for (int j = 0; j < kRtExperts; ++j) acc[j] = 0.0;
+      for (int sl = 0; sl < n_sl && ok; ++sl) {
+        const int b = sl & 1;
+        if (!mbar_wait(&tfull[b], (sl >> 1) & 1, p.ctrl, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t r[kRtExperts];
 #pragma unroll
-      for (int j = 0; j < kRtExperts; ++j) acc[j] += static_cast<double>(__uint_as_float(r[j]));
-      tc_fence_before();
-      mbar_arrive(&tempty[b]);
-    }
-    if (ok && t < p.T) {
-      double* dst = p.scores + t * p.E + e0;
+        for (int j0 = 0; j0 < kRtExperts; j0 += 16) tmem_ld16_nowait(trow + b * kRtExperts + j0, r + j0);
+        tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < kRtExperts; ++j)
-        if (j < ne) dst[j] = acc[j];
+        for (int j = 0; j < kRtExperts; ++j) acc[j] += static_cast<double>(__uint_as_float(r[j]));
+        tc_fence_before();
+        mbar_arrive(&tempty[b]);
+      }
+      if (ok && t < p.T) {
+        double* dst = p.scores + t * p.E + e0;
+#pragma unroll
+        for (int j = 0; j < kRtExperts; ++j)
+          if (j < ne) dst[j] = acc[j];
+      }
+    } else {
+      // sums of squares of this chunk's columns while the MMAs run: the x rows once per
+      // m tile (n == 0), the W_router rows once per n tile (m == 0)
+      const int c0 = kb_begin * kTileK, c1 = kb_end * kTileK;
+      if (blockIdx.y == 0)
+        sumsq_rows_bf16(p.x + t0 * p.H, p.H, rows, c0, c1, p.xss + blockIdx.z * p.T + t0, quarter, lane);
+      if (blockIdx.x == 0)
+        sumsq_rows_bf16(p.Wr + static_cast<int64_t>(e0) * p.H, p.H, ne, c0, c1,
+                        p.wss + static_cast<int64_t>(blockIdx.z) * p.E + e0, quarter, lane);
+      for (int sl = 0; sl < n_sl && ok; ++sl) {
+        const int b = sl & 1;
+        if (!mbar_wait(&tfull[b], (sl >> 1) & 1, p.ctrl, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t r[kRtExperts];
+#pragma unroll
+        for (int j0 = 0; j0 < kRtExperts; j0 += 16) tmem_ld16_nowait(trow + b * kRtExperts + j0, r + j0);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&tempty[b]);
+        if (t < p.T) {
+          float* dst = p.part + (static_cast<int64_t>(sl_begin + sl) * p.T + t) * p.E + e0;
+#pragma unroll
+          for (int j = 0; j < kRtExperts; ++j)
+            if (j < ne) dst[j] = __uint_as_float(r[j]);
+        }
+      }
+      // the last block of this (m, n) tile adds the partials of every chunk
+      __threadfence();
+      named_bar_sync(1, 128);
+      if (warp == 2 && lane == 0) {
+        const unsigned int done = atomicAdd(p.tile_done + blockIdx.x * gridDim.y + blockIdx.y, 1u);
+        *last_flag = (done == static_cast<unsigned int>(p.chunks - 1)) ? 1 : 0;
+      }
+      named_bar_sync(1, 128);
+      if (*last_flag) {
+        __threadfence();
+        const int et = threadIdx.x - 64;
+        for (int i = et; i < rows * ne; i += 128) {
+          const int tt = i / ne, j = i - tt * ne;
+          const float* src = p.part + (t0 + tt) * p.E + e0 + j;
+          const int64_t sstride = p.T * p.E;
+          double acc = 0.0;
+#pragma unroll 16
+          for (int sl = 0; sl < n_sl_all; ++sl) acc += static_cast<double>(__ldcg(src + sl * sstride));
+          p.scores[(t0 + tt) * p.E + e0 + j] = acc;
+        }
+        if (blockIdx.y == 0)
+          for (int i = et; i < rows; i += 128) {
+            double ss = 0.0;
+            for (int z = 0; z < p.chunks; ++z) ss += __ldcg(p.xss + z * p.T + t0 + i);
+            p.xnorm[t0 + i] = norm_ub_from_sumsq(ss, p.H);
+          }
+        if (blockIdx.x == 0)
+          for (int i = et; i < ne; i += 128) {
+            double ss = 0.0;
+            for (int z = 0; z < p.chunks; ++z) ss += __ldcg(p.wss + static_cast<int64_t>(z) * p.E + e0 + i);
+            p.wnorm[e0 + i] = norm_ub_from_sumsq(ss, p.H);
+          }
+      }
     }
   }
   pdl_trigger();
@@ -1016,6 +1139,30 @@ static cudaError_t allow_smem(K kern, size_t smem) {
 
 int router_slice_len(int /*H*/) { return kRtSliceSteps * kTileK; }
 
+// Reduction chunks of the tensor-core router: 1 when the (m, n) tiles fill the GPU or the
+// batch is too large for one block per tile to add the partials quickly, else the fewest
+// (at most 8, at least two slices each) that bring the blocks to one per SM.
+constexpr int64_t kRtSplitMaxTokens = 32;
+static int router_chunks(int64_t T, int E, int H) {
+  if (T > kRtSplitMaxTokens) return 1;
+  const int64_t tiles = ((T + kTileM - 1) / kTileM) * ((E + kRtExperts - 1) / kRtExperts);
+  const int n_sl = (H / kTileK + kRtSliceSteps - 1) / kRtSliceSteps;
+  int c = 1;
+  while (c < kRtMaxChunks && tiles * c < kRtSmTarget && 4 * c <= n_sl) c *= 2;
+  if (c == 1) return 1;
+  const int per = (n_sl + c - 1) / c;
+  return (n_sl + per - 1) / per;
+}
+
+size_t router_split_bytes(const moe_layer_shape& s) {
+  if (!router_tc_supported(s.dtype == MOE_BF16, s.T, s.E, s.H)) return 0;
+  const int c = router_chunks(s.T, s.E, s.H);
+  if (c == 1) return 0;
+  const size_t n_sl = static_cast<size_t>((s.H / kTileK + kRtSliceSteps - 1) / kRtSliceSteps);
+  const size_t T = static_cast<size_t>(s.T), E = static_cast<size_t>(s.E);
+  return static_cast<size_t>(c) * (T + E) * 8 + n_sl * T * E * 4;
+}
+
 static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
   using bf16 = __nv_bfloat16;
   RouterTcParams p{};
@@ -1031,11 +1178,31 @@ static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const bf16* x = static_cast<const bf16*>(a.x);
   const bf16* Wr = static_cast<const bf16*>(a.Wr);
-  e = launch_pdl(row_norm_ub_kernel<bf16>, dim3(static_cast<unsigned>(((a.T + a.E) * 32 + 255) / 256)),
-                 dim3(256), 0, st, x, a.T, a.xnorm, Wr, static_cast<int64_t>(a.E), a.wnorm, a.H);
-  if (e != cudaSuccess) return e;
+  const int n_sl = (a.H / kTileK + kRtSliceSteps - 1) / kRtSliceSteps;
+  const int chunks = a.rsplit ? router_chunks(a.T, a.E, a.H) : 1;
+  p.chunks = chunks;
+  p.chunk_slices = (n_sl + chunks - 1) / chunks;
+  int launches = 2;
+  if (chunks > 1) {
+    // the split blocks also produce the norm bounds
+    double* d = static_cast<double*>(a.rsplit);
+    p.x = x;
+    p.Wr = Wr;
+    p.xss = d;
+    p.wss = d + static_cast<int64_t>(chunks) * a.T;
+    p.part = reinterpret_cast<float*>(p.wss + static_cast<int64_t>(chunks) * a.E);
+    p.tile_done = a.group_done;
+    p.xnorm = a.xnorm;
+    p.wnorm = a.wnorm;
+  } else {
+    e = launch_pdl(row_norm_ub_kernel<bf16>, dim3(static_cast<unsigned>(((a.T + a.E) * 32 + 255) / 256)),
+                   dim3(256), 0, st, x, a.T, a.xnorm, Wr, static_cast<int64_t>(a.E), a.wnorm, a.H);
+    if (e != cudaSuccess) return e;
+    launches = 3;
+  }
   e = launch_pdl(router_gemm_tc_kernel,
-                 dim3(static_cast<unsigned>((a.T + kTileM - 1) / kTileM), (a.E + kRtExperts - 1) / kRtExperts),
+                 dim3(static_cast<unsigned>((a.T + kTileM - 1) / kTileM), (a.E + kRtExperts - 1) / kRtExperts,
+                      static_cast<unsigned>(chunks)),
                  dim3(192), static_cast<size_t>(kRtSmem), st, p);
   if (e != cudaSuccess) return e;
   // Each slice of L = 256 products is accumulated in fp32 from exact products, at most
@@ -1054,7 +1221,7 @@ static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
   const int epl = select_epl(a.E);
   e = epl == 4 ? sel(route_select_kernel<bf16, 4>) : epl == 12 ? sel(route_select_kernel<bf16, 12>)
                                                                 : sel(route_select_kernel<bf16, 32>);
-  count_launches(3);
+  count_launches(launches);
   return e;
 }
 
@@ -1074,7 +1241,10 @@ static cudaError_t launch_router_decode(const RouterArgs& a, cudaStream_t st) {
   return e;
 }
 
-int64_t router_group_counters(int64_t T) { return (T + kDecodeTok - 1) / kDecodeTok; }
+int64_t router_group_counters(int64_t T, int E) {
+  const int64_t tiles = ((T + kTileM - 1) / kTileM) * ((E + kRtExperts - 1) / kRtExperts);
+  return std::max<int64_t>((T + kDecodeTok - 1) / kDecodeTok, tiles);
+}
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;

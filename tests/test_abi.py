@@ -48,6 +48,9 @@ def test_workspace_bytes(lib):
     # x_perm, h, o (bf16) dominate; everything else is small
     assert n >= 2 * (P * H + P * I + P * H + T * I + T * H)
     assert n < 2 * (P * H + P * I + P * H + T * I + T * H) + 64 * 1024 * 1024
+    # 16-token tiles (decode) gather token rows from x: no permuted copy of x
+    d = moe.workspace_bytes(shape(T=4))
+    assert d < 2 * (4 * k * H) + 2 * (4 * k * I + 4 * k * H + 4 * I + 4 * H) + 64 * 1024 * 1024
     assert moe.workspace_bytes(shape(T=0)) > 0
     for bad in (shape(top_k=0), shape(top_k=289), shape(E=0), shape(H=4000), shape(I=1000),
                 shape(I_shared=100), shape(E=1025, top_k=8), shape(dtype=7), shape(T=-1)):

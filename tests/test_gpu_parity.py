@@ -45,6 +45,10 @@ SMALL = [
     dict(T=77, H=256, E=8, top_k=8, I=128, I_shared=128),
     dict(T=200, H=512, E=40, top_k=6, I=384, I_shared=0),
     dict(T=1000, H=256, E=64, top_k=8, I=128, I_shared=128),
+    # router reduction split over blocks: 2 chunks; 3 chunks with a ragged last slice and a
+    # ragged last expert tile
+    dict(T=30, H=1024, E=96, top_k=6, I=128, I_shared=128),
+    dict(T=3, H=2176, E=200, top_k=8, I=128, I_shared=128),
 ]
 
 
