@@ -46,6 +46,7 @@ struct TcParams {
   int rows_out[2];             // rows of out[0] (T*k) and out[1] (T)
   int max_items;               // upper bound of the schedule length (host-computed)
   int ksplit;                  // gate/up: slices of the reduction per tile (1 = no split)
+  int sched_smem;              // copy the schedule tables into shared memory (room permitting)
   int max_tiles;               // bound of tile ids (split partial buffers)
   float* partial;              // [max_tiles][ksplit][BN][256] fp32 gate|up partial sums
   unsigned int* tile_done;     // [max_tiles] slices finished per tile, zero before the launch
@@ -85,23 +86,33 @@ struct Item {
   int nvalid;  // tokens in the tile
 };
 
+// The schedule tables (item_start, group_order, offsets), read from shared-memory copies
+// when the launch has room for them, else from global memory.
+struct Sched {
+  const int32_t* item_start;   // [G + 1]
+  const int32_t* group_order;  // [G]
+  const int32_t* offsets;      // [E + 1]
+  bool in_smem;
+  __device__ __forceinline__ int ld(const int32_t* q) const { return in_smem ? *q : __ldg(q); }
+};
+
 template <int BN>
-__device__ __forceinline__ Item decode_item(const TcParams& p, int it) {
+__device__ __forceinline__ Item decode_item(const TcParams& p, const Sched& sc, int it) {
   int lo = 0, hi = p.G - 1;
   while (lo < hi) {  // last group slot whose first item is <= it
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(p.item_start + mid) <= it) lo = mid; else hi = mid - 1;
+    if (sc.ld(sc.item_start + mid) <= it) lo = mid; else hi = mid - 1;
   }
   Item r;
-  r.g = __ldg(p.group_order + lo);
+  r.g = sc.ld(sc.group_order + lo);
   r.sh = (r.g == p.E) ? 1 : 0;
   const int ks_n = p.ksplit;
-  const int local_item = it - __ldg(p.item_start + lo);
+  const int local_item = it - sc.ld(sc.item_start + lo);
   const int local = local_item / ks_n;  // slices of one tile are consecutive items
   r.ks = local_item - local * ks_n;
   r.tile = it / ks_n;                   // every group's item count is a multiple of ks_n
-  const int base = r.sh ? 0 : __ldg(p.offsets + r.g);
-  const int cnt = r.sh ? static_cast<int>(p.T) : __ldg(p.offsets + r.g + 1) - base;
+  const int base = r.sh ? 0 : sc.ld(sc.offsets + r.g);
+  const int cnt = r.sh ? static_cast<int>(p.T) : sc.ld(sc.offsets + r.g + 1) - base;
   const int ntile = (cnt + BN - 1) / BN;
   r.m = ntile > 0 ? local / ntile : 0;
   const int n = local - r.m * ntile;
@@ -118,8 +129,8 @@ __device__ __forceinline__ Item decode_item(const TcParams& p, int it) {
 }
 
 // schedule length, clamped to the host bound (a larger value is reported, not run)
-__device__ __forceinline__ int schedule_length(const TcParams& p) {
-  const int total = __ldg(p.item_start + p.G);
+__device__ __forceinline__ int schedule_length(const TcParams& p, const Sched& sc) {
+  const int total = sc.ld(sc.item_start + p.G);
   if (total < 0 || total > p.max_items) {
     if (threadIdx.x == 0 && blockIdx.x == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
     return 0;
@@ -191,7 +202,18 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();
-  const int total = schedule_length(p);
+  Sched sc{p.item_start, p.group_order, p.offsets, false};
+  if (p.sched_smem) {
+    // one parallel copy of the tables instead of a chain of dependent global reads per item
+    int32_t* tab = reinterpret_cast<int32_t*>(aux + C::kAuxBytes);
+    const int G = p.G;
+    for (int i = threadIdx.x; i <= G; i += blockDim.x) tab[i] = __ldg(p.item_start + i);
+    for (int i = threadIdx.x; i < G; i += blockDim.x) tab[G + 1 + i] = __ldg(p.group_order + i);
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) tab[2 * G + 1 + i] = __ldg(p.offsets + i);
+    __syncthreads();
+    sc = Sched{tab, tab + G + 1, tab + 2 * G + 1, true};
+  }
+  const int total = schedule_length(p, sc);
 
   if (warp == 0) {
     // ------------------------------- TMA producer -------------------------------------
@@ -202,7 +224,7 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
     uint32_t used = 0;  // stages that ever received a copy
     bool ok = true;
     for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-      const Item t = decode_item<BN>(p, it);
+      const Item t = decode_item<BN>(p, sc, it);
       if (!t.valid) {
         if (blockIdx.x == 0 && lane == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
         continue;
@@ -263,7 +285,7 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-        const Item t = decode_item<BN>(p, it);
+        const Item t = decode_item<BN>(p, sc, it);
         if (!t.valid) continue;
         const int n_mma = (t.nvalid + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(kTileM, n_mma);
@@ -304,7 +326,7 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int it = blockIdx.x; it < total; it += gridDim.x) {
-      const Item t = decode_item<BN>(p, it);
+      const Item t = decode_item<BN>(p, sc, it);
       if (!t.valid) continue;
       if (!GATED && et < BN)
         sw[et] = (t.sh || et >= t.nvalid) ? 1.0f : __ldg(p.row_w + t.row0 + et);
@@ -504,13 +526,17 @@ static bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, ui
 }
 
 template <bool GATED, int BN>
-static cudaError_t launch_tc(const TcParams& prm, int num_sms, cudaStream_t st) {
+static cudaError_t launch_tc(const TcParams& prm_in, int num_sms, cudaStream_t st) {
   using C = TcCfg<GATED, BN>;
   auto kern = expert_gemm_tc_kernel<GATED, BN>;
+  TcParams prm = prm_in;
+  const size_t tables = static_cast<size_t>(2 * prm.G + 1 + prm.E + 1) * sizeof(int32_t);
+  prm.sched_smem = (C::kSmemBytes + tables <= static_cast<size_t>(kMaxDynSmem)) ? 1 : 0;
+  const size_t smem = C::kSmemBytes + (prm.sched_smem ? tables : 0);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       C::kSmemBytes);
+                                       static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  e = launch_pdl(kern, dim3(num_sms), dim3(192), static_cast<size_t>(C::kSmemBytes), st, prm);
+  e = launch_pdl(kern, dim3(num_sms), dim3(192), smem, st, prm);
   count_launches(1);
   return e;
 }
