@@ -98,7 +98,7 @@ struct Layout {
   size_t ctrl, group_done, tile_done, wss, zero_end, scores, xnorm, wnorm, idx, w, blk_hist, counts,
       offsets, group_order, item_start_gu, item_start_dn, perm, inv_perm, row_w, row_tok, partial, spill, rsplit,
       x_perm, h, h_shared, o, o_shared, total;
-  int bn, ksplit;
+  int bn, bn_dn, ksplit;
   int64_t max_tiles;
 };
 
@@ -115,6 +115,7 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
     return at;
   };
   L.bn = choose_tile_n(s->T, s->top_k, s->E);
+  L.bn_dn = choose_tile_n_down(s->T, s->top_k, s->E);
   L.ksplit = s->dtype == MOE_BF16 ? choose_ksplit(s->T, s->top_k, s->E, s->I, s->I_shared, L.bn) : 1;
   L.max_tiles = expert_tile_bound(s->T, s->top_k, s->E, s->I, s->I_shared, L.bn);
   // control block and counters first: one memset per forward clears them
@@ -275,6 +276,7 @@ extern "C" moe_status moe_layer_forward(const moe_layer_shape* shape, const void
   da.I = s.I;
   da.Is = s.I_shared;
   da.bn = L.bn;
+  da.bn_dn = L.bn_dn;
   da.ksplit = L.ksplit;
   da.x = x;
   da.idx = ra.idx_ws;
@@ -318,6 +320,7 @@ extern "C" moe_status moe_layer_forward(const moe_layer_shape* shape, const void
   ea.x_perm = da.x_perm;
   ea.row_tok = da.row_tok;
   ea.bn = L.bn;
+  ea.bn_dn = L.bn_dn;
   ea.ksplit = L.ksplit;
   ea.partial = static_cast<float*>(at(L.partial));
   ea.tile_done = static_cast<unsigned int*>(at(L.tile_done));

@@ -77,7 +77,7 @@ __device__ int block_scan_pair(int v0, int v1, int* warp_tot, int& total) {
 
 struct ScheduleArgs {
   int64_t T;
-  int E, has_shared, mt_gu, mt_gu_shared, mt_dn, bn, ksplit;
+  int E, has_shared, mt_gu, mt_gu_shared, mt_dn, bn, bn_dn, ksplit;
   int32_t* offsets;
   int32_t* group_order;
   int32_t* item_start_gu;
@@ -139,7 +139,8 @@ __device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* order, int*
   auto tiles = [&](int r, bool gu) -> int {
     if (r >= G) return 0;
     const int g = order[r];
-    const int nt = (cnt[g] + a.bn - 1) / a.bn;
+    const int bn = gu ? a.bn : a.bn_dn;
+    const int nt = (cnt[g] + bn - 1) / bn;
     const int mt = gu ? (g < E ? a.mt_gu : a.mt_gu_shared) * a.ksplit : a.mt_dn;
     return nt * mt;
   };
@@ -342,6 +343,7 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st) {
   sa.mt_gu_shared = a.Is / kTileM;
   sa.mt_dn = a.H / kTileM;
   sa.bn = a.bn;
+  sa.bn_dn = a.bn_dn;
   sa.ksplit = a.ksplit;
   sa.offsets = a.offsets;
   sa.group_order = a.group_order;

@@ -60,19 +60,25 @@ struct TcCfg {
   static constexpr int kABytes = kTileM * kTileK * 2;  // 16 KB of weights per operand tile
   static constexpr int kBBytes = BN * kTileK * 2;      // token rows
   static constexpr int kStageBytes = (GATED ? 2 : 1) * kABytes + kBBytes;
-  static constexpr int kStagingBytes = BN * kTileM * 2;  // epilogue tile [BN][128] bf16
-  static constexpr int kAuxBytes = 1024;                 // barriers, TMEM slot, row weights
+  // tiles of up to 128 tokens stage the output tile [BN][128] bf16 in shared memory for
+  // 16-byte stores; 256-token tiles store straight from registers (each warp writes 64
+  // contiguous bytes per token) to leave shared memory to the pipeline
+  static constexpr bool kStaged = BN <= 128;
+  static constexpr int kStagingBytes = kStaged ? BN * kTileM * 2 : 0;
+  static constexpr int kAuxBytes = 512 + (BN * 4 > 512 ? BN * 4 : 512);  // barriers, TMEM slot | row weights
   static constexpr int kFit = (kMaxDynSmem - kStagingBytes - 1024 - kAuxBytes) / kStageBytes;
   static constexpr int kStages = kFit > 12 ? 12 : kFit;
   static constexpr int kAccCols = (GATED ? 2 : 1) * BN;  // TMEM columns per accumulator
-  static constexpr int kTmemCols = (2 * kAccCols <= 32) ? 32 : (2 * kAccCols <= 64) ? 64
-                                 : (2 * kAccCols <= 128) ? 128 : (2 * kAccCols <= 256) ? 256 : 512;
+  static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;  // double-buffered when it fits
+  static constexpr int kTmemNeed = kAccBufs * kAccCols;
+  static constexpr int kTmemCols = (kTmemNeed <= 32) ? 32 : (kTmemNeed <= 64) ? 64
+                                 : (kTmemNeed <= 128) ? 128 : (kTmemNeed <= 256) ? 256 : 512;
   static constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + kAuxBytes;
   static_assert(kStages >= 2, "pipeline too shallow");
   static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
-  static_assert(2 * kAccCols <= 512, "accumulators exceed tensor memory");
+  static_assert(kTmemNeed <= 512, "accumulators exceed tensor memory");
   static_assert(kSmemBytes <= kMaxDynSmem, "shared memory budget");
-  static_assert(BN % 16 == 0 && BN <= 128, "tile width");
+  static_assert(BN % 16 == 0 && BN <= 256, "tile width");
 };
 
 struct Item {
@@ -312,7 +318,7 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
         }
         if (!ok) break;
         mma_commit(&tfull[acc]);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
       }
       // all MMAs issued by this thread complete before the accumulators are freed
       mma_commit(drain);
@@ -328,13 +334,43 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
     for (int it = blockIdx.x; it < total; it += gridDim.x) {
       const Item t = decode_item<BN>(p, sc, it);
       if (!t.valid) continue;
-      if (!GATED && et < BN)
-        sw[et] = (t.sh || et >= t.nvalid) ? 1.0f : __ldg(p.row_w + t.row0 + et);
+      if (!GATED)
+        for (int n = et; n < BN; n += 128)
+          sw[n] = (t.sh || n >= t.nvalid) ? 1.0f : __ldg(p.row_w + t.row0 + n);
       if (!mbar_wait(&tfull[acc], acc_phase, p.ctrl, abort_flag)) break;
       tc_fence_after();
       named_bar_sync(1, 128);  // staging free (previous tile copied out), sw visible
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::kAccCols;
-      if (GATED && p.ksplit > 1) {
+      if (!C::kStaged) {
+        // rows of this thread's output column, one token at a time, straight to global
+        const int ld = p.ld_out[t.sh];
+        __nv_bfloat16* out = p.out[t.sh] + static_cast<int64_t>(t.row0) * ld + t.m * kTileM + r;
+        for (int c0 = 0; c0 < t.nvalid; c0 += 16) {
+          uint32_t a[16];
+          tmem_ld16_nowait(trow + c0, a);
+          float v[16];
+          if (GATED) {
+            uint32_t u[16];
+            tmem_ld16_nowait(trow + BN + c0, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = silu_mul(__uint_as_float(a[j]), __uint_as_float(u[j]));
+          } else {
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(a[j]) * sw[c0 + j];
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < t.nvalid) out[static_cast<int64_t>(c0 + j) * ld] = __float2bfloat16_rn(v[j]);
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+        if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
+        named_bar_sync(1, 128);  // sw free for the next tile
+        continue;
+      }
+      if (GATED && C::kStaged && p.ksplit > 1) {
         // this slice's gate|up partial sums -> its own fp32 slab; the last slice of the
         // tile adds the slabs, applies SiLU(gate)*up and writes the tile
         float* slab = p.partial + (static_cast<int64_t>(t.tile) * p.ksplit + t.ks) * BN * 256;
@@ -352,7 +388,7 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
         }
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
         __threadfence();
         named_bar_sync(1, 128);
         if (et == 0) sw[0] = (atomicAdd(p.tile_done + t.tile, 1u) == static_cast<unsigned>(p.ksplit - 1)) ? 1.f : 0.f;
@@ -403,7 +439,7 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);  // the accumulator may be overwritten now
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
       named_bar_sync(1, 128);  // staging tile complete
       // rows of 128 bf16 (256 B) -> out[row0 + n][m*128 ...], 16-byte coalesced stores
       const int ld = p.ld_out[t.sh];
@@ -544,6 +580,9 @@ static cudaError_t launch_tc(const TcParams& prm_in, int num_sms, cudaStream_t s
 template <bool GATED>
 static cudaError_t launch_tc_bn(const TcParams& prm, int bn, int num_sms, cudaStream_t st) {
   if (bn == 16) return launch_tc<GATED, 16>(prm, num_sms, st);
+  if constexpr (!GATED) {
+    if (bn == 256) return launch_tc<false, 256>(prm, num_sms, st);
+  }
   return launch_tc<GATED, 128>(prm, num_sms, st);
 }
 
@@ -627,10 +666,10 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   // down: A = W_down viewed as [E*H, I]; B = h [P, I] (shared: Ws_down [H, Is], h_shared)
   TcParams d{};
   ok = encode_2d_bf16(&d.tmA[0], a.Wd, static_cast<uint64_t>(a.E) * a.H, a.I, kTileM) &&
-       encode_2d_bf16(&d.tmB[0], a.h, P, a.I, a.bn);
+       encode_2d_bf16(&d.tmB[0], a.h, P, a.I, a.bn_dn);
   if (has_shared)
     ok = ok && encode_2d_bf16(&d.tmA[1], a.Wsd, a.H, a.Is, kTileM) &&
-         encode_2d_bf16(&d.tmB[1], a.h_shared, a.T, a.Is, a.bn);
+         encode_2d_bf16(&d.tmB[1], a.h_shared, a.T, a.Is, a.bn_dn);
   else {
     d.tmA[1] = d.tmA[0];
     d.tmB[1] = d.tmB[0];
@@ -654,10 +693,10 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   d.rows_out[0] = static_cast<int>(P);
   d.rows_out[1] = static_cast<int>(a.T);
   d.ksplit = 1;
-  d.max_tiles = static_cast<int>(expert_tile_bound(a.T, a.k, a.E, a.H, a.Is > 0 ? a.H : 0, a.bn));
+  d.max_tiles = static_cast<int>(expert_tile_bound(a.T, a.k, a.E, a.H, a.Is > 0 ? a.H : 0, a.bn_dn));
   d.max_items = d.max_tiles;
   d.ctrl = a.ctrl;
-  return launch_tc_bn<false>(d, a.bn, a.num_sms, st);
+  return launch_tc_bn<false>(d, a.bn_dn, a.num_sms, st);
 }
 
 }  // namespace moe

@@ -18,10 +18,17 @@ constexpr int kTokBlock = 256;
 // rows of weights per tcgen05 tile (MMA M) and reduction elements per pipeline stage
 constexpr int kTileM = 128;
 constexpr int kTileK = 64;
-// tokens per tcgen05 tile (MMA N upper bound): 16 when experts hold a few tokens each
-// (decode), 128 otherwise
+// tokens per tcgen05 tile of the gate/up GEMM (MMA N upper bound): 16 when experts hold a
+// few tokens each (decode), 128 otherwise
 inline int choose_tile_n(int64_t T, int k, int E) {
   return (T * k <= static_cast<int64_t>(6) * E) ? 16 : 128;
+}
+// tokens per tile of the down GEMM: as gate/up, but 256 when experts hold 256 or more on
+// average (long prefill: a third less operand traffic per MMA cycle; its accumulators stay
+// double-buffered in tensor memory, unlike gate/up's pair of 256-column ones)
+inline int choose_tile_n_down(int64_t T, int k, int E) {
+  const int bn = choose_tile_n(T, k, E);
+  return (bn == 128 && T * k >= static_cast<int64_t>(256) * E) ? 256 : bn;
 }
 
 struct RouterArgs {
@@ -59,7 +66,8 @@ struct DispatchArgs {
   int64_t T;
   int H, E, k;
   int I, Is;        // expert widths (Is = 0: no shared expert)
-  int bn;           // tokens per GEMM tile
+  int bn;           // tokens per gate/up GEMM tile
+  int bn_dn;        // tokens per down GEMM tile
   int ksplit;       // gate/up reduction slices
   const void* x;
   const int32_t* idx;   // [T, k]
@@ -98,7 +106,8 @@ struct ExpertArgs {
   const float* row_w;
   const int32_t* row_tok;  // [T*k] token of each routed row (bf16: gathered from x)
   const void* x_perm;      // fp32 path: routed rows of x in expert order
-  int bn;           // tokens per GEMM tile (16 or 128)
+  int bn;           // tokens per gate/up GEMM tile (16 or 128)
+  int bn_dn;        // tokens per down GEMM tile (16, 128 or 256)
   int ksplit;       // gate/up reduction slices (1, 2 or 4)
   float* partial;   // split partial sums (ksplit > 1)
   unsigned int* tile_done;  // per-tile slice counters, zero before the forward

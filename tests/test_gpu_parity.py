@@ -49,6 +49,8 @@ SMALL = [
     # ragged last expert tile
     dict(T=30, H=1024, E=96, top_k=6, I=128, I_shared=128),
     dict(T=3, H=2176, E=200, top_k=8, I=128, I_shared=128),
+    # 256-token tiles (about 350 tokens per expert: one full and one ragged tile each)
+    dict(T=700, H=256, E=8, top_k=4, I=256, I_shared=128),
 ]
 
 
