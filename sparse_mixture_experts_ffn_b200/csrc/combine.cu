@@ -20,6 +20,7 @@ __global__ void combine_kernel(const int32_t* __restrict__ inv_perm, const T* __
                                const T* __restrict__ o_shared, int64_t Tn, int H, int k,
                                T* __restrict__ y, Ctrl* ctrl) {
   pdl_wait();
+  pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
   constexpr int V = Vec16<T>::N;
   const int vpr = H / V;
   const int64_t total = Tn * vpr;
@@ -75,7 +76,6 @@ __global__ void combine_kernel(const int32_t* __restrict__ inv_perm, const T* __
     for (int j = 0; j < V; ++j) out.v[j] = from_f32<T>(acc[j]);
     reinterpret_cast<uint4*>(y + t * H)[v] = *reinterpret_cast<const uint4*>(&out);
   }
-  pdl_trigger();
 }
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st) {

@@ -64,7 +64,11 @@ __device__ __forceinline__ Vec16<T> ld16(const T* p) {
 // one may start its prologue while the previous one drains.  pdl_wait() blocks until every
 // preceding kernel of the stream has completed and its memory is visible; it must come
 // before the first read of anything an earlier kernel wrote.  pdl_trigger() lets the next
-// kernel launch early.
+// kernel launch early: the dispatch, expert GEMM and combine kernels call it right after
+// pdl_wait(), so the next kernel's blocks are placed and run their prologue (barriers,
+// tensor memory, descriptor prefetch) while this one works, then wait in pdl_wait() for it
+// to finish.  The routing kernels and the single-block dispatch do not call it (their
+// dependents launch when they exit), which measured faster for the short decode chain.
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {

@@ -27,6 +27,7 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ i
                                                    Ctrl* ctrl) {
   extern __shared__ int sh_hist[];
   pdl_wait();
+  pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
   for (int e = threadIdx.x; e < E; e += blockDim.x) sh_hist[e] = 0;
   __syncthreads();
   const int64_t a0 = static_cast<int64_t>(blockIdx.x) * kTokBlock * k;
@@ -42,7 +43,6 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ i
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     blk_hist[static_cast<int64_t>(blockIdx.x) * E + e] = sh_hist[e];
-  pdl_trigger();
 }
 
 // exclusive scan of up to 2 * blockDim.x values held two per thread; blockDim.x = 1024
@@ -197,6 +197,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScheduleArgs sa, int k, int 
   __shared__ int order[2048];
   __shared__ int warp_tot[33];
   pdl_wait();
+  pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
   const int E = sa.E;
   // each warp scans the block counts of one expert at a time (lanes over blocks)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -224,7 +225,6 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScheduleArgs sa, int k, int 
   if (sa.has_shared && threadIdx.x == 0) cnt[E] = static_cast<int>(sa.T);
   __syncthreads();
   build_schedule(sa, cnt, order, warp_tot);
-  pdl_trigger();
 }
 
 // Placement for large batches: block b owns the assignments of tokens [256b, 256b+256);
@@ -239,6 +239,7 @@ __global__ void __launch_bounds__(32 * kPermWarps) permute_kernel(
     int32_t* __restrict__ row_tok, int32_t* __restrict__ perm_user) {
   extern __shared__ int wcnt[];  // [kPermWarps][E]
   pdl_wait();
+  pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) wcnt[i] = 0;
   __syncthreads();
@@ -263,7 +264,6 @@ __global__ void __launch_bounds__(32 * kPermWarps) permute_kernel(
   }
   __syncthreads();
   place_assignments(idx, w, a0, a1, k, E, mine, perm, inv_perm, row_w, row_tok, perm_user);
-  pdl_trigger();
 }
 
 // Small batches: histogram, scans, schedule and placement in one block.
@@ -302,7 +302,6 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
   __syncthreads();
   if (threadIdx.x < 32)
     place_assignments(idx, w, 0, P, k, E, base, perm, inv_perm, row_w, row_tok, perm_user);
-  pdl_trigger();
 }
 
 // x_perm[pos, :] = x[row_tok[pos], :], 16-byte vectors
@@ -311,6 +310,7 @@ __global__ void gather_rows_kernel(const T* __restrict__ x, const int32_t* __res
                                    int64_t P, int64_t Tn, int H, T* __restrict__ x_perm,
                                    Ctrl* ctrl) {
   pdl_wait();
+  pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
   constexpr int V = Vec16<T>::N;
   const int vpr = H / V;
   const int64_t total = P * vpr;
@@ -326,7 +326,6 @@ __global__ void gather_rows_kernel(const T* __restrict__ x, const int32_t* __res
     const uint4 val = __ldg(reinterpret_cast<const uint4*>(x + t * H) + v);
     reinterpret_cast<uint4*>(x_perm + p * H)[v] = val;
   }
-  pdl_trigger();
 }
 
 // assignments up to which the single-block path is used

@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();
+  pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
   Sched sc{p.item_start, p.group_order, p.offsets, false};
   if (p.sched_smem) {
     // one parallel copy of the tables instead of a chain of dependent global reads per item
@@ -451,7 +452,6 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
       }
     }
   }
-  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -77,7 +77,6 @@ __global__ void row_norm_ub_kernel(const T* __restrict__ A, int64_t rows_a, doub
     const double ss = warp_sumsq((first ? A : B) + r * H, H);
     if ((threadIdx.x & 31) == 0) (first ? out_a : out_b)[r] = norm_ub_from_sumsq(ss, H);
   }
-  pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------------------
@@ -695,7 +694,6 @@ __global__ void __launch_bounds__(32 * kSelectWarps) route_select_kernel(
                            key_spill(spill, T_, E, t), bias, x + t * H, Wr, H, E, k, t, idx_ws, w_ws,
                            idx_user, w_user, exact_scratch[warp], ctrl);
   }
-  pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------------------
@@ -820,7 +818,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) router_decode_kernel(
                              idx_user, w_user, exact_scratch[warp], ctrl);
     }
   }
-  pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1095,7 +1092,6 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
       }
     }
   }
-  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
