@@ -95,7 +95,7 @@ static int num_sms_current_device() {
 static size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
-  size_t ctrl, group_done, tile_done, wss, zero_end, scores, xnorm, wnorm, idx, w, blk_hist, counts,
+  size_t ctrl, group_done, tile_done, item_counters, wss, zero_end, scores, xnorm, wnorm, idx, w, blk_hist, counts,
       offsets, group_order, item_start_gu, item_start_dn, perm, inv_perm, row_w, row_tok, partial, spill, rsplit,
       x_perm, h, h_shared, o, o_shared, total;
   int bn, bn_dn, ksplit;
@@ -124,6 +124,7 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.ctrl = take(sizeof(Ctrl));
   L.group_done = take(groups * 4);
   L.tile_done = take(L.ksplit > 1 ? static_cast<size_t>(L.max_tiles) * 4 : 0);
+  L.item_counters = take(2 * 4);
   // the small-batch router accumulates scores and row sums of squares atomically
   L.wss = take(tc_scores ? 0 : groups * E * 8);
   L.scores = take(T * E * 8);
@@ -324,6 +325,7 @@ extern "C" moe_status moe_layer_forward(const moe_layer_shape* shape, const void
   ea.ksplit = L.ksplit;
   ea.partial = static_cast<float*>(at(L.partial));
   ea.tile_done = static_cast<unsigned int*>(at(L.tile_done));
+  ea.item_counters = static_cast<unsigned int*>(at(L.item_counters));
   ea.h = at(L.h);
   ea.h_shared = at(L.h_shared);
   ea.o = at(L.o);

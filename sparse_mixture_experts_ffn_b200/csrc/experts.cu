@@ -50,10 +50,12 @@ struct TcParams {
   int max_tiles;               // bound of tile ids (split partial buffers)
   float* partial;              // [max_tiles][ksplit][BN][256] fp32 gate|up partial sums
   unsigned int* tile_done;     // [max_tiles] slices finished per tile, zero before the launch
+  unsigned int* item_counter;  // items claimed beyond the first gridDim.x, zero before the launch
   Ctrl* ctrl;
 };
 
 constexpr int kMaxDynSmem = 232448;  // 227 KB per block on sm_100
+constexpr int kRing = 4;             // item slots between the producer and the other roles
 
 template <bool GATED, int BN>
 struct TcCfg {
@@ -164,7 +166,10 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 //   warp 1      allocates tensor memory; one lane issues the tcgen05 MMAs
 //   warps 2..5  epilogue: tensor memory -> registers -> shared staging tile -> global
 // Accumulators are double-buffered in tensor memory, so the epilogue of one tile overlaps
-// the main loop of the next.
+// the main loop of the next.  Items are claimed dynamically: block b starts with item b and
+// then takes the next unclaimed one from a global counter, so blocks that draw short tiles
+// take more of them; the producer publishes each claimed item to the MMA and epilogue warps
+// through a ring of kRing shared-memory slots (index -1 ends the schedule).
 template <bool GATED, int BN>
 __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
   using C = TcCfg<GATED, BN>;
@@ -180,6 +185,9 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* ring_full = reinterpret_cast<uint64_t*>(aux + 384);  // [kRing]
+  uint64_t* ring_empty = ring_full + kRing;                     // [kRing]
+  volatile int* ring = reinterpret_cast<volatile int*>(ring_empty + kRing);  // [kRing] item ids
   float* sw = reinterpret_cast<float*>(aux + 512);  // [BN] routing weights of the tile rows
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -193,6 +201,10 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
       mbar_init(&tempty[a], 4 * 32);
     }
     mbar_init(drain, 1);
+    for (int q = 0; q < kRing; ++q) {
+      mbar_init(&ring_full[q], 1);
+      mbar_init(&ring_empty[q], 1 + 4);  // the MMA thread and one lane per epilogue warp
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -230,8 +242,29 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
     uint32_t phase = 0;
     uint32_t used = 0;  // stages that ever received a copy
     bool ok = true;
-    for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
-      const Item t = decode_item<BN>(p, sc, it);
+    int q = 0;
+    uint32_t qphase = 0;
+    // the item after the current one is claimed while the current one streams
+    int it = static_cast<int>(blockIdx.x);
+    int claimed = (lane == 0) ? static_cast<int>(atomicAdd(p.item_counter, 1u) + gridDim.x) : 0;
+    for (;;) {
+      if (it >= total || !ok) it = -1;
+      // publish the item (or the end) to the MMA and epilogue warps
+      int pub = 1;
+      if (lane == 0) {
+        pub = mbar_wait(&ring_empty[q], qphase ^ 1u, p.ctrl, abort_flag) ? 1 : 0;
+        if (pub) {
+          ring[q] = it;
+          mbar_arrive(&ring_full[q]);
+        }
+      }
+      pub = __shfl_sync(0xffffffffu, pub, 0);
+      if (++q == kRing) { q = 0; qphase ^= 1u; }
+      if (!pub || it < 0) break;
+      const int cur = it;
+      it = __shfl_sync(0xffffffffu, claimed, 0);
+      if (lane == 0 && it < total) claimed = static_cast<int>(atomicAdd(p.item_counter, 1u) + gridDim.x);
+      const Item t = decode_item<BN>(p, sc, cur);
       if (!t.valid) {
         if (blockIdx.x == 0 && lane == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
         continue;
@@ -291,7 +324,14 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      int q = 0;
+      uint32_t qphase = 0;
+      while (ok) {
+        if (!mbar_wait(&ring_full[q], qphase, p.ctrl, abort_flag)) break;
+        const int it = ring[q];
+        mbar_arrive(&ring_empty[q]);
+        if (++q == kRing) { q = 0; qphase ^= 1u; }
+        if (it < 0) break;
         const Item t = decode_item<BN>(p, sc, it);
         if (!t.valid) continue;
         const int n_mma = (t.nvalid + 15) & ~15;
@@ -332,7 +372,15 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
     const int et = threadIdx.x - 64;    // 0..127
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int it = blockIdx.x; it < total; it += gridDim.x) {
+    int q = 0;
+    uint32_t qphase = 0;
+    for (;;) {
+      if (!mbar_wait(&ring_full[q], qphase, p.ctrl, abort_flag)) break;
+      const int it = ring[q];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ring_empty[q]);
+      if (++q == kRing) { q = 0; qphase ^= 1u; }
+      if (it < 0) break;
       const Item t = decode_item<BN>(p, sc, it);
       if (!t.valid) continue;
       if (!GATED)
@@ -657,6 +705,7 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   g.max_items = g.max_tiles * a.ksplit;
   g.partial = a.partial;
   g.tile_done = a.tile_done;
+  g.item_counter = a.item_counters;
   g.ctrl = a.ctrl;
   g.ld_out[0] = a.I;
   g.ld_out[1] = a.Is;
@@ -695,6 +744,7 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   d.ksplit = 1;
   d.max_tiles = static_cast<int>(expert_tile_bound(a.T, a.k, a.E, a.H, a.Is > 0 ? a.H : 0, a.bn_dn));
   d.max_items = d.max_tiles;
+  d.item_counter = a.item_counters + 1;
   d.ctrl = a.ctrl;
   return launch_tc_bn<false>(d, a.bn_dn, a.num_sms, st);
 }

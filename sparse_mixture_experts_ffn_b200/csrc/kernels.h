@@ -111,6 +111,7 @@ struct ExpertArgs {
   int ksplit;       // gate/up reduction slices (1, 2 or 4)
   float* partial;   // split partial sums (ksplit > 1)
   unsigned int* tile_done;  // per-tile slice counters, zero before the forward
+  unsigned int* item_counters;  // [2] dynamic item claims of the two GEMMs, zero before the forward
   void* h;          // [T*k, I]
   void* h_shared;   // [T, Is]
   void* o;          // [T*k, H]
