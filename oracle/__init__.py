@@ -56,10 +56,11 @@ def _load():
                                              P, P, P, ctypes.c_int]
         lib.oracle_route.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, P, P, P, P]
         lib.oracle_dispatch.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, P, P, P, P]
-        lib.oracle_expert_act.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P]
+        D = ctypes.c_double
+        lib.oracle_expert_act.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, D, P]
         lib.oracle_moe_tokens.argtypes = [ctypes.c_int, ctypes.c_int64, P, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P,
-                                          P, P, ctypes.c_int]
+                                          P, D, D, P, ctypes.c_int]
         for f in (lib.oracle_exact_dot, lib.oracle_router_scores, lib.oracle_route,
                   lib.oracle_dispatch, lib.oracle_expert_act, lib.oracle_moe_tokens):
             f.restype = ctypes.c_int
@@ -142,17 +143,21 @@ def dispatch(idx: np.ndarray, E: int):
     return counts, offsets, perm, inv
 
 
-def expert_act(xrow: np.ndarray, Wgu_e: np.ndarray) -> np.ndarray:
-    """SiLU(x W_g^T) * (x W_u^T) of one token through one expert, fp64 [I]."""
+def expert_act(xrow: np.ndarray, Wgu_e: np.ndarray, swiglu_limit: float = 0.0) -> np.ndarray:
+    """SiLU(x W_g^T) * (x W_u^T) of one token through one expert, fp64 [I]; a SwiGLU limit
+    L > 0 first clamps gate to <= L and up to [-L, L]."""
     xrow, Wgu_e = _c(xrow), _c(Wgu_e)
     twoI, H = Wgu_e.shape
     out = np.empty(twoI // 2, np.float64)
-    _load().oracle_expert_act(_dtype_code(xrow), H, twoI // 2, _p(xrow), _p(Wgu_e), _p(out))
+    _load().oracle_expert_act(_dtype_code(xrow), H, twoI // 2, _p(xrow), _p(Wgu_e),
+                              float(swiglu_limit), _p(out))
     return out
 
 
-def moe_tokens(x, idx, w64, Wgu, Wd, Wsgu=None, Wsd=None, tokens=None, nthreads: int = 0):
-    """Layer output (fp64 [n, H]) for the listed tokens (all tokens when ``tokens`` is None)."""
+def moe_tokens(x, idx, w64, Wgu, Wd, Wsgu=None, Wsd=None, tokens=None, nthreads: int = 0,
+               swiglu_limit: float = 0.0, swiglu_limit_shared: float = 0.0):
+    """Layer output (fp64 [n, H]) for the listed tokens (all tokens when ``tokens`` is None).
+    swiglu_limit / swiglu_limit_shared: SwiGLU limits of the routed / shared experts (0: none)."""
     x, Wgu, Wd = _c(x), _c(Wgu), _c(Wd)
     Wsgu, Wsd = _c(Wsgu), _c(Wsd)
     idx = _c(idx, np.int32)
@@ -169,6 +174,7 @@ def moe_tokens(x, idx, w64, Wgu, Wd, Wsgu=None, Wsd=None, tokens=None, nthreads:
     y = np.empty((tok.shape[0], H), np.float64)
     rc = _load().oracle_moe_tokens(_dtype_code(x), tok.shape[0], _p(tok), H, E, k, twoI // 2, Is,
                                    _p(x), _p(idx), _p(w64), _p(Wgu), _p(Wd), _p(Wsgu), _p(Wsd),
+                                   float(swiglu_limit), float(swiglu_limit_shared),
                                    _p(y), nthreads or nthreads_default())
     if rc != 0:
         raise ValueError("moe_tokens: expert index out of range")
@@ -176,7 +182,7 @@ def moe_tokens(x, idx, w64, Wgu, Wd, Wsgu=None, Wsd=None, tokens=None, nthreads:
 
 
 def moe_forward(x, Wr, Wgu, Wd, Wsgu=None, Wsd=None, top_k=8, bias=None, tokens=None,
-                nthreads: int = 0):
+                nthreads: int = 0, swiglu_limit: float = 0.0, swiglu_limit_shared: float = 0.0):
     """The whole layer: routing for every token, output for ``tokens`` (default all).
 
     Returns a dict with scores, idx, w, w64, counts, offsets, perm, inv_perm and y (fp64).
@@ -184,6 +190,7 @@ def moe_forward(x, Wr, Wgu, Wd, Wsgu=None, Wsd=None, top_k=8, bias=None, tokens=
     s = router_scores(x, Wr, nthreads)
     idx, w, w64 = route(s, top_k, bias)
     counts, offsets, perm, inv = dispatch(idx, Wr.shape[0])
-    y = moe_tokens(x, idx, w64, Wgu, Wd, Wsgu, Wsd, tokens=tokens, nthreads=nthreads)
+    y = moe_tokens(x, idx, w64, Wgu, Wd, Wsgu, Wsd, tokens=tokens, nthreads=nthreads,
+                   swiglu_limit=swiglu_limit, swiglu_limit_shared=swiglu_limit_shared)
     return dict(scores=s, idx=idx, w=w, w64=w64, counts=counts, offsets=offsets, perm=perm,
                 inv_perm=inv, y=y)

@@ -27,7 +27,12 @@
  *   - key[t,e] = fp32(s[t,e] + b[e]) when a router bias is given, else s[t,e];
  *   - selection by (key descending, expert index ascending), stored by ascending index;
  *   - routing weights: softmax over the selected keys, in fp64;
- *   - expert FFNs and the combine: fp64, sequential accumulation.
+ *   - expert FFNs and the combine: fp64, sequential accumulation;
+ *   - SwiGLU limits (same table: swiglu_limits "0.0x46 + 7x2" for the routed experts,
+ *     swiglu_limits_shared "0.0x47 + 16x1" for the shared one): the page gives only the
+ *     values.  Read here as a clamp of the activation inputs when the limit L > 0:
+ *     gate <- min(gate, L), up <- min(max(up, -L), L), then SiLU(gate)*up; L = 0 means
+ *     no clamp (the value of almost every layer).
  *
  * Parity status: every function here is pinned by tests (exact rational sums,
  * brute-force subset enumeration, closed forms and invariants); none is unpinned.
@@ -309,8 +314,19 @@ int oracle_dispatch(int64_t T, int E, int k, const int32_t* idx, int32_t* counts
  *   a_i = SiLU(g_i) * u_i,      SiLU(z) = z / (1 + exp(-z))
  *   out_h += scale * sum_i a_i Wd[h, i]
  * ---------------------------------------------------------------------------------- */
+/* SiLU(gate) * up with the SwiGLU limit L (0: none) applied to the inputs. */
+static double swiglu(double g, double u, double limit) {
+  if (limit > 0.0) {
+    if (g > limit) g = limit;
+    if (u > limit) u = limit;
+    if (u < -limit) u = -limit;
+  }
+  return g / (1.0 + exp(-g)) * u;
+}
+
 static void gated_ffn_acc(int dtype, int H, int I, const void* xrow, const void* Wgu,
-                          const void* Wd, double scale, double* out, double* a /*[I]*/) {
+                          const void* Wd, double scale, double limit, double* out,
+                          double* a /*[I]*/) {
   for (int i = 0; i < I; ++i) {
     double g = 0.0, u = 0.0;
     for (int h = 0; h < H; ++h) {
@@ -318,7 +334,7 @@ static void gated_ffn_acc(int dtype, int H, int I, const void* xrow, const void*
       g += xv * to_f64(dtype, Wgu, (size_t)i * H + h);
       u += xv * to_f64(dtype, Wgu, (size_t)(I + i) * H + h);
     }
-    a[i] = g / (1.0 + exp(-g)) * u;
+    a[i] = swiglu(g, u, limit);
   }
   for (int h = 0; h < H; ++h) {
     double o = 0.0;
@@ -330,7 +346,7 @@ static void gated_ffn_acc(int dtype, int H, int I, const void* xrow, const void*
 /* The intermediate activation of one token through one expert (exposed so that the
    tests can pin the gate/up/SiLU step on its own). */
 int oracle_expert_act(int dtype, int H, int I, const void* xrow, const void* Wgu_e,
-                      double* act_out) {
+                      double limit, double* act_out) {
   for (int i = 0; i < I; ++i) {
     double g = 0.0, u = 0.0;
     for (int h = 0; h < H; ++h) {
@@ -338,7 +354,7 @@ int oracle_expert_act(int dtype, int H, int I, const void* xrow, const void* Wgu
       g += xv * to_f64(dtype, Wgu_e, (size_t)i * H + h);
       u += xv * to_f64(dtype, Wgu_e, (size_t)(I + i) * H + h);
     }
-    act_out[i] = g / (1.0 + exp(-g)) * u;
+    act_out[i] = swiglu(g, u, limit);
   }
   return 0;
 }
@@ -349,12 +365,13 @@ int oracle_expert_act(int dtype, int H, int I, const void* xrow, const void* Wgu
  * The shared expert (share_expert_dim) is always on with weight 1; pass NULL shared
  * weights for a layer without one.  Weight layouts: Wgu [E, 2I, H], Wd [E, H, I],
  * Wsgu [2Is, H], Wsd [H, Is].  tok[n] is the token whose output goes to y[n, :];
- * idx/w are indexed by token.
+ * idx/w are indexed by token.  limit / limit_shared: SwiGLU limits of the routed and the
+ * shared experts (0: none).
  * ---------------------------------------------------------------------------------- */
 int oracle_moe_tokens(int dtype, int64_t ntok, const int64_t* tok, int H, int E, int k, int I,
                       int Is, const void* x, const int32_t* idx, const double* w,
                       const void* Wgu, const void* Wd, const void* Wsgu, const void* Wsd,
-                      double* y, int nthreads) {
+                      double limit, double limit_shared, double* y, int nthreads) {
   size_t es = esize(dtype);
   int bad = 0;
 #ifdef _OPENMP
@@ -376,9 +393,9 @@ int oracle_moe_tokens(int dtype, int64_t ntok, const int64_t* tok, int H, int E,
       }
       const char* gu = (const char*)Wgu + (size_t)e * 2 * I * H * es;
       const char* d = (const char*)Wd + (size_t)e * H * I * es;
-      gated_ffn_acc(dtype, H, I, xr, gu, d, w[t * k + j], out, a);
+      gated_ffn_acc(dtype, H, I, xr, gu, d, w[t * k + j], limit, out, a);
     }
-    if (Wsgu && Wsd && Is > 0) gated_ffn_acc(dtype, H, Is, xr, Wsgu, Wsd, 1.0, out, a);
+    if (Wsgu && Wsd && Is > 0) gated_ffn_acc(dtype, H, Is, xr, Wsgu, Wsd, 1.0, limit_shared, out, a);
     free(a);
   }
   return bad ? -1 : 0;

@@ -252,11 +252,31 @@ def test_silu_gate_up_closed_form():
     assert abs(act[0] - 1.5 * float(ln3)) > 0.1
 
 
-def _numpy_ffn(x, Wgu, Wd):
+def test_swiglu_limit_closed_form():
+    """The SwiGLU limit L (llm-atlas page "Step-3.5-Flash", table "Champs bruts du
+    config.json": swiglu_limits, swiglu_limits_shared; values only) read as a clamp of the
+    activation inputs: gate <- min(gate, L), up <- clip(up, -L, L); L = 0 is no clamp."""
+    x = np.array([1.0], np.float32)
+    s7 = 7.0 / (1.0 + math.exp(-7.0))  # SiLU(7)
+    cases = [  # gate, up, L, expected
+        (10.0, 10.0, 7.0, s7 * 7.0),                                  # both clamped
+        (10.0, -10.0, 7.0, s7 * -7.0),                                # up clamped from below
+        (-10.0, 3.0, 7.0, -10.0 / (1.0 + math.exp(10.0)) * 3.0),     # gate has no lower clamp
+        (5.0, 5.0, 7.0, 5.0 / (1.0 + math.exp(-5.0)) * 5.0),         # inside the limit
+        (10.0, 10.0, 0.0, 10.0 / (1.0 + math.exp(-10.0)) * 10.0),    # L = 0: no clamp
+    ]
+    for g, u, L, want in cases:
+        act = oracle.expert_act(x, np.array([[g], [u]], np.float32), swiglu_limit=L)
+        assert abs(act[0] - want) <= 1e-12 * max(1.0, abs(want)), (g, u, L, act[0], want)
+
+
+def _numpy_ffn(x, Wgu, Wd, limit=0.0):
     """Dense gated FFN with numpy fp64 matmuls (a library routine, not the oracle)."""
     I = Wgu.shape[0] // 2
     g = x @ Wgu[:I].T
     u = x @ Wgu[I:].T
+    if limit > 0:
+        g, u = np.minimum(g, limit), np.clip(u, -limit, limit)
     return (silu(g) * u) @ Wd.T
 
 
@@ -281,6 +301,25 @@ def test_identical_experts_reduce_to_one_dense_ffn(dtype):
     x = _f64(d["x"])
     want = _numpy_ffn(x, _f64(Wgu[0]), _f64(Wd[0])) + _numpy_ffn(x, _f64(d["Ws_gate_up"]), _f64(d["Ws_down"]))
     assert np.allclose(r["y"], want, rtol=1e-10, atol=1e-12)
+
+
+def test_swiglu_limits_of_routed_and_shared_experts():
+    """Identical routed experts with limit 0.3 and a shared expert with limit 0.2 reduce to
+    two dense clamped FFNs (numpy); swapping the two limits would fail."""
+    cfg = _small("f32", w_std=0.2)
+    d = inputs.make_inputs(cfg)
+    Wgu = d["W_gate_up"][:1].expand(cfg.E, -1, -1).contiguous()
+    Wd = d["W_down"][:1].expand(cfg.E, -1, -1).contiguous()
+    r = oracle.moe_forward(to_oracle(d["x"]), to_oracle(d["W_router"]), to_oracle(Wgu), to_oracle(Wd),
+                           to_oracle(d["Ws_gate_up"]), to_oracle(d["Ws_down"]), top_k=cfg.top_k,
+                           swiglu_limit=0.3, swiglu_limit_shared=0.2)
+    x = _f64(d["x"])
+    want = _numpy_ffn(x, _f64(Wgu[0]), _f64(Wd[0]), 0.3) + _numpy_ffn(x, _f64(d["Ws_gate_up"]),
+                                                                        _f64(d["Ws_down"]), 0.2)
+    assert np.allclose(r["y"], want, rtol=1e-10, atol=1e-12)
+    unclamped = _numpy_ffn(x, _f64(Wgu[0]), _f64(Wd[0])) + _numpy_ffn(x, _f64(d["Ws_gate_up"]),
+                                                                       _f64(d["Ws_down"]))
+    assert np.abs(want - unclamped).max() > 1e-3  # the clamps are active on these inputs
 
 
 def test_top_k_equal_E_is_the_full_softmax_mixture():
