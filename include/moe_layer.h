@@ -110,6 +110,27 @@ MOE_API moe_status moe_layer_forward(const moe_layer_shape* shape, const void* x
                              moe_routing_out* routing, void* workspace, size_t workspace_bytes,
                              void* stream);
 
+/* Per-layer options of moe_layer_forward_ex().
+ *   swiglu_limit, swiglu_limit_shared: the SwiGLU limits of the routed experts and of the
+ *   shared expert (llm-atlas page "Step-3.5-Flash", table "Champs bruts du config.json":
+ *   swiglu_limits "0.0x46 + 7x2", swiglu_limits_shared "0.0x47 + 16x1"; the page gives
+ *   the values only).  A limit L > 0 clamps the activation inputs, gate to <= L and up to
+ *   [-L, L], before SiLU(gate)*up; 0 means no clamp.  Limits must be finite and >= 0. */
+typedef struct {
+  float swiglu_limit;
+  float swiglu_limit_shared;
+} moe_layer_options;
+
+/* moe_layer_forward() with per-layer options; options = NULL is moe_layer_forward().
+ * Errors as moe_layer_forward(), plus MOE_ERR_INVALID_ARG for a negative or non-finite
+ * limit. */
+MOE_API moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const void* x,
+                                        const void* W_router, const float* router_bias,
+                                        const void* W_gate_up, const void* W_down,
+                                        const void* Ws_gate_up, const void* Ws_down, void* y,
+                                        moe_routing_out* routing, const moe_layer_options* options,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then returns the device status word of the most recent
  * moe_layer_forward() that used this workspace (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or
  * MOE_ERR_DEVICE_BOUNDS), or MOE_ERR_CUDA if the stream itself reports an error. */

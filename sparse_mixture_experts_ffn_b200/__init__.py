@@ -24,7 +24,7 @@ STATUS_NAMES = {
     3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT",
     6: "MOE_ERR_DEVICE_BOUNDS",
 }
-EXPORTED = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_layer_check_status",
+EXPORTED = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_layer_forward_ex", "moe_layer_check_status",
             "moe_layer_route_stats", "moe_layer_workspace_layout", "moe_layer_profile_enable",
             "moe_layer_profile_read", "moe_layer_launch_count", "moe_status_string")
 STAGES = ("routing", "dispatch", "gate_up", "down", "combine")
@@ -34,6 +34,10 @@ class MoEShape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("H", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("I", ctypes.c_int32), ("I_shared", ctypes.c_int32), ("top_k", ctypes.c_int32),
                 ("dtype", ctypes.c_int32)]
+
+
+class MoEOptions(ctypes.Structure):
+    _fields_ = [("swiglu_limit", ctypes.c_float), ("swiglu_limit_shared", ctypes.c_float)]
 
 
 class MoERoutingOut(ctypes.Structure):
@@ -76,6 +80,10 @@ def load_library(path: str = LIB_PATH):
     lib.moe_layer_forward.argtypes = [ctypes.POINTER(MoEShape), P, P, P, P, P, P, P, P,
                                       ctypes.POINTER(MoERoutingOut), P, ctypes.c_size_t, P]
     lib.moe_layer_forward.restype = ctypes.c_int
+    lib.moe_layer_forward_ex.argtypes = [ctypes.POINTER(MoEShape), P, P, P, P, P, P, P, P,
+                                         ctypes.POINTER(MoERoutingOut), ctypes.POINTER(MoEOptions), P,
+                                         ctypes.c_size_t, P]
+    lib.moe_layer_forward_ex.restype = ctypes.c_int
     lib.moe_layer_check_status.argtypes = [P, P]
     lib.moe_layer_check_status.restype = ctypes.c_int
     lib.moe_layer_route_stats.argtypes = [P, ctypes.POINTER(MoERouteStats), P]
@@ -136,12 +144,14 @@ def alloc_workspace(shape: MoEShape, device):
 
 
 def moe_layer_forward(x, W_router, W_gate_up, W_down, Ws_gate_up=None, Ws_down=None, *, top_k,
-                      router_bias=None, y=None, workspace=None, routing=True, stream=None):
+                      router_bias=None, y=None, workspace=None, routing=True, stream=None,
+                      swiglu_limit=0.0, swiglu_limit_shared=0.0):
     """Run the MoE layer on the device.  Returns (y, Routing or None).
 
     Shapes: x [T,H], W_router [E,H], W_gate_up [E,2I,H], W_down [E,H,I], Ws_gate_up
     [2Is,H], Ws_down [H,Is] (or both None), router_bias [E] fp32 or None.  All CUDA,
-    contiguous, same dtype (bf16 or fp32).
+    contiguous, same dtype (bf16 or fp32).  swiglu_limit / swiglu_limit_shared: SwiGLU
+    limits of the routed / shared experts (gate <= L, up in [-L, L]; 0 = none).
     """
     import torch
     lib = load_library()
@@ -171,12 +181,14 @@ def moe_layer_forward(x, W_router, W_gate_up, W_down, Ws_gate_up=None, Ws_down=N
                              r.offsets.data_ptr(), r.perm.data_ptr())
     if stream is None:
         stream = torch.cuda.current_stream(x.device)
-    rc = lib.moe_layer_forward(ctypes.byref(shape), _ptr(x), _ptr(W_router), _ptr(router_bias),
-                               _ptr(W_gate_up), _ptr(W_down), _ptr(Ws_gate_up), _ptr(Ws_down),
-                               _ptr(y), ctypes.byref(rout) if rout is not None else None,
-                               _ptr(workspace), workspace.numel(), ctypes.c_void_p(stream.cuda_stream))
+    opts = MoEOptions(float(swiglu_limit), float(swiglu_limit_shared))
+    rc = lib.moe_layer_forward_ex(ctypes.byref(shape), _ptr(x), _ptr(W_router), _ptr(router_bias),
+                                  _ptr(W_gate_up), _ptr(W_down), _ptr(Ws_gate_up), _ptr(Ws_down),
+                                  _ptr(y), ctypes.byref(rout) if rout is not None else None,
+                                  ctypes.byref(opts), _ptr(workspace), workspace.numel(),
+                                  ctypes.c_void_p(stream.cuda_stream))
     if rc != MOE_OK:
-        raise MoEError(rc, "moe_layer_forward")
+        raise MoEError(rc, "moe_layer_forward_ex")
     return y, r
 
 

@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <float.h>
 #include <string.h>
 
 #include <atomic>
@@ -210,6 +211,20 @@ extern "C" moe_status moe_layer_forward(const moe_layer_shape* shape, const void
                                         const void* Ws_gate_up, const void* Ws_down, void* y,
                                         moe_routing_out* routing, void* workspace,
                                         size_t workspace_bytes, void* stream) {
+  return moe_layer_forward_ex(shape, x, W_router, router_bias, W_gate_up, W_down, Ws_gate_up, Ws_down,
+                              y, routing, nullptr, workspace, workspace_bytes, stream);
+}
+
+extern "C" moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const void* x,
+                                           const void* W_router, const float* router_bias,
+                                           const void* W_gate_up, const void* W_down,
+                                           const void* Ws_gate_up, const void* Ws_down, void* y,
+                                           moe_routing_out* routing, const moe_layer_options* options,
+                                           void* workspace, size_t workspace_bytes, void* stream) {
+  const moe_layer_options opt = options ? *options : moe_layer_options{0.0f, 0.0f};
+  if (!(opt.swiglu_limit >= 0.0f && opt.swiglu_limit <= FLT_MAX) ||
+      !(opt.swiglu_limit_shared >= 0.0f && opt.swiglu_limit_shared <= FLT_MAX))
+    return MOE_ERR_INVALID_ARG;  // negative, infinite or NaN
   const moe_status vs = validate_shape(shape);
   if (vs != MOE_OK) return vs;
   const moe_layer_shape& s = *shape;
@@ -325,6 +340,8 @@ extern "C" moe_status moe_layer_forward(const moe_layer_shape* shape, const void
   ea.ksplit = L.ksplit;
   ea.partial = static_cast<float*>(at(L.partial));
   ea.tile_done = static_cast<unsigned int*>(at(L.tile_done));
+  ea.swiglu_limit = opt.swiglu_limit;
+  ea.swiglu_limit_shared = opt.swiglu_limit_shared;
   ea.item_counters = static_cast<unsigned int*>(at(L.item_counters));
   ea.h = at(L.h);
   ea.h_shared = at(L.h_shared);

@@ -47,6 +47,7 @@ struct TcParams {
   int max_items;               // upper bound of the schedule length (host-computed)
   int ksplit;                  // gate/up: slices of the reduction per tile (1 = no split)
   int sched_smem;              // copy the schedule tables into shared memory (room permitting)
+  float limit[2];              // gate/up: SwiGLU limits, routed and shared (0: none)
   int max_tiles;               // bound of tile ids (split partial buffers)
   float* partial;              // [max_tiles][ksplit][BN][256] fp32 gate|up partial sums
   unsigned int* tile_done;     // [max_tiles] slices finished per tile, zero before the launch
@@ -146,7 +147,14 @@ __device__ __forceinline__ int schedule_length(const TcParams& p, const Sched& s
   return total;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) {
+// SiLU(gate) * up; a SwiGLU limit L > 0 first clamps gate to <= L and up to [-L, L]
+// (limits of llm-atlas page "Step-3.5-Flash", table "Champs bruts du config.json":
+// swiglu_limits, swiglu_limits_shared)
+__device__ __forceinline__ float swiglu(float g, float u, float L) {
+  if (L > 0.0f) {
+    g = fminf(g, L);
+    u = fminf(fmaxf(u, -L), L);
+  }
   return g / (1.0f + __expf(-g)) * u;
 }
 
@@ -403,7 +411,7 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
             tmem_ld16_nowait(trow + BN + c0, u);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = silu_mul(__uint_as_float(a[j]), __uint_as_float(u[j]));
+            for (int j = 0; j < 16; ++j) v[j] = swiglu(__uint_as_float(a[j]), __uint_as_float(u[j]), p.limit[t.sh]);
           } else {
             tmem_wait_ld();
 #pragma unroll
@@ -453,7 +461,7 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
             gs += __ldcg(tile_slabs + (static_cast<int64_t>(q) * BN + n) * 256 + r);
             us += __ldcg(tile_slabs + (static_cast<int64_t>(q) * BN + n) * 256 + 128 + r);
           }
-          staging[n * kTileM + r] = __float2bfloat16_rn(silu_mul(gs, us));
+          staging[n * kTileM + r] = __float2bfloat16_rn(swiglu(gs, us, p.limit[t.sh]));
         }
         named_bar_sync(1, 128);
         const int ld = p.ld_out[t.sh];
@@ -477,7 +485,7 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
           for (int j = 0; j < 16; ++j)
             if (c0 + j < t.nvalid)
               staging[(c0 + j) * kTileM + r] =
-                  __float2bfloat16_rn(silu_mul(__uint_as_float(a[j]), __uint_as_float(u[j])));
+                  __float2bfloat16_rn(swiglu(__uint_as_float(a[j]), __uint_as_float(u[j]), p.limit[t.sh]));
         } else {
           tmem_wait_ld();
 #pragma unroll
@@ -522,12 +530,14 @@ __global__ void gate_up_f32_kernel(const float* __restrict__ x_perm, const float
                                    const int32_t* __restrict__ offsets,
                                    const float* __restrict__ Wgu, const float* __restrict__ Wsgu,
                                    int64_t P, int64_t T, int H, int E, int I, int Is,
+                                   float limit, float limit_shared,
                                    float* __restrict__ h, float* __restrict__ hs) {
   const int64_t n_routed = P * I, total = n_routed + T * Is;
   for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < total;
        q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const float *xr, *wg, *wu;
     float* dst;
+    float L = limit;
     if (q < n_routed) {
       const int64_t p = q / I;
       const int i = static_cast<int>(q - p * I);
@@ -544,12 +554,17 @@ __global__ void gate_up_f32_kernel(const float* __restrict__ x_perm, const float
       wg = Wsgu + static_cast<int64_t>(i) * H;
       wu = wg + static_cast<int64_t>(Is) * H;
       dst = hs + qs;
+      L = limit_shared;
     }
     float g = 0.f, u = 0.f;
     for (int k = 0; k < H; ++k) {
       const float xv = __ldg(xr + k);
       g = fmaf(xv, __ldg(wg + k), g);
       u = fmaf(xv, __ldg(wu + k), u);
+    }
+    if (L > 0.0f) {
+      g = fminf(g, L);
+      u = fminf(fmaxf(u, -L), L);
     }
     *dst = g / (1.0f + expf(-g)) * u;
   }
@@ -653,8 +668,8 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
     gate_up_f32_kernel<<<static_cast<unsigned>(std::min<int64_t>((n1 + 255) / 256, 148 * 32)), 256, 0, st>>>(
         static_cast<const float*>(a.x_perm), static_cast<const float*>(a.x), a.offsets,
         static_cast<const float*>(a.Wgu), static_cast<const float*>(a.Wsgu), P,
-        has_shared ? a.T : 0, a.H, a.E, a.I, a.Is, static_cast<float*>(a.h),
-        static_cast<float*>(a.h_shared));
+        has_shared ? a.T : 0, a.H, a.E, a.I, a.Is, a.swiglu_limit, a.swiglu_limit_shared,
+        static_cast<float*>(a.h), static_cast<float*>(a.h_shared));
     count_launches(2);
     if (a.stage_mark) a.stage_mark(a.stage_mark_ctx, 3, st);
     const int64_t n2 = P * a.H + (has_shared ? a.T * a.H : 0);
@@ -686,6 +701,8 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   g.item_start = a.item_start_gu;
   g.row_w = a.row_w;
   g.row_tok = a.row_tok;
+  g.limit[0] = a.swiglu_limit;
+  g.limit[1] = a.swiglu_limit_shared;
   g.gather = gather ? 1 : 0;
   g.out[0] = static_cast<__nv_bfloat16*>(a.h);
   g.out[1] = static_cast<__nv_bfloat16*>(a.h_shared);

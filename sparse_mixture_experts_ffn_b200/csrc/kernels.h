@@ -112,6 +112,8 @@ struct ExpertArgs {
   float* partial;   // split partial sums (ksplit > 1)
   unsigned int* tile_done;  // per-tile slice counters, zero before the forward
   unsigned int* item_counters;  // [2] dynamic item claims of the two GEMMs, zero before the forward
+  float swiglu_limit;          // routed experts: gate <= L, up in [-L, L] before SiLU*up (0: none)
+  float swiglu_limit_shared;   // the same for the shared expert
   void* h;          // [T*k, I]
   void* h_shared;   // [T, Is]
   void* o;          // [T*k, H]

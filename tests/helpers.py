@@ -48,10 +48,11 @@ def oracle_routing(d: dict, top_k: int):
     return dict(scores=s, idx=idx, w=w, w64=w64, counts=counts, offsets=offsets, perm=perm, inv_perm=inv)
 
 
-def oracle_y(d: dict, routing: dict, tokens=None):
+def oracle_y(d: dict, routing: dict, tokens=None, swiglu_limit=0.0, swiglu_limit_shared=0.0):
     a = oracle_arrays({k: d.get(k) for k in ("x", "W_gate_up", "W_down", "Ws_gate_up", "Ws_down")})
     return oracle.moe_tokens(a["x"], routing["idx"], routing["w64"], a["W_gate_up"], a["W_down"],
-                             a["Ws_gate_up"], a["Ws_down"], tokens=tokens)
+                             a["Ws_gate_up"], a["Ws_down"], tokens=tokens, swiglu_limit=swiglu_limit,
+                             swiglu_limit_shared=swiglu_limit_shared)
 
 
 def assert_routing_exact(r_gpu, r_ref: dict, E: int, w_tol: float = None):

@@ -100,3 +100,20 @@ def test_status_strings(lib):
     for code, name in moe.STATUS_NAMES.items():
         assert moe.status_string(code).startswith(name)
     assert moe.status_string(99) == "unknown moe_status"
+
+
+def test_forward_ex_rejects_bad_swiglu_limits_before_any_launch(lib):
+    s = shape()
+    P = ctypes.c_void_p
+    n = moe.workspace_bytes(s)
+
+    def call(limit, limit_shared):
+        opts = moe.MoEOptions(limit, limit_shared)
+        return lib.moe_layer_forward_ex(ctypes.byref(s), P(16), P(16), None, P(16), P(16), P(16), P(16),
+                                        P(16), None, ctypes.byref(opts), P(256), n, None)
+
+    for bad in ((-1.0, 0.0), (0.0, -0.5), (float("nan"), 0.0), (0.0, float("inf"))):
+        assert call(*bad) == 1, bad
+    # NULL options is the plain forward (validation of the other arguments still runs)
+    assert lib.moe_layer_forward_ex(ctypes.byref(s), None, P(16), None, P(16), P(16), P(16), P(16),
+                                    P(16), None, None, P(256), n, None) == 1

@@ -61,6 +61,30 @@ def test_small_bf16_parity(sz):
     check_full(d, cfg.top_k, cfg.name)
 
 
+LIMIT_CASES = [
+    # 16-token tiles with the gate/up reduction split (the last slice applies the clamp)
+    dict(T=3, H=512, E=16, top_k=4, I=128, I_shared=128),
+    # 128-token gate/up tiles (staged epilogue), 128- and 256-token down tiles
+    dict(T=300, H=256, E=16, top_k=4, I=256, I_shared=128),
+    dict(T=700, H=256, E=8, top_k=4, I=256, I_shared=128),
+    dict(T=45, H=72, E=10, top_k=3, I=40, I_shared=24, dtype="f32", r_std=0.1),
+]
+
+
+@pytest.mark.parametrize("sz", LIMIT_CASES, ids=lambda s: "T{T}_H{H}_E{E}".format(**s) + s.get("dtype", ""))
+def test_swiglu_limits(sz):
+    """SwiGLU limits 0.3 (routed) and 0.2 (shared): gate <= L, up in [-L, L] before SiLU*up."""
+    cfg = inputs.small_config(**sz)
+    d = to_device(inputs.make_inputs(cfg, "cuda"))
+    y, r = run(d, cfg.top_k, swiglu_limit=0.3, swiglu_limit_shared=0.2)
+    ref = oracle_routing(d, cfg.top_k)
+    assert_routing_exact(r, ref, cfg.E)
+    y_ref = oracle_y(d, ref, swiglu_limit=0.3, swiglu_limit_shared=0.2)
+    assert_y_close(y, y_ref, "swiglu limits")
+    y_free = oracle_y(d, ref)
+    assert np.abs(y_ref - y_free).max() > 0.05 * np.abs(y_free).max()  # the clamps are active
+
+
 def test_small_bf16_with_router_bias():
     cfg = inputs.small_config(T=257, H=256, E=32, top_k=4, I=128, I_shared=128)
     d = inputs.make_inputs(cfg, "cuda")
