@@ -36,12 +36,13 @@ _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile moe_oracle.c into oracle/_build/libmoe_oracle.so with gcc -O2 -fopenmp."""
+    """Compile moe_oracle.c into oracle/_build/libmoe_oracle.so with gcc -O2 -fopenmp
+    (-ffp-contract=off: the fixed-sequence exponential fuses only where it says so)."""
     os.makedirs(_BUILD_DIR, exist_ok=True)
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
-                               "-o", tmp, _SRC, "-lm"])
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fopenmp", "-fPIC",
+                               "-shared", "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 
@@ -57,12 +58,16 @@ def _load():
         lib.oracle_route.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, P, P, P, P]
         lib.oracle_dispatch.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, P, P, P, P]
         D = ctypes.c_double
+        lib.oracle_route_mode.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int, D,
+                                          P, P, P]
+        lib.oracle_sigmoid32.argtypes = [ctypes.c_int64, P, P]
         lib.oracle_expert_act.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, D, P]
         lib.oracle_moe_tokens.argtypes = [ctypes.c_int, ctypes.c_int64, P, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P,
                                           P, D, D, P, ctypes.c_int]
         for f in (lib.oracle_exact_dot, lib.oracle_router_scores, lib.oracle_route,
-                  lib.oracle_dispatch, lib.oracle_expert_act, lib.oracle_moe_tokens):
+                  lib.oracle_dispatch, lib.oracle_expert_act, lib.oracle_moe_tokens,
+                  lib.oracle_route_mode, lib.oracle_sigmoid32):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -115,18 +120,34 @@ def router_scores(x: np.ndarray, Wr: np.ndarray, nthreads: int = 0) -> np.ndarra
     return s
 
 
-def route(scores: np.ndarray, top_k: int, bias: np.ndarray | None = None):
-    """Top-k routing of every token -> (idx int32 [T,k] ascending, w fp32 [T,k], w fp64 [T,k])."""
+ROUTERS = {"softmax": 0, "sigmoid": 1}
+
+
+def route(scores: np.ndarray, top_k: int, bias: np.ndarray | None = None, router: str = "softmax",
+          scale: float = 1.0):
+    """Top-k routing of every token -> (idx int32 [T,k] ascending, w fp32 [T,k], w fp64 [T,k]).
+
+    router="softmax": key = s (+ bias), w = softmax of the chosen keys.
+    router="sigmoid": p = sigma32(s), key = p (+ bias, selection only), w = scale * p / sum p."""
     s = _c(scores, np.float32)
     T, E = s.shape
     b = _c(bias, np.float32)
     idx = np.empty((T, top_k), np.int32)
     w = np.empty((T, top_k), np.float32)
     w64 = np.empty((T, top_k), np.float64)
-    rc = _load().oracle_route(T, E, top_k, _p(s), _p(b), _p(idx), _p(w), _p(w64))
+    rc = _load().oracle_route_mode(T, E, top_k, _p(s), _p(b), ROUTERS[router], float(scale), _p(idx),
+                                   _p(w), _p(w64))
     if rc != 0:
         raise ValueError("route: top_k must be in [1, E]")
     return idx, w, w64
+
+
+def sigmoid32(scores: np.ndarray) -> np.ndarray:
+    """fp32(1 / (1 + e^-s)) by the oracle's fixed-sequence exponential (0 below -110, 1 above 40)."""
+    s = _c(np.asarray(scores), np.float32)
+    p = np.empty_like(s)
+    _load().oracle_sigmoid32(s.size, _p(s), _p(p))
+    return p
 
 
 def dispatch(idx: np.ndarray, E: int):
@@ -182,13 +203,14 @@ def moe_tokens(x, idx, w64, Wgu, Wd, Wsgu=None, Wsd=None, tokens=None, nthreads:
 
 
 def moe_forward(x, Wr, Wgu, Wd, Wsgu=None, Wsd=None, top_k=8, bias=None, tokens=None,
-                nthreads: int = 0, swiglu_limit: float = 0.0, swiglu_limit_shared: float = 0.0):
+                nthreads: int = 0, swiglu_limit: float = 0.0, swiglu_limit_shared: float = 0.0,
+                router: str = "softmax", routed_scale: float = 1.0):
     """The whole layer: routing for every token, output for ``tokens`` (default all).
 
     Returns a dict with scores, idx, w, w64, counts, offsets, perm, inv_perm and y (fp64).
     """
     s = router_scores(x, Wr, nthreads)
-    idx, w, w64 = route(s, top_k, bias)
+    idx, w, w64 = route(s, top_k, bias, router=router, scale=routed_scale)
     counts, offsets, perm, inv = dispatch(idx, Wr.shape[0])
     y = moe_tokens(x, idx, w64, Wgu, Wd, Wsgu, Wsd, tokens=tokens, nthreads=nthreads,
                    swiglu_limit=swiglu_limit, swiglu_limit_shared=swiglu_limit_shared)

@@ -34,8 +34,12 @@
  *     gate <- min(gate, L), up <- min(max(up, -L), L), then SiLU(gate)*up; L = 0 means
  *     no clamp (the value of almost every layer).
  *
+ * The router as configured (sigmoid scores, selection-only bias, weights scaled by the
+ * routing factor) is a second routing mode, described above oracle_route_mode().
+ *
  * Parity status: every function here is pinned by tests (exact rational sums,
- * brute-force subset enumeration, closed forms and invariants); none is unpinned.
+ * brute-force subset enumeration, closed forms, high-precision decimal values and
+ * invariants); none is unpinned.
  */
 #include <math.h>
 #include <stdint.h>
@@ -238,15 +242,77 @@ static int beats(float ka, int a, float kb, int b) { /* a is ordered before b */
   return (ka > kb) || (ka == kb && a < b);
 }
 
-int oracle_route(int64_t T, int E, int k, const float* s, const float* bias, int32_t* idx_out,
-                 float* w_out, double* w64_out) {
-  if (k < 1 || k > E) return -1;
+/* ------------------------------------------------------------------------------------
+ * The router as configured on the llm-atlas page "Step-3.5-Flash", table "Champs bruts
+ * du config.json": moe_router_activation = sigmoid, use_moe_router_bias = true,
+ * moe_router_scaling_factor = 3, norm_expert_weight = true, need_fp32_gate = true.
+ * Reading (the page gives the fields only): the fp32 score of expert e is
+ *   p_e = sigma32(s_e) = fp32(1 / (1 + e^(-s_e))),
+ * the bias only steers the selection, key_e = fp32(p_e + b_e), and the weights are the
+ * chosen scores renormalised and scaled: w_j = scale * p_j / sum_{i in S} p_i (fp64).
+ *
+ * e^z is evaluated by a fixed sequence of IEEE fp64 operations, so that any IEEE
+ * implementation of the same steps (the CUDA library's own is one) returns the same
+ * bits: z = n ln2 + r with n = round(z / ln 2) and ln 2 split in two (the first part
+ * has 42 significant bits, so n * ln2_hi is exact for the |n| < 2^11 used here),
+ * |r| <= ln2/2 + tiny, then the degree-13 Taylor polynomial of e^r in Horner form with
+ * fused multiply-adds (truncation < 6e-18 relative), then an exact scaling by 2^n.
+ * The file is compiled with -ffp-contract=off: no other operation is fused.
+ * ---------------------------------------------------------------------------------- */
+static double exp_fixed(double z) {
+  const double inv_ln2 = 0x1.71547652b82fep+0; /* RN(1 / ln 2) */
+  const double ln2_hi = 0x1.62e42fefa3800p-1;  /* ln 2 = 0.693147180559945309417... cut to 42 bits */
+  const double ln2_lo = 0x1.ef35793c76730p-45; /* RN(ln 2 - ln2_hi) */
+  double n = nearbyint(z * inv_ln2);
+  double r = (z - n * ln2_hi) - n * ln2_lo;
+  double q = 1.0 / 6227020800.0; /* 1/13! */
+  q = fma(q, r, 1.0 / 479001600.0);
+  q = fma(q, r, 1.0 / 39916800.0);
+  q = fma(q, r, 1.0 / 3628800.0);
+  q = fma(q, r, 1.0 / 362880.0);
+  q = fma(q, r, 1.0 / 40320.0);
+  q = fma(q, r, 1.0 / 5040.0);
+  q = fma(q, r, 1.0 / 720.0);
+  q = fma(q, r, 1.0 / 120.0);
+  q = fma(q, r, 1.0 / 24.0);
+  q = fma(q, r, 1.0 / 6.0);
+  q = fma(q, r, 0.5);
+  q = fma(q, r, 1.0);
+  q = fma(q, r, 1.0);
+  uint64_t bits = (uint64_t)((int64_t)n + 1023) << 52; /* 2^n, a normal number here */
+  double two_n;
+  memcpy(&two_n, &bits, sizeof two_n);
+  return q * two_n;
+}
+
+/* sigma32(s): 0 below s = -110 (sigma < 2e-48 rounds to 0 in fp32), 1 above s = 40
+ * (1 - sigma < 5e-18 rounds to 1), else fp32(1 / (1 + e^(-s))). */
+static float sigmoid32(float sv) {
+  double z = (double)sv;
+  if (z < -110.0) return 0.0f;
+  if (z > 40.0) return 1.0f;
+  return (float)(1.0 / (1.0 + exp_fixed(-z)));
+}
+
+int oracle_sigmoid32(int64_t n, const float* s, float* p) {
+  for (int64_t i = 0; i < n; ++i) p[i] = sigmoid32(s[i]);
+  return 0;
+}
+
+/* mode 0: softmax router (above); mode 1: sigmoid router with selection-only bias and
+   weights scale * p / sum p. */
+int oracle_route_mode(int64_t T, int E, int k, const float* s, const float* bias, int mode,
+                      double scale, int32_t* idx_out, float* w_out, double* w64_out) {
+  if (k < 1 || k > E || (mode != 0 && mode != 1)) return -1;
 #pragma omp parallel for schedule(static)
   for (int64_t t = 0; t < T; ++t) {
     float* key = (float*)malloc(sizeof(float) * E);
+    float* prob = (float*)malloc(sizeof(float) * E);
     int* chosen = (int*)calloc(E, sizeof(int));
     for (int e = 0; e < E; ++e) {
       float v = s[t * E + e];
+      if (mode == 1) v = sigmoid32(v);
+      prob[e] = v;
       key[e] = bias ? (float)(v + bias[e]) : v; /* fp32 + fp32 -> RN fp32 */
     }
     /* k passes of "pick the best not yet chosen" */
@@ -267,16 +333,31 @@ int oracle_route(int64_t T, int E, int k, const float* s, const float* bias, int
         if ((double)key[e] > m) m = (double)key[e];
       }
     double z = 0.0;
-    for (j = 0; j < k; ++j) z += exp((double)key[idx_out[t * k + j]] - m);
-    for (j = 0; j < k; ++j) {
-      double w = exp((double)key[idx_out[t * k + j]] - m) / z;
-      if (w64_out) w64_out[t * k + j] = w;
-      if (w_out) w_out[t * k + j] = (float)w;
+    if (mode == 0) {
+      for (j = 0; j < k; ++j) z += exp((double)key[idx_out[t * k + j]] - m);
+      for (j = 0; j < k; ++j) {
+        double w = exp((double)key[idx_out[t * k + j]] - m) / z;
+        if (w64_out) w64_out[t * k + j] = w;
+        if (w_out) w_out[t * k + j] = (float)w;
+      }
+    } else {
+      for (j = 0; j < k; ++j) z += (double)prob[idx_out[t * k + j]];
+      for (j = 0; j < k; ++j) {
+        double w = z > 0.0 ? scale * (double)prob[idx_out[t * k + j]] / z : scale / k;
+        if (w64_out) w64_out[t * k + j] = w;
+        if (w_out) w_out[t * k + j] = (float)w;
+      }
     }
     free(key);
+    free(prob);
     free(chosen);
   }
   return 0;
+}
+
+int oracle_route(int64_t T, int E, int k, const float* s, const float* bias, int32_t* idx_out,
+                 float* w_out, double* w64_out) {
+  return oracle_route_mode(T, E, k, s, bias, 0, 1.0, idx_out, w_out, w64_out);
 }
 
 /* ------------------------------------------------------------------------------------

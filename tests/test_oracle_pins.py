@@ -430,3 +430,77 @@ def test_workload_table_matches_the_pages():
         assert (cfg.H, cfg.E, cfg.top_k, cfg.I, cfg.I_shared) == (
             c["hidden_size"], c["moe_num_experts"], c["moe_top_k"], c["moe_intermediate_size"],
             c["share_expert_dim"])
+
+
+# --------------------------------------------------------------------------------------
+# the router as configured: sigmoid scores, selection-only bias, renormalised and scaled
+# weights (llm-atlas page "Step-3.5-Flash", table "Champs bruts du config.json":
+# moe_router_activation, use_moe_router_bias, moe_router_scaling_factor)
+# --------------------------------------------------------------------------------------
+def _sigma32_reference(s):
+    """fp32 rounding of 1/(1+e^-s) evaluated with 40-digit decimal arithmetic."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 40
+    out = []
+    for v in np.asarray(s, np.float32).tolist():
+        out.append(float(1 / (1 + (-Decimal(v)).exp())))
+    return np.array(out, np.float64).astype(np.float32)
+
+
+def test_sigmoid32_against_high_precision_values():
+    rng = np.random.default_rng(7)
+    s = np.concatenate([rng.uniform(-110, 40, 400), rng.normal(0, 3, 400), [0.0, 1e-8, -1e-8, 17.0, -87.5]])
+    s = s.astype(np.float32)
+    p = oracle.sigmoid32(s)
+    want = _sigma32_reference(s)
+    # fp32 results equal the correctly rounded value (a near-tie could differ by one ulp)
+    ulps = np.abs(p.view(np.int32).astype(np.int64) - want.view(np.int32).astype(np.int64))
+    assert ulps.max() <= 1 and (ulps == 0).mean() >= 0.995, (ulps.max(), (ulps == 0).mean())
+
+
+def test_sigmoid32_special_values_and_monotonicity():
+    p = oracle.sigmoid32(np.array([0.0, 40.5, 1e30, -110.5, -1e30], np.float32))
+    assert p.tolist() == [0.5, 1.0, 1.0, 0.0, 0.0]
+    grid = np.sort(np.concatenate([np.linspace(-110, 40, 200001), np.linspace(-1, 1, 100001)])).astype(np.float32)
+    pg = oracle.sigmoid32(grid)
+    assert np.all(np.diff(pg.astype(np.float64)) >= 0)
+    s = np.linspace(-30, 30, 1001).astype(np.float32)
+    assert np.abs(oracle.sigmoid32(s).astype(np.float64) + oracle.sigmoid32(-s) - 1).max() < 2e-7
+
+
+@pytest.mark.parametrize("E", [5, 8])
+def test_sigmoid_router_selection_brute_force(E):
+    rng = np.random.default_rng(E)
+    for trial in range(40):
+        k = int(rng.integers(1, E + 1))
+        s = rng.normal(0, 2, (1, E)).astype(np.float32)
+        bias = rng.normal(0, 0.3, E).astype(np.float32) if trial % 2 else None
+        if trial % 5 == 0:  # saturated scores: equal p, ties toward the lower index
+            s[0, : E // 2] = 50.0
+        idx, _, _ = oracle.route(s, k, bias, router="sigmoid", scale=3.0)
+        p = oracle.sigmoid32(s[0])
+        key = p + (bias if bias is not None else np.float32(0))
+        key = key.astype(np.float32)
+        valid = []
+        for S in itertools.combinations(range(E), k):
+            rest = [f for f in range(E) if f not in S]
+            if all((key[e] > key[f]) or (key[e] == key[f] and e < f) for e in S for f in rest):
+                valid.append(S)
+        assert len(valid) == 1 and tuple(idx[0]) == valid[0]
+
+
+def test_sigmoid_router_weights_use_scores_not_keys():
+    """w_j = 3 p_j / sum_S p with p = sigma32(s); the bias steers the choice only."""
+    E, k = 8, 3
+    s = np.array([[-6.0, 2.0, 1.0, 0.5, 0.0, -1.0, 3.0, -2.0]], np.float32)
+    bias = np.zeros(E, np.float32)
+    bias[0] = 100.0  # expert 0 (a tiny score) is always chosen
+    idx, w, w64 = oracle.route(s, k, bias, router="sigmoid", scale=3.0)
+    p = oracle.sigmoid32(s[0]).astype(np.float64)
+    assert idx[0].tolist() == [0, 1, 6]
+    want = 3.0 * p[[0, 1, 6]] / p[[0, 1, 6]].sum()
+    assert np.allclose(w64[0], want, rtol=1e-15, atol=0)
+    assert abs(w64[0].sum() - 3.0) < 1e-14 and w64[0][0] < 0.01
+    # without the bias the same scores pick the three best p
+    idx2, _, w2 = oracle.route(s, k, None, router="sigmoid", scale=3.0)
+    assert idx2[0].tolist() == [1, 2, 6] and abs(w2[0].sum() - 3.0) < 1e-14
