@@ -188,15 +188,26 @@ def host_arrays(d):
     return {k: cv(v) for k, v in d.items()}
 
 
-def oracle_step(h, cfg, tokens):
+LAYER_DEFAULTS = dict(router="softmax", routed_scaling_factor=1.0, swiglu_limit=0.0, swiglu_limit_shared=0.0)
+
+
+def layer_options(args) -> dict:
+    """Per-layer options of the run (router mode and scale, SwiGLU limits)."""
+    return dict(router=args.router, routed_scaling_factor=args.routed_scale,
+                swiglu_limit=args.swiglu_limit, swiglu_limit_shared=args.swiglu_limit_shared)
+
+
+def oracle_step(h, cfg, tokens, opts=None):
     """The whole hot path for the listed tokens: exact router over all experts, top-k and
     weights, then the expert FFNs and the combine."""
     import oracle
+    o = dict(LAYER_DEFAULTS, **(opts or {}))
     x = h["x"][tokens]
     s = oracle.router_scores(x, h["W_router"])
     bias = None if h.get("bias") is None else h["bias"].astype(np.float32)
-    idx, w, w64 = oracle.route(s, cfg.top_k, bias)
-    return oracle.moe_tokens(x, idx, w64, h["W_gate_up"], h["W_down"], h["Ws_gate_up"], h["Ws_down"])
+    idx, w, w64 = oracle.route(s, cfg.top_k, bias, router=o["router"], scale=o["routed_scaling_factor"])
+    return oracle.moe_tokens(x, idx, w64, h["W_gate_up"], h["W_down"], h["Ws_gate_up"], h["Ws_down"],
+                             swiglu_limit=o["swiglu_limit"], swiglu_limit_shared=o["swiglu_limit_shared"])
 
 
 def run_reference(args, cfg):
@@ -215,10 +226,10 @@ def run_reference(args, cfg):
     cores = len(os.sched_getaffinity(0))
     per_step = 1  # tokens per step: one token's full pass through the layer
     for i in range(args.warmup):
-        oracle_step(h, cfg, [i % cfg.T])
+        oracle_step(h, cfg, [i % cfg.T], layer_options(args))
     t0 = time.perf_counter()
     for i in range(args.steps):
-        oracle_step(h, cfg, [i % cfg.T])
+        oracle_step(h, cfg, [i % cfg.T], layer_options(args))
     dt = time.perf_counter() - t0
     value = per_step * args.steps / dt
     sample = f"{per_step} token of {cfg.name} per step (exact router over {cfg.E} experts, top-{cfg.top_k}, {cfg.top_k} routed + 1 shared expert FFNs)"
@@ -226,20 +237,22 @@ def run_reference(args, cfg):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
             "data": "synthetic", "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E,
-                                             "top_k": cfg.top_k, "I": cfg.I, "I_shared": cfg.I_shared},
+                                             "top_k": cfg.top_k, "I": cfg.I, "I_shared": cfg.I_shared,
+                                             **({"layer_options": layer_options(args)}
+                                                if layer_options(args) != LAYER_DEFAULTS else {})},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
-def cpu_baseline(h, cfg, budget_s=10.0):
+def cpu_baseline(h, cfg, opts=None, budget_s=10.0):
     import oracle
     cores = len(os.sched_getaffinity(0))
     tokens = list(range(min(cfg.T, 8)))
     n, t0 = 0, time.perf_counter()
     while True:
-        oracle_step(h, cfg, tokens)
+        oracle_step(h, cfg, tokens, opts)
         n += 1
         if time.perf_counter() - t0 >= budget_s:
             break
@@ -262,6 +275,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--T", type=int, default=None, help="profiling variant: override the token count")
     ap.add_argument("--E", type=int, default=None, help="profiling variant: override the expert count")
+    ap.add_argument("--router", default="softmax", choices=["softmax", "sigmoid"],
+                    help="router mode (sigmoid: the router as configured, bias for the selection only)")
+    ap.add_argument("--routed-scale", type=float, default=1.0, help="sigmoid router: routed scaling factor")
+    ap.add_argument("--swiglu-limit", type=float, default=0.0, help="SwiGLU limit of the routed experts")
+    ap.add_argument("--swiglu-limit-shared", type=float, default=0.0, help="SwiGLU limit of the shared expert")
     ap.add_argument("--I", type=int, default=None,
                     help="profiling variant: override both expert widths (small weights, same router)")
     args = ap.parse_args()
@@ -310,7 +328,8 @@ def main():
 
     def step(xin, yout, routing=False):
         return moe.moe_layer_forward(xin, Wr, Wgu, Wd, Wsgu, Wsd, top_k=cfg.top_k, router_bias=bias,
-                                     y=yout, workspace=ws, routing=routing, stream=stream)
+                                     y=yout, workspace=ws, routing=routing, stream=stream,
+                                     **layer_options(args))
 
     _, r = step(x, y, routing=True)
     torch.cuda.synchronize()
@@ -412,6 +431,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
             "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "top_k": cfg.top_k,
                        "I": cfg.I, "I_shared": cfg.I_shared, "tokens_per_gpu": cfg.T,
+                       **({"layer_options": layer_options(args)} if layer_options(args) != LAYER_DEFAULTS else {}),
                        "l2": "flushed before every timed step (2x L2 write, outside the events)",
                        "parallelism": f"replicas x{world}"},
             "roofline": roof,
@@ -432,7 +452,7 @@ def main():
             oracle.build()
             h = host_arrays(dict(x=x, W_router=Wr, bias=bias, W_gate_up=Wgu, W_down=Wd, Ws_gate_up=Wsgu,
                                  Ws_down=Wsd))
-            line["cpu_baseline"] = cpu_baseline(h, cfg)
+            line["cpu_baseline"] = cpu_baseline(h, cfg, layer_options(args))
         print(json.dumps(line), flush=True)
     if pg:
         pg.barrier()

@@ -110,20 +110,32 @@ MOE_API moe_status moe_layer_forward(const moe_layer_shape* shape, const void* x
                              moe_routing_out* routing, void* workspace, size_t workspace_bytes,
                              void* stream);
 
-/* Per-layer options of moe_layer_forward_ex().
+/* Per-layer options of moe_layer_forward_ex().  All zero = moe_layer_forward().
  *   swiglu_limit, swiglu_limit_shared: the SwiGLU limits of the routed experts and of the
  *   shared expert (llm-atlas page "Step-3.5-Flash", table "Champs bruts du config.json":
  *   swiglu_limits "0.0x46 + 7x2", swiglu_limits_shared "0.0x47 + 16x1"; the page gives
  *   the values only).  A limit L > 0 clamps the activation inputs, gate to <= L and up to
- *   [-L, L], before SiLU(gate)*up; 0 means no clamp.  Limits must be finite and >= 0. */
+ *   [-L, L], before SiLU(gate)*up; 0 means no clamp.  Limits must be finite and >= 0.
+ *   router: MOE_ROUTER_SOFTMAX (0) or MOE_ROUTER_SIGMOID (1), the router as configured on
+ *   the same table (moe_router_activation = sigmoid, use_moe_router_bias,
+ *   moe_router_scaling_factor = 3): p_e = fp32(1 / (1 + e^-s_e)) of the fp32 logit s_e,
+ *   with e^z evaluated by a fixed sequence of fp64 operations (Cody-Waite reduction by a
+ *   42-bit ln 2 head and its tail, the degree-13 Taylor polynomial in fused
+ *   multiply-adds, scaling by 2^n; p = 0 below s = -110 and 1 above 40); the router bias
+ *   only steers the selection (key_e = fp32(p_e + b_e)); the weights are
+ *   routed_scaling_factor * p_j / sum of the chosen p (uniform if that sum is 0).
+ *   routed_scaling_factor: sigmoid router only; 0 is read as 1; else finite and > 0. */
+enum { MOE_ROUTER_SOFTMAX = 0, MOE_ROUTER_SIGMOID = 1 };
 typedef struct {
   float swiglu_limit;
   float swiglu_limit_shared;
+  int32_t router;
+  float routed_scaling_factor;
 } moe_layer_options;
 
 /* moe_layer_forward() with per-layer options; options = NULL is moe_layer_forward().
  * Errors as moe_layer_forward(), plus MOE_ERR_INVALID_ARG for a negative or non-finite
- * limit. */
+ * limit, an unknown router or a negative or non-finite scaling factor. */
 MOE_API moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const void* x,
                                         const void* W_router, const float* router_bias,
                                         const void* W_gate_up, const void* W_down,
@@ -198,8 +210,8 @@ MOE_API int64_t moe_layer_launch_count(void);
  * of the shape are not used.
  *
  * Scratch: a 16 MiB device array inside this library (present on every GPU that loads the
- * library, until the process exits).  The call needs about T * (24 * E + 8) bytes of it
- * (plus E / 2 per token for fp32 inputs), so batches of up to about 2400 tokens fit at
+ * library, until the process exits).  The call needs about T * (28 * E + 8) bytes of it
+ * (plus E / 2 per token for fp32 inputs), so batches of up to about 2000 tokens fit at
  * E = 288.  Larger batches return MOE_ERR_WORKSPACE_TOO_SMALL before anything is enqueued.
  * The array is shared by all calls: calls that may overlap on the GPU (several streams or
  * host threads) race and must be serialised by the caller.  Each call clears the part

@@ -37,7 +37,11 @@ class MoEShape(ctypes.Structure):
 
 
 class MoEOptions(ctypes.Structure):
-    _fields_ = [("swiglu_limit", ctypes.c_float), ("swiglu_limit_shared", ctypes.c_float)]
+    _fields_ = [("swiglu_limit", ctypes.c_float), ("swiglu_limit_shared", ctypes.c_float),
+                ("router", ctypes.c_int32), ("routed_scaling_factor", ctypes.c_float)]
+
+
+ROUTERS = {"softmax": 0, "sigmoid": 1}
 
 
 class MoERoutingOut(ctypes.Structure):
@@ -145,13 +149,16 @@ def alloc_workspace(shape: MoEShape, device):
 
 def moe_layer_forward(x, W_router, W_gate_up, W_down, Ws_gate_up=None, Ws_down=None, *, top_k,
                       router_bias=None, y=None, workspace=None, routing=True, stream=None,
-                      swiglu_limit=0.0, swiglu_limit_shared=0.0):
+                      swiglu_limit=0.0, swiglu_limit_shared=0.0, router="softmax",
+                      routed_scaling_factor=1.0):
     """Run the MoE layer on the device.  Returns (y, Routing or None).
 
     Shapes: x [T,H], W_router [E,H], W_gate_up [E,2I,H], W_down [E,H,I], Ws_gate_up
     [2Is,H], Ws_down [H,Is] (or both None), router_bias [E] fp32 or None.  All CUDA,
     contiguous, same dtype (bf16 or fp32).  swiglu_limit / swiglu_limit_shared: SwiGLU
     limits of the routed / shared experts (gate <= L, up in [-L, L]; 0 = none).
+    router="sigmoid": sigmoid scores, router_bias for the selection only, weights
+    routed_scaling_factor * p / sum p (the default "softmax" ignores the factor).
     """
     import torch
     lib = load_library()
@@ -181,7 +188,8 @@ def moe_layer_forward(x, W_router, W_gate_up, W_down, Ws_gate_up=None, Ws_down=N
                              r.offsets.data_ptr(), r.perm.data_ptr())
     if stream is None:
         stream = torch.cuda.current_stream(x.device)
-    opts = MoEOptions(float(swiglu_limit), float(swiglu_limit_shared))
+    opts = MoEOptions(float(swiglu_limit), float(swiglu_limit_shared), ROUTERS[router],
+                      float(routed_scaling_factor))
     rc = lib.moe_layer_forward_ex(ctypes.byref(shape), _ptr(x), _ptr(W_router), _ptr(router_bias),
                                   _ptr(W_gate_up), _ptr(W_down), _ptr(Ws_gate_up), _ptr(Ws_down),
                                   _ptr(y), ctypes.byref(rout) if rout is not None else None,

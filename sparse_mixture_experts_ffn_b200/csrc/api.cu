@@ -130,7 +130,7 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.wss = take(tc_scores ? 0 : groups * E * 8);
   L.scores = take(T * E * 8);
   L.zero_end = tc_scores ? L.scores : off;
-  L.spill = take(T * E * 16);
+  L.spill = take(T * E * 20);
   L.rsplit = take(router_split_bytes(*s));
   L.xnorm = take(T * 8);
   L.wnorm = take(E * 8);
@@ -221,10 +221,12 @@ extern "C" moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const v
                                            const void* Ws_gate_up, const void* Ws_down, void* y,
                                            moe_routing_out* routing, const moe_layer_options* options,
                                            void* workspace, size_t workspace_bytes, void* stream) {
-  const moe_layer_options opt = options ? *options : moe_layer_options{0.0f, 0.0f};
+  const moe_layer_options opt = options ? *options : moe_layer_options{0.0f, 0.0f, MOE_ROUTER_SOFTMAX, 0.0f};
   if (!(opt.swiglu_limit >= 0.0f && opt.swiglu_limit <= FLT_MAX) ||
-      !(opt.swiglu_limit_shared >= 0.0f && opt.swiglu_limit_shared <= FLT_MAX))
+      !(opt.swiglu_limit_shared >= 0.0f && opt.swiglu_limit_shared <= FLT_MAX) ||
+      !(opt.routed_scaling_factor >= 0.0f && opt.routed_scaling_factor <= FLT_MAX))
     return MOE_ERR_INVALID_ARG;  // negative, infinite or NaN
+  if (opt.router != MOE_ROUTER_SOFTMAX && opt.router != MOE_ROUTER_SIGMOID) return MOE_ERR_INVALID_ARG;
   const moe_status vs = validate_shape(shape);
   if (vs != MOE_OK) return vs;
   const moe_layer_shape& s = *shape;
@@ -271,6 +273,8 @@ extern "C" moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const v
   ra.scores64 = static_cast<double*>(at(L.scores));
   ra.wss = static_cast<double*>(at(L.wss));
   ra.spill = static_cast<float*>(at(L.spill));
+  ra.sigmoid = opt.router == MOE_ROUTER_SIGMOID ? 1 : 0;
+  ra.scale = opt.routed_scaling_factor > 0.0f ? opt.routed_scaling_factor : 1.0f;
   ra.rsplit = router_split_bytes(*shape) ? at(L.rsplit) : nullptr;
   ra.xnorm = static_cast<double*>(at(L.xnorm));
   ra.wnorm = static_cast<double*>(at(L.wnorm));

@@ -38,6 +38,8 @@ struct RouterArgs {
   const void* x;
   const void* Wr;
   const float* bias;
+  int sigmoid;       // 0: softmax router; 1: sigmoid router (bias for the selection only)
+  float scale;       // sigmoid router: routed scaling factor of the weights
   double* scores64;  // [T, E], zero before the forward on the small-batch path
   double* wss;       // [router_group_counters(T), E] zero before the forward
   double* xnorm;     // [T]
@@ -47,7 +49,7 @@ struct RouterArgs {
   float* w_ws;       // [T, k]
   int32_t* idx_user;
   float* w_user;
-  float* spill;      // [4, T, E] key state of tokens that need exact dots
+  float* spill;      // [5, T, E] key state of tokens that need exact dots
   void* rsplit;      // router_split_bytes(shape) bytes, or null: the reduction is not split
   Ctrl* ctrl;
 };

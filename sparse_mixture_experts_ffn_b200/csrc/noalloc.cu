@@ -90,7 +90,7 @@ extern "C" moe_status moe_layer_route_noalloc(const moe_layer_shape* shape, cons
   const size_t zero_end = tc ? o_scores : off;
   const size_t o_xnorm = take(T * 8);
   const size_t o_wnorm = take(E * 8);
-  const size_t o_spill = take(T * E * 16);
+  const size_t o_spill = take(T * E * 20);
   if (off > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE_TOO_SMALL;
 
   void* base = nullptr;
@@ -119,6 +119,8 @@ extern "C" moe_status moe_layer_route_noalloc(const moe_layer_shape* shape, cons
   ra.w_user = nullptr;
   ra.spill = reinterpret_cast<float*>(ws + o_spill);
   ra.rsplit = nullptr;  // the scratch holds no reduction-split partials
+  ra.sigmoid = 0;       // the softmax router
+  ra.scale = 1.0f;
   ra.ctrl = reinterpret_cast<Ctrl*>(ws + o_ctrl);
   return launch_router(ra, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

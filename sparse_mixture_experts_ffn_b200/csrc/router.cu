@@ -236,10 +236,77 @@ __device__ __forceinline__ uint32_t ordered(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-__device__ __forceinline__ float key_of(double s, const float* bias, int e) {
-  const float s32 = __double2float_rn(s);
-  return bias ? __fadd_rn(s32, bias[e]) : s32;
+// e^z for the sigmoid router, z in [-41, 111]: the fixed sequence of IEEE fp64 steps that
+// defines the router's sigmoid (Cody-Waite reduction z = n ln2 + r with ln 2 split into a
+// 42-bit head, so that n * ln2_hi is exact, and a tail; the degree-13 Taylor polynomial of
+// e^r by fused multiply-adds; an exact scaling by 2^n).  Every operation is an explicit
+// round-to-nearest intrinsic, so nothing is contracted or approximated and the result is
+// the same on any IEEE implementation of these steps.
+__device__ __forceinline__ double exp_fixed(double z) {
+  const double inv_ln2 = 0x1.71547652b82fep+0;  // RN(1 / ln 2)
+  const double ln2_hi = 0x1.62e42fefa3800p-1;   // ln 2 = 0.693147180559945309417..., 42 bits
+  const double ln2_lo = 0x1.ef35793c76730p-45;  // RN(ln 2 - ln2_hi)
+  const double n = rint(__dmul_rn(z, inv_ln2));
+  const double r = __dsub_rn(__dsub_rn(z, __dmul_rn(n, ln2_hi)), __dmul_rn(n, ln2_lo));
+  double q = 1.0 / 6227020800.0;  // 1/13!
+  q = __fma_rn(q, r, 1.0 / 479001600.0);
+  q = __fma_rn(q, r, 1.0 / 39916800.0);
+  q = __fma_rn(q, r, 1.0 / 3628800.0);
+  q = __fma_rn(q, r, 1.0 / 362880.0);
+  q = __fma_rn(q, r, 1.0 / 40320.0);
+  q = __fma_rn(q, r, 1.0 / 5040.0);
+  q = __fma_rn(q, r, 1.0 / 720.0);
+  q = __fma_rn(q, r, 1.0 / 120.0);
+  q = __fma_rn(q, r, 1.0 / 24.0);
+  q = __fma_rn(q, r, 1.0 / 6.0);
+  q = __fma_rn(q, r, 0.5);
+  q = __fma_rn(q, r, 1.0);
+  q = __fma_rn(q, r, 1.0);
+  const double two_n = __longlong_as_double((static_cast<long long>(n) + 1023) << 52);
+  return __dmul_rn(q, two_n);
 }
+
+// The router's fp32 sigmoid score of an fp32 logit: 0 below -110, 1 above 40, else
+// fp32(1 / (1 + e^-s)).  Not monotone by construction, but within one ulp of it (the fp64
+// value is within a few ulps of the true sigmoid), which the interval ends allow for.
+__device__ __forceinline__ float sigmoid32(float s32) {
+  const double z = static_cast<double>(s32);
+  if (z < -110.0) return 0.0f;
+  if (z > 40.0) return 1.0f;
+  return __double2float_rn(__ddiv_rn(1.0, __dadd_rn(1.0, exp_fixed(-z))));
+}
+
+// How router logits become selection keys and weights.
+//   softmax (sigmoid = 0): key = fp32(s) (+ bias), weights = softmax of the chosen keys;
+//   sigmoid (sigmoid = 1): p = sigmoid32(fp32(s)), key = fp32(p + bias) with the bias
+//     steering the choice only, weights = scale * p / sum of the chosen p
+//     (llm-atlas page "Step-3.5-Flash", table "Champs bruts du config.json":
+//     moe_router_activation, use_moe_router_bias, moe_router_scaling_factor).
+struct Keys {
+  const float* bias;
+  int sigmoid;
+  float scale;
+  __device__ __forceinline__ float score(double s) const {  // p, or the logit itself
+    const float s32 = __double2float_rn(s);
+    return sigmoid ? sigmoid32(s32) : s32;
+  }
+  // the key of a logit (exact when s is the exact logit rounded to fp32)
+  __device__ __forceinline__ float key(double s, int e) const {
+    const float v = score(s);
+    return bias ? __fadd_rn(v, bias[e]) : v;
+  }
+  // lower / upper ends of the keys of all logits >= s_lo / <= s_hi
+  __device__ __forceinline__ float key_lo(double s_lo, int e) const {
+    if (!sigmoid) return key(s_lo, e);
+    const float p = nextafterf(score(s_lo), -INFINITY);
+    return bias ? __fadd_rd(p, bias[e]) : p;
+  }
+  __device__ __forceinline__ float key_hi(double s_hi, int e) const {
+    if (!sigmoid) return key(s_hi, e);
+    const float p = nextafterf(score(s_hi), INFINITY);
+    return bias ? __fadd_ru(p, bias[e]) : p;
+  }
+};
 
 // a is ranked before b: larger key, then lower index
 __device__ __forceinline__ bool better(float ka, int a, float kb, int b) {
@@ -325,18 +392,22 @@ __device__ double warp_dot_f64_prefetch(const T* __restrict__ a, const T* __rest
 struct CandList {
   int e[32];
   float lo[32], hi[32], mid[32];
+  float p[32];  // sigmoid router: the score of the best estimate (weights)
 };
 
-template <typename T, int EPL>
+// SIG: the router mode as a compile-time constant (the softmax path carries no sigmoid code)
+template <typename T, int EPL, bool SIG>
 __device__ __forceinline__ bool select_token(const double* __restrict__ srow, double delta_coef,
                                              double delta_abs, bool refine_f64, double nx,
                                              const double* __restrict__ wnorm,
                                              const double* __restrict__ wss,
-                                             const float* __restrict__ bias, const T* __restrict__ xt,
+                                             const Keys kf_in, const T* __restrict__ xt,
                                              const T* __restrict__ Wr, int H, int E, int k, int64_t t,
                                              int32_t* __restrict__ idx_ws, float* __restrict__ w_ws,
                                              int32_t* __restrict__ idx_user, float* __restrict__ w_user,
                                              CandList& C, Ctrl* ctrl) {
+  Keys kf = kf_in;
+  kf.sigmoid = SIG ? 1 : 0;
   const int lane = threadIdx.x & 31;
   auto nw = [&](int e) -> double { return wss ? norm_ub_from_sumsq(wss[e], H) : wnorm[e]; };
   const double cdx = __dmul_ru(delta_coef, nx);
@@ -348,7 +419,7 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
     u[i] = 0;
     if (e < E) {
       const double d = __dadd_ru(__dmul_ru(cdx, nw(e)), delta_abs);
-      u[i] = ordered(key_of(__dadd_rd(srow[e], -d), bias, e));
+      u[i] = ordered(kf.key_lo(__dadd_rd(srow[e], -d), e));
     }
   }
   // 2. Lk
@@ -379,16 +450,17 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
-    float lo = 0.f, hi = 0.f, mid = 0.f;
+    float lo = 0.f, hi = 0.f, mid = 0.f, pv = 0.f;
     bool cand = false;
     if (e < E) {
       const double sh = srow[e];
       const double d = __dadd_ru(__dmul_ru(cdx, nw(e)), delta_abs);
-      hi = key_of(__dadd_ru(sh, d), bias, e);
+      hi = kf.key_hi(__dadd_ru(sh, d), e);
       cand = ordered(hi) >= lk;
       if (cand) {
-        lo = key_of(__dadd_rd(sh, -d), bias, e);
-        mid = key_of(sh, bias, e);
+        lo = kf.key_lo(__dadd_rd(sh, -d), e);
+        mid = kf.key(sh, e);
+        if (SIG) pv = kf.score(sh);
       }
     }
     const unsigned m = __ballot_sync(0xffffffffu, cand);
@@ -398,6 +470,7 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
       C.lo[pos] = lo;
       C.hi[pos] = hi;
       C.mid[pos] = mid;
+      if (SIG) C.p[pos] = pv;
     }
     cn += __popc(m);
   }
@@ -407,6 +480,7 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
   const bool mine = lane < cn;
   const int my_e = mine ? C.e[lane] : 0;
   float my_lo = mine ? C.lo[lane] : 0.f, my_hi = mine ? C.hi[lane] : 0.f, my_mid = mine ? C.mid[lane] : 0.f;
+  float my_p = (SIG && mine) ? C.p[lane] : 0.f;
   auto classify_mine = [&]() -> int {
     int cp = 0, cc = 0;
     for (int j = 0; j < cn; ++j) {
@@ -431,9 +505,10 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
         const double s64 = warp_dot_f64_prefetch(xt, Wr + static_cast<size_t>(e) * H, H);
         if (lane == src) {
           const double d = __dmul_ru(__dmul_ru(1.01 * H * kU53, nx), nw(e));
-          my_lo = key_of(__dadd_rd(s64, -d), bias, e);
-          my_hi = key_of(__dadd_ru(s64, d), bias, e);
-          my_mid = key_of(s64, bias, e);
+          my_lo = kf.key_lo(__dadd_rd(s64, -d), e);
+          my_hi = kf.key_hi(__dadd_ru(s64, d), e);
+          my_mid = kf.key(s64, e);
+          if (SIG) my_p = kf.score(s64);
           C.lo[lane] = my_lo;
           C.hi[lane] = my_hi;
           C.mid[lane] = my_mid;
@@ -468,12 +543,13 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
     }
     if (mine && my_e == be) st = ST_IN;
   }
-  // 7. renormalised softmax over the chosen keys; outputs in ascending expert order
+  // 7. weights: renormalised softmax over the chosen keys, or (sigmoid router) the chosen
+  //    scores renormalised and scaled; outputs in ascending expert order
   const bool in = st == ST_IN;
   float m = in ? my_mid : -FLT_MAX;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  const float ex = in ? expf(my_mid - m) : 0.0f;
+  const float ex = in ? (kf.sigmoid ? my_p : expf(my_mid - m)) : 0.0f;
   float z = ex;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
@@ -481,7 +557,7 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
   if (in) {
     const int pos = __popc(in_mask & ((1u << lane) - 1u));
     if (pos < k) {
-      const float w = ex / z;
+      const float w = !kf.sigmoid ? ex / z : (z > 0.0f ? kf.scale * ex / z : kf.scale / k);
       idx_ws[t * k + pos] = my_e;
       w_ws[t * k + pos] = w;
       if (idx_user) idx_user[t * k + pos] = my_e;
@@ -504,6 +580,7 @@ struct KeySpill {
   float* hi;
   float* mid;
   int* st;
+  float* p;  // sigmoid router: scores of the best estimates
 };
 
 __device__ __forceinline__ KeySpill key_spill(float* base, int64_t T, int E, int64_t t) {
@@ -513,6 +590,7 @@ __device__ __forceinline__ KeySpill key_spill(float* base, int64_t T, int E, int
   s.hi = base + n + t * E;
   s.mid = base + 2 * n + t * E;
   s.st = reinterpret_cast<int*>(base + 3 * n) + t * E;
+  s.p = base + 4 * n + t * E;
   return s;
 }
 
@@ -520,18 +598,20 @@ __device__ __forceinline__ KeySpill key_spill(float* base, int64_t T, int E, int
 // warp): intervals from the score estimates, fp64 recompute (when the estimates are not
 // fp64 sums) and exact dots for what stays undecided, classification, open slots,
 // weights and outputs.
-template <typename T>
+template <typename T, bool SIG>
 __device__ __noinline__ void select_token_slow(const double* __restrict__ srow, int64_t sstride,
                                                double delta_coef,
                                                double delta_abs, bool refine_f64, double nx,
                                                const double* __restrict__ wnorm,
                                                const double* __restrict__ wss, KeySpill sp,
-                                               const float* __restrict__ bias,
+                                               const Keys kf_in,
                                                const T* __restrict__ xt, const T* __restrict__ Wr,
                                                int H, int E, int k, int64_t t,
                                                int32_t* __restrict__ idx_ws, float* __restrict__ w_ws,
                                                int32_t* __restrict__ idx_user, float* __restrict__ w_user,
                                                unsigned char* exact_scratch, Ctrl* ctrl) {
+  Keys kf = kf_in;
+  kf.sigmoid = SIG ? 1 : 0;
   const int lane = threadIdx.x & 31;
   auto nw = [&](int e) -> double { return wss ? norm_ub_from_sumsq(wss[e], H) : wnorm[e]; };
   long long* bins = reinterpret_cast<long long*>(exact_scratch);
@@ -539,9 +619,10 @@ __device__ __noinline__ void select_token_slow(const double* __restrict__ srow, 
   for (int e = lane; e < E; e += 32) {
     const double sh = srow[e * sstride];
     const double d = __dadd_ru(__dmul_ru(__dmul_ru(delta_coef, nx), nw(e)), delta_abs);
-    sp.lo[e] = key_of(__dadd_rd(sh, -d), bias, e);
-    sp.hi[e] = key_of(__dadd_ru(sh, d), bias, e);
-    sp.mid[e] = key_of(sh, bias, e);
+    sp.lo[e] = kf.key_lo(__dadd_rd(sh, -d), e);
+    sp.hi[e] = kf.key_hi(__dadd_ru(sh, d), e);
+    sp.mid[e] = kf.key(sh, e);
+    sp.p[e] = kf.score(sh);
     sp.st[e] = ST_CAND;
   }
   __syncwarp();
@@ -581,17 +662,19 @@ __device__ __noinline__ void select_token_slow(const double* __restrict__ srow, 
         const int e = base + __ffs(mask) - 1;
         mask &= mask - 1;
         const T* we = Wr + static_cast<size_t>(e) * H;
-        float klo, khi, kmid;
+        float klo, khi, kmid, kp;
         if (pass == 0) {
           const double s64 = warp_dot_f64_prefetch(xt, we, H);
           const double d = __dmul_ru(__dmul_ru(1.01 * H * kU53, nx), nw(e));
-          klo = key_of(__dadd_rd(s64, -d), bias, e);
-          khi = key_of(__dadd_ru(s64, d), bias, e);
-          kmid = key_of(s64, bias, e);
+          klo = kf.key_lo(__dadd_rd(s64, -d), e);
+          khi = kf.key_hi(__dadd_ru(s64, d), e);
+          kmid = kf.key(s64, e);
+          kp = kf.score(s64);
           ++n_ref;
         } else {
           const float s32 = warp_exact_dot_rn32(xt, we, H, bins, limbs);
-          klo = khi = kmid = bias ? __fadd_rn(s32, bias[e]) : s32;
+          klo = khi = kmid = kf.key(s32, e);
+          kp = kf.score(s32);
           ++n_exact;
         }
         __syncwarp();
@@ -599,6 +682,7 @@ __device__ __noinline__ void select_token_slow(const double* __restrict__ srow, 
           sp.lo[e] = klo;
           sp.hi[e] = khi;
           sp.mid[e] = kmid;
+          sp.p[e] = kp;
         }
         __syncwarp();
       }
@@ -640,7 +724,7 @@ __device__ __noinline__ void select_token_slow(const double* __restrict__ srow, 
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float z = 0.0f;
   for (int e = lane; e < E; e += 32)
-    if (sp.st[e] == ST_IN) z += expf(sp.mid[e] - m);
+    if (sp.st[e] == ST_IN) z += kf.sigmoid ? sp.p[e] : expf(sp.mid[e] - m);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
   int written = 0;
@@ -651,7 +735,8 @@ __device__ __noinline__ void select_token_slow(const double* __restrict__ srow, 
     if (ch) {
       const int pos = written + __popc(mask & ((1u << lane) - 1u));
       if (pos < k) {
-        const float w = expf(sp.mid[e] - m) / z;
+        const float w = !kf.sigmoid ? expf(sp.mid[e] - m) / z
+                                    : (z > 0.0f ? kf.scale * sp.p[e] / z : kf.scale / k);
         idx_ws[t * k + pos] = e;
         w_ws[t * k + pos] = w;
         if (idx_user) idx_user[t * k + pos] = e;
@@ -673,11 +758,11 @@ __device__ __noinline__ void select_token_slow(const double* __restrict__ srow, 
 // ---------------------------------------------------------------------------------------
 constexpr int kSelectWarps = 4;
 
-template <typename T, int EPL>
+template <typename T, int EPL, bool SIG>
 __global__ void __launch_bounds__(32 * kSelectWarps) route_select_kernel(
     const double* __restrict__ scores, double delta_coef, double delta_abs,
     const double* __restrict__ xnorm, const double* __restrict__ wnorm,
-    const float* __restrict__ bias, const T* __restrict__ x, const T* __restrict__ Wr,
+    const Keys kf, const T* __restrict__ x, const T* __restrict__ Wr,
     int64_t T_, int H, int E, int k, int32_t* __restrict__ idx_ws, float* __restrict__ w_ws,
     int32_t* __restrict__ idx_user, float* __restrict__ w_user, float* __restrict__ spill,
     Ctrl* ctrl) {
@@ -687,11 +772,11 @@ __global__ void __launch_bounds__(32 * kSelectWarps) route_select_kernel(
   const int warp = threadIdx.x >> 5;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kSelectWarps + warp;
   if (t < T_) {
-    if (!select_token<T, EPL>(scores + t * E, delta_coef, delta_abs, true, xnorm[t], wnorm, nullptr,
-                              bias, x + t * H, Wr, H, E, k, t, idx_ws, w_ws, idx_user, w_user,
+    if (!select_token<T, EPL, SIG>(scores + t * E, delta_coef, delta_abs, true, xnorm[t], wnorm, nullptr,
+                              kf, x + t * H, Wr, H, E, k, t, idx_ws, w_ws, idx_user, w_user,
                               cands[warp], ctrl))
-      select_token_slow<T>(scores + t * E, 1, delta_coef, delta_abs, true, xnorm[t], wnorm, nullptr,
-                           key_spill(spill, T_, E, t), bias, x + t * H, Wr, H, E, k, t, idx_ws, w_ws,
+      select_token_slow<T, SIG>(scores + t * E, 1, delta_coef, delta_abs, true, xnorm[t], wnorm, nullptr,
+                           key_spill(spill, T_, E, t), kf, x + t * H, Wr, H, E, k, t, idx_ws, w_ws,
                            idx_user, w_user, exact_scratch[warp], ctrl);
   }
 }
@@ -710,9 +795,9 @@ constexpr int kDecodeExp = 16;
 constexpr int kDecodeSplit = 4;
 constexpr int kDecodeThreads = 256;
 
-template <typename T, int EPL>
+template <typename T, int EPL, bool SIG>
 __global__ void __launch_bounds__(kDecodeThreads, 1) router_decode_kernel(
-    const T* __restrict__ x, const T* __restrict__ Wr, const float* __restrict__ bias, int64_t T_,
+    const T* __restrict__ x, const T* __restrict__ Wr, const Keys kf, int64_t T_,
     int H, int E, int k, double* __restrict__ scores, double* __restrict__ wss,
     unsigned int* __restrict__ group_done, int32_t* __restrict__ idx_ws, float* __restrict__ w_ws,
     int32_t* __restrict__ idx_user, float* __restrict__ w_user, float* __restrict__ spill, Ctrl* ctrl) {
@@ -811,10 +896,10 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) router_decode_kernel(
       const T* xt = x + t * H;
       const double nx = norm_ub_from_sumsq(warp_sumsq(xt, H), H);
       // fp64 scores: |s^ - s| <= 1.01 * H * 2^-53 * ||x|| ||w|| (any summation order)
-      if (!select_token<T, EPL>(scores + t * E, 1.01 * H * kU53, 0.0, false, nx, nullptr, wss_g, bias,
+      if (!select_token<T, EPL, SIG>(scores + t * E, 1.01 * H * kU53, 0.0, false, nx, nullptr, wss_g, kf,
                                 xt, Wr, H, E, k, t, idx_ws, w_ws, idx_user, w_user, cands[warp], ctrl))
-        select_token_slow<T>(scores + t * E, 1, 1.01 * H * kU53, 0.0, false, nx, nullptr, wss_g,
-                             key_spill(spill, T_, E, t), bias, xt, Wr, H, E, k, t, idx_ws, w_ws,
+        select_token_slow<T, SIG>(scores + t * E, 1, 1.01 * H * kU53, 0.0, false, nx, nullptr, wss_g,
+                             key_spill(spill, T_, E, t), kf, xt, Wr, H, E, k, t, idx_ws, w_ws,
                              idx_user, w_user, exact_scratch[warp], ctrl);
     }
   }
@@ -1211,12 +1296,17 @@ static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
   auto sel = [&](auto kern) {
     return launch_pdl(kern, dim3(sgrid), dim3(32 * kSelectWarps), 0, st, static_cast<const double*>(a.scores64),
                       coef, a.H * 2.350988701644575e-38, static_cast<const double*>(a.xnorm),
-                      static_cast<const double*>(a.wnorm), a.bias, x, Wr, a.T, a.H, a.E, a.k, a.idx_ws,
+                      static_cast<const double*>(a.wnorm), Keys{a.bias, a.sigmoid, a.scale}, x, Wr, a.T, a.H,
+                      a.E, a.k, a.idx_ws,
                       a.w_ws, a.idx_user, a.w_user, a.spill, a.ctrl);
   };
   const int epl = select_epl(a.E);
-  e = epl == 4 ? sel(route_select_kernel<bf16, 4>) : epl == 12 ? sel(route_select_kernel<bf16, 12>)
-                                                                : sel(route_select_kernel<bf16, 32>);
+  if (a.sigmoid)
+    e = epl == 4 ? sel(route_select_kernel<bf16, 4, true>) : epl == 12 ? sel(route_select_kernel<bf16, 12, true>)
+                                                                      : sel(route_select_kernel<bf16, 32, true>);
+  else
+    e = epl == 4 ? sel(route_select_kernel<bf16, 4, false>) : epl == 12 ? sel(route_select_kernel<bf16, 12, false>)
+                                                                       : sel(route_select_kernel<bf16, 32, false>);
   count_launches(launches);
   return e;
 }
@@ -1227,12 +1317,18 @@ static cudaError_t launch_router_decode(const RouterArgs& a, cudaStream_t st) {
                   kDecodeSplit);
   auto go = [&](auto kern) {
     return launch_pdl(kern, grid, dim3(kDecodeThreads), 0, st, static_cast<const T*>(a.x),
-                      static_cast<const T*>(a.Wr), a.bias, a.T, a.H, a.E, a.k, a.scores64, a.wss,
+                      static_cast<const T*>(a.Wr), Keys{a.bias, a.sigmoid, a.scale}, a.T, a.H, a.E, a.k,
+                      a.scores64, a.wss,
                       a.group_done, a.idx_ws, a.w_ws, a.idx_user, a.w_user, a.spill, a.ctrl);
   };
   const int epl = select_epl(a.E);
-  const cudaError_t e = epl == 4 ? go(router_decode_kernel<T, 4>)
-                        : epl == 12 ? go(router_decode_kernel<T, 12>) : go(router_decode_kernel<T, 32>);
+  cudaError_t e;
+  if (a.sigmoid)
+    e = epl == 4 ? go(router_decode_kernel<T, 4, true>)
+        : epl == 12 ? go(router_decode_kernel<T, 12, true>) : go(router_decode_kernel<T, 32, true>);
+  else
+    e = epl == 4 ? go(router_decode_kernel<T, 4, false>)
+        : epl == 12 ? go(router_decode_kernel<T, 12, false>) : go(router_decode_kernel<T, 32, false>);
   count_launches(1);
   return e;
 }

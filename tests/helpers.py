@@ -38,12 +38,12 @@ def oracle_arrays(d: dict):
     return {k: to_oracle(v) if v is not None else None for k, v in d.items()}
 
 
-def oracle_routing(d: dict, top_k: int):
+def oracle_routing(d: dict, top_k: int, router: str = "softmax", scale: float = 1.0):
     """Exact routing of every token by the oracle."""
     a = oracle_arrays({"x": d["x"], "W_router": d["W_router"]})
     s = oracle.router_scores(a["x"], a["W_router"])
     bias = None if d.get("bias") is None else d["bias"].detach().cpu().numpy().astype(np.float32)
-    idx, w, w64 = oracle.route(s, top_k, bias)
+    idx, w, w64 = oracle.route(s, top_k, bias, router=router, scale=scale)
     counts, offsets, perm, inv = oracle.dispatch(idx, d["W_router"].shape[0])
     return dict(scores=s, idx=idx, w=w, w64=w64, counts=counts, offsets=offsets, perm=perm, inv_perm=inv)
 

@@ -107,12 +107,13 @@ def test_forward_ex_rejects_bad_swiglu_limits_before_any_launch(lib):
     P = ctypes.c_void_p
     n = moe.workspace_bytes(s)
 
-    def call(limit, limit_shared):
-        opts = moe.MoEOptions(limit, limit_shared)
+    def call(limit, limit_shared, router=0, scale=0.0):
+        opts = moe.MoEOptions(limit, limit_shared, router, scale)
         return lib.moe_layer_forward_ex(ctypes.byref(s), P(16), P(16), None, P(16), P(16), P(16), P(16),
                                         P(16), None, ctypes.byref(opts), P(256), n, None)
 
-    for bad in ((-1.0, 0.0), (0.0, -0.5), (float("nan"), 0.0), (0.0, float("inf"))):
+    for bad in ((-1.0, 0.0), (0.0, -0.5), (float("nan"), 0.0), (0.0, float("inf")), (0.0, 0.0, 2),
+                (0.0, 0.0, 1, -3.0), (0.0, 0.0, 1, float("nan"))):
         assert call(*bad) == 1, bad
     # NULL options is the plain forward (validation of the other arguments still runs)
     assert lib.moe_layer_forward_ex(ctypes.byref(s), None, P(16), None, P(16), P(16), P(16), P(16),

@@ -85,6 +85,30 @@ def test_swiglu_limits(sz):
     assert np.abs(y_ref - y_free).max() > 0.05 * np.abs(y_free).max()  # the clamps are active
 
 
+SIGMOID_CASES = [
+    dict(T=257, H=256, E=32, top_k=4, I=128, I_shared=128),                  # tensor-core scores
+    dict(T=3, H=2176, E=200, top_k=8, I=128, I_shared=128),                  # split reduction
+    dict(T=45, H=72, E=10, top_k=3, I=40, I_shared=24, dtype="f32", r_std=0.1),  # fp64 scores
+]
+
+
+@pytest.mark.parametrize("with_bias", [False, True])
+@pytest.mark.parametrize("sz", SIGMOID_CASES, ids=lambda s: "T{T}_H{H}_E{E}".format(**s) + s.get("dtype", ""))
+def test_sigmoid_router(sz, with_bias):
+    """The router as configured: p = sigma32(s), bias for the selection only, weights
+    3 * p / sum p; indices, counts, offsets and perm bit-exact against the oracle."""
+    cfg = inputs.small_config(**sz)
+    d = inputs.make_inputs(cfg, "cuda")
+    if with_bias:
+        d["bias"] = torch.linspace(-0.2, 0.2, cfg.E, dtype=torch.float32)
+    d = to_device(d)
+    y, r = run(d, cfg.top_k, router="sigmoid", routed_scaling_factor=3.0)
+    ref = oracle_routing(d, cfg.top_k, router="sigmoid", scale=3.0)
+    assert_routing_exact(r, ref, cfg.E)
+    assert_y_close(y, oracle_y(d, ref), "sigmoid router")
+    assert torch.allclose(r.topk_w.sum(1), torch.full((cfg.T,), 3.0, device=r.topk_w.device), rtol=1e-5)
+
+
 def test_small_bf16_with_router_bias():
     cfg = inputs.small_config(T=257, H=256, E=32, top_k=4, I=128, I_shared=128)
     d = inputs.make_inputs(cfg, "cuda")
