@@ -236,6 +236,30 @@ def test_full_size_workload(name):
     print(name, "route stats", stats)
 
 
+@pytest.mark.parametrize("name", ["decode_t4", "prefill_t16384_skew"])
+def test_full_size_layer_as_configured(name):
+    """The last layers as configured: sigmoid router with the routing factor 3 and a bias
+    for the selection, SwiGLU limits 7 (routed) and 16 (shared)."""
+    cfg = inputs.CONFIGS[name]
+    d = inputs.make_inputs(cfg, "cuda")
+    if d.get("bias") is None:
+        d["bias"] = torch.linspace(-0.05, 0.05, cfg.E, dtype=torch.float32)
+    d = to_device(d)
+    opts = dict(router="sigmoid", routed_scaling_factor=3.0, swiglu_limit=7.0, swiglu_limit_shared=16.0)
+    shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared, cfg.top_k, torch.bfloat16)
+    ws = moe.alloc_workspace(shape, "cuda")
+    y, r = run(d, cfg.top_k, workspace=ws, **opts)
+    assert moe.check_status(ws) == moe.MOE_OK
+    ref = oracle_routing(d, cfg.top_k, router="sigmoid", scale=3.0)
+    assert_routing_exact(r, ref, cfg.E)
+    rng = np.random.default_rng(cfg.seed)
+    tokens = np.arange(cfg.T) if cfg.T <= 128 else np.unique(
+        np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 30, replace=False)]))
+    y_ref = oracle_y(d, ref, tokens=tokens, swiglu_limit=7.0, swiglu_limit_shared=16.0)
+    assert_y_close(y[torch.as_tensor(tokens, device=y.device)], y_ref, name + " as configured")
+    print(name, "as configured, route stats", moe.route_stats(ws))
+
+
 # ------------------------------------------------------------------------------------
 # the tensor-core router's error bound
 # ------------------------------------------------------------------------------------
