@@ -223,6 +223,16 @@ MOE_API moe_status moe_layer_route_noalloc(const moe_layer_shape* shape, const v
                                            const void* W_router, const float* router_bias,
                                            int32_t* topk_idx, float* topk_w, void* stream);
 
+/* Self-test of the device-side failure detection.  Every wait of the library's kernels
+ * gives up after 2 s, records MOE_ERR_DEVICE_TIMEOUT in the workspace's status word and
+ * lets its kernel return, so a stalled pipeline ends with an error that
+ * moe_layer_check_status() reports instead of a hang.  This call clears the status word of
+ * `workspace` (at least 256-byte aligned, >= 64 bytes) and runs one kernel whose wait, the
+ * same code, is on a barrier that nothing completes: about 2 s later the status reads
+ * MOE_ERR_DEVICE_TIMEOUT and the stream and context remain usable.  No counterpart on the
+ * source pages. */
+MOE_API moe_status moe_layer_selftest_wait_timeout(void* workspace, size_t workspace_bytes, void* stream);
+
 /* Human-readable name of a status code (static string). */
 MOE_API const char* moe_status_string(moe_status status);
 

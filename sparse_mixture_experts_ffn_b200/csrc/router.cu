@@ -267,8 +267,7 @@ __device__ __forceinline__ double exp_fixed(double z) {
 }
 
 // The router's fp32 sigmoid score of an fp32 logit: 0 below -110, 1 above 40, else
-// fp32(1 / (1 + e^-s)).  Not monotone by construction, but within one ulp of it (the fp64
-// value is within a few ulps of the true sigmoid), which the interval ends allow for.
+// fp32(1 / (1 + e^-s)), within a few fp64 ulps of the exact sigmoid before the rounding.
 __device__ __forceinline__ float sigmoid32(float s32) {
   const double z = static_cast<double>(s32);
   if (z < -110.0) return 0.0f;
@@ -295,15 +294,22 @@ struct Keys {
     const float v = score(s);
     return bias ? __fadd_rn(v, bias[e]) : v;
   }
-  // lower / upper ends of the keys of all logits >= s_lo / <= s_hi
+  // Lower / upper ends of the keys of all logits >= s_lo / <= s_hi.  For the sigmoid the
+  // ends come from an fp32 evaluation, 1 / (1 + expf(-z)) (expf within 2 ulps over its whole
+  // range, as CUDA documents it; one rounding each for the add and the IEEE division), widened
+  // by a relative 2^-20: that covers its error against the exact sigmoid and the fp64
+  // definition's rounding to fp32, at a tenth of the cost of the fp64 evaluation.  Below
+  // z = -80 the ends are 0 and 2^-115 > sigma(-80).
   __device__ __forceinline__ float key_lo(double s_lo, int e) const {
     if (!sigmoid) return key(s_lo, e);
-    const float p = nextafterf(score(s_lo), -INFINITY);
+    const float z = __double2float_rd(s_lo);
+    const float p = z < -80.0f ? 0.0f : __fmul_rd(__fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-z))), 1.0f - 0x1p-20f);
     return bias ? __fadd_rd(p, bias[e]) : p;
   }
   __device__ __forceinline__ float key_hi(double s_hi, int e) const {
     if (!sigmoid) return key(s_hi, e);
-    const float p = nextafterf(score(s_hi), INFINITY);
+    const float z = __double2float_ru(s_hi);
+    const float p = z < -80.0f ? 0x1p-115f : __fmul_ru(__fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-z))), 1.0f + 0x1p-20f);
     return bias ? __fadd_ru(p, bias[e]) : p;
   }
 };

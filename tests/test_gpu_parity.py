@@ -329,3 +329,23 @@ def test_decode_tiles_with_popular_experts():
     ref = oracle_routing(d, cfg.top_k)
     assert_routing_exact(r, ref, cfg.E)
     assert_y_close(y, oracle_y(d, ref), "popular experts, 16-token tiles")
+
+
+def test_bounded_wait_times_out_with_a_readable_status():
+    """A wait on a barrier that nothing completes gives up (about 2 s), the status word
+    reads MOE_ERR_DEVICE_TIMEOUT, and the context still runs the layer correctly."""
+    import ctypes
+    import time
+    lib = moe.load_library()
+    lib.moe_layer_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    lib.moe_layer_selftest_wait_timeout.restype = ctypes.c_int
+    ws = torch.zeros(1 << 12, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    t0 = time.perf_counter()
+    rc = lib.moe_layer_selftest_wait_timeout(ctypes.c_void_p(ws.data_ptr()), ws.numel(),
+                                             ctypes.c_void_p(stream.cuda_stream))
+    assert rc == moe.MOE_OK
+    assert moe.check_status(ws) == 5  # MOE_ERR_DEVICE_TIMEOUT
+    assert 1.5 < time.perf_counter() - t0 < 30.0
+    cfg = inputs.small_config(T=64, H=256, E=16, top_k=4, I=128, I_shared=128)
+    check_full(to_device(inputs.make_inputs(cfg, "cuda")), cfg.top_k, "after a timeout")
