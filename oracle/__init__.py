@@ -61,13 +61,17 @@ def _load():
         lib.oracle_route_mode.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int, D,
                                           P, P, P]
         lib.oracle_sigmoid32.argtypes = [ctypes.c_int64, P, P]
+        lib.oracle_exact_dot_mixed.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P]
+        lib.oracle_router_scores_mixed.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                                   ctypes.c_int, P, P, P, ctypes.c_int]
         lib.oracle_expert_act.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, D, P]
         lib.oracle_moe_tokens.argtypes = [ctypes.c_int, ctypes.c_int64, P, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P,
                                           P, D, D, P, ctypes.c_int]
         for f in (lib.oracle_exact_dot, lib.oracle_router_scores, lib.oracle_route,
                   lib.oracle_dispatch, lib.oracle_expert_act, lib.oracle_moe_tokens,
-                  lib.oracle_route_mode, lib.oracle_sigmoid32):
+                  lib.oracle_route_mode, lib.oracle_sigmoid32, lib.oracle_exact_dot_mixed,
+                  lib.oracle_router_scores_mixed):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -96,25 +100,27 @@ def nthreads_default() -> int:
 
 
 def exact_dot(x: np.ndarray, w: np.ndarray) -> np.float32:
-    """Exact sum_h x[h]*w[h] rounded once to fp32 (nearest, ties to even)."""
+    """Exact sum_h x[h]*w[h] rounded once to fp32 (nearest, ties to even); each of x and w
+    bf16 (uint16 bit patterns) or float32."""
     x, w = _c(x), _c(w)
-    assert x.shape == w.shape and x.ndim == 1 and x.dtype == w.dtype
+    assert x.shape == w.shape and x.ndim == 1
     out = np.zeros(1, np.float32)
-    rc = _load().oracle_exact_dot(_dtype_code(x), x.shape[0], _p(x), _p(w), _p(out))
+    rc = _load().oracle_exact_dot_mixed(_dtype_code(x), _dtype_code(w), x.shape[0], _p(x), _p(w), _p(out))
     if rc != 0:
         raise ValueError("exact_dot: non-finite input")
     return out[0]
 
 
 def router_scores(x: np.ndarray, Wr: np.ndarray, nthreads: int = 0) -> np.ndarray:
-    """s[t,e] = RN32(exact x[t] . Wr[e]) for every token t and expert e -> float32 [T,E]."""
+    """s[t,e] = RN32(exact x[t] . Wr[e]) for every token t and expert e -> float32 [T,E]
+    (x and Wr each bf16 or float32: fp32 router weights with bf16 tokens are allowed)."""
     x, Wr = _c(x), _c(Wr)
     T, H = x.shape
     E, H2 = Wr.shape
-    assert H == H2 and x.dtype == Wr.dtype
+    assert H == H2
     s = np.empty((T, E), np.float32)
-    rc = _load().oracle_router_scores(_dtype_code(x), T, H, E, _p(x), _p(Wr), _p(s),
-                                      nthreads or nthreads_default())
+    rc = _load().oracle_router_scores_mixed(_dtype_code(x), _dtype_code(Wr), T, H, E, _p(x), _p(Wr), _p(s),
+                                            nthreads or nthreads_default())
     if rc != 0:
         raise ValueError("router_scores: non-finite input")
     return s

@@ -65,8 +65,9 @@
 
 /* smallest product exponent: fp32 subnormal * subnormal = 2^-149 * 2^-149 */
 #define BIN_EMIN (-298)
-/* largest exponent a bin can receive: bf16 max 2^120*2^120 = 2^240, fp32 hi half 2^232 */
-#define BIN_EMAX 241
+/* largest exponent a bin can receive: bf16 max 2^120*2^120 = 2^240, fp32 hi half 2^232,
+   bf16 x fp32 hi half 2^248 */
+#define BIN_EMAX 249
 #define NBINS (BIN_EMAX - BIN_EMIN + 1)
 /* room for the carries of up to 2^62 in magnitude above the top bin */
 #define NBITS (NBINS + 72)
@@ -159,21 +160,15 @@ static float round_bins_to_f32(const int64_t* bins) {
   return negative ? -f : f;
 }
 
-/* Exact sum_h x[h]*w[h] rounded once to fp32.  Returns 0 on success, -1 on a
-   non-finite input, -2 if the length could overflow a bin. */
-static int exact_dot_f32(int dtype, int n, const void* x, const void* w, float* out) {
+/* Exact sum_h x[h]*w[h] rounded once to fp32, x and w each bf16 or fp32.  Returns 0 on
+   success, -1 on a non-finite input, -2 if the length could overflow a bin. */
+static int exact_dot_mixed(int dtype_x, int dtype_w, int n, const void* x, const void* w, float* out) {
   int64_t bins[NBINS];
   memset(bins, 0, sizeof(bins));
   if (n > (1 << 30)) return -2;
   for (int h = 0; h < n; ++h) {
-    dyadic a, b;
-    if (dtype == OR_BF16) {
-      a = decode_bf16(((const uint16_t*)x)[h]);
-      b = decode_bf16(((const uint16_t*)w)[h]);
-    } else {
-      a = decode_f32(((const uint32_t*)x)[h]);
-      b = decode_f32(((const uint32_t*)w)[h]);
-    }
+    dyadic a = dtype_x == OR_BF16 ? decode_bf16(((const uint16_t*)x)[h]) : decode_f32(((const uint32_t*)x)[h]);
+    dyadic b = dtype_w == OR_BF16 ? decode_bf16(((const uint16_t*)w)[h]) : decode_f32(((const uint32_t*)w)[h]);
     if (!a.finite || !b.finite) return -1;
     if (a.m == 0 || b.m == 0) continue;
     int64_t p = (int64_t)a.m * (int64_t)b.m; /* |p| < 2^48 */
@@ -188,9 +183,16 @@ static int exact_dot_f32(int dtype, int n, const void* x, const void* w, float* 
   return 0;
 }
 
+static int exact_dot_f32(int dtype, int n, const void* x, const void* w, float* out) {
+  return exact_dot_mixed(dtype, dtype, n, x, w, out);
+}
+
 /* Exposed for the tests that pin the exact dot product on its own. */
 int oracle_exact_dot(int dtype, int n, const void* x, const void* w, float* out) {
   return exact_dot_f32(dtype, n, x, w, out);
+}
+int oracle_exact_dot_mixed(int dtype_x, int dtype_w, int n, const void* x, const void* w, float* out) {
+  return exact_dot_mixed(dtype_x, dtype_w, n, x, w, out);
 }
 
 static size_t esize(int dtype) { return dtype == OR_BF16 ? 2 : 4; }
@@ -207,12 +209,13 @@ static double to_f64(int dtype, const void* base, size_t i) {
 
 /* ------------------------------------------------------------------------------------
  * Router scores: s[t,e] = RN32(exact sum_h x[t,h] W_r[e,h]) for every token and expert
- * (router logits; fp32 scores per need_fp32_gate).
+ * (router logits; fp32 scores per need_fp32_gate).  The router matrix may be fp32 with
+ * bf16 tokens (need_fp32_gate read as fp32 router weights).
  * ---------------------------------------------------------------------------------- */
-int oracle_router_scores(int dtype, int64_t T, int H, int E, const void* x, const void* Wr,
-                         float* s_out, int nthreads) {
+int oracle_router_scores_mixed(int dtype_x, int dtype_w, int64_t T, int H, int E, const void* x,
+                               const void* Wr, float* s_out, int nthreads) {
   int err = 0;
-  size_t es = esize(dtype);
+  size_t es = esize(dtype_x), ews = esize(dtype_w);
 #ifdef _OPENMP
   if (nthreads > 0) omp_set_num_threads(nthreads);
 #endif
@@ -221,12 +224,17 @@ int oracle_router_scores(int dtype, int64_t T, int H, int E, const void* x, cons
     int64_t t = te / E;
     int e = (int)(te % E);
     const char* xr = (const char*)x + (size_t)t * H * es;
-    const char* wr = (const char*)Wr + (size_t)e * H * es;
+    const char* wr = (const char*)Wr + (size_t)e * H * ews;
     float s;
-    if (exact_dot_f32(dtype, H, xr, wr, &s) != 0) err |= 1;
+    if (exact_dot_mixed(dtype_x, dtype_w, H, xr, wr, &s) != 0) err |= 1;
     s_out[te] = s;
   }
   return err ? -1 : 0;
+}
+
+int oracle_router_scores(int dtype, int64_t T, int H, int E, const void* x, const void* Wr,
+                         float* s_out, int nthreads) {
+  return oracle_router_scores_mixed(dtype, dtype, T, H, E, x, Wr, s_out, nthreads);
 }
 
 /* ------------------------------------------------------------------------------------

@@ -94,6 +94,26 @@ def test_exact_dot_matches_rational_sum(dtype):
         assert got.tobytes() == want.tobytes() or (got == 0 and want == 0), (trial, got, want)
 
 
+def test_exact_dot_mixed_bf16_tokens_fp32_router_weights():
+    """need_fp32_gate read as fp32 router weights with bf16 tokens: the exact sum of bf16 x
+    fp32 products (subnormals, extreme exponents, cancellation) against rational arithmetic."""
+    rng = np.random.default_rng(4321)
+    for trial in range(300):
+        n = int(rng.integers(1, 80))
+        x = random_wide_vector(rng, n, "bf16")
+        w = random_wide_vector(rng, n, "f32")
+        got = oracle.exact_dot(x, w)
+        want = brute_dot(x, w)
+        assert got.tobytes() == want.tobytes() or (got == 0 and want == 0), (trial, got, want)
+    # router scores with fp32 weights are the same exact dots
+    xs = np.stack([random_wide_vector(rng, 48, "bf16") for _ in range(3)])
+    ws = np.stack([random_wide_vector(rng, 48, "f32") for _ in range(5)])
+    s = oracle.router_scores(xs, ws)
+    for t in range(3):
+        for e in range(5):
+            assert s[t, e].tobytes() == brute_dot(xs[t], ws[e]).tobytes() or (s[t, e] == 0 and brute_dot(xs[t], ws[e]) == 0)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_exact_dot_router_like_vectors(dtype):
     rng = np.random.default_rng(99)
