@@ -197,6 +197,15 @@ def layer_options(args) -> dict:
                 swiglu_limit=args.swiglu_limit, swiglu_limit_shared=args.swiglu_limit_shared)
 
 
+def config_options(args) -> dict:
+    """The options as reported in the JSON line's config (empty for the defaults)."""
+    o = layer_options(args)
+    out = {"layer_options": o} if o != LAYER_DEFAULTS else {}
+    if getattr(args, "fp32_router", False):
+        out["router_weights"] = "fp32"
+    return out
+
+
 def oracle_step(h, cfg, tokens, opts=None):
     """The whole hot path for the listed tokens: exact router over all experts, top-k and
     weights, then the expert FFNs and the combine."""
@@ -217,8 +226,10 @@ def run_reference(args, cfg):
     import oracle
     oracle.build()
     d = inputs.make_inputs(cfg, "cpu") if cfg.T * cfg.H * cfg.E < 5e7 else None
+    if d is not None and args.fp32_router:
+        d["W_router"] = inputs.make_routing_inputs(cfg, router_fp32=True)[1]
     if d is None:
-        x, Wr, bias = inputs.make_routing_inputs(cfg)
+        x, Wr, bias = inputs.make_routing_inputs(cfg, router_fp32=args.fp32_router)
         dev = "cuda" if torch.cuda.is_available() else "cpu"
         Wgu, Wd, Wsgu, Wsd = inputs.make_expert_weights(cfg, dev)
         d = dict(x=x, W_router=Wr, bias=bias, W_gate_up=Wgu, W_down=Wd, Ws_gate_up=Wsgu, Ws_down=Wsd)
@@ -238,8 +249,7 @@ def run_reference(args, cfg):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
             "data": "synthetic", "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E,
                                              "top_k": cfg.top_k, "I": cfg.I, "I_shared": cfg.I_shared,
-                                             **({"layer_options": layer_options(args)}
-                                                if layer_options(args) != LAYER_DEFAULTS else {})},
+                                             **config_options(args)},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -278,6 +288,7 @@ def main():
     ap.add_argument("--router", default="softmax", choices=["softmax", "sigmoid"],
                     help="router mode (sigmoid: the router as configured, bias for the selection only)")
     ap.add_argument("--routed-scale", type=float, default=1.0, help="sigmoid router: routed scaling factor")
+    ap.add_argument("--fp32-router", action="store_true", help="fp32 router weights (bf16 tokens and experts)")
     ap.add_argument("--swiglu-limit", type=float, default=0.0, help="SwiGLU limit of the routed experts")
     ap.add_argument("--swiglu-limit-shared", type=float, default=0.0, help="SwiGLU limit of the shared expert")
     ap.add_argument("--I", type=int, default=None,
@@ -315,7 +326,7 @@ def main():
     moe.load_library()
 
     # ---- inputs (resident in HBM); each rank is a replica with its own tokens -------------
-    x, Wr, bias = inputs.make_routing_inputs(rank_config(cfg, rank))
+    x, Wr, bias = inputs.make_routing_inputs(rank_config(cfg, rank), router_fp32=args.fp32_router)
     Wgu, Wd, Wsgu, Wsd = inputs.make_expert_weights(cfg, dev)
     x, Wr = x.to(dev), Wr.to(dev)
     bias = None if bias is None else bias.to(dev)
@@ -431,7 +442,7 @@ def main():
             "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
             "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "top_k": cfg.top_k,
                        "I": cfg.I, "I_shared": cfg.I_shared, "tokens_per_gpu": cfg.T,
-                       **({"layer_options": layer_options(args)} if layer_options(args) != LAYER_DEFAULTS else {}),
+                       **config_options(args),
                        "l2": "flushed before every timed step (2x L2 write, outside the events)",
                        "parallelism": f"replicas x{world}"},
             "roofline": roof,

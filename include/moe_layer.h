@@ -124,13 +124,19 @@ MOE_API moe_status moe_layer_forward(const moe_layer_shape* shape, const void* x
  *   multiply-adds, scaling by 2^n; p = 0 below s = -110 and 1 above 40); the router bias
  *   only steers the selection (key_e = fp32(p_e + b_e)); the weights are
  *   routed_scaling_factor * p_j / sum of the chosen p (uniform if that sum is 0).
- *   routed_scaling_factor: sigmoid router only; 0 is read as 1; else finite and > 0. */
+ *   routed_scaling_factor: sigmoid router only; 0 is read as 1; else finite and > 0.
+ *   router_weights_fp32: 1 = W_router is fp32 [E, H] while the tokens and experts are bf16
+ *   (need_fp32_gate on the same table, read as fp32 router weights).  The scores stay the
+ *   exact dot rounded once to fp32; the weights are split into three bf16 parts for the
+ *   tensor cores.  Needs E <= 512 and H a multiple of 64 (else MOE_ERR_UNSUPPORTED_SHAPE);
+ *   ignored for fp32 layers, whose router is fp32 already. */
 enum { MOE_ROUTER_SOFTMAX = 0, MOE_ROUTER_SIGMOID = 1 };
 typedef struct {
   float swiglu_limit;
   float swiglu_limit_shared;
   int32_t router;
   float routed_scaling_factor;
+  int32_t router_weights_fp32;
 } moe_layer_options;
 
 /* moe_layer_forward() with per-layer options; options = NULL is moe_layer_forward().

@@ -38,7 +38,8 @@ class MoEShape(ctypes.Structure):
 
 class MoEOptions(ctypes.Structure):
     _fields_ = [("swiglu_limit", ctypes.c_float), ("swiglu_limit_shared", ctypes.c_float),
-                ("router", ctypes.c_int32), ("routed_scaling_factor", ctypes.c_float)]
+                ("router", ctypes.c_int32), ("routed_scaling_factor", ctypes.c_float),
+                ("router_weights_fp32", ctypes.c_int32)]
 
 
 ROUTERS = {"softmax": 0, "sigmoid": 1}
@@ -151,6 +152,7 @@ def moe_layer_forward(x, W_router, W_gate_up, W_down, Ws_gate_up=None, Ws_down=N
                       router_bias=None, y=None, workspace=None, routing=True, stream=None,
                       swiglu_limit=0.0, swiglu_limit_shared=0.0, router="softmax",
                       routed_scaling_factor=1.0):
+    # W_router may be fp32 while the layer is bf16 (fp32 router weights)
     """Run the MoE layer on the device.  Returns (y, Routing or None).
 
     Shapes: x [T,H], W_router [E,H], W_gate_up [E,2I,H], W_down [E,H,I], Ws_gate_up
@@ -188,8 +190,9 @@ def moe_layer_forward(x, W_router, W_gate_up, W_down, Ws_gate_up=None, Ws_down=N
                              r.offsets.data_ptr(), r.perm.data_ptr())
     if stream is None:
         stream = torch.cuda.current_stream(x.device)
+    w32 = 1 if (x.dtype == torch.bfloat16 and W_router.dtype == torch.float32) else 0
     opts = MoEOptions(float(swiglu_limit), float(swiglu_limit_shared), ROUTERS[router],
-                      float(routed_scaling_factor))
+                      float(routed_scaling_factor), w32)
     rc = lib.moe_layer_forward_ex(ctypes.byref(shape), _ptr(x), _ptr(W_router), _ptr(router_bias),
                                   _ptr(W_gate_up), _ptr(W_down), _ptr(Ws_gate_up), _ptr(Ws_down),
                                   _ptr(y), ctypes.byref(rout) if rout is not None else None,

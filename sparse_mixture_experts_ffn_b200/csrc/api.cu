@@ -97,7 +97,7 @@ static size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255);
 
 struct Layout {
   size_t ctrl, group_done, tile_done, item_counters, wss, zero_end, scores, xnorm, wnorm, idx, w, blk_hist, counts,
-      offsets, group_order, item_start_gu, item_start_dn, perm, inv_perm, row_w, row_tok, partial, spill, rsplit,
+      offsets, group_order, item_start_gu, item_start_dn, perm, inv_perm, row_w, row_tok, partial, spill, rsplit, w3,
       x_perm, h, h_shared, o, o_shared, total;
   int bn, bn_dn, ksplit;
   int64_t max_tiles;
@@ -132,6 +132,7 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.zero_end = tc_scores ? L.scores : off;
   L.spill = take(T * E * 20);
   L.rsplit = take(router_split_bytes(*s));
+  L.w3 = take(router_w3_bytes(*s));
   L.xnorm = take(T * 8);
   L.wnorm = take(E * 8);
   L.idx = take(P * 4);
@@ -221,15 +222,18 @@ extern "C" moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const v
                                            const void* Ws_gate_up, const void* Ws_down, void* y,
                                            moe_routing_out* routing, const moe_layer_options* options,
                                            void* workspace, size_t workspace_bytes, void* stream) {
-  const moe_layer_options opt = options ? *options : moe_layer_options{0.0f, 0.0f, MOE_ROUTER_SOFTMAX, 0.0f};
+  const moe_layer_options opt = options ? *options : moe_layer_options{0.0f, 0.0f, MOE_ROUTER_SOFTMAX, 0.0f, 0};
   if (!(opt.swiglu_limit >= 0.0f && opt.swiglu_limit <= FLT_MAX) ||
       !(opt.swiglu_limit_shared >= 0.0f && opt.swiglu_limit_shared <= FLT_MAX) ||
       !(opt.routed_scaling_factor >= 0.0f && opt.routed_scaling_factor <= FLT_MAX))
     return MOE_ERR_INVALID_ARG;  // negative, infinite or NaN
   if (opt.router != MOE_ROUTER_SOFTMAX && opt.router != MOE_ROUTER_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (opt.router_weights_fp32 != 0 && opt.router_weights_fp32 != 1) return MOE_ERR_INVALID_ARG;
   const moe_status vs = validate_shape(shape);
   if (vs != MOE_OK) return vs;
   const moe_layer_shape& s = *shape;
+  // fp32 router weights with bf16 tokens run on the tensor-core router only
+  if (opt.router_weights_fp32 && s.dtype == MOE_BF16 && !router_w32_supported(s)) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (s.T == 0) return MOE_OK;  // empty batch: nothing to read or write
   if (!x || !W_router || !W_gate_up || !W_down || !y || !workspace) return MOE_ERR_INVALID_ARG;
   const bool has_shared = s.I_shared > 0;
@@ -274,6 +278,8 @@ extern "C" moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const v
   ra.wss = static_cast<double*>(at(L.wss));
   ra.spill = static_cast<float*>(at(L.spill));
   ra.sigmoid = opt.router == MOE_ROUTER_SIGMOID ? 1 : 0;
+  ra.w32 = bf16 && opt.router_weights_fp32;
+  ra.w3 = at(L.w3);
   ra.scale = opt.routed_scaling_factor > 0.0f ? opt.routed_scaling_factor : 1.0f;
   ra.rsplit = router_split_bytes(*shape) ? at(L.rsplit) : nullptr;
   ra.xnorm = static_cast<double*>(at(L.xnorm));

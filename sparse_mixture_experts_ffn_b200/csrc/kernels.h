@@ -51,6 +51,8 @@ struct RouterArgs {
   float* w_user;
   float* spill;      // [5, T, E] key state of tokens that need exact dots
   void* rsplit;      // router_split_bytes(shape) bytes, or null: the reduction is not split
+  bool w32;          // bf16 tokens with fp32 router weights (Wr is float [E, H])
+  void* w3;          // router_w3_bytes(shape): the fp32 weights split into 3 bf16 parts
   Ctrl* ctrl;
 };
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
@@ -58,6 +60,10 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
 int64_t router_group_counters(int64_t T, int E);
 // scratch of the reduction-split tensor-core router (0 when a batch fills the GPU unsplit)
 size_t router_split_bytes(const moe_layer_shape& s);
+// the bf16 split of fp32 router weights for the tensor-core router (0 when it is not used)
+size_t router_w3_bytes(const moe_layer_shape& s);
+// whether fp32 router weights can be used with this shape (bf16 tokens, tensor-core router)
+bool router_w32_supported(const moe_layer_shape& s);
 // whether the router scores of this shape come from the tensor cores (else fp64)
 bool router_scores_f32(const moe_layer_shape& s);
 // products per fp32-accumulated slice of the tensor-core router scores

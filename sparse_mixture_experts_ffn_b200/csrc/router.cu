@@ -140,8 +140,8 @@ __device__ __forceinline__ void bin_add(long long* bins, int q, long long v) {
   atomicAdd(reinterpret_cast<unsigned long long*>(&bins[q - kQMin]), static_cast<unsigned long long>(v));
 }
 
-template <typename T>
-__device__ __noinline__ float warp_exact_dot_rn32(const T* __restrict__ a, const T* __restrict__ b, int H,
+template <typename TA, typename TB>
+__device__ __noinline__ float warp_exact_dot_rn32(const TA* __restrict__ a, const TB* __restrict__ b, int H,
                                      long long* bins /* kNBins, warp-private smem */,
                                      uint32_t* limbs /* kNLimbs, warp-private smem */) {
   const int lane = threadIdx.x & 31;
@@ -162,7 +162,7 @@ __device__ __noinline__ float warp_exact_dot_rn32(const T* __restrict__ a, const
       int m1, q1, m2, q2;
       decode(a[h], m1, q1);
       decode(b[h], m2, q2);
-      const long long p = static_cast<long long>(m1) * m2;  // |p| < 2^48
+      const long long p = static_cast<long long>(m1) * m2;  // |p| < 2^48 (bf16 x fp32: < 2^32)
       if (p == 0) continue;
       const int q = q1 + q2;
       if (q >= anchor) {
@@ -345,6 +345,48 @@ __device__ __forceinline__ void put(V (&a)[EPL], int i, V v) {
 }
 
 // fp64 dot with four 16-byte loads per operand in flight per lane
+// eight consecutive elements as floats (one 16-byte load of bf16, two of fp32)
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&o)[8]) {
+  const Vec16<__nv_bfloat16> v = ld16(p);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) o[j] = __bfloat162float(v.v[j]);
+}
+__device__ __forceinline__ void load8(const float* p, float (&o)[8]) {
+  const Vec16<float> v0 = ld16(p), v1 = ld16(p + 4);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    o[j] = v0.v[j];
+    o[4 + j] = v1.v[j];
+  }
+}
+
+// fp64 dot of two rows of different types (bf16 tokens, fp32 router weights): exact
+// products, fp64 accumulation; H a multiple of 8
+template <typename TA, typename TB>
+__device__ double warp_dot_f64_prefetch(const TA* __restrict__ a, const TB* __restrict__ b, int H) {
+  const int lane = threadIdx.x & 31;
+  double acc = 0.0;
+  const int n8 = H / 8;
+  for (int v = lane; v < n8; v += 64) {
+    float av[2][8], bv[2][8];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      if (v + 32 * u < n8) {
+        load8(a + (v + 32 * u) * 8, av[u]);
+        load8(b + (v + 32 * u) * 8, bv[u]);
+      }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (v + 32 * u >= n8) break;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc = fma(static_cast<double>(av[u][j]), static_cast<double>(bv[u][j]), acc);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  return acc;
+}
+
 template <typename T>
 __device__ double warp_dot_f64_prefetch(const T* __restrict__ a, const T* __restrict__ b, int H) {
   const int lane = threadIdx.x & 31;
@@ -402,13 +444,13 @@ struct CandList {
 };
 
 // SIG: the router mode as a compile-time constant (the softmax path carries no sigmoid code)
-template <typename T, int EPL, bool SIG>
+template <typename T, typename TW, int EPL, bool SIG>
 __device__ __forceinline__ bool select_token(const double* __restrict__ srow, double delta_coef,
                                              double delta_abs, bool refine_f64, double nx,
                                              const double* __restrict__ wnorm,
                                              const double* __restrict__ wss,
                                              const Keys kf_in, const T* __restrict__ xt,
-                                             const T* __restrict__ Wr, int H, int E, int k, int64_t t,
+                                             const TW* __restrict__ Wr, int H, int E, int k, int64_t t,
                                              int32_t* __restrict__ idx_ws, float* __restrict__ w_ws,
                                              int32_t* __restrict__ idx_user, float* __restrict__ w_user,
                                              CandList& C, Ctrl* ctrl) {
@@ -604,14 +646,14 @@ __device__ __forceinline__ KeySpill key_spill(float* base, int64_t T, int E, int
 // warp): intervals from the score estimates, fp64 recompute (when the estimates are not
 // fp64 sums) and exact dots for what stays undecided, classification, open slots,
 // weights and outputs.
-template <typename T, bool SIG>
+template <typename T, typename TW, bool SIG>
 __device__ __noinline__ void select_token_slow(const double* __restrict__ srow, int64_t sstride,
                                                double delta_coef,
                                                double delta_abs, bool refine_f64, double nx,
                                                const double* __restrict__ wnorm,
                                                const double* __restrict__ wss, KeySpill sp,
                                                const Keys kf_in,
-                                               const T* __restrict__ xt, const T* __restrict__ Wr,
+                                               const T* __restrict__ xt, const TW* __restrict__ Wr,
                                                int H, int E, int k, int64_t t,
                                                int32_t* __restrict__ idx_ws, float* __restrict__ w_ws,
                                                int32_t* __restrict__ idx_user, float* __restrict__ w_user,
@@ -667,7 +709,7 @@ __device__ __noinline__ void select_token_slow(const double* __restrict__ srow, 
       while (mask) {
         const int e = base + __ffs(mask) - 1;
         mask &= mask - 1;
-        const T* we = Wr + static_cast<size_t>(e) * H;
+        const TW* we = Wr + static_cast<size_t>(e) * H;
         float klo, khi, kmid, kp;
         if (pass == 0) {
           const double s64 = warp_dot_f64_prefetch(xt, we, H);
@@ -764,11 +806,11 @@ __device__ __noinline__ void select_token_slow(const double* __restrict__ srow, 
 // ---------------------------------------------------------------------------------------
 constexpr int kSelectWarps = 4;
 
-template <typename T, int EPL, bool SIG>
+template <typename T, typename TW, int EPL, bool SIG>
 __global__ void __launch_bounds__(32 * kSelectWarps) route_select_kernel(
     const double* __restrict__ scores, double delta_coef, double delta_abs,
     const double* __restrict__ xnorm, const double* __restrict__ wnorm,
-    const Keys kf, const T* __restrict__ x, const T* __restrict__ Wr,
+    const Keys kf, const T* __restrict__ x, const TW* __restrict__ Wr,
     int64_t T_, int H, int E, int k, int32_t* __restrict__ idx_ws, float* __restrict__ w_ws,
     int32_t* __restrict__ idx_user, float* __restrict__ w_user, float* __restrict__ spill,
     Ctrl* ctrl) {
@@ -778,10 +820,10 @@ __global__ void __launch_bounds__(32 * kSelectWarps) route_select_kernel(
   const int warp = threadIdx.x >> 5;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kSelectWarps + warp;
   if (t < T_) {
-    if (!select_token<T, EPL, SIG>(scores + t * E, delta_coef, delta_abs, true, xnorm[t], wnorm, nullptr,
+    if (!select_token<T, TW, EPL, SIG>(scores + t * E, delta_coef, delta_abs, true, xnorm[t], wnorm, nullptr,
                               kf, x + t * H, Wr, H, E, k, t, idx_ws, w_ws, idx_user, w_user,
                               cands[warp], ctrl))
-      select_token_slow<T, SIG>(scores + t * E, 1, delta_coef, delta_abs, true, xnorm[t], wnorm, nullptr,
+      select_token_slow<T, TW, SIG>(scores + t * E, 1, delta_coef, delta_abs, true, xnorm[t], wnorm, nullptr,
                            key_spill(spill, T_, E, t), kf, x + t * H, Wr, H, E, k, t, idx_ws, w_ws,
                            idx_user, w_user, exact_scratch[warp], ctrl);
   }
@@ -902,9 +944,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) router_decode_kernel(
       const T* xt = x + t * H;
       const double nx = norm_ub_from_sumsq(warp_sumsq(xt, H), H);
       // fp64 scores: |s^ - s| <= 1.01 * H * 2^-53 * ||x|| ||w|| (any summation order)
-      if (!select_token<T, EPL, SIG>(scores + t * E, 1.01 * H * kU53, 0.0, false, nx, nullptr, wss_g, kf,
+      if (!select_token<T, T, EPL, SIG>(scores + t * E, 1.01 * H * kU53, 0.0, false, nx, nullptr, wss_g, kf,
                                 xt, Wr, H, E, k, t, idx_ws, w_ws, idx_user, w_user, cands[warp], ctrl))
-        select_token_slow<T, SIG>(scores + t * E, 1, 1.01 * H * kU53, 0.0, false, nx, nullptr, wss_g,
+        select_token_slow<T, T, SIG>(scores + t * E, 1, 1.01 * H * kU53, 0.0, false, nx, nullptr, wss_g,
                              key_spill(spill, T_, E, t), kf, xt, Wr, H, E, k, t, idx_ws, w_ws,
                              idx_user, w_user, exact_scratch[warp], ctrl);
     }
@@ -940,10 +982,12 @@ constexpr int kRtMaxChunks = 8;
 constexpr int kRtSmTarget = 148;                     // blocks that fill the GPU
 
 struct RouterTcParams {
-  CUtensorMap tmX;   // x [T, H], box {64, 16}
-  CUtensorMap tmW;   // W_router [E, H], box {64, 64}
+  CUtensorMap tmX;   // x [T, Hx], box {64, 16}
+  CUtensorMap tmW;   // W_router [E, H] (fp32 weights: their bf16 split [E, 3 Hx]), box {64, 64}
   int64_t T;
-  int H, E;
+  int H, E;          // H: length of the reduction (Hx, or 3 Hx for split fp32 weights)
+  int Hx;            // tokens' hidden size; reduction step kb reads x columns (kb mod Hx/64)
+  int w_given;       // W_router norms precomputed (split fp32 weights): no W sums of squares
   double* scores;    // [T, E]
   // split only
   int chunks, chunk_slices;
@@ -1052,8 +1096,9 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
         if (!mbar_wait(&empty[stage], phase ^ 1u, p.ctrl, abort_flag)) break;
         unsigned char* st = smem + stage * kRtStageBytes;
         mbar_arrive_expect_tx(&full[stage], bytes);
+        const int xcol = (kb % (p.Hx / kTileK)) * kTileK;
         for (int b = 0; b < nbox; ++b)
-          tma_load_2d(st + b * kRtRowBox * kTileK * 2, &p.tmX, kb * kTileK,
+          tma_load_2d(st + b * kRtRowBox * kTileK * 2, &p.tmX, xcol,
                       static_cast<int32_t>(t0 + b * kRtRowBox), &full[stage]);
         tma_load_2d(st + kRtABytes, &p.tmW, kb * kTileK, e0, &full[stage]);
         used |= 1u << stage;
@@ -1126,9 +1171,10 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
       // sums of squares of this chunk's columns while the MMAs run: the x rows once per
       // m tile (n == 0), the W_router rows once per n tile (m == 0)
       const int c0 = kb_begin * kTileK, c1 = kb_end * kTileK;
-      if (blockIdx.y == 0)
-        sumsq_rows_bf16(p.x + t0 * p.H, p.H, rows, c0, c1, p.xss + blockIdx.z * p.T + t0, quarter, lane);
-      if (blockIdx.x == 0)
+      if (blockIdx.y == 0)  // x columns once (the split fp32 weights repeat them)
+        sumsq_rows_bf16(p.x + t0 * p.Hx, p.Hx, rows, min(c0, p.Hx), min(c1, p.Hx),
+                        p.xss + blockIdx.z * p.T + t0, quarter, lane);
+      if (blockIdx.x == 0 && !p.w_given)
         sumsq_rows_bf16(p.Wr + static_cast<int64_t>(e0) * p.H, p.H, ne, c0, c1,
                         p.wss + static_cast<int64_t>(blockIdx.z) * p.E + e0, quarter, lane);
       for (int sl = 0; sl < n_sl && ok; ++sl) {
@@ -1172,9 +1218,9 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
           for (int i = et; i < rows; i += 128) {
             double ss = 0.0;
             for (int z = 0; z < p.chunks; ++z) ss += __ldcg(p.xss + z * p.T + t0 + i);
-            p.xnorm[t0 + i] = norm_ub_from_sumsq(ss, p.H);
+            p.xnorm[t0 + i] = norm_ub_from_sumsq(ss, p.Hx);
           }
-        if (blockIdx.x == 0)
+        if (blockIdx.x == 0 && !p.w_given)
           for (int i = et; i < ne; i += 128) {
             double ss = 0.0;
             for (int z = 0; z < p.chunks; ++z) ss += __ldcg(p.wss + static_cast<int64_t>(z) * p.E + e0 + i);
@@ -1241,40 +1287,122 @@ static int router_chunks(int64_t T, int E, int H) {
   return (n_sl + per - 1) / per;
 }
 
+static size_t split_bytes_for(int64_t T, int E, int K) {
+  const int c = router_chunks(T, E, K);
+  if (c == 1) return 0;
+  const size_t n_sl = static_cast<size_t>((K / kTileK + kRtSliceSteps - 1) / kRtSliceSteps);
+  return static_cast<size_t>(c) * (static_cast<size_t>(T) + E) * 8 + n_sl * static_cast<size_t>(T) * E * 4;
+}
+
+// room for both reduction lengths: H, and 3H for split fp32 router weights
 size_t router_split_bytes(const moe_layer_shape& s) {
   if (!router_tc_supported(s.dtype == MOE_BF16, s.T, s.E, s.H)) return 0;
-  const int c = router_chunks(s.T, s.E, s.H);
-  if (c == 1) return 0;
-  const size_t n_sl = static_cast<size_t>((s.H / kTileK + kRtSliceSteps - 1) / kRtSliceSteps);
-  const size_t T = static_cast<size_t>(s.T), E = static_cast<size_t>(s.E);
-  return static_cast<size_t>(c) * (T + E) * 8 + n_sl * T * E * 4;
+  return std::max(split_bytes_for(s.T, s.E, s.H), split_bytes_for(s.T, s.E, 3 * s.H));
+}
+
+bool router_w32_supported(const moe_layer_shape& s) {
+  return router_tc_supported(s.dtype == MOE_BF16, s.T > 0 ? s.T : 1, s.E, s.H);
+}
+
+size_t router_w3_bytes(const moe_layer_shape& s) {
+  if (!router_tc_supported(s.dtype == MOE_BF16, s.T, s.E, s.H)) return 0;
+  return static_cast<size_t>(s.E) * 3 * s.H * 2;
+}
+
+// fp32 router weights on the bf16 tensor cores: W = hi + mid + lo, each part bf16, so that
+// x . W is the bf16 GEMM of x against [hi | mid | lo] over 3H (every part is an exact fp32
+// difference; lo is exact unless W falls below the bf16 normal range, and whatever it misses
+// goes into the norm bound).  One warp per expert row also bounds the row's norm for the
+// selection: ||hi|| + ||mid|| + ||lo|| (all products of the split counted), plus the
+// unrepresented rest scaled by 1/coef, so that coef * |x| * bound still covers it.
+__global__ void split_w32_kernel(const float* __restrict__ W, int E, int H, __nv_bfloat16* __restrict__ W3,
+                                 double* __restrict__ wnorm, double rest_scale) {
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int e = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
+  if (e < E) {
+    const float* w = W + static_cast<int64_t>(e) * H;
+    __nv_bfloat16* out = W3 + static_cast<int64_t>(e) * 3 * H;
+    double ss[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int v = lane; v < H / 4; v += 32) {
+      const Vec16<float> w4 = ld16(w + v * 4);
+      __nv_bfloat16 part[3][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float x0 = w4.v[j];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(x0);
+        const float r1 = __fsub_rn(x0, __bfloat162float(hi));
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const float r2 = __fsub_rn(r1, __bfloat162float(mid));
+        const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+        const double r3 = static_cast<double>(r2) - static_cast<double>(__bfloat162float(lo));
+        part[0][j] = hi;
+        part[1][j] = mid;
+        part[2][j] = lo;
+        const double dh = __bfloat162float(hi), dm = __bfloat162float(mid), dl = __bfloat162float(lo);
+        ss[0] = fma(dh, dh, ss[0]);
+        ss[1] = fma(dm, dm, ss[1]);
+        ss[2] = fma(dl, dl, ss[2]);
+        ss[3] = fma(r3, r3, ss[3]);
+      }
+#pragma unroll
+      for (int q = 0; q < 3; ++q)
+        *reinterpret_cast<uint2*>(out + static_cast<int64_t>(q) * H + v * 4) = *reinterpret_cast<const uint2*>(part[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss[q] += __shfl_xor_sync(0xffffffffu, ss[q], o);
+    if (lane == 0) {
+      double b = __dadd_ru(norm_ub_from_sumsq(ss[0], H), norm_ub_from_sumsq(ss[1], H));
+      b = __dadd_ru(b, norm_ub_from_sumsq(ss[2], H));
+      b = __dadd_ru(b, __dmul_ru(norm_ub_from_sumsq(ss[3], H), rest_scale));
+      wnorm[e] = b;
+    }
+  }
 }
 
 static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
   using bf16 = __nv_bfloat16;
   RouterTcParams p{};
+  const int Kg = a.w32 ? 3 * a.H : a.H;  // length of the GEMM's reduction
   p.T = a.T;
-  p.H = a.H;
+  p.H = Kg;
+  p.Hx = a.H;
   p.E = a.E;
+  p.w_given = a.w32 ? 1 : 0;
   p.scores = a.scores64;
   p.ctrl = a.ctrl;
+  const bf16* x = static_cast<const bf16*>(a.x);
+  const bf16* Wg = static_cast<const bf16*>(a.w32 ? a.w3 : a.Wr);  // the GEMM's B operand
   if (!encode_bf16_rows(&p.tmX, a.x, a.T, a.H, kRtRowBox) ||
-      !encode_bf16_rows(&p.tmW, a.Wr, a.E, a.H, kRtExperts))
+      !encode_bf16_rows(&p.tmW, Wg, a.E, Kg, kRtExperts))
     return cudaErrorInvalidValue;
   cudaError_t e = allow_smem(router_gemm_tc_kernel, kRtSmem);
   if (e != cudaSuccess) return e;
-  const bf16* x = static_cast<const bf16*>(a.x);
-  const bf16* Wr = static_cast<const bf16*>(a.Wr);
-  const int n_sl = (a.H / kTileK + kRtSliceSteps - 1) / kRtSliceSteps;
-  const int chunks = a.rsplit ? router_chunks(a.T, a.E, a.H) : 1;
+  // Each slice of L = 256 products is accumulated in fp32 from exact products, at most
+  // 2^-23 relative per accumulation step (truncation included), so its error is
+  // <= 2 L 2^-23 * sum|x w| over the slice; adding the K/L partials in fp64 costs at most
+  // 2 (K/L) 2^-53 more; K 2^-125 covers partial sums flushed below the normal range.
+  const double slice = static_cast<double>(kRtSliceSteps) * kTileK;
+  const double coef = 2.0 * slice * kU23 + 2.0 * (Kg / slice + 1) * kU53;
+  int launches = 2;
+  if (a.w32) {
+    e = launch_pdl(split_w32_kernel, dim3(static_cast<unsigned>((a.E * 32 + 255) / 256)), dim3(256), 0, st,
+                   static_cast<const float*>(a.Wr), a.E, a.H, static_cast<bf16*>(a.w3), a.wnorm,
+                   (1.0 / coef) * (1.0 + 0x1p-40));  // >= 1 / coef
+    if (e != cudaSuccess) return e;
+    ++launches;
+  }
+  const int n_sl = (Kg / kTileK + kRtSliceSteps - 1) / kRtSliceSteps;
+  const int chunks = a.rsplit ? router_chunks(a.T, a.E, Kg) : 1;
   p.chunks = chunks;
   p.chunk_slices = (n_sl + chunks - 1) / chunks;
-  int launches = 2;
   if (chunks > 1) {
     // the split blocks also produce the norm bounds
     double* d = static_cast<double*>(a.rsplit);
     p.x = x;
-    p.Wr = Wr;
+    p.Wr = Wg;
     p.xss = d;
     p.wss = d + static_cast<int64_t>(chunks) * a.T;
     p.part = reinterpret_cast<float*>(p.wss + static_cast<int64_t>(chunks) * a.E);
@@ -1282,37 +1410,42 @@ static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
     p.xnorm = a.xnorm;
     p.wnorm = a.wnorm;
   } else {
-    e = launch_pdl(row_norm_ub_kernel<bf16>, dim3(static_cast<unsigned>(((a.T + a.E) * 32 + 255) / 256)),
-                   dim3(256), 0, st, x, a.T, a.xnorm, Wr, static_cast<int64_t>(a.E), a.wnorm, a.H);
+    const int64_t wrows = a.w32 ? 0 : a.E;  // split fp32 weights come with their norm bounds
+    e = launch_pdl(row_norm_ub_kernel<bf16>, dim3(static_cast<unsigned>(((a.T + wrows) * 32 + 255) / 256)),
+                   dim3(256), 0, st, x, a.T, a.xnorm, Wg, wrows, a.wnorm, a.H);
     if (e != cudaSuccess) return e;
-    launches = 3;
+    ++launches;
   }
   e = launch_pdl(router_gemm_tc_kernel,
                  dim3(static_cast<unsigned>((a.T + kTileM - 1) / kTileM), (a.E + kRtExperts - 1) / kRtExperts,
                       static_cast<unsigned>(chunks)),
                  dim3(192), static_cast<size_t>(kRtSmem), st, p);
   if (e != cudaSuccess) return e;
-  // Each slice of L = 256 products is accumulated in fp32 from exact products, at most
-  // 2^-23 relative per accumulation step (truncation included), so its error is
-  // <= 2 L 2^-23 * sum|x w| over the slice; adding the H/L partials in fp64 costs at most
-  // 2 (H/L) 2^-53 more; H 2^-125 covers partial sums flushed below the normal range.
-  const double slice = static_cast<double>(kRtSliceSteps) * kTileK;
-  const double coef = 2.0 * slice * kU23 + 2.0 * (a.H / slice + 1) * kU53;
   const unsigned sgrid = static_cast<unsigned>((a.T + kSelectWarps - 1) / kSelectWarps);
-  auto sel = [&](auto kern) {
+  auto sel = [&](auto kern, auto* Wsel) {
     return launch_pdl(kern, dim3(sgrid), dim3(32 * kSelectWarps), 0, st, static_cast<const double*>(a.scores64),
-                      coef, a.H * 2.350988701644575e-38, static_cast<const double*>(a.xnorm),
-                      static_cast<const double*>(a.wnorm), Keys{a.bias, a.sigmoid, a.scale}, x, Wr, a.T, a.H,
+                      coef, Kg * 2.350988701644575e-38, static_cast<const double*>(a.xnorm),
+                      static_cast<const double*>(a.wnorm), Keys{a.bias, a.sigmoid, a.scale}, x, Wsel, a.T, a.H,
                       a.E, a.k, a.idx_ws,
                       a.w_ws, a.idx_user, a.w_user, a.spill, a.ctrl);
   };
   const int epl = select_epl(a.E);
-  if (a.sigmoid)
-    e = epl == 4 ? sel(route_select_kernel<bf16, 4, true>) : epl == 12 ? sel(route_select_kernel<bf16, 12, true>)
-                                                                      : sel(route_select_kernel<bf16, 32, true>);
-  else
-    e = epl == 4 ? sel(route_select_kernel<bf16, 4, false>) : epl == 12 ? sel(route_select_kernel<bf16, 12, false>)
-                                                                       : sel(route_select_kernel<bf16, 32, false>);
+  const bf16* Wb = static_cast<const bf16*>(a.Wr);
+  const float* Wf = static_cast<const float*>(a.Wr);
+  if (a.w32) {  // the recomputations read the fp32 weights themselves
+    if (a.sigmoid)
+      e = epl == 4 ? sel(route_select_kernel<bf16, float, 4, true>, Wf)
+          : epl == 12 ? sel(route_select_kernel<bf16, float, 12, true>, Wf) : sel(route_select_kernel<bf16, float, 32, true>, Wf);
+    else
+      e = epl == 4 ? sel(route_select_kernel<bf16, float, 4, false>, Wf)
+          : epl == 12 ? sel(route_select_kernel<bf16, float, 12, false>, Wf) : sel(route_select_kernel<bf16, float, 32, false>, Wf);
+  } else if (a.sigmoid) {
+    e = epl == 4 ? sel(route_select_kernel<bf16, bf16, 4, true>, Wb)
+        : epl == 12 ? sel(route_select_kernel<bf16, bf16, 12, true>, Wb) : sel(route_select_kernel<bf16, bf16, 32, true>, Wb);
+  } else {
+    e = epl == 4 ? sel(route_select_kernel<bf16, bf16, 4, false>, Wb)
+        : epl == 12 ? sel(route_select_kernel<bf16, bf16, 12, false>, Wb) : sel(route_select_kernel<bf16, bf16, 32, false>, Wb);
+  }
   count_launches(launches);
   return e;
 }

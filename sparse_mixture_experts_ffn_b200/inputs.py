@@ -92,14 +92,17 @@ def skew_bias(cfg: MoEConfig, beta: float = SKEW_BETA) -> torch.Tensor:
     return (beta * torch.log(z)).to(torch.float32)
 
 
-def make_routing_inputs(cfg: MoEConfig, beta: float | None = None):
-    """x [T,H], W_router [E,H] (working dtype) and router bias [E] fp32 or None, on the CPU."""
+def make_routing_inputs(cfg: MoEConfig, beta: float | None = None, router_fp32: bool = False):
+    """x [T,H], W_router [E,H] (working dtype; fp32 with router_fp32, the same draws unrounded)
+    and router bias [E] fp32 or None, on the CPU."""
     g = torch.Generator().manual_seed(cfg.seed)
     x = torch.randn(cfg.T, cfg.H, generator=g, dtype=torch.float32) * cfg.x_std
     if cfg.rms_norm:
         x = x * torch.rsqrt(x.pow(2).mean(dim=-1, keepdim=True) + 1e-6)
     x = x.to(cfg.torch_dtype)
-    Wr = (torch.randn(cfg.E, cfg.H, generator=g, dtype=torch.float32) * cfg.r_std).to(cfg.torch_dtype)
+    Wr = torch.randn(cfg.E, cfg.H, generator=g, dtype=torch.float32) * cfg.r_std
+    if not router_fp32:
+        Wr = Wr.to(cfg.torch_dtype)
     bias = skew_bias(cfg, SKEW_BETA if beta is None else beta) if cfg.skew else None
     return x, Wr, bias
 

@@ -109,6 +109,31 @@ def test_sigmoid_router(sz, with_bias):
     assert torch.allclose(r.topk_w.sum(1), torch.full((cfg.T,), 3.0, device=r.topk_w.device), rtol=1e-5)
 
 
+FP32_ROUTER_CASES = [
+    dict(T=257, H=256, E=32, top_k=4, I=128, I_shared=128),    # unsplit tensor-core scores
+    dict(T=3, H=2176, E=200, top_k=8, I=128, I_shared=128),    # reduction split over blocks
+]
+
+
+@pytest.mark.parametrize("router", ["softmax", "sigmoid"])
+@pytest.mark.parametrize("sz", FP32_ROUTER_CASES, ids=lambda s: "T{T}_H{H}_E{E}".format(**s))
+def test_fp32_router_weights(sz, router):
+    """bf16 layer with fp32 router weights (need_fp32_gate): the scores are the exact dots of
+    bf16 tokens and fp32 weights; indices bit-exact against the oracle."""
+    cfg = inputs.small_config(**sz)
+    d = inputs.make_inputs(cfg, "cuda")
+    g = torch.Generator().manual_seed(cfg.seed + 31)
+    d["W_router"] = torch.randn(cfg.E, cfg.H, generator=g) * cfg.r_std  # fp32, not bf16-rounded
+    if router == "sigmoid":
+        d["bias"] = torch.linspace(-0.1, 0.1, cfg.E, dtype=torch.float32)
+    d = to_device(d)
+    scale = 3.0 if router == "sigmoid" else 1.0
+    y, r = run(d, cfg.top_k, router=router, routed_scaling_factor=scale)
+    ref = oracle_routing(d, cfg.top_k, router=router, scale=scale)
+    assert_routing_exact(r, ref, cfg.E)
+    assert_y_close(y, oracle_y(d, ref), "fp32 router weights")
+
+
 def test_small_bf16_with_router_bias():
     cfg = inputs.small_config(T=257, H=256, E=32, top_k=4, I=128, I_shared=128)
     d = inputs.make_inputs(cfg, "cuda")
@@ -238,12 +263,15 @@ def test_full_size_workload(name):
 
 @pytest.mark.parametrize("name", ["decode_t4", "prefill_t16384_skew"])
 def test_full_size_layer_as_configured(name):
-    """The last layers as configured: sigmoid router with the routing factor 3 and a bias
-    for the selection, SwiGLU limits 7 (routed) and 16 (shared)."""
+    """The last layers as configured: fp32 router weights, sigmoid router with the routing
+    factor 3 and a bias for the selection, SwiGLU limits 7 (routed) and 16 (shared)."""
     cfg = inputs.CONFIGS[name]
     d = inputs.make_inputs(cfg, "cuda")
     if d.get("bias") is None:
         d["bias"] = torch.linspace(-0.05, 0.05, cfg.E, dtype=torch.float32)
+    # need_fp32_gate: fp32 router weights
+    g = torch.Generator().manual_seed(cfg.seed + 31)
+    d["W_router"] = torch.randn(cfg.E, cfg.H, generator=g) * cfg.r_std
     d = to_device(d)
     opts = dict(router="sigmoid", routed_scaling_factor=3.0, swiglu_limit=7.0, swiglu_limit_shared=16.0)
     shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared, cfg.top_k, torch.bfloat16)
