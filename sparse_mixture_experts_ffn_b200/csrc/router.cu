@@ -312,6 +312,18 @@ struct Keys {
     const float p = z < -80.0f ? 0x1p-115f : __fmul_ru(__fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-z))), 1.0f + 0x1p-20f);
     return bias ? __fadd_ru(p, bias[e]) : p;
   }
+  // The same ends for a refined (fp64) score, tight: the fp64 definition itself, widened by
+  // one ulp of p for its at most one-ulp departure from monotonicity.
+  __device__ __forceinline__ float key_lo_ref(double s_lo, int e) const {
+    if (!sigmoid) return key(s_lo, e);
+    const float p = nextafterf(sigmoid32(__double2float_rd(s_lo)), -INFINITY);
+    return bias ? __fadd_rd(p, bias[e]) : p;
+  }
+  __device__ __forceinline__ float key_hi_ref(double s_hi, int e) const {
+    if (!sigmoid) return key(s_hi, e);
+    const float p = nextafterf(sigmoid32(__double2float_ru(s_hi)), INFINITY);
+    return bias ? __fadd_ru(p, bias[e]) : p;
+  }
 };
 
 // a is ranked before b: larger key, then lower index
@@ -553,8 +565,8 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
         const double s64 = warp_dot_f64_prefetch(xt, Wr + static_cast<size_t>(e) * H, H);
         if (lane == src) {
           const double d = __dmul_ru(__dmul_ru(1.01 * H * kU53, nx), nw(e));
-          my_lo = kf.key_lo(__dadd_rd(s64, -d), e);
-          my_hi = kf.key_hi(__dadd_ru(s64, d), e);
+          my_lo = kf.key_lo_ref(__dadd_rd(s64, -d), e);
+          my_hi = kf.key_hi_ref(__dadd_ru(s64, d), e);
           my_mid = kf.key(s64, e);
           if (SIG) my_p = kf.score(s64);
           C.lo[lane] = my_lo;
@@ -714,8 +726,8 @@ __device__ __noinline__ void select_token_slow(const double* __restrict__ srow, 
         if (pass == 0) {
           const double s64 = warp_dot_f64_prefetch(xt, we, H);
           const double d = __dmul_ru(__dmul_ru(1.01 * H * kU53, nx), nw(e));
-          klo = kf.key_lo(__dadd_rd(s64, -d), e);
-          khi = kf.key_hi(__dadd_ru(s64, d), e);
+          klo = kf.key_lo_ref(__dadd_rd(s64, -d), e);
+          khi = kf.key_hi_ref(__dadd_ru(s64, d), e);
           kmid = kf.key(s64, e);
           kp = kf.score(s64);
           ++n_ref;
@@ -978,7 +990,7 @@ constexpr int kRtBBytes = kRtExperts * kTileK * 2;   // 8 KB of W_router
 constexpr int kRtStageBytes = kRtABytes + kRtBBytes;
 constexpr int kRtSmem = kRtStages * kRtStageBytes + 1024 + 256;
 constexpr int kRtRowBox = 16;                        // token rows per TMA box
-constexpr int kRtMaxChunks = 8;
+constexpr int kRtMaxChunks = 16;
 constexpr int kRtSmTarget = 148;                     // blocks that fill the GPU
 
 struct RouterTcParams {
@@ -1315,50 +1327,56 @@ size_t router_w3_bytes(const moe_layer_shape& s) {
 // goes into the norm bound).  One warp per expert row also bounds the row's norm for the
 // selection: ||hi|| + ||mid|| + ||lo|| (all products of the split counted), plus the
 // unrepresented rest scaled by 1/coef, so that coef * |x| * bound still covers it.
-__global__ void split_w32_kernel(const float* __restrict__ W, int E, int H, __nv_bfloat16* __restrict__ W3,
-                                 double* __restrict__ wnorm, double rest_scale) {
+__global__ void __launch_bounds__(256) split_w32_kernel(const float* __restrict__ W, int E, int H,
+                                                         __nv_bfloat16* __restrict__ W3,
+                                                         double* __restrict__ wnorm, double rest_scale) {
+  __shared__ double red[8][4];
   pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int e = static_cast<int>((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5);
-  if (e < E) {
-    const float* w = W + static_cast<int64_t>(e) * H;
-    __nv_bfloat16* out = W3 + static_cast<int64_t>(e) * 3 * H;
-    double ss[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int v = lane; v < H / 4; v += 32) {
-      const Vec16<float> w4 = ld16(w + v * 4);
-      __nv_bfloat16 part[3][4];
+  const int e = blockIdx.x;  // one block per expert row, four floats per thread and step
+  const float* w = W + static_cast<int64_t>(e) * H;
+  __nv_bfloat16* out = W3 + static_cast<int64_t>(e) * 3 * H;
+  double ss[4] = {0.0, 0.0, 0.0, 0.0};
+  for (int v = threadIdx.x; v < H / 4; v += blockDim.x) {
+    const Vec16<float> w4 = ld16(w + v * 4);
+    __nv_bfloat16 part[3][4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float x0 = w4.v[j];
-        const __nv_bfloat16 hi = __float2bfloat16_rn(x0);
-        const float r1 = __fsub_rn(x0, __bfloat162float(hi));
-        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-        const float r2 = __fsub_rn(r1, __bfloat162float(mid));
-        const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
-        const double r3 = static_cast<double>(r2) - static_cast<double>(__bfloat162float(lo));
-        part[0][j] = hi;
-        part[1][j] = mid;
-        part[2][j] = lo;
-        const double dh = __bfloat162float(hi), dm = __bfloat162float(mid), dl = __bfloat162float(lo);
-        ss[0] = fma(dh, dh, ss[0]);
-        ss[1] = fma(dm, dm, ss[1]);
-        ss[2] = fma(dl, dl, ss[2]);
-        ss[3] = fma(r3, r3, ss[3]);
-      }
-#pragma unroll
-      for (int q = 0; q < 3; ++q)
-        *reinterpret_cast<uint2*>(out + static_cast<int64_t>(q) * H + v * 4) = *reinterpret_cast<const uint2*>(part[q]);
+    for (int j = 0; j < 4; ++j) {
+      const float x0 = w4.v[j];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x0);
+      const float r1 = __fsub_rn(x0, __bfloat162float(hi));
+      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+      const float r2 = __fsub_rn(r1, __bfloat162float(mid));
+      const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+      const double r3 = static_cast<double>(r2) - static_cast<double>(__bfloat162float(lo));
+      part[0][j] = hi;
+      part[1][j] = mid;
+      part[2][j] = lo;
+      const double dh = __bfloat162float(hi), dm = __bfloat162float(mid), dl = __bfloat162float(lo);
+      ss[0] = fma(dh, dh, ss[0]);
+      ss[1] = fma(dm, dm, ss[1]);
+      ss[2] = fma(dl, dl, ss[2]);
+      ss[3] = fma(r3, r3, ss[3]);
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
+    for (int q = 0; q < 3; ++q)
+      *reinterpret_cast<uint2*>(out + static_cast<int64_t>(q) * H + v * 4) = *reinterpret_cast<const uint2*>(part[q]);
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss[q] += __shfl_xor_sync(0xffffffffu, ss[q], o);
-    if (lane == 0) {
-      double b = __dadd_ru(norm_ub_from_sumsq(ss[0], H), norm_ub_from_sumsq(ss[1], H));
-      b = __dadd_ru(b, norm_ub_from_sumsq(ss[2], H));
-      b = __dadd_ru(b, __dmul_ru(norm_ub_from_sumsq(ss[3], H), rest_scale));
-      wnorm[e] = b;
-    }
+  for (int q = 0; q < 4; ++q) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss[q] += __shfl_xor_sync(0xffffffffu, ss[q], o);
+    if (lane == 0) red[warp][q] = ss[q];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int w8 = 0; w8 < static_cast<int>(blockDim.x >> 5); ++w8)
+      for (int q = 0; q < 4; ++q) t[q] += red[w8][q];
+    double b = __dadd_ru(norm_ub_from_sumsq(t[0], H), norm_ub_from_sumsq(t[1], H));
+    b = __dadd_ru(b, norm_ub_from_sumsq(t[2], H));
+    b = __dadd_ru(b, __dmul_ru(norm_ub_from_sumsq(t[3], H), rest_scale));
+    wnorm[e] = b;
   }
 }
 
@@ -1388,7 +1406,7 @@ static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
   const double coef = 2.0 * slice * kU23 + 2.0 * (Kg / slice + 1) * kU53;
   int launches = 2;
   if (a.w32) {
-    e = launch_pdl(split_w32_kernel, dim3(static_cast<unsigned>((a.E * 32 + 255) / 256)), dim3(256), 0, st,
+    e = launch_pdl(split_w32_kernel, dim3(static_cast<unsigned>(a.E)), dim3(256), 0, st,
                    static_cast<const float*>(a.Wr), a.E, a.H, static_cast<bf16*>(a.w3), a.wnorm,
                    (1.0 / coef) * (1.0 + 0x1p-40));  // >= 1 / coef
     if (e != cudaSuccess) return e;
