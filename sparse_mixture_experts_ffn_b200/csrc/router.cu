@@ -1286,14 +1286,14 @@ int router_slice_len(int /*H*/) { return kRtSliceSteps * kTileK; }
 
 // Reduction chunks of the tensor-core router: 1 when the (m, n) tiles fill the GPU or the
 // batch is too large for one block per tile to add the partials quickly, else the fewest
-// (at most 8, at least two slices each) that bring the blocks to one per SM.
+// (at most 16, at least one slice each) that bring the blocks to one per SM.
 constexpr int64_t kRtSplitMaxTokens = 32;
 static int router_chunks(int64_t T, int E, int H) {
   if (T > kRtSplitMaxTokens) return 1;
   const int64_t tiles = ((T + kTileM - 1) / kTileM) * ((E + kRtExperts - 1) / kRtExperts);
   const int n_sl = (H / kTileK + kRtSliceSteps - 1) / kRtSliceSteps;
   int c = 1;
-  while (c < kRtMaxChunks && tiles * c < kRtSmTarget && 4 * c <= n_sl) c *= 2;
+  while (c < kRtMaxChunks && tiles * c < kRtSmTarget && 2 * c <= n_sl) c *= 2;
   if (c == 1) return 1;
   const int per = (n_sl + c - 1) / c;
   return (n_sl + per - 1) / per;
