@@ -420,11 +420,15 @@ def main():
         e2e_value = job_tokens_per_s(cfg.T, world, e_steps, e2e_ms)
         gu_ms = stage_ms["gate_up"] / max(calls, 1)
         dn_ms = stage_ms["down"] / max(calls, 1)
-        tensor_bound = alg["gate_up_flops"] / (peaks["bf16_tflops"] * 1e12) > alg["gate_up_bytes"] / (peaks["hbm_gbs"] * 1e9)
+        # the GEMM is timed inside the long step loop, where the part runs at its power cap:
+        # the sustained bf16 figure is its tensor-core peak
+        tc_peak = peaks["bf16_tflops_sustained"]
+        tensor_bound = alg["gate_up_flops"] / (tc_peak * 1e12) > alg["gate_up_bytes"] / (peaks["hbm_gbs"] * 1e9)
         if tensor_bound:
             achieved = alg["gate_up_flops"] / (gu_ms / 1e3) / 1e12
-            roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": achieved / peaks["bf16_tflops"]}
+            roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                    "frac": achieved / tc_peak, "peak_kind": "sustained bf16 (cuBLAS, seconds-long loop)",
+                    "frac_of_burst": achieved / peaks["bf16_tflops"]}
         else:
             achieved = alg["gate_up_bytes"] / (gu_ms / 1e3) / 1e9
             roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
