@@ -142,7 +142,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctrl* 
 }
 
 // ---------------------------------------------------------------------------------------
-// TMA (cp.async.bulk.tensor), no multicast
+// TMA (cp.async.bulk.tensor), each copy into this CTA's own shared memory
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t c0,
                                             int32_t c1, uint64_t* bar) {
