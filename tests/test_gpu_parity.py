@@ -134,6 +134,30 @@ def test_fp32_router_weights(sz, router):
     assert_y_close(y, oracle_y(d, ref), "fp32 router weights")
 
 
+EDGE_CASES = [
+    dict(T=40, H=256, E=1024, top_k=8, I=128, I_shared=128),   # the most experts: fp64 router kernel
+    dict(T=33, H=256, E=513, top_k=4, I=128, I_shared=0),      # one past the tensor-core router
+    dict(T=33, H=256, E=512, top_k=4, I=128, I_shared=128),    # the largest tensor-core router
+    dict(T=50, H=256, E=1, top_k=1, I=128, I_shared=128),      # a single expert
+    dict(T=3, H=512, E=16, top_k=4, I=256, I_shared=0),        # split decode GEMM, no shared expert
+]
+
+
+@pytest.mark.parametrize("router", ["softmax", "sigmoid"])
+@pytest.mark.parametrize("sz", EDGE_CASES, ids=lambda s: "T{T}_E{E}_k{top_k}_Is{I_shared}".format(**s))
+def test_edge_shapes(sz, router):
+    cfg = inputs.small_config(**sz)
+    d = to_device(inputs.make_inputs(cfg, "cuda", shared=sz["I_shared"] > 0))
+    scale = 3.0 if router == "sigmoid" else 1.0
+    shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared, cfg.top_k, torch.bfloat16)
+    ws = moe.alloc_workspace(shape, "cuda")
+    y, r = run(d, cfg.top_k, workspace=ws, router=router, routed_scaling_factor=scale)
+    assert moe.check_status(ws) == moe.MOE_OK
+    ref = oracle_routing(d, cfg.top_k, router=router, scale=scale)
+    assert_routing_exact(r, ref, cfg.E)
+    assert_y_close(y, oracle_y(d, ref), f"edge {sz} {router}")
+
+
 def test_small_bf16_with_router_bias():
     cfg = inputs.small_config(T=257, H=256, E=32, top_k=4, I=128, I_shared=128)
     d = inputs.make_inputs(cfg, "cuda")
