@@ -304,7 +304,8 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
     place_assignments(idx, w, 0, P, k, E, base, perm, inv_perm, row_w, row_tok, perm_user);
 }
 
-// x_perm[pos, :] = x[row_tok[pos], :], 16-byte vectors
+// x_perm[pos, :] = x[row_tok[pos], :], 16-byte vectors: one warp per row at a time (no
+// per-vector index arithmetic), four vectors in flight per lane
 template <typename T>
 __global__ void gather_rows_kernel(const T* __restrict__ x, const int32_t* __restrict__ row_tok,
                                    int64_t P, int64_t Tn, int H, T* __restrict__ x_perm,
@@ -313,18 +314,25 @@ __global__ void gather_rows_kernel(const T* __restrict__ x, const int32_t* __res
   pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
   constexpr int V = Vec16<T>::N;
   const int vpr = H / V;
-  const int64_t total = P * vpr;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t p = i / vpr;
-    const int v = static_cast<int>(i - p * vpr);
-    const int64_t t = row_tok[p];
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t p = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; p < P; p += warps) {
+    const int64_t t = __ldg(row_tok + p);
     if (t < 0 || t >= Tn) {
-      set_status(ctrl, MOE_ERR_DEVICE_BOUNDS);
+      if (lane == 0) set_status(ctrl, MOE_ERR_DEVICE_BOUNDS);
       continue;
     }
-    const uint4 val = __ldg(reinterpret_cast<const uint4*>(x + t * H) + v);
-    reinterpret_cast<uint4*>(x_perm + p * H)[v] = val;
+    const uint4* src = reinterpret_cast<const uint4*>(x + t * H);
+    uint4* dst = reinterpret_cast<uint4*>(x_perm + p * H);
+    int v = lane;
+    for (; v + 96 < vpr; v += 128) {
+      uint4 r[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) r[u] = __ldg(src + v + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) dst[v + 32 * u] = r[u];
+    }
+    for (; v < vpr; v += 32) dst[v] = __ldg(src + v);
   }
 }
 
@@ -383,8 +391,7 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st) {
     count_launches(launches);
     return cudaSuccess;
   }
-  const int64_t vec = P * (a.H / (a.bf16 ? 8 : 4));
-  const int blocks = static_cast<int>(std::min<int64_t>((vec + 255) / 256, 148 * 16));
+  const int blocks = static_cast<int>(std::min<int64_t>((P + 7) / 8, 148 * 16));  // a warp per row
   if (a.bf16)
     e = launch_pdl(gather_rows_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st,
                    static_cast<const __nv_bfloat16*>(a.x), static_cast<const int32_t*>(a.row_tok), P,
