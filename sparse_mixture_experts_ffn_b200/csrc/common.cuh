@@ -67,8 +67,8 @@ __device__ __forceinline__ Vec16<T> ld16(const T* p) {
 // kernel launch early: the dispatch, expert GEMM and combine kernels call it right after
 // pdl_wait(), so the next kernel's blocks are placed and run their prologue (barriers,
 // tensor memory, descriptor prefetch) while this one works, then wait in pdl_wait() for it
-// to finish.  The routing kernels and the single-block dispatch do not call it (their
-// dependents launch when they exit), which measured faster for the short decode chain.
+// to finish.  The routing kernels do not call it (their dependents launch when they exit),
+// which measured faster for the short decode chain.
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {

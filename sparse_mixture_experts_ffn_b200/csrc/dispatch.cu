@@ -277,6 +277,7 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
   __shared__ int base[1024];
   __shared__ int warp_tot[33];
   pdl_wait();
+  pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
   const int E = sa.E;
   const int64_t P = sa.T * k;
   for (int e = threadIdx.x; e < E + 1; e += blockDim.x) cnt[e] = 0;
