@@ -5,7 +5,9 @@
 
 One step = one full forward of the layer (routing, dispatch, both grouped expert GEMMs,
 combine) over one batch of synthetic tokens with all inputs resident in HBM.  The L2 is
-flushed (a 2x-L2 write) before every timed step, outside the timed events.  Each step is
+flushed before every timed step, outside the timed events: a 2x-L2 write, then a 2x-L2 read,
+so that the write-back of the flush's own dirty lines also happens outside the events (it
+would otherwise land in the step: 15 us of a 226 us decode step).  Each step is
 timed with CUDA events on the launching stream; the sum over K steps, max over ranks,
 gives ``value`` = tokens of all ranks / time.  ``e2e`` repeats the measurement through the
 public API with the step's tokens copied from pinned host memory and the output read
@@ -334,7 +336,14 @@ def main():
     ws = moe.alloc_workspace(shape, dev)
     y = torch.empty_like(x)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(flush_w.numel() // 4, dtype=torch.int32, device=dev)
+    flush_sink = torch.zeros(1, dtype=torch.int64, device=dev)
+
+    def flush():
+        # evict everything, then leave the L2 holding clean lines of an unrelated buffer
+        flush_w.zero_()
+        flush_sink.add_(flush_r.sum())
     stream = torch.cuda.current_stream(dev)
 
     def step(xin, yout, routing=False):
@@ -352,7 +361,7 @@ def main():
     alg = algorithmic(cfg, counts)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step(x, y)
     torch.cuda.synchronize()
 
@@ -368,7 +377,7 @@ def main():
         launches0 = moe.launch_count()
         with ClockSampler(local) as clocks:
             for i in range(args.steps):
-                flush.zero_()
+                flush()
                 starts[i].record(stream)
                 step(x, y)
                 ends[i].record(stream)
@@ -402,7 +411,7 @@ def main():
     if pg:
         pg.barrier()
     for i in range(e_steps):
-        flush.zero_()
+        flush()
         es_[i].record(stream)
         x_dev.copy_(x_host, non_blocking=True)
         step(x_dev, y)
@@ -447,7 +456,7 @@ def main():
             "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "top_k": cfg.top_k,
                        "I": cfg.I, "I_shared": cfg.I_shared, "tokens_per_gpu": cfg.T,
                        **config_options(args),
-                       "l2": "flushed before every timed step (2x L2 write, outside the events)",
+                       "l2": "flushed before every timed step, outside the events: 2x L2 write, then 2x L2 read",
                        "parallelism": f"replicas x{world}"},
             "roofline": roof,
             "layer": {"touched_experts": alg["touched"], "algorithmic_bytes": alg["layer_bytes"],
