@@ -13,7 +13,10 @@ moe_intermediate_size, share_expert_dim; "FFN / MoE" paragraph of the same page)
 * key[t,e]      = fp32(s[t,e] + b[e]) with an optional router bias b;
 * selection     = the top_k keys, ties toward the lower expert index, stored ascending;
 * weights       = softmax over the selected keys (renormalised to sum to 1), fp64;
-* output        y_t = sum_j w_j SiLU(x W_g^T) * (x W_u^T) W_d^T + shared expert, fp64.
+* output        y_t = sum_j w_j SiLU(x W_g^T) * (x W_u^T) W_d^T + shared expert, fp64;
+* FP8 weights   (the low-precision expert weights for decode) E4M3 codes with one E8M0
+                power-of-two scale per 128 x 128 block, decoded exactly (``dequant_e4m3``,
+                ``moe_tokens_fp8``).
 
 bf16 arrays are passed as ``numpy.uint16`` bit patterns; fp32 as ``numpy.float32``.
 """
@@ -68,10 +71,14 @@ def _load():
         lib.oracle_moe_tokens.argtypes = [ctypes.c_int, ctypes.c_int64, P, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, P, P,
                                           P, D, D, P, ctypes.c_int]
+        lib.oracle_dequant_e4m3.argtypes = [ctypes.c_int64, ctypes.c_int, P, P, P]
+        lib.oracle_moe_tokens_fp8.argtypes = [ctypes.c_int64, P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, P, P, P, P, P, P, P, P, P, P, P,
+                                              D, D, P, ctypes.c_int]
         for f in (lib.oracle_exact_dot, lib.oracle_router_scores, lib.oracle_route,
                   lib.oracle_dispatch, lib.oracle_expert_act, lib.oracle_moe_tokens,
                   lib.oracle_route_mode, lib.oracle_sigmoid32, lib.oracle_exact_dot_mixed,
-                  lib.oracle_router_scores_mixed):
+                  lib.oracle_router_scores_mixed, lib.oracle_dequant_e4m3, lib.oracle_moe_tokens_fp8):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -205,6 +212,58 @@ def moe_tokens(x, idx, w64, Wgu, Wd, Wsgu=None, Wsd=None, tokens=None, nthreads:
                                    _p(y), nthreads or nthreads_default())
     if rc != 0:
         raise ValueError("moe_tokens: expert index out of range")
+    return y
+
+
+def fp8_scale_shape(R: int, K: int):
+    """Shape of the scale table of an FP8 weight matrix [R, K]: one scale per 128 x 128 block."""
+    return ((R + 127) // 128, (K + 127) // 128)
+
+
+def dequant_e4m3(q: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """The fp64 weights [R, K] that FP8 E4M3 codes q [R, K] (uint8) with E8M0 block scales
+    s [ceil(R/128), ceil(K/128)] (uint8) stand for: e4m3(q[r, c]) * 2^(s[r//128, c//128] - 127)."""
+    q, s = _c(q, np.uint8), _c(s, np.uint8)
+    R, K = q.shape
+    assert s.shape == fp8_scale_shape(R, K)
+    out = np.empty((R, K), np.float64)
+    _load().oracle_dequant_e4m3(R, K, _p(q), _p(s), _p(out))
+    return out
+
+
+def moe_tokens_fp8(x, idx, w64, Wgu, Wd, Wsgu=None, Wsd=None, tokens=None, nthreads: int = 0,
+                   swiglu_limit: float = 0.0, swiglu_limit_shared: float = 0.0):
+    """moe_tokens with bf16 tokens and FP8 expert weights.  Each weight argument is a pair
+    (codes uint8, scales uint8): Wgu ([E, 2I, H], [E, ceil(2I/128), ceil(H/128)]),
+    Wd ([E, H, I], [E, ceil(H/128), ceil(I/128)]), Wsgu ([2Is, H], ...), Wsd ([H, Is], ...)."""
+    x = _c(x)
+    assert x.dtype == np.uint16, "tokens are bf16 bit patterns"
+    (gq, gs), (dq, ds) = Wgu, Wd
+    gq, gs, dq, ds = (_c(a, np.uint8) for a in (gq, gs, dq, ds))
+    T, H = x.shape
+    E, twoI, H2 = gq.shape
+    I = twoI // 2
+    assert H2 == H and dq.shape == (E, H, I)
+    assert gs.shape == (E,) + fp8_scale_shape(twoI, H) and ds.shape == (E,) + fp8_scale_shape(H, I)
+    sgq = sgs = sdq = sds = None
+    Is = 0
+    if Wsgu is not None:
+        (sgq, sgs), (sdq, sds) = Wsgu, Wsd
+        sgq, sgs, sdq, sds = (_c(a, np.uint8) for a in (sgq, sgs, sdq, sds))
+        Is = sgq.shape[0] // 2
+        assert sgq.shape == (2 * Is, H) and sdq.shape == (H, Is)
+        assert sgs.shape == fp8_scale_shape(2 * Is, H) and sds.shape == fp8_scale_shape(H, Is)
+    idx = _c(idx, np.int32)
+    w64 = _c(w64, np.float64)
+    k = idx.shape[1]
+    tok = np.arange(T, dtype=np.int64) if tokens is None else _c(np.asarray(tokens), np.int64)
+    y = np.empty((tok.shape[0], H), np.float64)
+    rc = _load().oracle_moe_tokens_fp8(tok.shape[0], _p(tok), H, E, k, I, Is, _p(x), _p(idx), _p(w64),
+                                       _p(gq), _p(gs), _p(dq), _p(ds), _p(sgq), _p(sgs), _p(sdq), _p(sds),
+                                       float(swiglu_limit), float(swiglu_limit_shared), _p(y),
+                                       nthreads or nthreads_default())
+    if rc != 0:
+        raise ValueError("moe_tokens_fp8: expert index out of range")
     return y
 
 

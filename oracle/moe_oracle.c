@@ -449,6 +449,126 @@ int oracle_expert_act(int dtype, int H, int I, const void* xrow, const void* Wgu
 }
 
 /* ------------------------------------------------------------------------------------
+ * Blockwise FP8 expert weights (the low-precision expert weights for decode).
+ *
+ * A weight matrix W [R, K] is stored as one byte per element, an FP8 E4M3 code, plus one
+ * scale byte per 128 x 128 block, an E8M0 power of two; the weight it stands for is
+ *   W[r, c] = e4m3(q[r, c]) * e8m0(s[r / 128, c / 128]),  s laid out [ceil(R/128), ceil(K/128)].
+ * Formats (OCP 8-bit floating point and microscaling formats):
+ *   E4M3: sign, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 holds the
+ *         subnormals m/8 * 2^-6; no infinities; S.1111.111 is NaN; largest finite 448;
+ *   E8M0: an unsigned biased exponent, 2^(v - 127); v = 255 is NaN.
+ * Every such product is exact in fp64.  The layer is then the same gated FFNs on these
+ * weights (the tokens stay bf16), in fp64 as above.
+ * ---------------------------------------------------------------------------------- */
+static double decode_e4m3(uint8_t c) {
+  int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = ldexp((double)m, -9); /* m/8 * 2^-6 */
+  else
+    v = ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+  return sgn ? -v : v;
+}
+
+static double decode_e8m0(uint8_t v) { return v == 255 ? NAN : ldexp(1.0, (int)v - 127); }
+
+/* the two decodings of every byte, filled once (before any parallel region) */
+static double e4m3_val[256], e8m0_val[256];
+static int fp8_tables_ready = 0;
+static void fp8_tables(void) {
+  if (fp8_tables_ready) return;
+  for (int c = 0; c < 256; ++c) {
+    e4m3_val[c] = decode_e4m3((uint8_t)c);
+    e8m0_val[c] = decode_e8m0((uint8_t)c);
+  }
+  fp8_tables_ready = 1;
+}
+
+typedef struct {
+  const uint8_t* q; /* [R, K] codes */
+  const uint8_t* s; /* [ceil(R/128), ceil(K/128)] scales */
+  int K;
+} fp8_mat;
+
+static double fp8_at(fp8_mat w, size_t r, int c) {
+  int kb = (w.K + 127) / 128;
+  return e4m3_val[w.q[r * (size_t)w.K + c]] * e8m0_val[w.s[(r / 128) * (size_t)kb + c / 128]];
+}
+
+int oracle_dequant_e4m3(int64_t R, int K, const uint8_t* q, const uint8_t* s, double* out) {
+  fp8_mat w = {q, s, K};
+  fp8_tables();
+  for (int64_t r = 0; r < R; ++r)
+    for (int c = 0; c < K; ++c) out[r * (int64_t)K + c] = fp8_at(w, (size_t)r, c);
+  return 0;
+}
+
+/* gated_ffn_acc with FP8 weights: gu is [2I, H] (gate rows, then up rows), d is [H, I] */
+static void gated_ffn_acc_fp8(int H, int I, const uint16_t* xrow, fp8_mat gu, fp8_mat d, double scale,
+                              double limit, double* out, double* a /*[I]*/) {
+  for (int i = 0; i < I; ++i) {
+    double g = 0.0, u = 0.0;
+    for (int h = 0; h < H; ++h) {
+      double xv = to_f64(OR_BF16, xrow, h);
+      g += xv * fp8_at(gu, (size_t)i, h);
+      u += xv * fp8_at(gu, (size_t)(I + i), h);
+    }
+    a[i] = swiglu(g, u, limit);
+  }
+  for (int h = 0; h < H; ++h) {
+    double o = 0.0;
+    for (int i = 0; i < I; ++i) o += a[i] * fp8_at(d, (size_t)h, i);
+    out[h] += scale * o;
+  }
+}
+
+/* oracle_moe_tokens with bf16 tokens and FP8 weights.  Per routed expert e the codes are
+   Wgu_q[e] [2I, H] and Wd_q[e] [H, I]; the scale tables are Wgu_s[e] [ceil(2I/128),
+   ceil(H/128)] and Wd_s[e] [ceil(H/128), ceil(I/128)], stacked by expert like the codes. */
+int oracle_moe_tokens_fp8(int64_t ntok, const int64_t* tok, int H, int E, int k, int I, int Is,
+                          const uint16_t* x, const int32_t* idx, const double* w,
+                          const uint8_t* Wgu_q, const uint8_t* Wgu_s, const uint8_t* Wd_q,
+                          const uint8_t* Wd_s, const uint8_t* Wsgu_q, const uint8_t* Wsgu_s,
+                          const uint8_t* Wsd_q, const uint8_t* Wsd_s, double limit,
+                          double limit_shared, double* y, int nthreads) {
+  const size_t gu_sc = (size_t)((2 * I + 127) / 128) * ((H + 127) / 128);
+  const size_t d_sc = (size_t)((H + 127) / 128) * ((I + 127) / 128);
+  int bad = 0;
+  fp8_tables();
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+  for (int64_t n = 0; n < ntok; ++n) {
+    int64_t t = tok[n];
+    const uint16_t* xr = x + (size_t)t * H;
+    double* out = y + (size_t)n * H;
+    int Imax = I > Is ? I : Is;
+    double* a = (double*)malloc(sizeof(double) * (Imax > 0 ? Imax : 1));
+    for (int h = 0; h < H; ++h) out[h] = 0.0;
+    for (int j = 0; j < k; ++j) {
+      int e = idx[t * k + j];
+      if (e < 0 || e >= E) {
+        bad |= 1;
+        continue;
+      }
+      fp8_mat gu = {Wgu_q + (size_t)e * 2 * I * H, Wgu_s + (size_t)e * gu_sc, H};
+      fp8_mat d = {Wd_q + (size_t)e * H * I, Wd_s + (size_t)e * d_sc, I};
+      gated_ffn_acc_fp8(H, I, xr, gu, d, w[t * k + j], limit, out, a);
+    }
+    if (Wsgu_q && Wsd_q && Is > 0) {
+      fp8_mat gu = {Wsgu_q, Wsgu_s, H};
+      fp8_mat d = {Wsd_q, Wsd_s, Is};
+      gated_ffn_acc_fp8(H, Is, xr, gu, d, 1.0, limit_shared, out, a);
+    }
+    free(a);
+  }
+  return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------------------
  * Layer output for a list of tokens, given their routing:
  *   y_t = sum_j w[t,j] * FFN_{idx[t,j]}(x_t) + FFN_shared(x_t)      (fp64)
  * The shared expert (share_expert_dim) is always on with weight 1; pass NULL shared

@@ -127,6 +127,51 @@ def make_expert_weights(cfg: MoEConfig, device="cpu", shared: bool = True):
     return Wgu, Wd, Wsgu, Wsd
 
 
+FP8_BLOCK = 128  # one E8M0 scale per 128 x 128 block of an FP8 weight matrix
+
+
+def fp8_blockwise(w: torch.Tensor):
+    """(codes uint8 [R, K], scales uint8 [ceil(R/128), ceil(K/128)]) of a weight matrix in the
+    blockwise FP8 format: E4M3 codes by torch's own cast, and per block the E8M0 scale
+    2^ceil(log2(amax / 448)) that brings the block's largest magnitude within E4M3's range."""
+    R, K = w.shape
+    rb, kb = -(-R // FP8_BLOCK), -(-K // FP8_BLOCK)
+    wf = torch.zeros(rb * FP8_BLOCK, kb * FP8_BLOCK, dtype=torch.float32, device=w.device)
+    wf[:R, :K] = w.float()
+    blocks = wf.view(rb, FP8_BLOCK, kb, FP8_BLOCK)
+    amax = blocks.abs().amax(dim=(1, 3)).clamp_min(2.0 ** -100)
+    exp = torch.ceil(torch.log2(amax / 448.0)).clamp(-127, 127)
+    scaled = blocks * torch.exp2(-exp)[:, None, :, None]
+    codes = scaled.view(rb * FP8_BLOCK, kb * FP8_BLOCK)[:R, :K].to(torch.float8_e4m3fn)
+    return codes.view(torch.uint8).contiguous(), (exp + 127).to(torch.uint8).contiguous()
+
+
+def make_fp8_expert_weights(cfg: MoEConfig, device="cpu", shared: bool = True):
+    """The expert weights of ``make_expert_weights`` (same draws) in the blockwise FP8 format:
+    a dict of (codes, scales) pairs W_gate_up ([E,2I,H], [E,ceil(2I/128),ceil(H/128)]),
+    W_down ([E,H,I], [E,ceil(H/128),ceil(I/128)]) and, with ``shared``, Ws_gate_up and
+    Ws_down.  Drawn and converted one expert at a time."""
+    device = torch.device(device)
+    g = torch.Generator(device=device).manual_seed(cfg.seed + 7919)
+    E, H, I, Is = cfg.E, cfg.H, cfg.I, cfg.I_shared
+    dt = cfg.torch_dtype
+
+    def stack(rows, cols):
+        q = torch.empty(E, rows, cols, dtype=torch.uint8, device=device)
+        s = torch.empty(E, -(-rows // FP8_BLOCK), -(-cols // FP8_BLOCK), dtype=torch.uint8, device=device)
+        for e in range(E):
+            q[e], s[e] = fp8_blockwise((torch.randn(rows, cols, generator=g, device=device) * cfg.w_std).to(dt))
+        return q, s
+
+    out = {"W_gate_up": stack(2 * I, H), "W_down": stack(H, I)}
+    if shared:
+        out["Ws_gate_up"] = fp8_blockwise((torch.randn(2 * Is, H, generator=g, device=device) * cfg.w_std).to(dt))
+        out["Ws_down"] = fp8_blockwise((torch.randn(H, Is, generator=g, device=device) * cfg.w_std).to(dt))
+    else:
+        out["Ws_gate_up"] = out["Ws_down"] = None
+    return out
+
+
 def make_inputs(cfg: MoEConfig, device="cpu", shared: bool = True):
     """All inputs of one workload as a dict of tensors on ``device``."""
     x, Wr, bias = make_routing_inputs(cfg)

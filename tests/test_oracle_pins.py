@@ -524,3 +524,94 @@ def test_sigmoid_router_weights_use_scores_not_keys():
     # without the bias the same scores pick the three best p
     idx2, _, w2 = oracle.route(s, k, None, router="sigmoid", scale=3.0)
     assert idx2[0].tolist() == [1, 2, 6] and abs(w2[0].sum() - 3.0) < 1e-14
+
+
+# --------------------------------------------------------------------------------------
+# blockwise FP8 expert weights: E4M3 codes, one E8M0 scale per 128 x 128 block
+# --------------------------------------------------------------------------------------
+def torch_e4m3(codes: np.ndarray) -> np.ndarray:
+    """Library decoding of E4M3 codes (torch.float8_e4m3fn) to fp64."""
+    return torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e4m3fn).double().numpy()
+
+
+def torch_e8m0(codes: np.ndarray) -> np.ndarray:
+    """Library decoding of E8M0 scale codes (torch.float8_e8m0fnu) to fp64."""
+    return torch.from_numpy(np.ascontiguousarray(codes, np.uint8)).view(torch.float8_e8m0fnu).double().numpy()
+
+
+def test_e4m3_decoding_of_all_codes_matches_the_library():
+    q = np.arange(256, dtype=np.uint8).reshape(2, 128)
+    got = oracle.dequant_e4m3(q, np.full((1, 1), 127, np.uint8))  # scale 2^0
+    ref = torch_e4m3(q)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan) and nan.sum() == 2  # S.1111.111 only
+    assert np.array_equal(got[~nan], ref[~nan])
+    # landmarks of the format: 1.0, the largest finite value, the smallest subnormal, -0
+    assert got[0, 0x38] == 1.0 and got[0, 0x7E] == 448.0 and got[0, 0x01] == 2.0 ** -9
+    assert got[1, 0] == 0.0 and math.copysign(1.0, got[1, 0]) == -1.0
+
+
+def test_e8m0_scales_match_the_library():
+    v = np.arange(255, dtype=np.uint8)
+    q = np.full((1, 255 * 128), 0x38, np.uint8)  # every weight 1.0, one block per scale
+    got = oracle.dequant_e4m3(q, v.reshape(1, 255))[0, ::128]
+    assert np.array_equal(got, torch_e8m0(v))
+    assert got[127] == 1.0 and got[0] == 2.0 ** -127
+
+
+def test_fp8_block_scales_index_row_and_column_blocks():
+    """Ragged 3 x 4 block grid, a different scale per block: the decoded matrix must equal the
+    library decoding of each code times its own block's scale, built by block expansion."""
+    rng = np.random.default_rng(7)
+    R, K = 320, 448
+    q = rng.integers(0, 256, size=(R, K), dtype=np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0x3C  # no NaN codes
+    s = rng.integers(100, 150, size=oracle.fp8_scale_shape(R, K), dtype=np.uint8)
+    assert s.shape == (3, 4)
+    expanded = np.kron(torch_e8m0(s), np.ones((128, 128)))[:R, :K]
+    ref = torch_e4m3(q) * expanded
+    assert np.array_equal(oracle.dequant_e4m3(q, s), ref)
+
+
+def _fp8_layer(rng, E, H, I, Is):
+    def mat(*shape):
+        q = rng.integers(0, 256, size=shape, dtype=np.uint8)
+        q[(q & 0x7F) == 0x7F] = 0xB8  # no NaN codes
+        s = rng.integers(118, 128, size=shape[:-2] + oracle.fp8_scale_shape(*shape[-2:]), dtype=np.uint8)
+        return q, s
+    return mat(E, 2 * I, H), mat(E, H, I), mat(2 * Is, H), mat(H, Is)
+
+
+def _as_bf16_bits(w: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(w).to(torch.bfloat16)
+    assert np.array_equal(t.double().numpy(), w), "FP8 weights must be exact in bf16"
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def test_fp8_layer_equals_the_bf16_layer_on_the_decoded_weights():
+    """Every E4M3 value times a power of two in the test's range is exact in bf16, so the FP8
+    layer must give the bf16 layer's output bit for bit once the weights are decoded by the
+    library (per expert, with per-expert scale tables and gate rows before up rows)."""
+    rng = np.random.default_rng(11)
+    E, H, I, Is, T, k = 4, 256, 256, 128, 5, 2
+    gu, dn, sgu, sdn = _fp8_layer(rng, E, H, I, Is)
+
+    def decode(q, s):  # library decoding, block expansion per matrix
+        if q.ndim == 3:
+            return np.stack([decode(q[e], s[e]) for e in range(q.shape[0])])
+        return torch_e4m3(q) * np.kron(torch_e8m0(s), np.ones((128, 128)))[: q.shape[0], : q.shape[1]]
+
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    idx = np.array([[0, 3], [1, 2], [2, 3], [0, 1], [3, 0]], np.int32)
+    w64 = rng.random((T, k))
+    y8 = oracle.moe_tokens_fp8(xb, idx, w64, gu, dn, sgu, sdn, swiglu_limit=7.0)
+    yb = oracle.moe_tokens(xb, idx, w64, _as_bf16_bits(decode(*gu)), _as_bf16_bits(decode(*dn)),
+                           _as_bf16_bits(decode(*sgu)), _as_bf16_bits(decode(*sdn)), swiglu_limit=7.0)
+    assert np.array_equal(y8, yb)
+    # the shared expert alone: routed down-projections of zero give the shared output
+    zq = np.zeros_like(dn[0])
+    y_sh = oracle.moe_tokens_fp8(xb, idx, w64, gu, (zq, dn[1]), sgu, sdn)
+    y_ref = oracle.moe_tokens(xb, idx, w64, _as_bf16_bits(decode(*gu)), _as_bf16_bits(np.zeros((E, H, I))),
+                              _as_bf16_bits(decode(*sgu)), _as_bf16_bits(decode(*sdn)))
+    assert np.array_equal(y_sh, y_ref)
