@@ -149,6 +149,45 @@ MOE_API moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const void
                                         moe_routing_out* routing, const moe_layer_options* options,
                                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* Expert weights in the blockwise FP8 format, for moe_layer_forward_fp8().  Each weight
+ * matrix W [R, K] of the layer is given as
+ *   codes  [R, K] bytes: FP8 E4M3 (OCP 8-bit floating point: sign, 4 exponent bits with
+ *          bias 7, 3 mantissa bits, subnormals at exponent 0, largest finite 448; the two
+ *          NaN codes S.1111.111 are outside the contract);
+ *   scales [R/128, K/128] bytes: one E8M0 scale per 128 x 128 block (OCP microscaling
+ *          formats: the power of two 2^(v - 127)), codes v in [10, 134];
+ * and stands for W[r, c] = e4m3(codes[r, c]) * 2^(scales[r/128, c/128] - 127).  Every such
+ * value is exact in bf16, so the layer computes exactly what moe_layer_forward() computes
+ * on bf16 weights holding the decoded values.  Matrices, as in moe_layer_forward():
+ *   W_gate_up  [E, 2*I, H]      scales [E, 2*I/128, H/128]
+ *   W_down     [E, H, I]        scales [E, H/128, I/128]
+ *   Ws_gate_up [2*I_shared, H]  scales [2*I_shared/128, H/128]   (NULL iff I_shared == 0)
+ *   Ws_down    [H, I_shared]    scales [H/128, I_shared/128]     (NULL iff I_shared == 0)
+ * Code arrays 16-byte aligned; scale arrays any alignment; all device memory owned by
+ * the caller and read only.  This format is the low-precision expert-weight option for
+ * decode; the source pages deploy 4-bit weights in a third-party format instead. */
+typedef struct {
+  const void* W_gate_up;
+  const void* W_gate_up_scale;
+  const void* W_down;
+  const void* W_down_scale;
+  const void* Ws_gate_up;
+  const void* Ws_gate_up_scale;
+  const void* Ws_down;
+  const void* Ws_down_scale;
+} moe_fp8_weights;
+
+/* moe_layer_forward_ex() with FP8 expert weights (moe_fp8_weights).  The shape's dtype
+ * must be MOE_BF16 (x, W_router and y as before); H, I and I_shared must be multiples of
+ * 128 and at most 8192.  The workspace is that of moe_layer_workspace_bytes(shape).
+ * Errors as moe_layer_forward_ex(), plus MOE_ERR_UNSUPPORTED_SHAPE for another dtype or
+ * sizes outside those bounds and MOE_ERR_INVALID_ARG for a missing or misaligned array. */
+MOE_API moe_status moe_layer_forward_fp8(const moe_layer_shape* shape, const void* x,
+                                         const void* W_router, const float* router_bias,
+                                         const moe_fp8_weights* weights, void* y,
+                                         moe_routing_out* routing, const moe_layer_options* options,
+                                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronises `stream`, then returns the device status word of the most recent
  * moe_layer_forward() that used this workspace (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or
  * MOE_ERR_DEVICE_BOUNDS), or MOE_ERR_CUDA if the stream itself reports an error. */

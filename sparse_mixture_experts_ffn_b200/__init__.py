@@ -24,7 +24,8 @@ STATUS_NAMES = {
     3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT",
     6: "MOE_ERR_DEVICE_BOUNDS",
 }
-EXPORTED = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_layer_forward_ex", "moe_layer_check_status",
+EXPORTED = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_layer_forward_ex", "moe_layer_forward_fp8",
+            "moe_layer_check_status",
             "moe_layer_route_stats", "moe_layer_workspace_layout", "moe_layer_profile_enable",
             "moe_layer_profile_read", "moe_layer_launch_count", "moe_status_string")
 STAGES = ("routing", "dispatch", "gate_up", "down", "combine")
@@ -43,6 +44,13 @@ class MoEOptions(ctypes.Structure):
 
 
 ROUTERS = {"softmax": 0, "sigmoid": 1}
+
+
+class MoEFp8Weights(ctypes.Structure):
+    _fields_ = [("W_gate_up", ctypes.c_void_p), ("W_gate_up_scale", ctypes.c_void_p),
+                ("W_down", ctypes.c_void_p), ("W_down_scale", ctypes.c_void_p),
+                ("Ws_gate_up", ctypes.c_void_p), ("Ws_gate_up_scale", ctypes.c_void_p),
+                ("Ws_down", ctypes.c_void_p), ("Ws_down_scale", ctypes.c_void_p)]
 
 
 class MoERoutingOut(ctypes.Structure):
@@ -89,6 +97,10 @@ def load_library(path: str = LIB_PATH):
                                          ctypes.POINTER(MoERoutingOut), ctypes.POINTER(MoEOptions), P,
                                          ctypes.c_size_t, P]
     lib.moe_layer_forward_ex.restype = ctypes.c_int
+    lib.moe_layer_forward_fp8.argtypes = [ctypes.POINTER(MoEShape), P, P, P, ctypes.POINTER(MoEFp8Weights), P,
+                                          ctypes.POINTER(MoERoutingOut), ctypes.POINTER(MoEOptions), P,
+                                          ctypes.c_size_t, P]
+    lib.moe_layer_forward_fp8.restype = ctypes.c_int
     lib.moe_layer_check_status.argtypes = [P, P]
     lib.moe_layer_check_status.restype = ctypes.c_int
     lib.moe_layer_route_stats.argtypes = [P, ctypes.POINTER(MoERouteStats), P]
@@ -162,15 +174,49 @@ def moe_layer_forward(x, W_router, W_gate_up, W_down, Ws_gate_up=None, Ws_down=N
     router="sigmoid": sigmoid scores, router_bias for the selection only, weights
     routed_scaling_factor * p / sum p (the default "softmax" ignores the factor).
     """
+    I = W_gate_up.shape[1] // 2
+    Is = 0 if Ws_gate_up is None else Ws_gate_up.shape[0] // 2
+    tensors = (("W_gate_up", W_gate_up), ("W_down", W_down), ("Ws_gate_up", Ws_gate_up), ("Ws_down", Ws_down))
+    return _forward("moe_layer_forward_ex", (W_gate_up, W_down, Ws_gate_up, Ws_down), tensors, x, W_router, I, Is,
+                    top_k, router_bias, y, workspace, routing, stream, swiglu_limit, swiglu_limit_shared, router,
+                    routed_scaling_factor)
+
+
+def moe_layer_forward_fp8(x, W_router, weights, *, top_k, router_bias=None, y=None, workspace=None,
+                          routing=True, stream=None, swiglu_limit=0.0, swiglu_limit_shared=0.0,
+                          router="softmax", routed_scaling_factor=1.0):
+    """moe_layer_forward with expert weights in the blockwise FP8 format.
+
+    ``weights``: a dict with W_gate_up, W_down, Ws_gate_up, Ws_down, each a pair (codes
+    uint8, scales uint8) -- E4M3 codes of the matrix and one E8M0 scale per 128 x 128 block,
+    shapes as in include/moe_layer.h (the shared pairs may be None) -- as made by
+    ``inputs.fp8_blockwise``.  x and W_router bf16 (W_router may be fp32).
+    """
+    import torch
+    gu, dn = weights["W_gate_up"], weights["W_down"]
+    sgu, sdn = weights.get("Ws_gate_up"), weights.get("Ws_down")
+    for pair in (gu, dn, sgu, sdn):
+        if pair is not None and (pair[0].dtype != torch.uint8 or pair[1].dtype != torch.uint8):
+            raise ValueError("FP8 weights are (codes, scales) pairs of uint8 tensors")
+    I = gu[0].shape[1] // 2
+    Is = 0 if sgu is None else sgu[0].shape[0] // 2
+    parts = (gu, dn, sgu, sdn)
+    names = ("W_gate_up", "W_down", "Ws_gate_up", "Ws_down")
+    tensors = tuple((f"{n}{suffix}", None if pr is None else pr[i])
+                    for n, pr in zip(names, parts) for i, suffix in ((0, ""), (1, "_scale")))
+    return _forward("moe_layer_forward_fp8", parts, tensors, x, W_router, I, Is, top_k, router_bias, y,
+                    workspace, routing, stream, swiglu_limit, swiglu_limit_shared, router,
+                    routed_scaling_factor)
+
+
+def _forward(entry, weights, tensors, x, W_router, I, Is, top_k, router_bias, y, workspace, routing, stream,
+             swiglu_limit, swiglu_limit_shared, router, routed_scaling_factor):
     import torch
     lib = load_library()
     T, H = x.shape
     E = W_router.shape[0]
-    I = W_gate_up.shape[1] // 2
-    Is = 0 if Ws_gate_up is None else Ws_gate_up.shape[0] // 2
     shape = make_shape(T, H, E, I, Is, top_k, x.dtype)
-    for name, t in (("x", x), ("W_router", W_router), ("W_gate_up", W_gate_up), ("W_down", W_down),
-                    ("Ws_gate_up", Ws_gate_up), ("Ws_down", Ws_down), ("router_bias", router_bias)):
+    for name, t in (("x", x), ("W_router", W_router), ("router_bias", router_bias)) + tuple(tensors):
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError(f"{name} must be a contiguous CUDA tensor")
     if y is None:
@@ -193,13 +239,16 @@ def moe_layer_forward(x, W_router, W_gate_up, W_down, Ws_gate_up=None, Ws_down=N
     w32 = 1 if (x.dtype == torch.bfloat16 and W_router.dtype == torch.float32) else 0
     opts = MoEOptions(float(swiglu_limit), float(swiglu_limit_shared), ROUTERS[router],
                       float(routed_scaling_factor), w32)
-    rc = lib.moe_layer_forward_ex(ctypes.byref(shape), _ptr(x), _ptr(W_router), _ptr(router_bias),
-                                  _ptr(W_gate_up), _ptr(W_down), _ptr(Ws_gate_up), _ptr(Ws_down),
-                                  _ptr(y), ctypes.byref(rout) if rout is not None else None,
-                                  ctypes.byref(opts), _ptr(workspace), workspace.numel(),
-                                  ctypes.c_void_p(stream.cuda_stream))
+    common = (ctypes.byref(shape), _ptr(x), _ptr(W_router), _ptr(router_bias))
+    tail = (_ptr(y), ctypes.byref(rout) if rout is not None else None, ctypes.byref(opts), _ptr(workspace),
+            workspace.numel(), ctypes.c_void_p(stream.cuda_stream))
+    if entry == "moe_layer_forward_fp8":
+        fw = MoEFp8Weights(*[None if pr is None else pr[i].data_ptr() for pr in weights for i in (0, 1)])
+        rc = lib.moe_layer_forward_fp8(*common, ctypes.byref(fw), *tail)
+    else:
+        rc = lib.moe_layer_forward_ex(*common, *(_ptr(w) for w in weights), *tail)
     if rc != MOE_OK:
-        raise MoEError(rc, "moe_layer_forward_ex")
+        raise MoEError(rc, entry)
     return y, r
 
 

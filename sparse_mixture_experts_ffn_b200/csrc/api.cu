@@ -118,6 +118,8 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.bn = choose_tile_n(s->T, s->top_k, s->E);
   L.bn_dn = choose_tile_n_down(s->T, s->top_k, s->E);
   L.ksplit = s->dtype == MOE_BF16 ? choose_ksplit(s->T, s->top_k, s->E, s->I, s->I_shared, L.bn) : 1;
+  // every slice of the reduction keeps at least one 64-column k-block (H = 128 has two)
+  while (L.ksplit > 1 && L.ksplit > s->H / kTileK) L.ksplit /= 2;
   L.max_tiles = expert_tile_bound(s->T, s->top_k, s->E, s->I, s->I_shared, L.bn);
   // control block and counters first: one memset per forward clears them
   const bool tc_scores = router_scores_f32(*s);
@@ -216,12 +218,27 @@ extern "C" moe_status moe_layer_forward(const moe_layer_shape* shape, const void
                               y, routing, nullptr, workspace, workspace_bytes, stream);
 }
 
-extern "C" moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const void* x,
-                                           const void* W_router, const float* router_bias,
-                                           const void* W_gate_up, const void* W_down,
-                                           const void* Ws_gate_up, const void* Ws_down, void* y,
-                                           moe_routing_out* routing, const moe_layer_options* options,
-                                           void* workspace, size_t workspace_bytes, void* stream) {
+namespace moe {
+
+// The four expert weight matrices: bf16/fp32 in the layer's dtype, or FP8 codes with their
+// block scales.
+struct ExpertWeights {
+  const void* Wgu;
+  const void* Wd;
+  const void* Wsgu;
+  const void* Wsd;
+  bool w8;
+  const void* scale[4];  // FP8: of Wgu, Wd, Wsgu, Wsd
+};
+
+static moe_status forward_impl(const moe_layer_shape* shape, const void* x, const void* W_router,
+                               const float* router_bias, const ExpertWeights& wt, void* y,
+                               moe_routing_out* routing, const moe_layer_options* options,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  const void* W_gate_up = wt.Wgu;
+  const void* W_down = wt.Wd;
+  const void* Ws_gate_up = wt.Wsgu;
+  const void* Ws_down = wt.Wsd;
   const moe_layer_options opt = options ? *options : moe_layer_options{0.0f, 0.0f, MOE_ROUTER_SOFTMAX, 0.0f, 0};
   if (!(opt.swiglu_limit >= 0.0f && opt.swiglu_limit <= FLT_MAX) ||
       !(opt.swiglu_limit_shared >= 0.0f && opt.swiglu_limit_shared <= FLT_MAX) ||
@@ -244,9 +261,13 @@ extern "C" moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const v
       (reinterpret_cast<uintptr_t>(router_bias) & 3u) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return MOE_ERR_INVALID_ARG;
+  if (wt.w8 && (!wt.scale[0] || !wt.scale[1] || (has_shared && (!wt.scale[2] || !wt.scale[3]))))
+    return MOE_ERR_INVALID_ARG;
   Layout L;
   make_layout(shape, L);
   if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  // FP8 weights run on 16- and 128-token tiles only
+  const int bn_dn = wt.w8 ? std::min(L.bn_dn, 128) : L.bn_dn;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
@@ -302,7 +323,7 @@ extern "C" moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const v
   da.I = s.I;
   da.Is = s.I_shared;
   da.bn = L.bn;
-  da.bn_dn = L.bn_dn;
+  da.bn_dn = bn_dn;
   da.ksplit = L.ksplit;
   da.x = x;
   da.idx = ra.idx_ws;
@@ -338,6 +359,11 @@ extern "C" moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const v
   ea.Wd = W_down;
   ea.Wsgu = Ws_gate_up;
   ea.Wsd = Ws_down;
+  ea.w8 = wt.w8;
+  ea.Wgu_scale = wt.scale[0];
+  ea.Wd_scale = wt.scale[1];
+  ea.Wsgu_scale = wt.scale[2];
+  ea.Wsd_scale = wt.scale[3];
   ea.offsets = da.offsets;
   ea.group_order = da.group_order;
   ea.item_start_gu = da.item_start_gu;
@@ -346,7 +372,7 @@ extern "C" moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const v
   ea.x_perm = da.x_perm;
   ea.row_tok = da.row_tok;
   ea.bn = L.bn;
-  ea.bn_dn = L.bn_dn;
+  ea.bn_dn = bn_dn;
   ea.ksplit = L.ksplit;
   ea.partial = static_cast<float*>(at(L.partial));
   ea.tile_done = static_cast<unsigned int*>(at(L.tile_done));
@@ -378,6 +404,38 @@ extern "C" moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const v
   if (launch_combine(ca, st) != cudaSuccess) return MOE_ERR_CUDA;
   marks.mark(5, st);
   return MOE_OK;
+}
+
+}  // namespace moe
+
+extern "C" moe_status moe_layer_forward_ex(const moe_layer_shape* shape, const void* x,
+                                           const void* W_router, const float* router_bias,
+                                           const void* W_gate_up, const void* W_down,
+                                           const void* Ws_gate_up, const void* Ws_down, void* y,
+                                           moe_routing_out* routing, const moe_layer_options* options,
+                                           void* workspace, size_t workspace_bytes, void* stream) {
+  const ExpertWeights wt{W_gate_up, W_down, Ws_gate_up, Ws_down, false, {nullptr, nullptr, nullptr, nullptr}};
+  return forward_impl(shape, x, W_router, router_bias, wt, y, routing, options, workspace, workspace_bytes,
+                      stream);
+}
+
+extern "C" moe_status moe_layer_forward_fp8(const moe_layer_shape* shape, const void* x,
+                                            const void* W_router, const float* router_bias,
+                                            const moe_fp8_weights* weights, void* y,
+                                            moe_routing_out* routing, const moe_layer_options* options,
+                                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (!shape || !weights) return MOE_ERR_INVALID_ARG;
+  const moe_layer_shape& s = *shape;
+  if (s.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED_SHAPE;
+  // the GEMM producer keeps one item's block scales in two registers per lane: at most
+  // 64 scale blocks (8192 columns) along a reduction
+  if (s.H > 8192 || s.I > 8192 || s.I_shared > 8192 || s.H % 128 || s.I % 128 || s.I_shared % 128)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  const moe_fp8_weights& w = *weights;
+  const ExpertWeights wt{w.W_gate_up, w.W_down, w.Ws_gate_up, w.Ws_down, true,
+                         {w.W_gate_up_scale, w.W_down_scale, w.Ws_gate_up_scale, w.Ws_down_scale}};
+  return forward_impl(shape, x, W_router, router_bias, wt, y, routing, options, workspace, workspace_bytes,
+                      stream);
 }
 
 extern "C" moe_status moe_layer_check_status(void* workspace, void* stream) {

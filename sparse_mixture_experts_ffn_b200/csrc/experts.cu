@@ -7,6 +7,13 @@
 //   down:     o[p, c]  = w_p * (h_p . Wd[e, c])                     (routing weight fused)
 // with fp32 accumulators in tensor memory and bf16 outputs.  The shared expert
 // (share_expert_dim, always on, weight 1) is one more group over all T tokens.
+//
+// FP8 weights (the low-precision expert weights for decode): each weight matrix is
+// E4M3 codes plus one E8M0 power-of-two scale per 128 x 128 block.  TMA brings the codes
+// (half the bytes of bf16); four more warps turn each 128 x 64 code tile into the bf16
+// tile the MMA reads, scale applied, in the layout 128-byte-swizzled TMA would have
+// written.  Every decoded weight is exact in bf16, so the GEMM is the bf16 GEMM of the
+// decoded weights, with bf16 tokens as before.
 // Sources: llm-atlas page "Step-3.5-Flash", "Champs bruts du config.json":
 // moe_intermediate_size 1280, share_expert_dim 1280, hidden_size 4096, norm_expert_weight.
 //
@@ -52,33 +59,48 @@ struct TcParams {
   float* partial;              // [max_tiles][ksplit][BN][256] fp32 gate|up partial sums
   unsigned int* tile_done;     // [max_tiles] slices finished per tile, zero before the launch
   unsigned int* item_counter;  // items claimed beyond the first gridDim.x, zero before the launch
+  const uint8_t* scaleA[2];    // FP8 weights: E8M0 block scales of the A matrices, routed
+                               // (stacked by expert) and shared
+  int s_rows_per_group;        // FP8 weights: scale rows (128-row blocks) per routed expert
+  int s_ld[2];                 // FP8 weights: scale columns (128-column blocks), routed and shared
   Ctrl* ctrl;
 };
 
 constexpr int kMaxDynSmem = 232448;  // 227 KB per block on sm_100
 constexpr int kRing = 4;             // item slots between the producer and the other roles
 
-template <bool GATED, int BN>
+template <bool GATED, int BN, bool W8 = false>
 struct TcCfg {
-  static constexpr int kABytes = kTileM * kTileK * 2;  // 16 KB of weights per operand tile
+  static constexpr int kMats = GATED ? 2 : 1;           // weight tiles per stage (gate, up)
+  static constexpr int kABytes = kTileM * kTileK * 2;  // 16 KB of bf16 weights per operand tile
+  static constexpr int kA8Bytes = kTileM * kTileK;     // the same tile as FP8 codes
   static constexpr int kBBytes = BN * kTileK * 2;      // token rows
-  static constexpr int kStageBytes = (GATED ? 2 : 1) * kABytes + kBBytes;
+  // one TMA stage: the weight tiles as loaded (bf16, or FP8 codes), then the token rows
+  static constexpr int kBOffset = kMats * (W8 ? kA8Bytes : kABytes);
+  static constexpr int kStageBytes = kBOffset + kBBytes;
+  // FP8: stages of converted bf16 weight tiles between the converters and the MMA
+  static constexpr int kConvStages = W8 ? 2 : 0;
+  static constexpr int kConvBytes = kMats * kABytes;
+  static constexpr int kThreads = W8 ? 320 : 192;
   // tiles of up to 128 tokens stage the output tile [BN][128] bf16 in shared memory for
   // 16-byte stores; 256-token tiles store straight from registers (each warp writes 64
   // contiguous bytes per token) to leave shared memory to the pipeline
   static constexpr bool kStaged = BN <= 128;
   static constexpr int kStagingBytes = kStaged ? BN * kTileM * 2 : 0;
   static constexpr int kAuxBytes = 512 + (BN * 4 > 512 ? BN * 4 : 512);  // barriers, TMEM slot | row weights
-  static constexpr int kFit = (kMaxDynSmem - kStagingBytes - 1024 - kAuxBytes) / kStageBytes;
+  static constexpr int kFit =
+      (kMaxDynSmem - kStagingBytes - 1024 - kAuxBytes - kConvStages * kConvBytes) / kStageBytes;
   static constexpr int kStages = kFit > 12 ? 12 : kFit;
   static constexpr int kAccCols = (GATED ? 2 : 1) * BN;  // TMEM columns per accumulator
   static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;  // double-buffered when it fits
   static constexpr int kTmemNeed = kAccBufs * kAccCols;
   static constexpr int kTmemCols = (kTmemNeed <= 32) ? 32 : (kTmemNeed <= 64) ? 64
                                  : (kTmemNeed <= 128) ? 128 : (kTmemNeed <= 256) ? 256 : 512;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + kAuxBytes;
+  static constexpr int kSmemBytes =
+      kStages * kStageBytes + kConvStages * kConvBytes + kStagingBytes + 1024 + kAuxBytes;
   static_assert(kStages >= 2, "pipeline too shallow");
-  static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(kStageBytes % 1024 == 0 && kBOffset % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(!W8 || BN <= 128, "FP8 weights: staged tiles only");
   static_assert(kTmemNeed <= 512, "accumulators exceed tensor memory");
   static_assert(kSmemBytes <= kMaxDynSmem, "shared memory budget");
   static_assert(BN % 16 == 0 && BN <= 256, "tile width");
@@ -158,6 +180,51 @@ __device__ __forceinline__ float swiglu(float g, float u, float L) {
   return g / (1.0f + __expf(-g)) * u;
 }
 
+// Two E4M3 codes (bytes `sel` picks from w) -> two bf16 bit patterns, the low code in
+// the low half, each standing for its code times 2^-120.  An E4M3 code is a sign, a
+// 4-bit exponent e (bias 7) and a 3-bit mantissa m; moving its exponent and mantissa
+// fields into bf16's (bias 127) gives 2^(e-127) (1 + m/8) for e > 0 and, for e = 0, the
+// bf16 subnormal 2^-126 m/8 = the code's subnormal m/8 * 2^-6 times the same 2^-120.
+__device__ __forceinline__ uint32_t e4m3x2_bits(uint32_t w, uint32_t sel) {
+  const uint32_t v = __byte_perm(w, 0u, sel);  // one code in the high byte of each half
+  return (v & 0x80008000u) | ((v >> 4) & 0x07F007F0u);
+}
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&a), y = *reinterpret_cast<__nv_bfloat162*>(&b);
+  __nv_bfloat162 r = __hmul2(x, y);
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// One 128 x 64 FP8 code tile (rows of 64 bytes, as TMA loads it without swizzling) ->
+// the bf16 tile [128][64] the MMA reads: rows of 128 bytes whose 16-byte chunk c sits at
+// chunk c ^ (row % 8), the layout of a 128-byte-swizzled TMA load.  `scale` is the
+// block's E8M0 code v: the weights are code * 2^(v - 127) = bits * 2^(v - 7), a product
+// exact in bf16 for v <= 134.  128 threads, four 16-code chunks each.
+__device__ __forceinline__ void fp8_tile_to_bf16(const unsigned char* src, unsigned char* dst, int ct,
+                                                 uint32_t scale) {
+  const uint32_t mb = (scale + 120u) << 7;  // bf16 2^(v - 7)
+  const uint32_t mult = mb | (mb << 16);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int qd = ct + 128 * i;  // row qd / 4, codes 16 (qd % 4) .. + 15 of the row
+    const int r = qd >> 2, j = qd & 3;
+    const uint4 w = *reinterpret_cast<const uint4*>(src + r * 64 + j * 16);
+    uint4 o0, o1;
+    o0.x = bf16x2_mul(e4m3x2_bits(w.x, 0x1404u), mult);
+    o0.y = bf16x2_mul(e4m3x2_bits(w.x, 0x3424u), mult);
+    o0.z = bf16x2_mul(e4m3x2_bits(w.y, 0x1404u), mult);
+    o0.w = bf16x2_mul(e4m3x2_bits(w.y, 0x3424u), mult);
+    o1.x = bf16x2_mul(e4m3x2_bits(w.z, 0x1404u), mult);
+    o1.y = bf16x2_mul(e4m3x2_bits(w.z, 0x3424u), mult);
+    o1.z = bf16x2_mul(e4m3x2_bits(w.w, 0x1404u), mult);
+    o1.w = bf16x2_mul(e4m3x2_bits(w.w, 0x3424u), mult);
+    unsigned char* row = dst + r * 128;
+    *reinterpret_cast<uint4*>(row + (((2 * j) ^ (r & 7)) << 4)) = o0;
+    *reinterpret_cast<uint4*>(row + (((2 * j + 1) ^ (r & 7)) << 4)) = o1;
+  }
+}
+
 // Wait without looking at the abort flag (teardown: in-flight copies must land).
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, Ctrl* ctrl) {
   const uint64_t t0 = globaltimer_ns();
@@ -169,23 +236,25 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   }
 }
 
-// Persistent grouped GEMM: 192 threads, one block per SM.
+// Persistent grouped GEMM: 192 threads (320 with FP8 weights), one block per SM.
 //   warp 0      TMA producer (one lane): weight tiles (gate and up for GATED) and token rows
 //   warp 1      allocates tensor memory; one lane issues the tcgen05 MMAs
 //   warps 2..5  epilogue: tensor memory -> registers -> shared staging tile -> global
+//   warps 6..9  FP8 weights only: code tiles -> bf16 tiles
 // Accumulators are double-buffered in tensor memory, so the epilogue of one tile overlaps
 // the main loop of the next.  Items are claimed dynamically: block b starts with item b and
 // then takes the next unclaimed one from a global counter, so blocks that draw short tiles
 // take more of them; the producer publishes each claimed item to the MMA and epilogue warps
 // through a ring of kRing shared-memory slots (index -1 ends the schedule).
-template <bool GATED, int BN>
-__global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
-  using C = TcCfg<GATED, BN>;
+template <bool GATED, int BN, bool W8>
+__global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
+  using C = TcCfg<GATED, BN, W8>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   unsigned char* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
-  __nv_bfloat16* staging = reinterpret_cast<__nv_bfloat16*>(smem + C::kStages * C::kStageBytes);
-  unsigned char* aux = smem + C::kStages * C::kStageBytes + C::kStagingBytes;
+  unsigned char* conv = smem + C::kStages * C::kStageBytes;  // FP8: converted weight tiles
+  __nv_bfloat16* staging = reinterpret_cast<__nv_bfloat16*>(conv + C::kConvStages * C::kConvBytes);
+  unsigned char* aux = conv + C::kConvStages * C::kConvBytes + C::kStagingBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(aux);
   uint64_t* empty = full + C::kStages;
   uint64_t* tfull = empty + C::kStages;
@@ -193,6 +262,10 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* cfull = reinterpret_cast<uint64_t*>(aux + 256);  // FP8: [kConvStages] converted
+  uint64_t* cempty = cfull + 2;                              // FP8: [kConvStages] consumed
+  volatile uint32_t* sc_stage = reinterpret_cast<volatile uint32_t*>(aux + 288);  // FP8: [kStages]
+                                                         // scale codes of each stage's tiles
   uint64_t* ring_full = reinterpret_cast<uint64_t*>(aux + 384);  // [kRing]
   uint64_t* ring_empty = ring_full + kRing;                     // [kRing]
   volatile int* ring = reinterpret_cast<volatile int*>(ring_empty + kRing);  // [kRing] item ids
@@ -211,7 +284,12 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
     mbar_init(drain, 1);
     for (int q = 0; q < kRing; ++q) {
       mbar_init(&ring_full[q], 1);
-      mbar_init(&ring_empty[q], 1 + 4);  // the MMA thread and one lane per epilogue warp
+      // the MMA thread and one lane per epilogue (and converter) warp
+      mbar_init(&ring_empty[q], 1 + 4 + (W8 ? 4 : 0));
+    }
+    for (int c = 0; c < C::kConvStages; ++c) {
+      mbar_init(&cfull[c], 128);  // every converter thread
+      mbar_init(&cempty[c], 1);   // the MMA commit
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -291,26 +369,47 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
       const int arow = t.sh ? t.m * kTileM : t.g * p.a_rows_per_group + t.m * kTileM;
       const int kb_n = p.kblocks[t.sh];
       const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
+      // FP8: the item's block scales, one 128-column block per lane (and lane + 32)
+      uint32_t sg[2] = {0u, 0u}, su[2] = {0u, 0u};
+      const int sc0 = kb0 >> 1;  // 128-column scale blocks hold two 64-column k-blocks
+      if (W8) {
+        const int ld = p.s_ld[t.sh];
+        const uint8_t* sbase = p.scaleA[t.sh] + static_cast<int64_t>(t.sh ? 0 : t.g) * p.s_rows_per_group * ld;
+        const uint8_t* srow_g = sbase + static_cast<int64_t>(t.m) * ld;
+        const uint8_t* srow_u = sbase + static_cast<int64_t>(t.m + p.a_up_offset[t.sh] / kTileM) * ld;
+        const int nblk = kb1 > kb0 ? ((kb1 - 1) >> 1) - sc0 + 1 : 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          if (lane + 32 * h < nblk) {
+            sg[h] = __ldg(srow_g + sc0 + lane + 32 * h);
+            if (GATED) su[h] = __ldg(srow_u + sc0 + lane + 32 * h);
+          }
+      }
       for (int kb = kb0; kb < kb1; ++kb) {
         unsigned char* st = smem + stage * C::kStageBytes;
+        uint32_t scw = 0;
+        if (W8) {
+          const int rel = (kb >> 1) - sc0;  // < 64: the host bounds K by 64 scale blocks
+          scw = __shfl_sync(0xffffffffu, rel < 32 ? sg[0] : sg[1], rel & 31);
+          if (GATED) scw |= __shfl_sync(0xffffffffu, rel < 32 ? su[0] : su[1], rel & 31) << 8;
+        }
         int good = 1;
         if (lane == 0) {
           good = mbar_wait(&empty[stage], phase ^ 1u, p.ctrl, abort_flag) ? 1 : 0;
           if (good) {
+            if (W8) sc_stage[stage] = scw;  // published by the arrive below
             mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
             tma_load_2d(st, &p.tmA[t.sh], kb * kTileK, arow, &full[stage]);
             if (GATED)
-              tma_load_2d(st + C::kABytes, &p.tmA[t.sh], kb * kTileK, arow + p.a_up_offset[t.sh],
-                          &full[stage]);
-            if (!gath)
-              tma_load_2d(st + (GATED ? 2 : 1) * C::kABytes, &p.tmB[t.sh], kb * kTileK, t.row0,
-                          &full[stage]);
+              tma_load_2d(st + (W8 ? C::kA8Bytes : C::kABytes), &p.tmA[t.sh], kb * kTileK,
+                          arow + p.a_up_offset[t.sh], &full[stage]);
+            if (!gath) tma_load_2d(st + C::kBOffset, &p.tmB[t.sh], kb * kTileK, t.row0, &full[stage]);
           }
         }
         good = __shfl_sync(0xffffffffu, good, 0);
         if (!good) { ok = false; break; }
         if (gath && lane < BN / 4)
-          tma_gather4_2d(st + (GATED ? 2 : 1) * C::kABytes + lane * 4 * kTileK * 2, &p.tmB[0], kb * kTileK,
+          tma_gather4_2d(st + C::kBOffset + lane * 4 * kTileK * 2, &p.tmB[0], kb * kTileK,
                          tok[0], tok[1], tok[2], tok[3], &full[stage]);
         used |= 1u << stage;
         if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
@@ -329,8 +428,8 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
   } else if (warp == 1) {
     // ------------------------------- MMA issuer ---------------------------------------
     if (lane == 0) {
-      int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0;
+      int stage = 0, acc = 0, cs = 0;
+      uint32_t phase = 0, acc_phase = 0, cphase = 0;
       bool ok = true;
       int q = 0;
       uint32_t qphase = 0;
@@ -350,10 +449,12 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
         const int kb_n = p.kblocks[t.sh];
         const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, p.ctrl, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&full[stage], phase, p.ctrl, abort_flag) ||
+              (W8 && !mbar_wait(&cfull[cs], cphase, p.ctrl, abort_flag))) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t b0 = a0 + (GATED ? 2 : 1) * C::kABytes;
+          const uint32_t s0 = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t a0 = W8 ? smem_u32(conv + cs * C::kConvBytes) : s0;
+          const uint32_t b0 = s0 + C::kBOffset;
 #pragma unroll
           for (int kk = 0; kk < kTileK / 16; ++kk) {
             const uint32_t accum = (kb != kb0 || kk) ? 1u : 0u;
@@ -364,6 +465,10 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
           }
           mma_commit(&empty[stage]);
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+          if (W8) {
+            mma_commit(&cempty[cs]);
+            if (++cs == C::kConvStages) { cs = 0; cphase ^= 1u; }
+          }
         }
         if (!ok) break;
         mma_commit(&tfull[acc]);
@@ -372,6 +477,39 @@ __global__ void __launch_bounds__(192, 1) expert_gemm_tc_kernel(const __grid_con
       // all MMAs issued by this thread complete before the accumulators are freed
       mma_commit(drain);
       mbar_wait_drain(drain, 0, p.ctrl);
+    }
+  } else if (W8 && warp >= 6) {
+    // ------------------------- FP8 code tiles -> bf16 (warps 6..9) ---------------------
+    const int ct = threadIdx.x - 192;  // 0..127
+    int stage = 0, cs = 0;
+    uint32_t phase = 0, cphase = 0;
+    int q = 0;
+    uint32_t qphase = 0;
+    bool ok = true;
+    while (ok) {
+      if (!mbar_wait(&ring_full[q], qphase, p.ctrl, abort_flag)) break;
+      const int it = ring[q];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ring_empty[q]);
+      if (++q == kRing) { q = 0; qphase ^= 1u; }
+      if (it < 0) break;
+      const Item t = decode_item<BN>(p, sc, it);
+      if (!t.valid) continue;
+      const int kb_n = p.kblocks[t.sh];
+      const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&full[stage], phase, p.ctrl, abort_flag) ||
+            !mbar_wait(&cempty[cs], cphase ^ 1u, p.ctrl, abort_flag)) { ok = false; break; }
+        const uint32_t scw = sc_stage[stage];
+        const unsigned char* src = smem + stage * C::kStageBytes;
+        unsigned char* dst = conv + cs * C::kConvBytes;
+        fp8_tile_to_bf16(src, dst, ct, scw & 0xFFu);
+        if (GATED) fp8_tile_to_bf16(src + C::kA8Bytes, dst + C::kABytes, ct, (scw >> 8) & 0xFFu);
+        fence_proxy_async_smem();  // the tensor cores read these bytes next
+        mbar_arrive(&cfull[cs]);
+        if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        if (++cs == C::kConvStages) { cs = 0; cphase ^= 1u; }
+      }
     }
   } else {
     // ------------------------------- epilogue (warps 2..5) ----------------------------
@@ -624,10 +762,25 @@ static bool encode_2d_bf16(CUtensorMap* map, const void* base, uint64_t rows, ui
   return r == CUDA_SUCCESS;
 }
 
-template <bool GATED, int BN>
+// FP8 code matrix [rows, cols] (bytes): 128-row x 64-byte boxes, no swizzling (the
+// converters read the rows and write the swizzled bf16 layout themselves)
+static bool encode_2d_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn fn = get_encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileK), static_cast<cuuint32_t>(kTileM)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool GATED, int BN, bool W8>
 static cudaError_t launch_tc(const TcParams& prm_in, int num_sms, cudaStream_t st) {
-  using C = TcCfg<GATED, BN>;
-  auto kern = expert_gemm_tc_kernel<GATED, BN>;
+  using C = TcCfg<GATED, BN, W8>;
+  auto kern = expert_gemm_tc_kernel<GATED, BN, W8>;
   TcParams prm = prm_in;
   const size_t tables = static_cast<size_t>(2 * prm.G + 1 + prm.E + 1) * sizeof(int32_t);
   prm.sched_smem = (C::kSmemBytes + tables <= static_cast<size_t>(kMaxDynSmem)) ? 1 : 0;
@@ -635,18 +788,22 @@ static cudaError_t launch_tc(const TcParams& prm_in, int num_sms, cudaStream_t s
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  e = launch_pdl(kern, dim3(num_sms), dim3(192), smem, st, prm);
+  e = launch_pdl(kern, dim3(num_sms), dim3(C::kThreads), smem, st, prm);
   count_launches(1);
   return e;
 }
 
 template <bool GATED>
-static cudaError_t launch_tc_bn(const TcParams& prm, int bn, int num_sms, cudaStream_t st) {
-  if (bn == 16) return launch_tc<GATED, 16>(prm, num_sms, st);
-  if constexpr (!GATED) {
-    if (bn == 256) return launch_tc<false, 256>(prm, num_sms, st);
+static cudaError_t launch_tc_bn(const TcParams& prm, int bn, bool w8, int num_sms, cudaStream_t st) {
+  if (w8) {  // FP8 weights: 16- and 128-token tiles
+    if (bn == 16) return launch_tc<GATED, 16, true>(prm, num_sms, st);
+    return launch_tc<GATED, 128, true>(prm, num_sms, st);
   }
-  return launch_tc<GATED, 128>(prm, num_sms, st);
+  if (bn == 16) return launch_tc<GATED, 16, false>(prm, num_sms, st);
+  if constexpr (!GATED) {
+    if (bn == 256) return launch_tc<false, 256, false>(prm, num_sms, st);
+  }
+  return launch_tc<GATED, 128, false>(prm, num_sms, st);
 }
 
 // Upper bound of the tiles of one grouped GEMM whose weight matrices have `rows` rows per
@@ -685,11 +842,15 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   // (16-token tiles) or x_perm [P, H] (shared: x [T, H] in order)
   TcParams g{};
   const bool gather = a.bn == 16;
-  bool ok = encode_2d_bf16(&g.tmA[0], a.Wgu, static_cast<uint64_t>(a.E) * 2 * a.I, a.H, kTileM) &&
+  // weight matrices: bf16 rows, or FP8 code rows with their block scales
+  auto encode_w = [&](CUtensorMap* m, const void* w, uint64_t rows, uint64_t cols) {
+    return a.w8 ? encode_2d_u8(m, w, rows, cols) : encode_2d_bf16(m, w, rows, cols, kTileM);
+  };
+  bool ok = encode_w(&g.tmA[0], a.Wgu, static_cast<uint64_t>(a.E) * 2 * a.I, a.H) &&
             (gather ? encode_2d_bf16(&g.tmB[0], a.x, a.T, a.H, 1)
                     : encode_2d_bf16(&g.tmB[0], a.x_perm, P, a.H, a.bn));
   if (has_shared)
-    ok = ok && encode_2d_bf16(&g.tmA[1], a.Wsgu, 2ull * a.Is, a.H, kTileM) &&
+    ok = ok && encode_w(&g.tmA[1], a.Wsgu, 2ull * a.Is, a.H) &&
          encode_2d_bf16(&g.tmB[1], a.x, a.T, a.H, a.bn);
   else {
     g.tmA[1] = g.tmA[0];
@@ -726,15 +887,19 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   g.ctrl = a.ctrl;
   g.ld_out[0] = a.I;
   g.ld_out[1] = a.Is;
-  cudaError_t e = launch_tc_bn<true>(g, a.bn, a.num_sms, st);
+  g.scaleA[0] = static_cast<const uint8_t*>(a.Wgu_scale);
+  g.scaleA[1] = static_cast<const uint8_t*>(a.Wsgu_scale);
+  g.s_rows_per_group = 2 * a.I / kTileM;
+  g.s_ld[0] = g.s_ld[1] = (a.H + 127) / 128;
+  cudaError_t e = launch_tc_bn<true>(g, a.bn, a.w8, a.num_sms, st);
   if (e != cudaSuccess) return e;
   if (a.stage_mark) a.stage_mark(a.stage_mark_ctx, 3, st);
   // down: A = W_down viewed as [E*H, I]; B = h [P, I] (shared: Ws_down [H, Is], h_shared)
   TcParams d{};
-  ok = encode_2d_bf16(&d.tmA[0], a.Wd, static_cast<uint64_t>(a.E) * a.H, a.I, kTileM) &&
+  ok = encode_w(&d.tmA[0], a.Wd, static_cast<uint64_t>(a.E) * a.H, a.I) &&
        encode_2d_bf16(&d.tmB[0], a.h, P, a.I, a.bn_dn);
   if (has_shared)
-    ok = ok && encode_2d_bf16(&d.tmA[1], a.Wsd, a.H, a.Is, kTileM) &&
+    ok = ok && encode_w(&d.tmA[1], a.Wsd, a.H, a.Is) &&
          encode_2d_bf16(&d.tmB[1], a.h_shared, a.T, a.Is, a.bn_dn);
   else {
     d.tmA[1] = d.tmA[0];
@@ -763,7 +928,12 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   d.max_items = d.max_tiles;
   d.item_counter = a.item_counters + 1;
   d.ctrl = a.ctrl;
-  return launch_tc_bn<false>(d, a.bn_dn, a.num_sms, st);
+  d.scaleA[0] = static_cast<const uint8_t*>(a.Wd_scale);
+  d.scaleA[1] = static_cast<const uint8_t*>(a.Wsd_scale);
+  d.s_rows_per_group = a.H / kTileM;
+  d.s_ld[0] = (a.I + 127) / 128;
+  d.s_ld[1] = (a.Is + 127) / 128;
+  return launch_tc_bn<false>(d, a.bn_dn, a.w8, a.num_sms, st);
 }
 
 }  // namespace moe

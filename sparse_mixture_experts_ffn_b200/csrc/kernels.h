@@ -107,6 +107,11 @@ struct ExpertArgs {
   const void* Wd;    // [E, H, I]
   const void* Wsgu;  // [2Is, H] or null
   const void* Wsd;   // [H, Is]
+  bool w8;           // the four weight matrices are FP8 E4M3 codes with E8M0 block scales
+  const void* Wgu_scale;   // FP8: [E, 2I/128, H/128]
+  const void* Wd_scale;    // FP8: [E, H/128, I/128]
+  const void* Wsgu_scale;  // FP8: [2Is/128, H/128]
+  const void* Wsd_scale;   // FP8: [H/128, Is/128]
   const int32_t* offsets;
   const int32_t* group_order;
   const int32_t* item_start_gu;

@@ -118,3 +118,26 @@ def test_forward_ex_rejects_bad_swiglu_limits_before_any_launch(lib):
     # NULL options is the plain forward (validation of the other arguments still runs)
     assert lib.moe_layer_forward_ex(ctypes.byref(s), None, P(16), None, P(16), P(16), P(16), P(16),
                                     P(16), None, None, P(256), n, None) == 1
+
+
+def test_forward_fp8_rejects_bad_arguments_before_any_launch(lib):
+    P = ctypes.c_void_p
+
+    def call(s, scales=(1, 1, 1, 1), codes=(16, 16, 16, 16), weights=True, ws_bytes=None):
+        n = moe.workspace_bytes(s) if ws_bytes is None else ws_bytes
+        fw = moe.MoEFp8Weights(codes[0], scales[0], codes[1], scales[1], codes[2], scales[2], codes[3],
+                               scales[3])
+        return lib.moe_layer_forward_fp8(ctypes.byref(s), P(16), P(16), None,
+                                         ctypes.byref(fw) if weights else None, P(16), None, None, P(256),
+                                         n or 1, None)
+
+    assert call(shape(), weights=False) == 1
+    assert call(shape(dtype=moe.MOE_F32)) == 2        # FP8 weights go with bf16 tokens only
+    assert call(shape(H=4160)) == 2                   # not a multiple of 128
+    assert call(shape(I=1344)) == 2
+    assert call(shape(H=8320)) == 2                   # more than 64 scale blocks per reduction
+    assert call(shape(), scales=(None, 1, 1, 1)) == 1  # a scale table missing
+    assert call(shape(), scales=(1, 1, 1, None)) == 1
+    assert call(shape(), codes=(24, 16, 16, 16)) == 1  # codes misaligned
+    assert call(shape(), ws_bytes=moe.workspace_bytes(shape()) - 1) == 3
+    assert call(shape(T=0)) == 0                      # empty batch: nothing to do

@@ -140,6 +140,7 @@ EDGE_CASES = [
     dict(T=33, H=256, E=512, top_k=4, I=128, I_shared=128),    # the largest tensor-core router
     dict(T=50, H=256, E=1, top_k=1, I=128, I_shared=128),      # a single expert
     dict(T=3, H=512, E=16, top_k=4, I=256, I_shared=0),        # split decode GEMM, no shared expert
+    dict(T=2, H=128, E=16, top_k=4, I=128, I_shared=128),      # two k-blocks: the split stops at 2
 ]
 
 
@@ -310,6 +311,106 @@ def test_full_size_layer_as_configured(name):
     y_ref = oracle_y(d, ref, tokens=tokens, swiglu_limit=7.0, swiglu_limit_shared=16.0)
     assert_y_close(y[torch.as_tensor(tokens, device=y.device)], y_ref, name + " as configured")
     print(name, "as configured, route stats", moe.route_stats(ws))
+
+
+# ------------------------------------------------------------------------------------
+# FP8 expert weights (E4M3 codes, one E8M0 scale per 128 x 128 block)
+# ------------------------------------------------------------------------------------
+def fp8_inputs(cfg, shared=True):
+    x, Wr, bias = inputs.make_routing_inputs(cfg)
+    d = to_device(dict(x=x, W_router=Wr, bias=bias))
+    d["fp8"] = inputs.make_fp8_expert_weights(cfg, "cuda", shared=shared)
+    return d
+
+
+def oracle_y_fp8(d, routing, tokens=None, swiglu_limit=0.0, swiglu_limit_shared=0.0):
+    import oracle
+    from conftest import to_oracle
+
+    def host(pair):
+        return None if pair is None else tuple(t.cpu().numpy() for t in pair)
+
+    w = d["fp8"]
+    return oracle.moe_tokens_fp8(to_oracle(d["x"]), routing["idx"], routing["w64"], host(w["W_gate_up"]),
+                                 host(w["W_down"]), host(w["Ws_gate_up"]), host(w["Ws_down"]), tokens=tokens,
+                                 swiglu_limit=swiglu_limit, swiglu_limit_shared=swiglu_limit_shared)
+
+
+def run_fp8(d, top_k, tokens=None, what="", **kw):
+    x = d["x"]
+    w = d["fp8"]
+    I = w["W_gate_up"][0].shape[1] // 2
+    Is = 0 if w.get("Ws_gate_up") is None else w["Ws_gate_up"][0].shape[0] // 2
+    ws = moe.alloc_workspace(moe.make_shape(x.shape[0], x.shape[1], d["W_router"].shape[0], I, Is, top_k,
+                                            x.dtype), x.device)
+    y, r = moe.moe_layer_forward_fp8(x, d["W_router"], w, top_k=top_k, router_bias=d.get("bias"),
+                                     workspace=ws, **kw)
+    assert moe.check_status(ws) == moe.MOE_OK
+    ref = oracle_routing(d, top_k)
+    assert_routing_exact(r, ref, d["W_router"].shape[0])
+    limits = {k: kw[k] for k in ("swiglu_limit", "swiglu_limit_shared") if k in kw}
+    y_ref = oracle_y_fp8(d, ref, tokens=tokens, **limits)
+    yt = y if tokens is None else y[torch.as_tensor(tokens, device=y.device)]
+    return assert_y_close(yt, y_ref, what)
+
+
+FP8_CASES = [
+    # 16-token tiles, gate/up reduction split in 4 (each slice two k-blocks of one scale block)
+    dict(T=3, H=512, E=16, top_k=4, I=128, I_shared=128),
+    # 17 scale blocks along H, 200 experts, split reduction with ragged slices
+    dict(T=3, H=2176, E=200, top_k=8, I=128, I_shared=128),
+    # 128-token tiles; 3 scale blocks along H, 2 row blocks per gate and up half
+    dict(T=129, H=384, E=12, top_k=1, I=256, I_shared=256),
+    dict(T=300, H=256, E=16, top_k=4, I=256, I_shared=128),
+    # long-prefill grouping (the bf16 down GEMM would take 256-token tiles; FP8 keeps 128)
+    dict(T=700, H=256, E=8, top_k=4, I=256, I_shared=128),
+    # no shared expert, 3 row blocks per half
+    dict(T=200, H=512, E=40, top_k=6, I=384, I_shared=0),
+    # one scale block along H, split reduction of two k-blocks
+    dict(T=2, H=128, E=16, top_k=4, I=128, I_shared=128),
+]
+
+
+@pytest.mark.parametrize("sz", FP8_CASES, ids=lambda s: "T{T}_H{H}_E{E}_k{top_k}_I{I}_Is{I_shared}".format(**s))
+def test_fp8_weights_parity(sz):
+    cfg = inputs.small_config(**sz)
+    d = fp8_inputs(cfg, shared=sz["I_shared"] > 0)
+    run_fp8(d, cfg.top_k, what=cfg.name + " fp8")
+
+
+def test_fp8_weights_with_swiglu_limits():
+    cfg = inputs.small_config(T=300, H=256, E=16, top_k=4, I=256, I_shared=128)
+    d = fp8_inputs(cfg)
+    run_fp8(d, cfg.top_k, what="fp8 limits", swiglu_limit=0.3, swiglu_limit_shared=0.2)
+
+
+@pytest.mark.parametrize("T", [3, 300])
+def test_fp8_subnormal_and_zero_codes(T):
+    """Weights made only of E4M3 subnormals (exponent field 0) and zeros, with scales far
+    from 1: the output is nonzero only if the conversion keeps the subnormals."""
+    cfg = inputs.small_config(T=T, H=256, E=16, top_k=4, I=128, I_shared=128)
+    d = fp8_inputs(cfg)
+    g = torch.Generator(device="cuda").manual_seed(5)
+    for k, (q, sc) in list(d["fp8"].items()):
+        codes = torch.randint(0, 8, q.shape, generator=g, device="cuda", dtype=torch.int32)  # m, e = 0
+        sign = torch.randint(0, 2, q.shape, generator=g, device="cuda", dtype=torch.int32) << 7
+        scale = torch.randint(125, 134, sc.shape, generator=g, device="cuda", dtype=torch.int32)
+        d["fp8"][k] = ((codes | sign).to(torch.uint8), scale.to(torch.uint8))
+    rel_max, _ = run_fp8(d, cfg.top_k, what="fp8 subnormals")
+    y, _ = moe.moe_layer_forward_fp8(d["x"], d["W_router"], d["fp8"], top_k=cfg.top_k, routing=False)
+    assert float(y.float().abs().max()) > 0
+
+
+@pytest.mark.parametrize("name", ["decode_t4", "decode_t128", "prefill_t4096"])
+def test_fp8_full_size_workload(name):
+    cfg = inputs.CONFIGS[name]
+    d = fp8_inputs(cfg)
+    if cfg.T <= 4:
+        tokens = None
+    else:
+        rng = np.random.default_rng(cfg.seed)
+        tokens = np.unique(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 30, replace=False)]))
+    run_fp8(d, cfg.top_k, tokens=tokens, what=name + " fp8")
 
 
 # ------------------------------------------------------------------------------------
