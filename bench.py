@@ -111,17 +111,21 @@ class ClockSampler:
 # ------------------------------------------------------------------------------------------
 # algorithmic bytes / flops
 # ------------------------------------------------------------------------------------------
-def algorithmic(cfg, counts: np.ndarray):
-    """Bytes and FLOPs of the layer and of its gate/up GEMM for one step (no padding)."""
+def algorithmic(cfg, counts: np.ndarray, fp8: bool = False):
+    """Bytes and FLOPs of the layer and of its gate/up GEMM for one step (no padding).
+    fp8: expert weights as E4M3 codes (1 byte) plus one scale byte per 128 x 128 block."""
     es = 2 if cfg.dtype == "bf16" else 4
     H, I, Is, E, T, k = cfg.H, cfg.I, cfg.I_shared, cfg.E, cfg.T, cfg.top_k
     touched = int((counts > 0).sum())
     P = T * k
-    layer_bytes = (touched * 3 * H * I + 3 * H * Is + E * H + 2 * T * H) * es
+
+    def wb(n):  # bytes of n expert weights
+        return n + n // (128 * 128) if fp8 else n * es
+    layer_bytes = wb(touched * 3 * H * I + 3 * H * Is) + (E * H + 2 * T * H) * es
     layer_flops = 2 * T * E * H + P * 6 * H * I + T * 6 * H * Is
-    gu_bytes = (touched * 2 * I * H + 2 * Is * H + P * H + T * H + P * I + T * Is) * es
+    gu_bytes = wb(touched * 2 * I * H + 2 * Is * H) + (P * H + T * H + P * I + T * Is) * es
     gu_flops = P * 4 * H * I + T * 4 * H * Is
-    dn_bytes = (touched * H * I + H * Is + P * I + T * Is + P * H + T * H) * es
+    dn_bytes = wb(touched * H * I + H * Is) + (P * I + T * Is + P * H + T * H) * es
     dn_flops = P * 2 * H * I + T * 2 * H * Is
     return dict(touched=touched, layer_bytes=layer_bytes, layer_flops=layer_flops,
                 gate_up_bytes=gu_bytes, gate_up_flops=gu_flops, down_bytes=dn_bytes, down_flops=dn_flops)
@@ -185,6 +189,8 @@ def host_arrays(d):
     def cv(t):
         if t is None:
             return None
+        if isinstance(t, tuple):  # FP8 weights: (codes, scales)
+            return tuple(cv(u) for u in t)
         t = t.detach().cpu().contiguous()
         return t.view(torch.int16).numpy().view(_np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
     return {k: cv(v) for k, v in d.items()}
@@ -205,20 +211,25 @@ def config_options(args) -> dict:
     out = {"layer_options": o} if o != LAYER_DEFAULTS else {}
     if getattr(args, "fp32_router", False):
         out["router_weights"] = "fp32"
+    if getattr(args, "weights", "bf16") == "fp8":
+        out["expert_weights"] = "fp8: E4M3 codes, one E8M0 scale per 128x128 block (bf16 tensor-core math)"
     return out
 
 
 def oracle_step(h, cfg, tokens, opts=None):
     """The whole hot path for the listed tokens: exact router over all experts, top-k and
-    weights, then the expert FFNs and the combine."""
+    weights, then the expert FFNs and the combine.  FP8 weights come as (codes, scales)."""
     import oracle
     o = dict(LAYER_DEFAULTS, **(opts or {}))
     x = h["x"][tokens]
     s = oracle.router_scores(x, h["W_router"])
     bias = None if h.get("bias") is None else h["bias"].astype(np.float32)
     idx, w, w64 = oracle.route(s, cfg.top_k, bias, router=o["router"], scale=o["routed_scaling_factor"])
-    return oracle.moe_tokens(x, idx, w64, h["W_gate_up"], h["W_down"], h["Ws_gate_up"], h["Ws_down"],
-                             swiglu_limit=o["swiglu_limit"], swiglu_limit_shared=o["swiglu_limit_shared"])
+    lim = dict(swiglu_limit=o["swiglu_limit"], swiglu_limit_shared=o["swiglu_limit_shared"])
+    if isinstance(h["W_gate_up"], tuple):
+        return oracle.moe_tokens_fp8(x, idx, w64, h["W_gate_up"], h["W_down"], h["Ws_gate_up"], h["Ws_down"],
+                                     **lim)
+    return oracle.moe_tokens(x, idx, w64, h["W_gate_up"], h["W_down"], h["Ws_gate_up"], h["Ws_down"], **lim)
 
 
 def run_reference(args, cfg):
@@ -230,11 +241,14 @@ def run_reference(args, cfg):
     d = inputs.make_inputs(cfg, "cpu") if cfg.T * cfg.H * cfg.E < 5e7 else None
     if d is not None and args.fp32_router:
         d["W_router"] = inputs.make_routing_inputs(cfg, router_fp32=True)[1]
-    if d is None:
+    if d is None or args.weights == "fp8":
         x, Wr, bias = inputs.make_routing_inputs(cfg, router_fp32=args.fp32_router)
         dev = "cuda" if torch.cuda.is_available() else "cpu"
-        Wgu, Wd, Wsgu, Wsd = inputs.make_expert_weights(cfg, dev)
-        d = dict(x=x, W_router=Wr, bias=bias, W_gate_up=Wgu, W_down=Wd, Ws_gate_up=Wsgu, Ws_down=Wsd)
+        if args.weights == "fp8":
+            d = dict(x=x, W_router=Wr, bias=bias, **inputs.make_fp8_expert_weights(cfg, dev))
+        else:
+            Wgu, Wd, Wsgu, Wsd = inputs.make_expert_weights(cfg, dev)
+            d = dict(x=x, W_router=Wr, bias=bias, W_gate_up=Wgu, W_down=Wd, Ws_gate_up=Wsgu, Ws_down=Wsd)
     h = host_arrays(d)
     cores = len(os.sched_getaffinity(0))
     per_step = 1  # tokens per step: one token's full pass through the layer
@@ -293,6 +307,8 @@ def main():
     ap.add_argument("--fp32-router", action="store_true", help="fp32 router weights (bf16 tokens and experts)")
     ap.add_argument("--swiglu-limit", type=float, default=0.0, help="SwiGLU limit of the routed experts")
     ap.add_argument("--swiglu-limit-shared", type=float, default=0.0, help="SwiGLU limit of the shared expert")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
+                    help="expert weights: bf16, or FP8 E4M3 codes with one E8M0 scale per 128x128 block")
     ap.add_argument("--I", type=int, default=None,
                     help="profiling variant: override both expert widths (small weights, same router)")
     args = ap.parse_args()
@@ -329,7 +345,12 @@ def main():
 
     # ---- inputs (resident in HBM); each rank is a replica with its own tokens -------------
     x, Wr, bias = inputs.make_routing_inputs(rank_config(cfg, rank), router_fp32=args.fp32_router)
-    Wgu, Wd, Wsgu, Wsd = inputs.make_expert_weights(cfg, dev)
+    fp8 = args.weights == "fp8"
+    if fp8:
+        W8 = inputs.make_fp8_expert_weights(cfg, dev)
+        Wgu, Wd, Wsgu, Wsd = W8["W_gate_up"], W8["W_down"], W8["Ws_gate_up"], W8["Ws_down"]
+    else:
+        Wgu, Wd, Wsgu, Wsd = inputs.make_expert_weights(cfg, dev)
     x, Wr = x.to(dev), Wr.to(dev)
     bias = None if bias is None else bias.to(dev)
     shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared, cfg.top_k, cfg.torch_dtype)
@@ -347,6 +368,9 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     def step(xin, yout, routing=False):
+        if fp8:
+            return moe.moe_layer_forward_fp8(xin, Wr, W8, top_k=cfg.top_k, router_bias=bias, y=yout,
+                                             workspace=ws, routing=routing, stream=stream, **layer_options(args))
         return moe.moe_layer_forward(xin, Wr, Wgu, Wd, Wsgu, Wsd, top_k=cfg.top_k, router_bias=bias,
                                      y=yout, workspace=ws, routing=routing, stream=stream,
                                      **layer_options(args))
@@ -358,7 +382,7 @@ def main():
         raise RuntimeError(f"device status {moe.status_string(status)}")
     counts = r.counts.cpu().numpy()
     route_stats = moe.route_stats(ws)
-    alg = algorithmic(cfg, counts)
+    alg = algorithmic(cfg, counts, fp8)
 
     for _ in range(args.warmup):
         flush()
@@ -442,9 +466,10 @@ def main():
             achieved = alg["gate_up_bytes"] / (gu_ms / 1e3) / 1e9
             roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": achieved / peaks["hbm_gbs"]}
-        roof.update({"kernel": "expert_gemm_tc_kernel<gated> (gate/up GEMM + SiLU*up)",
+        roof.update({"kernel": "expert_gemm_tc_kernel<gated%s> (gate/up GEMM + SiLU*up)" % (", fp8" if fp8 else ""),
                      "timing": "CUDA events around each launch, stage-timed pass of the same steps",
-                     "traffic": ncu_traffic("gate_up", cfg.name), "peak_source": peaks["source"],
+                     "traffic": ncu_traffic("gate_up", cfg.name + ("+fp8" if fp8 else "")),
+                     "peak_source": peaks["source"],
                      "ms_per_launch": gu_ms, "algorithmic_bytes": alg["gate_up_bytes"],
                      "algorithmic_flops": alg["gate_up_flops"]})
         layer_s = ms_per_step / 1e3
