@@ -121,6 +121,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the thread sleep until the phase completes (or about 0.5 ms pass)
+// instead of returning at once, so that waiting warps leave the issue slots to the
+// warps that compute.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(500000)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Gives up after kWaitLimitNs,
 // records MOE_ERR_DEVICE_TIMEOUT and returns false; also returns false at once if
 // another thread of the block already gave up (*abort != 0).
@@ -137,6 +152,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctrl* 
         *abort = 1;
         return false;
       }
+    }
+  }
+}
+
+// mbar_wait with sleeping polls (same limit, status and abort behaviour).
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, Ctrl* ctrl,
+                                                volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      set_status(ctrl, MOE_ERR_DEVICE_TIMEOUT);
+      *abort = 1;
+      return false;
     }
   }
 }

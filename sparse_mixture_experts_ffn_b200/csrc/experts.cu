@@ -67,6 +67,7 @@ struct TcParams {
 };
 
 constexpr int kMaxDynSmem = 232448;  // 227 KB per block on sm_100
+constexpr int kConvGroups = 2;       // FP8: converter groups of four warps
 constexpr int kRing = 4;             // item slots between the producer and the other roles
 
 template <bool GATED, int BN, bool W8 = false>
@@ -78,10 +79,14 @@ struct TcCfg {
   // one TMA stage: the weight tiles as loaded (bf16, or FP8 codes), then the token rows
   static constexpr int kBOffset = kMats * (W8 ? kA8Bytes : kABytes);
   static constexpr int kStageBytes = kBOffset + kBBytes;
-  // FP8: stages of converted bf16 weight tiles between the converters and the MMA
+  // FP8: stages of converted bf16 weight tiles plus a copy of the token rows, between the
+  // converters and the MMA.  The converters free each TMA stage as soon as they have read
+  // it, so every TMA stage is either in flight or waiting for conversion.
   static constexpr int kConvStages = W8 ? 2 : 0;
-  static constexpr int kConvBytes = kMats * kABytes;
-  static constexpr int kThreads = W8 ? 320 : 192;
+  static constexpr int kConvBOffset = kMats * kABytes;
+  static constexpr int kConvBytes = kConvBOffset + kBBytes;
+  static constexpr int kThreads = W8 ? 192 + 128 * kConvGroups : 192;
+  static constexpr int kConvMod = kConvStages > 0 ? kConvStages : 1;  // a divisor in every variant
   // tiles of up to 128 tokens stage the output tile [BN][128] bf16 in shared memory for
   // 16-byte stores; 256-token tiles store straight from registers (each warp writes 64
   // contiguous bytes per token) to leave shared memory to the pipeline
@@ -101,6 +106,8 @@ struct TcCfg {
   static_assert(kStages >= 2, "pipeline too shallow");
   static_assert(kStageBytes % 1024 == 0 && kBOffset % 1024 == 0, "stages must keep 1024-byte alignment");
   static_assert(!W8 || BN <= 128, "FP8 weights: staged tiles only");
+  static_assert(kConvStages <= 6 && kStages <= 12, "barrier and scale slots in the aux block");
+  static_assert(kConvBytes % 1024 == 0, "converted stages keep the 1024-byte swizzle alignment");
   static_assert(kTmemNeed <= 512, "accumulators exceed tensor memory");
   static_assert(kSmemBytes <= kMaxDynSmem, "shared memory budget");
   static_assert(BN % 16 == 0 && BN <= 256, "tile width");
@@ -236,18 +243,19 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   }
 }
 
-// Persistent grouped GEMM: 192 threads (320 with FP8 weights), one block per SM.
+// Persistent grouped GEMM: 192 threads (448 with FP8 weights), one block per SM.
 //   warp 0      TMA producer (one lane): weight tiles (gate and up for GATED) and token rows
 //   warp 1      allocates tensor memory; one lane issues the tcgen05 MMAs
 //   warps 2..5  epilogue: tensor memory -> registers -> shared staging tile -> global
-//   warps 6..9  FP8 weights only: code tiles -> bf16 tiles
+//   warps 6..13 FP8 weights only: code tiles -> bf16 tiles, two groups of four warps
+//               taking alternate k-steps
 // Accumulators are double-buffered in tensor memory, so the epilogue of one tile overlaps
 // the main loop of the next.  Items are claimed dynamically: block b starts with item b and
 // then takes the next unclaimed one from a global counter, so blocks that draw short tiles
 // take more of them; the producer publishes each claimed item to the MMA and epilogue warps
 // through a ring of kRing shared-memory slots (index -1 ends the schedule).
 template <bool GATED, int BN, bool W8>
-__global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(W8 ? 192 + 128 * kConvGroups : 192, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
   using C = TcCfg<GATED, BN, W8>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -263,8 +271,8 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint64_t* cfull = reinterpret_cast<uint64_t*>(aux + 256);  // FP8: [kConvStages] converted
-  uint64_t* cempty = cfull + 2;                              // FP8: [kConvStages] consumed
-  volatile uint32_t* sc_stage = reinterpret_cast<volatile uint32_t*>(aux + 288);  // FP8: [kStages]
+  uint64_t* cempty = cfull + 6;                              // FP8: [kConvStages] consumed
+  volatile uint32_t* sc_stage = reinterpret_cast<volatile uint32_t*>(aux + 464);  // FP8: [kStages]
                                                          // scale codes of each stage's tiles
   uint64_t* ring_full = reinterpret_cast<uint64_t*>(aux + 384);  // [kRing]
   uint64_t* ring_empty = ring_full + kRing;                     // [kRing]
@@ -275,7 +283,7 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], W8 ? 4 : 1);  // the MMA commit, or (FP8) the four converter warps
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
@@ -285,10 +293,10 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
     for (int q = 0; q < kRing; ++q) {
       mbar_init(&ring_full[q], 1);
       // the MMA thread and one lane per epilogue (and converter) warp
-      mbar_init(&ring_empty[q], 1 + 4 + (W8 ? 4 : 0));
+      mbar_init(&ring_empty[q], 1 + 4 + (W8 ? 4 * kConvGroups : 0));
     }
     for (int c = 0; c < C::kConvStages; ++c) {
-      mbar_init(&cfull[c], 128);  // every converter thread
+      mbar_init(&cfull[c], 4);    // one lane per warp of the converter group
       mbar_init(&cempty[c], 1);   // the MMA commit
     }
     *abort_flag = 0;
@@ -319,6 +327,10 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
     sc = Sched{tab, tab + G + 1, tab + 2 * G + 1, true};
   }
   const int total = schedule_length(p, sc);
+  // FP8: waiting threads sleep in their polls, leaving the issue slots to the converters
+  auto wait = [&](uint64_t* bar, uint32_t parity) {
+    return W8 ? mbar_wait_sleep(bar, parity, p.ctrl, abort_flag) : mbar_wait(bar, parity, p.ctrl, abort_flag);
+  };
 
   if (warp == 0) {
     // ------------------------------- TMA producer -------------------------------------
@@ -330,6 +342,26 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
     bool ok = true;
     int q = 0;
     uint32_t qphase = 0;
+    // FP8: block scales of an item (one 128-column block per lane, and lane + 32)
+    auto load_scales = [&](const Item& t, uint32_t* g, uint32_t* u) {
+      const int kbn = p.kblocks[t.sh];
+      const int k0 = t.ks * kbn / p.ksplit, k1 = (t.ks + 1) * kbn / p.ksplit;
+      const int c0 = k0 >> 1, nblk = k1 > k0 ? ((k1 - 1) >> 1) - c0 + 1 : 0;
+      const int ld = p.s_ld[t.sh];
+      const uint8_t* sbase = p.scaleA[t.sh] + static_cast<int64_t>(t.sh ? 0 : t.g) * p.s_rows_per_group * ld;
+      const uint8_t* srow_g = sbase + static_cast<int64_t>(t.m) * ld;
+      const uint8_t* srow_u = sbase + static_cast<int64_t>(t.m + p.a_up_offset[t.sh] / kTileM) * ld;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        g[h] = u[h] = 0u;
+        if (lane + 32 * h < nblk) {
+          g[h] = __ldg(srow_g + c0 + lane + 32 * h);
+          if (GATED) u[h] = __ldg(srow_u + c0 + lane + 32 * h);
+        }
+      }
+    };
+    int pf_it = -1;  // FP8: the item whose scales pf_sg / pf_su hold
+    uint32_t pf_sg[2] = {0u, 0u}, pf_su[2] = {0u, 0u};
     // the item after the current one is claimed while the current one streams
     int it = static_cast<int>(blockIdx.x);
     int claimed = (lane == 0) ? static_cast<int>(atomicAdd(p.item_counter, 1u) + gridDim.x) : 0;
@@ -338,7 +370,7 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
       // publish the item (or the end) to the MMA and epilogue warps
       int pub = 1;
       if (lane == 0) {
-        pub = mbar_wait(&ring_empty[q], qphase ^ 1u, p.ctrl, abort_flag) ? 1 : 0;
+        pub = wait(&ring_empty[q], qphase ^ 1u) ? 1 : 0;
         if (pub) {
           ring[q] = it;
           mbar_arrive(&ring_full[q]);
@@ -369,21 +401,24 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
       const int arow = t.sh ? t.m * kTileM : t.g * p.a_rows_per_group + t.m * kTileM;
       const int kb_n = p.kblocks[t.sh];
       const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
-      // FP8: the item's block scales, one 128-column block per lane (and lane + 32)
+      // FP8: the item's block scales, one 128-column block per lane (and lane + 32),
+      // loaded one item ahead so that their latency overlaps the previous item's stream
       uint32_t sg[2] = {0u, 0u}, su[2] = {0u, 0u};
       const int sc0 = kb0 >> 1;  // 128-column scale blocks hold two 64-column k-blocks
       if (W8) {
-        const int ld = p.s_ld[t.sh];
-        const uint8_t* sbase = p.scaleA[t.sh] + static_cast<int64_t>(t.sh ? 0 : t.g) * p.s_rows_per_group * ld;
-        const uint8_t* srow_g = sbase + static_cast<int64_t>(t.m) * ld;
-        const uint8_t* srow_u = sbase + static_cast<int64_t>(t.m + p.a_up_offset[t.sh] / kTileM) * ld;
-        const int nblk = kb1 > kb0 ? ((kb1 - 1) >> 1) - sc0 + 1 : 0;
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          if (lane + 32 * h < nblk) {
-            sg[h] = __ldg(srow_g + sc0 + lane + 32 * h);
-            if (GATED) su[h] = __ldg(srow_u + sc0 + lane + 32 * h);
+        if (pf_it == cur) {
+          sg[0] = pf_sg[0]; sg[1] = pf_sg[1]; su[0] = pf_su[0]; su[1] = pf_su[1];
+        } else {
+          load_scales(t, sg, su);
+        }
+        pf_it = -1;
+        if (it < total) {
+          const Item tn = decode_item<BN>(p, sc, it);
+          if (tn.valid) {
+            load_scales(tn, pf_sg, pf_su);
+            pf_it = it;
           }
+        }
       }
       for (int kb = kb0; kb < kb1; ++kb) {
         unsigned char* st = smem + stage * C::kStageBytes;
@@ -395,7 +430,7 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
         }
         int good = 1;
         if (lane == 0) {
-          good = mbar_wait(&empty[stage], phase ^ 1u, p.ctrl, abort_flag) ? 1 : 0;
+          good = wait(&empty[stage], phase ^ 1u) ? 1 : 0;
           if (good) {
             if (W8) sc_stage[stage] = scw;  // published by the arrive below
             mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
@@ -434,7 +469,7 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
       int q = 0;
       uint32_t qphase = 0;
       while (ok) {
-        if (!mbar_wait(&ring_full[q], qphase, p.ctrl, abort_flag)) break;
+        if (!wait(&ring_full[q], qphase)) break;
         const int it = ring[q];
         mbar_arrive(&ring_empty[q]);
         if (++q == kRing) { q = 0; qphase ^= 1u; }
@@ -443,18 +478,17 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
         if (!t.valid) continue;
         const int n_mma = (t.nvalid + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(kTileM, n_mma);
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, p.ctrl, abort_flag)) break;
+        if (!wait(&tempty[acc], acc_phase ^ 1u)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + acc * C::kAccCols;
         const int kb_n = p.kblocks[t.sh];
         const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, p.ctrl, abort_flag) ||
-              (W8 && !mbar_wait(&cfull[cs], cphase, p.ctrl, abort_flag))) { ok = false; break; }
+          if (!(W8 ? wait(&cfull[cs], cphase) : wait(&full[stage], phase))) { ok = false; break; }
           tc_fence_after();
-          const uint32_t s0 = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t a0 = W8 ? smem_u32(conv + cs * C::kConvBytes) : s0;
-          const uint32_t b0 = s0 + C::kBOffset;
+          const uint32_t s0 = W8 ? smem_u32(conv + cs * C::kConvBytes) : smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t a0 = s0;
+          const uint32_t b0 = s0 + (W8 ? C::kConvBOffset : C::kBOffset);
 #pragma unroll
           for (int kk = 0; kk < kTileK / 16; ++kk) {
             const uint32_t accum = (kb != kb0 || kk) ? 1u : 0u;
@@ -463,11 +497,12 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
             if (GATED)
               mma_bf16(d0 + BN, sw128_kmajor_desc(a0 + C::kABytes + kk * 32), bdesc, idesc, accum);
           }
-          mma_commit(&empty[stage]);
-          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
           if (W8) {
             mma_commit(&cempty[cs]);
             if (++cs == C::kConvStages) { cs = 0; cphase ^= 1u; }
+          } else {
+            mma_commit(&empty[stage]);
+            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
           }
         }
         if (!ok) break;
@@ -479,15 +514,17 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
       mbar_wait_drain(drain, 0, p.ctrl);
     }
   } else if (W8 && warp >= 6) {
-    // ------------------------- FP8 code tiles -> bf16 (warps 6..9) ---------------------
-    const int ct = threadIdx.x - 192;  // 0..127
-    int stage = 0, cs = 0;
-    uint32_t phase = 0, cphase = 0;
+    // ------------------------ FP8 code tiles -> bf16 (warps 6..13) --------------------
+    // Group g converts the block's k-steps n with n % 2 == g, so one group's waits and
+    // fences overlap the other group's conversion.
+    const uint32_t grp = static_cast<uint32_t>(warp - 6) >> 2;  // < kConvGroups
+    const int ct = threadIdx.x - 192 - 128 * static_cast<int>(grp);  // 0..127 within the group
+    uint32_t n = 0;  // k-steps of this block so far, over all items
     int q = 0;
     uint32_t qphase = 0;
     bool ok = true;
     while (ok) {
-      if (!mbar_wait(&ring_full[q], qphase, p.ctrl, abort_flag)) break;
+      if (!wait(&ring_full[q], qphase)) break;
       const int it = ring[q];
       __syncwarp();
       if (lane == 0) mbar_arrive(&ring_empty[q]);
@@ -497,18 +534,27 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
       if (!t.valid) continue;
       const int kb_n = p.kblocks[t.sh];
       const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
-      for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&full[stage], phase, p.ctrl, abort_flag) ||
-            !mbar_wait(&cempty[cs], cphase ^ 1u, p.ctrl, abort_flag)) { ok = false; break; }
+      for (int kb = kb0; kb < kb1; ++kb, ++n) {
+        if (n % kConvGroups != grp) continue;
+        const int stage = static_cast<int>(n % C::kStages), cs = static_cast<int>(n % C::kConvMod);
+        const uint32_t phase = (n / C::kStages) & 1u, cphase = (n / C::kConvMod) & 1u;
+        if (!wait(&full[stage], phase) || !wait(&cempty[cs], cphase ^ 1u)) { ok = false; break; }
         const uint32_t scw = sc_stage[stage];
         const unsigned char* src = smem + stage * C::kStageBytes;
         unsigned char* dst = conv + cs * C::kConvBytes;
         fp8_tile_to_bf16(src, dst, ct, scw & 0xFFu);
         if (GATED) fp8_tile_to_bf16(src + C::kA8Bytes, dst + C::kABytes, ct, (scw >> 8) & 0xFFu);
+        // the token rows, byte for byte (both copies sit at 1024-byte-aligned offsets, so the
+        // 128-byte swizzle TMA wrote them in stays valid)
+        for (int i = ct; i < C::kBBytes / 16; i += 128)
+          reinterpret_cast<uint4*>(dst + C::kConvBOffset)[i] =
+              reinterpret_cast<const uint4*>(src + C::kBOffset)[i];
         fence_proxy_async_smem();  // the tensor cores read these bytes next
-        mbar_arrive(&cfull[cs]);
-        if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
-        if (++cs == C::kConvStages) { cs = 0; cphase ^= 1u; }
+        __syncwarp();              // the warp's reads and writes, then one arrival each
+        if (lane == 0) {
+          mbar_arrive(&empty[stage]);  // the TMA stage may be refilled
+          mbar_arrive(&cfull[cs]);
+        }
       }
     }
   } else {
@@ -521,7 +567,7 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
     int q = 0;
     uint32_t qphase = 0;
     for (;;) {
-      if (!mbar_wait(&ring_full[q], qphase, p.ctrl, abort_flag)) break;
+      if (!wait(&ring_full[q], qphase)) break;
       const int it = ring[q];
       __syncwarp();
       if (lane == 0) mbar_arrive(&ring_empty[q]);
@@ -532,7 +578,7 @@ __global__ void __launch_bounds__(W8 ? 320 : 192, 1) expert_gemm_tc_kernel(const
       if (!GATED)
         for (int n = et; n < BN; n += 128)
           sw[n] = (t.sh || n >= t.nvalid) ? 1.0f : __ldg(p.row_w + t.row0 + n);
-      if (!mbar_wait(&tfull[acc], acc_phase, p.ctrl, abort_flag)) break;
+      if (!wait(&tfull[acc], acc_phase)) break;
       tc_fence_after();
       named_bar_sync(1, 128);  // staging free (previous tile copied out), sw visible
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::kAccCols;
