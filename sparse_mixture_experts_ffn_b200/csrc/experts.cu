@@ -81,8 +81,10 @@ struct TcCfg {
   static constexpr int kStageBytes = kBOffset + kBBytes;
   // FP8: stages of converted bf16 weight tiles plus a copy of the token rows, between the
   // converters and the MMA.  The converters free each TMA stage as soon as they have read
-  // it, so every TMA stage is either in flight or waiting for conversion.
-  static constexpr int kConvStages = W8 ? 2 : 0;
+  // it, so every TMA stage is either in flight or waiting for conversion.  More converted
+  // stages than converter groups let a group start its next step before the MMA has
+  // finished its previous one (16-token tiles; 128-token ones lack the room).
+  static constexpr int kConvStages = W8 ? (BN <= 16 ? (GATED ? 3 : 4) : 2) : 0;
   static constexpr int kConvBOffset = kMats * kABytes;
   static constexpr int kConvBytes = kConvBOffset + kBBytes;
   static constexpr int kThreads = W8 ? 192 + 128 * kConvGroups : 192;
