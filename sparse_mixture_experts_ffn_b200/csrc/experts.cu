@@ -10,9 +10,9 @@
 //
 // FP8 weights (the low-precision expert weights for decode): each weight matrix is
 // E4M3 codes plus one E8M0 power-of-two scale per 128 x 128 block.  TMA brings the codes
-// (half the bytes of bf16); four more warps turn each 128 x 64 code tile into the bf16
-// tile the MMA reads, scale applied, in the layout 128-byte-swizzled TMA would have
-// written.  Every decoded weight is exact in bf16, so the GEMM is the bf16 GEMM of the
+// (half the bytes of bf16); eight more warps, in two groups taking alternate k-blocks, turn
+// each 128 x 64 code tile into the bf16 tile the MMA reads, scale applied, in the layout
+// 128-byte-swizzled TMA would have written.  Every decoded weight is exact in bf16, so the GEMM is the bf16 GEMM of the
 // decoded weights, with bf16 tokens as before.
 // Sources: llm-atlas page "Step-3.5-Flash", "Champs bruts du config.json":
 // moe_intermediate_size 1280, share_expert_dim 1280, hidden_size 4096, norm_expert_weight.
