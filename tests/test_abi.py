@@ -141,3 +141,43 @@ def test_forward_fp8_rejects_bad_arguments_before_any_launch(lib):
     assert call(shape(), codes=(24, 16, 16, 16)) == 1  # codes misaligned
     assert call(shape(), ws_bytes=moe.workspace_bytes(shape()) - 1) == 3
     assert call(shape(T=0)) == 0                      # empty batch: nothing to do
+
+
+C_TYPES = {"int64_t": ctypes.c_int64, "int32_t": ctypes.c_int32, "float": ctypes.c_float,
+           "size_t": ctypes.c_size_t}
+
+
+def header_structs():
+    """{struct name: [(field, C type), ...]} parsed from the typedef'd structs of the header."""
+    text = open(os.path.join(ROOT, "include", "moe_layer.h")).read()
+    out = {}
+    for body, name in re.findall(r"typedef struct \{(.*?)\}\s*(\w+);", text, flags=re.S):
+        fields = []
+        for decl in re.sub(r"/\*.*?\*/", "", body, flags=re.S).split(";"):
+            decl = decl.strip()
+            if not decl:
+                continue
+            m = re.match(r"(const\s+)?(\w+)\s*(\*?)\s*(.*)", decl)
+            ctype = "pointer" if m.group(3) else m.group(2)
+            for f in m.group(4).split(","):
+                fields.append((f.strip().lstrip("*"), ctype))
+        out[name] = fields
+    return out
+
+
+@pytest.mark.parametrize("c_name, py_struct", [
+    ("moe_layer_shape", moe.MoEShape), ("moe_routing_out", moe.MoERoutingOut),
+    ("moe_layer_options", moe.MoEOptions), ("moe_fp8_weights", moe.MoEFp8Weights),
+    ("moe_route_stats", moe.MoERouteStats), ("moe_workspace_layout", moe.MoEWorkspaceLayout)])
+def test_binding_structs_match_the_header(c_name, py_struct):
+    """Every ctypes structure of the binding has the header's fields, in order, with the same
+    C types (pointers as pointers), so that the marshalled bytes are what the library reads."""
+    fields = header_structs()[c_name]
+    py = py_struct._fields_
+    assert [f for f, _ in fields] == [f for f, _ in py], c_name
+    for (f, ctype), (_, pytype) in zip(fields, py):
+        if ctype == "pointer":
+            assert pytype is ctypes.c_void_p, (c_name, f)
+        else:
+            assert ctypes.sizeof(pytype) == ctypes.sizeof(C_TYPES[ctype]), (c_name, f)
+            assert (pytype is ctypes.c_float) == (ctype == "float"), (c_name, f)

@@ -1,0 +1,38 @@
+"""The seeded input generators (CPU): the FP8 expert weights stand for the bf16 draws they
+were cast from, within E4M3's rounding, and are reproducible."""
+import numpy as np
+import torch
+
+import oracle
+from sparse_mixture_experts_ffn_b200 import inputs
+
+
+def test_fp8_weights_round_the_bf16_draws():
+    cfg = inputs.small_config(T=4, H=384, E=3, top_k=2, I=256, I_shared=128)
+    w8 = inputs.make_fp8_expert_weights(cfg)
+    wb = dict(zip(("W_gate_up", "W_down", "Ws_gate_up", "Ws_down"), inputs.make_expert_weights(cfg)))
+    for name, (q, s) in w8.items():
+        ref = wb[name].double().numpy()
+        qn, sn = q.numpy(), s.numpy()
+        mats = [(qn[e], sn[e], ref[e]) for e in range(qn.shape[0])] if qn.ndim == 3 else [(qn, sn, ref)]
+        for qm, sm, rm in mats:
+            d = oracle.dequant_e4m3(qm, sm)
+            assert not np.isnan(d).any(), name
+            # each block: scale = 2^ceil(log2(amax / 448)), so amax / scale lies in (224, 448]
+            scale = 2.0 ** (sm.astype(np.float64) - 127)
+            blocks = np.abs(rm).reshape(sm.shape[0], 128, sm.shape[1], 128).max(axis=(1, 3))
+            assert np.all(blocks / scale <= 448) and np.all(blocks / scale > 224), name
+            # E4M3 keeps 4 significant bits: nearest rounding is within 2^-4 relative above
+            # its normal range (2^-6 of the scale) and within half its subnormal step below
+            big = np.abs(rm) >= np.kron(scale, np.ones((128, 128))) * 2.0 ** -6
+            err = np.abs(d - rm)
+            assert np.all(err[big] <= np.abs(rm[big]) * 2.0 ** -4), name
+            assert np.all(err[~big] <= np.kron(scale, np.ones((128, 128)))[~big] * 2.0 ** -10), name
+
+
+def test_fp8_weights_are_reproducible():
+    cfg = inputs.small_config(T=4, H=256, E=2, top_k=1, I=128, I_shared=128)
+    a, b = inputs.make_fp8_expert_weights(cfg), inputs.make_fp8_expert_weights(cfg)
+    for k in a:
+        for u, v in zip(a[k], b[k]):
+            assert torch.equal(u, v), k
