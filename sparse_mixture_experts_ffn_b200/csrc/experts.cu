@@ -110,6 +110,7 @@ struct TcCfg {
   static_assert(!W8 || BN <= 128, "FP8 weights: staged tiles only");
   static_assert(kConvStages <= 6 && kStages <= 12, "barrier and scale slots in the aux block");
   static_assert(kConvBytes % 1024 == 0, "converted stages keep the 1024-byte swizzle alignment");
+  static_assert(kStages >= kConvStages, "the converters' wait order relies on it");
   static_assert(kTmemNeed <= 512, "accumulators exceed tensor memory");
   static_assert(kSmemBytes <= kMaxDynSmem, "shared memory budget");
   static_assert(BN % 16 == 0 && BN <= 256, "tile width");
@@ -540,7 +541,11 @@ __global__ void __launch_bounds__(W8 ? 192 + 128 * kConvGroups : 192, 1) expert_
         if (n % kConvGroups != grp) continue;
         const int stage = static_cast<int>(n % C::kStages), cs = static_cast<int>(n % C::kConvMod);
         const uint32_t phase = (n / C::kStages) & 1u, cphase = (n / C::kConvMod) & 1u;
-        if (!wait(&full[stage], phase) || !wait(&cempty[cs], cphase ^ 1u)) { ok = false; break; }
+        // the converted stage first: once the MMA has consumed step n - kConvStages, every
+        // earlier use of this TMA stage (n - kStages <= n - kConvStages) has completed, so
+        // the parity wait on it below cannot mistake an older phase for this one, whichever
+        // group took the stage's previous use
+        if (!wait(&cempty[cs], cphase ^ 1u) || !wait(&full[stage], phase)) { ok = false; break; }
         const uint32_t scw = sc_stage[stage];
         const unsigned char* src = smem + stage * C::kStageBytes;
         unsigned char* dst = conv + cs * C::kConvBytes;
