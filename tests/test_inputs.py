@@ -36,3 +36,20 @@ def test_fp8_weights_are_reproducible():
     for k in a:
         for u, v in zip(a[k], b[k]):
             assert torch.equal(u, v), k
+
+
+def test_bench_algorithmic_bytes_closed_form():
+    """The benchmark's algorithmic byte and FLOP counts, against their closed forms for a
+    decode batch: bf16 weights at 2 bytes, FP8 at 1 byte plus one scale byte per 128x128 block."""
+    import bench
+    cfg = inputs.CONFIGS["decode_t4"]
+    counts = np.zeros(cfg.E, np.int64)
+    counts[:32] = 1
+    H, I, Is, E, T, k = cfg.H, cfg.I, cfg.I_shared, cfg.E, cfg.T, cfg.top_k
+    b = bench.algorithmic(cfg, counts)
+    f = bench.algorithmic(cfg, counts, fp8=True)
+    weights = 32 * 3 * H * I + 3 * H * Is
+    assert b["layer_bytes"] == 2 * weights + 2 * (E * H + 2 * T * H)
+    assert f["layer_bytes"] == weights + weights // (128 * 128) + 2 * (E * H + 2 * T * H)
+    assert b["layer_flops"] == f["layer_flops"] == 2 * T * E * H + T * k * 6 * H * I + T * 6 * H * Is
+    assert b["gate_up_bytes"] == 2 * (32 * 2 * I * H + 2 * Is * H) + 2 * (T * k * H + T * H + T * k * I + T * Is)

@@ -615,3 +615,29 @@ def test_fp8_layer_equals_the_bf16_layer_on_the_decoded_weights():
     y_ref = oracle.moe_tokens(xb, idx, w64, _as_bf16_bits(decode(*gu)), _as_bf16_bits(np.zeros((E, H, I))),
                               _as_bf16_bits(decode(*sgu)), _as_bf16_bits(decode(*sdn)))
     assert np.array_equal(y_sh, y_ref)
+
+
+def test_e8m0_nan_code_and_negative_zero_codes():
+    """E8M0 255 is NaN (like the library's float8_e8m0fnu); a -0 code times any scale is -0."""
+    q = np.full((1, 256), 0x80, np.uint8)
+    got = oracle.dequant_e4m3(q, np.array([[255, 3]], np.uint8))
+    assert np.isnan(got[0, :128]).all() and np.isnan(torch_e8m0(np.array([255], np.uint8))).all()
+    assert (got[0, 128:] == 0).all() and (np.signbit(got[0, 128:])).all()
+
+
+def test_fp8_layer_token_subset_and_permutation():
+    """Invariants of the FP8 layer: a token subset gives the same rows as the full batch, and
+    permuting the tokens (with their routing) permutes the outputs."""
+    rng = np.random.default_rng(12)
+    E, H, I, Is, T, k = 3, 256, 128, 128, 6, 2
+    gu, dn, sgu, sdn = _fp8_layer(rng, E, H, I, Is)
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    idx = np.array([[0, 1], [1, 2], [0, 2], [2, 0], [1, 0], [0, 1]], np.int32)
+    w64 = rng.random((T, k))
+    full = oracle.moe_tokens_fp8(xb, idx, w64, gu, dn, sgu, sdn)
+    sub = oracle.moe_tokens_fp8(xb, idx, w64, gu, dn, sgu, sdn, tokens=[4, 1])
+    assert np.array_equal(sub, full[[4, 1]])
+    perm = rng.permutation(T)
+    permuted = oracle.moe_tokens_fp8(np.ascontiguousarray(xb[perm]), idx[perm], w64[perm], gu, dn, sgu, sdn)
+    assert np.array_equal(permuted, full[perm])
