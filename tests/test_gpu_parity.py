@@ -502,3 +502,23 @@ def test_bounded_wait_times_out_with_a_readable_status():
     assert 1.5 < time.perf_counter() - t0 < 30.0
     cfg = inputs.small_config(T=64, H=256, E=16, top_k=4, I=128, I_shared=128)
     check_full(to_device(inputs.make_inputs(cfg, "cuda")), cfg.top_k, "after a timeout")
+
+
+def test_fp8_weights_layer_as_configured_decode():
+    """FP8 expert weights under the last layers' configuration at decode size: fp32 router
+    weights, sigmoid router with the routing factor 3 and a selection bias, SwiGLU limits 7
+    (routed) and 16 (shared)."""
+    import oracle
+    from conftest import to_oracle
+    cfg = inputs.CONFIGS["decode_t4"]
+    d = fp8_inputs(cfg)
+    d["bias"] = torch.linspace(-0.05, 0.05, cfg.E, dtype=torch.float32, device="cuda")
+    g = torch.Generator().manual_seed(cfg.seed + 31)
+    d["W_router"] = (torch.randn(cfg.E, cfg.H, generator=g) * cfg.r_std).cuda()
+    opts = dict(router="sigmoid", routed_scaling_factor=3.0, swiglu_limit=7.0, swiglu_limit_shared=16.0)
+    y, r = moe.moe_layer_forward_fp8(d["x"], d["W_router"], d["fp8"], top_k=cfg.top_k, router_bias=d["bias"],
+                                     **opts)
+    ref = oracle_routing(d, cfg.top_k, router="sigmoid", scale=3.0)
+    assert_routing_exact(r, ref, cfg.E)
+    y_ref = oracle_y_fp8(d, ref, swiglu_limit=7.0, swiglu_limit_shared=16.0)
+    assert_y_close(y, y_ref, "decode_t4 fp8 as configured")
