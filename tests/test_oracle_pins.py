@@ -641,3 +641,97 @@ def test_fp8_layer_token_subset_and_permutation():
     perm = rng.permutation(T)
     permuted = oracle.moe_tokens_fp8(np.ascontiguousarray(xb[perm]), idx[perm], w64[perm], gu, dn, sgu, sdn)
     assert np.array_equal(permuted, full[perm])
+
+
+# --------------------------------------------------------------------------------------
+# the routed-expert gather and the weighted combine, restated with numpy
+# --------------------------------------------------------------------------------------
+def _numpy_layer(x, idx, w, Wgu, Wd, Wsgu=None, Wsd=None):
+    """y_t = sum_j w[t, j] * FFN_{idx[t, j]}(x_t) + shared(x_t), written independently of the
+    oracle with numpy fp64 matmuls: for each expert, the (token, slot) pairs routed to it
+    are found with numpy and their weighted FFN rows are scattered back with np.add.at
+    (the definition of the layer on the llm-atlas page "Step-3.5-Flash", "Champs bruts du
+    config.json": moe_top_k, norm_expert_weight; the weights are inputs here)."""
+    T, H = x.shape
+    y = np.zeros((T, H))
+    for e in np.unique(idx):
+        tok, slot = np.nonzero(idx == e)
+        np.add.at(y, tok, w[tok, slot][:, None] * _numpy_ffn(x[tok], Wgu[e], Wd[e]))
+    if Wsgu is not None:
+        y += _numpy_ffn(x, Wsgu, Wsd)
+    return y
+
+
+def _hand_routing(T, E, k, rng):
+    """Distinct experts per token in a scrambled order (no slot j holds expert j) with
+    deliberately unequal weights."""
+    idx = np.empty((T, k), np.int32)
+    for t in range(T):
+        while True:
+            c = rng.choice(E, size=k, replace=False)
+            if not np.any(c == np.arange(k)):
+                break
+        idx[t] = np.sort(c)[::-1]  # descending, unlike the oracle's own ascending routing
+    w = rng.dirichlet(np.linspace(0.5, 4.0, k), size=T)
+    return idx, w
+
+
+@pytest.mark.parametrize("case", ["tiny_f32_t64", "bf16_k3_of_8", "decode_shaped_bf16"])
+@pytest.mark.parametrize("routing", ["oracle", "hand"])
+def test_routed_gather_matches_a_numpy_restatement(case, routing):
+    """The routed experts' gather (expert idx[t, j] with weight w[t, j]) and the combine of
+    oracle.moe_tokens against an independent numpy restatement, with top_k < E and distinct
+    experts, so that reading the slot index j as the expert, or pairing weights with the
+    wrong slot, fails.  Cases: the tiny fp32 workload (top-2 of 16); bf16 top-3 of 8;
+    decode-shaped routing (H = 4096, top-8 of 288) with narrow experts."""
+    rng = np.random.default_rng(21)
+    if case == "tiny_f32_t64":
+        cfg = inputs.CONFIGS["tiny_f32_t64"]
+    elif case == "bf16_k3_of_8":
+        cfg = _small("bf16", T=40, H=128, E=8, top_k=3, I=64, I_shared=32, w_std=0.1)
+    else:
+        cfg = inputs.small_config(T=4, H=4096, E=288, top_k=8, I=32, I_shared=32, seed=1, w_std=0.05)
+    d = inputs.make_inputs(cfg)
+    xo = to_oracle(d["x"])
+    if routing == "oracle":
+        s = oracle.router_scores(xo, to_oracle(d["W_router"]))
+        idx, _, w64 = oracle.route(s, cfg.top_k)
+    else:
+        idx, w64 = _hand_routing(cfg.T, cfg.E, cfg.top_k, rng)
+    assert cfg.top_k < cfg.E
+    assert len(np.unique(idx.ravel())) > cfg.top_k  # tokens use different experts
+    args = [to_oracle(d[k]) for k in ("W_gate_up", "W_down", "Ws_gate_up", "Ws_down")]
+    got = oracle.moe_tokens(xo, idx, w64, *args)
+    want = _numpy_layer(_f64(d["x"]), idx, w64, _f64(d["W_gate_up"]), _f64(d["W_down"]),
+                        _f64(d["Ws_gate_up"]), _f64(d["Ws_down"]))
+    rel = np.abs(got - want).max() / np.abs(want).max()
+    assert rel <= 1e-5, rel
+    # the pin separates the experts: treating slot j as expert j, or reversing the weights'
+    # pairing with the slots, moves the output far outside the tolerance
+    wrong_e = _numpy_layer(_f64(d["x"]), np.tile(np.arange(cfg.top_k, dtype=np.int32), (cfg.T, 1)), w64,
+                           _f64(d["W_gate_up"]), _f64(d["W_down"]), _f64(d["Ws_gate_up"]), _f64(d["Ws_down"]))
+    wrong_w = _numpy_layer(_f64(d["x"]), idx, w64[:, ::-1], _f64(d["W_gate_up"]), _f64(d["W_down"]),
+                           _f64(d["Ws_gate_up"]), _f64(d["Ws_down"]))
+    for wrong in (wrong_e, wrong_w):
+        assert np.abs(wrong - want).max() / np.abs(want).max() > 1e-3
+
+
+def test_fp8_routed_gather_matches_a_numpy_restatement():
+    """oracle.moe_tokens_fp8 against the numpy restatement on weights decoded by the library's
+    E4M3 / E8M0 decoders (block expansion per matrix), with a hand routing of distinct
+    experts in scrambled slots and unequal weights."""
+    rng = np.random.default_rng(22)
+    E, H, I, Is, T, k = 6, 256, 128, 128, 7, 3
+    gu, dn, sgu, sdn = _fp8_layer(rng, E, H, I, Is)
+
+    def decode(q, s):
+        if q.ndim == 3:
+            return np.stack([decode(q[e], s[e]) for e in range(q.shape[0])])
+        return torch_e4m3(q) * np.kron(torch_e8m0(s), np.ones((128, 128)))[: q.shape[0], : q.shape[1]]
+
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    idx, w64 = _hand_routing(T, E, k, rng)
+    got = oracle.moe_tokens_fp8(xb, idx, w64, gu, dn, sgu, sdn)
+    want = _numpy_layer(x.double().numpy(), idx, w64, decode(*gu), decode(*dn), decode(*sgu), decode(*sdn))
+    assert np.abs(got - want).max() / np.abs(want).max() <= 1e-5
