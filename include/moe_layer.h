@@ -251,8 +251,12 @@ MOE_API int64_t moe_layer_launch_count(void);
  * experts of each token (ascending index, same certified selection) and their
  * renormalised softmax weights -- and writes
  *   topk_idx [T, top_k] int32 and topk_w [T, top_k] fp32 (device pointers, caller-owned).
- * x, W_router and router_bias are as for moe_layer_forward(); the I and I_shared fields
- * of the shape are not used.
+ * x, W_router and router_bias are as for moe_layer_forward() without options: W_router has
+ * the shape's dtype (fp32 router weights with bf16 tokens are not accepted here, since
+ * nothing tells this call they are fp32), and the router is the softmax router, with
+ * router_bias added to the score for both the selection and the weights.  The sigmoid
+ * router of moe_layer_forward_ex() is not available through this entry point.  The I and
+ * I_shared fields of the shape are not used.
  *
  * Scratch: a 16 MiB device array inside this library (present on every GPU that loads the
  * library, until the process exits).  The call needs about T * (28 * E + 8) bytes of it

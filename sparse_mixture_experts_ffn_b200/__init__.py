@@ -164,20 +164,22 @@ def moe_layer_forward(x, W_router, W_gate_up, W_down, Ws_gate_up=None, Ws_down=N
                       router_bias=None, y=None, workspace=None, routing=True, stream=None,
                       swiglu_limit=0.0, swiglu_limit_shared=0.0, router="softmax",
                       routed_scaling_factor=1.0):
-    # W_router may be fp32 while the layer is bf16 (fp32 router weights)
     """Run the MoE layer on the device.  Returns (y, Routing or None).
 
     Shapes: x [T,H], W_router [E,H], W_gate_up [E,2I,H], W_down [E,H,I], Ws_gate_up
     [2Is,H], Ws_down [H,Is] (or both None), router_bias [E] fp32 or None.  All CUDA,
-    contiguous, same dtype (bf16 or fp32).  swiglu_limit / swiglu_limit_shared: SwiGLU
+    contiguous, on x's device, same dtype (bf16 or fp32); W_router may be fp32 with bf16
+    tokens (fp32 router weights).  Mismatched shapes, dtypes or devices raise ValueError
+    before anything is launched.  swiglu_limit / swiglu_limit_shared: SwiGLU
     limits of the routed / shared experts (gate <= L, up in [-L, L]; 0 = none).
     router="sigmoid": sigmoid scores, router_bias for the selection only, weights
     routed_scaling_factor * p / sum p (the default "softmax" ignores the factor).
     """
+    if W_gate_up.dim() != 3 or (Ws_gate_up is not None and Ws_gate_up.dim() != 2):
+        raise ValueError("W_gate_up must be [E, 2I, H] and Ws_gate_up [2Is, H]")
     I = W_gate_up.shape[1] // 2
     Is = 0 if Ws_gate_up is None else Ws_gate_up.shape[0] // 2
-    tensors = (("W_gate_up", W_gate_up), ("W_down", W_down), ("Ws_gate_up", Ws_gate_up), ("Ws_down", Ws_down))
-    return _forward("moe_layer_forward_ex", (W_gate_up, W_down, Ws_gate_up, Ws_down), tensors, x, W_router, I, Is,
+    return _forward("moe_layer_forward_ex", (W_gate_up, W_down, Ws_gate_up, Ws_down), x, W_router, I, Is,
                     top_k, router_bias, y, workspace, routing, stream, swiglu_limit, swiglu_limit_shared, router,
                     routed_scaling_factor)
 
@@ -198,27 +200,87 @@ def moe_layer_forward_fp8(x, W_router, weights, *, top_k, router_bias=None, y=No
     for pair in (gu, dn, sgu, sdn):
         if pair is not None and (pair[0].dtype != torch.uint8 or pair[1].dtype != torch.uint8):
             raise ValueError("FP8 weights are (codes, scales) pairs of uint8 tensors")
+    if gu[0].dim() != 3 or (sgu is not None and sgu[0].dim() != 2):
+        raise ValueError("W_gate_up codes must be [E, 2I, H] and Ws_gate_up codes [2Is, H]")
     I = gu[0].shape[1] // 2
     Is = 0 if sgu is None else sgu[0].shape[0] // 2
-    parts = (gu, dn, sgu, sdn)
-    names = ("W_gate_up", "W_down", "Ws_gate_up", "Ws_down")
-    tensors = tuple((f"{n}{suffix}", None if pr is None else pr[i])
-                    for n, pr in zip(names, parts) for i, suffix in ((0, ""), (1, "_scale")))
-    return _forward("moe_layer_forward_fp8", parts, tensors, x, W_router, I, Is, top_k, router_bias, y,
+    return _forward("moe_layer_forward_fp8", (gu, dn, sgu, sdn), x, W_router, I, Is, top_k, router_bias, y,
                     workspace, routing, stream, swiglu_limit, swiglu_limit_shared, router,
                     routed_scaling_factor)
 
 
-def _forward(entry, weights, tensors, x, W_router, I, Is, top_k, router_bias, y, workspace, routing, stream,
+def _check_args(x, W_router, router_bias, y, weights, I, Is, fp8: bool):
+    """Validate shapes, dtypes and devices before anything reaches the C ABI, which sees only
+    pointers: a mismatch there would make the kernels read past an allocation.  Raises
+    ValueError.  ``weights`` are (W_gate_up, W_down, Ws_gate_up, Ws_down): tensors in x's
+    dtype, or (codes, scales) uint8 pairs for FP8 weights (shared pair None without a
+    shared expert)."""
+    import torch
+
+    def shape_of(t):
+        return tuple(t.shape)
+
+    if x.dim() != 2:
+        raise ValueError(f"x must be [T, H], got {shape_of(x)}")
+    T, H = x.shape
+    if x.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError(f"x must be bf16 or fp32, got {x.dtype}")
+    if fp8 and x.dtype != torch.bfloat16:
+        raise ValueError("FP8 expert weights need bf16 tokens")
+    if W_router.dim() != 2 or W_router.shape[1] != H:
+        raise ValueError(f"W_router must be [E, {H}], got {shape_of(W_router)}")
+    E = W_router.shape[0]
+    router_dtypes = (x.dtype, torch.float32) if x.dtype == torch.bfloat16 else (x.dtype,)
+    if W_router.dtype not in router_dtypes:
+        raise ValueError(f"W_router must be {x.dtype}" + (" or fp32" if len(router_dtypes) > 1 else "") +
+                         f", got {W_router.dtype}")
+    if router_bias is not None and (router_bias.dtype != torch.float32 or shape_of(router_bias) != (E,)):
+        raise ValueError(f"router_bias must be fp32 [{E}], got {router_bias.dtype} {shape_of(router_bias)}")
+    if y is not None and (y.dtype != x.dtype or shape_of(y) != (T, H)):
+        raise ValueError(f"y must be {x.dtype} [{T}, {H}], got {y.dtype} {shape_of(y)}")
+    Wgu, Wd, Wsgu, Wsd = weights
+    if (Wsgu is None) != (Wsd is None):
+        raise ValueError("give both shared-expert matrices or neither")
+    mats = [("W_gate_up", Wgu, (E, 2 * I, H)), ("W_down", Wd, (E, H, I))]
+    if Wsgu is not None:
+        mats += [("Ws_gate_up", Wsgu, (2 * Is, H)), ("Ws_down", Wsd, (H, Is))]
+    checked = [("x", x), ("W_router", W_router), ("router_bias", router_bias), ("y", y)]
+    for name, w, want in mats:
+        if w is None:
+            raise ValueError(f"{name} is required")
+        if fp8:
+            codes, scales = w
+            sshape = want[:-2] + tuple(-(-n // 128) for n in want[-2:])
+            for part, t, shp in (("codes", codes, want), ("scales", scales, sshape)):
+                if t.dtype != torch.uint8 or shape_of(t) != shp:
+                    raise ValueError(f"{name} {part} must be uint8 {list(shp)}, got {t.dtype} {shape_of(t)}")
+            checked += [(name, codes), (name + "_scale", scales)]
+        else:
+            if w.dtype != x.dtype or shape_of(w) != want:
+                raise ValueError(f"{name} must be {x.dtype} {list(want)}, got {w.dtype} {shape_of(w)}")
+            checked.append((name, w))
+    for name, t in checked:
+        if t is None:
+            continue
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if t.device != x.device:
+            raise ValueError(f"{name} is on {t.device}, x on {x.device}")
+    if not x.is_cuda:
+        raise ValueError("the tensors must be CUDA tensors (the layer runs only on the GPU)")
+
+
+def _forward(entry, weights, x, W_router, I, Is, top_k, router_bias, y, workspace, routing, stream,
              swiglu_limit, swiglu_limit_shared, router, routed_scaling_factor):
     import torch
+    _check_args(x, W_router, router_bias, y, weights, I, Is, entry == "moe_layer_forward_fp8")
+    if workspace is not None and (workspace.device != x.device or workspace.dtype != torch.uint8
+                                  or not workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous uint8 tensor on x's device")
     lib = load_library()
     T, H = x.shape
     E = W_router.shape[0]
     shape = make_shape(T, H, E, I, Is, top_k, x.dtype)
-    for name, t in (("x", x), ("W_router", W_router), ("router_bias", router_bias)) + tuple(tensors):
-        if t is not None and (not t.is_cuda or not t.is_contiguous()):
-            raise ValueError(f"{name} must be a contiguous CUDA tensor")
     if y is None:
         y = torch.empty_like(x)
     if workspace is None:

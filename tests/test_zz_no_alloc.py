@@ -57,6 +57,33 @@ def test_noalloc_routing_matches_forward(lib, case):
         assert float(rel.max()) <= W_REL_TOL, f"call {call}: weights differ by {float(rel.max()):.2e}"
 
 
+def test_noalloc_routing_with_a_router_bias_matches_the_oracle(lib):
+    """The skewed long-prefill workload's router bias (added to the scores, for the selection
+    and the weights) on a decode-sized batch: indices bit-exact against the oracle's exact
+    routing, weights within the routing-weight tolerance, on two calls in a row."""
+    from helpers import oracle_routing
+    big = inputs.CONFIGS["prefill_t16384_skew"]
+    cfg = inputs.with_sizes(big, T=4)
+    x, Wr, bias = inputs.make_routing_inputs(cfg)
+    assert bias is not None
+    d = dict(x=x.cuda(), W_router=Wr.cuda(), bias=bias.cuda())
+    ref = oracle_routing(d, cfg.top_k)
+    shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared, cfg.top_k, cfg.torch_dtype)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for call in range(2):
+        idx = torch.full((cfg.T, cfg.top_k), -1, dtype=torch.int32, device="cuda")
+        w = torch.full((cfg.T, cfg.top_k), -1.0, dtype=torch.float32, device="cuda")
+        rc = lib.moe_layer_route_noalloc(ctypes.byref(shape), ctypes.c_void_p(d["x"].data_ptr()),
+                                         ctypes.c_void_p(d["W_router"].data_ptr()),
+                                         ctypes.c_void_p(d["bias"].data_ptr()),
+                                         ctypes.c_void_p(idx.data_ptr()), ctypes.c_void_p(w.data_ptr()), stream)
+        assert rc == moe.MOE_OK, moe.status_string(rc)
+        torch.cuda.synchronize()
+        assert np.array_equal(idx.cpu().numpy(), ref["idx"]), f"call {call}: indices differ"
+        rel = np.abs(w.cpu().numpy().astype(np.float64) - ref["w64"]) / np.abs(ref["w64"])
+        assert float(rel.max()) <= W_REL_TOL, f"call {call}: weights differ by {float(rel.max()):.2e}"
+
+
 def test_noalloc_rejects_batches_beyond_its_scratch(lib):
     shape = moe.make_shape(100000, 4096, 288, 1280, 1280, 8, torch.bfloat16)
     P = ctypes.c_void_p
