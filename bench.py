@@ -50,62 +50,96 @@ def log(*a):
 # clocks during the timed region
 # ------------------------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock, power and clock-event reasons of one GPU, read through NVML (read-only
+    queries) every ``period_s`` in a background thread while the ``with`` block runs.
+    Falls back to ``nvidia-smi -lms`` if NVML cannot be loaded."""
+    REASONS = {  # NVML clock-event reason bits that the run record names
+        0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown",
+    }
     FIELDS = ("clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
               "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
               "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, period_s: float = 0.005):
         self.dev = device_index
+        self.period = period_s
+        self.samples = []  # (sm_mhz, sm_max_mhz, reason names)
         self.proc = None
-        self.lines = []
+        self._stop = threading.Event()
+        self._t = None
+        self.source = None
+
+    def _uuid(self):
+        uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+        return uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
 
     def __enter__(self):
         try:
-            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
-            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self._uuid())
+            smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+
+            def poll():
+                while not self._stop.is_set():
+                    try:
+                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        bits = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((float(sm), float(smax),
+                                             [n for b, n in self.REASONS.items() if bits & b]))
+                    except Exception:  # pragma: no cover - a failed query is skipped
+                        pass
+                    self._stop.wait(self.period)
+            self.source = f"nvml every {self.period * 1e3:.0f} ms"
+            self._t = threading.Thread(target=poll, daemon=True)
+            self._t.start()
+            return self
+        except Exception as e:  # pragma: no cover - no NVML on this host
+            log("NVML unavailable, falling back to nvidia-smi:", e)
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", sel, "--query-gpu=" + ",".join(self.FIELDS),
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                ["nvidia-smi", "-i", self._uuid(), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "10"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self._t = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi -lms 10"
+            self._t = threading.Thread(target=self._read_smi, daemon=True)
             self._t.start()
         except Exception as e:  # pragma: no cover - no nvidia-smi
             log("clock sampler unavailable:", e)
             self.proc = None
         return self
 
-    def _read(self):
+    def _read_smi(self):
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            parts = [q.strip() for q in line.strip().split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                self.samples.append((float(parts[0]), float(parts[1]),
+                                     [n for n, v in zip(names, parts[4:]) if v.lower() == "active"]))
+            except ValueError:
+                continue
 
     def __exit__(self, *exc):
+        self._stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self._t is not None:
             self._t.join(timeout=2)
 
-    def summary(self):
-        sm, smax, reasons = [], [], set()
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) != len(self.FIELDS):
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for name, v in zip(names, parts[4:]):
-                if v.lower() == "active":
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+    def summary(self, since: int = 0):
+        """Median SM clock, the max clock and every reason seen, over samples[since:]."""
+        rows = self.samples[since:]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted({n for r in rows for n in r[2]}), "samples": len(rows), "source": self.source}
 
 
 # ------------------------------------------------------------------------------------------
@@ -232,34 +266,45 @@ def oracle_step(h, cfg, tokens, opts=None):
     return oracle.moe_tokens(x, idx, w64, h["W_gate_up"], h["W_down"], h["Ws_gate_up"], h["Ws_down"], **lim)
 
 
+def sample_tokens(cfg) -> list:
+    """The bounded token sample that the oracle times: the first min(T, 8) tokens of the
+    workload (the whole batch of the T = 4 decode)."""
+    return list(range(min(cfg.T, 8)))
+
+
+def host_inputs(cfg, args, dev):
+    """The workload's inputs for the oracle, as host arrays (weights drawn on the GPU when
+    there is one, as the CUDA path draws them)."""
+    x, Wr, bias = inputs.make_routing_inputs(cfg, router_fp32=args.fp32_router)
+    if args.weights == "fp8":
+        d = dict(x=x, W_router=Wr, bias=bias, **inputs.make_fp8_expert_weights(cfg, dev))
+    else:
+        Wgu, Wd, Wsgu, Wsd = inputs.make_expert_weights(cfg, dev)
+        d = dict(x=x, W_router=Wr, bias=bias, W_gate_up=Wgu, W_down=Wd, Ws_gate_up=Wsgu, Ws_down=Wsd)
+    return host_arrays(d)
+
+
 def run_reference(args, cfg):
+    """The reference arm: the CPU oracle as it stands, timed on the host cores; each step is
+    one pass of the whole layer over the workload's bounded token sample."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     import oracle
     oracle.build()
-    d = inputs.make_inputs(cfg, "cpu") if cfg.T * cfg.H * cfg.E < 5e7 else None
-    if d is not None and args.fp32_router:
-        d["W_router"] = inputs.make_routing_inputs(cfg, router_fp32=True)[1]
-    if d is None or args.weights == "fp8":
-        x, Wr, bias = inputs.make_routing_inputs(cfg, router_fp32=args.fp32_router)
-        dev = "cuda" if torch.cuda.is_available() else "cpu"
-        if args.weights == "fp8":
-            d = dict(x=x, W_router=Wr, bias=bias, **inputs.make_fp8_expert_weights(cfg, dev))
-        else:
-            Wgu, Wd, Wsgu, Wsd = inputs.make_expert_weights(cfg, dev)
-            d = dict(x=x, W_router=Wr, bias=bias, W_gate_up=Wgu, W_down=Wd, Ws_gate_up=Wsgu, Ws_down=Wsd)
-    h = host_arrays(d)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    h = host_inputs(cfg, args, dev)
     cores = len(os.sched_getaffinity(0))
-    per_step = 1  # tokens per step: one token's full pass through the layer
-    for i in range(args.warmup):
-        oracle_step(h, cfg, [i % cfg.T], layer_options(args))
+    tokens = sample_tokens(cfg)
+    for _ in range(args.warmup):
+        oracle_step(h, cfg, tokens, layer_options(args))
     t0 = time.perf_counter()
-    for i in range(args.steps):
-        oracle_step(h, cfg, [i % cfg.T], layer_options(args))
+    for _ in range(args.steps):
+        oracle_step(h, cfg, tokens, layer_options(args))
     dt = time.perf_counter() - t0
-    value = per_step * args.steps / dt
-    sample = f"{per_step} token of {cfg.name} per step (exact router over {cfg.E} experts, top-{cfg.top_k}, {cfg.top_k} routed + 1 shared expert FFNs)"
+    value = len(tokens) * args.steps / dt
+    sample = (f"{len(tokens)} tokens of {cfg.name} per step (tokens 0..{len(tokens) - 1}): exact router over "
+              f"{cfg.E} experts, top-{cfg.top_k}, routed + shared expert FFNs in fp64")
     line = {"metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
@@ -272,78 +317,77 @@ def run_reference(args, cfg):
     return 0
 
 
-def cpu_baseline(h, cfg, opts=None, budget_s=10.0):
+def cpu_baseline(h, cfg, opts=None, budget_s=8.0):
+    """The oracle on the host cores, repeated over the workload's bounded token sample for
+    about ``budget_s`` seconds (at least twice)."""
     import oracle
     cores = len(os.sched_getaffinity(0))
-    tokens = list(range(min(cfg.T, 8)))
+    tokens = sample_tokens(cfg)
+    oracle_step(h, cfg, tokens, opts)  # warm-up: page in the weights
     n, t0 = 0, time.perf_counter()
     while True:
         oracle_step(h, cfg, tokens, opts)
         n += 1
-        if time.perf_counter() - t0 >= budget_s:
+        if n >= 2 and time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
     return {"value": len(tokens) * n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{len(tokens)} tokens of {cfg.name} x {n} repetitions ({dt:.1f} s): exact router over "
-                      f"{cfg.E} experts, top-{cfg.top_k}, routed + shared expert FFNs in fp64"}
+            "sample": f"{len(tokens)} tokens of {cfg.name} (tokens 0..{len(tokens) - 1}) x {n} repetitions "
+                      f"({dt:.1f} s): exact router over {cfg.E} experts, top-{cfg.top_k}, routed + shared "
+                      f"expert FFNs in fp64"}
 
 
 # ------------------------------------------------------------------------------------------
 # the CUDA path
 # ------------------------------------------------------------------------------------------
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=None)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.CONFIGS))
-    ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--T", type=int, default=None, help="profiling variant: override the token count")
-    ap.add_argument("--E", type=int, default=None, help="profiling variant: override the expert count")
-    ap.add_argument("--router", default="softmax", choices=["softmax", "sigmoid"],
-                    help="router mode (sigmoid: the router as configured, bias for the selection only)")
-    ap.add_argument("--routed-scale", type=float, default=1.0, help="sigmoid router: routed scaling factor")
-    ap.add_argument("--fp32-router", action="store_true", help="fp32 router weights (bf16 tokens and experts)")
-    ap.add_argument("--swiglu-limit", type=float, default=0.0, help="SwiGLU limit of the routed experts")
-    ap.add_argument("--swiglu-limit-shared", type=float, default=0.0, help="SwiGLU limit of the shared expert")
-    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
-                    help="expert weights: bf16, or FP8 E4M3 codes with one E8M0 scale per 128x128 block")
-    ap.add_argument("--I", type=int, default=None,
-                    help="profiling variant: override both expert widths (small weights, same router)")
-    args = ap.parse_args()
-    cfg = inputs.CONFIGS[args.workload]
-    if args.T is not None or args.E is not None or args.I is not None:
-        T = cfg.T if args.T is None else args.T
-        E = cfg.E if args.E is None else args.E
-        I = cfg.I if args.I is None else args.I
-        cfg = inputs.with_sizes(cfg, T=T, E=E, I=I, I_shared=I, name=f"{cfg.name}[T={T},E={E},I={I}]")
-    if args.steps is None:
-        args.steps = DEFAULT_STEPS.get(cfg.name, 100)
-    args.warmup = max(args.warmup, 3)
-    if args.impl == "reference":
-        return run_reference(args, cfg)
+BF16_WORKLOADS = ("decode_t4", "decode_t128", "prefill_t4096", "prefill_t16384_skew")
 
+
+def roofline(alg, peaks, gu_ms, fp8, workload):
+    """Roofline of the dominant kernel, the gate/up GEMM: its algorithmic bytes or FLOPs per
+    launch over its average launch time, against the measured copy bandwidth when the
+    launch is HBM-bound and the sustained bf16 tensor peak when it is tensor-bound."""
+    tc_peak = peaks["bf16_tflops_sustained"]
+    tensor_bound = alg["gate_up_flops"] / (tc_peak * 1e12) > alg["gate_up_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    if tensor_bound:
+        achieved = alg["gate_up_flops"] / (gu_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": achieved / tc_peak, "peak_kind": "sustained bf16 (cuBLAS, seconds-long loop)",
+                "frac_of_burst": achieved / peaks["bf16_tflops"]}
+    else:
+        achieved = alg["gate_up_bytes"] / (gu_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    roof.update({"kernel": "expert_gemm_tc_kernel<gated%s> (gate/up GEMM + SiLU*up)" % (", fp8" if fp8 else ""),
+                 "timing": "CUDA events around each launch, stage-timed pass of the same steps",
+                 "traffic": ncu_traffic("gate_up", workload + ("+fp8" if fp8 else "")),
+                 "peak_source": peaks["source"],
+                 "ms_per_launch": gu_ms, "algorithmic_bytes": alg["gate_up_bytes"],
+                 "algorithmic_flops": alg["gate_up_flops"]})
+    return roof
+
+
+def layer_roofline(alg, peaks, ms_per_step):
+    """The whole step against both roofs: bytes / time, FLOPs / time, and the fraction of the
+    attainable time max(bytes / measured HBM bandwidth, FLOPs / sustained bf16 peak)."""
+    s = ms_per_step / 1e3
+    floor = max(alg["layer_bytes"] / (peaks["hbm_gbs"] * 1e9), alg["layer_flops"] / (peaks["bf16_tflops_sustained"] * 1e12))
+    return {"touched_experts": alg["touched"], "algorithmic_bytes": alg["layer_bytes"],
+            "algorithmic_flops": alg["layer_flops"],
+            "hbm_gbs": alg["layer_bytes"] / s / 1e9, "hbm_frac": alg["layer_bytes"] / s / 1e9 / peaks["hbm_gbs"],
+            "hbm_frac_of_8000": alg["layer_bytes"] / s / 1e9 / 8000.0,
+            "tflops": alg["layer_flops"] / s / 1e12,
+            "tensor_frac_sustained": alg["layer_flops"] / s / 1e12 / peaks["bf16_tflops_sustained"],
+            "tensor_frac_burst": alg["layer_flops"] / s / 1e12 / peaks["bf16_tflops"],
+            "frac_of_attainable": floor / s}
+
+
+def measure(cfg, args, dev, pg, world, rank, local, clocks):
+    """Everything measured on one workload: the plain timed pass (the value), a stage-timed
+    pass (per-kernel durations), the end-to-end pass through host buffers and, on rank 0 at
+    N = 1, the oracle's CPU baseline.  Returns the workload's record (rank 0) or None."""
     import sparse_mixture_experts_ffn_b200 as moe
-    from sparse_mixture_experts_ffn_b200 import build
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-        pg = dist
-    if rank == 0 or world == 1:
-        build.build()
-    if pg:
-        pg.barrier()
-    moe.load_library()
-
-    # ---- inputs (resident in HBM); each rank is a replica with its own tokens -------------
+    steps = args.steps if args.steps is not None else DEFAULT_STEPS.get(cfg.name, 100)
     x, Wr, bias = inputs.make_routing_inputs(rank_config(cfg, rank), router_fp32=args.fp32_router)
     fp8 = args.weights == "fp8"
     if fp8:
@@ -379,7 +423,7 @@ def main():
     torch.cuda.synchronize()
     status = moe.check_status(ws)
     if status != moe.MOE_OK:
-        raise RuntimeError(f"device status {moe.status_string(status)}")
+        raise RuntimeError(f"{cfg.name}: device status {moe.status_string(status)}")
     counts = r.counts.cpu().numpy()
     route_stats = moe.route_stats(ws)
     alg = algorithmic(cfg, counts, fp8)
@@ -389,33 +433,33 @@ def main():
         step(x, y)
     torch.cuda.synchronize()
 
-    # ---- kernel-only timed region (the headline value) -----------------------------------
     def timed_pass(profile: bool):
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
         moe.profile_read()
         moe.profile_enable(profile)
         if pg:
             pg.barrier()
         torch.cuda.synchronize()
         launches0 = moe.launch_count()
-        with ClockSampler(local) as clocks:
-            for i in range(args.steps):
-                flush()
-                starts[i].record(stream)
-                step(x, y)
-                ends[i].record(stream)
-            torch.cuda.synchronize()
+        since = len(clocks.samples)
+        for i in range(steps):
+            flush()
+            starts[i].record(stream)
+            step(x, y)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        clk = clocks.summary(since)
         if pg:
             pg.barrier()
         launches = moe.launch_count() - launches0
         moe.profile_enable(False)
         calls, stage_ms = moe.profile_read()
         elapsed = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), pg, dev)
-        return elapsed, launches, clocks, calls, stage_ms
+        return elapsed, launches, clk, calls, stage_ms
 
     # pass 1: the step as a user runs it, kernels chained with programmatic launches
-    elapsed_ms, launches, clocks, _, _ = timed_pass(False)
+    elapsed_ms, launches, clk, _, _ = timed_pass(False)
     # pass 2: the same steps with a CUDA event pair around every stage, for the per-kernel
     # durations (the events end the programmatic overlap between stages, so this pass is slower)
     elapsed_prof_ms, _, _, calls, stage_ms = timed_pass(True)
@@ -425,7 +469,7 @@ def main():
     x_host = x.cpu().pin_memory()
     y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     x_dev = torch.empty_like(x)
-    e_steps = max(3, min(args.steps, 500))
+    e_steps = max(3, min(steps, 500))
     es_, ee_ = ([torch.cuda.Event(enable_timing=True) for _ in range(e_steps)] for _ in range(2))
     for _ in range(3):
         x_dev.copy_(x_host, non_blocking=True)
@@ -445,63 +489,125 @@ def main():
     e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(es_, ee_)), pg, dev)
     if pg:
         pg.barrier()
-
+    rec = None
     if rank == 0:
         peaks = measured_peaks()
-        ms_per_step = elapsed_ms / args.steps
-        value = job_tokens_per_s(cfg.T, world, args.steps, elapsed_ms)
-        e2e_value = job_tokens_per_s(cfg.T, world, e_steps, e2e_ms)
+        ms_per_step = elapsed_ms / steps
         gu_ms = stage_ms["gate_up"] / max(calls, 1)
-        dn_ms = stage_ms["down"] / max(calls, 1)
-        # the GEMM is timed inside the long step loop, where the part runs at its power cap:
-        # the sustained bf16 figure is its tensor-core peak
-        tc_peak = peaks["bf16_tflops_sustained"]
-        tensor_bound = alg["gate_up_flops"] / (tc_peak * 1e12) > alg["gate_up_bytes"] / (peaks["hbm_gbs"] * 1e9)
-        if tensor_bound:
-            achieved = alg["gate_up_flops"] / (gu_ms / 1e3) / 1e12
-            roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                    "frac": achieved / tc_peak, "peak_kind": "sustained bf16 (cuBLAS, seconds-long loop)",
-                    "frac_of_burst": achieved / peaks["bf16_tflops"]}
-        else:
-            achieved = alg["gate_up_bytes"] / (gu_ms / 1e3) / 1e9
-            roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm_gbs"]}
-        roof.update({"kernel": "expert_gemm_tc_kernel<gated%s> (gate/up GEMM + SiLU*up)" % (", fp8" if fp8 else ""),
-                     "timing": "CUDA events around each launch, stage-timed pass of the same steps",
-                     "traffic": ncu_traffic("gate_up", cfg.name + ("+fp8" if fp8 else "")),
-                     "peak_source": peaks["source"],
-                     "ms_per_launch": gu_ms, "algorithmic_bytes": alg["gate_up_bytes"],
-                     "algorithmic_flops": alg["gate_up_flops"]})
-        layer_s = ms_per_step / 1e3
+        rec = {
+            "workload": cfg.name, "T": cfg.T, "steps": steps, "ms_per_step": ms_per_step,
+            "value": job_tokens_per_s(cfg.T, world, steps, elapsed_ms), "unit": UNIT,
+            "ms_per_step_stage_timed": elapsed_prof_ms / steps,
+            "roofline": roofline(alg, peaks, gu_ms, fp8, cfg.name),
+            "layer": dict(layer_roofline(alg, peaks, ms_per_step),
+                          stage_ms_per_step={k: v / max(calls, 1) for k, v in stage_ms.items()},
+                          route_stats=route_stats, device_status=moe.status_string(status)),
+            "e2e": {"value": job_tokens_per_s(cfg.T, world, e_steps, e2e_ms), "unit": UNIT,
+                    "h2d_bytes_per_step": x.numel() * x.element_size(),
+                    "d2h_bytes_per_step": y.numel() * y.element_size(), "steps": e_steps},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+    del ws, y, flush_w, flush_r, x_host
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        h = host_arrays(dict(x=x, W_router=Wr, bias=bias, W_gate_up=Wgu, W_down=Wd, Ws_gate_up=Wsgu,
+                             Ws_down=Wsd))
+        del Wgu, Wd, Wsgu, Wsd
+        if fp8:
+            del W8
+        torch.cuda.empty_cache()
+        rec["cpu_baseline"] = cpu_baseline(h, cfg, layer_options(args))
+    return rec
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=None, choices=sorted(inputs.CONFIGS),
+                    help="one workload only (default: the four bf16 workloads, decode_t4 as the headline)")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--T", type=int, default=None, help="profiling variant: override the token count")
+    ap.add_argument("--E", type=int, default=None, help="profiling variant: override the expert count")
+    ap.add_argument("--router", default="softmax", choices=["softmax", "sigmoid"],
+                    help="router mode (sigmoid: the router as configured, bias for the selection only)")
+    ap.add_argument("--routed-scale", type=float, default=1.0, help="sigmoid router: routed scaling factor")
+    ap.add_argument("--fp32-router", action="store_true", help="fp32 router weights (bf16 tokens and experts)")
+    ap.add_argument("--swiglu-limit", type=float, default=0.0, help="SwiGLU limit of the routed experts")
+    ap.add_argument("--swiglu-limit-shared", type=float, default=0.0, help="SwiGLU limit of the shared expert")
+    ap.add_argument("--weights", default="bf16", choices=["bf16", "fp8"],
+                    help="expert weights: bf16, or FP8 E4M3 codes with one E8M0 scale per 128x128 block")
+    ap.add_argument("--I", type=int, default=None,
+                    help="profiling variant: override both expert widths (small weights, same router)")
+    args = ap.parse_args()
+    names = [args.workload] if args.workload else list(BF16_WORKLOADS)
+    cfgs = []
+    for name in names:
+        cfg = inputs.CONFIGS[name]
+        if args.T is not None or args.E is not None or args.I is not None:
+            T = cfg.T if args.T is None else args.T
+            E = cfg.E if args.E is None else args.E
+            I = cfg.I if args.I is None else args.I
+            cfg = inputs.with_sizes(cfg, T=T, E=E, I=I, I_shared=I, name=f"{cfg.name}[T={T},E={E},I={I}]")
+        cfgs.append(cfg)
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        if args.steps is None:
+            args.steps = 20
+        return run_reference(args, cfgs[0])
+
+    import sparse_mixture_experts_ffn_b200 as moe
+    from sparse_mixture_experts_ffn_b200 import build
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+    if rank == 0 or world == 1:
+        build.build()
+    if pg:
+        pg.barrier()
+    moe.load_library()
+
+    recs = []
+    with ClockSampler(local) as clocks:
+        for cfg in cfgs:
+            recs.append(measure(cfg, args, dev, pg, world, rank, local, clocks))
+            torch.cuda.empty_cache()
+    if rank == 0:
+        head = recs[0]
+        cfg = cfgs[0]
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "ms_per_step_stage_timed": elapsed_prof_ms / args.steps, "higher_is_better": True,
+            "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": head["steps"],
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "ms_per_step_stage_timed": head["ms_per_step_stage_timed"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
             "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "top_k": cfg.top_k,
                        "I": cfg.I, "I_shared": cfg.I_shared, "tokens_per_gpu": cfg.T,
                        **config_options(args),
                        "l2": "flushed before every timed step, outside the events: 2x L2 write, then 2x L2 read",
                        "parallelism": f"replicas x{world}"},
-            "roofline": roof,
-            "layer": {"touched_experts": alg["touched"], "algorithmic_bytes": alg["layer_bytes"],
-                      "algorithmic_flops": alg["layer_flops"],
-                      "hbm_gbs": alg["layer_bytes"] / layer_s / 1e9,
-                      "hbm_frac": alg["layer_bytes"] / layer_s / 1e9 / peaks["hbm_gbs"],
-                      "tflops": alg["layer_flops"] / layer_s / 1e12,
-                      "stage_ms_per_step": {k: v / max(calls, 1) for k, v in stage_ms.items()},
-                      "route_stats": route_stats, "device_status": moe.status_string(status)},
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": x.numel() * x.element_size(),
-                    "d2h_bytes_per_step": y.numel() * y.element_size(), "steps": e_steps},
-            "gpu_launches": int(launches),
-            "clocks": clocks.summary(),
+            "roofline": head["roofline"],
+            "layer": head["layer"],
+            "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"],
+            "clocks": head["clocks"],
         }
-        if world == 1 and not args.no_cpu_baseline:
-            import oracle
-            oracle.build()
-            h = host_arrays(dict(x=x, W_router=Wr, bias=bias, W_gate_up=Wgu, W_down=Wd, Ws_gate_up=Wsgu,
-                                 Ws_down=Wsd))
-            line["cpu_baseline"] = cpu_baseline(h, cfg, layer_options(args))
+        if "cpu_baseline" in head:
+            line["cpu_baseline"] = head["cpu_baseline"]
+        if len(recs) > 1:
+            line["per_workload"] = {r["workload"]: r for r in recs}
+            line["clocks_all_workloads"] = clocks.summary()
         print(json.dumps(line), flush=True)
     if pg:
         pg.barrier()

@@ -70,3 +70,29 @@ def assert_routing_exact(r_gpu, r_ref: dict, E: int, w_tol: float = None):
 
 def to_device(d: dict, device="cuda"):
     return {k: (v.to(device).contiguous() if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+def tile_class_tokens(ref: dict, T: int, top_k: int, n_random: int, seed: int, top: int = 5,
+                      tiles=(16, 128, 256)):
+    """Tokens whose outputs a full-size test checks, chosen from the exact routing so that
+    every kind of expert-GEMM tile is hit: for each of the `top` most-loaded experts and
+    each token-tile width in `tiles`, the last row of its last (ragged) tile and the first
+    row of that tile; the rows at the starts of 256-token tiles of the most-loaded expert;
+    the first and the last token (the shared expert's first and ragged last tiles); and
+    `n_random` random tokens."""
+    counts, offsets, perm = ref["counts"], ref["offsets"], ref["perm"]
+    picks = [0, T - 1]
+    for e in np.argsort(-counts, kind="stable")[:top]:
+        c = int(counts[e])
+        if c == 0:
+            continue
+        for bn in tiles:
+            last = (c - 1) // bn * bn
+            for r in (last, c - 1):
+                picks.append(int(perm[offsets[e] + r]) // top_k)
+    e0 = int(np.argmax(counts))
+    for r in range(0, int(counts[e0]), 256):
+        picks.append(int(perm[offsets[e0] + r]) // top_k)
+    rng = np.random.default_rng(seed)
+    picks += rng.choice(T, min(n_random, T), replace=False).tolist()
+    return np.unique(np.asarray(picks, np.int64))

@@ -6,7 +6,8 @@ import pytest
 import torch
 
 import sparse_mixture_experts_ffn_b200 as moe
-from helpers import (assert_routing_exact, assert_y_close, oracle_routing, oracle_y, to_device)
+from helpers import (assert_routing_exact, assert_y_close, oracle_routing, oracle_y, tile_class_tokens,
+                     to_device)
 from sparse_mixture_experts_ffn_b200 import inputs
 
 pytestmark = pytest.mark.gpu
@@ -276,11 +277,7 @@ def test_full_size_workload(name):
     stats = moe.route_stats(ws)
     ref = oracle_routing(d, cfg.top_k)
     assert_routing_exact(r, ref, cfg.E)
-    if cfg.T <= 128:
-        tokens = np.arange(cfg.T)
-    else:
-        rng = np.random.default_rng(cfg.seed)
-        tokens = np.unique(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 46, replace=False)]))
+    tokens = np.arange(cfg.T) if cfg.T <= 128 else tile_class_tokens(ref, cfg.T, cfg.top_k, 40, cfg.seed)
     y_ref = oracle_y(d, ref, tokens=tokens)
     assert_y_close(y[torch.as_tensor(tokens, device=y.device)], y_ref, name)
     print(name, "route stats", stats)
@@ -305,9 +302,7 @@ def test_full_size_layer_as_configured(name):
     assert moe.check_status(ws) == moe.MOE_OK
     ref = oracle_routing(d, cfg.top_k, router="sigmoid", scale=3.0)
     assert_routing_exact(r, ref, cfg.E)
-    rng = np.random.default_rng(cfg.seed)
-    tokens = np.arange(cfg.T) if cfg.T <= 128 else np.unique(
-        np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 30, replace=False)]))
+    tokens = np.arange(cfg.T) if cfg.T <= 128 else tile_class_tokens(ref, cfg.T, cfg.top_k, 20, cfg.seed)
     y_ref = oracle_y(d, ref, tokens=tokens, swiglu_limit=7.0, swiglu_limit_shared=16.0)
     assert_y_close(y[torch.as_tensor(tokens, device=y.device)], y_ref, name + " as configured")
     print(name, "as configured, route stats", moe.route_stats(ws))
@@ -405,11 +400,10 @@ def test_fp8_subnormal_and_zero_codes(T):
 def test_fp8_full_size_workload(name):
     cfg = inputs.CONFIGS[name]
     d = fp8_inputs(cfg)
-    if cfg.T <= 4:
+    if cfg.T <= 128:
         tokens = None
     else:
-        rng = np.random.default_rng(cfg.seed)
-        tokens = np.unique(np.concatenate([[0, cfg.T - 1], rng.choice(cfg.T, 30, replace=False)]))
+        tokens = tile_class_tokens(oracle_routing(d, cfg.top_k), cfg.T, cfg.top_k, 20, cfg.seed, tiles=(16, 128))
     run_fp8(d, cfg.top_k, tokens=tokens, what=name + " fp8")
 
 
