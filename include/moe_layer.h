@@ -188,6 +188,49 @@ MOE_API moe_status moe_layer_forward_fp8(const moe_layer_shape* shape, const voi
                                          moe_routing_out* routing, const moe_layer_options* options,
                                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Expert parallelism: the layer split over G GPUs (one process per GPU), each holding a
+ * contiguous range of the routed experts.  The source pages say only that multi-GPU setups
+ * serve the model (q4km.ai model page, hardware section); the split is this library's.
+ * Every rank sees the same tokens (for example after an all-gather of the ranks' batches),
+ * routes them over all E experts as moe_layer_forward() does, computes the routed experts
+ * it holds and, on a range of token rows, the shared expert, and writes its fp32 share:
+ *   y_partial[t] = sum_{j: expert_begin <= idx[t,j] < expert_end} w[t,j] FFN_idx[t,j](x_t)
+ *                + [shared_begin <= t < shared_end] shared(x_t)
+ * The sum of the shares over the ranks (in rank order: moe_layer_sum_partials(), or a
+ * reduce-scatter) is the layer's output, when the ranks' expert ranges partition [0, E)
+ * and their shared ranges partition [0, T).                                               */
+typedef struct {
+  int32_t expert_begin;  /* first routed expert held by this rank */
+  int32_t expert_end;    /* one past the last; 0 <= begin < end <= E */
+  int64_t shared_begin;  /* token rows [shared_begin, shared_end) get the shared expert */
+  int64_t shared_end;    /* 0 <= begin <= end <= T (an empty range adds no shared expert) */
+} moe_ep_range;
+
+/* One rank's share of the layer (see moe_ep_range).  As moe_layer_forward_ex(), except:
+ *   W_gate_up  [expert_end - expert_begin, 2*I, H] bf16: this rank's routed experts only
+ *   W_down     [expert_end - expert_begin, H, I]   bf16
+ *   y_partial  [T, H] fp32, written (16-byte aligned); there is no y argument
+ * x, W_router (all E experts), router_bias, the shared expert's matrices, routing,
+ * options and the workspace (moe_layer_workspace_bytes(shape)) are as for
+ * moe_layer_forward_ex(); the routing outputs cover all E experts.  The shape's dtype must
+ * be MOE_BF16 (else MOE_ERR_UNSUPPORTED_SHAPE); a range outside the bounds above returns
+ * MOE_ERR_INVALID_ARG before anything is enqueued. */
+MOE_API moe_status moe_layer_forward_ep(const moe_layer_shape* shape, const void* x, const void* W_router,
+                                        const float* router_bias, const void* W_gate_up, const void* W_down,
+                                        const void* Ws_gate_up, const void* Ws_down, const moe_ep_range* range,
+                                        float* y_partial, moe_routing_out* routing,
+                                        const moe_layer_options* options, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+
+/* y = sum_{r < n_parts} parts[r], the n_parts fp32 [T, H] buffers added element by element
+ * in index order (fp32), stored in `dtype` (MOE_BF16 or MOE_F32).  `parts` is a HOST array
+ * of n_parts device pointers (1 <= n_parts <= 16), each 16-byte aligned; they may point to
+ * other GPUs' memory mapped into this process (peer access over NVLink), so the ranks'
+ * shares of moe_layer_forward_ep() can be added where they lie.  H must be a multiple of 8.
+ * Used by expert parallelism; no counterpart on the source pages. */
+MOE_API moe_status moe_layer_sum_partials(int64_t T, int32_t H, int32_t dtype, int32_t n_parts,
+                                          const float* const* parts, void* y, void* stream);
+
 /* Synchronises `stream`, then returns the device status word of the most recent
  * moe_layer_forward() that used this workspace (MOE_OK, MOE_ERR_DEVICE_TIMEOUT or
  * MOE_ERR_DEVICE_BOUNDS), or MOE_ERR_CUDA if the stream itself reports an error. */

@@ -25,7 +25,7 @@ STATUS_NAMES = {
     6: "MOE_ERR_DEVICE_BOUNDS",
 }
 EXPORTED = ("moe_layer_workspace_bytes", "moe_layer_forward", "moe_layer_forward_ex", "moe_layer_forward_fp8",
-            "moe_layer_check_status",
+            "moe_layer_forward_ep", "moe_layer_sum_partials", "moe_layer_check_status",
             "moe_layer_route_stats", "moe_layer_workspace_layout", "moe_layer_profile_enable",
             "moe_layer_profile_read", "moe_layer_launch_count", "moe_status_string")
 STAGES = ("routing", "dispatch", "gate_up", "down", "combine")
@@ -51,6 +51,11 @@ class MoEFp8Weights(ctypes.Structure):
                 ("W_down", ctypes.c_void_p), ("W_down_scale", ctypes.c_void_p),
                 ("Ws_gate_up", ctypes.c_void_p), ("Ws_gate_up_scale", ctypes.c_void_p),
                 ("Ws_down", ctypes.c_void_p), ("Ws_down_scale", ctypes.c_void_p)]
+
+
+class MoEEpRange(ctypes.Structure):
+    _fields_ = [("expert_begin", ctypes.c_int32), ("expert_end", ctypes.c_int32),
+                ("shared_begin", ctypes.c_int64), ("shared_end", ctypes.c_int64)]
 
 
 class MoERoutingOut(ctypes.Structure):
@@ -101,6 +106,13 @@ def load_library(path: str = LIB_PATH):
                                           ctypes.POINTER(MoERoutingOut), ctypes.POINTER(MoEOptions), P,
                                           ctypes.c_size_t, P]
     lib.moe_layer_forward_fp8.restype = ctypes.c_int
+    lib.moe_layer_forward_ep.argtypes = [ctypes.POINTER(MoEShape), P, P, P, P, P, P, P, ctypes.POINTER(MoEEpRange),
+                                         P, ctypes.POINTER(MoERoutingOut), ctypes.POINTER(MoEOptions), P,
+                                         ctypes.c_size_t, P]
+    lib.moe_layer_forward_ep.restype = ctypes.c_int
+    lib.moe_layer_sum_partials.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.POINTER(ctypes.c_void_p), P, P]
+    lib.moe_layer_sum_partials.restype = ctypes.c_int
     lib.moe_layer_check_status.argtypes = [P, P]
     lib.moe_layer_check_status.restype = ctypes.c_int
     lib.moe_layer_route_stats.argtypes = [P, ctypes.POINTER(MoERouteStats), P]
@@ -209,6 +221,99 @@ def moe_layer_forward_fp8(x, W_router, weights, *, top_k, router_bias=None, y=No
                     routed_scaling_factor)
 
 
+def expert_range(E: int, world: int, rank: int) -> tuple:
+    """The routed experts [begin, end) that rank `rank` of `world` holds under expert
+    parallelism: contiguous, sizes differing by at most one."""
+    return rank * E // world, (rank + 1) * E // world
+
+
+def moe_layer_forward_ep(x, W_router, W_gate_up, W_down, Ws_gate_up=None, Ws_down=None, *, top_k,
+                         expert_begin, shared_rows=(0, 0), router_bias=None, y_partial=None, workspace=None,
+                         routing=False, stream=None, swiglu_limit=0.0, swiglu_limit_shared=0.0,
+                         router="softmax", routed_scaling_factor=1.0):
+    """One rank's fp32 share of the layer under expert parallelism (moe_layer_forward_ep in
+    include/moe_layer.h).  W_gate_up [n, 2I, H] and W_down [n, H, I] hold the routed experts
+    [expert_begin, expert_begin + n) only; W_router holds all E.  The shared expert is added
+    on the token rows [shared_rows[0], shared_rows[1]).  Returns (y_partial fp32 [T, H],
+    Routing or None); the shares of ranks whose expert and shared ranges partition the
+    experts and the tokens add up to the layer's output."""
+    import torch
+    if W_gate_up.dim() != 3 or W_down.dim() != 3 or (Ws_gate_up is not None and Ws_gate_up.dim() != 2):
+        raise ValueError("W_gate_up must be [n, 2I, H], W_down [n, H, I] and Ws_gate_up [2Is, H]")
+    if x.dtype != torch.bfloat16:
+        raise ValueError("expert parallelism runs bf16 layers")
+    n = W_gate_up.shape[0]
+    E = W_router.shape[0]
+    e0 = int(expert_begin)
+    if not (0 <= e0 and e0 + n <= E and n >= 1):
+        raise ValueError(f"experts [{e0}, {e0 + n}) outside [0, {E})")
+    I = W_gate_up.shape[1] // 2
+    Is = 0 if Ws_gate_up is None else Ws_gate_up.shape[0] // 2
+    _check_args(x, W_router[e0:e0 + n], router_bias[e0:e0 + n] if router_bias is not None else None, None,
+                (W_gate_up, W_down, Ws_gate_up, Ws_down), I, Is, False)
+    if router_bias is not None and (router_bias.dtype != torch.float32 or tuple(router_bias.shape) != (E,)):
+        raise ValueError(f"router_bias must be fp32 [{E}]")
+    T, H = x.shape
+    s0, s1 = int(shared_rows[0]), int(shared_rows[1])
+    if not (0 <= s0 <= s1 <= T):
+        raise ValueError(f"shared rows [{s0}, {s1}) outside [0, {T}]")
+    if y_partial is None:
+        y_partial = torch.empty(T, H, dtype=torch.float32, device=x.device)
+    elif y_partial.dtype != torch.float32 or tuple(y_partial.shape) != (T, H) or y_partial.device != x.device:
+        raise ValueError(f"y_partial must be fp32 [{T}, {H}] on x's device")
+    lib = load_library()
+    shape = make_shape(T, H, E, I, Is, top_k, x.dtype)
+    if workspace is None:
+        workspace = alloc_workspace(shape, x.device)
+    r, rout = _routing_buffers(T, E, top_k, x.device) if routing else (None, None)
+    if stream is None:
+        stream = torch.cuda.current_stream(x.device)
+    w32 = 1 if W_router.dtype == torch.float32 else 0
+    opts = MoEOptions(float(swiglu_limit), float(swiglu_limit_shared), ROUTERS[router],
+                      float(routed_scaling_factor), w32)
+    rng = MoEEpRange(e0, e0 + n, s0, s1)
+    rc = lib.moe_layer_forward_ep(ctypes.byref(shape), _ptr(x), _ptr(W_router), _ptr(router_bias), _ptr(W_gate_up),
+                                  _ptr(W_down), _ptr(Ws_gate_up), _ptr(Ws_down), ctypes.byref(rng), _ptr(y_partial),
+                                  ctypes.byref(rout) if rout is not None else None, ctypes.byref(opts),
+                                  _ptr(workspace), workspace.numel(), ctypes.c_void_p(stream.cuda_stream))
+    if rc != MOE_OK:
+        raise MoEError(rc, "moe_layer_forward_ep")
+    return y_partial, r
+
+
+def sum_partials(parts, y, stream=None):
+    """y = parts[0] + parts[1] + ... (fp32, in order), stored in y's dtype (bf16 or fp32).
+    Each part is an fp32 tensor of y's shape on y's device."""
+    import torch
+    if not parts or len(parts) > 16:
+        raise ValueError("1 to 16 parts")
+    for t in parts:
+        if t.dtype != torch.float32 or t.shape != y.shape or t.device != y.device or not t.is_contiguous():
+            raise ValueError("parts must be contiguous fp32 tensors of y's shape on y's device")
+    if y.dim() != 2 or not y.is_contiguous() or y.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("y must be a contiguous bf16 or fp32 [T, H] tensor")
+    if stream is None:
+        stream = torch.cuda.current_stream(y.device)
+    arr = (ctypes.c_void_p * len(parts))(*[t.data_ptr() for t in parts])
+    rc = load_library().moe_layer_sum_partials(y.shape[0], y.shape[1], MOE_BF16 if y.dtype == torch.bfloat16
+                                               else MOE_F32, len(parts), arr, _ptr(y),
+                                               ctypes.c_void_p(stream.cuda_stream))
+    if rc != MOE_OK:
+        raise MoEError(rc, "moe_layer_sum_partials")
+    return y
+
+
+def _routing_buffers(T, E, top_k, dev):
+    import torch
+    r = Routing(torch.empty(T, top_k, dtype=torch.int32, device=dev),
+                torch.empty(T, top_k, dtype=torch.float32, device=dev),
+                torch.empty(E, dtype=torch.int32, device=dev),
+                torch.empty(E + 1, dtype=torch.int32, device=dev),
+                torch.empty(T * top_k, dtype=torch.int32, device=dev))
+    return r, MoERoutingOut(r.topk_idx.data_ptr(), r.topk_w.data_ptr(), r.counts.data_ptr(),
+                            r.offsets.data_ptr(), r.perm.data_ptr())
+
+
 def _check_args(x, W_router, router_bias, y, weights, I, Is, fp8: bool):
     """Validate shapes, dtypes and devices before anything reaches the C ABI, which sees only
     pointers: a mismatch there would make the kernels read past an allocation.  Raises
@@ -285,17 +390,7 @@ def _forward(entry, weights, x, W_router, I, Is, top_k, router_bias, y, workspac
         y = torch.empty_like(x)
     if workspace is None:
         workspace = alloc_workspace(shape, x.device)
-    r = None
-    rout = None
-    if routing:
-        dev = x.device
-        r = Routing(torch.empty(T, top_k, dtype=torch.int32, device=dev),
-                    torch.empty(T, top_k, dtype=torch.float32, device=dev),
-                    torch.empty(E, dtype=torch.int32, device=dev),
-                    torch.empty(E + 1, dtype=torch.int32, device=dev),
-                    torch.empty(T * top_k, dtype=torch.int32, device=dev))
-        rout = MoERoutingOut(r.topk_idx.data_ptr(), r.topk_w.data_ptr(), r.counts.data_ptr(),
-                             r.offsets.data_ptr(), r.perm.data_ptr())
+    r, rout = _routing_buffers(T, E, top_k, x.device) if routing else (None, None)
     if stream is None:
         stream = torch.cuda.current_stream(x.device)
     w32 = 1 if (x.dtype == torch.bfloat16 and W_router.dtype == torch.float32) else 0

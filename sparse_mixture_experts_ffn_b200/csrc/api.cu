@@ -231,10 +231,14 @@ struct ExpertWeights {
   const void* scale[4];  // FP8: of Wgu, Wd, Wsgu, Wsd
 };
 
+// ep = nullptr: the whole layer into y.  Otherwise (expert parallelism) the weights hold the
+// routed experts [ep->expert_begin, ep->expert_end) only, and this rank's fp32 share of the
+// output goes to y_partial (y is not used).
 static moe_status forward_impl(const moe_layer_shape* shape, const void* x, const void* W_router,
                                const float* router_bias, const ExpertWeights& wt, void* y,
                                moe_routing_out* routing, const moe_layer_options* options,
-                               void* workspace, size_t workspace_bytes, void* stream) {
+                               void* workspace, size_t workspace_bytes, void* stream,
+                               const moe_ep_range* ep = nullptr, float* y_partial = nullptr) {
   const void* W_gate_up = wt.Wgu;
   const void* W_down = wt.Wd;
   const void* Ws_gate_up = wt.Wsgu;
@@ -251,13 +255,25 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   const moe_layer_shape& s = *shape;
   // fp32 router weights with bf16 tokens run on the tensor-core router only
   if (opt.router_weights_fp32 && s.dtype == MOE_BF16 && !router_w32_supported(s)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  int e_lo = 0, e_hi = s.E;
+  int64_t sh_lo = 0, sh_hi = s.T;
+  if (ep) {
+    if (s.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED_SHAPE;
+    e_lo = ep->expert_begin;
+    e_hi = ep->expert_end;
+    sh_lo = ep->shared_begin;
+    sh_hi = ep->shared_end;
+    if (e_lo < 0 || e_hi > s.E || e_lo >= e_hi || sh_lo < 0 || sh_hi > s.T || sh_lo > sh_hi)
+      return MOE_ERR_INVALID_ARG;
+  }
   if (s.T == 0) return MOE_OK;  // empty batch: nothing to read or write
-  if (!x || !W_router || !W_gate_up || !W_down || !y || !workspace) return MOE_ERR_INVALID_ARG;
+  if (!x || !W_router || !W_gate_up || !W_down || !workspace) return MOE_ERR_INVALID_ARG;
+  if (ep ? (!y_partial || !aligned16(y_partial)) : !y) return MOE_ERR_INVALID_ARG;
   const bool has_shared = s.I_shared > 0;
   if (has_shared != (Ws_gate_up != nullptr) || has_shared != (Ws_down != nullptr))
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(W_router) || !aligned16(W_gate_up) || !aligned16(W_down) ||
-      !aligned16(y) || (has_shared && (!aligned16(Ws_gate_up) || !aligned16(Ws_down))) ||
+      (!ep && !aligned16(y)) || (has_shared && (!aligned16(Ws_gate_up) || !aligned16(Ws_down))) ||
       (reinterpret_cast<uintptr_t>(router_bias) & 3u) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return MOE_ERR_INVALID_ARG;
@@ -325,6 +341,9 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   da.bn = L.bn;
   da.bn_dn = bn_dn;
   da.ksplit = L.ksplit;
+  da.e_lo = e_lo;
+  da.e_hi = e_hi;
+  da.shared_rows = static_cast<int>(sh_hi - sh_lo);
   da.x = x;
   da.idx = ra.idx_ws;
   da.w = ra.w_ws;
@@ -354,6 +373,10 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   ea.k = s.top_k;
   ea.I = s.I;
   ea.Is = s.I_shared;
+  ea.e_lo = e_lo;
+  ea.e_hi = e_hi;
+  ea.shared_base = sh_lo;
+  ea.shared_rows = sh_hi - sh_lo;
   ea.x = x;
   ea.Wgu = W_gate_up;
   ea.Wd = W_down;
@@ -401,6 +424,14 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   ca.o_shared = ea.o_shared;
   ca.y = y;
   ca.ctrl = ctrl;
+  if (ep) {
+    ca.y_partial = y_partial;
+    ca.offsets = da.offsets;
+    ca.e_lo = e_lo;
+    ca.e_hi = e_hi;
+    ca.shared_lo = sh_lo;
+    ca.shared_hi = sh_hi;
+  }
   if (launch_combine(ca, st) != cudaSuccess) return MOE_ERR_CUDA;
   marks.mark(5, st);
   return MOE_OK;
@@ -436,6 +467,33 @@ extern "C" moe_status moe_layer_forward_fp8(const moe_layer_shape* shape, const 
                          {w.W_gate_up_scale, w.W_down_scale, w.Ws_gate_up_scale, w.Ws_down_scale}};
   return forward_impl(shape, x, W_router, router_bias, wt, y, routing, options, workspace, workspace_bytes,
                       stream);
+}
+
+extern "C" moe_status moe_layer_forward_ep(const moe_layer_shape* shape, const void* x,
+                                           const void* W_router, const float* router_bias,
+                                           const void* W_gate_up, const void* W_down,
+                                           const void* Ws_gate_up, const void* Ws_down,
+                                           const moe_ep_range* range, float* y_partial,
+                                           moe_routing_out* routing, const moe_layer_options* options,
+                                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!range) return MOE_ERR_INVALID_ARG;
+  const ExpertWeights wt{W_gate_up, W_down, Ws_gate_up, Ws_down, false, {nullptr, nullptr, nullptr, nullptr}};
+  return forward_impl(shape, x, W_router, router_bias, wt, nullptr, routing, options, workspace, workspace_bytes,
+                      stream, range, y_partial);
+}
+
+extern "C" moe_status moe_layer_sum_partials(int64_t T, int32_t H, int32_t dtype, int32_t n_parts,
+                                             const float* const* parts, void* y, void* stream) {
+  if (T < 0 || H < 1 || H % 8 || (dtype != MOE_F32 && dtype != MOE_BF16)) return MOE_ERR_INVALID_ARG;
+  if (n_parts < 1 || n_parts > kMaxParts || !parts) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!y || !aligned16(y)) return MOE_ERR_INVALID_ARG;
+  for (int r = 0; r < n_parts; ++r)
+    if (!parts[r] || !aligned16(parts[r])) return MOE_ERR_INVALID_ARG;
+  return launch_sum_partials(parts, n_parts, T * static_cast<int64_t>(H), dtype == MOE_BF16, y,
+                             static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }
 
 extern "C" moe_status moe_layer_check_status(void* workspace, void* stream) {

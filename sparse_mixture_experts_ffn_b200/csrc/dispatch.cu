@@ -78,6 +78,8 @@ __device__ int block_scan_pair(int v0, int v1, int* warp_tot, int& total) {
 struct ScheduleArgs {
   int64_t T;
   int E, has_shared, mt_gu, mt_gu_shared, mt_dn, bn, bn_dn, ksplit;
+  int e_lo, e_hi;   // routed experts that get tiles (expert parallelism: this rank's range)
+  int shared_rows;  // rows of the shared-expert group
   int32_t* offsets;
   int32_t* group_order;
   int32_t* item_start_gu;
@@ -140,6 +142,7 @@ __device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* order, int*
     if (r >= G) return 0;
     const int g = order[r];
     const int bn = gu ? a.bn : a.bn_dn;
+    if (g < E && (g < a.e_lo || g >= a.e_hi)) return 0;  // another rank's expert
     const int nt = (cnt[g] + bn - 1) / bn;
     const int mt = gu ? (g < E ? a.mt_gu : a.mt_gu_shared) * a.ksplit : a.mt_dn;
     return nt * mt;
@@ -222,7 +225,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScheduleArgs sa, int k, int 
       if (counts_user) counts_user[e] = run;
     }
   }
-  if (sa.has_shared && threadIdx.x == 0) cnt[E] = static_cast<int>(sa.T);
+  if (sa.has_shared && threadIdx.x == 0) cnt[E] = sa.shared_rows;
   __syncthreads();
   build_schedule(sa, cnt, order, warp_tot);
 }
@@ -295,7 +298,7 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
     counts[e] = cnt[e];
     if (counts_user) counts_user[e] = cnt[e];
   }
-  if (sa.has_shared && threadIdx.x == 0) cnt[E] = static_cast<int>(sa.T);
+  if (sa.has_shared && threadIdx.x == 0) cnt[E] = sa.shared_rows;
   __syncthreads();
   build_schedule(sa, cnt, order, warp_tot);
   __syncthreads();
@@ -305,10 +308,12 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
     place_assignments(idx, w, 0, P, k, E, base, perm, inv_perm, row_w, row_tok, perm_user);
 }
 
-// x_perm[pos, :] = x[row_tok[pos], :], 16-byte vectors: one warp per row at a time (no
-// per-vector index arithmetic), four vectors in flight per lane
+// x_perm[pos, :] = x[row_tok[pos], :] for the rows of experts [e_lo, e_hi) (all experts,
+// or one rank's range under expert parallelism), 16-byte vectors: one warp per row at a
+// time (no per-vector index arithmetic), four vectors in flight per lane
 template <typename T>
 __global__ void gather_rows_kernel(const T* __restrict__ x, const int32_t* __restrict__ row_tok,
+                                   const int32_t* __restrict__ offsets, int e_lo, int e_hi,
                                    int64_t P, int64_t Tn, int H, T* __restrict__ x_perm,
                                    Ctrl* ctrl) {
   pdl_wait();
@@ -317,7 +322,13 @@ __global__ void gather_rows_kernel(const T* __restrict__ x, const int32_t* __res
   const int vpr = H / V;
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t p = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; p < P; p += warps) {
+  const int64_t p_lo = __ldg(offsets + e_lo), p_hi = __ldg(offsets + e_hi);
+  if (p_lo < 0 || p_hi > P || p_lo > p_hi) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(ctrl, MOE_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  for (int64_t p = p_lo + ((static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5); p < p_hi;
+       p += warps) {
     const int64_t t = __ldg(row_tok + p);
     if (t < 0 || t >= Tn) {
       if (lane == 0) set_status(ctrl, MOE_ERR_DEVICE_BOUNDS);
@@ -353,6 +364,9 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st) {
   sa.bn = a.bn;
   sa.bn_dn = a.bn_dn;
   sa.ksplit = a.ksplit;
+  sa.e_lo = a.e_lo;
+  sa.e_hi = a.e_hi;
+  sa.shared_rows = a.shared_rows;
   sa.offsets = a.offsets;
   sa.group_order = a.group_order;
   sa.item_start_gu = a.item_start_gu;
@@ -395,11 +409,13 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st) {
   const int blocks = static_cast<int>(std::min<int64_t>((P + 7) / 8, 148 * 16));  // a warp per row
   if (a.bf16)
     e = launch_pdl(gather_rows_kernel<__nv_bfloat16>, dim3(blocks), dim3(256), 0, st,
-                   static_cast<const __nv_bfloat16*>(a.x), static_cast<const int32_t*>(a.row_tok), P,
-                   a.T, a.H, static_cast<__nv_bfloat16*>(a.x_perm), a.ctrl);
+                   static_cast<const __nv_bfloat16*>(a.x), static_cast<const int32_t*>(a.row_tok),
+                   static_cast<const int32_t*>(a.offsets), a.e_lo, a.e_hi, P, a.T, a.H,
+                   static_cast<__nv_bfloat16*>(a.x_perm), a.ctrl);
   else
     e = launch_pdl(gather_rows_kernel<float>, dim3(blocks), dim3(256), 0, st,
-                   static_cast<const float*>(a.x), static_cast<const int32_t*>(a.row_tok), P, a.T, a.H,
+                   static_cast<const float*>(a.x), static_cast<const int32_t*>(a.row_tok),
+                   static_cast<const int32_t*>(a.offsets), a.e_lo, a.e_hi, P, a.T, a.H,
                    static_cast<float*>(a.x_perm), a.ctrl);
   count_launches(launches + 1);
   return e;

@@ -46,6 +46,9 @@ struct TcParams {
   int ld_out[2];               // row stride of out (elements), routed and shared
   int E, G;
   int64_t T;
+  int g_lo, g_hi;              // routed experts held in the weight matrices: [g_lo, g_hi)
+                               // (all E, or one rank's range under expert parallelism)
+  int sh_base, sh_rows;        // rows of the shared-expert group: [sh_base, sh_base + sh_rows)
   int kblocks[2];              // reduction length / kTileK, routed and shared
   int a_rows_per_group;        // rows of one routed expert's weight matrix
   int a_up_offset[2];          // gate/up: row offset of the up block (I or Is)
@@ -152,14 +155,15 @@ __device__ __forceinline__ Item decode_item(const TcParams& p, const Sched& sc, 
   const int local = local_item / ks_n;  // slices of one tile are consecutive items
   r.ks = local_item - local * ks_n;
   r.tile = it / ks_n;                   // every group's item count is a multiple of ks_n
-  const int base = r.sh ? 0 : sc.ld(sc.offsets + r.g);
-  const int cnt = r.sh ? static_cast<int>(p.T) : sc.ld(sc.offsets + r.g + 1) - base;
+  const int base = r.sh ? p.sh_base : sc.ld(sc.offsets + r.g);
+  const int cnt = r.sh ? p.sh_rows : sc.ld(sc.offsets + r.g + 1) - base;
   const int ntile = (cnt + BN - 1) / BN;
   r.m = ntile > 0 ? local / ntile : 0;
   const int n = local - r.m * ntile;
   r.row0 = base + n * BN;
   r.nvalid = min(BN, cnt - n * BN);
-  r.valid = (r.g >= 0 && r.g < p.G && ntile > 0 && r.m >= 0 && r.m < p.mt[r.sh] && r.nvalid >= 1 &&
+  r.valid = (r.g >= 0 && r.g < p.G && (r.sh || (r.g >= p.g_lo && r.g < p.g_hi)) && ntile > 0 && r.m >= 0 &&
+             r.m < p.mt[r.sh] && r.nvalid >= 1 &&
              r.row0 >= 0 && r.row0 + r.nvalid <= p.rows_out[r.sh] &&
              (ks_n == 1 || (r.tile >= 0 && r.tile < p.max_tiles))) ? 1 : 0;
   if (!r.valid) {
@@ -351,7 +355,7 @@ __global__ void __launch_bounds__(W8 ? 192 + 128 * kConvGroups : 192, 1) expert_
       const int k0 = t.ks * kbn / p.ksplit, k1 = (t.ks + 1) * kbn / p.ksplit;
       const int c0 = k0 >> 1, nblk = k1 > k0 ? ((k1 - 1) >> 1) - c0 + 1 : 0;
       const int ld = p.s_ld[t.sh];
-      const uint8_t* sbase = p.scaleA[t.sh] + static_cast<int64_t>(t.sh ? 0 : t.g) * p.s_rows_per_group * ld;
+      const uint8_t* sbase = p.scaleA[t.sh] + static_cast<int64_t>(t.sh ? 0 : t.g - p.g_lo) * p.s_rows_per_group * ld;
       const uint8_t* srow_g = sbase + static_cast<int64_t>(t.m) * ld;
       const uint8_t* srow_u = sbase + static_cast<int64_t>(t.m + p.a_up_offset[t.sh] / kTileM) * ld;
 #pragma unroll
@@ -401,7 +405,7 @@ __global__ void __launch_bounds__(W8 ? 192 + 128 * kConvGroups : 192, 1) expert_
           tok[q] = (v < 0 || v >= p.T) ? 0 : v;  // padding rows repeat the first token
         }
       }
-      const int arow = t.sh ? t.m * kTileM : t.g * p.a_rows_per_group + t.m * kTileM;
+      const int arow = t.sh ? t.m * kTileM : (t.g - p.g_lo) * p.a_rows_per_group + t.m * kTileM;
       const int kb_n = p.kblocks[t.sh];
       const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
       // FP8: the item's block scales, one 128-column block per lane (and lane + 32),
@@ -899,7 +903,8 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   auto encode_w = [&](CUtensorMap* m, const void* w, uint64_t rows, uint64_t cols) {
     return a.w8 ? encode_2d_u8(m, w, rows, cols) : encode_2d_bf16(m, w, rows, cols, kTileM);
   };
-  bool ok = encode_w(&g.tmA[0], a.Wgu, static_cast<uint64_t>(a.E) * 2 * a.I, a.H) &&
+  const uint64_t n_local = static_cast<uint64_t>(a.e_hi - a.e_lo);  // routed experts held
+  bool ok = encode_w(&g.tmA[0], a.Wgu, n_local * 2 * a.I, a.H) &&
             (gather ? encode_2d_bf16(&g.tmB[0], a.x, a.T, a.H, 1)
                     : encode_2d_bf16(&g.tmB[0], a.x_perm, P, a.H, a.bn));
   if (has_shared)
@@ -923,6 +928,10 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   g.E = a.E;
   g.G = G;
   g.T = a.T;
+  g.g_lo = a.e_lo;
+  g.g_hi = a.e_hi;
+  g.sh_base = static_cast<int>(a.shared_base);
+  g.sh_rows = static_cast<int>(a.shared_rows);
   g.kblocks[0] = g.kblocks[1] = a.H / kTileK;
   g.a_rows_per_group = 2 * a.I;
   g.a_up_offset[0] = a.I;
@@ -949,7 +958,7 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   if (a.stage_mark) a.stage_mark(a.stage_mark_ctx, 3, st);
   // down: A = W_down viewed as [E*H, I]; B = h [P, I] (shared: Ws_down [H, Is], h_shared)
   TcParams d{};
-  ok = encode_w(&d.tmA[0], a.Wd, static_cast<uint64_t>(a.E) * a.H, a.I) &&
+  ok = encode_w(&d.tmA[0], a.Wd, n_local * a.H, a.I) &&
        encode_2d_bf16(&d.tmB[0], a.h, P, a.I, a.bn_dn);
   if (has_shared)
     ok = ok && encode_w(&d.tmA[1], a.Wsd, a.H, a.Is) &&
@@ -969,6 +978,10 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   d.E = a.E;
   d.G = G;
   d.T = a.T;
+  d.g_lo = a.e_lo;
+  d.g_hi = a.e_hi;
+  d.sh_base = static_cast<int>(a.shared_base);
+  d.sh_rows = static_cast<int>(a.shared_rows);
   d.kblocks[0] = a.I / kTileK;
   d.kblocks[1] = has_shared ? a.Is / kTileK : 0;
   d.a_rows_per_group = a.H;

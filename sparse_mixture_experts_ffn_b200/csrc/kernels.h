@@ -77,6 +77,8 @@ struct DispatchArgs {
   int bn;           // tokens per gate/up GEMM tile
   int bn_dn;        // tokens per down GEMM tile
   int ksplit;       // gate/up reduction slices
+  int e_lo, e_hi;   // routed experts whose rows are computed: [0, E), or one rank's range
+  int shared_rows;  // rows of the shared-expert group (T, or one rank's token slice)
   const void* x;
   const int32_t* idx;   // [T, k]
   const float* w;       // [T, k]
@@ -102,6 +104,9 @@ struct ExpertArgs {
   bool bf16;
   int64_t T;
   int H, E, k, I, Is;
+  int e_lo, e_hi;          // routed experts whose weights Wgu / Wd hold: [e_lo, e_hi)
+  int64_t shared_base;     // token rows [shared_base, shared_base + shared_rows) get the
+  int64_t shared_rows;     // shared expert (all T rows without expert parallelism)
   const void* x;
   const void* Wgu;   // [E, 2I, H]
   const void* Wd;    // [E, H, I]
@@ -160,8 +165,20 @@ struct CombineArgs {
   const void* o_shared;
   void* y;
   Ctrl* ctrl;
+  // expert parallelism: when y_partial is set, the fp32 share of the experts [e_lo, e_hi)
+  // and of the shared expert on token rows [shared_lo, shared_hi) is written there instead
+  float* y_partial = nullptr;
+  const int32_t* offsets = nullptr;
+  int e_lo = 0, e_hi = 0;
+  int64_t shared_lo = 0, shared_hi = 0;
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
+
+// the most partial outputs that moe_layer_sum_partials adds in one call
+constexpr int kMaxParts = 16;
+// y = sum of n fp32 buffers of `count` elements (count a multiple of 4), in order, as bf16 or fp32
+cudaError_t launch_sum_partials(const float* const* parts, int n, int64_t count, bool bf16, void* y,
+                                cudaStream_t st);
 
 // adds n to the process-wide count of kernels launched by this library
 void count_launches(int n);

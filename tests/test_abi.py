@@ -168,7 +168,8 @@ def header_structs():
 @pytest.mark.parametrize("c_name, py_struct", [
     ("moe_layer_shape", moe.MoEShape), ("moe_routing_out", moe.MoERoutingOut),
     ("moe_layer_options", moe.MoEOptions), ("moe_fp8_weights", moe.MoEFp8Weights),
-    ("moe_route_stats", moe.MoERouteStats), ("moe_workspace_layout", moe.MoEWorkspaceLayout)])
+    ("moe_route_stats", moe.MoERouteStats), ("moe_workspace_layout", moe.MoEWorkspaceLayout),
+    ("moe_ep_range", moe.MoEEpRange)])
 def test_binding_structs_match_the_header(c_name, py_struct):
     """Every ctypes structure of the binding has the header's fields, in order, with the same
     C types (pointers as pointers), so that the marshalled bytes are what the library reads."""
@@ -181,3 +182,36 @@ def test_binding_structs_match_the_header(c_name, py_struct):
         else:
             assert ctypes.sizeof(pytype) == ctypes.sizeof(C_TYPES[ctype]), (c_name, f)
             assert (pytype is ctypes.c_float) == (ctype == "float"), (c_name, f)
+
+
+def test_forward_ep_and_sum_partials_reject_bad_arguments_before_any_launch(lib):
+    P = ctypes.c_void_p
+
+    def ep(s, rng, yp=16, ws_bytes=None):
+        nb = moe.workspace_bytes(s) if ws_bytes is None else ws_bytes
+        r = None if rng is None else ctypes.byref(moe.MoEEpRange(*rng))
+        return lib.moe_layer_forward_ep(ctypes.byref(s), P(16), P(16), None, P(16), P(16), P(16), P(16), r,
+                                        P(yp), None, None, P(256), nb if nb else 1 << 40, None)
+    s = shape(T=64)
+    assert ep(s, None) == 1                           # no range
+    assert ep(s, (0, 0, 0, 64)) == 1                  # empty expert range
+    assert ep(s, (10, 289, 0, 64)) == 1               # past E
+    assert ep(s, (-1, 8, 0, 64)) == 1
+    assert ep(s, (0, 36, 10, 5)) == 1                 # shared rows reversed
+    assert ep(s, (0, 36, 0, 65)) == 1                 # shared rows past T
+    assert ep(s, (0, 36, 0, 64), yp=None) == 1        # no partial output
+    assert ep(s, (0, 36, 0, 64), yp=24) == 1          # misaligned partial output
+    assert ep(shape(T=64, dtype=moe.MOE_F32, H=72, I=40, I_shared=24), (0, 36, 0, 64)) == 2  # bf16 only
+    assert ep(s, (0, 36, 0, 64), ws_bytes=moe.workspace_bytes(s) - 1) == 3
+    assert ep(shape(T=0), (0, 36, 0, 0)) == 0          # empty batch
+
+    def sp(T, H, dtype, ptrs, y=16):
+        arr = (ctypes.c_void_p * max(len(ptrs), 1))(*ptrs)
+        return lib.moe_layer_sum_partials(T, H, dtype, len(ptrs), arr, P(y), None)
+    assert sp(4, 64, moe.MOE_BF16, []) == 1
+    assert sp(4, 64, moe.MOE_BF16, [16] * 17) == 1    # more than 16 parts
+    assert sp(4, 60, moe.MOE_BF16, [16]) == 1         # H not a multiple of 8
+    assert sp(4, 64, 9, [16]) == 1
+    assert sp(4, 64, moe.MOE_BF16, [16, 24]) == 1     # misaligned part
+    assert sp(4, 64, moe.MOE_BF16, [16], y=None) == 1
+    assert sp(0, 64, moe.MOE_BF16, [16]) == 0
