@@ -96,7 +96,7 @@ static int num_sms_current_device() {
 static size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
-  size_t ctrl, group_done, tile_done, item_counters, wss, zero_end, scores, xnorm, wnorm, idx, w, blk_hist, counts,
+  size_t ctrl, group_done, tile_done, item_counters, wss, zero_end, scores, fwss, xnorm, wnorm, idx, w, blk_hist, counts,
       offsets, group_order, item_start_gu, item_start_dn, perm, inv_perm, row_w, row_tok, partial, spill, rsplit, w3,
       x_perm, h, h_shared, o, o_shared, total;
   int bn, bn_dn, ksplit;
@@ -132,6 +132,7 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.wss = take(tc_scores ? 0 : groups * E * 8);
   L.scores = take(T * E * 8);
   L.zero_end = tc_scores ? L.scores : off;
+  L.fwss = take(E * 8);  // the fused small-batch routing's sums of squares of W_router rows
   L.spill = take(T * E * 20);
   L.rsplit = take(router_split_bytes(*s));
   L.w3 = take(router_w3_bytes(*s));
@@ -150,7 +151,8 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.row_w = take(P * 4);
   L.row_tok = take(P * 4);
   L.partial = take(L.ksplit > 1 ? static_cast<size_t>(L.max_tiles) * L.ksplit * L.bn * 256 * 4 : 0);
-  // 16-token bf16 tiles gather their token rows from x; wider tiles and fp32 read a copy
+  // bf16 GEMMs gather their token rows from x; fp32, and FP8 weights with 128-token tiles,
+  // read a permuted copy (the workspace size does not depend on the weight format)
   L.x_perm = take(s->dtype == MOE_BF16 && L.bn == 16 ? 0 : P * H * es);
   L.h = take(P * I * es);
   L.h_shared = take(T * Is * es);
@@ -204,7 +206,10 @@ extern "C" moe_status moe_layer_workspace_layout(const moe_layer_shape* shape,
   out->o_shared = L.o_shared;
   out->row_w = L.row_w;
   out->scores = L.scores;
-  out->scores_slice = router_scores_f32(*shape) ? router_slice_len(shape->H) : 0;
+  // fp32 slices on the tensor-core router; fp64 sums on the fused small-batch path (with bf16
+  // router weights) and the CUDA-core router
+  out->scores_slice = router_scores_f32(*shape) && !route_dispatch_fused_supported(*shape, false, L.bn)
+                          ? router_slice_len(shape->H) : 0;
   return MOE_OK;
 }
 
@@ -284,6 +289,11 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
   // FP8 weights run on 16- and 128-token tiles only
   const int bn_dn = wt.w8 ? std::min(L.bn_dn, 128) : L.bn_dn;
+  // long prefill: both GEMMs on 256-row tiles over pairs of SMs (gate/up reads the gathered
+  // copy of x)
+  const bool pair = s.dtype == MOE_BF16 && !wt.w8 && L.ksplit == 1 &&
+                    choose_pair(s.T, s.top_k, s.E, s.H, s.I, s.I_shared);
+  const bool pair_gu = pair, pair_dn = pair;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
@@ -327,8 +337,6 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   ra.idx_user = routing ? routing->topk_idx : nullptr;
   ra.w_user = routing ? routing->topk_w : nullptr;
   ra.ctrl = ctrl;
-  if (launch_router(ra, st) != cudaSuccess) return MOE_ERR_CUDA;
-  marks.mark(1, st);
 
   DispatchArgs da{};
   da.bf16 = bf16;
@@ -341,9 +349,12 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   da.bn = L.bn;
   da.bn_dn = bn_dn;
   da.ksplit = L.ksplit;
+  da.pair_gu = pair_gu;
+  da.pair_dn = pair_dn;
   da.e_lo = e_lo;
   da.e_hi = e_hi;
   da.shared_rows = static_cast<int>(sh_hi - sh_lo);
+  da.need_x_perm = !bf16 || (wt.w8 && L.bn == 128) || pair_gu;
   da.x = x;
   da.idx = ra.idx_ws;
   da.w = ra.w_ws;
@@ -362,7 +373,20 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   da.offsets_user = routing ? routing->offsets : nullptr;
   da.perm_user = routing ? routing->perm : nullptr;
   da.ctrl = ctrl;
-  if (launch_dispatch(da, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (route_dispatch_fused_supported(s, ra.w32, L.bn)) {
+    if (has_shared && !wt.w8) {  // bf16 shared gate/up rows: read first by the gate/up GEMM
+      ra.prefetch = Ws_gate_up;
+      ra.prefetch_bytes = static_cast<int64_t>(2) * s.I_shared * s.H * 2;
+    }
+    // small bf16 batches: routing and dispatch in one launch (the stage marks 0-1 time it)
+    if (launch_route_dispatch_small(ra, da, static_cast<double*>(at(L.fwss)), st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    marks.mark(1, st);
+  } else {
+    if (launch_router(ra, st) != cudaSuccess) return MOE_ERR_CUDA;
+    marks.mark(1, st);
+    if (launch_dispatch(da, st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
   marks.mark(2, st);
 
   ExpertArgs ea{};
@@ -394,6 +418,8 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   ea.row_w = da.row_w;
   ea.x_perm = da.x_perm;
   ea.row_tok = da.row_tok;
+  ea.pair_gu = pair_gu;
+  ea.pair_dn = pair_dn;
   ea.bn = L.bn;
   ea.bn_dn = bn_dn;
   ea.ksplit = L.ksplit;

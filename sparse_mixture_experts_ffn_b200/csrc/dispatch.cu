@@ -17,6 +17,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "dispatch_common.cuh"
 #include "kernels.h"
 
 namespace moe {
@@ -43,152 +44,6 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ i
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     blk_hist[static_cast<int64_t>(blockIdx.x) * E + e] = sh_hist[e];
-}
-
-// exclusive scan of up to 2 * blockDim.x values held two per thread; blockDim.x = 1024
-__device__ int block_scan_pair(int v0, int v1, int* warp_tot, int& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int v = v0 + v1;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) warp_tot[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int s = warp_tot[lane];
-    int si = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, si, o);
-      if (lane >= o) si += y;
-    }
-    warp_tot[lane] = si - s;
-    if (lane == 31) warp_tot[32] = si;
-  }
-  __syncthreads();
-  const int excl = warp_tot[warp] + incl - v;
-  total = warp_tot[32];
-  __syncthreads();
-  return excl;  // exclusive prefix of v0; v1's is excl + v0
-}
-
-struct ScheduleArgs {
-  int64_t T;
-  int E, has_shared, mt_gu, mt_gu_shared, mt_dn, bn, bn_dn, ksplit;
-  int e_lo, e_hi;   // routed experts that get tiles (expert parallelism: this rank's range)
-  int shared_rows;  // rows of the shared-expert group
-  int32_t* offsets;
-  int32_t* group_order;
-  int32_t* item_start_gu;
-  int32_t* item_start_dn;
-  int32_t* offsets_user;
-};
-
-// From the group sizes cnt[0..G) (routed experts, then the shared expert with all T
-// tokens): offsets of the routed experts, the largest-first group order and the tile
-// prefix sums of both grouped GEMMs (gate/up tiles counted ksplit times, once per slice
-// of the reduction).  Block of 1024 threads; cnt/order in shared memory.
-__device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* order, int* warp_tot) {
-  const int E = a.E, G = E + (a.has_shared ? 1 : 0);
-  {
-    const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
-    const int v0 = i0 < E ? cnt[i0] : 0, v1 = i1 < E ? cnt[i1] : 0;
-    int total;
-    const int ex = block_scan_pair(v0, v1, warp_tot, total);
-    if (i0 < E) a.offsets[i0] = ex;
-    if (i1 < E) a.offsets[i1] = ex + v0;
-    if (a.offsets_user) {
-      if (i0 < E) a.offsets_user[i0] = ex;
-      if (i1 < E) a.offsets_user[i1] = ex + v0;
-    }
-    if (threadIdx.x == 0) {
-      a.offsets[E] = total;
-      if (a.offsets_user) a.offsets_user[E] = total;
-    }
-  }
-  // largest group first: rank by (count desc, index asc).  Groups without tokens take the
-  // last places in index order; the others are first compacted (in index order) into the
-  // leading places of order[] and ranked among themselves only.
-  {
-    const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
-    const int z0 = (i0 < G && cnt[i0] > 0) ? 1 : 0, z1 = (i1 < G && cnt[i1] > 0) ? 1 : 0;
-    int nnz;
-    const int nz_ex = block_scan_pair(z0, z1, warp_tot, nnz);
-    if (i0 < G) order[z0 ? nz_ex : nnz + (i0 - nz_ex)] = i0;
-    if (i1 < G) order[z1 ? nz_ex + z0 : nnz + (i1 - nz_ex - z0)] = i1;
-    __syncthreads();
-    auto rank_of = [&](int g) {
-      const int c = cnt[g];
-      int r = 0;
-      for (int j = 0; j < nnz; ++j) {
-        const int h = order[j];
-        const int ch = cnt[h];
-        r += (ch > c) || (ch == c && h < g);
-      }
-      return r;
-    };
-    const int r0 = z0 ? rank_of(i0) : -1, r1 = z1 ? rank_of(i1) : -1;
-    __syncthreads();
-    if (r0 >= 0) order[r0] = i0;
-    if (r1 >= 0) order[r1] = i1;
-    __syncthreads();
-  }
-  for (int r = threadIdx.x; r < G; r += blockDim.x) a.group_order[r] = order[r];
-  const int r0 = 2 * threadIdx.x, r1 = r0 + 1;
-  auto tiles = [&](int r, bool gu) -> int {
-    if (r >= G) return 0;
-    const int g = order[r];
-    const int bn = gu ? a.bn : a.bn_dn;
-    if (g < E && (g < a.e_lo || g >= a.e_hi)) return 0;  // another rank's expert
-    const int nt = (cnt[g] + bn - 1) / bn;
-    const int mt = gu ? (g < E ? a.mt_gu : a.mt_gu_shared) * a.ksplit : a.mt_dn;
-    return nt * mt;
-  };
-  int total;
-  int a0 = tiles(r0, true), a1 = tiles(r1, true);
-  int ex = block_scan_pair(a0, a1, warp_tot, total);
-  if (r0 < G) a.item_start_gu[r0] = ex;
-  if (r1 < G) a.item_start_gu[r1] = ex + a0;
-  if (threadIdx.x == 0) a.item_start_gu[G] = total;
-  a0 = tiles(r0, false);
-  a1 = tiles(r1, false);
-  ex = block_scan_pair(a0, a1, warp_tot, total);
-  if (r0 < G) a.item_start_dn[r0] = ex;
-  if (r1 < G) a.item_start_dn[r1] = ex + a0;
-  if (threadIdx.x == 0) a.item_start_dn[G] = total;
-}
-
-// Stable placement of the assignments [a0, a1) by one warp, 32 at a time, in (token,
-// slot) order: equal experts inside a chunk get consecutive positions in lane order.
-// base[e] holds the next free position of expert e and is advanced.
-__device__ void place_assignments(const int32_t* __restrict__ idx, const float* __restrict__ w,
-                                  int64_t a0, int64_t a1, int k, int E, int* base,
-                                  int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
-                                  float* __restrict__ row_w, int32_t* __restrict__ row_tok,
-                                  int32_t* __restrict__ perm_user) {
-  const int lane = threadIdx.x & 31;
-  for (int64_t c = a0; c < a1; c += 32) {
-    const int64_t a = c + lane;
-    int e = (a < a1) ? idx[a] : -1;
-    if (e < 0 || e >= E) e = -1;  // reported by the histogram
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    int pos = 0;
-    if (e >= 0) pos = base[e] + rank;
-    __syncwarp();
-    if (e >= 0 && rank == 0) base[e] += __popc(peers);
-    __syncwarp();
-    if (e >= 0) {
-      perm[pos] = static_cast<int32_t>(a);
-      inv_perm[a] = pos;
-      row_w[pos] = w[a];
-      row_tok[pos] = static_cast<int32_t>(a / k);
-      if (perm_user) perm_user[pos] = static_cast<int32_t>(a);
-    }
-  }
 }
 
 // One block of 1024 threads: per-expert block prefixes, counts and the schedule.
@@ -275,37 +130,10 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
     int32_t* __restrict__ counts, int32_t* __restrict__ counts_user, int32_t* __restrict__ perm,
     int32_t* __restrict__ inv_perm, float* __restrict__ row_w, int32_t* __restrict__ row_tok,
     int32_t* __restrict__ perm_user, Ctrl* ctrl) {
-  __shared__ int cnt[2048];
-  __shared__ int order[2048];
-  __shared__ int base[1024];
-  __shared__ int warp_tot[33];
+  __shared__ SmallDispatchSmem sm;
   pdl_wait();
   pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
-  const int E = sa.E;
-  const int64_t P = sa.T * k;
-  for (int e = threadIdx.x; e < E + 1; e += blockDim.x) cnt[e] = 0;
-  __syncthreads();
-  for (int64_t a = threadIdx.x; a < P; a += blockDim.x) {
-    const int e = idx[a];
-    if (e < 0 || e >= E) {
-      set_status(ctrl, MOE_ERR_DEVICE_BOUNDS);
-      continue;
-    }
-    atomicAdd(&cnt[e], 1);
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    counts[e] = cnt[e];
-    if (counts_user) counts_user[e] = cnt[e];
-  }
-  if (sa.has_shared && threadIdx.x == 0) cnt[E] = sa.shared_rows;
-  __syncthreads();
-  build_schedule(sa, cnt, order, warp_tot);
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) base[e] = sa.offsets[e];
-  __syncthreads();
-  if (threadIdx.x < 32)
-    place_assignments(idx, w, 0, P, k, E, base, perm, inv_perm, row_w, row_tok, perm_user);
+  dispatch_small_block(sa, idx, w, k, counts, counts_user, perm, inv_perm, row_w, row_tok, perm_user, ctrl, sm);
 }
 
 // x_perm[pos, :] = x[row_tok[pos], :] for the rows of experts [e_lo, e_hi) (all experts,
@@ -354,24 +182,7 @@ constexpr int64_t kSmallDispatch = 4096;
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   const int64_t P = a.T * a.k;
-  ScheduleArgs sa{};
-  sa.T = a.T;
-  sa.E = a.E;
-  sa.has_shared = a.Is > 0 ? 1 : 0;
-  sa.mt_gu = a.I / kTileM;
-  sa.mt_gu_shared = a.Is / kTileM;
-  sa.mt_dn = a.H / kTileM;
-  sa.bn = a.bn;
-  sa.bn_dn = a.bn_dn;
-  sa.ksplit = a.ksplit;
-  sa.e_lo = a.e_lo;
-  sa.e_hi = a.e_hi;
-  sa.shared_rows = a.shared_rows;
-  sa.offsets = a.offsets;
-  sa.group_order = a.group_order;
-  sa.item_start_gu = a.item_start_gu;
-  sa.item_start_dn = a.item_start_dn;
-  sa.offsets_user = a.offsets_user;
+  const ScheduleArgs sa = schedule_args(a);
   cudaError_t e;
   int launches = 0;
   if (P <= kSmallDispatch) {
@@ -399,10 +210,10 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     launches = 3;
   }
-  // 16-token bf16 tiles gather their token rows from x inside the GEMM (row-gather TMA,
-  // four rows per copy); wider tiles, whose copies would be too many, and the fp32 path
-  // read a permuted copy
-  if (a.bf16 && a.bn == 16) {
+  // bf16 GEMMs gather their token rows from x themselves (16-token tiles: row-gather TMA,
+  // four rows per copy; 128-token tiles: gather warps); FP8 weights with 128-token tiles and
+  // the fp32 path read a permuted copy
+  if (a.bf16 && !a.need_x_perm) {
     count_launches(launches);
     return cudaSuccess;
   }

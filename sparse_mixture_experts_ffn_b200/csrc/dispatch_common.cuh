@@ -1,0 +1,233 @@
+// dispatch_common.cuh -- the device code of the dispatch step shared by the dispatch
+// kernels and the fused small-batch routing kernel: block scans, the tile schedule of the
+// grouped expert GEMMs and the stable placement of the assignments.
+//
+// Definitions (the routing of llm-atlas page "Step-3.5-Flash", "Champs bruts du
+// config.json": moe_num_experts, moe_top_k): counts[e] = #{(t,j): idx[t,j] = e};
+// offsets[0] = 0, offsets[e+1] = offsets[e] + counts[e]; perm[offsets[e] + r] = t*k + j for
+// the r-th token (ascending t) routed to e; inv_perm is its inverse.
+#pragma once
+
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+// exclusive scan of up to 2 * blockDim.x values held two per thread (blockDim.x a multiple
+// of 32, at most 1024)
+static __device__ int block_scan_pair(int v0, int v1, int* warp_tot, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int v = v0 + v1;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int s = (lane < static_cast<int>(blockDim.x >> 5)) ? warp_tot[lane] : 0;  // fewer warps: zeros
+    int si = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, si, o);
+      if (lane >= o) si += y;
+    }
+    warp_tot[lane] = si - s;
+    if (lane == 31) warp_tot[32] = si;
+  }
+  __syncthreads();
+  const int excl = warp_tot[warp] + incl - v;
+  total = warp_tot[32];
+  __syncthreads();
+  return excl;  // exclusive prefix of v0; v1's is excl + v0
+}
+
+struct ScheduleArgs {
+  int64_t T;
+  int E, has_shared, mt_gu, mt_gu_shared, mt_dn, bn, bn_dn, ksplit;
+  int e_lo, e_hi;   // routed experts that get tiles (expert parallelism: this rank's range)
+  int shared_rows;  // rows of the shared-expert group
+  int32_t* offsets;
+  int32_t* group_order;
+  int32_t* item_start_gu;
+  int32_t* item_start_dn;
+  int32_t* offsets_user;
+};
+
+// From the group sizes cnt[0..G) (routed experts, then the shared expert with all T
+// tokens): offsets of the routed experts, the largest-first group order and the tile
+// prefix sums of both grouped GEMMs (gate/up tiles counted ksplit times, once per slice
+// of the reduction).  One block with 2 * blockDim.x >= G + 1; cnt/order in shared memory.
+static __device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* order, int* warp_tot) {
+  const int E = a.E, G = E + (a.has_shared ? 1 : 0);
+  {
+    const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
+    const int v0 = i0 < E ? cnt[i0] : 0, v1 = i1 < E ? cnt[i1] : 0;
+    int total;
+    const int ex = block_scan_pair(v0, v1, warp_tot, total);
+    if (i0 < E) a.offsets[i0] = ex;
+    if (i1 < E) a.offsets[i1] = ex + v0;
+    if (a.offsets_user) {
+      if (i0 < E) a.offsets_user[i0] = ex;
+      if (i1 < E) a.offsets_user[i1] = ex + v0;
+    }
+    if (threadIdx.x == 0) {
+      a.offsets[E] = total;
+      if (a.offsets_user) a.offsets_user[E] = total;
+    }
+  }
+  // largest group first: rank by (count desc, index asc).  Groups without tokens take the
+  // last places in index order; the others are first compacted (in index order) into the
+  // leading places of order[] and ranked among themselves only.
+  {
+    const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
+    const int z0 = (i0 < G && cnt[i0] > 0) ? 1 : 0, z1 = (i1 < G && cnt[i1] > 0) ? 1 : 0;
+    int nnz;
+    const int nz_ex = block_scan_pair(z0, z1, warp_tot, nnz);
+    if (i0 < G) order[z0 ? nz_ex : nnz + (i0 - nz_ex)] = i0;
+    if (i1 < G) order[z1 ? nz_ex + z0 : nnz + (i1 - nz_ex - z0)] = i1;
+    __syncthreads();
+    auto rank_of = [&](int g) {
+      const int c = cnt[g];
+      int r = 0;
+      for (int j = 0; j < nnz; ++j) {
+        const int h = order[j];
+        const int ch = cnt[h];
+        r += (ch > c) || (ch == c && h < g);
+      }
+      return r;
+    };
+    const int r0 = z0 ? rank_of(i0) : -1, r1 = z1 ? rank_of(i1) : -1;
+    __syncthreads();
+    if (r0 >= 0) order[r0] = i0;
+    if (r1 >= 0) order[r1] = i1;
+    __syncthreads();
+  }
+  for (int r = threadIdx.x; r < G; r += blockDim.x) a.group_order[r] = order[r];
+  const int r0 = 2 * threadIdx.x, r1 = r0 + 1;
+  auto tiles = [&](int r, bool gu) -> int {
+    if (r >= G) return 0;
+    const int g = order[r];
+    const int bn = gu ? a.bn : a.bn_dn;
+    if (g < E && (g < a.e_lo || g >= a.e_hi)) return 0;  // another rank's expert
+    const int nt = (cnt[g] + bn - 1) / bn;
+    const int mt = gu ? (g < E ? a.mt_gu : a.mt_gu_shared) * a.ksplit : a.mt_dn;
+    return nt * mt;
+  };
+  int total;
+  int a0 = tiles(r0, true), a1 = tiles(r1, true);
+  int ex = block_scan_pair(a0, a1, warp_tot, total);
+  if (r0 < G) a.item_start_gu[r0] = ex;
+  if (r1 < G) a.item_start_gu[r1] = ex + a0;
+  if (threadIdx.x == 0) a.item_start_gu[G] = total;
+  a0 = tiles(r0, false);
+  a1 = tiles(r1, false);
+  ex = block_scan_pair(a0, a1, warp_tot, total);
+  if (r0 < G) a.item_start_dn[r0] = ex;
+  if (r1 < G) a.item_start_dn[r1] = ex + a0;
+  if (threadIdx.x == 0) a.item_start_dn[G] = total;
+}
+
+// Stable placement of the assignments [a0, a1) by one warp, 32 at a time, in (token,
+// slot) order: equal experts inside a chunk get consecutive positions in lane order.
+// base[e] holds the next free position of expert e and is advanced.
+static __device__ void place_assignments(const int32_t* __restrict__ idx, const float* __restrict__ w,
+                                  int64_t a0, int64_t a1, int k, int E, int* base,
+                                  int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
+                                  float* __restrict__ row_w, int32_t* __restrict__ row_tok,
+                                  int32_t* __restrict__ perm_user) {
+  const int lane = threadIdx.x & 31;
+  for (int64_t c = a0; c < a1; c += 32) {
+    const int64_t a = c + lane;
+    int e = (a < a1) ? idx[a] : -1;
+    if (e < 0 || e >= E) e = -1;  // reported by the histogram
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    int pos = 0;
+    if (e >= 0) pos = base[e] + rank;
+    __syncwarp();
+    if (e >= 0 && rank == 0) base[e] += __popc(peers);
+    __syncwarp();
+    if (e >= 0) {
+      perm[pos] = static_cast<int32_t>(a);
+      inv_perm[a] = pos;
+      row_w[pos] = w[a];
+      row_tok[pos] = static_cast<int32_t>(a / k);
+      if (perm_user) perm_user[pos] = static_cast<int32_t>(a);
+    }
+  }
+}
+
+// shared memory of the single-block dispatch
+struct SmallDispatchSmem {
+  int cnt[2048];
+  int order[2048];
+  int base[1024];
+  int warp_tot[33];
+};
+
+// The whole dispatch of a small batch by one block of 1024 threads: histogram, counts,
+// offsets and the tile schedule, then the stable placement (one warp).
+static __device__ void dispatch_small_block(const ScheduleArgs& sa, const int32_t* __restrict__ idx,
+                                            const float* __restrict__ w, int k, int32_t* __restrict__ counts,
+                                            int32_t* __restrict__ counts_user, int32_t* __restrict__ perm,
+                                            int32_t* __restrict__ inv_perm, float* __restrict__ row_w,
+                                            int32_t* __restrict__ row_tok, int32_t* __restrict__ perm_user,
+                                            Ctrl* ctrl, SmallDispatchSmem& sm) {
+  const int E = sa.E;
+  const int64_t P = sa.T * k;
+  for (int e = threadIdx.x; e < E + 1; e += blockDim.x) sm.cnt[e] = 0;
+  __syncthreads();
+  for (int64_t a = threadIdx.x; a < P; a += blockDim.x) {
+    const int e = idx[a];
+    if (e < 0 || e >= E) {
+      set_status(ctrl, MOE_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    atomicAdd(&sm.cnt[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    counts[e] = sm.cnt[e];
+    if (counts_user) counts_user[e] = sm.cnt[e];
+  }
+  if (sa.has_shared && threadIdx.x == 0) sm.cnt[E] = sa.shared_rows;
+  __syncthreads();
+  build_schedule(sa, sm.cnt, sm.order, sm.warp_tot);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) sm.base[e] = sa.offsets[e];
+  __syncthreads();
+  if (threadIdx.x < 32)
+    place_assignments(idx, w, 0, P, k, E, sm.base, perm, inv_perm, row_w, row_tok, perm_user);
+}
+
+// The schedule arguments of a dispatch (tile shapes of both grouped GEMMs).
+inline ScheduleArgs schedule_args(const DispatchArgs& a) {
+  ScheduleArgs sa{};
+  sa.T = a.T;
+  sa.E = a.E;
+  sa.has_shared = a.Is > 0 ? 1 : 0;
+  const int tm_gu = a.pair_gu ? 2 * kTileM : kTileM;  // weight rows per tile
+  const int tm_dn = a.pair_dn ? 2 * kTileM : kTileM;
+  sa.mt_gu = a.I / tm_gu;
+  sa.mt_gu_shared = a.Is / tm_gu;
+  sa.mt_dn = a.H / tm_dn;
+  sa.bn = a.pair_gu ? 128 : a.bn;  // pair tiles: 128 tokens for gate/up, 256 for down
+  sa.bn_dn = a.pair_dn ? 256 : a.bn_dn;
+  sa.ksplit = a.ksplit;
+  sa.e_lo = a.e_lo;
+  sa.e_hi = a.e_hi;
+  sa.shared_rows = a.shared_rows;
+  sa.offsets = a.offsets;
+  sa.group_order = a.group_order;
+  sa.item_start_gu = a.item_start_gu;
+  sa.item_start_dn = a.item_start_dn;
+  sa.offsets_user = a.offsets_user;
+  return sa;
+}
+
+}  // namespace moe

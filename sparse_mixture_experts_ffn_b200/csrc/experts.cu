@@ -42,6 +42,8 @@ struct TcParams {
   const float* row_w;          // routing weight per routed row (down projection only)
   const int32_t* row_tok;      // token of each routed row (gather)
   int gather;                  // routed token rows gathered from x by tmB[0] (gate/up)
+  const __nv_bfloat16* x;      // tokens [T, H] (gate/up with 128-token tiles: rows gathered
+                               // by the gather warps, routed and shared alike)
   __nv_bfloat16* out[2];       // [0] routed rows, [1] shared rows
   int ld_out[2];               // row stride of out (elements), routed and shared
   int E, G;
@@ -62,6 +64,13 @@ struct TcParams {
   float* partial;              // [max_tiles][ksplit][BN][256] fp32 gate|up partial sums
   unsigned int* tile_done;     // [max_tiles] slices finished per tile, zero before the launch
   unsigned int* item_counter;  // items claimed beyond the first gridDim.x, zero before the launch
+  // gate/up: the down GEMM's schedule and weights, so that a block out of work brings the
+  // weight rows of the down GEMM's item blockIdx.x into L2 (null: no prefetch)
+  const int32_t* pf_item_start;    // [G + 1] item prefix of the down GEMM
+  const unsigned char* pf_w[2];    // W_down (this launch's experts), Ws_down
+  int pf_bn, pf_mt;                // tokens per down tile, weight tiles per group
+  int64_t pf_rows_per_group;       // rows of one routed expert's down matrix (H)
+  int64_t pf_row_bytes[2];         // bytes of one row: routed (I), shared (I_shared)
   const uint8_t* scaleA[2];    // FP8 weights: E8M0 block scales of the A matrices, routed
                                // (stacked by expert) and shared
   int s_rows_per_group;        // FP8 weights: scale rows (128-row blocks) per routed expert
@@ -90,7 +99,10 @@ struct TcCfg {
   static constexpr int kConvStages = W8 ? (BN <= 16 ? (GATED ? 3 : 4) : 2) : 0;
   static constexpr int kConvBOffset = kMats * kABytes;
   static constexpr int kConvBytes = kConvBOffset + kBBytes;
-  static constexpr int kThreads = W8 ? 192 + 128 * kConvGroups : 192;
+  // bf16 gate/up with 128-token tiles: four more warps gather the tiles' token rows from x
+  // (cp.async, 16 bytes per lane), so no permuted copy of x is written and read back
+  static constexpr bool kCpGather = GATED && BN == 128 && !W8;
+  static constexpr int kThreads = W8 ? 192 + 128 * kConvGroups : (kCpGather ? 192 + 128 : 192);
   static constexpr int kConvMod = kConvStages > 0 ? kConvStages : 1;  // a divisor in every variant
   // tiles of up to 128 tokens stage the output tile [BN][128] bf16 in shared memory for
   // 16-byte stores; 256-token tiles store straight from registers (each warp writes 64
@@ -261,8 +273,21 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 // then takes the next unclaimed one from a global counter, so blocks that draw short tiles
 // take more of them; the producer publishes each claimed item to the MMA and epilogue warps
 // through a ring of kRing shared-memory slots (index -1 ends the schedule).
+// 16 bytes global -> shared, bypassing L1; `bytes` = 0 fills the 16 bytes with zeros
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src, uint32_t bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src),
+               "r"(bytes)
+               : "memory");
+}
+// the mbarrier receives one arrival once every cp.async issued so far by this thread has
+// landed (counted in the barrier's expected arrivals)
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 template <bool GATED, int BN, bool W8>
-__global__ void __launch_bounds__(W8 ? 192 + 128 * kConvGroups : 192, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
   using C = TcCfg<GATED, BN, W8>;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -289,7 +314,7 @@ __global__ void __launch_bounds__(W8 ? 192 + 128 * kConvGroups : 192, 1) expert_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], C::kCpGather ? 1 + 128 : 1);  // + one per gather thread
       mbar_init(&empty[s], W8 ? 4 : 1);  // the MMA commit, or (FP8) the four converter warps
     }
     for (int a = 0; a < 2; ++a) {
@@ -300,7 +325,7 @@ __global__ void __launch_bounds__(W8 ? 192 + 128 * kConvGroups : 192, 1) expert_
     for (int q = 0; q < kRing; ++q) {
       mbar_init(&ring_full[q], 1);
       // the MMA thread and one lane per epilogue (and converter) warp
-      mbar_init(&ring_empty[q], 1 + 4 + (W8 ? 4 * kConvGroups : 0));
+      mbar_init(&ring_empty[q], 1 + 4 + (W8 ? 4 * kConvGroups : 0) + (C::kCpGather ? 4 : 0));
     }
     for (int c = 0; c < C::kConvStages; ++c) {
       mbar_init(&cfull[c], 4);    // one lane per warp of the converter group
@@ -440,12 +465,13 @@ __global__ void __launch_bounds__(W8 ? 192 + 128 * kConvGroups : 192, 1) expert_
           good = wait(&empty[stage], phase ^ 1u) ? 1 : 0;
           if (good) {
             if (W8) sc_stage[stage] = scw;  // published by the arrive below
-            mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+            mbar_arrive_expect_tx(&full[stage], C::kCpGather ? C::kBOffset : C::kStageBytes);
             tma_load_2d(st, &p.tmA[t.sh], kb * kTileK, arow, &full[stage]);
             if (GATED)
               tma_load_2d(st + (W8 ? C::kA8Bytes : C::kABytes), &p.tmA[t.sh], kb * kTileK,
                           arow + p.a_up_offset[t.sh], &full[stage]);
-            if (!gath) tma_load_2d(st + C::kBOffset, &p.tmB[t.sh], kb * kTileK, t.row0, &full[stage]);
+            if (!gath && !C::kCpGather)
+              tma_load_2d(st + C::kBOffset, &p.tmB[t.sh], kb * kTileK, t.row0, &full[stage]);
           }
         }
         good = __shfl_sync(0xffffffffu, good, 0);
@@ -458,6 +484,24 @@ __global__ void __launch_bounds__(W8 ? 192 + 128 * kConvGroups : 192, 1) expert_
       }
     }
     __syncwarp();
+    if (GATED && !W8 && p.pf_item_start && lane == 0 && static_cast<int>(blockIdx.x) < __ldg(p.pf_item_start + p.G)) {
+      // out of work: the rows of the down GEMM's item blockIdx.x (its first wave) into L2
+      const int itd = static_cast<int>(blockIdx.x);
+      int lo = 0, hi = p.G - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(p.pf_item_start + mid) <= itd) lo = mid; else hi = mid - 1;
+      }
+      const int g = sc.ld(sc.group_order + lo);
+      const int sh = (g == p.E) ? 1 : 0;
+      const int cnt = sh ? p.sh_rows : sc.ld(sc.offsets + g + 1) - sc.ld(sc.offsets + g);
+      const int ntile = (cnt + p.pf_bn - 1) / p.pf_bn;
+      const int m = ntile > 0 ? (itd - __ldg(p.pf_item_start + lo)) / ntile : -1;
+      if (m >= 0 && m < p.pf_mt && (sh || (g >= p.g_lo && g < p.g_hi))) {
+        const int64_t row = (sh ? 0 : (g - p.g_lo) * p.pf_rows_per_group) + static_cast<int64_t>(m) * kTileM;
+        prefetch_l2(p.pf_w[sh] + row * p.pf_row_bytes[sh], static_cast<uint64_t>(kTileM) * p.pf_row_bytes[sh]);
+      }
+    }
     // every copy issued must have landed before the block exits
     if (lane == 0)
       for (int s = 0; s < C::kStages; ++s) {
@@ -493,6 +537,9 @@ __global__ void __launch_bounds__(W8 ? 192 + 128 * kConvGroups : 192, 1) expert_
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!(W8 ? wait(&cfull[cs], cphase) : wait(&full[stage], phase))) { ok = false; break; }
           tc_fence_after();
+          // token rows written by the gather warps' cp.async: order them before the
+          // tensor cores' (async-proxy) reads of the stage
+          if (C::kCpGather) fence_proxy_async_smem();
           const uint32_t s0 = W8 ? smem_u32(conv + cs * C::kConvBytes) : smem_u32(smem + stage * C::kStageBytes);
           const uint32_t a0 = s0;
           const uint32_t b0 = s0 + (W8 ? C::kConvBOffset : C::kBOffset);
@@ -520,6 +567,62 @@ __global__ void __launch_bounds__(W8 ? 192 + 128 * kConvGroups : 192, 1) expert_
       mma_commit(drain);
       mbar_wait_drain(drain, 0, p.ctrl);
     }
+  } else if (C::kCpGather && warp >= 6) {
+    // --------------------- token-row gather (warps 6..9, 128-token tiles) ---------------
+    // Each k-step's B tile is 128 token rows x 64 columns (128 bytes a row), written where a
+    // 128-byte-swizzled TMA load would put them: chunk c of row n at chunk c ^ (n % 8).
+    // Lane l of gather warp w copies chunk l % 8 of rows 32w + 4i + l / 8 (i = 0..7), so a
+    // warp's eight lanes per row read one 128-byte line.  Rows past the tile's tokens are
+    // zero-filled.  Routed rows come from x[row_tok[row]], shared-expert rows from x[row].
+    const int gw = warp - 6;
+    const int c = lane & 7;
+    int stage = 0;
+    uint32_t phase = 0;
+    int q = 0;
+    uint32_t qphase = 0;
+    bool ok = true;
+    while (ok) {
+      if (!wait(&ring_full[q], qphase)) break;
+      const int it = ring[q];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ring_empty[q]);
+      if (++q == kRing) { q = 0; qphase ^= 1u; }
+      if (it < 0) break;
+      const Item t = decode_item<BN>(p, sc, it);
+      if (!t.valid) continue;
+      const __nv_bfloat16* src[8];
+      uint32_t nbytes[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int n = 32 * gw + 4 * i + (lane >> 3);
+        int64_t tok = 0;
+        nbytes[i] = 0;
+        if (n < t.nvalid) {
+          tok = t.sh ? static_cast<int64_t>(t.row0 + n) : static_cast<int64_t>(__ldg(p.row_tok + t.row0 + n));
+          if (tok < 0 || tok >= p.T) {
+            set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
+            tok = 0;
+          } else {
+            nbytes[i] = 16;
+          }
+        }
+        src[i] = p.x + tok * (static_cast<int64_t>(p.kblocks[0]) * kTileK) + c * 8;
+      }
+      const int kb_n = p.kblocks[t.sh];
+      const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!wait(&empty[stage], phase ^ 1u)) { ok = false; break; }
+        unsigned char* bt = smem + stage * C::kStageBytes + C::kBOffset;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int n = 32 * gw + 4 * i + (lane >> 3);
+          cp_async16(bt + n * 128 + ((c ^ (n & 7)) << 4), src[i] + kb * kTileK, nbytes[i]);
+        }
+        cp_async_arrive_noinc(&full[stage]);
+        if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    cp_async_wait_all();  // this thread's copies land before the block exits
   } else if (W8 && warp >= 6) {
     // ------------------------ FP8 code tiles -> bf16 (warps 6..13) --------------------
     // Group g converts the block's k-steps n with n % 2 == g, so one group's waits and
@@ -710,6 +813,215 @@ __global__ void __launch_bounds__(W8 ? 192 + 128 * kConvGroups : 192, 1) expert_
 }
 
 // ---------------------------------------------------------------------------------------
+// Pair tiles for long prefill (on average 256 or more tokens per expert): a cluster of two
+// CTAs on two SMs computes one 256-row weight tile x BN-token tile with tcgen05.mma
+// cta_group::2.  CTA c of the pair holds weight rows [128c, 128c + 128) of the tile and
+// token rows [c BN/2, (c + 1) BN/2) in its own shared memory; the even CTA's single MMA
+// thread multiplies the pair's 256 x BN tile, each CTA's tensor memory receiving its own 128
+// weight rows for all BN tokens.  Each SM thus loads half the token rows a single-SM tile of
+// the same shape would:
+//   gate/up (BN = 128): the CTA's 128 gate rows and its 128 up rows of the same
+//            intermediate units, two MMAs per step sharing the token rows (x_perm, the
+//            routed rows of x in expert order; the shared expert's rows of x); accumulators
+//            gate | up, 256 columns, two buffers;
+//   down (BN = 256): one MMA per step, 256 columns, two buffers; the routing weight in
+//            the epilogue.
+// Work items (group, 256-row weight tile, token tile) are taken in a fixed order, pair q
+// doing items q, q + pairs, ...; both CTAs walk the same sequence.  TMA loads of both CTAs
+// complete on the even CTA's barrier; the MMA commits arrive on both CTAs' barriers; both
+// epilogues release an accumulator on the even CTA's barrier.
+// ---------------------------------------------------------------------------------------
+template <bool GATED>
+struct PairCfg {
+  static constexpr int BN = GATED ? 128 : 256;          // tokens per pair tile
+  static constexpr int kMats = GATED ? 2 : 1;
+  static constexpr int kABytes = kTileM * kTileK * 2;  // this CTA's 128 rows of one matrix
+  static constexpr int kBRows = BN / 2;                // this CTA's token rows
+  static constexpr int kBBytes = kBRows * kTileK * 2;
+  static constexpr int kBOffset = kMats * kABytes;
+  static constexpr int kStageBytes = kBOffset + kBBytes;
+  static constexpr int kThreads = 192;
+  static constexpr int kChunk = 32;                    // tokens per epilogue chunk
+  static constexpr int kStagingBytes = kChunk * kTileM * 2;
+  static constexpr int kAuxBytes = 2048;               // barriers, TMEM slot, row weights
+  static constexpr int kFit = (kMaxDynSmem - kStagingBytes - 1024 - kAuxBytes) / kStageBytes;
+  static constexpr int kStages = kFit > 8 ? 8 : kFit;
+  static constexpr int kAccCols = (GATED ? 2 : 1) * BN;
+  static constexpr int kAccBufs = 2;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + kAuxBytes;
+  static_assert(kStages >= 3 && kSmemBytes <= kMaxDynSmem, "shared memory budget");
+  static_assert(kStageBytes % 1024 == 0 && kBOffset % 1024 == 0, "stages keep the swizzle alignment");
+  static_assert(kAccBufs * kAccCols <= 512, "tensor memory");
+};
+
+template <bool GATED>
+__global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_kernel(const __grid_constant__ TcParams p) {
+  using C = PairCfg<GATED>;
+  constexpr int BN = C::BN;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  unsigned char* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+  __nv_bfloat16* staging = reinterpret_cast<__nv_bfloat16*>(smem + C::kStages * C::kStageBytes);
+  unsigned char* aux = smem + C::kStages * C::kStageBytes + C::kStagingBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(aux);   // [kStages], used on the even CTA
+  uint64_t* empty = full + 8;                          // [kStages]
+  uint64_t* tfull = empty + 8;                         // [2]
+  uint64_t* tempty = tfull + 2;                        // [2], used on the even CTA
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* sw = reinterpret_cast<float*>(aux + 1024);    // [256] routing weights of the tile
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();             // 0: the pair's MMA issuer
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);   // the even CTA's expect_tx; bytes of both CTAs
+      mbar_init(&empty[s], 1);  // the pair's MMA commit
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * 4);  // one lane per epilogue warp of each CTA
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, 512);
+  tc_fence_before();
+  cluster_sync();  // barriers initialised in both CTAs before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+  const Sched sc{p.item_start, p.group_order, p.offsets, false};
+  const int total = schedule_length(p, sc);
+  const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
+
+  if (warp == 0) {
+    // ------------------------------- TMA producer (both CTAs) -------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int it = pair; it < total && ok; it += npairs) {
+        const Item t = decode_item<BN>(p, sc, it);
+        if (!t.valid) {
+          if (blockIdx.x == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
+          continue;
+        }
+        const int arow = (t.sh ? 0 : (t.g - p.g_lo) * p.a_rows_per_group) + t.m * 256 + static_cast<int>(rank) * 128;
+        const int brow = t.row0 + static_cast<int>(rank) * C::kBRows;
+        for (int kb = 0; kb < p.kblocks[t.sh]; ++kb) {
+          if (!mbar_wait_cluster(&empty[stage], phase ^ 1u, p.ctrl, abort_flag)) { ok = false; break; }
+          unsigned char* st = smem + stage * C::kStageBytes;
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
+          tma_load_2d_pair(st, &p.tmA[t.sh], kb * kTileK, arow, fb);
+          if (GATED) tma_load_2d_pair(st + C::kABytes, &p.tmA[t.sh], kb * kTileK, arow + p.a_up_offset[t.sh], fb);
+          tma_load_2d_pair(st + C::kBOffset, &p.tmB[t.sh], kb * kTileK, brow, fb);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (rank == 0 && lane == 0) {
+      // ----------------------------- MMA issuer (even CTA) ----------------------------
+      const uint32_t idesc = idesc_bf16_f32(256, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int it = pair; it < total && ok; it += npairs) {
+        const Item t = decode_item<BN>(p, sc, it);
+        if (!t.valid) continue;
+        if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, p.ctrl, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + acc * C::kAccCols;
+        for (int kb = 0; kb < p.kblocks[t.sh]; ++kb) {
+          if (!mbar_wait_cluster(&full[stage], phase, p.ctrl, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t b0 = a0 + C::kBOffset;
+#pragma unroll
+          for (int kk = 0; kk < kTileK / 16; ++kk) {
+            const uint32_t accum = (kb || kk) ? 1u : 0u;
+            const uint64_t bdesc = sw128_kmajor_desc(b0 + kk * 32);
+            mma_bf16_pair(d0, sw128_kmajor_desc(a0 + kk * 32), bdesc, idesc, accum);
+            if (GATED) mma_bf16_pair(d0 + BN, sw128_kmajor_desc(a0 + C::kABytes + kk * 32), bdesc, idesc, accum);
+          }
+          mma_commit_pair(&empty[stage]);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit_pair(&tfull[acc]);
+        if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
+      }
+      mma_commit_pair(drain);  // every MMA of the pair done before the accumulators are freed
+      mbar_wait_drain(drain, 0, p.ctrl);
+    }
+  } else {
+    // ------------------------------- epilogue (warps 2..5, both CTAs) -----------------
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // this CTA's weight row = output column
+    const int et = threadIdx.x - 64;
+    const uint32_t tempty_even0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_even1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int it = pair; it < total; it += npairs) {
+      const Item t = decode_item<BN>(p, sc, it);
+      if (!t.valid) continue;
+      if (!GATED) {
+        for (int n = et; n < BN; n += 128) sw[n] = (t.sh || n >= t.nvalid) ? 1.0f : __ldg(p.row_w + t.row0 + n);
+        named_bar_sync(1, 128);
+      }
+      if (!mbar_wait_cluster(&tfull[acc], acc_phase, p.ctrl, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::kAccCols;
+      const int ld = p.ld_out[t.sh];
+      __nv_bfloat16* out = p.out[t.sh] + static_cast<int64_t>(t.row0) * ld + t.m * 256 + static_cast<int>(rank) * 128;
+      for (int c0 = 0; c0 < t.nvalid; c0 += C::kChunk) {
+        uint32_t a[32];
+        tmem_ld16_nowait(trow + c0, a);
+        tmem_ld16_nowait(trow + c0 + 16, a + 16);
+        uint32_t u[GATED ? 32 : 1];
+        if (GATED) {
+          tmem_ld16_nowait(trow + BN + c0, u);
+          tmem_ld16_nowait(trow + BN + c0 + 16, u + 16);
+        }
+        tmem_wait_ld();
+        if (c0 + C::kChunk >= t.nvalid) {  // the accumulator has been read: release it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(acc ? tempty_even1 : tempty_even0);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          float v;
+          if (GATED) v = swiglu(__uint_as_float(a[j]), __uint_as_float(u[GATED ? j : 0]), p.limit[t.sh]);
+          else v = __uint_as_float(a[j]) * sw[c0 + j];
+          staging[j * kTileM + r] = __float2bfloat16_rn(v);
+        }
+        named_bar_sync(1, 128);
+        // rows of 128 bf16 (256 B) -> out[row0 + c0 + j][...], 16-byte coalesced stores
+        const int rows = min(C::kChunk, t.nvalid - c0);
+        const uint4* src = reinterpret_cast<const uint4*>(staging);
+        for (int i = et; i < rows * 16; i += 128) {
+          const int j = i >> 4, cc = i & 15;
+          *reinterpret_cast<uint4*>(out + static_cast<int64_t>(c0 + j) * ld + cc * 8) = src[j * 16 + cc];
+        }
+        named_bar_sync(1, 128);  // staging (and sw) free again
+      }
+      if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the pair's MMAs may still read its operands
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, 512);
+}
+
+// ---------------------------------------------------------------------------------------
 // fp32 CUDA-core path
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ int group_of_row(const int32_t* offsets, int E, int p) {
@@ -851,6 +1163,31 @@ static cudaError_t launch_tc(const TcParams& prm_in, int num_sms, cudaStream_t s
 }
 
 template <bool GATED>
+static cudaError_t launch_pair(const TcParams& prm, int num_sms, cudaStream_t st) {
+  using C = PairCfg<GATED>;
+  auto kern = expert_gemm_pair_kernel<GATED>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, kern, prm);
+  count_launches(1);
+  return e;
+}
+
+template <bool GATED>
 static cudaError_t launch_tc_bn(const TcParams& prm, int bn, bool w8, int num_sms, cudaStream_t st) {
   if (w8) {  // FP8 weights: 16- and 128-token tiles
     if (bn == 16) return launch_tc<GATED, 16, true>(prm, num_sms, st);
@@ -899,6 +1236,13 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   // (16-token tiles) or x_perm [P, H] (shared: x [T, H] in order)
   TcParams g{};
   const bool gather = a.bn == 16;
+  // bf16 128-token tiles gather their token rows inside the kernel (no x_perm); FP8 weights
+  // read the permuted copy
+  const bool cp_gather = !a.pair_gu && a.bn == 128 && !a.w8;
+  // token rows per B copy (pair tiles: each CTA's half; the gate/up pair kernel gathers its
+  // rows itself and never uses its B maps)
+  const uint32_t box_gu = a.pair_gu ? 64 : static_cast<uint32_t>(a.bn);
+  const uint32_t box_dn = a.pair_dn ? 128 : static_cast<uint32_t>(a.bn_dn);
   // weight matrices: bf16 rows, or FP8 code rows with their block scales
   auto encode_w = [&](CUtensorMap* m, const void* w, uint64_t rows, uint64_t cols) {
     return a.w8 ? encode_2d_u8(m, w, rows, cols) : encode_2d_bf16(m, w, rows, cols, kTileM);
@@ -906,10 +1250,10 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   const uint64_t n_local = static_cast<uint64_t>(a.e_hi - a.e_lo);  // routed experts held
   bool ok = encode_w(&g.tmA[0], a.Wgu, n_local * 2 * a.I, a.H) &&
             (gather ? encode_2d_bf16(&g.tmB[0], a.x, a.T, a.H, 1)
-                    : encode_2d_bf16(&g.tmB[0], a.x_perm, P, a.H, a.bn));
+                    : encode_2d_bf16(&g.tmB[0], cp_gather ? a.x : a.x_perm, cp_gather ? a.T : P, a.H, box_gu));
   if (has_shared)
     ok = ok && encode_w(&g.tmA[1], a.Wsgu, 2ull * a.Is, a.H) &&
-         encode_2d_bf16(&g.tmB[1], a.x, a.T, a.H, a.bn);
+         encode_2d_bf16(&g.tmB[1], a.x, a.T, a.H, box_gu);
   else {
     g.tmA[1] = g.tmA[0];
     g.tmB[1] = g.tmB[0];
@@ -923,6 +1267,17 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   g.limit[0] = a.swiglu_limit;
   g.limit[1] = a.swiglu_limit_shared;
   g.gather = gather ? 1 : 0;
+  g.x = static_cast<const __nv_bfloat16*>(a.x);
+  if (!a.w8 && !a.pair_dn) {
+    g.pf_item_start = a.item_start_dn;
+    g.pf_w[0] = static_cast<const unsigned char*>(a.Wd);
+    g.pf_w[1] = static_cast<const unsigned char*>(has_shared ? a.Wsd : a.Wd);
+    g.pf_bn = a.bn_dn;
+    g.pf_mt = a.H / kTileM;
+    g.pf_rows_per_group = a.H;
+    g.pf_row_bytes[0] = static_cast<int64_t>(a.I) * 2;
+    g.pf_row_bytes[1] = static_cast<int64_t>(a.Is) * 2;
+  }
   g.out[0] = static_cast<__nv_bfloat16*>(a.h);
   g.out[1] = static_cast<__nv_bfloat16*>(a.h_shared);
   g.E = a.E;
@@ -953,16 +1308,22 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   g.scaleA[1] = static_cast<const uint8_t*>(a.Wsgu_scale);
   g.s_rows_per_group = 2 * a.I / kTileM;
   g.s_ld[0] = g.s_ld[1] = (a.H + 127) / 128;
-  cudaError_t e = launch_tc_bn<true>(g, a.bn, a.w8, a.num_sms, st);
+  if (a.pair_gu) {  // 256-row weight tiles over pairs of SMs, 128-token tiles
+    g.mt[0] = a.I / 256;
+    g.mt[1] = a.Is / 256;
+    g.max_tiles = static_cast<int>(expert_tile_bound(a.T, a.k, a.E, a.I / 2, a.Is / 2, 128));
+    g.max_items = g.max_tiles;
+  }
+  cudaError_t e = a.pair_gu ? launch_pair<true>(g, a.num_sms, st) : launch_tc_bn<true>(g, a.bn, a.w8, a.num_sms, st);
   if (e != cudaSuccess) return e;
   if (a.stage_mark) a.stage_mark(a.stage_mark_ctx, 3, st);
   // down: A = W_down viewed as [E*H, I]; B = h [P, I] (shared: Ws_down [H, Is], h_shared)
   TcParams d{};
   ok = encode_w(&d.tmA[0], a.Wd, n_local * a.H, a.I) &&
-       encode_2d_bf16(&d.tmB[0], a.h, P, a.I, a.bn_dn);
+       encode_2d_bf16(&d.tmB[0], a.h, P, a.I, box_dn);
   if (has_shared)
     ok = ok && encode_w(&d.tmA[1], a.Wsd, a.H, a.Is) &&
-         encode_2d_bf16(&d.tmB[1], a.h_shared, a.T, a.Is, a.bn_dn);
+         encode_2d_bf16(&d.tmB[1], a.h_shared, a.T, a.Is, box_dn);
   else {
     d.tmA[1] = d.tmA[0];
     d.tmB[1] = d.tmB[0];
@@ -999,6 +1360,12 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   d.s_rows_per_group = a.H / kTileM;
   d.s_ld[0] = (a.I + 127) / 128;
   d.s_ld[1] = (a.Is + 127) / 128;
+  if (a.pair_dn) {
+    d.mt[0] = d.mt[1] = a.H / 256;
+    d.max_tiles = static_cast<int>(expert_tile_bound(a.T, a.k, a.E, a.H / 2, a.Is > 0 ? a.H / 2 : 0, 256));
+    d.max_items = d.max_tiles;
+    return launch_pair<false>(d, a.num_sms, st);
+  }
   return launch_tc_bn<false>(d, a.bn_dn, a.w8, a.num_sms, st);
 }
 

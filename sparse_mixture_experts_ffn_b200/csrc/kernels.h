@@ -30,6 +30,11 @@ inline int choose_tile_n_down(int64_t T, int k, int E) {
   const int bn = choose_tile_n(T, k, E);
   return (bn == 128 && T * k >= static_cast<int64_t>(256) * E) ? 256 : bn;
 }
+// long prefill (256 or more tokens per expert on average) with bf16 weights whose sizes are
+// multiples of 256: both GEMMs use 256 x 256 tiles over pairs of SMs
+inline bool choose_pair(int64_t T, int k, int E, int H, int I, int Is) {
+  return T * k >= static_cast<int64_t>(256) * E && H % 256 == 0 && I % 256 == 0 && Is % 256 == 0;
+}
 
 struct RouterArgs {
   bool bf16;
@@ -53,6 +58,8 @@ struct RouterArgs {
   void* rsplit;      // router_split_bytes(shape) bytes, or null: the reduction is not split
   bool w32;          // bf16 tokens with fp32 router weights (Wr is float [E, H])
   void* w3;          // router_w3_bytes(shape): the fp32 weights split into 3 bf16 parts
+  const void* prefetch = nullptr;  // fused small-batch routing: bytes to bring into L2 meanwhile
+  int64_t prefetch_bytes = 0;      // (a multiple of 16)
   Ctrl* ctrl;
 };
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
@@ -74,11 +81,14 @@ struct DispatchArgs {
   int64_t T;
   int H, E, k;
   int I, Is;        // expert widths (Is = 0: no shared expert)
+  bool pair_gu;     // gate/up GEMM on 256-row x 128-token tiles over pairs of SMs
+  bool pair_dn;     // down GEMM on 256-row x 256-token tiles over pairs of SMs
   int bn;           // tokens per gate/up GEMM tile
   int bn_dn;        // tokens per down GEMM tile
   int ksplit;       // gate/up reduction slices
   int e_lo, e_hi;   // routed experts whose rows are computed: [0, E), or one rank's range
   int shared_rows;  // rows of the shared-expert group (T, or one rank's token slice)
+  bool need_x_perm; // the GEMMs read a permuted copy of x (fp32; FP8 weights with 128-token tiles)
   const void* x;
   const int32_t* idx;   // [T, k]
   const float* w;       // [T, k]
@@ -99,6 +109,12 @@ struct DispatchArgs {
   Ctrl* ctrl;
 };
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st);
+
+// Small bf16 batches: routing and dispatch in one launch (replaces launch_router and
+// launch_dispatch).  wss: [E] fp64 scratch for the experts' sums of squares.
+bool route_dispatch_fused_supported(const moe_layer_shape& s, bool w32, int bn);
+cudaError_t launch_route_dispatch_small(const RouterArgs& a, const DispatchArgs& da, double* wss,
+                                        cudaStream_t st);
 
 struct ExpertArgs {
   bool bf16;
@@ -124,6 +140,8 @@ struct ExpertArgs {
   const float* row_w;
   const int32_t* row_tok;  // [T*k] token of each routed row (bf16: gathered from x)
   const void* x_perm;      // fp32 path: routed rows of x in expert order
+  bool pair_gu;     // long prefill: gate/up on 256-row x 128-token tiles over pairs of SMs
+  bool pair_dn;     // long prefill: down on 256-row x 256-token tiles over pairs of SMs
   int bn;           // tokens per gate/up GEMM tile (16 or 128)
   int bn_dn;        // tokens per down GEMM tile (16, 128 or 256)
   int ksplit;       // gate/up reduction slices (1, 2 or 4)

@@ -21,6 +21,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "dispatch_common.cuh"
 #include "kernels.h"
 
 namespace moe {
@@ -966,6 +967,158 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) router_decode_kernel(
 }
 
 // ---------------------------------------------------------------------------------------
+// Small bf16 batches (decode, at most 32 tokens): routing and dispatch in one launch.
+// Block b scores the experts [4b, 4b + 4), four warps per expert, each warp over a quarter
+// of the hidden dimension: products exact in fp64, fp64 accumulation, the quarters added in
+// a fixed order, so |s^ - s| <= 1.01 H 2^-53 ||x|| ||w|| in any case and the scores are the
+// same on every run.  The block also keeps each expert's sum of squares (its norm bound).
+// The last block to finish (a counter) selects every token -- one warp per token, the
+// certified selection on these fp64 scores, exact recomputation where it cannot decide --
+// and then dispatches the batch in the same block (counts, offsets, the tile schedule and
+// the stable permutation), so the router GEMM, the selection and the dispatch are one
+// launch instead of three.
+// ---------------------------------------------------------------------------------------
+constexpr int kFusedMaxTokens = 32;
+constexpr int kFusedThreads = 512;
+constexpr int kFusedExperts = kFusedThreads / 32 / 4;  // experts per block (four warps each)
+constexpr int kFusedSelWarps = 8;                      // selecting warps of the last block
+
+struct FusedRouteSmem {
+  union {
+    double part[kFusedExperts][4][kFusedMaxTokens + 1];  // per quarter: T partial scores, sum of squares
+    struct {
+      __align__(16) unsigned char exact_scratch[kFusedSelWarps][kExactScratch];
+      CandList cands[kFusedSelWarps];
+    } sel;
+    SmallDispatchSmem disp;
+  };
+  int is_last;
+};
+
+template <int EPL, bool SIG>
+__global__ void __launch_bounds__(kFusedThreads, 1) route_dispatch_small_kernel(
+    const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wr, const Keys kf, int T,
+    int H, int E, int k, double* __restrict__ scores, double* __restrict__ wss, unsigned int* __restrict__ done,
+    int32_t* __restrict__ idx_ws, float* __restrict__ w_ws, int32_t* __restrict__ idx_user,
+    float* __restrict__ w_user, float* __restrict__ spill, const ScheduleArgs sa, int32_t* __restrict__ counts,
+    int32_t* __restrict__ counts_user, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
+    float* __restrict__ row_w, int32_t* __restrict__ row_tok, int32_t* __restrict__ perm_user,
+    const unsigned char* __restrict__ pf, int64_t pf_bytes, Ctrl* ctrl) {
+  __shared__ FusedRouteSmem sm;
+  // the memory stream is idle while the batch is routed: bring this block's slice of `pf`
+  // (the shared expert's gate/up weights, which the expert GEMM reads first) into L2
+  if (pf && threadIdx.x == 0) {
+    const int64_t per = ((pf_bytes + gridDim.x - 1) / gridDim.x + 15) & ~static_cast<int64_t>(15);
+    const int64_t b0 = per * blockIdx.x, b1 = b0 + per < pf_bytes ? b0 + per : pf_bytes;
+    if (b1 > b0) prefetch_l2(pf + b0, static_cast<uint64_t>(b1 - b0));
+  }
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int el = warp >> 2, qt = warp & 3;
+  const int e = blockIdx.x * kFusedExperts + el;
+  constexpr int V = 8;  // bf16 per 16-byte vector
+  if (e < E) {
+    const int nv = H / V, per = nv / 4;  // H is a multiple of 128: per is a multiple of 4
+    const int v0 = qt * per, v1 = v0 + per;
+    const __nv_bfloat16* w = Wr + static_cast<int64_t>(e) * H;
+    double ss = 0.0;
+    for (int tg = 0; tg < T; tg += 8) {
+      double acc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = 0.0;
+      for (int v = v0 + lane; v < v1; v += 32) {
+        const Vec16<__nv_bfloat16> wv = ld16(w + v * V);
+        double wd[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i) wd[i] = static_cast<double>(__bfloat162float(wv.v[i]));
+        if (tg == 0) {
+#pragma unroll
+          for (int i = 0; i < V; ++i) ss = fma(wd[i], wd[i], ss);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (tg + j >= T) break;
+          const Vec16<__nv_bfloat16> xv = ld16(x + static_cast<int64_t>(tg + j) * H + v * V);
+#pragma unroll
+          for (int i = 0; i < V; ++i) acc[j] = fma(static_cast<double>(__bfloat162float(xv.v[i])), wd[i], acc[j]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+        if (lane == 0 && tg + j < T) sm.part[el][qt][tg + j] = acc[j];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) sm.part[el][qt][kFusedMaxTokens] = ss;
+  }
+  __syncthreads();
+  // the quarters in a fixed order: scores [T, E] and the experts' sums of squares
+  for (int i = threadIdx.x; i < kFusedExperts * (T + 1); i += blockDim.x) {
+    const int q = i / (T + 1), t = i - q * (T + 1);
+    const int eq = blockIdx.x * kFusedExperts + q;
+    if (eq >= E) continue;
+    const int slot = t < T ? t : kFusedMaxTokens;
+    const double v = ((sm.part[q][0][slot] + sm.part[q][1][slot]) + sm.part[q][2][slot]) + sm.part[q][3][slot];
+    if (t < T) scores[static_cast<int64_t>(t) * E + eq] = v;
+    else wss[eq] = v;
+  }
+  // the last block selects and dispatches
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) sm.is_last = atomicAdd(done, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!sm.is_last) return;
+  __threadfence();
+  pdl_trigger();  // the expert GEMM's blocks may take their SMs during the selection
+  for (int t = warp; t < T && warp < kFusedSelWarps; t += kFusedSelWarps) {
+    const __nv_bfloat16* xt = x + static_cast<int64_t>(t) * H;
+    const double nx = norm_ub_from_sumsq(warp_sumsq(xt, H), H);
+    if (!select_token<__nv_bfloat16, __nv_bfloat16, EPL, SIG>(scores + static_cast<int64_t>(t) * E, 1.01 * H * kU53,
+                                                              0.0, false, nx, nullptr, wss, kf, xt, Wr, H, E, k, t,
+                                                              idx_ws, w_ws, idx_user, w_user, sm.sel.cands[warp], ctrl))
+      select_token_slow<__nv_bfloat16, __nv_bfloat16, SIG>(scores + static_cast<int64_t>(t) * E, 1, 1.01 * H * kU53,
+                                                          0.0, false, nx, nullptr, wss, key_spill(spill, T, E, t), kf,
+                                                          xt, Wr, H, E, k, t, idx_ws, w_ws, idx_user, w_user,
+                                                          sm.sel.exact_scratch[warp], ctrl);
+  }
+  __syncthreads();  // idx_ws / w_ws written by this block are visible to all its threads
+  dispatch_small_block(sa, idx_ws, w_ws, k, counts, counts_user, perm, inv_perm, row_w, row_tok, perm_user, ctrl,
+                       sm.disp);
+}
+
+bool route_dispatch_fused_supported(const moe_layer_shape& s, bool w32, int bn) {
+  return s.dtype == MOE_BF16 && !w32 && s.T >= 1 && s.T <= kFusedMaxTokens && s.E + 1 <= 2 * kFusedThreads &&
+         bn == 16;
+}
+
+cudaError_t launch_route_dispatch_small(const RouterArgs& a, const DispatchArgs& da, double* wss,
+                                        cudaStream_t st) {
+  const ScheduleArgs sa = schedule_args(da);
+  const unsigned grid = static_cast<unsigned>((a.E + kFusedExperts - 1) / kFusedExperts);
+  auto go = [&](auto kern) {
+    return launch_pdl(kern, dim3(grid), dim3(kFusedThreads), 0, st, static_cast<const __nv_bfloat16*>(a.x),
+                      static_cast<const __nv_bfloat16*>(a.Wr), Keys{a.bias, a.sigmoid, a.scale},
+                      static_cast<int>(a.T), a.H, a.E, a.k, a.scores64, wss, a.group_done, a.idx_ws, a.w_ws,
+                      a.idx_user, a.w_user, a.spill, sa, da.counts, da.counts_user, da.perm, da.inv_perm, da.row_w,
+                      da.row_tok, da.perm_user, static_cast<const unsigned char*>(a.prefetch), a.prefetch_bytes,
+                      a.ctrl);
+  };
+  const int epl = select_epl(a.E);
+  cudaError_t e;
+  if (a.sigmoid)
+    e = epl == 4 ? go(route_dispatch_small_kernel<4, true>)
+        : epl == 12 ? go(route_dispatch_small_kernel<12, true>) : go(route_dispatch_small_kernel<32, true>);
+  else
+    e = epl == 4 ? go(route_dispatch_small_kernel<4, false>)
+        : epl == 12 ? go(route_dispatch_small_kernel<12, false>) : go(route_dispatch_small_kernel<32, false>);
+  count_launches(1);
+  return e;
+}
+
+// ---------------------------------------------------------------------------------------
 // tcgen05 router GEMM.  Block (m, n, z) scores the tokens [128m, 128m+128) against the
 // experts [64n, 64n+64) over chunk z of the reduction.  Every slice of kRtSliceSteps
 // 64-product steps is accumulated in fp32 in one of two tensor-memory buffers and then
@@ -995,6 +1148,7 @@ constexpr int kRtSmTarget = 148;                     // blocks that fill the GPU
 
 struct RouterTcParams {
   CUtensorMap tmX;   // x [T, Hx], box {64, 16}
+  CUtensorMap tmX128;  // x [T, Hx], box {64, 128}: one copy per k-step for a full token tile
   CUtensorMap tmW;   // W_router [E, H] (fp32 weights: their bf16 split [E, 3 Hx]), box {64, 64}
   int64_t T;
   int H, E;          // H: length of the reduction (Hx, or 3 Hx for split fp32 weights)
@@ -1082,8 +1236,12 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTileM;
-  const int e0 = blockIdx.y * kRtExperts;
+  // blocks are numbered expert tile fastest: the blocks that share a token tile run side by
+  // side, so its rows of x are read from HBM once and then from L2
+  const int n_tiles = (p.E + kRtExperts - 1) / kRtExperts;
+  const int mi = static_cast<int>(blockIdx.x / n_tiles), ni = static_cast<int>(blockIdx.x % n_tiles);
+  const int64_t t0 = static_cast<int64_t>(mi) * kTileM;
+  const int e0 = ni * kRtExperts;
   const int ne = min(kRtExperts, p.E - e0);
   const int kb_all = p.H / kTileK;
   const int n_sl_all = (kb_all + kRtSliceSteps - 1) / kRtSliceSteps;
@@ -1099,7 +1257,7 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&p.tmX);
+      tma_prefetch_desc(rows == kTileM ? &p.tmX128 : &p.tmX);
       tma_prefetch_desc(&p.tmW);
       const uint32_t bytes = nbox * kRtRowBox * kTileK * 2 + kRtBBytes;
       int stage = 0;
@@ -1109,9 +1267,13 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
         unsigned char* st = smem + stage * kRtStageBytes;
         mbar_arrive_expect_tx(&full[stage], bytes);
         const int xcol = (kb % (p.Hx / kTileK)) * kTileK;
-        for (int b = 0; b < nbox; ++b)
-          tma_load_2d(st + b * kRtRowBox * kTileK * 2, &p.tmX, xcol,
-                      static_cast<int32_t>(t0 + b * kRtRowBox), &full[stage]);
+        if (rows == kTileM) {
+          tma_load_2d(st, &p.tmX128, xcol, static_cast<int32_t>(t0), &full[stage]);
+        } else {
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(st + b * kRtRowBox * kTileK * 2, &p.tmX, xcol,
+                        static_cast<int32_t>(t0 + b * kRtRowBox), &full[stage]);
+        }
         tma_load_2d(st + kRtABytes, &p.tmW, kb * kTileK, e0, &full[stage]);
         used |= 1u << stage;
         if (++stage == kRtStages) { stage = 0; phase ^= 1u; }
@@ -1183,10 +1345,10 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
       // sums of squares of this chunk's columns while the MMAs run: the x rows once per
       // m tile (n == 0), the W_router rows once per n tile (m == 0)
       const int c0 = kb_begin * kTileK, c1 = kb_end * kTileK;
-      if (blockIdx.y == 0)  // x columns once (the split fp32 weights repeat them)
+      if (ni == 0)  // x columns once (the split fp32 weights repeat them)
         sumsq_rows_bf16(p.x + t0 * p.Hx, p.Hx, rows, min(c0, p.Hx), min(c1, p.Hx),
                         p.xss + blockIdx.z * p.T + t0, quarter, lane);
-      if (blockIdx.x == 0 && !p.w_given)
+      if (mi == 0 && !p.w_given)
         sumsq_rows_bf16(p.Wr + static_cast<int64_t>(e0) * p.H, p.H, ne, c0, c1,
                         p.wss + static_cast<int64_t>(blockIdx.z) * p.E + e0, quarter, lane);
       for (int sl = 0; sl < n_sl && ok; ++sl) {
@@ -1210,7 +1372,7 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
       __threadfence();
       named_bar_sync(1, 128);
       if (warp == 2 && lane == 0) {
-        const unsigned int done = atomicAdd(p.tile_done + blockIdx.x * gridDim.y + blockIdx.y, 1u);
+        const unsigned int done = atomicAdd(p.tile_done + blockIdx.x, 1u);
         *last_flag = (done == static_cast<unsigned int>(p.chunks - 1)) ? 1 : 0;
       }
       named_bar_sync(1, 128);
@@ -1226,13 +1388,13 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
           for (int sl = 0; sl < n_sl_all; ++sl) acc += static_cast<double>(__ldcg(src + sl * sstride));
           p.scores[(t0 + tt) * p.E + e0 + j] = acc;
         }
-        if (blockIdx.y == 0)
+        if (ni == 0)
           for (int i = et; i < rows; i += 128) {
             double ss = 0.0;
             for (int z = 0; z < p.chunks; ++z) ss += __ldcg(p.xss + z * p.T + t0 + i);
             p.xnorm[t0 + i] = norm_ub_from_sumsq(ss, p.Hx);
           }
-        if (blockIdx.x == 0 && !p.w_given)
+        if (mi == 0 && !p.w_given)
           for (int i = et; i < ne; i += 128) {
             double ss = 0.0;
             for (int z = 0; z < p.chunks; ++z) ss += __ldcg(p.wss + static_cast<int64_t>(z) * p.E + e0 + i);
@@ -1394,8 +1556,10 @@ static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
   const bf16* x = static_cast<const bf16*>(a.x);
   const bf16* Wg = static_cast<const bf16*>(a.w32 ? a.w3 : a.Wr);  // the GEMM's B operand
   if (!encode_bf16_rows(&p.tmX, a.x, a.T, a.H, kRtRowBox) ||
+      (a.T >= kTileM && !encode_bf16_rows(&p.tmX128, a.x, a.T, a.H, kTileM)) ||
       !encode_bf16_rows(&p.tmW, Wg, a.E, Kg, kRtExperts))
     return cudaErrorInvalidValue;
+  if (a.T < kTileM) p.tmX128 = p.tmX;  // no full token tile: never used
   cudaError_t e = allow_smem(router_gemm_tc_kernel, kRtSmem);
   if (e != cudaSuccess) return e;
   // Each slice of L = 256 products is accumulated in fp32 from exact products, at most
@@ -1435,7 +1599,7 @@ static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
     ++launches;
   }
   e = launch_pdl(router_gemm_tc_kernel,
-                 dim3(static_cast<unsigned>((a.T + kTileM - 1) / kTileM), (a.E + kRtExperts - 1) / kRtExperts,
+                 dim3(static_cast<unsigned>(((a.T + kTileM - 1) / kTileM) * ((a.E + kRtExperts - 1) / kRtExperts)), 1,
                       static_cast<unsigned>(chunks)),
                  dim3(192), static_cast<size_t>(kRtSmem), st, p);
   if (e != cudaSuccess) return e;

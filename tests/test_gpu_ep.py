@@ -41,6 +41,7 @@ CASES = [
     dict(T=3, H=512, E=16, top_k=4, I=128, I_shared=128, world=4),      # 16-token tiles, split gate/up
     dict(T=700, H=256, E=8, top_k=4, I=256, I_shared=128, world=3),     # 256-token down tiles, uneven ranges
     dict(T=200, H=512, E=40, top_k=6, I=384, I_shared=0, world=5),      # no shared expert
+    dict(T=700, H=256, E=8, top_k=4, I=256, I_shared=256, world=3),     # tiles over pairs of SMs
 ]
 
 

@@ -52,6 +52,10 @@ SMALL = [
     dict(T=3, H=2176, E=200, top_k=8, I=128, I_shared=128),
     # 256-token tiles (about 350 tokens per expert: one full and one ragged tile each)
     dict(T=700, H=256, E=8, top_k=4, I=256, I_shared=128),
+    # 256 x 256 tiles over pairs of SMs (widths multiples of 256): ragged token tiles, a
+    # shared expert of one weight tile; no shared expert and two weight tiles per expert
+    dict(T=700, H=256, E=8, top_k=4, I=256, I_shared=256),
+    dict(T=1100, H=512, E=6, top_k=2, I=512, I_shared=0),
 ]
 
 
