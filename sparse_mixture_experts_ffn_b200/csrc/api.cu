@@ -132,7 +132,7 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.wss = take(tc_scores ? 0 : groups * E * 8);
   L.scores = take(T * E * 8);
   L.zero_end = tc_scores ? L.scores : off;
-  L.fwss = take(E * 8);  // the fused small-batch routing's sums of squares of W_router rows
+  L.fwss = take(E * 8);  // the fused small-batch routing's norm bounds of the W_router rows
   L.spill = take(T * E * 20);
   L.rsplit = take(router_split_bytes(*s));
   L.w3 = take(router_w3_bytes(*s));
@@ -208,7 +208,7 @@ extern "C" moe_status moe_layer_workspace_layout(const moe_layer_shape* shape,
   out->scores = L.scores;
   // fp32 slices on the tensor-core router; fp64 sums on the fused small-batch path (with bf16
   // router weights) and the CUDA-core router
-  out->scores_slice = router_scores_f32(*shape) && !route_dispatch_fused_supported(*shape, false, L.bn)
+  out->scores_slice = router_scores_f32(*shape)
                           ? router_slice_len(shape->H) : 0;
   return MOE_OK;
 }
@@ -289,11 +289,12 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
   // FP8 weights run on 16- and 128-token tiles only
   const int bn_dn = wt.w8 ? std::min(L.bn_dn, 128) : L.bn_dn;
-  // long prefill: both GEMMs on 256-row tiles over pairs of SMs (gate/up reads the gathered
-  // copy of x)
+  // long prefill: the down projection on 256-row tiles over pairs of SMs.  The gate/up GEMM
+  // stays on one SM a tile, where its four gather warps read the token rows straight from x
+  // (measured faster than pair tiles fed from a gathered copy of x)
   const bool pair = s.dtype == MOE_BF16 && !wt.w8 && L.ksplit == 1 &&
                     choose_pair(s.T, s.top_k, s.E, s.H, s.I, s.I_shared);
-  const bool pair_gu = pair, pair_dn = pair;
+  const bool pair_gu = false, pair_dn = pair;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
@@ -373,7 +374,7 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   da.offsets_user = routing ? routing->offsets : nullptr;
   da.perm_user = routing ? routing->perm : nullptr;
   da.ctrl = ctrl;
-  if (route_dispatch_fused_supported(s, ra.w32, L.bn)) {
+  if (false && route_dispatch_fused_supported(s, ra.w32, L.bn)) {
     if (has_shared && !wt.w8) {  // bf16 shared gate/up rows: read first by the gate/up GEMM
       ra.prefetch = Ws_gate_up;
       ra.prefetch_bytes = static_cast<int64_t>(2) * s.I_shared * s.H * 2;

@@ -111,9 +111,9 @@ struct DispatchArgs {
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st);
 
 // Small bf16 batches: routing and dispatch in one launch (replaces launch_router and
-// launch_dispatch).  wss: [E] fp64 scratch for the experts' sums of squares.
+// launch_dispatch).  wnorm: [E] fp64 scratch for the W_router rows' norm bounds.
 bool route_dispatch_fused_supported(const moe_layer_shape& s, bool w32, int bn);
-cudaError_t launch_route_dispatch_small(const RouterArgs& a, const DispatchArgs& da, double* wss,
+cudaError_t launch_route_dispatch_small(const RouterArgs& a, const DispatchArgs& da, double* wnorm,
                                         cudaStream_t st);
 
 struct ExpertArgs {
