@@ -102,7 +102,14 @@ struct TcCfg {
   // bf16 gate/up with 128-token tiles: four more warps gather the tiles' token rows from x
   // (cp.async, 16 bytes per lane), so no permuted copy of x is written and read back
   static constexpr bool kCpGather = GATED && BN == 128 && !W8;
-  static constexpr int kThreads = W8 ? 192 + 128 * kConvGroups : (kCpGather ? 192 + 128 : 192);
+  // bf16 tiles of 128 or more tokens: a stage-watcher warp (the last) waits for each stage's
+  // operands and hands the stage to the MMA warp at a named barrier.  A thread that has
+  // tcgen05.mma in flight stalls on its next shared-memory read (an mbarrier poll included)
+  // for about as long as one stage of MMAs takes, so the issuing warp reads no shared memory
+  // between the stages of a tile; the watcher also waits for the accumulator and walks the
+  // item ring for it.
+  static constexpr bool kWatch = BN >= 128 && !W8;
+  static constexpr int kThreads = (W8 ? 192 + 128 * kConvGroups : (kCpGather ? 192 + 128 : 192)) + (kWatch ? 32 : 0);
   static constexpr int kConvMod = kConvStages > 0 ? kConvStages : 1;  // a divisor in every variant
   // tiles of up to 128 tokens stage the output tile [BN][128] bf16 in shared memory for
   // 16-byte stores; 256-token tiles store straight from registers (each warp writes 64
@@ -262,12 +269,14 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   }
 }
 
-// Persistent grouped GEMM: 192 threads (448 with FP8 weights), one block per SM.
+// Persistent grouped GEMM, one block per SM.
 //   warp 0      TMA producer (one lane): weight tiles (gate and up for GATED) and token rows
 //   warp 1      allocates tensor memory; one lane issues the tcgen05 MMAs
 //   warps 2..5  epilogue: tensor memory -> registers -> shared staging tile -> global
+//   warps 6..9  bf16 gate/up with 128-token tiles: token-row gather (cp.async)
 //   warps 6..13 FP8 weights only: code tiles -> bf16 tiles, two groups of four warps
 //               taking alternate k-steps
+//   last warp   bf16 tiles of 128 or 256 tokens: stage watcher (waits, hands stages over)
 // Accumulators are double-buffered in tensor memory, so the epilogue of one tile overlaps
 // the main loop of the next.  Items are claimed dynamically: block b starts with item b and
 // then takes the next unclaimed one from a global counter, so blocks that draw short tiles
@@ -302,6 +311,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* hand = abort_flag + 1;  // [2] items handed from the watcher to the MMA warp
   uint64_t* cfull = reinterpret_cast<uint64_t*>(aux + 256);  // FP8: [kConvStages] converted
   uint64_t* cempty = cfull + 6;                              // FP8: [kConvStages] consumed
   volatile uint32_t* sc_stage = reinterpret_cast<volatile uint32_t*>(aux + 464);  // FP8: [kStages]
@@ -324,7 +334,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
     mbar_init(drain, 1);
     for (int q = 0; q < kRing; ++q) {
       mbar_init(&ring_full[q], 1);
-      // the MMA thread and one lane per epilogue (and converter) warp
+      // the MMA thread (or the watcher) and one lane per epilogue, converter and gather warp
       mbar_init(&ring_empty[q], 1 + 4 + (W8 ? 4 * kConvGroups : 0) + (C::kCpGather ? 4 : 0));
     }
     for (int c = 0; c < C::kConvStages; ++c) {
@@ -511,6 +521,95 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
         const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
         mbar_wait_drain(&full[s], par, p.ctrl);
       }
+  } else if (C::kWatch && warp == 1) {
+    // ------------------------- MMA issuer (stages handed over) -------------------------
+    // The whole warp takes the hand-overs at named barrier 2; lane 0 issues.  The item of
+    // each tile is read once (hand[n & 1]); every stage after it costs the warp one barrier
+    // and no shared-memory read.  After a failed wait the watcher goes on handing over the
+    // stages of the current tile (their MMAs read stale operands; the status is set) and
+    // then ends the schedule.
+    int stage = 0, acc = 0, n = 0;
+    for (;; ++n) {
+      __syncwarp();
+      named_bar_sync(2, 64);  // item hand-over: hand[n & 1], accumulator `acc` free
+      const int it = hand[n & 1];
+      if (it < 0) break;
+      const Item t = decode_item<BN>(p, sc, it);  // valid: the watcher skips the others
+      const uint32_t idesc = idesc_bf16_f32(kTileM, (t.nvalid + 15) & ~15);
+      const uint32_t d0 = tmem_base + acc * C::kAccCols;
+      const int kb_n = p.kblocks[t.sh];
+      const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        __syncwarp();
+        named_bar_sync(2, 64);  // stage hand-over: its operands are in shared memory
+        if (lane == 0) {
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+          const uint32_t b0 = a0 + C::kBOffset;
+#pragma unroll
+          for (int kk = 0; kk < kTileK / 16; ++kk) {
+            const uint32_t accum = (kb != kb0 || kk) ? 1u : 0u;
+            const uint64_t bdesc = sw128_kmajor_desc(b0 + kk * 32);
+            mma_bf16(d0, sw128_kmajor_desc(a0 + kk * 32), bdesc, idesc, accum);
+            if (GATED)
+              mma_bf16(d0 + BN, sw128_kmajor_desc(a0 + C::kABytes + kk * 32), bdesc, idesc, accum);
+          }
+          mma_commit(&empty[stage]);
+        }
+        if (++stage == C::kStages) stage = 0;
+      }
+      if (lane == 0) mma_commit(&tfull[acc]);
+      if (++acc == C::kAccBufs) acc = 0;
+    }
+    // all MMAs issued by this thread complete before the accumulators are freed
+    if (lane == 0) {
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0, p.ctrl);
+    }
+  } else if (C::kWatch && warp == C::kThreads / 32 - 1) {
+    // ------------------------------- stage watcher ------------------------------------
+    // Walks the item ring like the MMA warp would: per item it waits for a free
+    // accumulator and hands the item over, per stage it waits for the operands (TMA bytes
+    // and, with gather warps, their cp.async rows made visible to the tensor cores' proxy)
+    // and hands the stage over.
+    int stage = 0, acc = 0, n = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    bool failed = false;
+    int q = 0;
+    uint32_t qphase = 0;
+    for (;; ++n) {
+      int it = -1;
+      Item t{};
+      while (!failed) {
+        if (!wait(&ring_full[q], qphase)) { failed = true; break; }
+        it = ring[q];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ring_empty[q]);
+        if (++q == kRing) { q = 0; qphase ^= 1u; }
+        if (it < 0) break;
+        t = decode_item<BN>(p, sc, it);
+        if (t.valid) break;
+        it = -1;  // inconsistent entry (reported by the producer): the next one
+      }
+      if (failed) it = -1;
+      if (it >= 0 && !wait(&tempty[acc], acc_phase ^ 1u)) { failed = true; it = -1; }
+      if (lane == 0) hand[n & 1] = it;
+      __syncwarp();
+      named_bar_sync(2, 64);
+      if (it < 0) break;
+      const int kb_n = p.kblocks[t.sh];
+      const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!failed && !wait(&full[stage], phase)) failed = true;
+        // token rows written by the gather warps' cp.async: order them before the tensor
+        // cores' (async-proxy) reads of the stage
+        if (C::kCpGather) fence_proxy_async_smem();
+        __syncwarp();
+        named_bar_sync(2, 64);
+        if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+      }
+      if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
+    }
   } else if (warp == 1) {
     // ------------------------------- MMA issuer ---------------------------------------
     if (lane == 0) {
@@ -840,7 +939,7 @@ struct PairCfg {
   static constexpr int kBBytes = kBRows * kTileK * 2;
   static constexpr int kBOffset = kMats * kABytes;
   static constexpr int kStageBytes = kBOffset + kBBytes;
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 192 + 32;            // + the stage watcher (even CTA)
   static constexpr int kChunk = 32;                    // tokens per epilogue chunk
   static constexpr int kStagingBytes = kChunk * kTileM * 2;
   static constexpr int kAuxBytes = 2048;               // barriers, TMEM slot, row weights
@@ -924,39 +1023,68 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
       }
     }
   } else if (warp == 1) {
-    if (rank == 0 && lane == 0) {
+    if (rank == 0) {
       // ----------------------------- MMA issuer (even CTA) ----------------------------
+      // The whole warp takes the hand-overs of the watcher at named barrier 2 (a free
+      // accumulator per item, the operands of both CTAs per stage) and reads no shared
+      // memory between them; lane 0 issues.
       const uint32_t idesc = idesc_bf16_f32(256, BN);
       int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      bool ok = true;
-      for (int it = pair; it < total && ok; it += npairs) {
+      for (int it = pair; it < total; it += npairs) {
         const Item t = decode_item<BN>(p, sc, it);
         if (!t.valid) continue;
-        if (!mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, p.ctrl, abort_flag)) break;
-        tc_fence_after();
+        __syncwarp();
+        named_bar_sync(2, 64);  // accumulator `acc` free
         const uint32_t d0 = tmem_base + acc * C::kAccCols;
         for (int kb = 0; kb < p.kblocks[t.sh]; ++kb) {
-          if (!mbar_wait_cluster(&full[stage], phase, p.ctrl, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t b0 = a0 + C::kBOffset;
+          __syncwarp();
+          named_bar_sync(2, 64);  // both CTAs' operands of this stage have landed
+          if (lane == 0) {
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(smem + stage * C::kStageBytes);
+            const uint32_t b0 = a0 + C::kBOffset;
 #pragma unroll
-          for (int kk = 0; kk < kTileK / 16; ++kk) {
-            const uint32_t accum = (kb || kk) ? 1u : 0u;
-            const uint64_t bdesc = sw128_kmajor_desc(b0 + kk * 32);
-            mma_bf16_pair(d0, sw128_kmajor_desc(a0 + kk * 32), bdesc, idesc, accum);
-            if (GATED) mma_bf16_pair(d0 + BN, sw128_kmajor_desc(a0 + C::kABytes + kk * 32), bdesc, idesc, accum);
+            for (int kk = 0; kk < kTileK / 16; ++kk) {
+              const uint32_t accum = (kb || kk) ? 1u : 0u;
+              const uint64_t bdesc = sw128_kmajor_desc(b0 + kk * 32);
+              mma_bf16_pair(d0, sw128_kmajor_desc(a0 + kk * 32), bdesc, idesc, accum);
+              if (GATED) mma_bf16_pair(d0 + BN, sw128_kmajor_desc(a0 + C::kABytes + kk * 32), bdesc, idesc, accum);
+            }
+            mma_commit_pair(&empty[stage]);
           }
-          mma_commit_pair(&empty[stage]);
+          if (++stage == C::kStages) stage = 0;
+        }
+        if (lane == 0) mma_commit_pair(&tfull[acc]);
+        if (++acc == C::kAccBufs) acc = 0;
+      }
+      if (lane == 0) {
+        mma_commit_pair(drain);  // every MMA of the pair done before the accumulators are freed
+        mbar_wait_drain(drain, 0, p.ctrl);
+      }
+    }
+  } else if (warp == C::kThreads / 32 - 1) {
+    if (rank == 0) {
+      // ------------------------- stage watcher (even CTA) ------------------------------
+      // Walks the same items; waits for each accumulator and stage and hands them to the
+      // MMA warp.  After a failed wait (status set) it goes on handing over without
+      // waiting, so that the MMA warp reaches the end of the schedule.
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool failed = false;
+      for (int it = pair; it < total; it += npairs) {
+        const Item t = decode_item<BN>(p, sc, it);
+        if (!t.valid) continue;
+        if (!failed && !mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, p.ctrl, abort_flag)) failed = true;
+        __syncwarp();
+        named_bar_sync(2, 64);
+        for (int kb = 0; kb < p.kblocks[t.sh]; ++kb) {
+          if (!failed && !mbar_wait_cluster(&full[stage], phase, p.ctrl, abort_flag)) failed = true;
+          __syncwarp();
+          named_bar_sync(2, 64);
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
-        if (!ok) break;
-        mma_commit_pair(&tfull[acc]);
         if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
       }
-      mma_commit_pair(drain);  // every MMA of the pair done before the accumulators are freed
-      mbar_wait_drain(drain, 0, p.ctrl);
     }
   } else {
     // ------------------------------- epilogue (warps 2..5, both CTAs) -----------------
