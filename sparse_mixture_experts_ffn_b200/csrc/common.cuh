@@ -300,6 +300,18 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// named barrier that also counts the participants whose `pred` is true and returns the count
+// to all of them: a small number passed from one warp to another without a memory access
+__device__ __forceinline__ uint32_t named_bar_popc(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %1, 0;\n\tbarrier.cta.red.popc.u32 %0, %2, %3, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+      : "memory");
+  return r;
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* out) {
   uint32_t r[16];
   asm volatile(

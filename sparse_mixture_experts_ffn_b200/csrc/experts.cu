@@ -192,6 +192,12 @@ __device__ __forceinline__ Item decode_item(const TcParams& p, const Sched& sc, 
   return r;
 }
 
+// The shape of a valid tile as a number 1..32 for the MMA warp: (shared expert) * 16 +
+// (16-token MMA columns - 1); 0 ends the schedule.  Tiles of up to 256 tokens.
+__device__ __forceinline__ uint32_t tile_code(const Item& t) {
+  return static_cast<uint32_t>(t.sh) * 16u + static_cast<uint32_t>((t.nvalid + 15) >> 4);
+}
+
 // schedule length, clamped to the host bound (a larger value is reported, not run)
 __device__ __forceinline__ int schedule_length(const TcParams& p, const Sched& sc) {
   const int total = sc.ld(sc.item_start + p.G);
@@ -525,7 +531,10 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
     // ------------------------- MMA issuer (stages handed over) -------------------------
     // The whole warp takes the hand-overs at named barrier 2; lane 0 issues.  The item of
     // each tile is read once (hand[n & 1]); every stage after it costs the warp one barrier
-    // and no shared-memory read.  After a failed wait the watcher goes on handing over the
+    // and no shared-memory read.  (The pause that the read and the decode cost once a tile
+    // measured faster here than passing the tile in the barrier, as the pair kernel does:
+    // it lets the copies into shared memory, which compete with the tensor cores' operand
+    // reads, catch up.)  After a failed wait the watcher goes on handing over the
     // stages of the current tile (their MMAs read stale operands; the status is set) and
     // then ends the schedule.
     int stage = 0, acc = 0, n = 0;
@@ -1025,18 +1034,19 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
   } else if (warp == 1) {
     if (rank == 0) {
       // ----------------------------- MMA issuer (even CTA) ----------------------------
-      // The whole warp takes the hand-overs of the watcher at named barrier 2 (a free
-      // accumulator per item, the operands of both CTAs per stage) and reads no shared
-      // memory between them; lane 0 issues.
+      // The whole warp takes the hand-overs of the watcher at named barrier 2 (per tile a
+      // free accumulator and tile_code(), per stage the operands of both CTAs) and reads no
+      // memory; lane 0 issues.  Pair tiles always run all BN columns.
       const uint32_t idesc = idesc_bf16_f32(256, BN);
+      const int kb_routed = p.kblocks[0], kb_shared = p.kblocks[1];  // in registers before any MMA
       int stage = 0, acc = 0;
-      for (int it = pair; it < total; it += npairs) {
-        const Item t = decode_item<BN>(p, sc, it);
-        if (!t.valid) continue;
+      for (;;) {
         __syncwarp();
-        named_bar_sync(2, 64);  // accumulator `acc` free
+        const uint32_t code = named_bar_popc(2, 64, false);  // accumulator `acc` free
+        if (code == 0) break;
+        const int kb_n = code > 16 ? kb_shared : kb_routed;
         const uint32_t d0 = tmem_base + acc * C::kAccCols;
-        for (int kb = 0; kb < p.kblocks[t.sh]; ++kb) {
+        for (int kb = 0; kb < kb_n; ++kb) {
           __syncwarp();
           named_bar_sync(2, 64);  // both CTAs' operands of this stage have landed
           if (lane == 0) {
@@ -1076,7 +1086,7 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
         if (!t.valid) continue;
         if (!failed && !mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, p.ctrl, abort_flag)) failed = true;
         __syncwarp();
-        named_bar_sync(2, 64);
+        named_bar_popc(2, 64, static_cast<uint32_t>(lane) < tile_code(t));
         for (int kb = 0; kb < p.kblocks[t.sh]; ++kb) {
           if (!failed && !mbar_wait_cluster(&full[stage], phase, p.ctrl, abort_flag)) failed = true;
           __syncwarp();
@@ -1085,6 +1095,8 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
         }
         if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
       }
+      __syncwarp();
+      named_bar_popc(2, 64, false);  // the end of the schedule
     }
   } else {
     // ------------------------------- epilogue (warps 2..5, both CTAs) -----------------
