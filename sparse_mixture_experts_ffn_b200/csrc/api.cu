@@ -96,11 +96,11 @@ static int num_sms_current_device() {
 static size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
-  size_t ctrl, group_done, tile_done, item_counters, wss, zero_end, scores, fwss, xnorm, wnorm, idx, w, blk_hist, counts,
-      offsets, group_order, item_start_gu, item_start_dn, perm, inv_perm, row_w, row_tok, partial, spill, rsplit, w3,
+  size_t ctrl, group_done, tile_done, item_counters, wss, zero_end, scores, xnorm, wnorm, idx, w, blk_hist, counts,
+      offsets, group_order, item_start_gu, item_start_dn, info_gu, info_dn, perm, inv_perm, row_w, row_tok, partial, spill, rsplit, w3,
       x_perm, h, h_shared, o, o_shared, total;
   int bn, bn_dn, ksplit;
-  int64_t max_tiles;
+  int64_t max_tiles, cap_gu, cap_dn;
 };
 
 static bool make_layout(const moe_layer_shape* s, Layout& L) {
@@ -132,7 +132,6 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.wss = take(tc_scores ? 0 : groups * E * 8);
   L.scores = take(T * E * 8);
   L.zero_end = tc_scores ? L.scores : off;
-  L.fwss = take(E * 8);  // the fused small-batch routing's norm bounds of the W_router rows
   L.spill = take(T * E * 20);
   L.rsplit = take(router_split_bytes(*s));
   L.w3 = take(router_w3_bytes(*s));
@@ -146,6 +145,12 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.group_order = take((E + 1) * 4);
   L.item_start_gu = take((E + 2) * 4);
   L.item_start_dn = take((E + 2) * 4);
+  // tile descriptors: room for the longest schedules (128-row tiles; the down GEMM's
+  // narrowest token tiles, which FP8 weights use)
+  L.cap_gu = L.max_tiles * L.ksplit;
+  L.cap_dn = expert_tile_bound(s->T, s->top_k, s->E, s->H, Is ? s->H : 0, std::min(L.bn_dn, 128));
+  L.info_gu = take(static_cast<size_t>(L.cap_gu) * 16);
+  L.info_dn = take(static_cast<size_t>(L.cap_dn) * 16);
   L.perm = take(P * 4);
   L.inv_perm = take(P * 4);
   L.row_w = take(P * 4);
@@ -206,10 +211,8 @@ extern "C" moe_status moe_layer_workspace_layout(const moe_layer_shape* shape,
   out->o_shared = L.o_shared;
   out->row_w = L.row_w;
   out->scores = L.scores;
-  // fp32 slices on the tensor-core router; fp64 sums on the fused small-batch path (with bf16
-  // router weights) and the CUDA-core router
-  out->scores_slice = router_scores_f32(*shape)
-                          ? router_slice_len(shape->H) : 0;
+  // fp32 slices on the tensor-core router; fp64 sums on the CUDA-core router
+  out->scores_slice = router_scores_f32(*shape) ? router_slice_len(shape->H) : 0;
   return MOE_OK;
 }
 
@@ -365,6 +368,10 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   da.group_order = static_cast<int32_t*>(at(L.group_order));
   da.item_start_gu = static_cast<int32_t*>(at(L.item_start_gu));
   da.item_start_dn = static_cast<int32_t*>(at(L.item_start_dn));
+  da.info_gu = static_cast<int4*>(at(L.info_gu));
+  da.info_dn = static_cast<int4*>(at(L.info_dn));
+  da.cap_gu = static_cast<int>(L.cap_gu);
+  da.cap_dn = static_cast<int>(L.cap_dn);
   da.perm = static_cast<int32_t*>(at(L.perm));
   da.inv_perm = static_cast<int32_t*>(at(L.inv_perm));
   da.row_w = static_cast<float*>(at(L.row_w));
@@ -374,20 +381,9 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   da.offsets_user = routing ? routing->offsets : nullptr;
   da.perm_user = routing ? routing->perm : nullptr;
   da.ctrl = ctrl;
-  if (false && route_dispatch_fused_supported(s, ra.w32, L.bn)) {
-    if (has_shared && !wt.w8) {  // bf16 shared gate/up rows: read first by the gate/up GEMM
-      ra.prefetch = Ws_gate_up;
-      ra.prefetch_bytes = static_cast<int64_t>(2) * s.I_shared * s.H * 2;
-    }
-    // small bf16 batches: routing and dispatch in one launch (the stage marks 0-1 time it)
-    if (launch_route_dispatch_small(ra, da, static_cast<double*>(at(L.fwss)), st) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    marks.mark(1, st);
-  } else {
-    if (launch_router(ra, st) != cudaSuccess) return MOE_ERR_CUDA;
-    marks.mark(1, st);
-    if (launch_dispatch(da, st) != cudaSuccess) return MOE_ERR_CUDA;
-  }
+  if (launch_router(ra, st) != cudaSuccess) return MOE_ERR_CUDA;
+  marks.mark(1, st);
+  if (launch_dispatch(da, st) != cudaSuccess) return MOE_ERR_CUDA;
   marks.mark(2, st);
 
   ExpertArgs ea{};
@@ -416,6 +412,8 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   ea.group_order = da.group_order;
   ea.item_start_gu = da.item_start_gu;
   ea.item_start_dn = da.item_start_dn;
+  ea.info_gu = da.info_gu;
+  ea.info_dn = da.info_dn;
   ea.row_w = da.row_w;
   ea.x_perm = da.x_perm;
   ea.row_tok = da.row_tok;

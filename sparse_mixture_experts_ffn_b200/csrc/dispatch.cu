@@ -54,6 +54,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScheduleArgs sa, int k, int 
   __shared__ int cnt[2048];
   __shared__ int order[2048];
   __shared__ int warp_tot[33];
+  __shared__ ScheduleSmem ss;
   pdl_wait();
   pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
   const int E = sa.E;
@@ -82,7 +83,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScheduleArgs sa, int k, int 
   }
   if (sa.has_shared && threadIdx.x == 0) cnt[E] = sa.shared_rows;
   __syncthreads();
-  build_schedule(sa, cnt, order, warp_tot);
+  build_schedule(sa, cnt, order, warp_tot, ss);  // the tile descriptors: permute_kernel
 }
 
 // Placement for large batches: block b owns the assignments of tokens [256b, 256b+256);
@@ -94,10 +95,33 @@ __global__ void __launch_bounds__(32 * kPermWarps) permute_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ w, int64_t T, int k, int E,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ blk_hist,
     int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm, float* __restrict__ row_w,
-    int32_t* __restrict__ row_tok, int32_t* __restrict__ perm_user) {
-  extern __shared__ int wcnt[];  // [kPermWarps][E]
+    int32_t* __restrict__ row_tok, int32_t* __restrict__ perm_user, const ScheduleArgs sa,
+    const int32_t* __restrict__ counts) {
+  extern __shared__ int wcnt[];  // [kPermWarps][E], then the schedule tables
   pdl_wait();
   pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
+  {
+    // the tile descriptors of both GEMMs, spread over every block: first the schedule
+    // tables into shared memory (G <= E + 1 groups)
+    const int G = E + (sa.has_shared ? 1 : 0);
+    int* t_cnt = wcnt + kPermWarps * E;  // [E + 1]
+    int* t_off = t_cnt + E + 1;          // [E + 1]
+    int* t_order = t_off + E + 1;        // [G]
+    int* t_gu = t_order + G;             // [G + 1]
+    int* t_dn = t_gu + G + 1;            // [G + 1]
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) {
+      t_cnt[i] = i < E ? counts[i] : sa.shared_rows;
+      t_off[i] = offsets[i];
+    }
+    for (int i = threadIdx.x; i <= G; i += blockDim.x) {
+      if (i < G) t_order[i] = sa.group_order[i];
+      t_gu[i] = sa.item_start_gu[i];
+      t_dn[i] = sa.item_start_dn[i];
+    }
+    __syncthreads();
+    write_item_tables(sa, t_cnt, t_order, t_off, t_gu, t_dn, blockIdx.x * blockDim.x + threadIdx.x,
+                      gridDim.x * blockDim.x);
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kPermWarps * E; i += blockDim.x) wcnt[i] = 0;
   __syncthreads();
@@ -198,7 +222,7 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st) {
     e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, sa, a.k, nblk, a.blk_hist, a.counts,
                    a.counts_user);
     if (e != cudaSuccess) return e;
-    const size_t smem_p = smem_e * kPermWarps;
+    const size_t smem_p = smem_e * kPermWarps + sizeof(int) * (5 * static_cast<size_t>(a.E) + 8);
     if (smem_p > 48 * 1024) {
       e = cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem_p));
@@ -206,7 +230,8 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st) {
     }
     e = launch_pdl(permute_kernel, dim3(nblk), dim3(32 * kPermWarps), smem_p, st, a.idx, a.w, a.T, a.k,
                    a.E, static_cast<const int32_t*>(a.offsets), static_cast<const int32_t*>(a.blk_hist),
-                   a.perm, a.inv_perm, a.row_w, a.row_tok, a.perm_user);
+                   a.perm, a.inv_perm, a.row_w, a.row_tok, a.perm_user, sa,
+                   static_cast<const int32_t*>(a.counts));
     if (e != cudaSuccess) return e;
     launches = 3;
   }

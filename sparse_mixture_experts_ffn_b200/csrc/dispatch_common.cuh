@@ -56,27 +56,41 @@ struct ScheduleArgs {
   int32_t* item_start_gu;
   int32_t* item_start_dn;
   int32_t* offsets_user;
+  // one descriptor per tile of each grouped GEMM, in schedule order (see write_item_tables)
+  int4* info_gu;
+  int4* info_dn;
+  int cap_gu, cap_dn;  // their capacities (host bounds of the schedule lengths)
+  Ctrl* ctrl;
+};
+
+// shared-memory scratch of build_schedule / write_item_tables (groups G <= 2048)
+struct ScheduleSmem {
+  int istart_gu[2049];
+  int istart_dn[2049];
+  int off[2049];
 };
 
 // From the group sizes cnt[0..G) (routed experts, then the shared expert with all T
 // tokens): offsets of the routed experts, the largest-first group order and the tile
 // prefix sums of both grouped GEMMs (gate/up tiles counted ksplit times, once per slice
-// of the reduction).  One block with 2 * blockDim.x >= G + 1; cnt/order in shared memory.
-static __device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* order, int* warp_tot) {
+// of the reduction).  One block with 2 * blockDim.x >= G + 1; cnt/order in shared memory,
+// and the offsets and prefixes also kept in ss for write_item_tables.
+static __device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* order, int* warp_tot,
+                                      ScheduleSmem& ss) {
   const int E = a.E, G = E + (a.has_shared ? 1 : 0);
   {
     const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
     const int v0 = i0 < E ? cnt[i0] : 0, v1 = i1 < E ? cnt[i1] : 0;
     int total;
     const int ex = block_scan_pair(v0, v1, warp_tot, total);
-    if (i0 < E) a.offsets[i0] = ex;
-    if (i1 < E) a.offsets[i1] = ex + v0;
+    if (i0 < E) a.offsets[i0] = ss.off[i0] = ex;
+    if (i1 < E) a.offsets[i1] = ss.off[i1] = ex + v0;
     if (a.offsets_user) {
       if (i0 < E) a.offsets_user[i0] = ex;
       if (i1 < E) a.offsets_user[i1] = ex + v0;
     }
     if (threadIdx.x == 0) {
-      a.offsets[E] = total;
+      a.offsets[E] = ss.off[E] = total;
       if (a.offsets_user) a.offsets_user[E] = total;
     }
   }
@@ -121,15 +135,60 @@ static __device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* orde
   int total;
   int a0 = tiles(r0, true), a1 = tiles(r1, true);
   int ex = block_scan_pair(a0, a1, warp_tot, total);
-  if (r0 < G) a.item_start_gu[r0] = ex;
-  if (r1 < G) a.item_start_gu[r1] = ex + a0;
-  if (threadIdx.x == 0) a.item_start_gu[G] = total;
+  if (r0 < G) a.item_start_gu[r0] = ss.istart_gu[r0] = ex;
+  if (r1 < G) a.item_start_gu[r1] = ss.istart_gu[r1] = ex + a0;
+  if (threadIdx.x == 0) a.item_start_gu[G] = ss.istart_gu[G] = total;
   a0 = tiles(r0, false);
   a1 = tiles(r1, false);
   ex = block_scan_pair(a0, a1, warp_tot, total);
-  if (r0 < G) a.item_start_dn[r0] = ex;
-  if (r1 < G) a.item_start_dn[r1] = ex + a0;
-  if (threadIdx.x == 0) a.item_start_dn[G] = total;
+  if (r0 < G) a.item_start_dn[r0] = ss.istart_dn[r0] = ex;
+  if (r1 < G) a.item_start_dn[r1] = ss.istart_dn[r1] = ex + a0;
+  if (threadIdx.x == 0) a.item_start_dn[G] = ss.istart_dn[G] = total;
+}
+
+// One descriptor per tile of a grouped GEMM, so that a GEMM role finds its tile with one
+// load instead of searching the group prefixes: item `it` of group slot r (group g =
+// order[r], items [istart[r], istart[r + 1])) is local tile l = it - istart[r]; slice
+// ks = l % ksplit, weight tile m = (l / ksplit) / ntile, token tile n = (l / ksplit) % ntile
+// with ntile = ceil(cnt[g] / bn).  Stored {g, m, first row, rows | ks << 16}; the first
+// row of a shared-expert tile is relative to that group's first row.  Threads t0, t0 +
+// stride, ... of the caller write the items of both GEMMs; the tables (cnt[E] = rows of the
+// shared group, off = routed offsets, the prefixes) come from build_schedule.
+static __device__ void write_item_tables(const ScheduleArgs& a, const int* cnt, const int* order,
+                                         const int* off, const int* istart_gu, const int* istart_dn,
+                                         int t0, int stride) {
+  const int E = a.E, G = E + (a.has_shared ? 1 : 0);
+  for (int which = 0; which < 2; ++which) {
+    const int* istart = which ? istart_dn : istart_gu;
+    int4* info = which ? a.info_dn : a.info_gu;
+    const int cap = which ? a.cap_dn : a.cap_gu;
+    const int bn = which ? a.bn_dn : a.bn;
+    const int ks_n = which ? 1 : a.ksplit;
+    const int total = istart[G];
+    if (total > cap) {  // the GEMM reports it too and runs nothing
+      if (t0 == 0) set_status(a.ctrl, MOE_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    for (int it = t0; it < total; it += stride) {
+      int lo = 0, hi = G - 1;
+      while (lo < hi) {  // last group slot whose first item is <= it
+        const int mid = (lo + hi + 1) >> 1;
+        if (istart[mid] <= it) lo = mid; else hi = mid - 1;
+      }
+      const int g = order[lo];
+      const int rows = cnt[g];
+      const int ntile = (rows + bn - 1) / bn;  // >= 1: groups without rows have no items
+      if (ntile < 1) {  // inconsistent prefixes: an invalid descriptor, reported by the GEMM
+        info[it] = make_int4(-1, 0, 0, 0);
+        continue;
+      }
+      const int l = it - istart[lo];
+      const int tile = l / ks_n, ks = l - tile * ks_n;
+      const int m = tile / ntile, n = tile - m * ntile;
+      const int row0 = (g < E ? off[g] : 0) + n * bn;
+      info[it] = make_int4(g, m, row0, min(bn, rows - n * bn) | (ks << 16));
+    }
+  }
 }
 
 // Stable placement of the assignments [a0, a1) by one warp, 32 at a time, in (token,
@@ -168,6 +227,7 @@ struct SmallDispatchSmem {
   int order[2048];
   int base[1024];
   int warp_tot[33];
+  ScheduleSmem sched;
 };
 
 // The whole dispatch of a small batch by one block of 1024 threads: histogram, counts,
@@ -197,9 +257,11 @@ static __device__ void dispatch_small_block(const ScheduleArgs& sa, const int32_
   }
   if (sa.has_shared && threadIdx.x == 0) sm.cnt[E] = sa.shared_rows;
   __syncthreads();
-  build_schedule(sa, sm.cnt, sm.order, sm.warp_tot);
+  build_schedule(sa, sm.cnt, sm.order, sm.warp_tot, sm.sched);
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) sm.base[e] = sa.offsets[e];
+  write_item_tables(sa, sm.cnt, sm.order, sm.sched.off, sm.sched.istart_gu, sm.sched.istart_dn, threadIdx.x,
+                    blockDim.x);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) sm.base[e] = sm.sched.off[e];
   __syncthreads();
   if (threadIdx.x < 32)
     place_assignments(idx, w, 0, P, k, E, sm.base, perm, inv_perm, row_w, row_tok, perm_user);
@@ -227,6 +289,11 @@ inline ScheduleArgs schedule_args(const DispatchArgs& a) {
   sa.item_start_gu = a.item_start_gu;
   sa.item_start_dn = a.item_start_dn;
   sa.offsets_user = a.offsets_user;
+  sa.info_gu = a.info_gu;
+  sa.info_dn = a.info_dn;
+  sa.cap_gu = a.cap_gu;
+  sa.cap_dn = a.cap_dn;
+  sa.ctrl = a.ctrl;
   return sa;
 }
 

@@ -36,9 +36,8 @@ struct TcParams {
   CUtensorMap tmA[2];  // weights: [0] routed (all experts stacked), [1] shared expert
   CUtensorMap tmB[2];  // activations: [0] routed rows in expert order (gather: x rows,
                        // one-row box), [1] shared rows
-  const int32_t* offsets;      // [E + 1]
-  const int32_t* group_order;  // [G]
-  const int32_t* item_start;   // [G + 1]
+  const int32_t* item_start;   // [G + 1] tiles per group slot (prefix); [G] = schedule length
+  const int4* item_info;       // [schedule length] tile descriptors {g, m, first row, rows | ks << 16}
   const float* row_w;          // routing weight per routed row (down projection only)
   const int32_t* row_tok;      // token of each routed row (gather)
   int gather;                  // routed token rows gathered from x by tmB[0] (gate/up)
@@ -58,7 +57,6 @@ struct TcParams {
   int rows_out[2];             // rows of out[0] (T*k) and out[1] (T)
   int max_items;               // upper bound of the schedule length (host-computed)
   int ksplit;                  // gate/up: slices of the reduction per tile (1 = no split)
-  int sched_smem;              // copy the schedule tables into shared memory (room permitting)
   float limit[2];              // gate/up: SwiGLU limits, routed and shared (0: none)
   int max_tiles;               // bound of tile ids (split partial buffers)
   float* partial;              // [max_tiles][ksplit][BN][256] fp32 gate|up partial sums
@@ -67,8 +65,9 @@ struct TcParams {
   // gate/up: the down GEMM's schedule and weights, so that a block out of work brings the
   // weight rows of the down GEMM's item blockIdx.x into L2 (null: no prefetch)
   const int32_t* pf_item_start;    // [G + 1] item prefix of the down GEMM
+  const int4* pf_info;             // its tile descriptors
   const unsigned char* pf_w[2];    // W_down (this launch's experts), Ws_down
-  int pf_bn, pf_mt;                // tokens per down tile, weight tiles per group
+  int pf_mt;                       // weight tiles per group of the down GEMM
   int64_t pf_rows_per_group;       // rows of one routed expert's down matrix (H)
   int64_t pf_row_bytes[2];         // bytes of one row: routed (I), shared (I_shared)
   const uint8_t* scaleA[2];    // FP8 weights: E8M0 block scales of the A matrices, routed
@@ -149,42 +148,23 @@ struct Item {
   int nvalid;  // tokens in the tile
 };
 
-// The schedule tables (item_start, group_order, offsets), read from shared-memory copies
-// when the launch has room for them, else from global memory.
-struct Sched {
-  const int32_t* item_start;   // [G + 1]
-  const int32_t* group_order;  // [G]
-  const int32_t* offsets;      // [E + 1]
-  bool in_smem;
-  __device__ __forceinline__ int ld(const int32_t* q) const { return in_smem ? *q : __ldg(q); }
-};
-
+// Tile `it` of the schedule from its descriptor (written by the dispatch step), checked
+// against this launch's bounds: an inconsistent descriptor is reported and skipped.
 template <int BN>
-__device__ __forceinline__ Item decode_item(const TcParams& p, const Sched& sc, int it) {
-  int lo = 0, hi = p.G - 1;
-  while (lo < hi) {  // last group slot whose first item is <= it
-    const int mid = (lo + hi + 1) >> 1;
-    if (sc.ld(sc.item_start + mid) <= it) lo = mid; else hi = mid - 1;
-  }
+__device__ __forceinline__ Item decode_item(const TcParams& p, int it) {
+  const int4 d = __ldg(p.item_info + it);
   Item r;
-  r.g = sc.ld(sc.group_order + lo);
+  r.g = d.x;
   r.sh = (r.g == p.E) ? 1 : 0;
-  const int ks_n = p.ksplit;
-  const int local_item = it - sc.ld(sc.item_start + lo);
-  const int local = local_item / ks_n;  // slices of one tile are consecutive items
-  r.ks = local_item - local * ks_n;
-  r.tile = it / ks_n;                   // every group's item count is a multiple of ks_n
-  const int base = r.sh ? p.sh_base : sc.ld(sc.offsets + r.g);
-  const int cnt = r.sh ? p.sh_rows : sc.ld(sc.offsets + r.g + 1) - base;
-  const int ntile = (cnt + BN - 1) / BN;
-  r.m = ntile > 0 ? local / ntile : 0;
-  const int n = local - r.m * ntile;
-  r.row0 = base + n * BN;
-  r.nvalid = min(BN, cnt - n * BN);
-  r.valid = (r.g >= 0 && r.g < p.G && (r.sh || (r.g >= p.g_lo && r.g < p.g_hi)) && ntile > 0 && r.m >= 0 &&
-             r.m < p.mt[r.sh] && r.nvalid >= 1 &&
+  r.m = d.y;
+  r.row0 = d.z + (r.sh ? p.sh_base : 0);
+  r.nvalid = d.w & 0xFFFF;
+  r.ks = d.w >> 16;
+  r.tile = it / p.ksplit;  // every group's item count is a multiple of ksplit
+  r.valid = (r.g >= 0 && r.g < p.G && (r.sh || (r.g >= p.g_lo && r.g < p.g_hi)) && r.m >= 0 &&
+             r.m < p.mt[r.sh] && r.nvalid >= 1 && r.nvalid <= BN && r.ks < p.ksplit &&
              r.row0 >= 0 && r.row0 + r.nvalid <= p.rows_out[r.sh] &&
-             (ks_n == 1 || (r.tile >= 0 && r.tile < p.max_tiles))) ? 1 : 0;
+             (p.ksplit == 1 || (r.tile >= 0 && r.tile < p.max_tiles))) ? 1 : 0;
   if (!r.valid) {
     r.nvalid = 0;
     r.sh = 0;
@@ -199,8 +179,8 @@ __device__ __forceinline__ uint32_t tile_code(const Item& t) {
 }
 
 // schedule length, clamped to the host bound (a larger value is reported, not run)
-__device__ __forceinline__ int schedule_length(const TcParams& p, const Sched& sc) {
-  const int total = sc.ld(sc.item_start + p.G);
+__device__ __forceinline__ int schedule_length(const TcParams& p) {
+  const int total = __ldg(p.item_start + p.G);
   if (total < 0 || total > p.max_items) {
     if (threadIdx.x == 0 && blockIdx.x == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
     return 0;
@@ -363,18 +343,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();
   pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
-  Sched sc{p.item_start, p.group_order, p.offsets, false};
-  if (p.sched_smem) {
-    // one parallel copy of the tables instead of a chain of dependent global reads per item
-    int32_t* tab = reinterpret_cast<int32_t*>(aux + C::kAuxBytes);
-    const int G = p.G;
-    for (int i = threadIdx.x; i <= G; i += blockDim.x) tab[i] = __ldg(p.item_start + i);
-    for (int i = threadIdx.x; i < G; i += blockDim.x) tab[G + 1 + i] = __ldg(p.group_order + i);
-    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) tab[2 * G + 1 + i] = __ldg(p.offsets + i);
-    __syncthreads();
-    sc = Sched{tab, tab + G + 1, tab + 2 * G + 1, true};
-  }
-  const int total = schedule_length(p, sc);
+  const int total = schedule_length(p);
   // FP8: waiting threads sleep in their polls, leaving the issue slots to the converters
   auto wait = [&](uint64_t* bar, uint32_t parity) {
     return W8 ? mbar_wait_sleep(bar, parity, p.ctrl, abort_flag) : mbar_wait(bar, parity, p.ctrl, abort_flag);
@@ -430,7 +399,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
       const int cur = it;
       it = __shfl_sync(0xffffffffu, claimed, 0);
       if (lane == 0 && it < total) claimed = static_cast<int>(atomicAdd(p.item_counter, 1u) + gridDim.x);
-      const Item t = decode_item<BN>(p, sc, cur);
+      const Item t = decode_item<BN>(p, cur);
       if (!t.valid) {
         if (blockIdx.x == 0 && lane == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
         continue;
@@ -461,7 +430,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
         }
         pf_it = -1;
         if (it < total) {
-          const Item tn = decode_item<BN>(p, sc, it);
+          const Item tn = decode_item<BN>(p, it);
           if (tn.valid) {
             load_scales(tn, pf_sg, pf_su);
             pf_it = it;
@@ -502,18 +471,10 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
     __syncwarp();
     if (GATED && !W8 && p.pf_item_start && lane == 0 && static_cast<int>(blockIdx.x) < __ldg(p.pf_item_start + p.G)) {
       // out of work: the rows of the down GEMM's item blockIdx.x (its first wave) into L2
-      const int itd = static_cast<int>(blockIdx.x);
-      int lo = 0, hi = p.G - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(p.pf_item_start + mid) <= itd) lo = mid; else hi = mid - 1;
-      }
-      const int g = sc.ld(sc.group_order + lo);
+      const int4 d = __ldg(p.pf_info + blockIdx.x);
+      const int g = d.x, m = d.y;
       const int sh = (g == p.E) ? 1 : 0;
-      const int cnt = sh ? p.sh_rows : sc.ld(sc.offsets + g + 1) - sc.ld(sc.offsets + g);
-      const int ntile = (cnt + p.pf_bn - 1) / p.pf_bn;
-      const int m = ntile > 0 ? (itd - __ldg(p.pf_item_start + lo)) / ntile : -1;
-      if (m >= 0 && m < p.pf_mt && (sh || (g >= p.g_lo && g < p.g_hi))) {
+      if (g >= 0 && m >= 0 && m < p.pf_mt && (sh || (g >= p.g_lo && g < p.g_hi))) {
         const int64_t row = (sh ? 0 : (g - p.g_lo) * p.pf_rows_per_group) + static_cast<int64_t>(m) * kTileM;
         prefetch_l2(p.pf_w[sh] + row * p.pf_row_bytes[sh], static_cast<uint64_t>(kTileM) * p.pf_row_bytes[sh]);
       }
@@ -543,7 +504,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
       named_bar_sync(2, 64);  // item hand-over: hand[n & 1], accumulator `acc` free
       const int it = hand[n & 1];
       if (it < 0) break;
-      const Item t = decode_item<BN>(p, sc, it);  // valid: the watcher skips the others
+      const Item t = decode_item<BN>(p, it);  // valid: the watcher skips the others
       const uint32_t idesc = idesc_bf16_f32(kTileM, (t.nvalid + 15) & ~15);
       const uint32_t d0 = tmem_base + acc * C::kAccCols;
       const int kb_n = p.kblocks[t.sh];
@@ -596,7 +557,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
         if (lane == 0) mbar_arrive(&ring_empty[q]);
         if (++q == kRing) { q = 0; qphase ^= 1u; }
         if (it < 0) break;
-        t = decode_item<BN>(p, sc, it);
+        t = decode_item<BN>(p, it);
         if (t.valid) break;
         it = -1;  // inconsistent entry (reported by the producer): the next one
       }
@@ -633,7 +594,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
         mbar_arrive(&ring_empty[q]);
         if (++q == kRing) { q = 0; qphase ^= 1u; }
         if (it < 0) break;
-        const Item t = decode_item<BN>(p, sc, it);
+        const Item t = decode_item<BN>(p, it);
         if (!t.valid) continue;
         const int n_mma = (t.nvalid + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(kTileM, n_mma);
@@ -696,7 +657,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
       if (lane == 0) mbar_arrive(&ring_empty[q]);
       if (++q == kRing) { q = 0; qphase ^= 1u; }
       if (it < 0) break;
-      const Item t = decode_item<BN>(p, sc, it);
+      const Item t = decode_item<BN>(p, it);
       if (!t.valid) continue;
       const __nv_bfloat16* src[8];
       uint32_t nbytes[8];
@@ -748,7 +709,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
       if (lane == 0) mbar_arrive(&ring_empty[q]);
       if (++q == kRing) { q = 0; qphase ^= 1u; }
       if (it < 0) break;
-      const Item t = decode_item<BN>(p, sc, it);
+      const Item t = decode_item<BN>(p, it);
       if (!t.valid) continue;
       const int kb_n = p.kblocks[t.sh];
       const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
@@ -795,7 +756,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
       if (lane == 0) mbar_arrive(&ring_empty[q]);
       if (++q == kRing) { q = 0; qphase ^= 1u; }
       if (it < 0) break;
-      const Item t = decode_item<BN>(p, sc, it);
+      const Item t = decode_item<BN>(p, it);
       if (!t.valid) continue;
       if (!GATED)
         for (int n = et; n < BN; n += 128)
@@ -1001,8 +962,7 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();
   pdl_trigger();
-  const Sched sc{p.item_start, p.group_order, p.offsets, false};
-  const int total = schedule_length(p, sc);
+  const int total = schedule_length(p);
   const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
 
   if (warp == 0) {
@@ -1012,7 +972,7 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
       uint32_t phase = 0;
       bool ok = true;
       for (int it = pair; it < total && ok; it += npairs) {
-        const Item t = decode_item<BN>(p, sc, it);
+        const Item t = decode_item<BN>(p, it);
         if (!t.valid) {
           if (blockIdx.x == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
           continue;
@@ -1082,7 +1042,7 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
       uint32_t phase = 0, acc_phase = 0;
       bool failed = false;
       for (int it = pair; it < total; it += npairs) {
-        const Item t = decode_item<BN>(p, sc, it);
+        const Item t = decode_item<BN>(p, it);
         if (!t.valid) continue;
         if (!failed && !mbar_wait_cluster(&tempty[acc], acc_phase ^ 1u, p.ctrl, abort_flag)) failed = true;
         __syncwarp();
@@ -1108,7 +1068,7 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int it = pair; it < total; it += npairs) {
-      const Item t = decode_item<BN>(p, sc, it);
+      const Item t = decode_item<BN>(p, it);
       if (!t.valid) continue;
       if (!GATED) {
         for (int n = et; n < BN; n += 128) sw[n] = (t.sh || n >= t.nvalid) ? 1.0f : __ldg(p.row_w + t.row0 + n);
@@ -1291,9 +1251,7 @@ static cudaError_t launch_tc(const TcParams& prm_in, int num_sms, cudaStream_t s
   using C = TcCfg<GATED, BN, W8>;
   auto kern = expert_gemm_tc_kernel<GATED, BN, W8>;
   TcParams prm = prm_in;
-  const size_t tables = static_cast<size_t>(2 * prm.G + 1 + prm.E + 1) * sizeof(int32_t);
-  prm.sched_smem = (C::kSmemBytes + tables <= static_cast<size_t>(kMaxDynSmem)) ? 1 : 0;
-  const size_t smem = C::kSmemBytes + (prm.sched_smem ? tables : 0);
+  const size_t smem = C::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -1399,9 +1357,8 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
     g.tmB[1] = g.tmB[0];
   }
   if (!ok) return cudaErrorInvalidValue;
-  g.offsets = a.offsets;
-  g.group_order = a.group_order;
   g.item_start = a.item_start_gu;
+  g.item_info = a.info_gu;
   g.row_w = a.row_w;
   g.row_tok = a.row_tok;
   g.limit[0] = a.swiglu_limit;
@@ -1410,9 +1367,9 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   g.x = static_cast<const __nv_bfloat16*>(a.x);
   if (!a.w8 && !a.pair_dn) {
     g.pf_item_start = a.item_start_dn;
+    g.pf_info = a.info_dn;
     g.pf_w[0] = static_cast<const unsigned char*>(a.Wd);
     g.pf_w[1] = static_cast<const unsigned char*>(has_shared ? a.Wsd : a.Wd);
-    g.pf_bn = a.bn_dn;
     g.pf_mt = a.H / kTileM;
     g.pf_rows_per_group = a.H;
     g.pf_row_bytes[0] = static_cast<int64_t>(a.I) * 2;
@@ -1469,9 +1426,8 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
     d.tmB[1] = d.tmB[0];
   }
   if (!ok) return cudaErrorInvalidValue;
-  d.offsets = a.offsets;
-  d.group_order = a.group_order;
   d.item_start = a.item_start_dn;
+  d.item_info = a.info_dn;
   d.row_w = a.row_w;
   d.out[0] = static_cast<__nv_bfloat16*>(a.o);
   d.out[1] = static_cast<__nv_bfloat16*>(a.o_shared);

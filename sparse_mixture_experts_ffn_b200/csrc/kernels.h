@@ -58,8 +58,6 @@ struct RouterArgs {
   void* rsplit;      // router_split_bytes(shape) bytes, or null: the reduction is not split
   bool w32;          // bf16 tokens with fp32 router weights (Wr is float [E, H])
   void* w3;          // router_w3_bytes(shape): the fp32 weights split into 3 bf16 parts
-  const void* prefetch = nullptr;  // fused small-batch routing: bytes to bring into L2 meanwhile
-  int64_t prefetch_bytes = 0;      // (a multiple of 16)
   Ctrl* ctrl;
 };
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
@@ -98,6 +96,9 @@ struct DispatchArgs {
   int32_t* group_order;     // [G]   groups sorted by row count, descending
   int32_t* item_start_gu;   // [G+1] tcgen05 tiles of the gate/up GEMM per group (prefix)
   int32_t* item_start_dn;   // [G+1] tiles of the down GEMM
+  int4* info_gu;            // [cap_gu] one descriptor per gate/up tile, in schedule order
+  int4* info_dn;            // [cap_dn] the same for the down GEMM
+  int cap_gu, cap_dn;
   int32_t* perm;        // [T*k]
   int32_t* inv_perm;    // [T*k]
   float* row_w;         // [T*k]
@@ -109,12 +110,6 @@ struct DispatchArgs {
   Ctrl* ctrl;
 };
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st);
-
-// Small bf16 batches: routing and dispatch in one launch (replaces launch_router and
-// launch_dispatch).  wnorm: [E] fp64 scratch for the W_router rows' norm bounds.
-bool route_dispatch_fused_supported(const moe_layer_shape& s, bool w32, int bn);
-cudaError_t launch_route_dispatch_small(const RouterArgs& a, const DispatchArgs& da, double* wnorm,
-                                        cudaStream_t st);
 
 struct ExpertArgs {
   bool bf16;
@@ -137,6 +132,8 @@ struct ExpertArgs {
   const int32_t* group_order;
   const int32_t* item_start_gu;
   const int32_t* item_start_dn;
+  const int4* info_gu;
+  const int4* info_dn;
   const float* row_w;
   const int32_t* row_tok;  // [T*k] token of each routed row (bf16: gathered from x)
   const void* x_perm;      // fp32 path: routed rows of x in expert order

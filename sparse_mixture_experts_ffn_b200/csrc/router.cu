@@ -9,9 +9,11 @@
 // recomputed, in fp64 (delta ~ 2^-41 relative) and, if that is still not conclusive, with
 // an exact integer dot product.
 //
-//   small batches: one fused kernel computes fp64 scores of all experts; the last block
-//                  of each token group to finish selects for those tokens;
-//   large batches: a tcgen05 GEMM (fp32 accumulation) scores, then a selection kernel.
+//   bf16 tokens: a tcgen05 GEMM (fp32 accumulation over short slices, the slices added in
+//                fp64; small batches split the reduction over blocks) scores, then a
+//                selection kernel;
+//   fp32 tokens, or more experts than tensor memory holds: one kernel computes fp64 scores
+//                on the CUDA cores; the last block of each token group selects for them.
 #include <algorithm>
 
 #include <cuda_bf16.h>
@@ -21,7 +23,6 @@
 #include <stdint.h>
 
 #include "common.cuh"
-#include "dispatch_common.cuh"
 #include "kernels.h"
 
 namespace moe {
@@ -964,175 +965,6 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) router_decode_kernel(
                              idx_user, w_user, exact_scratch[warp], ctrl);
     }
   }
-}
-
-// ---------------------------------------------------------------------------------------
-// Small bf16 batches (decode, at most 32 tokens): routing and dispatch in one launch.
-// Block b scores the experts [4b, 4b + 4), four warps per expert, each warp over a quarter
-// of the hidden dimension: products exact in fp64, fp64 accumulation, the quarters added in
-// a fixed order, so |s^ - s| <= 1.01 H 2^-53 ||x|| ||w|| in any case and the scores are the
-// same on every run.  The block also writes each expert's norm bound (from the fp64 sum of
-// squares), so that the selection reads the bounds instead of taking square roots.
-// The last block to finish (a counter) selects every token -- one warp per token, the
-// certified selection on these fp64 scores, exact recomputation where it cannot decide --
-// and then dispatches the batch in the same block (counts, offsets, the tile schedule and
-// the stable permutation), so the router GEMM, the selection and the dispatch are one
-// launch instead of three.
-// ---------------------------------------------------------------------------------------
-constexpr int kFusedMaxTokens = 32;
-constexpr int kFusedThreads = 512;
-constexpr int kFusedExperts = kFusedThreads / 32 / 4;  // experts per block (four warps each)
-constexpr int kFusedSelWarps = 8;                      // selecting warps of the last block
-
-struct FusedRouteSmem {
-  union {
-    double part[kFusedExperts][4][kFusedMaxTokens + 1];  // per quarter: T partial scores, sum of squares
-    struct {
-      __align__(16) unsigned char exact_scratch[kFusedSelWarps][kExactScratch];
-      CandList cands[kFusedSelWarps];
-    } sel;
-    SmallDispatchSmem disp;
-  };
-  int is_last;
-};
-
-template <int EPL, bool SIG>
-__global__ void __launch_bounds__(kFusedThreads, 1) route_dispatch_small_kernel(
-    const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ Wr, const Keys kf, int T,
-    int H, int E, int k, double* __restrict__ scores, double* __restrict__ wnorm, unsigned int* __restrict__ done,
-    int32_t* __restrict__ idx_ws, float* __restrict__ w_ws, int32_t* __restrict__ idx_user,
-    float* __restrict__ w_user, float* __restrict__ spill, const ScheduleArgs sa, int32_t* __restrict__ counts,
-    int32_t* __restrict__ counts_user, int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
-    float* __restrict__ row_w, int32_t* __restrict__ row_tok, int32_t* __restrict__ perm_user,
-    const unsigned char* __restrict__ pf, int64_t pf_bytes, Ctrl* ctrl) {
-  __shared__ FusedRouteSmem sm;
-  pdl_wait();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int el = warp >> 2, qt = warp & 3;
-  const int e = blockIdx.x * kFusedExperts + el;
-  constexpr int V = 8;  // bf16 per 16-byte vector
-  if (e < E) {
-    const int nv = H / V, per = nv / 4;  // H is a multiple of 128: per is a multiple of 4
-    const int v0 = qt * per;
-    const __nv_bfloat16* w = Wr + static_cast<int64_t>(e) * H;
-    double ss = 0.0;
-    for (int tg = 0; tg < T; tg += 8) {
-      double acc[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[j] = 0.0;
-      // rounds of four 16-byte vectors per lane (one round at H = 4096), every load of a
-      // round issued before its arithmetic
-      for (int ub = 0; ub < per; ub += 128) {
-        Vec16<__nv_bfloat16> wv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int vi = ub + 32 * u + lane;
-          if (vi < per) wv[u] = ld16(w + (v0 + vi) * V);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int vi = ub + 32 * u + lane;
-          if (vi >= per) continue;
-          Vec16<__nv_bfloat16> xv[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (tg + j < T) xv[j] = ld16(x + static_cast<int64_t>(tg + j) * H + (v0 + vi) * V);
-          double wd[V];
-#pragma unroll
-          for (int i = 0; i < V; ++i) wd[i] = static_cast<double>(__bfloat162float(wv[u].v[i]));
-          if (tg == 0) {
-#pragma unroll
-            for (int i = 0; i < V; ++i) ss = fma(wd[i], wd[i], ss);
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (tg + j < T) {
-#pragma unroll
-              for (int i = 0; i < V; ++i) acc[j] = fma(static_cast<double>(__bfloat162float(xv[j].v[i])), wd[i], acc[j]);
-            }
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
-        if (lane == 0 && tg + j < T) sm.part[el][qt][tg + j] = acc[j];
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) sm.part[el][qt][kFusedMaxTokens] = ss;
-  }
-  __syncthreads();
-  // the memory stream is idle while the batch is selected: bring this block's slice of `pf`
-  // (the shared expert's gate/up weights, which the expert GEMM reads first) into L2, after
-  // this block's own W_router loads so as not to delay them
-  if (pf && threadIdx.x == 0) {
-    const int64_t per = ((pf_bytes + gridDim.x - 1) / gridDim.x + 15) & ~static_cast<int64_t>(15);
-    const int64_t b0 = per * blockIdx.x, b1 = b0 + per < pf_bytes ? b0 + per : pf_bytes;
-    if (b1 > b0) prefetch_l2(pf + b0, static_cast<uint64_t>(b1 - b0));
-  }
-  // the quarters in a fixed order: scores [T, E] and the experts' sums of squares
-  for (int i = threadIdx.x; i < kFusedExperts * (T + 1); i += blockDim.x) {
-    const int q = i / (T + 1), t = i - q * (T + 1);
-    const int eq = blockIdx.x * kFusedExperts + q;
-    if (eq >= E) continue;
-    const int slot = t < T ? t : kFusedMaxTokens;
-    const double v = ((sm.part[q][0][slot] + sm.part[q][1][slot]) + sm.part[q][2][slot]) + sm.part[q][3][slot];
-    if (t < T) scores[static_cast<int64_t>(t) * E + eq] = v;
-    else wnorm[eq] = norm_ub_from_sumsq(v, H);
-  }
-  // the last block selects and dispatches
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) sm.is_last = atomicAdd(done, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!sm.is_last) return;
-  __threadfence();
-  pdl_trigger();  // the expert GEMM's blocks may take their SMs during the selection
-  for (int t = warp; t < T && warp < kFusedSelWarps; t += kFusedSelWarps) {
-    const __nv_bfloat16* xt = x + static_cast<int64_t>(t) * H;
-    const double nx = norm_ub_from_sumsq(warp_sumsq(xt, H), H);
-    if (!select_token<__nv_bfloat16, __nv_bfloat16, EPL, SIG>(scores + static_cast<int64_t>(t) * E, 1.01 * H * kU53,
-                                                              0.0, false, nx, wnorm, nullptr, kf, xt, Wr, H, E, k, t,
-                                                              idx_ws, w_ws, idx_user, w_user, sm.sel.cands[warp], ctrl))
-      select_token_slow<__nv_bfloat16, __nv_bfloat16, SIG>(scores + static_cast<int64_t>(t) * E, 1, 1.01 * H * kU53,
-                                                          0.0, false, nx, wnorm, nullptr, key_spill(spill, T, E, t), kf,
-                                                          xt, Wr, H, E, k, t, idx_ws, w_ws, idx_user, w_user,
-                                                          sm.sel.exact_scratch[warp], ctrl);
-  }
-  __syncthreads();  // idx_ws / w_ws written by this block are visible to all its threads
-  dispatch_small_block(sa, idx_ws, w_ws, k, counts, counts_user, perm, inv_perm, row_w, row_tok, perm_user, ctrl,
-                       sm.disp);
-}
-
-bool route_dispatch_fused_supported(const moe_layer_shape& s, bool w32, int bn) {
-  return s.dtype == MOE_BF16 && !w32 && s.T >= 1 && s.T <= kFusedMaxTokens && s.E + 1 <= 2 * kFusedThreads &&
-         bn == 16;
-}
-
-cudaError_t launch_route_dispatch_small(const RouterArgs& a, const DispatchArgs& da, double* wnorm,
-                                        cudaStream_t st) {
-  const ScheduleArgs sa = schedule_args(da);
-  const unsigned grid = static_cast<unsigned>((a.E + kFusedExperts - 1) / kFusedExperts);
-  auto go = [&](auto kern) {
-    return launch_pdl(kern, dim3(grid), dim3(kFusedThreads), 0, st, static_cast<const __nv_bfloat16*>(a.x),
-                      static_cast<const __nv_bfloat16*>(a.Wr), Keys{a.bias, a.sigmoid, a.scale},
-                      static_cast<int>(a.T), a.H, a.E, a.k, a.scores64, wnorm, a.group_done, a.idx_ws, a.w_ws,
-                      a.idx_user, a.w_user, a.spill, sa, da.counts, da.counts_user, da.perm, da.inv_perm, da.row_w,
-                      da.row_tok, da.perm_user, static_cast<const unsigned char*>(a.prefetch), a.prefetch_bytes,
-                      a.ctrl);
-  };
-  const int epl = select_epl(a.E);
-  cudaError_t e;
-  if (a.sigmoid)
-    e = epl == 4 ? go(route_dispatch_small_kernel<4, true>)
-        : epl == 12 ? go(route_dispatch_small_kernel<12, true>) : go(route_dispatch_small_kernel<32, true>);
-  else
-    e = epl == 4 ? go(route_dispatch_small_kernel<4, false>)
-        : epl == 12 ? go(route_dispatch_small_kernel<12, false>) : go(route_dispatch_small_kernel<32, false>);
-  count_launches(1);
-  return e;
 }
 
 // ---------------------------------------------------------------------------------------
