@@ -84,12 +84,19 @@ constexpr int kRing = 4;             // item slots between the producer and the 
 template <bool GATED, int BN, bool W8 = false>
 struct TcCfg {
   static constexpr int kMats = GATED ? 2 : 1;           // weight tiles per stage (gate, up)
-  static constexpr int kABytes = kTileM * kTileK * 2;  // 16 KB of bf16 weights per operand tile
-  static constexpr int kA8Bytes = kTileM * kTileK;     // the same tile as FP8 codes
-  static constexpr int kBBytes = BN * kTileK * 2;      // token rows
+  // k-blocks (64 columns, one 128-byte swizzle atom wide) per stage.  bf16 16-token tiles
+  // stream their weights from HBM: two adjacent k-blocks per stage, so that each weight row
+  // is requested 256 contiguous bytes at a time rather than 128
+  static constexpr int kKB = (BN == 16 && !W8) ? 2 : 1;
+  static constexpr int kAtomA = kTileM * kTileK * 2;   // one k-block of 128 weight rows (16 KB)
+  static constexpr int kAtomB = BN * kTileK * 2;       // one k-block of the token rows
+  static constexpr int kABytes = kKB * kAtomA;         // bf16 weights per operand tile and stage
+  static constexpr int kA8Bytes = kTileM * kTileK;     // one k-block as FP8 codes
+  static constexpr int kBBytes = kKB * kAtomB;         // token rows
   // one TMA stage: the weight tiles as loaded (bf16, or FP8 codes), then the token rows
   static constexpr int kBOffset = kMats * (W8 ? kA8Bytes : kABytes);
   static constexpr int kStageBytes = kBOffset + kBBytes;
+  static constexpr int kKBytes = kStageBytes / kKB;     // bytes of one k-block of a stage
   // FP8: stages of converted bf16 weight tiles plus a copy of the token rows, between the
   // converters and the MMA.  The converters free each TMA stage as soon as they have read
   // it, so every TMA stage is either in flight or waiting for conversion.  More converted
@@ -437,8 +444,9 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
           }
         }
       }
-      for (int kb = kb0; kb < kb1; ++kb) {
+      for (int kb = kb0; kb < kb1; kb += C::kKB) {
         unsigned char* st = smem + stage * C::kStageBytes;
+        const int nk = min(C::kKB, kb1 - kb);  // k-blocks in this stage
         uint32_t scw = 0;
         if (W8) {
           const int rel = (kb >> 1) - sc0;  // < 64: the host bounds K by 64 scale blocks
@@ -450,20 +458,24 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
           good = wait(&empty[stage], phase ^ 1u) ? 1 : 0;
           if (good) {
             if (W8) sc_stage[stage] = scw;  // published by the arrive below
-            mbar_arrive_expect_tx(&full[stage], C::kCpGather ? C::kBOffset : C::kStageBytes);
-            tma_load_2d(st, &p.tmA[t.sh], kb * kTileK, arow, &full[stage]);
-            if (GATED)
-              tma_load_2d(st + (W8 ? C::kA8Bytes : C::kABytes), &p.tmA[t.sh], kb * kTileK,
-                          arow + p.a_up_offset[t.sh], &full[stage]);
-            if (!gath && !C::kCpGather)
-              tma_load_2d(st + C::kBOffset, &p.tmB[t.sh], kb * kTileK, t.row0, &full[stage]);
+            mbar_arrive_expect_tx(&full[stage], C::kCpGather ? C::kBOffset : nk * C::kKBytes);
+            for (int j = 0; j < nk; ++j) {
+              tma_load_2d(st + j * C::kAtomA, &p.tmA[t.sh], (kb + j) * kTileK, arow, &full[stage]);
+              if (GATED)
+                tma_load_2d(st + (W8 ? C::kA8Bytes : C::kABytes) + j * C::kAtomA, &p.tmA[t.sh],
+                            (kb + j) * kTileK, arow + p.a_up_offset[t.sh], &full[stage]);
+              if (!gath && !C::kCpGather)
+                tma_load_2d(st + C::kBOffset + j * C::kAtomB, &p.tmB[t.sh], (kb + j) * kTileK, t.row0,
+                            &full[stage]);
+            }
           }
         }
         good = __shfl_sync(0xffffffffu, good, 0);
         if (!good) { ok = false; break; }
         if (gath && lane < BN / 4)
-          tma_gather4_2d(st + C::kBOffset + lane * 4 * kTileK * 2, &p.tmB[0], kb * kTileK,
-                         tok[0], tok[1], tok[2], tok[3], &full[stage]);
+          for (int j = 0; j < nk; ++j)
+            tma_gather4_2d(st + C::kBOffset + j * C::kAtomB + lane * 4 * kTileK * 2, &p.tmB[0], (kb + j) * kTileK,
+                           tok[0], tok[1], tok[2], tok[3], &full[stage]);
         used |= 1u << stage;
         if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
       }
@@ -603,22 +615,25 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
         const uint32_t d0 = tmem_base + acc * C::kAccCols;
         const int kb_n = p.kblocks[t.sh];
         const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; kb += C::kKB) {
           if (!(W8 ? wait(&cfull[cs], cphase) : wait(&full[stage], phase))) { ok = false; break; }
           tc_fence_after();
           // token rows written by the gather warps' cp.async: order them before the
           // tensor cores' (async-proxy) reads of the stage
           if (C::kCpGather) fence_proxy_async_smem();
           const uint32_t s0 = W8 ? smem_u32(conv + cs * C::kConvBytes) : smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t a0 = s0;
-          const uint32_t b0 = s0 + (W8 ? C::kConvBOffset : C::kBOffset);
+          const int nk = min(C::kKB, kb1 - kb);
+          for (int j = 0; j < nk; ++j) {
+            const uint32_t a0 = s0 + j * C::kAtomA;
+            const uint32_t b0 = s0 + (W8 ? C::kConvBOffset : C::kBOffset) + j * C::kAtomB;
 #pragma unroll
-          for (int kk = 0; kk < kTileK / 16; ++kk) {
-            const uint32_t accum = (kb != kb0 || kk) ? 1u : 0u;
-            const uint64_t bdesc = sw128_kmajor_desc(b0 + kk * 32);
-            mma_bf16(d0, sw128_kmajor_desc(a0 + kk * 32), bdesc, idesc, accum);
-            if (GATED)
-              mma_bf16(d0 + BN, sw128_kmajor_desc(a0 + C::kABytes + kk * 32), bdesc, idesc, accum);
+            for (int kk = 0; kk < kTileK / 16; ++kk) {
+              const uint32_t accum = (kb != kb0 || j || kk) ? 1u : 0u;
+              const uint64_t bdesc = sw128_kmajor_desc(b0 + kk * 32);
+              mma_bf16(d0, sw128_kmajor_desc(a0 + kk * 32), bdesc, idesc, accum);
+              if (GATED)
+                mma_bf16(d0 + BN, sw128_kmajor_desc(a0 + C::kABytes + kk * 32), bdesc, idesc, accum);
+            }
           }
           if (W8) {
             mma_commit(&cempty[cs]);
