@@ -58,28 +58,29 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScheduleArgs sa, int k, int 
   pdl_wait();
   pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
   const int E = sa.E;
-  // each warp scans the block counts of one expert at a time (lanes over blocks)
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int e = warp; e < E; e += blockDim.x / 32) {
-    int run = 0;
-    for (int b0 = 0; b0 < nblk; b0 += 32) {
-      const int b = b0 + lane;
-      const int64_t i = static_cast<int64_t>(b) * E + e;
-      const int c = (b < nblk) ? blk_hist[i] : 0;
-      int incl = c;
+  // thread e scans the block counts of expert e (loads coalesced across experts), sixteen
+  // blocks' counts in flight at a time
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0, b = 0;
+    for (; b + 16 <= nblk; b += 16) {
+      int v[16];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+      for (int j = 0; j < 16; ++j) v[j] = blk_hist[static_cast<int64_t>(b + j) * E + e];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        blk_hist[static_cast<int64_t>(b + j) * E + e] = run;
+        run += v[j];
       }
-      if (b < nblk) blk_hist[i] = run + incl - c;
-      run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-      cnt[e] = run;
-      counts[e] = run;
-      if (counts_user) counts_user[e] = run;
+    for (; b < nblk; ++b) {
+      const int64_t i = static_cast<int64_t>(b) * E + e;
+      const int c = blk_hist[i];
+      blk_hist[i] = run;
+      run += c;
     }
+    cnt[e] = run;
+    counts[e] = run;
+    if (counts_user) counts_user[e] = run;
   }
   if (sa.has_shared && threadIdx.x == 0) cnt[E] = sa.shared_rows;
   __syncthreads();

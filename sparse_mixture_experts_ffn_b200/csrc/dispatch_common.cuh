@@ -64,11 +64,12 @@ struct ScheduleArgs {
 };
 
 // shared-memory scratch of build_schedule / write_item_tables (groups G <= 2048)
-struct ScheduleSmem {
-  int istart_gu[2049];
+struct __align__(16) ScheduleSmem {
+  int istart_gu[2049];  // istart_gu and istart_dn (contiguous) also hold the sort keys
   int istart_dn[2049];
   int off[2049];
 };
+static_assert(sizeof(int) * 2 * 2049 >= sizeof(unsigned long long) * 2048, "room for the sort keys");
 
 // From the group sizes cnt[0..G) (routed experts, then the shared expert with all T
 // tokens): offsets of the routed experts, the largest-first group order and the tile
@@ -94,32 +95,64 @@ static __device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* orde
       if (a.offsets_user) a.offsets_user[E] = total;
     }
   }
-  // largest group first: rank by (count desc, index asc).  Groups without tokens take the
-  // last places in index order; the others are first compacted (in index order) into the
-  // leading places of order[] and ranked among themselves only.
+  // largest group first: order by (count desc, index asc), groups without rows last in
+  // index order.  The groups with rows are first compacted (in index order) into the leading
+  // places of order[], the others after them.  Few groups with rows (small batches): each
+  // is ranked by a count over the others; many: one ascending bitonic sort of the keys
+  // (~count << 32 | index) over the next power of two >= G, padded with keys above every
+  // real one, two keys a thread.
   {
     const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
     const int z0 = (i0 < G && cnt[i0] > 0) ? 1 : 0, z1 = (i1 < G && cnt[i1] > 0) ? 1 : 0;
     int nnz;
     const int nz_ex = block_scan_pair(z0, z1, warp_tot, nnz);
-    if (i0 < G) order[z0 ? nz_ex : nnz + (i0 - nz_ex)] = i0;
-    if (i1 < G) order[z1 ? nz_ex + z0 : nnz + (i1 - nz_ex - z0)] = i1;
-    __syncthreads();
-    auto rank_of = [&](int g) {
-      const int c = cnt[g];
-      int r = 0;
-      for (int j = 0; j < nnz; ++j) {
-        const int h = order[j];
-        const int ch = cnt[h];
-        r += (ch > c) || (ch == c && h < g);
+    if (nnz <= 64) {
+      if (i0 < G) order[z0 ? nz_ex : nnz + (i0 - nz_ex)] = i0;
+      if (i1 < G) order[z1 ? nz_ex + z0 : nnz + (i1 - nz_ex - z0)] = i1;
+      __syncthreads();
+      auto rank_of = [&](int g) {
+        const int c = cnt[g];
+        int r = 0;
+        for (int j = 0; j < nnz; ++j) {
+          const int h = order[j];
+          const int ch = cnt[h];
+          r += (ch > c) || (ch == c && h < g);
+        }
+        return r;
+      };
+      const int r0 = z0 ? rank_of(i0) : -1, r1 = z1 ? rank_of(i1) : -1;
+      __syncthreads();
+      if (r0 >= 0) order[r0] = i0;
+      if (r1 >= 0) order[r1] = i1;
+      __syncthreads();
+    } else {
+      // [n <= 2048] keys in the prefix arrays, which are written only after the sort
+      unsigned long long* key = reinterpret_cast<unsigned long long*>(ss.istart_gu);
+      int n = 1;
+      while (n < G) n <<= 1;
+      for (int i = threadIdx.x; i < n; i += blockDim.x)
+        key[i] = i < G ? (static_cast<unsigned long long>(~static_cast<uint32_t>(cnt[i])) << 32) |
+                             static_cast<uint32_t>(i)
+                       : ~0ull;
+      __syncthreads();
+      for (int size = 2; size <= n; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          for (int t = threadIdx.x; t < (n >> 1); t += blockDim.x) {
+            // pair (i, i + stride) of the stride-sized half blocks; ascending where i & size is 0
+            const int i = 2 * t - (t & (stride - 1));
+            const unsigned long long x = key[i], y = key[i + stride];
+            const bool up = (i & size) == 0;
+            if ((x > y) == up) {
+              key[i] = y;
+              key[i + stride] = x;
+            }
+          }
+          __syncthreads();
+        }
       }
-      return r;
-    };
-    const int r0 = z0 ? rank_of(i0) : -1, r1 = z1 ? rank_of(i1) : -1;
-    __syncthreads();
-    if (r0 >= 0) order[r0] = i0;
-    if (r1 >= 0) order[r1] = i1;
-    __syncthreads();
+      for (int i = threadIdx.x; i < G; i += blockDim.x) order[i] = static_cast<int>(key[i] & 0xFFFFFFFFu);
+      __syncthreads();
+    }
   }
   for (int r = threadIdx.x; r < G; r += blockDim.x) a.group_order[r] = order[r];
   const int r0 = 2 * threadIdx.x, r1 = r0 + 1;
