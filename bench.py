@@ -177,20 +177,32 @@ def measured_peaks():
         return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
-def ncu_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it still matches the source."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
-    try:
-        with open(path) as f:
-            d = json.load(f)
-        ent = d[f"{kernel}@{workload}"]
-        import hashlib
-        src = os.path.join(ROOT, ent["source"])
-        if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != ent["source_sha"]:
-            return None
-        return float(ent["dram_bytes_per_launch"])
-    except Exception:
-        return None
+def ncu_traffic(kernel: str, workload: str, algorithmic_bytes: float):
+    """DRAM bytes per launch of `kernel` on `workload`, from a committed ncu summary under
+    profiles/: a line `traffic-ratio <kernel> <workload> <ratio> <source> <sha256[:16]>`
+    gives the kernel's DRAM bytes over its algorithmic bytes, measured by ncu on a small
+    variant of the workload (the ratio carries over: the bytes per weight tile and token row
+    do not depend on the number of experts).  None when no summary matches or the kernel's
+    source has changed since the capture."""
+    import glob
+    import hashlib
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        try:
+            lines = open(path).read().splitlines()
+        except OSError:
+            continue
+        for line in lines:
+            f = line.strip().strip("`").split()
+            if len(f) != 6 or f[0] != "traffic-ratio" or f[1] != kernel or f[2] != workload:
+                continue
+            try:
+                src = open(os.path.join(ROOT, f[4]), "rb").read()
+            except OSError:
+                return None
+            if hashlib.sha256(src).hexdigest()[:16] != f[5]:
+                return None
+            return float(f[3]) * algorithmic_bytes
+    return None
 
 
 # ------------------------------------------------------------------------------------------
@@ -360,7 +372,7 @@ def roofline(alg, peaks, gu_ms, fp8, workload):
                 "frac": achieved / peaks["hbm_gbs"]}
     roof.update({"kernel": "expert_gemm_tc_kernel<gated%s> (gate/up GEMM + SiLU*up)" % (", fp8" if fp8 else ""),
                  "timing": "CUDA events around each launch, stage-timed pass of the same steps",
-                 "traffic": ncu_traffic("gate_up", workload + ("+fp8" if fp8 else "")),
+                 "traffic": ncu_traffic("gate_up", workload + ("+fp8" if fp8 else ""), alg["gate_up_bytes"]),
                  "peak_source": peaks["source"],
                  "ms_per_launch": gu_ms, "algorithmic_bytes": alg["gate_up_bytes"],
                  "algorithmic_flops": alg["gate_up_flops"]})
