@@ -292,12 +292,11 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
   // FP8 weights run on 16- and 128-token tiles only
   const int bn_dn = wt.w8 ? std::min(L.bn_dn, 128) : L.bn_dn;
-  // long prefill: the down projection on 256-row tiles over pairs of SMs.  The gate/up GEMM
-  // stays on one SM a tile, where its four gather warps read the token rows straight from x
-  // (measured faster than pair tiles fed from a gathered copy of x)
+  // long prefill: the down projection on 256-row x 256-token tiles over pairs of SMs (the
+  // gate/up GEMM stays on one SM a tile, where its gather warps read the token rows from x)
   const bool pair = s.dtype == MOE_BF16 && !wt.w8 && L.ksplit == 1 &&
                     choose_pair(s.T, s.top_k, s.E, s.H, s.I, s.I_shared);
-  const bool pair_gu = false, pair_dn = pair;
+  const bool pair_dn = pair;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
@@ -353,12 +352,11 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   da.bn = L.bn;
   da.bn_dn = bn_dn;
   da.ksplit = L.ksplit;
-  da.pair_gu = pair_gu;
   da.pair_dn = pair_dn;
   da.e_lo = e_lo;
   da.e_hi = e_hi;
   da.shared_rows = static_cast<int>(sh_hi - sh_lo);
-  da.need_x_perm = !bf16 || (wt.w8 && L.bn == 128) || pair_gu;
+  da.need_x_perm = !bf16 || (wt.w8 && L.bn == 128);
   da.x = x;
   da.idx = ra.idx_ws;
   da.w = ra.w_ws;
@@ -417,7 +415,6 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   ea.row_w = da.row_w;
   ea.x_perm = da.x_perm;
   ea.row_tok = da.row_tok;
-  ea.pair_gu = pair_gu;
   ea.pair_dn = pair_dn;
   ea.bn = L.bn;
   ea.bn_dn = bn_dn;

@@ -306,12 +306,11 @@ inline ScheduleArgs schedule_args(const DispatchArgs& a) {
   sa.T = a.T;
   sa.E = a.E;
   sa.has_shared = a.Is > 0 ? 1 : 0;
-  const int tm_gu = a.pair_gu ? 2 * kTileM : kTileM;  // weight rows per tile
   const int tm_dn = a.pair_dn ? 2 * kTileM : kTileM;
-  sa.mt_gu = a.I / tm_gu;
-  sa.mt_gu_shared = a.Is / tm_gu;
+  sa.mt_gu = a.I / kTileM;
+  sa.mt_gu_shared = a.Is / kTileM;
   sa.mt_dn = a.H / tm_dn;
-  sa.bn = a.pair_gu ? 128 : a.bn;  // pair tiles: 128 tokens for gate/up, 256 for down
+  sa.bn = a.bn;
   sa.bn_dn = a.pair_dn ? 256 : a.bn_dn;
   sa.ksplit = a.ksplit;
   sa.e_lo = a.e_lo;

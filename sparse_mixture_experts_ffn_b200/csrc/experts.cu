@@ -897,32 +897,25 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
 }
 
 // ---------------------------------------------------------------------------------------
-// Pair tiles for long prefill (on average 256 or more tokens per expert): a cluster of two
-// CTAs on two SMs computes one 256-row weight tile x BN-token tile with tcgen05.mma
-// cta_group::2.  CTA c of the pair holds weight rows [128c, 128c + 128) of the tile and
-// token rows [c BN/2, (c + 1) BN/2) in its own shared memory; the even CTA's single MMA
-// thread multiplies the pair's 256 x BN tile, each CTA's tensor memory receiving its own 128
-// weight rows for all BN tokens.  Each SM thus loads half the token rows a single-SM tile of
-// the same shape would:
-//   gate/up (BN = 128): the CTA's 128 gate rows and its 128 up rows of the same
-//            intermediate units, two MMAs per step sharing the token rows (x_perm, the
-//            routed rows of x in expert order; the shared expert's rows of x); accumulators
-//            gate | up, 256 columns, two buffers;
-//   down (BN = 256): one MMA per step, 256 columns, two buffers; the routing weight in
-//            the epilogue.
+// Pair tiles for the down GEMM of long prefill (on average 256 or more tokens per expert): a
+// cluster of two CTAs on two SMs computes one 256-row weight tile x 256-token tile with
+// tcgen05.mma cta_group::2.  CTA c of the pair holds weight rows [128c, 128c + 128) of the
+// tile and token rows [128c, 128c + 128) in its own shared memory; the even CTA's MMA warp
+// multiplies the pair's 256 x 256 tile, each CTA's tensor memory receiving its own 128 weight
+// rows for all 256 tokens (two 256-column accumulators).  Each SM thus loads, and its tensor
+// cores read, half the token rows a single-SM tile of the same shape would.  The routing
+// weight is applied in the epilogue.
 // Work items (group, 256-row weight tile, token tile) are taken in a fixed order, pair q
 // doing items q, q + pairs, ...; both CTAs walk the same sequence.  TMA loads of both CTAs
 // complete on the even CTA's barrier; the MMA commits arrive on both CTAs' barriers; both
 // epilogues release an accumulator on the even CTA's barrier.
 // ---------------------------------------------------------------------------------------
-template <bool GATED>
 struct PairCfg {
-  static constexpr int BN = GATED ? 128 : 256;          // tokens per pair tile
-  static constexpr int kMats = GATED ? 2 : 1;
-  static constexpr int kABytes = kTileM * kTileK * 2;  // this CTA's 128 rows of one matrix
+  static constexpr int BN = 256;                       // tokens per pair tile
+  static constexpr int kABytes = kTileM * kTileK * 2;  // this CTA's 128 weight rows
   static constexpr int kBRows = BN / 2;                // this CTA's token rows
   static constexpr int kBBytes = kBRows * kTileK * 2;
-  static constexpr int kBOffset = kMats * kABytes;
+  static constexpr int kBOffset = kABytes;
   static constexpr int kStageBytes = kBOffset + kBBytes;
   static constexpr int kThreads = 192 + 32;            // + the stage watcher (even CTA)
   static constexpr int kChunk = 32;                    // tokens per epilogue chunk
@@ -930,7 +923,7 @@ struct PairCfg {
   static constexpr int kAuxBytes = 2048;               // barriers, TMEM slot, row weights
   static constexpr int kFit = (kMaxDynSmem - kStagingBytes - 1024 - kAuxBytes) / kStageBytes;
   static constexpr int kStages = kFit > 8 ? 8 : kFit;
-  static constexpr int kAccCols = (GATED ? 2 : 1) * BN;
+  static constexpr int kAccCols = BN;
   static constexpr int kAccBufs = 2;
   static constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + kAuxBytes;
   static_assert(kStages >= 3 && kSmemBytes <= kMaxDynSmem, "shared memory budget");
@@ -938,9 +931,8 @@ struct PairCfg {
   static_assert(kAccBufs * kAccCols <= 512, "tensor memory");
 };
 
-template <bool GATED>
-__global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_kernel(const __grid_constant__ TcParams p) {
-  using C = PairCfg<GATED>;
+__global__ void __launch_bounds__(PairCfg::kThreads, 1) expert_gemm_pair_kernel(const __grid_constant__ TcParams p) {
+  using C = PairCfg;
   constexpr int BN = C::BN;
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -1000,7 +992,6 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
           const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
           if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
           tma_load_2d_pair(st, &p.tmA[t.sh], kb * kTileK, arow, fb);
-          if (GATED) tma_load_2d_pair(st + C::kABytes, &p.tmA[t.sh], kb * kTileK, arow + p.a_up_offset[t.sh], fb);
           tma_load_2d_pair(st + C::kBOffset, &p.tmB[t.sh], kb * kTileK, brow, fb);
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
@@ -1033,7 +1024,6 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
               const uint32_t accum = (kb || kk) ? 1u : 0u;
               const uint64_t bdesc = sw128_kmajor_desc(b0 + kk * 32);
               mma_bf16_pair(d0, sw128_kmajor_desc(a0 + kk * 32), bdesc, idesc, accum);
-              if (GATED) mma_bf16_pair(d0 + BN, sw128_kmajor_desc(a0 + C::kABytes + kk * 32), bdesc, idesc, accum);
             }
             mma_commit_pair(&empty[stage]);
           }
@@ -1085,10 +1075,8 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
     for (int it = pair; it < total; it += npairs) {
       const Item t = decode_item<BN>(p, it);
       if (!t.valid) continue;
-      if (!GATED) {
-        for (int n = et; n < BN; n += 128) sw[n] = (t.sh || n >= t.nvalid) ? 1.0f : __ldg(p.row_w + t.row0 + n);
-        named_bar_sync(1, 128);
-      }
+      for (int n = et; n < BN; n += 128) sw[n] = (t.sh || n >= t.nvalid) ? 1.0f : __ldg(p.row_w + t.row0 + n);
+      named_bar_sync(1, 128);
       if (!mbar_wait_cluster(&tfull[acc], acc_phase, p.ctrl, abort_flag)) break;
       tc_fence_after();
       const uint32_t trow = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * C::kAccCols;
@@ -1098,11 +1086,6 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
         uint32_t a[32];
         tmem_ld16_nowait(trow + c0, a);
         tmem_ld16_nowait(trow + c0 + 16, a + 16);
-        uint32_t u[GATED ? 32 : 1];
-        if (GATED) {
-          tmem_ld16_nowait(trow + BN + c0, u);
-          tmem_ld16_nowait(trow + BN + c0 + 16, u + 16);
-        }
         tmem_wait_ld();
         if (c0 + C::kChunk >= t.nvalid) {  // the accumulator has been read: release it
           tc_fence_before();
@@ -1110,12 +1093,8 @@ __global__ void __launch_bounds__(PairCfg<GATED>::kThreads, 1) expert_gemm_pair_
           if (lane == 0) mbar_arrive_remote(acc ? tempty_even1 : tempty_even0);
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float v;
-          if (GATED) v = swiglu(__uint_as_float(a[j]), __uint_as_float(u[GATED ? j : 0]), p.limit[t.sh]);
-          else v = __uint_as_float(a[j]) * sw[c0 + j];
-          staging[j * kTileM + r] = __float2bfloat16_rn(v);
-        }
+        for (int j = 0; j < 32; ++j)
+          staging[j * kTileM + r] = __float2bfloat16_rn(__uint_as_float(a[j]) * sw[c0 + j]);
         named_bar_sync(1, 128);
         // rows of 128 bf16 (256 B) -> out[row0 + c0 + j][...], 16-byte coalesced stores
         const int rows = min(C::kChunk, t.nvalid - c0);
@@ -1275,10 +1254,9 @@ static cudaError_t launch_tc(const TcParams& prm_in, int num_sms, cudaStream_t s
   return e;
 }
 
-template <bool GATED>
 static cudaError_t launch_pair(const TcParams& prm, int num_sms, cudaStream_t st) {
-  using C = PairCfg<GATED>;
-  auto kern = expert_gemm_pair_kernel<GATED>;
+  using C = PairCfg;
+  auto kern = expert_gemm_pair_kernel;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -1351,10 +1329,10 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   const bool gather = a.bn == 16;
   // bf16 128-token tiles gather their token rows inside the kernel (no x_perm); FP8 weights
   // read the permuted copy
-  const bool cp_gather = !a.pair_gu && a.bn == 128 && !a.w8;
+  const bool cp_gather = a.bn == 128 && !a.w8;
   // token rows per B copy (pair tiles: each CTA's half; the gate/up pair kernel gathers its
   // rows itself and never uses its B maps)
-  const uint32_t box_gu = a.pair_gu ? 64 : static_cast<uint32_t>(a.bn);
+  const uint32_t box_gu = static_cast<uint32_t>(a.bn);
   const uint32_t box_dn = a.pair_dn ? 128 : static_cast<uint32_t>(a.bn_dn);
   // weight matrices: bf16 rows, or FP8 code rows with their block scales
   auto encode_w = [&](CUtensorMap* m, const void* w, uint64_t rows, uint64_t cols) {
@@ -1420,13 +1398,7 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   g.scaleA[1] = static_cast<const uint8_t*>(a.Wsgu_scale);
   g.s_rows_per_group = 2 * a.I / kTileM;
   g.s_ld[0] = g.s_ld[1] = (a.H + 127) / 128;
-  if (a.pair_gu) {  // 256-row weight tiles over pairs of SMs, 128-token tiles
-    g.mt[0] = a.I / 256;
-    g.mt[1] = a.Is / 256;
-    g.max_tiles = static_cast<int>(expert_tile_bound(a.T, a.k, a.E, a.I / 2, a.Is / 2, 128));
-    g.max_items = g.max_tiles;
-  }
-  cudaError_t e = a.pair_gu ? launch_pair<true>(g, a.num_sms, st) : launch_tc_bn<true>(g, a.bn, a.w8, a.num_sms, st);
+  cudaError_t e = launch_tc_bn<true>(g, a.bn, a.w8, a.num_sms, st);
   if (e != cudaSuccess) return e;
   if (a.stage_mark) a.stage_mark(a.stage_mark_ctx, 3, st);
   // down: A = W_down viewed as [E*H, I]; B = h [P, I] (shared: Ws_down [H, Is], h_shared)
@@ -1475,7 +1447,7 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
     d.mt[0] = d.mt[1] = a.H / 256;
     d.max_tiles = static_cast<int>(expert_tile_bound(a.T, a.k, a.E, a.H / 2, a.Is > 0 ? a.H / 2 : 0, 256));
     d.max_items = d.max_tiles;
-    return launch_pair<false>(d, a.num_sms, st);
+    return launch_pair(d, a.num_sms, st);
   }
   return launch_tc_bn<false>(d, a.bn_dn, a.w8, a.num_sms, st);
 }

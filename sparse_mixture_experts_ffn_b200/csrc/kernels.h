@@ -79,7 +79,6 @@ struct DispatchArgs {
   int64_t T;
   int H, E, k;
   int I, Is;        // expert widths (Is = 0: no shared expert)
-  bool pair_gu;     // gate/up GEMM on 256-row x 128-token tiles over pairs of SMs
   bool pair_dn;     // down GEMM on 256-row x 256-token tiles over pairs of SMs
   int bn;           // tokens per gate/up GEMM tile
   int bn_dn;        // tokens per down GEMM tile
@@ -137,7 +136,6 @@ struct ExpertArgs {
   const float* row_w;
   const int32_t* row_tok;  // [T*k] token of each routed row (bf16: gathered from x)
   const void* x_perm;      // fp32 path: routed rows of x in expert order
-  bool pair_gu;     // long prefill: gate/up on 256-row x 128-token tiles over pairs of SMs
   bool pair_dn;     // long prefill: down on 256-row x 256-token tiles over pairs of SMs
   int bn;           // tokens per gate/up GEMM tile (16 or 128)
   int bn_dn;        // tokens per down GEMM tile (16, 128 or 256)
