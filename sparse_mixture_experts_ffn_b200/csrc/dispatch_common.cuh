@@ -226,30 +226,43 @@ static __device__ void write_item_tables(const ScheduleArgs& a, const int* cnt, 
 
 // Stable placement of the assignments [a0, a1) by one warp, 32 at a time, in (token,
 // slot) order: equal experts inside a chunk get consecutive positions in lane order.
-// base[e] holds the next free position of expert e and is advanced.
+// base[e] holds the next free position of expert e and is advanced.  The indices and weights
+// of four chunks are loaded before the first of them is placed.
 static __device__ void place_assignments(const int32_t* __restrict__ idx, const float* __restrict__ w,
                                   int64_t a0, int64_t a1, int k, int E, int* base,
                                   int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
                                   float* __restrict__ row_w, int32_t* __restrict__ row_tok,
                                   int32_t* __restrict__ perm_user) {
   const int lane = threadIdx.x & 31;
-  for (int64_t c = a0; c < a1; c += 32) {
-    const int64_t a = c + lane;
-    int e = (a < a1) ? idx[a] : -1;
-    if (e < 0 || e >= E) e = -1;  // reported by the histogram
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    int pos = 0;
-    if (e >= 0) pos = base[e] + rank;
-    __syncwarp();
-    if (e >= 0 && rank == 0) base[e] += __popc(peers);
-    __syncwarp();
-    if (e >= 0) {
-      perm[pos] = static_cast<int32_t>(a);
-      inv_perm[a] = pos;
-      row_w[pos] = w[a];
-      row_tok[pos] = static_cast<int32_t>(a / k);
-      if (perm_user) perm_user[pos] = static_cast<int32_t>(a);
+  constexpr int kAhead = 4;
+  for (int64_t c0 = a0; c0 < a1; c0 += 32 * kAhead) {
+    int ev[kAhead];
+    float wv[kAhead];
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u) {
+      const int64_t a = c0 + 32 * u + lane;
+      ev[u] = (a < a1) ? idx[a] : -1;
+      wv[u] = (a < a1) ? w[a] : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u) {
+      const int64_t a = c0 + 32 * u + lane;
+      int e = ev[u];
+      if (e < 0 || e >= E) e = -1;  // reported by the histogram
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      int pos = 0;
+      if (e >= 0) pos = base[e] + rank;
+      __syncwarp();
+      if (e >= 0 && rank == 0) base[e] += __popc(peers);
+      __syncwarp();
+      if (e >= 0) {
+        perm[pos] = static_cast<int32_t>(a);
+        inv_perm[a] = pos;
+        row_w[pos] = wv[u];
+        row_tok[pos] = static_cast<int32_t>(a / k);
+        if (perm_user) perm_user[pos] = static_cast<int32_t>(a);
+      }
     }
   }
 }
@@ -263,8 +276,8 @@ struct SmallDispatchSmem {
   ScheduleSmem sched;
 };
 
-// The whole dispatch of a small batch by one block of 1024 threads: histogram, counts,
-// offsets and the tile schedule, then the stable placement (one warp).
+// The whole dispatch of a small batch by one block (2 * blockDim.x >= G + 1): histogram,
+// counts, offsets, the tile schedule and descriptors, then the stable placement (one warp).
 static __device__ void dispatch_small_block(const ScheduleArgs& sa, const int32_t* __restrict__ idx,
                                             const float* __restrict__ w, int k, int32_t* __restrict__ counts,
                                             int32_t* __restrict__ counts_user, int32_t* __restrict__ perm,
