@@ -53,3 +53,23 @@ def test_bench_algorithmic_bytes_closed_form():
     assert f["layer_bytes"] == weights + weights // (128 * 128) + 2 * (E * H + 2 * T * H)
     assert b["layer_flops"] == f["layer_flops"] == 2 * T * E * H + T * k * 6 * H * I + T * 6 * H * Is
     assert b["gate_up_bytes"] == 2 * (32 * 2 * I * H + 2 * Is * H) + 2 * (T * k * H + T * H + T * k * I + T * Is)
+
+
+def test_bench_traffic_ratio_follows_its_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from a `traffic-ratio` line of a committed ncu summary, scaled
+    to the launch's algorithmic bytes, and is null once the kernel source no longer matches
+    the hash recorded with the capture."""
+    import hashlib
+
+    import bench
+    src = tmp_path / "kernel.cu"
+    src.write_bytes(b"the kernel as captured\n")
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "profiles" / "gemm.md").write_text(
+        "# capture\n\n    traffic-ratio gate_up decode_t4 1.25 kernel.cu %s\n" % sha)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.ncu_traffic("gate_up", "decode_t4", 1000.0) == 1250.0
+    assert bench.ncu_traffic("gate_up", "decode_t128", 1000.0) is None  # no capture
+    src.write_bytes(b"the kernel, changed since\n")
+    assert bench.ncu_traffic("gate_up", "decode_t4", 1000.0) is None
