@@ -177,15 +177,43 @@ def measured_peaks():
         return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
+def code_digest(src: bytes) -> str:
+    """sha256[:16] of a C/C++/CUDA source with its comments removed and every run of
+    whitespace folded to one space: edits to comments or layout keep the digest, any change
+    to the code (a token added, removed or altered) moves it.  String and character literals
+    are kept as written, so a `//` inside one is not taken for a comment."""
+    import hashlib
+    t = src.decode("utf-8", "replace")
+    out, i, n = [], 0, len(t)
+    while i < n:
+        c = t[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and t[j] != c:
+                j += 2 if t[j] == "\\" else 1
+            out.append(t[i:j + 1])
+            i = j + 1
+        elif t.startswith("//", i):
+            j = t.find("\n", i)
+            i = n if j < 0 else j
+        elif t.startswith("/*", i):
+            j = t.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return hashlib.sha256(" ".join("".join(out).split()).encode()).hexdigest()[:16]
+
+
 def ncu_traffic(kernel: str, workload: str, algorithmic_bytes: float):
     """DRAM bytes per launch of `kernel` on `workload`, from a committed ncu summary under
-    profiles/: a line `traffic-ratio <kernel> <workload> <ratio> <source> <sha256[:16]>`
-    gives the kernel's DRAM bytes over its algorithmic bytes, measured by ncu on a small
-    variant of the workload (the ratio carries over: the bytes per weight tile and token row
-    do not depend on the number of experts).  None when no summary matches or the kernel's
-    source has changed since the capture."""
+    profiles/: a line `traffic-ratio <kernel> <workload> <ratio> <source> <digest>` gives
+    the kernel's DRAM bytes over its algorithmic bytes, measured by ncu on a small variant
+    of the workload (the ratio carries over: the bytes per weight tile and token row do not
+    depend on the number of experts).  <digest> is code_digest() of the kernel source at
+    the capture.  None when no summary matches or the kernel's code has changed since."""
     import glob
-    import hashlib
     for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         try:
             lines = open(path).read().splitlines()
@@ -199,7 +227,7 @@ def ncu_traffic(kernel: str, workload: str, algorithmic_bytes: float):
                 src = open(os.path.join(ROOT, f[4]), "rb").read()
             except OSError:
                 return None
-            if hashlib.sha256(src).hexdigest()[:16] != f[5]:
+            if code_digest(src) != f[5]:
                 return None
             return float(f[3]) * algorithmic_bytes
     return None

@@ -253,8 +253,9 @@ MOE_API moe_status moe_layer_route_stats(void* workspace, moe_route_stats* out, 
 
 /* Byte offsets of the intermediate buffers inside the workspace (for inspection by
  * tests; layout is private and may change between versions).  Sizes in elements:
- *   x_perm [T*top_k, H] dtype (no bytes when the bf16 GEMMs use 16-token tiles, which read
- *   token rows straight from x), h [T*top_k, I] dtype, h_shared [T, I_shared] dtype,
+ *   x_perm [T*top_k, H] dtype (no bytes when the bf16 GEMMs use 16-token tiles; written only
+ *   for fp32 layers and FP8 weights with 128-token tiles: bf16 GEMMs gather their token rows
+ *   from x), h [T*top_k, I] dtype, h_shared [T, I_shared] dtype,
  *   o [T*top_k, H] dtype, o_shared [T, H] dtype, row_w [T*top_k] fp32 (routing weight
  *   of each row of x_perm/h/o in expert order), scores: the fp64 router score estimates
  *   before selection.  scores_slice > 0 for tensor-core scoring (bf16): the H products

@@ -2,7 +2,8 @@
 //
 // bf16: one persistent, warp-specialised tcgen05 kernel per projection.  Weights are the
 // A operand (128 rows per tile, "swap-AB"), the tokens routed to an expert the B operand
-// (up to 128 per tile), so an expert's few tokens never pad a 128-row tile:
+// (16, 128 or 256 per tile), so an expert's few tokens never pad a 128-row tile; the long
+// prefill's down GEMM runs 256-row x 256-token tiles over pairs of SMs (cta_group::2):
 //   gate/up:  h[p, i]  = SiLU(x_p . Wg[e, i]) * (x_p . Wu[e, i])     (SiLU(gate) * up)
 //   down:     o[p, c]  = w_p * (h_p . Wd[e, c])                     (routing weight fused)
 // with fp32 accumulators in tensor memory and bf16 outputs.  The shared expert
@@ -1324,14 +1325,14 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   }
   const int G = a.E + (has_shared ? 1 : 0);
   // gate/up: A = W_gate_up viewed as [E*2I, H]; B = rows of x [T, H] gathered by token
-  // (16-token tiles) or x_perm [P, H] (shared: x [T, H] in order)
+  // (row-gather TMA for 16-token tiles, gather warps for 128-token tiles) or, for FP8 weights
+  // with 128-token tiles, x_perm [P, H]; the shared expert's rows are x [T, H] in order
   TcParams g{};
   const bool gather = a.bn == 16;
   // bf16 128-token tiles gather their token rows inside the kernel (no x_perm); FP8 weights
   // read the permuted copy
   const bool cp_gather = a.bn == 128 && !a.w8;
-  // token rows per B copy (pair tiles: each CTA's half; the gate/up pair kernel gathers its
-  // rows itself and never uses its B maps)
+  // token rows per B copy (down pair tiles: each CTA's half)
   const uint32_t box_gu = static_cast<uint32_t>(a.bn);
   const uint32_t box_dn = a.pair_dn ? 128 : static_cast<uint32_t>(a.bn_dn);
   // weight matrices: bf16 rows, or FP8 code rows with their block scales

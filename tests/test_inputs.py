@@ -57,19 +57,24 @@ def test_bench_algorithmic_bytes_closed_form():
 
 def test_bench_traffic_ratio_follows_its_source(tmp_path, monkeypatch):
     """roofline.traffic comes from a `traffic-ratio` line of a committed ncu summary, scaled
-    to the launch's algorithmic bytes, and is null once the kernel source no longer matches
-    the hash recorded with the capture."""
-    import hashlib
-
+    to the launch's algorithmic bytes, and is null once the kernel's code no longer matches
+    the digest recorded with the capture; edits to comments and layout keep it."""
     import bench
     src = tmp_path / "kernel.cu"
-    src.write_bytes(b"the kernel as captured\n")
-    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    src.write_bytes(b'int k(int a) { return a + 1; }  // as captured\nconst char* s = "x//y";\n')
+    digest = bench.code_digest(src.read_bytes())
     (tmp_path / "profiles").mkdir()
     (tmp_path / "profiles" / "gemm.md").write_text(
-        "# capture\n\n    traffic-ratio gate_up decode_t4 1.25 kernel.cu %s\n" % sha)
+        "# capture\n\n    traffic-ratio gate_up decode_t4 1.25 kernel.cu %s\n" % digest)
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.ncu_traffic("gate_up", "decode_t4", 1000.0) == 1250.0
     assert bench.ncu_traffic("gate_up", "decode_t128", 1000.0) is None  # no capture
-    src.write_bytes(b"the kernel, changed since\n")
+    # comments reworded, a block comment added, lines re-indented: same code, same digest
+    src.write_bytes(b'/* kernel */\nint k(int a) {\n    return a + 1;  // reworded\n}\n'
+                    b'const char* s = "x//y";\n')
+    assert bench.ncu_traffic("gate_up", "decode_t4", 1000.0) == 1250.0
+    # a change inside a string literal is a change of the code
+    src.write_bytes(b'int k(int a) { return a + 1; }\nconst char* s = "x/y";\n')
+    assert bench.ncu_traffic("gate_up", "decode_t4", 1000.0) is None
+    src.write_bytes(b'int k(int a) { return a + 2; }\nconst char* s = "x//y";\n')
     assert bench.ncu_traffic("gate_up", "decode_t4", 1000.0) is None
