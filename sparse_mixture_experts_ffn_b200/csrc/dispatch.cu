@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScheduleArgs sa, int k, int 
                                                     int32_t* __restrict__ counts_user) {
   __shared__ int cnt[2048];
   __shared__ int order[2048];
-  __shared__ int warp_tot[33];
+  __shared__ unsigned long long warp_tot[33];
   __shared__ ScheduleSmem ss;
   pdl_wait();
   pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
@@ -200,6 +200,7 @@ __global__ void gather_rows_kernel(const T* __restrict__ x, const int32_t* __res
     for (; v < vpr; v += 32) dst[v] = __ldg(src + v);
   }
 }
+
 
 // assignments up to which the single-block path is used
 constexpr int64_t kSmallDispatch = 4096;

@@ -1,6 +1,6 @@
 // dispatch_common.cuh -- the device code of the dispatch step shared by the dispatch
-// kernels and the fused small-batch routing kernel: block scans, the tile schedule of the
-// grouped expert GEMMs and the stable placement of the assignments.
+// kernels: block scans, the tile schedule of the grouped expert GEMMs and the stable
+// placement of the assignments.
 //
 // Definitions (the routing of llm-atlas page "Step-3.5-Flash", "Champs bruts du
 // config.json": moe_num_experts, moe_top_k): counts[e] = #{(t,j): idx[t,j] = e};
@@ -16,31 +16,33 @@
 namespace moe {
 
 // exclusive scan of up to 2 * blockDim.x values held two per thread (blockDim.x a multiple
-// of 32, at most 1024)
-static __device__ int block_scan_pair(int v0, int v1, int* warp_tot, int& total) {
+// of 32, at most 1024); V = unsigned long long scans two 32-bit counts packed in one value
+// (high and low halves) at once, as long as the low half's total stays below 2^32
+template <typename V>
+static __device__ V block_scan_pair(V v0, V v1, V* warp_tot, V& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int v = v0 + v1;
-  int incl = v;
+  const V v = v0 + v1;
+  V incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    const V y = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += y;
   }
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const int s = (lane < static_cast<int>(blockDim.x >> 5)) ? warp_tot[lane] : 0;  // fewer warps: zeros
-    int si = s;
+    const V s = (lane < static_cast<int>(blockDim.x >> 5)) ? warp_tot[lane] : V(0);  // fewer warps: zeros
+    V si = s;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, si, o);
+      const V y = __shfl_up_sync(0xffffffffu, si, o);
       if (lane >= o) si += y;
     }
     warp_tot[lane] = si - s;
     if (lane == 31) warp_tot[32] = si;
   }
   __syncthreads();
-  const int excl = warp_tot[warp] + incl - v;
+  const V excl = warp_tot[warp] + incl - v;
   total = warp_tot[32];
   __syncthreads();
   return excl;  // exclusive prefix of v0; v1's is excl + v0
@@ -74,21 +76,32 @@ static_assert(sizeof(int) * 2 * 2049 >= sizeof(unsigned long long) * 2048, "room
 // From the group sizes cnt[0..G) (routed experts, then the shared expert with all T
 // tokens): offsets of the routed experts, the largest-first group order and the tile
 // prefix sums of both grouped GEMMs (gate/up tiles counted ksplit times, once per slice
-// of the reduction).  One block with 2 * blockDim.x >= G + 1; cnt/order in shared memory,
-// and the offsets and prefixes also kept in ss for write_item_tables.
-static __device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* order, int* warp_tot,
-                                      ScheduleSmem& ss) {
+// of the reduction).  One block with 2 * blockDim.x >= G + 1 and blockDim.x / 64 a power
+// of two; cnt/order in shared memory, and the offsets and prefixes also kept in ss for the
+// descriptor writers.  Returns the number of groups with rows (they lead the order).
+static __device__ int build_schedule(const ScheduleArgs& a, int* cnt, int* order, unsigned long long* warp_tot,
+                                     ScheduleSmem& ss) {
+  using u64 = unsigned long long;
   const int E = a.E, G = E + (a.has_shared ? 1 : 0);
+  const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
+  // one scan for the routed offsets (low halves: the counts, whose total T*k < 2^31) and the
+  // places of the groups with rows (high halves: 1 per such group)
+  const int z0 = (i0 < G && cnt[i0] > 0) ? 1 : 0, z1 = (i1 < G && cnt[i1] > 0) ? 1 : 0;
+  int nz_ex, nnz;
   {
-    const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
-    const int v0 = i0 < E ? cnt[i0] : 0, v1 = i1 < E ? cnt[i1] : 0;
-    int total;
-    const int ex = block_scan_pair(v0, v1, warp_tot, total);
+    const u64 v0 = (static_cast<u64>(z0) << 32) | static_cast<uint32_t>(i0 < E ? cnt[i0] : 0);
+    const u64 v1 = (static_cast<u64>(z1) << 32) | static_cast<uint32_t>(i1 < E ? cnt[i1] : 0);
+    u64 tot;
+    const u64 ex64 = block_scan_pair(v0, v1, warp_tot, tot);
+    const int ex = static_cast<int>(ex64 & 0xFFFFFFFFu), total = static_cast<int>(tot & 0xFFFFFFFFu);
+    nz_ex = static_cast<int>(ex64 >> 32);
+    nnz = static_cast<int>(tot >> 32);
+    const int c0 = static_cast<int>(v0 & 0xFFFFFFFFu);
     if (i0 < E) a.offsets[i0] = ss.off[i0] = ex;
-    if (i1 < E) a.offsets[i1] = ss.off[i1] = ex + v0;
+    if (i1 < E) a.offsets[i1] = ss.off[i1] = ex + c0;
     if (a.offsets_user) {
       if (i0 < E) a.offsets_user[i0] = ex;
-      if (i1 < E) a.offsets_user[i1] = ex + v0;
+      if (i1 < E) a.offsets_user[i1] = ex + c0;
     }
     if (threadIdx.x == 0) {
       a.offsets[E] = ss.off[E] = total;
@@ -96,66 +109,62 @@ static __device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* orde
     }
   }
   // largest group first: order by (count desc, index asc), groups without rows last in
-  // index order.  The groups with rows are first compacted (in index order) into the leading
-  // places of order[], the others after them.  Few groups with rows (small batches): each
-  // is ranked by a count over the others; many: one ascending bitonic sort of the keys
-  // (~count << 32 | index) over the next power of two >= G, padded with keys above every
-  // real one, two keys a thread.
-  {
-    const int i0 = 2 * threadIdx.x, i1 = i0 + 1;
-    const int z0 = (i0 < G && cnt[i0] > 0) ? 1 : 0, z1 = (i1 < G && cnt[i1] > 0) ? 1 : 0;
-    int nnz;
-    const int nz_ex = block_scan_pair(z0, z1, warp_tot, nnz);
-    if (nnz <= 64) {
-      if (i0 < G) order[z0 ? nz_ex : nnz + (i0 - nz_ex)] = i0;
-      if (i1 < G) order[z1 ? nz_ex + z0 : nnz + (i1 - nz_ex - z0)] = i1;
-      __syncthreads();
-      auto rank_of = [&](int g) {
-        const int c = cnt[g];
-        int r = 0;
-        for (int j = 0; j < nnz; ++j) {
-          const int h = order[j];
-          const int ch = cnt[h];
-          r += (ch > c) || (ch == c && h < g);
-        }
-        return r;
-      };
-      const int r0 = z0 ? rank_of(i0) : -1, r1 = z1 ? rank_of(i1) : -1;
-      __syncthreads();
-      if (r0 >= 0) order[r0] = i0;
-      if (r1 >= 0) order[r1] = i1;
-      __syncthreads();
-    } else {
-      // [n <= 2048] keys in the prefix arrays, which are written only after the sort
-      unsigned long long* key = reinterpret_cast<unsigned long long*>(ss.istart_gu);
-      int n = 1;
-      while (n < G) n <<= 1;
-      for (int i = threadIdx.x; i < n; i += blockDim.x)
-        key[i] = i < G ? (static_cast<unsigned long long>(~static_cast<uint32_t>(cnt[i])) << 32) |
-                             static_cast<uint32_t>(i)
-                       : ~0ull;
-      __syncthreads();
-      for (int size = 2; size <= n; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-          for (int t = threadIdx.x; t < (n >> 1); t += blockDim.x) {
-            // pair (i, i + stride) of the stride-sized half blocks; ascending where i & size is 0
-            const int i = 2 * t - (t & (stride - 1));
-            const unsigned long long x = key[i], y = key[i + stride];
-            const bool up = (i & size) == 0;
-            if ((x > y) == up) {
-              key[i] = y;
-              key[i + stride] = x;
-            }
-          }
-          __syncthreads();
-        }
+  // index order.  Keys ~count << 32 | index rank the groups with rows.  Few of them (small
+  // batches): compacted into a list of at most 64 keys, each ranked by blockDim.x / 64
+  // threads that compare it with 64 / (blockDim.x / 64) keys each and add their counts; many:
+  // one ascending bitonic sort of every group's key over the next power of two >= G, padded
+  // with keys above every real one.
+  auto key_of = [&](int g) -> u64 {
+    return (static_cast<u64>(~static_cast<uint32_t>(cnt[g])) << 32) | static_cast<uint32_t>(g);
+  };
+  if (nnz <= 64) {
+    u64* ckey = reinterpret_cast<u64*>(ss.istart_gu);  // written only after the ranking
+    if (z0) ckey[nz_ex] = key_of(i0);
+    if (z1) ckey[nz_ex + z0] = key_of(i1);
+    if (i0 < G && !z0) order[nnz + (i0 - nz_ex)] = i0;
+    if (i1 < G && !z1) order[nnz + (i1 - nz_ex - z0)] = i1;
+    __syncthreads();
+    const int parts = static_cast<int>(blockDim.x >> 6), per = 64 / parts;
+    const int slot = static_cast<int>(threadIdx.x) / parts, part = static_cast<int>(threadIdx.x) - slot * parts;
+    int r = 0;
+    u64 kg = 0;
+    if (slot < nnz) {
+      kg = ckey[slot];
+      for (int q = 0; q < per; ++q) {
+        const int h = part * per + q;
+        r += (h < nnz && ckey[h] < kg) ? 1 : 0;
       }
-      for (int i = threadIdx.x; i < G; i += blockDim.x) order[i] = static_cast<int>(key[i] & 0xFFFFFFFFu);
-      __syncthreads();
     }
+    for (int o = parts >> 1; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+    if (slot < nnz && part == 0) order[r] = static_cast<int>(kg & 0xFFFFFFFFu);
+    __syncthreads();
+  } else {
+    // [n <= 2048] keys in the prefix arrays, which are written only after the sort
+    u64* key = reinterpret_cast<u64*>(ss.istart_gu);
+    int n = 1;
+    while (n < G) n <<= 1;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) key[i] = i < G ? key_of(i) : ~0ull;
+    __syncthreads();
+    for (int size = 2; size <= n; size <<= 1) {
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        for (int t = threadIdx.x; t < (n >> 1); t += blockDim.x) {
+          // pair (i, i + stride) of the stride-sized half blocks; ascending where i & size is 0
+          const int i = 2 * t - (t & (stride - 1));
+          const u64 x = key[i], y = key[i + stride];
+          const bool up = (i & size) == 0;
+          if ((x > y) == up) {
+            key[i] = y;
+            key[i + stride] = x;
+          }
+        }
+        __syncthreads();
+      }
+    }
+    for (int i = threadIdx.x; i < G; i += blockDim.x) order[i] = static_cast<int>(key[i] & 0xFFFFFFFFu);
+    __syncthreads();
   }
   for (int r = threadIdx.x; r < G; r += blockDim.x) a.group_order[r] = order[r];
-  const int r0 = 2 * threadIdx.x, r1 = r0 + 1;
+  // tiles of group slot r in each GEMM; one scan for both (gate/up high, down low halves)
   auto tiles = [&](int r, bool gu) -> int {
     if (r >= G) return 0;
     const int g = order[r];
@@ -165,18 +174,27 @@ static __device__ void build_schedule(const ScheduleArgs& a, int* cnt, int* orde
     const int mt = gu ? (g < E ? a.mt_gu : a.mt_gu_shared) * a.ksplit : a.mt_dn;
     return nt * mt;
   };
-  int total;
-  int a0 = tiles(r0, true), a1 = tiles(r1, true);
-  int ex = block_scan_pair(a0, a1, warp_tot, total);
-  if (r0 < G) a.item_start_gu[r0] = ss.istart_gu[r0] = ex;
-  if (r1 < G) a.item_start_gu[r1] = ss.istart_gu[r1] = ex + a0;
-  if (threadIdx.x == 0) a.item_start_gu[G] = ss.istart_gu[G] = total;
-  a0 = tiles(r0, false);
-  a1 = tiles(r1, false);
-  ex = block_scan_pair(a0, a1, warp_tot, total);
-  if (r0 < G) a.item_start_dn[r0] = ss.istart_dn[r0] = ex;
-  if (r1 < G) a.item_start_dn[r1] = ss.istart_dn[r1] = ex + a0;
-  if (threadIdx.x == 0) a.item_start_dn[G] = ss.istart_dn[G] = total;
+  const int r0 = i0, r1 = i1;
+  const int gu0 = tiles(r0, true), gu1 = tiles(r1, true);
+  const u64 v0 = (static_cast<u64>(gu0) << 32) | static_cast<uint32_t>(tiles(r0, false));
+  const u64 v1 = (static_cast<u64>(gu1) << 32) | static_cast<uint32_t>(tiles(r1, false));
+  u64 tot;
+  const u64 ex64 = block_scan_pair(v0, v1, warp_tot, tot);
+  const int ex_gu = static_cast<int>(ex64 >> 32), ex_dn = static_cast<int>(ex64 & 0xFFFFFFFFu);
+  const int dn0 = static_cast<int>(v0 & 0xFFFFFFFFu);
+  if (r0 < G) {
+    a.item_start_gu[r0] = ss.istart_gu[r0] = ex_gu;
+    a.item_start_dn[r0] = ss.istart_dn[r0] = ex_dn;
+  }
+  if (r1 < G) {
+    a.item_start_gu[r1] = ss.istart_gu[r1] = ex_gu + gu0;
+    a.item_start_dn[r1] = ss.istart_dn[r1] = ex_dn + dn0;
+  }
+  if (threadIdx.x == 0) {
+    a.item_start_gu[G] = ss.istart_gu[G] = static_cast<int>(tot >> 32);
+    a.item_start_dn[G] = ss.istart_dn[G] = static_cast<int>(tot & 0xFFFFFFFFu);
+  }
+  return nnz;
 }
 
 // One descriptor per tile of a grouped GEMM, so that a GEMM role finds its tile with one
@@ -220,6 +238,40 @@ static __device__ void write_item_tables(const ScheduleArgs& a, const int* cnt, 
       const int m = tile / ntile, n = tile - m * ntile;
       const int row0 = (g < E ? off[g] : 0) + n * bn;
       info[it] = make_int4(g, m, row0, min(bn, rows - n * bn) | (ks << 16));
+    }
+  }
+}
+
+// The same descriptors written by one block, a warp per (GEMM, group slot) with its lanes
+// over the slot's items: no search.  Only the first nslots slots of the order have items
+// (the groups with rows).
+static __device__ void write_item_tables_by_slot(const ScheduleArgs& a, const int* cnt, const int* order,
+                                                 const int* off, const int* istart_gu, const int* istart_dn,
+                                                 int nslots) {
+  const int E = a.E, G = E + (a.has_shared ? 1 : 0);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = static_cast<int>(blockDim.x >> 5);
+  const bool ok_gu = istart_gu[G] <= a.cap_gu, ok_dn = istart_dn[G] <= a.cap_dn;
+  if ((!ok_gu || !ok_dn) && threadIdx.x == 0) set_status(a.ctrl, MOE_ERR_DEVICE_BOUNDS);  // the GEMM runs nothing
+  for (int job = warp; job < 2 * nslots; job += nwarps) {
+    const int which = job >= nslots ? 1 : 0, r = job - which * nslots;
+    if (!(which ? ok_dn : ok_gu)) continue;
+    const int* istart = which ? istart_dn : istart_gu;
+    int4* info = which ? a.info_dn : a.info_gu;
+    const int bn = which ? a.bn_dn : a.bn;
+    const int ks_n = which ? 1 : a.ksplit;
+    const int i0 = istart[r], n_items = istart[r + 1] - i0;
+    if (n_items <= 0) continue;
+    const int g = order[r], rows = cnt[g];
+    const int ntile = (rows + bn - 1) / bn;
+    const int rbase = g < E ? off[g] : 0;
+    for (int l = lane; l < n_items; l += 32) {
+      if (ntile < 1) {  // inconsistent prefixes: an invalid descriptor, reported by the GEMM
+        info[i0 + l] = make_int4(-1, 0, 0, 0);
+        continue;
+      }
+      const int tile = l / ks_n, ks = l - tile * ks_n;
+      const int m = tile / ntile, n = tile - m * ntile;
+      info[i0 + l] = make_int4(g, m, rbase + n * bn, min(bn, rows - n * bn) | (ks << 16));
     }
   }
 }
@@ -272,7 +324,7 @@ struct SmallDispatchSmem {
   int cnt[2048];
   int order[2048];
   int base[1024];
-  int warp_tot[33];
+  unsigned long long warp_tot[33];
   ScheduleSmem sched;
 };
 
@@ -303,10 +355,14 @@ static __device__ void dispatch_small_block(const ScheduleArgs& sa, const int32_
   }
   if (sa.has_shared && threadIdx.x == 0) sm.cnt[E] = sa.shared_rows;
   __syncthreads();
-  build_schedule(sa, sm.cnt, sm.order, sm.warp_tot, sm.sched);
+  const int nnz = build_schedule(sa, sm.cnt, sm.order, sm.warp_tot, sm.sched);
   __syncthreads();
-  write_item_tables(sa, sm.cnt, sm.order, sm.sched.off, sm.sched.istart_gu, sm.sched.istart_dn, threadIdx.x,
-                    blockDim.x);
+  // few groups with rows: a warp per group slot; many: items spread evenly over the threads
+  if (nnz <= 64)
+    write_item_tables_by_slot(sa, sm.cnt, sm.order, sm.sched.off, sm.sched.istart_gu, sm.sched.istart_dn, nnz);
+  else
+    write_item_tables(sa, sm.cnt, sm.order, sm.sched.off, sm.sched.istart_gu, sm.sched.istart_dn, threadIdx.x,
+                      blockDim.x);
   for (int e = threadIdx.x; e < E; e += blockDim.x) sm.base[e] = sm.sched.off[e];
   __syncthreads();
   if (threadIdx.x < 32)

@@ -159,8 +159,7 @@ struct Item {
 // Tile `it` of the schedule from its descriptor (written by the dispatch step), checked
 // against this launch's bounds: an inconsistent descriptor is reported and skipped.
 template <int BN>
-__device__ __forceinline__ Item decode_item(const TcParams& p, int it) {
-  const int4 d = __ldg(p.item_info + it);
+__device__ __forceinline__ Item decode_item_info(const TcParams& p, const int4 d, int it) {
   Item r;
   r.g = d.x;
   r.sh = (r.g == p.E) ? 1 : 0;
@@ -178,6 +177,10 @@ __device__ __forceinline__ Item decode_item(const TcParams& p, int it) {
     r.sh = 0;
   }
   return r;
+}
+template <int BN>
+__device__ __forceinline__ Item decode_item(const TcParams& p, int it) {
+  return decode_item_info<BN>(p, __ldg(p.item_info + it), it);
 }
 
 // The shape of a valid tile as a number 1..32 for the MMA warp: (shared expert) * 16 +
@@ -351,6 +354,10 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();
   pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
+  // the producer requests its first item's descriptor (item blockIdx.x, within the table's
+  // capacity) together with the schedule length, so that both arrive in one round trip
+  int4 first_info = make_int4(-1, 0, 0, 0);
+  if (warp == 0 && static_cast<int>(blockIdx.x) < p.max_items) first_info = __ldg(p.item_info + blockIdx.x);
   const int total = schedule_length(p);
   // FP8: waiting threads sleep in their polls, leaving the issue slots to the converters
   auto wait = [&](uint64_t* bar, uint32_t parity) {
@@ -387,8 +394,10 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
     };
     int pf_it = -1;  // FP8: the item whose scales pf_sg / pf_su hold
     uint32_t pf_sg[2] = {0u, 0u}, pf_su[2] = {0u, 0u};
-    // the item after the current one is claimed while the current one streams
+    // the item after the current one is claimed, and its descriptor loaded, while the
+    // current one streams
     int it = static_cast<int>(blockIdx.x);
+    int4 info = first_info;  // descriptor of item `it`
     int claimed = (lane == 0) ? static_cast<int>(atomicAdd(p.item_counter, 1u) + gridDim.x) : 0;
     for (;;) {
       if (it >= total || !ok) it = -1;
@@ -405,9 +414,10 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
       if (++q == kRing) { q = 0; qphase ^= 1u; }
       if (!pub || it < 0) break;
       const int cur = it;
+      const Item t = decode_item_info<BN>(p, info, cur);
       it = __shfl_sync(0xffffffffu, claimed, 0);
       if (lane == 0 && it < total) claimed = static_cast<int>(atomicAdd(p.item_counter, 1u) + gridDim.x);
-      const Item t = decode_item<BN>(p, cur);
+      if (it < total) info = __ldg(p.item_info + it);
       if (!t.valid) {
         if (blockIdx.x == 0 && lane == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
         continue;

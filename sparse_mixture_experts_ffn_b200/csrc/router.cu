@@ -992,7 +992,7 @@ constexpr int kRtBBytes = kRtExperts * kTileK * 2;   // 8 KB of W_router
 constexpr int kRtStageBytes = kRtABytes + kRtBBytes;
 constexpr int kRtSmem = kRtStages * kRtStageBytes + 1024 + 256;
 constexpr int kRtRowBox = 16;                        // token rows per TMA box
-constexpr int kRtMaxChunks = 16;
+constexpr int kRtMaxChunks = 16;                      // a tile's last block adds them in one pass
 constexpr int kRtSmTarget = 148;                     // blocks that fill the GPU
 
 struct RouterTcParams {
@@ -1217,38 +1217,12 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
             if (j < ne) dst[j] = __uint_as_float(r[j]);
         }
       }
-      // the last block of this (m, n) tile adds the partials of every chunk
+      // the last block of this (m, n) tile adds the partials of every chunk (below)
       __threadfence();
       named_bar_sync(1, 128);
       if (warp == 2 && lane == 0) {
         const unsigned int done = atomicAdd(p.tile_done + blockIdx.x, 1u);
         *last_flag = (done == static_cast<unsigned int>(p.chunks - 1)) ? 1 : 0;
-      }
-      named_bar_sync(1, 128);
-      if (*last_flag) {
-        __threadfence();
-        const int et = threadIdx.x - 64;
-        for (int i = et; i < rows * ne; i += 128) {
-          const int tt = i / ne, j = i - tt * ne;
-          const float* src = p.part + (t0 + tt) * p.E + e0 + j;
-          const int64_t sstride = p.T * p.E;
-          double acc = 0.0;
-#pragma unroll 16
-          for (int sl = 0; sl < n_sl_all; ++sl) acc += static_cast<double>(__ldcg(src + sl * sstride));
-          p.scores[(t0 + tt) * p.E + e0 + j] = acc;
-        }
-        if (ni == 0)
-          for (int i = et; i < rows; i += 128) {
-            double ss = 0.0;
-            for (int z = 0; z < p.chunks; ++z) ss += __ldcg(p.xss + z * p.T + t0 + i);
-            p.xnorm[t0 + i] = norm_ub_from_sumsq(ss, p.Hx);
-          }
-        if (mi == 0 && !p.w_given)
-          for (int i = et; i < ne; i += 128) {
-            double ss = 0.0;
-            for (int z = 0; z < p.chunks; ++z) ss += __ldcg(p.wss + static_cast<int64_t>(z) * p.E + e0 + i);
-            p.wnorm[e0 + i] = norm_ub_from_sumsq(ss, p.H);
-          }
       }
     }
   }
@@ -1256,6 +1230,62 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem_base, kCols);
+  if (!split || !*last_flag) return;
+  // Last block of the tile: the scores (each the fp64 sum of its slices' fp32 partials, in
+  // slice order: the unsplit kernel's result bit for bit) and the norm bounds (fp64 sums of
+  // the chunks' sums of squares, in chunk order), by all six warps.  Every load of a thread
+  // is issued before the first of its values is used: first the sums of squares of the norm
+  // bound it owns (threads from the last one down), then two scores at a time.
+  __threadfence();
+  const int np = rows * ne, nxj = (ni == 0) ? rows : 0, nwj = (mi == 0 && !p.w_given) ? ne : 0;
+  const int nthr = static_cast<int>(blockDim.x);
+  const int jn = nthr - 1 - static_cast<int>(threadIdx.x);  // this thread's norm bound, if < nxj + nwj
+  const bool has_norm = jn < nxj + nwj;  // every bound has its thread: rows + ne <= 32 + 64 < 192
+  const bool norm_x = jn < nxj;
+  double nv[16];
+  {
+    const double* src = norm_x ? p.xss + t0 + jn : p.wss + e0 + (jn - nxj);
+    const int64_t nst = norm_x ? p.T : static_cast<int64_t>(p.E);
+#pragma unroll
+    for (int z = 0; z < 16; ++z) nv[z] = (has_norm && z < p.chunks) ? __ldcg(src + z * nst) : 0.0;
+  }
+  const int64_t sstride = p.T * p.E;
+  for (int j0 = threadIdx.x; j0 < np; j0 += 2 * nthr) {
+    const int j1 = j0 + nthr;
+    const bool h1 = j1 < np;
+    const int ta = j0 / ne, ea = j0 - ta * ne;
+    const int tb = h1 ? j1 / ne : ta, eb = h1 ? j1 - tb * ne : ea;
+    const float* pa = p.part + (t0 + ta) * p.E + e0 + ea;
+    const float* pb = p.part + (t0 + tb) * p.E + e0 + eb;
+    double acc_a = 0.0, acc_b = 0.0;
+    for (int b = 0; b < n_sl_all; b += 16) {
+      float va[16], vb[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const bool in = b + q < n_sl_all;
+        va[q] = in ? __ldcg(pa + (b + q) * sstride) : 0.0f;
+        vb[q] = in ? __ldcg(pb + (b + q) * sstride) : 0.0f;
+      }
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (b + q < n_sl_all) {
+          acc_a += static_cast<double>(va[q]);
+          acc_b += static_cast<double>(vb[q]);
+        }
+    }
+    p.scores[(t0 + ta) * p.E + e0 + ea] = acc_a;
+    if (h1) p.scores[(t0 + tb) * p.E + e0 + eb] = acc_b;
+  }
+  if (has_norm) {
+    double ss = 0.0;
+#pragma unroll
+    for (int z = 0; z < 16; ++z)
+      if (z < p.chunks) ss += nv[z];
+    if (norm_x)
+      p.xnorm[t0 + jn] = norm_ub_from_sumsq(ss, p.Hx);
+    else
+      p.wnorm[e0 + jn - nxj] = norm_ub_from_sumsq(ss, p.H);
+  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1299,6 +1329,7 @@ int router_slice_len(int /*H*/) { return kRtSliceSteps * kTileK; }
 // batch is too large for one block per tile to add the partials quickly, else the fewest
 // (at most 16, at least one slice each) that bring the blocks to one per SM.
 constexpr int64_t kRtSplitMaxTokens = 32;
+static_assert(kRtSplitMaxTokens + kRtExperts <= 192, "one thread per norm bound in a tile's last block");
 static int router_chunks(int64_t T, int E, int H) {
   if (T > kRtSplitMaxTokens) return 1;
   const int64_t tiles = ((T + kTileM - 1) / kTileM) * ((E + kRtExperts - 1) / kRtExperts);
@@ -1391,6 +1422,28 @@ __global__ void __launch_bounds__(256) split_w32_kernel(const float* __restrict_
   }
 }
 
+// The selection of the tensor-core scores: one warp per token.
+template <typename TW, int EPL, bool SIG>
+static cudaError_t launch_select(const RouterArgs& a, const TW* Wsel, double coef, int Kg, cudaStream_t st) {
+  using bf16 = __nv_bfloat16;
+  const double delta_abs = Kg * 2.350988701644575e-38;
+  const bf16* x = static_cast<const bf16*>(a.x);
+  const Keys kf{a.bias, a.sigmoid, a.scale};
+  const unsigned sgrid = static_cast<unsigned>((a.T + kSelectWarps - 1) / kSelectWarps);
+  return launch_pdl(route_select_kernel<bf16, TW, EPL, SIG>, dim3(sgrid), dim3(32 * kSelectWarps), 0, st,
+                    static_cast<const double*>(a.scores64), coef, delta_abs, static_cast<const double*>(a.xnorm),
+                    static_cast<const double*>(a.wnorm), kf, x, Wsel, a.T, a.H, a.E, a.k, a.idx_ws, a.w_ws,
+                    a.idx_user, a.w_user, a.spill, a.ctrl);
+}
+
+template <typename TW, bool SIG>
+static cudaError_t launch_select_epl(const RouterArgs& a, const TW* Wsel, double coef, int Kg, cudaStream_t st) {
+  const int epl = select_epl(a.E);
+  return epl == 4    ? launch_select<TW, 4, SIG>(a, Wsel, coef, Kg, st)
+         : epl == 12 ? launch_select<TW, 12, SIG>(a, Wsel, coef, Kg, st)
+                     : launch_select<TW, 32, SIG>(a, Wsel, coef, Kg, st);
+}
+
 static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
   using bf16 = __nv_bfloat16;
   RouterTcParams p{};
@@ -1452,31 +1505,13 @@ static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
                       static_cast<unsigned>(chunks)),
                  dim3(192), static_cast<size_t>(kRtSmem), st, p);
   if (e != cudaSuccess) return e;
-  const unsigned sgrid = static_cast<unsigned>((a.T + kSelectWarps - 1) / kSelectWarps);
-  auto sel = [&](auto kern, auto* Wsel) {
-    return launch_pdl(kern, dim3(sgrid), dim3(32 * kSelectWarps), 0, st, static_cast<const double*>(a.scores64),
-                      coef, Kg * 2.350988701644575e-38, static_cast<const double*>(a.xnorm),
-                      static_cast<const double*>(a.wnorm), Keys{a.bias, a.sigmoid, a.scale}, x, Wsel, a.T, a.H,
-                      a.E, a.k, a.idx_ws,
-                      a.w_ws, a.idx_user, a.w_user, a.spill, a.ctrl);
-  };
-  const int epl = select_epl(a.E);
-  const bf16* Wb = static_cast<const bf16*>(a.Wr);
   const float* Wf = static_cast<const float*>(a.Wr);
-  if (a.w32) {  // the recomputations read the fp32 weights themselves
-    if (a.sigmoid)
-      e = epl == 4 ? sel(route_select_kernel<bf16, float, 4, true>, Wf)
-          : epl == 12 ? sel(route_select_kernel<bf16, float, 12, true>, Wf) : sel(route_select_kernel<bf16, float, 32, true>, Wf);
-    else
-      e = epl == 4 ? sel(route_select_kernel<bf16, float, 4, false>, Wf)
-          : epl == 12 ? sel(route_select_kernel<bf16, float, 12, false>, Wf) : sel(route_select_kernel<bf16, float, 32, false>, Wf);
-  } else if (a.sigmoid) {
-    e = epl == 4 ? sel(route_select_kernel<bf16, bf16, 4, true>, Wb)
-        : epl == 12 ? sel(route_select_kernel<bf16, bf16, 12, true>, Wb) : sel(route_select_kernel<bf16, bf16, 32, true>, Wb);
-  } else {
-    e = epl == 4 ? sel(route_select_kernel<bf16, bf16, 4, false>, Wb)
-        : epl == 12 ? sel(route_select_kernel<bf16, bf16, 12, false>, Wb) : sel(route_select_kernel<bf16, bf16, 32, false>, Wb);
-  }
+  if (a.w32)  // the recomputations read the fp32 weights themselves
+    e = a.sigmoid ? launch_select_epl<float, true>(a, Wf, coef, Kg, st)
+                  : launch_select_epl<float, false>(a, Wf, coef, Kg, st);
+  else
+    e = a.sigmoid ? launch_select_epl<bf16, true>(a, static_cast<const bf16*>(a.Wr), coef, Kg, st)
+                  : launch_select_epl<bf16, false>(a, static_cast<const bf16*>(a.Wr), coef, Kg, st);
   count_launches(launches);
   return e;
 }
