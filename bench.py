@@ -383,27 +383,44 @@ def cpu_baseline(h, cfg, opts=None, budget_s=8.0):
 BF16_WORKLOADS = ("decode_t4", "decode_t128", "prefill_t4096", "prefill_t16384_skew")
 
 
-def roofline(alg, peaks, gu_ms, fp8, workload):
-    """Roofline of the dominant kernel, the gate/up GEMM: its algorithmic bytes or FLOPs per
-    launch over its average launch time, against the measured copy bandwidth when the
-    launch is HBM-bound and the sustained bf16 tensor peak when it is tensor-bound."""
+def gemms_in_one_launch(cfg, fp8: bool) -> bool:
+    """Whether the library runs both expert GEMMs as one launch on this workload: bf16
+    weights with 16-token tiles, which it takes when experts hold at most six assignments
+    on average (T * top_k <= 6 E).  The gate/up stage then times both GEMMs and the down
+    stage is empty."""
+    return not fp8 and cfg.T * cfg.top_k <= 6 * cfg.E
+
+
+def roofline(alg, peaks, gu_ms, fp8, workload, fused=False):
+    """Roofline of the dominant kernel, the gate/up GEMM (with 16-token tiles: the one launch
+    of both GEMMs): its algorithmic bytes or FLOPs per launch over its average launch time,
+    against the measured copy bandwidth when the launch is HBM-bound and the sustained bf16
+    tensor peak when it is tensor-bound."""
     tc_peak = peaks["bf16_tflops_sustained"]
-    tensor_bound = alg["gate_up_flops"] / (tc_peak * 1e12) > alg["gate_up_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    nbytes = alg["gate_up_bytes"] + (alg["down_bytes"] if fused else 0)
+    nflops = alg["gate_up_flops"] + (alg["down_flops"] if fused else 0)
+    tensor_bound = nflops / (tc_peak * 1e12) > nbytes / (peaks["hbm_gbs"] * 1e9)
     if tensor_bound:
-        achieved = alg["gate_up_flops"] / (gu_ms / 1e3) / 1e12
+        achieved = nflops / (gu_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": achieved / tc_peak, "peak_kind": "sustained bf16 (cuBLAS, seconds-long loop)",
                 "frac_of_burst": achieved / peaks["bf16_tflops"]}
     else:
-        achieved = alg["gate_up_bytes"] / (gu_ms / 1e3) / 1e9
+        achieved = nbytes / (gu_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
-    roof.update({"kernel": "expert_gemm_tc_kernel<gated%s> (gate/up GEMM + SiLU*up)" % (", fp8" if fp8 else ""),
+    if fused:
+        kernel = "expert_gemm_tc_kernel<gated, 16 tokens, both GEMMs> (gate/up + SiLU*up, then down)"
+        key = "gemm_fused"
+    else:
+        kernel = "expert_gemm_tc_kernel<gated%s> (gate/up GEMM + SiLU*up)" % (", fp8" if fp8 else "")
+        key = "gate_up"
+    roof.update({"kernel": kernel,
                  "timing": "CUDA events around each launch, stage-timed pass of the same steps",
-                 "traffic": ncu_traffic("gate_up", workload + ("+fp8" if fp8 else ""), alg["gate_up_bytes"]),
+                 "traffic": ncu_traffic(key, workload + ("+fp8" if fp8 else ""), nbytes),
                  "peak_source": peaks["source"],
-                 "ms_per_launch": gu_ms, "algorithmic_bytes": alg["gate_up_bytes"],
-                 "algorithmic_flops": alg["gate_up_flops"]})
+                 "ms_per_launch": gu_ms, "algorithmic_bytes": nbytes,
+                 "algorithmic_flops": nflops})
     return roof
 
 
@@ -538,7 +555,7 @@ def measure(cfg, args, dev, pg, world, rank, local, clocks):
             "workload": cfg.name, "T": cfg.T, "steps": steps, "ms_per_step": ms_per_step,
             "value": job_tokens_per_s(cfg.T, world, steps, elapsed_ms), "unit": UNIT,
             "ms_per_step_stage_timed": elapsed_prof_ms / steps,
-            "roofline": roofline(alg, peaks, gu_ms, fp8, cfg.name),
+            "roofline": roofline(alg, peaks, gu_ms, fp8, cfg.name, gemms_in_one_launch(cfg, fp8)),
             "layer": dict(layer_roofline(alg, peaks, ms_per_step),
                           stage_ms_per_step={k: v / max(calls, 1) for k, v in stage_ms.items()},
                           route_stats=route_stats, device_status=moe.status_string(status)),

@@ -96,7 +96,7 @@ static int num_sms_current_device() {
 static size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
-  size_t ctrl, group_done, tile_done, item_counters, wss, zero_end, scores, xnorm, wnorm, idx, w, blk_hist, counts,
+  size_t ctrl, group_done, tile_done, item_counters, gu_done, wss, zero_end, scores, xnorm, wnorm, idx, w, blk_hist, counts,
       offsets, group_order, item_start_gu, item_start_dn, info_gu, info_dn, perm, inv_perm, row_w, row_tok, partial, spill, rsplit, w3,
       x_perm, h, h_shared, o, o_shared, total;
   int bn, bn_dn, ksplit;
@@ -128,6 +128,7 @@ static bool make_layout(const moe_layer_shape* s, Layout& L) {
   L.group_done = take(groups * 4);
   L.tile_done = take(L.ksplit > 1 ? static_cast<size_t>(L.max_tiles) * 4 : 0);
   L.item_counters = take(2 * 4);
+  L.gu_done = take((E + 1) * 4);  // gate/up tiles finished per group (one launch for both GEMMs)
   // the small-batch router accumulates scores and row sums of squares atomically
   L.wss = take(tc_scores ? 0 : groups * E * 8);
   L.scores = take(T * E * 8);
@@ -424,6 +425,8 @@ static moe_status forward_impl(const moe_layer_shape* shape, const void* x, cons
   ea.swiglu_limit = opt.swiglu_limit;
   ea.swiglu_limit_shared = opt.swiglu_limit_shared;
   ea.item_counters = static_cast<unsigned int*>(at(L.item_counters));
+  ea.gu_done = static_cast<unsigned int*>(at(L.gu_done));
+  ea.counts = static_cast<const int32_t*>(at(L.counts));
   ea.h = at(L.h);
   ea.h_shared = at(L.h_shared);
   ea.o = at(L.o);

@@ -238,6 +238,18 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Orders this thread's global-memory accesses against those of the asynchronous proxy
+// (TMA copies): a writer's ordinary stores before a TMA load that reads them on another SM
+// (with a release / acquire pair between the two threads), on either side.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ unsigned int ld_acquire_gpu(const unsigned int* addr) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+  return v;
+}
+
 // Shared-memory matrix descriptor of a K-major operand tile stored the way TMA writes it
 // with 128-byte swizzling: rows of 64 bf16 (128 B), 8-row swizzle atoms 1024 B apart.
 //   bits  0-13 start address >> 4     bits 16-29 leading byte offset >> 4 (unused here)

@@ -71,6 +71,10 @@ struct TcParams {
   int pf_mt;                       // weight tiles per group of the down GEMM
   int64_t pf_rows_per_group;       // rows of one routed expert's down matrix (H)
   int64_t pf_row_bytes[2];         // bytes of one row: routed (I), shared (I_shared)
+  // both projections in one launch (16-token tiles): a down item of group g waits until
+  // every gate/up tile of g has written its h rows
+  unsigned int* gu_done;           // [G] gate/up tiles finished per group, zero before the launch
+  const int32_t* counts;           // [E] rows per routed expert (its gate/up token tiles)
   const uint8_t* scaleA[2];    // FP8 weights: E8M0 block scales of the A matrices, routed
                                // (stacked by expert) and shared
   int s_rows_per_group;        // FP8 weights: scale rows (128-row blocks) per routed expert
@@ -82,22 +86,25 @@ constexpr int kMaxDynSmem = 232448;  // 227 KB per block on sm_100
 constexpr int kConvGroups = 2;       // FP8: converter groups of four warps
 constexpr int kRing = 4;             // item slots between the producer and the other roles
 
-template <bool GATED, int BN, bool W8 = false>
+template <bool GATED, int BN, bool W8 = false, bool FUSED = false>
 struct TcCfg {
   static constexpr int kMats = GATED ? 2 : 1;           // weight tiles per stage (gate, up)
   // k-blocks (64 columns, one 128-byte swizzle atom wide) per stage.  bf16 16-token tiles
   // stream their weights from HBM: two adjacent k-blocks per stage, so that each weight row
   // is requested 256 contiguous bytes at a time rather than 128
   static constexpr int kKB = (BN == 16 && !W8) ? 2 : 1;
+  // both GEMMs in one launch: a down tile has no up rows, so it fills a stage's weight room
+  // with four k-blocks of its one matrix (and the token-row room holds four k-blocks too)
+  static constexpr int kDnKB = FUSED ? 2 * kKB : kKB;
   static constexpr int kAtomA = kTileM * kTileK * 2;   // one k-block of 128 weight rows (16 KB)
   static constexpr int kAtomB = BN * kTileK * 2;       // one k-block of the token rows
   static constexpr int kABytes = kKB * kAtomA;         // bf16 weights per operand tile and stage
   static constexpr int kA8Bytes = kTileM * kTileK;     // one k-block as FP8 codes
-  static constexpr int kBBytes = kKB * kAtomB;         // token rows
+  static constexpr int kBBytes = kDnKB * kAtomB;       // token rows
   // one TMA stage: the weight tiles as loaded (bf16, or FP8 codes), then the token rows
   static constexpr int kBOffset = kMats * (W8 ? kA8Bytes : kABytes);
   static constexpr int kStageBytes = kBOffset + kBBytes;
-  static constexpr int kKBytes = kStageBytes / kKB;     // bytes of one k-block of a stage
+  static constexpr int kKBytes = kMats * (W8 ? kA8Bytes : kAtomA) + kAtomB;  // bytes of one k-block
   // FP8: stages of converted bf16 weight tiles plus a copy of the token rows, between the
   // converters and the MMA.  The converters free each TMA stage as soon as they have read
   // it, so every TMA stage is either in flight or waiting for conversion.  More converted
@@ -143,6 +150,7 @@ struct TcCfg {
   static_assert(kTmemNeed <= 512, "accumulators exceed tensor memory");
   static_assert(kSmemBytes <= kMaxDynSmem, "shared memory budget");
   static_assert(BN % 16 == 0 && BN <= 256, "tile width");
+  static_assert(!FUSED || (GATED && kDnKB * kAtomA <= kBOffset), "a down stage fits the gate/up weight room");
 };
 
 struct Item {
@@ -266,6 +274,14 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
   }
 }
 
+// An epilogue thread's stores of h rows, ordered before the release of the group's count
+// (after a barrier of the four epilogue warps) and before the TMA loads that read them on
+// other SMs once the count is acquired.
+__device__ __forceinline__ void release_rows_stored() {
+  fence_proxy_async_global();
+  __threadfence();
+}
+
 // Persistent grouped GEMM, one block per SM.
 //   warp 0      TMA producer (one lane): weight tiles (gate and up for GATED) and token rows
 //   warp 1      allocates tensor memory; one lane issues the tcgen05 MMAs
@@ -292,9 +308,16 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-template <bool GATED, int BN, bool W8>
-__global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm_tc_kernel(const __grid_constant__ TcParams p) {
-  using C = TcCfg<GATED, BN, W8>;
+// FUSED (bf16 16-token tiles): one launch runs both projections.  p holds the gate/up
+// GEMM's parameters and pdn the down GEMM's; items [0, n_gu) of the schedule are gate/up
+// tiles, the rest down tiles (item n_gu + i is down tile i).  A down item's producer waits
+// until every gate/up tile of its group has written its h rows (gu_done, released after the
+// rows are stored) before it loads them; the weights of the down GEMM need no wait.
+template <bool GATED, int BN, bool W8, bool FUSED = false>
+__global__ void __launch_bounds__(TcCfg<GATED, BN, W8, FUSED>::kThreads, 1)
+    expert_gemm_tc_kernel(const __grid_constant__ TcParams p, const __grid_constant__ TcParams pdn) {
+  using C = TcCfg<GATED, BN, W8, FUSED>;
+  static_assert(!FUSED || (GATED && BN == 16 && !W8), "one launch for both projections: bf16 16-token tiles");
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   unsigned char* smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
@@ -358,7 +381,19 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
   // capacity) together with the schedule length, so that both arrive in one round trip
   int4 first_info = make_int4(-1, 0, 0, 0);
   if (warp == 0 && static_cast<int>(blockIdx.x) < p.max_items) first_info = __ldg(p.item_info + blockIdx.x);
-  const int total = schedule_length(p);
+  int n_gu, total;  // gate/up items, all items
+  if constexpr (FUSED) {
+    const int a = __ldg(p.item_start + p.G), b = __ldg(pdn.item_start + pdn.G);
+    const bool lengths_ok = a >= 0 && a <= p.max_items && b >= 0 && b <= pdn.max_items;
+    if (!lengths_ok && threadIdx.x == 0 && blockIdx.x == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
+    n_gu = lengths_ok ? a : 0;
+    total = lengths_ok ? a + b : 0;
+  } else {
+    n_gu = total = schedule_length(p);
+  }
+  // the launch parameters of item `it` (gate/up or down) and its index in that schedule
+  auto prm_of = [&](int it) -> const TcParams& { return (FUSED && it >= n_gu) ? pdn : p; };
+  auto local_of = [&](int it) { return (FUSED && it >= n_gu) ? it - n_gu : it; };
   // FP8: waiting threads sleep in their polls, leaving the issue slots to the converters
   auto wait = [&](uint64_t* bar, uint32_t parity) {
     return W8 ? mbar_wait_sleep(bar, parity, p.ctrl, abort_flag) : mbar_wait(bar, parity, p.ctrl, abort_flag);
@@ -398,6 +433,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
     // current one streams
     int it = static_cast<int>(blockIdx.x);
     int4 info = first_info;  // descriptor of item `it`
+    if (FUSED && it >= n_gu && it < total) info = __ldg(pdn.item_info + (it - n_gu));  // a down item first
     int claimed = (lane == 0) ? static_cast<int>(atomicAdd(p.item_counter, 1u) + gridDim.x) : 0;
     for (;;) {
       if (it >= total || !ok) it = -1;
@@ -414,15 +450,42 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
       if (++q == kRing) { q = 0; qphase ^= 1u; }
       if (!pub || it < 0) break;
       const int cur = it;
-      const Item t = decode_item_info<BN>(p, info, cur);
+      const bool dn = FUSED && cur >= n_gu;  // a down item of the fused launch
+      const TcParams& pp = prm_of(cur);
+      const Item t = decode_item_info<BN>(pp, info, local_of(cur));
       it = __shfl_sync(0xffffffffu, claimed, 0);
       if (lane == 0 && it < total) claimed = static_cast<int>(atomicAdd(p.item_counter, 1u) + gridDim.x);
-      if (it < total) info = __ldg(p.item_info + it);
+      if (it < total) info = __ldg(prm_of(it).item_info + local_of(it));
       if (!t.valid) {
         if (blockIdx.x == 0 && lane == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
         continue;
       }
-      const bool gath = GATED && p.gather && !t.sh;
+      const bool gated = GATED && !dn;
+      if (FUSED && dn) {
+        // every gate/up tile of the group has stored its h rows: ceil(rows / BN) token tiles
+        // times the group's gate/up weight tiles
+        int dep = 1;
+        if (lane == 0) {
+          const int rows = t.sh ? p.sh_rows : __ldg(p.counts + t.g);
+          const unsigned int need = static_cast<unsigned int>((rows + BN - 1) / BN * p.mt[t.sh]);
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_gpu(p.gu_done + t.g) < need) {
+            if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
+              set_status(p.ctrl, MOE_ERR_DEVICE_TIMEOUT);
+              *abort_flag = 1;
+              dep = 0;
+              break;
+            }
+            __nanosleep(100);
+          }
+          fence_proxy_async_global();  // the h rows, stored by other SMs, before the TMA reads
+        }
+        if (!__shfl_sync(0xffffffffu, dep, 0)) {
+          ok = false;
+          continue;
+        }
+      }
+      const bool gath = gated && pp.gather && !t.sh;
       int tok[4] = {0, 0, 0, 0};
       if (gath && lane < BN / 4) {
 #pragma unroll
@@ -433,9 +496,11 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
           tok[q] = (v < 0 || v >= p.T) ? 0 : v;  // padding rows repeat the first token
         }
       }
-      const int arow = t.sh ? t.m * kTileM : (t.g - p.g_lo) * p.a_rows_per_group + t.m * kTileM;
-      const int kb_n = p.kblocks[t.sh];
-      const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
+      const int arow = t.sh ? t.m * kTileM : (t.g - pp.g_lo) * pp.a_rows_per_group + t.m * kTileM;
+      const int kb_n = pp.kblocks[t.sh];
+      const int kb0 = t.ks * kb_n / pp.ksplit, kb1 = (t.ks + 1) * kb_n / pp.ksplit;
+      // bytes of one k-block of a stage (a down item of the fused launch has no up rows)
+      const uint32_t kbytes = (FUSED && dn) ? C::kAtomA + C::kAtomB : C::kKBytes;
       // FP8: the item's block scales, one 128-column block per lane (and lane + 32),
       // loaded one item ahead so that their latency overlaps the previous item's stream
       uint32_t sg[2] = {0u, 0u}, su[2] = {0u, 0u};
@@ -455,9 +520,10 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
           }
         }
       }
-      for (int kb = kb0; kb < kb1; kb += C::kKB) {
+      const int kstep = (FUSED && dn) ? C::kDnKB : C::kKB;  // k-blocks per stage
+      for (int kb = kb0; kb < kb1; kb += kstep) {
         unsigned char* st = smem + stage * C::kStageBytes;
-        const int nk = min(C::kKB, kb1 - kb);  // k-blocks in this stage
+        const int nk = min(kstep, kb1 - kb);  // k-blocks in this stage
         uint32_t scw = 0;
         if (W8) {
           const int rel = (kb >> 1) - sc0;  // < 64: the host bounds K by 64 scale blocks
@@ -469,14 +535,14 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
           good = wait(&empty[stage], phase ^ 1u) ? 1 : 0;
           if (good) {
             if (W8) sc_stage[stage] = scw;  // published by the arrive below
-            mbar_arrive_expect_tx(&full[stage], C::kCpGather ? C::kBOffset : nk * C::kKBytes);
+            mbar_arrive_expect_tx(&full[stage], C::kCpGather ? C::kBOffset : nk * kbytes);
             for (int j = 0; j < nk; ++j) {
-              tma_load_2d(st + j * C::kAtomA, &p.tmA[t.sh], (kb + j) * kTileK, arow, &full[stage]);
-              if (GATED)
-                tma_load_2d(st + (W8 ? C::kA8Bytes : C::kABytes) + j * C::kAtomA, &p.tmA[t.sh],
-                            (kb + j) * kTileK, arow + p.a_up_offset[t.sh], &full[stage]);
+              tma_load_2d(st + j * C::kAtomA, &pp.tmA[t.sh], (kb + j) * kTileK, arow, &full[stage]);
+              if (gated)
+                tma_load_2d(st + (W8 ? C::kA8Bytes : C::kABytes) + j * C::kAtomA, &pp.tmA[t.sh],
+                            (kb + j) * kTileK, arow + pp.a_up_offset[t.sh], &full[stage]);
               if (!gath && !C::kCpGather)
-                tma_load_2d(st + C::kBOffset + j * C::kAtomB, &p.tmB[t.sh], (kb + j) * kTileK, t.row0,
+                tma_load_2d(st + C::kBOffset + j * C::kAtomB, &pp.tmB[t.sh], (kb + j) * kTileK, t.row0,
                             &full[stage]);
             }
           }
@@ -617,23 +683,26 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
         mbar_arrive(&ring_empty[q]);
         if (++q == kRing) { q = 0; qphase ^= 1u; }
         if (it < 0) break;
-        const Item t = decode_item<BN>(p, it);
+        const TcParams& pp = prm_of(it);
+        const bool gated = GATED && !(FUSED && it >= n_gu);
+        const Item t = decode_item<BN>(pp, local_of(it));
         if (!t.valid) continue;
         const int n_mma = (t.nvalid + 15) & ~15;
         const uint32_t idesc = idesc_bf16_f32(kTileM, n_mma);
         if (!wait(&tempty[acc], acc_phase ^ 1u)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + acc * C::kAccCols;
-        const int kb_n = p.kblocks[t.sh];
-        const int kb0 = t.ks * kb_n / p.ksplit, kb1 = (t.ks + 1) * kb_n / p.ksplit;
-        for (int kb = kb0; kb < kb1; kb += C::kKB) {
+        const int kb_n = pp.kblocks[t.sh];
+        const int kb0 = t.ks * kb_n / pp.ksplit, kb1 = (t.ks + 1) * kb_n / pp.ksplit;
+        const int kstep = gated ? C::kKB : C::kDnKB;  // k-blocks per stage
+        for (int kb = kb0; kb < kb1; kb += kstep) {
           if (!(W8 ? wait(&cfull[cs], cphase) : wait(&full[stage], phase))) { ok = false; break; }
           tc_fence_after();
           // token rows written by the gather warps' cp.async: order them before the
           // tensor cores' (async-proxy) reads of the stage
           if (C::kCpGather) fence_proxy_async_smem();
           const uint32_t s0 = W8 ? smem_u32(conv + cs * C::kConvBytes) : smem_u32(smem + stage * C::kStageBytes);
-          const int nk = min(C::kKB, kb1 - kb);
+          const int nk = min(kstep, kb1 - kb);
           for (int j = 0; j < nk; ++j) {
             const uint32_t a0 = s0 + j * C::kAtomA;
             const uint32_t b0 = s0 + (W8 ? C::kConvBOffset : C::kBOffset) + j * C::kAtomB;
@@ -642,7 +711,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
               const uint32_t accum = (kb != kb0 || j || kk) ? 1u : 0u;
               const uint64_t bdesc = sw128_kmajor_desc(b0 + kk * 32);
               mma_bf16(d0, sw128_kmajor_desc(a0 + kk * 32), bdesc, idesc, accum);
-              if (GATED)
+              if (gated)
                 mma_bf16(d0 + BN, sw128_kmajor_desc(a0 + C::kABytes + kk * 32), bdesc, idesc, accum);
             }
           }
@@ -782,11 +851,13 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
       if (lane == 0) mbar_arrive(&ring_empty[q]);
       if (++q == kRing) { q = 0; qphase ^= 1u; }
       if (it < 0) break;
-      const Item t = decode_item<BN>(p, it);
+      const TcParams& pp = prm_of(it);
+      const bool gated = GATED && !(FUSED && it >= n_gu);
+      const Item t = decode_item<BN>(pp, local_of(it));
       if (!t.valid) continue;
-      if (!GATED)
+      if (!gated)
         for (int n = et; n < BN; n += 128)
-          sw[n] = (t.sh || n >= t.nvalid) ? 1.0f : __ldg(p.row_w + t.row0 + n);
+          sw[n] = (t.sh || n >= t.nvalid) ? 1.0f : __ldg(pp.row_w + t.row0 + n);
       if (!wait(&tfull[acc], acc_phase)) break;
       tc_fence_after();
       named_bar_sync(1, 128);  // staging free (previous tile copied out), sw visible
@@ -820,7 +891,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
         named_bar_sync(1, 128);  // sw free for the next tile
         continue;
       }
-      if (GATED && C::kStaged && p.ksplit > 1) {
+      if (gated && C::kStaged && p.ksplit > 1) {
         // this slice's gate|up partial sums -> its own fp32 slab; the last slice of the
         // tile adds the slabs, applies SiLU(gate)*up and writes the tile
         float* slab = p.partial + (static_cast<int64_t>(t.tile) * p.ksplit + t.ks) * BN * 256;
@@ -864,13 +935,15 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
           const int n = i >> 4, c = i & 15;
           *reinterpret_cast<uint4*>(out + static_cast<int64_t>(n) * ld + c * 8) = src[n * 16 + c];
         }
+        if (FUSED) release_rows_stored();
         named_bar_sync(1, 128);  // staging and sw[0] free for the next tile
+        if (FUSED && et == 0) atomicAdd(p.gu_done + t.g, 1u);  // the tile's h rows are stored
         continue;
       }
       for (int c0 = 0; c0 < t.nvalid; c0 += 16) {
         uint32_t a[16];
         tmem_ld16_nowait(trow + c0, a);
-        if (GATED) {
+        if (gated) {
           uint32_t u[16];
           tmem_ld16_nowait(trow + BN + c0, u);
           tmem_wait_ld();
@@ -878,7 +951,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
           for (int j = 0; j < 16; ++j)
             if (c0 + j < t.nvalid)
               staging[(c0 + j) * kTileM + r] =
-                  __float2bfloat16_rn(swiglu(__uint_as_float(a[j]), __uint_as_float(u[j]), p.limit[t.sh]));
+                  __float2bfloat16_rn(swiglu(__uint_as_float(a[j]), __uint_as_float(u[j]), pp.limit[t.sh]));
         } else {
           tmem_wait_ld();
 #pragma unroll
@@ -892,12 +965,17 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8>::kThreads, 1) expert_gemm
       if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
       named_bar_sync(1, 128);  // staging tile complete
       // rows of 128 bf16 (256 B) -> out[row0 + n][m*128 ...], 16-byte coalesced stores
-      const int ld = p.ld_out[t.sh];
-      __nv_bfloat16* out = p.out[t.sh] + static_cast<int64_t>(t.row0) * ld + t.m * kTileM;
+      const int ld = pp.ld_out[t.sh];
+      __nv_bfloat16* out = pp.out[t.sh] + static_cast<int64_t>(t.row0) * ld + t.m * kTileM;
       const uint4* src = reinterpret_cast<const uint4*>(staging);
       for (int i = et; i < t.nvalid * 16; i += 128) {
         const int n = i >> 4, c = i & 15;
         *reinterpret_cast<uint4*>(out + static_cast<int64_t>(n) * ld + c * 8) = src[n * 16 + c];
+      }
+      if (FUSED && gated) {
+        release_rows_stored();
+        named_bar_sync(1, 128);
+        if (et == 0) atomicAdd(p.gu_done + t.g, 1u);  // the tile's h rows are stored
       }
     }
   }
@@ -1260,7 +1338,19 @@ static cudaError_t launch_tc(const TcParams& prm_in, int num_sms, cudaStream_t s
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  e = launch_pdl(kern, dim3(num_sms), dim3(C::kThreads), smem, st, prm);
+  e = launch_pdl(kern, dim3(num_sms), dim3(C::kThreads), smem, st, prm, prm);
+  count_launches(1);
+  return e;
+}
+
+// both projections of bf16 16-token tiles in one launch (gu: gate/up, dn: down)
+static cudaError_t launch_fused(const TcParams& gu, const TcParams& dn, int num_sms, cudaStream_t st) {
+  using C = TcCfg<true, 16, false, true>;
+  auto kern = expert_gemm_tc_kernel<true, 16, false, true>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(C::kSmemBytes));
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(kern, dim3(num_sms), dim3(C::kThreads), static_cast<size_t>(C::kSmemBytes), st, gu, dn);
   count_launches(1);
   return e;
 }
@@ -1369,7 +1459,12 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   g.limit[1] = a.swiglu_limit_shared;
   g.gather = gather ? 1 : 0;
   g.x = static_cast<const __nv_bfloat16*>(a.x);
-  if (!a.w8 && !a.pair_dn) {
+  // bf16 16-token tiles (decode): both projections in one launch, each down tile starting
+  // as soon as its group's gate/up tiles are done
+  const bool fused = !a.w8 && !a.pair_dn && a.bn == 16 && a.bn_dn == 16 && a.gu_done && a.counts;
+  g.gu_done = a.gu_done;
+  g.counts = a.counts;
+  if (!a.w8 && !a.pair_dn && !fused) {
     g.pf_item_start = a.item_start_dn;
     g.pf_info = a.info_dn;
     g.pf_w[0] = static_cast<const unsigned char*>(a.Wd);
@@ -1409,9 +1504,11 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
   g.scaleA[1] = static_cast<const uint8_t*>(a.Wsgu_scale);
   g.s_rows_per_group = 2 * a.I / kTileM;
   g.s_ld[0] = g.s_ld[1] = (a.H + 127) / 128;
-  cudaError_t e = launch_tc_bn<true>(g, a.bn, a.w8, a.num_sms, st);
-  if (e != cudaSuccess) return e;
-  if (a.stage_mark) a.stage_mark(a.stage_mark_ctx, 3, st);
+  if (!fused) {
+    cudaError_t e = launch_tc_bn<true>(g, a.bn, a.w8, a.num_sms, st);
+    if (e != cudaSuccess) return e;
+    if (a.stage_mark) a.stage_mark(a.stage_mark_ctx, 3, st);
+  }
   // down: A = W_down viewed as [E*H, I]; B = h [P, I] (shared: Ws_down [H, Is], h_shared)
   TcParams d{};
   ok = encode_w(&d.tmA[0], a.Wd, n_local * a.H, a.I) &&
@@ -1459,6 +1556,11 @@ cudaError_t launch_experts(const ExpertArgs& a, cudaStream_t st) {
     d.max_tiles = static_cast<int>(expert_tile_bound(a.T, a.k, a.E, a.H / 2, a.Is > 0 ? a.H / 2 : 0, 256));
     d.max_items = d.max_tiles;
     return launch_pair(d, a.num_sms, st);
+  }
+  if (fused) {
+    const cudaError_t e = launch_fused(g, d, a.num_sms, st);
+    if (e == cudaSuccess && a.stage_mark) a.stage_mark(a.stage_mark_ctx, 3, st);  // no boundary between them
+    return e;
   }
   return launch_tc_bn<false>(d, a.bn_dn, a.w8, a.num_sms, st);
 }

@@ -143,6 +143,8 @@ struct ExpertArgs {
   float* partial;   // split partial sums (ksplit > 1)
   unsigned int* tile_done;  // per-tile slice counters, zero before the forward
   unsigned int* item_counters;  // [2] dynamic item claims of the two GEMMs, zero before the forward
+  unsigned int* gu_done;   // [E + 1] gate/up tiles finished per group, zero before the forward
+  const int32_t* counts;   // [E] rows per routed expert
   float swiglu_limit;          // routed experts: gate <= L, up in [-L, L] before SiLU*up (0: none)
   float swiglu_limit_shared;   // the same for the shared expert
   void* h;          // [T*k, I]
