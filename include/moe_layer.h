@@ -272,8 +272,9 @@ MOE_API moe_status moe_layer_workspace_layout(const moe_layer_shape* shape, moe_
  * CUDA events on its stream at the boundaries of its five stages:
  *   0 routing  (router scores, certified top-k, softmax weights)
  *   1 dispatch (histogram, scan, stable permutation, row gather)
- *   2 gate/up  (grouped GEMM with the SiLU(gate)*up epilogue)
- *   3 down     (grouped GEMM with the routing-weight epilogue)
+ *   2 gate/up  (grouped GEMM with the SiLU(gate)*up epilogue; with 16-token tiles, bf16
+ *              weights, both GEMMs, which then run as one launch)
+ *   3 down     (grouped GEMM with the routing-weight epilogue; empty when stage 2 ran both)
  *   4 combine  (unpermute and sum)
  * moe_layer_profile_read() waits for the recorded events, adds each stage's elapsed
  * milliseconds since the previous read into ms[0..n_stages), forgets them and returns

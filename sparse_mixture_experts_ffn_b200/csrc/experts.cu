@@ -279,7 +279,7 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 // other SMs once the count is acquired.
 __device__ __forceinline__ void release_rows_stored() {
   fence_proxy_async_global();
-  __threadfence();
+  fence_acq_rel_gpu();
 }
 
 // Persistent grouped GEMM, one block per SM.
@@ -435,6 +435,10 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8, FUSED>::kThreads, 1)
     int4 info = first_info;  // descriptor of item `it`
     if (FUSED && it >= n_gu && it < total) info = __ldg(pdn.item_info + (it - n_gu));  // a down item first
     int claimed = (lane == 0) ? static_cast<int>(atomicAdd(p.item_counter, 1u) + gridDim.x) : 0;
+    // fused launch: the gate/up tiles finished in the group of the next (down) item, read
+    // during the current item's second stage so that the next item seldom waits for it
+    int pre_g = -1;
+    unsigned int pre_seen = 0;
     for (;;) {
       if (it >= total || !ok) it = -1;
       // publish the item (or the end) to the MMA and epilogue warps
@@ -453,38 +457,43 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8, FUSED>::kThreads, 1)
       const bool dn = FUSED && cur >= n_gu;  // a down item of the fused launch
       const TcParams& pp = prm_of(cur);
       const Item t = decode_item_info<BN>(pp, info, local_of(cur));
-      it = __shfl_sync(0xffffffffu, claimed, 0);
-      if (lane == 0 && it < total) claimed = static_cast<int>(atomicAdd(p.item_counter, 1u) + gridDim.x);
-      if (it < total) info = __ldg(prm_of(it).item_info + local_of(it));
+      // the next item's claim and descriptor, taken once this item's first stage is issued
+      // (at the first item the claim is still in flight)
+      bool next_taken = false;
+      auto take_next = [&]() {
+        if (next_taken) return;
+        next_taken = true;
+        it = __shfl_sync(0xffffffffu, claimed, 0);
+        if (lane == 0 && it < total) claimed = static_cast<int>(atomicAdd(p.item_counter, 1u) + gridDim.x);
+        if (it < total) info = __ldg(prm_of(it).item_info + local_of(it));
+      };
       if (!t.valid) {
         if (blockIdx.x == 0 && lane == 0) set_status(p.ctrl, MOE_ERR_DEVICE_BOUNDS);
+        take_next();
         continue;
       }
       const bool gated = GATED && !dn;
-      if (FUSED && dn) {
-        // every gate/up tile of the group has stored its h rows: ceil(rows / BN) token tiles
-        // times the group's gate/up weight tiles
-        int dep = 1;
-        if (lane == 0) {
-          const int rows = t.sh ? p.sh_rows : __ldg(p.counts + t.g);
-          const unsigned int need = static_cast<unsigned int>((rows + BN - 1) / BN * p.mt[t.sh]);
-          const uint64_t t0 = globaltimer_ns();
-          while (ld_acquire_gpu(p.gu_done + t.g) < need) {
-            if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
-              set_status(p.ctrl, MOE_ERR_DEVICE_TIMEOUT);
-              *abort_flag = 1;
-              dep = 0;
-              break;
-            }
-            __nanosleep(100);
+      // a down item of the fused launch (lane 0): every gate/up tile of its group has stored
+      // its h rows -- ceil(rows / BN) token tiles times the group's gate/up weight tiles
+      auto rows_ready = [&]() -> bool {
+        const int rows = t.sh ? p.sh_rows : __ldg(p.counts + t.g);
+        const unsigned int need = static_cast<unsigned int>((rows + BN - 1) / BN * p.mt[t.sh]);
+        if (pre_g == t.g && pre_seen >= need) {
+          fence_proxy_async_global();
+          return true;
+        }
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_gpu(p.gu_done + t.g) < need) {
+          if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
+            set_status(p.ctrl, MOE_ERR_DEVICE_TIMEOUT);
+            *abort_flag = 1;
+            return false;
           }
-          fence_proxy_async_global();  // the h rows, stored by other SMs, before the TMA reads
+          __nanosleep(100);
         }
-        if (!__shfl_sync(0xffffffffu, dep, 0)) {
-          ok = false;
-          continue;
-        }
-      }
+        fence_proxy_async_global();  // the h rows, stored by other SMs, before the TMA reads
+        return true;
+      };
       const bool gath = gated && pp.gather && !t.sh;
       int tok[4] = {0, 0, 0, 0};
       if (gath && lane < BN / 4) {
@@ -506,6 +515,7 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8, FUSED>::kThreads, 1)
       uint32_t sg[2] = {0u, 0u}, su[2] = {0u, 0u};
       const int sc0 = kb0 >> 1;  // 128-column scale blocks hold two 64-column k-blocks
       if (W8) {
+        take_next();  // the next item's scales are loaded now
         if (pf_it == cur) {
           sg[0] = pf_sg[0]; sg[1] = pf_sg[1]; su[0] = pf_su[0]; su[1] = pf_su[1];
         } else {
@@ -541,10 +551,14 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8, FUSED>::kThreads, 1)
               if (gated)
                 tma_load_2d(st + (W8 ? C::kA8Bytes : C::kABytes) + j * C::kAtomA, &pp.tmA[t.sh],
                             (kb + j) * kTileK, arow + pp.a_up_offset[t.sh], &full[stage]);
-              if (!gath && !C::kCpGather)
+            }
+            // a down item's h rows once its group's gate/up tiles are done (its first
+            // weight k-blocks are in flight meanwhile)
+            if (FUSED && dn && kb == kb0 && !rows_ready()) good = 0;
+            if (good && !gath && !C::kCpGather)
+              for (int j = 0; j < nk; ++j)
                 tma_load_2d(st + C::kBOffset + j * C::kAtomB, &pp.tmB[t.sh], (kb + j) * kTileK, t.row0,
                             &full[stage]);
-            }
           }
         }
         good = __shfl_sync(0xffffffffu, good, 0);
@@ -555,7 +569,16 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8, FUSED>::kThreads, 1)
                            tok[0], tok[1], tok[2], tok[3], &full[stage]);
         used |= 1u << stage;
         if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        if (kb == kb0) take_next();
+        if (FUSED && lane == 0 && kb == kb0 + kstep) {
+          pre_g = -1;
+          if (it >= n_gu && it < total && info.x >= 0 && info.x <= p.E) {  // the next item is a down item
+            pre_g = info.x;
+            pre_seen = ld_acquire_gpu(p.gu_done + pre_g);
+          }
+        }
       }
+      take_next();
     }
     __syncwarp();
     if (GATED && !W8 && p.pf_item_start && lane == 0 && static_cast<int>(blockIdx.x) < __ldg(p.pf_item_start + p.G)) {
@@ -910,14 +933,14 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8, FUSED>::kThreads, 1)
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
         if (++acc == C::kAccBufs) { acc = 0; acc_phase ^= 1u; }
-        __threadfence();
+        fence_acq_rel_gpu();
         named_bar_sync(1, 128);
         if (et == 0) sw[0] = (atomicAdd(p.tile_done + t.tile, 1u) == static_cast<unsigned>(p.ksplit - 1)) ? 1.f : 0.f;
         named_bar_sync(1, 128);
         const bool last_slice = sw[0] != 0.f;
         named_bar_sync(1, 128);  // the flag is read by all before it can be rewritten
         if (!last_slice) continue;  // another slice finishes this tile
-        __threadfence();
+        fence_acq_rel_gpu();
         const float* tile_slabs = p.partial + static_cast<int64_t>(t.tile) * p.ksplit * BN * 256;
         for (int n = 0; n < t.nvalid; ++n) {
           float gs = 0.f, us = 0.f;

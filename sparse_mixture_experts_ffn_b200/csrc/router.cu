@@ -944,7 +944,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) router_decode_kernel(
     }
   }
   // last block of the token group?
-  __threadfence();
+  fence_acq_rel_gpu();
   __syncthreads();
   if (threadIdx.x == 0) {
     const unsigned prev = atomicAdd(&group_done[g], 1u);
@@ -952,7 +952,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1) router_decode_kernel(
   }
   __syncthreads();
   if (is_last) {
-    __threadfence();
+    fence_acq_rel_gpu();
     for (int tt = warp; tt < nt; tt += kDecodeThreads / 32) {
       const int64_t t = t0 + tt;
       const T* xt = x + t * H;
@@ -1218,7 +1218,7 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
         }
       }
       // the last block of this (m, n) tile adds the partials of every chunk (below)
-      __threadfence();
+      fence_acq_rel_gpu();
       named_bar_sync(1, 128);
       if (warp == 2 && lane == 0) {
         const unsigned int done = atomicAdd(p.tile_done + blockIdx.x, 1u);
@@ -1236,7 +1236,7 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
   // the chunks' sums of squares, in chunk order), by all six warps.  Every load of a thread
   // is issued before the first of its values is used: first the sums of squares of the norm
   // bound it owns (threads from the last one down), then two scores at a time.
-  __threadfence();
+  fence_acq_rel_gpu();
   const int np = rows * ne, nxj = (ni == 0) ? rows : 0, nwj = (mi == 0 && !p.w_given) ? ne : 0;
   const int nthr = static_cast<int>(blockDim.x);
   const int jn = nthr - 1 - static_cast<int>(threadIdx.x);  // this thread's norm bound, if < nxj + nwj
