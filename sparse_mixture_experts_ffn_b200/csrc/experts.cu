@@ -369,6 +369,12 @@ __global__ void __launch_bounds__(TcCfg<GATED, BN, W8, FUSED>::kThreads, 1)
     tma_prefetch_desc(&p.tmB[0]);
     tma_prefetch_desc(&p.tmA[1]);
     tma_prefetch_desc(&p.tmB[1]);
+    if (FUSED) {
+      tma_prefetch_desc(&pdn.tmA[0]);
+      tma_prefetch_desc(&pdn.tmB[0]);
+      tma_prefetch_desc(&pdn.tmA[1]);
+      tma_prefetch_desc(&pdn.tmB[1]);
+    }
   }
   if (warp == 1) tmem_alloc(tmem_slot, C::kTmemCols);
   tc_fence_before();
