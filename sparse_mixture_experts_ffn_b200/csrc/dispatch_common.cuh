@@ -48,6 +48,10 @@ static __device__ V block_scan_pair(V v0, V v1, V* warp_tot, V& total) {
   return excl;  // exclusive prefix of v0; v1's is excl + v0
 }
 
+// log2 of a power of two (token tile widths 16, 128, 256 and reduction splits 1, 2, 4 are),
+// so that tile counts and item coordinates take shifts and masks instead of divisions
+__device__ __forceinline__ int log2_pow2(int x) { return __ffs(x) - 1; }
+
 struct ScheduleArgs {
   int64_t T;
   int E, has_shared, mt_gu, mt_gu_shared, mt_dn, bn, bn_dn, ksplit;
@@ -170,7 +174,7 @@ static __device__ int build_schedule(const ScheduleArgs& a, int* cnt, int* order
     const int g = order[r];
     const int bn = gu ? a.bn : a.bn_dn;
     if (g < E && (g < a.e_lo || g >= a.e_hi)) return 0;  // another rank's expert
-    const int nt = (cnt[g] + bn - 1) / bn;
+    const int nt = (cnt[g] + bn - 1) >> log2_pow2(bn);
     const int mt = gu ? (g < E ? a.mt_gu : a.mt_gu_shared) * a.ksplit : a.mt_dn;
     return nt * mt;
   };
@@ -228,14 +232,14 @@ static __device__ void write_item_tables(const ScheduleArgs& a, const int* cnt, 
       }
       const int g = order[lo];
       const int rows = cnt[g];
-      const int ntile = (rows + bn - 1) / bn;  // >= 1: groups without rows have no items
+      const int ntile = (rows + bn - 1) >> log2_pow2(bn);  // >= 1: groups without rows have no items
       if (ntile < 1) {  // inconsistent prefixes: an invalid descriptor, reported by the GEMM
         info[it] = make_int4(-1, 0, 0, 0);
         continue;
       }
       const int l = it - istart[lo];
-      const int tile = l / ks_n, ks = l - tile * ks_n;
-      const int m = tile / ntile, n = tile - m * ntile;
+      const int tile = l >> log2_pow2(ks_n), ks = l & (ks_n - 1);
+      const int m = ntile == 1 ? tile : tile / ntile, n = tile - m * ntile;
       const int row0 = (g < E ? off[g] : 0) + n * bn;
       info[it] = make_int4(g, m, row0, min(bn, rows - n * bn) | (ks << 16));
     }
@@ -262,15 +266,16 @@ static __device__ void write_item_tables_by_slot(const ScheduleArgs& a, const in
     const int i0 = istart[r], n_items = istart[r + 1] - i0;
     if (n_items <= 0) continue;
     const int g = order[r], rows = cnt[g];
-    const int ntile = (rows + bn - 1) / bn;
+    const int ntile = (rows + bn - 1) >> log2_pow2(bn);
     const int rbase = g < E ? off[g] : 0;
+    const int ksh = log2_pow2(ks_n);
     for (int l = lane; l < n_items; l += 32) {
       if (ntile < 1) {  // inconsistent prefixes: an invalid descriptor, reported by the GEMM
         info[i0 + l] = make_int4(-1, 0, 0, 0);
         continue;
       }
-      const int tile = l / ks_n, ks = l - tile * ks_n;
-      const int m = tile / ntile, n = tile - m * ntile;
+      const int tile = l >> ksh, ks = l & (ks_n - 1);
+      const int m = ntile == 1 ? tile : tile / ntile, n = tile - m * ntile;  // one token tile: no division
       info[i0 + l] = make_int4(g, m, rbase + n * bn, min(bn, rows - n * bn) | (ks << 16));
     }
   }

@@ -484,25 +484,25 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
       u[i] = ordered(kf.key_lo(__dadd_rd(srow[e], -d), e));
     }
   }
-  // 2. Lk
+  // 2. Lk: each lane sorts its lower bounds in descending order; each of k rounds takes the
+  //    warp's largest head and shifts that lane's list by one (0 marks an empty slot)
   uint32_t lk = 0;
   {
-    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i)
+#pragma unroll
+      for (int j = i + 1; j < EPL; ++j) {
+        const uint32_t a = u[i], b = u[j];
+        u[i] = max(a, b);
+        u[j] = min(a, b);
+      }
     for (int r = 0; r < k; ++r) {
-      uint32_t best = 0;
-#pragma unroll
-      for (int i = 0; i < EPL; ++i)
-        if (!(taken & (1u << i))) best = max(best, u[i]);
-      const uint32_t gbest = __reduce_max_sync(0xffffffffu, best);
-      const unsigned holders = __ballot_sync(0xffffffffu, best == gbest);
+      const uint32_t gbest = __reduce_max_sync(0xffffffffu, u[0]);
+      const unsigned holders = __ballot_sync(0xffffffffu, u[0] == gbest);
       if (lane == __ffs(holders) - 1) {
-        bool done = false;
 #pragma unroll
-        for (int i = 0; i < EPL; ++i)
-          if (!done && !(taken & (1u << i)) && u[i] == gbest) {
-            taken |= 1u << i;
-            done = true;
-          }
+        for (int i = 0; i + 1 < EPL; ++i) u[i] = u[i + 1];
+        u[EPL - 1] = 0;
       }
       lk = gbest;
     }

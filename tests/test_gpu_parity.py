@@ -50,6 +50,9 @@ SMALL = [
     # ragged last expert tile
     dict(T=30, H=1024, E=96, top_k=6, I=128, I_shared=128),
     dict(T=3, H=2176, E=200, top_k=8, I=128, I_shared=128),
+    # 16-token tiles (both GEMMs in one launch) without a shared expert, the gate/up
+    # reduction split: fewer items than blocks, so blocks start on down tiles and wait
+    dict(T=5, H=256, E=32, top_k=4, I=256, I_shared=0),
     # 256-token tiles (about 350 tokens per expert: one full and one ragged tile each)
     dict(T=700, H=256, E=8, top_k=4, I=256, I_shared=128),
     # 256 x 256 tiles over pairs of SMs (widths multiples of 256): ragged token tiles, a
@@ -205,6 +208,24 @@ def test_group_sizes_at_tile_edges():
     ref = oracle_routing(d, 1)
     assert_routing_exact(r, ref, E)
     assert_y_close(y, oracle_y(d, ref), "tile edges")
+
+
+def test_decode_forward_launch_count():
+    """16-token tiles with bf16 weights run five launches: router GEMM, selection, dispatch, one
+    launch of both expert GEMMs, combine (the decode shape: 4 tokens, 288 experts, top-8)."""
+    cfg = inputs.small_config(T=4, H=512, E=288, top_k=8, I=128, I_shared=128)
+    d = to_device(inputs.make_inputs(cfg, "cuda", shared=True))
+    ws = moe.alloc_workspace(moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.I, cfg.I_shared, cfg.top_k, torch.bfloat16), "cuda")
+    run(d, cfg.top_k, workspace=ws)  # first call: one-time setup launches, if any
+    torch.cuda.synchronize()
+    n0 = moe.launch_count()
+    y, r = run(d, cfg.top_k, workspace=ws)
+    torch.cuda.synchronize()
+    assert moe.launch_count() - n0 == 5
+    assert moe.check_status(ws) == moe.MOE_OK
+    ref = oracle_routing(d, cfg.top_k)
+    assert_routing_exact(r, ref, cfg.E)
+    assert_y_close(y, oracle_y(d, ref), cfg.name)
 
 
 def test_ties_and_zero_input():
