@@ -473,16 +473,19 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
   const int lane = threadIdx.x & 31;
   auto nw = [&](int e) -> double { return wss ? norm_ub_from_sumsq(wss[e], H) : wnorm[e]; };
   const double cdx = __dmul_ru(delta_coef, nx);
-  // 1. lower bounds
+  // 1. lower bounds (the estimates and their error bounds stay in registers for step 3)
   uint32_t u[EPL];
+  double sh_r[EPL], d_r[EPL];
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
-    u[i] = 0;
-    if (e < E) {
-      const double d = __dadd_ru(__dmul_ru(cdx, nw(e)), delta_abs);
-      u[i] = ordered(kf.key_lo(__dadd_rd(srow[e], -d), e));
-    }
+    sh_r[i] = (e < E) ? srow[e] : 0.0;
+    d_r[i] = (e < E) ? __dadd_ru(__dmul_ru(cdx, nw(e)), delta_abs) : 0.0;
+  }
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    u[i] = (e < E) ? ordered(kf.key_lo(__dadd_rd(sh_r[i], -d_r[i]), e)) : 0u;
   }
   // 2. Lk: each lane sorts its lower bounds in descending order; each of k rounds takes the
   //    warp's largest head and shifts that lane's list by one (0 marks an empty slot)
@@ -507,32 +510,27 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
       lk = gbest;
     }
   }
-  // 3. candidates, compacted in ascending expert order
+  // 3. candidates, compacted in ascending expert order (their keys first, then the places)
   int cn = 0;
+  bool cand_r[EPL];
+  float hi_r[EPL];
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
-    float lo = 0.f, hi = 0.f, mid = 0.f, pv = 0.f;
-    bool cand = false;
-    if (e < E) {
-      const double sh = srow[e];
-      const double d = __dadd_ru(__dmul_ru(cdx, nw(e)), delta_abs);
-      hi = kf.key_hi(__dadd_ru(sh, d), e);
-      cand = ordered(hi) >= lk;
-      if (cand) {
-        lo = kf.key_lo(__dadd_rd(sh, -d), e);
-        mid = kf.key(sh, e);
-        if (SIG) pv = kf.score(sh);
-      }
-    }
-    const unsigned m = __ballot_sync(0xffffffffu, cand);
+    hi_r[i] = (e < E) ? kf.key_hi(__dadd_ru(sh_r[i], d_r[i]), e) : 0.f;
+    cand_r[i] = (e < E) && ordered(hi_r[i]) >= lk;
+  }
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const int e = lane + 32 * i;
+    const unsigned m = __ballot_sync(0xffffffffu, cand_r[i]);
     const int pos = cn + __popc(m & ((1u << lane) - 1u));
-    if (cand && pos < 32) {
+    if (cand_r[i] && pos < 32) {
       C.e[pos] = e;
-      C.lo[pos] = lo;
-      C.hi[pos] = hi;
-      C.mid[pos] = mid;
-      if (SIG) C.p[pos] = pv;
+      C.lo[pos] = kf.key_lo(__dadd_rd(sh_r[i], -d_r[i]), e);
+      C.hi[pos] = hi_r[i];
+      C.mid[pos] = kf.key(sh_r[i], e);
+      if (SIG) C.p[pos] = kf.score(sh_r[i]);
     }
     cn += __popc(m);
   }
@@ -545,6 +543,7 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
   float my_p = (SIG && mine) ? C.p[lane] : 0.f;
   auto classify_mine = [&]() -> int {
     int cp = 0, cc = 0;
+#pragma unroll 4
     for (int j = 0; j < cn; ++j) {
       if (j == lane) continue;
       const int f = C.e[j];
