@@ -284,12 +284,14 @@ static __device__ void write_item_tables_by_slot(const ScheduleArgs& a, const in
 // Stable placement of the assignments [a0, a1) by one warp, 32 at a time, in (token,
 // slot) order: equal experts inside a chunk get consecutive positions in lane order.
 // base[e] holds the next free position of expert e and is advanced.  The indices and weights
-// of four chunks are loaded before the first of them is placed.
+// of four chunks are loaded before the first of them is placed; those of the lane's first
+// assignment (a0 + lane) may come loaded already (e_first / w_first, when have_first).
 static __device__ void place_assignments(const int32_t* __restrict__ idx, const float* __restrict__ w,
                                   int64_t a0, int64_t a1, int k, int E, int* base,
                                   int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm,
                                   float* __restrict__ row_w, int32_t* __restrict__ row_tok,
-                                  int32_t* __restrict__ perm_user) {
+                                  int32_t* __restrict__ perm_user, bool have_first = false,
+                                  int e_first = 0, float w_first = 0.0f) {
   const int lane = threadIdx.x & 31;
   constexpr int kAhead = 4;
   for (int64_t c0 = a0; c0 < a1; c0 += 32 * kAhead) {
@@ -298,8 +300,9 @@ static __device__ void place_assignments(const int32_t* __restrict__ idx, const 
 #pragma unroll
     for (int u = 0; u < kAhead; ++u) {
       const int64_t a = c0 + 32 * u + lane;
-      ev[u] = (a < a1) ? idx[a] : -1;
-      wv[u] = (a < a1) ? w[a] : 0.0f;
+      const bool pre = have_first && c0 == a0 && u == 0;
+      ev[u] = (a < a1) ? (pre ? e_first : idx[a]) : -1;
+      wv[u] = (a < a1) ? (pre ? w_first : w[a]) : 0.0f;
     }
 #pragma unroll
     for (int u = 0; u < kAhead; ++u) {
@@ -343,10 +346,15 @@ static __device__ void dispatch_small_block(const ScheduleArgs& sa, const int32_
                                             Ctrl* ctrl, SmallDispatchSmem& sm) {
   const int E = sa.E;
   const int64_t P = sa.T * k;
+  // this thread's first assignment (and, for the placing warp, its weight), requested before
+  // the counters are cleared
+  const bool has_first = static_cast<int64_t>(threadIdx.x) < P;
+  const int e_first = has_first ? idx[threadIdx.x] : 0;
+  const float w_first = (has_first && threadIdx.x < 32) ? w[threadIdx.x] : 0.0f;
   for (int e = threadIdx.x; e < E + 1; e += blockDim.x) sm.cnt[e] = 0;
   __syncthreads();
   for (int64_t a = threadIdx.x; a < P; a += blockDim.x) {
-    const int e = idx[a];
+    const int e = (a == threadIdx.x) ? e_first : idx[a];
     if (e < 0 || e >= E) {
       set_status(ctrl, MOE_ERR_DEVICE_BOUNDS);
       continue;
@@ -371,7 +379,8 @@ static __device__ void dispatch_small_block(const ScheduleArgs& sa, const int32_
   for (int e = threadIdx.x; e < E; e += blockDim.x) sm.base[e] = sm.sched.off[e];
   __syncthreads();
   if (threadIdx.x < 32)
-    place_assignments(idx, w, 0, P, k, E, sm.base, perm, inv_perm, row_w, row_tok, perm_user);
+    place_assignments(idx, w, 0, P, k, E, sm.base, perm, inv_perm, row_w, row_tok, perm_user, true, e_first,
+                      w_first);
 }
 
 // The schedule arguments of a dispatch (tile shapes of both grouped GEMMs).
