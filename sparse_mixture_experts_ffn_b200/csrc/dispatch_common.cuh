@@ -306,6 +306,7 @@ static __device__ void place_assignments(const int32_t* __restrict__ idx, const 
     }
 #pragma unroll
     for (int u = 0; u < kAhead; ++u) {
+      if (c0 + 32 * u >= a1) break;  // no assignments left (the same for every lane)
       const int64_t a = c0 + 32 * u + lane;
       int e = ev[u];
       if (e < 0 || e >= E) e = -1;  // reported by the histogram

@@ -545,11 +545,11 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
     int cp = 0, cc = 0;
 #pragma unroll 4
     for (int j = 0; j < cn; ++j) {
-      if (j == lane) continue;
       const int f = C.e[j];
       const float hf = C.hi[j], lf = C.lo[j];
-      cp += (hf > my_lo) || (hf == my_lo && f < my_e);
-      cc += (lf > my_hi) || (lf == my_hi && f < my_e);
+      const bool other = j != lane;
+      cp += other && ((hf > my_lo) || (hf == my_lo && f < my_e));
+      cc += other && ((lf > my_hi) || (lf == my_hi && f < my_e));
     }
     return (cp < k) ? ST_IN : (cc >= k ? ST_OUT : ST_UNDECIDED);
   };
@@ -1242,11 +1242,11 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
   const bool has_norm = jn < nxj + nwj;  // every bound has its thread: rows + ne <= 32 + 64 < 192
   const bool norm_x = jn < nxj;
   double nv[16];
-  {
+  if (has_norm) {  // 16 loads, none of them conditional (chunks past the last repeat it, unused)
     const double* src = norm_x ? p.xss + t0 + jn : p.wss + e0 + (jn - nxj);
     const int64_t nst = norm_x ? p.T : static_cast<int64_t>(p.E);
 #pragma unroll
-    for (int z = 0; z < 16; ++z) nv[z] = (has_norm && z < p.chunks) ? __ldcg(src + z * nst) : 0.0;
+    for (int z = 0; z < 16; ++z) nv[z] = __ldcg(src + min(z, p.chunks - 1) * nst);
   }
   const int64_t sstride = p.T * p.E;
   for (int j0 = threadIdx.x; j0 < np; j0 += 2 * nthr) {
@@ -1257,20 +1257,23 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
     const float* pa = p.part + (t0 + ta) * p.E + e0 + ea;
     const float* pb = p.part + (t0 + tb) * p.E + e0 + eb;
     double acc_a = 0.0, acc_b = 0.0;
-    for (int b = 0; b < n_sl_all; b += 16) {
+    int b = 0;
+    for (; b + 16 <= n_sl_all; b += 16) {  // 32 unconditional loads, then the sums in slice order
       float va[16], vb[16];
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        const bool in = b + q < n_sl_all;
-        va[q] = in ? __ldcg(pa + (b + q) * sstride) : 0.0f;
-        vb[q] = in ? __ldcg(pb + (b + q) * sstride) : 0.0f;
+        va[q] = __ldcg(pa + (b + q) * sstride);
+        vb[q] = __ldcg(pb + (b + q) * sstride);
       }
 #pragma unroll
-      for (int q = 0; q < 16; ++q)
-        if (b + q < n_sl_all) {
-          acc_a += static_cast<double>(va[q]);
-          acc_b += static_cast<double>(vb[q]);
-        }
+      for (int q = 0; q < 16; ++q) {
+        acc_a += static_cast<double>(va[q]);
+        acc_b += static_cast<double>(vb[q]);
+      }
+    }
+    for (; b < n_sl_all; ++b) {
+      acc_a += static_cast<double>(__ldcg(pa + b * sstride));
+      acc_b += static_cast<double>(__ldcg(pb + b * sstride));
     }
     p.scores[(t0 + ta) * p.E + e0 + ea] = acc_a;
     if (h1) p.scores[(t0 + tb) * p.E + e0 + eb] = acc_b;
