@@ -291,29 +291,34 @@ struct Keys {
     const float s32 = __double2float_rn(s);
     return sigmoid ? sigmoid32(s32) : s32;
   }
-  // the key of a logit (exact when s is the exact logit rounded to fp32)
-  __device__ __forceinline__ float key(double s, int e) const {
+  // the bias of expert e (0 without one), for the *_b forms below that take it loaded
+  __device__ __forceinline__ float bias_of(int e) const { return bias ? bias[e] : 0.0f; }
+  // the key of a logit (exact when s is the exact logit rounded to fp32); b = bias_of(e)
+  __device__ __forceinline__ float key_b(double s, float b) const {
     const float v = score(s);
-    return bias ? __fadd_rn(v, bias[e]) : v;
+    return bias ? __fadd_rn(v, b) : v;
   }
+  __device__ __forceinline__ float key(double s, int e) const { return key_b(s, bias_of(e)); }
   // Lower / upper ends of the keys of all logits >= s_lo / <= s_hi.  For the sigmoid the
   // ends come from an fp32 evaluation, 1 / (1 + expf(-z)) (expf within 2 ulps over its whole
   // range, as CUDA documents it; one rounding each for the add and the IEEE division), widened
   // by a relative 2^-20: that covers its error against the exact sigmoid and the fp64
   // definition's rounding to fp32, at a tenth of the cost of the fp64 evaluation.  Below
   // z = -80 the ends are 0 and 2^-115 > sigma(-80).
-  __device__ __forceinline__ float key_lo(double s_lo, int e) const {
-    if (!sigmoid) return key(s_lo, e);
+  __device__ __forceinline__ float key_lo_b(double s_lo, float b) const {
+    if (!sigmoid) return key_b(s_lo, b);
     const float z = __double2float_rd(s_lo);
     const float p = z < -80.0f ? 0.0f : __fmul_rd(__fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-z))), 1.0f - 0x1p-20f);
-    return bias ? __fadd_rd(p, bias[e]) : p;
+    return bias ? __fadd_rd(p, b) : p;
   }
-  __device__ __forceinline__ float key_hi(double s_hi, int e) const {
-    if (!sigmoid) return key(s_hi, e);
+  __device__ __forceinline__ float key_hi_b(double s_hi, float b) const {
+    if (!sigmoid) return key_b(s_hi, b);
     const float z = __double2float_ru(s_hi);
     const float p = z < -80.0f ? 0x1p-115f : __fmul_ru(__fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-z))), 1.0f + 0x1p-20f);
-    return bias ? __fadd_ru(p, bias[e]) : p;
+    return bias ? __fadd_ru(p, b) : p;
   }
+  __device__ __forceinline__ float key_lo(double s_lo, int e) const { return key_lo_b(s_lo, bias_of(e)); }
+  __device__ __forceinline__ float key_hi(double s_hi, int e) const { return key_hi_b(s_hi, bias_of(e)); }
   // The same ends for a refined (fp64) score, tight: the fp64 definition itself, widened by
   // one ulp of p for its at most one-ulp departure from monotonicity.
   __device__ __forceinline__ float key_lo_ref(double s_lo, int e) const {
@@ -476,16 +481,18 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
   // 1. lower bounds (the estimates and their error bounds stay in registers for step 3)
   uint32_t u[EPL];
   double sh_r[EPL], d_r[EPL];
+  float b_r[EPL];  // the experts' biases, loaded once
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
     sh_r[i] = (e < E) ? srow[e] : 0.0;
     d_r[i] = (e < E) ? __dadd_ru(__dmul_ru(cdx, nw(e)), delta_abs) : 0.0;
+    b_r[i] = (e < E) ? kf.bias_of(e) : 0.0f;
   }
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
-    u[i] = (e < E) ? ordered(kf.key_lo(__dadd_rd(sh_r[i], -d_r[i]), e)) : 0u;
+    u[i] = (e < E) ? ordered(kf.key_lo_b(__dadd_rd(sh_r[i], -d_r[i]), b_r[i])) : 0u;
   }
   // 2. Lk: each lane sorts its lower bounds in descending order; each of k rounds takes the
   //    warp's largest head and shifts that lane's list by one (0 marks an empty slot)
@@ -517,7 +524,7 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
-    hi_r[i] = (e < E) ? kf.key_hi(__dadd_ru(sh_r[i], d_r[i]), e) : 0.f;
+    hi_r[i] = (e < E) ? kf.key_hi_b(__dadd_ru(sh_r[i], d_r[i]), b_r[i]) : 0.f;
     cand_r[i] = (e < E) && ordered(hi_r[i]) >= lk;
   }
 #pragma unroll
@@ -527,9 +534,9 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
     const int pos = cn + __popc(m & ((1u << lane) - 1u));
     if (cand_r[i] && pos < 32) {
       C.e[pos] = e;
-      C.lo[pos] = kf.key_lo(__dadd_rd(sh_r[i], -d_r[i]), e);
+      C.lo[pos] = kf.key_lo_b(__dadd_rd(sh_r[i], -d_r[i]), b_r[i]);
       C.hi[pos] = hi_r[i];
-      C.mid[pos] = kf.key(sh_r[i], e);
+      C.mid[pos] = kf.key_b(sh_r[i], b_r[i]);
       if (SIG) C.p[pos] = kf.score(sh_r[i]);
     }
     cn += __popc(m);
