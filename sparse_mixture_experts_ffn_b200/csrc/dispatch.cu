@@ -212,7 +212,9 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st) {
   cudaError_t e;
   int launches = 0;
   if (P <= kSmallDispatch) {
-    e = launch_pdl(dispatch_small_kernel, dim3(1), dim3(1024), 0, st, sa, a.idx, a.w, a.k, a.counts,
+    // tiny batches: 16 warps (shorter block barriers; the scans hold two groups a thread)
+    const unsigned nthr = (P <= 64 && a.E + 2 <= 1024) ? 512 : 1024;
+    e = launch_pdl(dispatch_small_kernel, dim3(1), dim3(nthr), 0, st, sa, a.idx, a.w, a.k, a.counts,
                    a.counts_user, a.perm, a.inv_perm, a.row_w, a.row_tok, a.perm_user, a.ctrl);
     if (e != cudaSuccess) return e;
     launches = 1;

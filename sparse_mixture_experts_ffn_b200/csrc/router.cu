@@ -548,19 +548,20 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
   const int my_e = mine ? C.e[lane] : 0;
   float my_lo = mine ? C.lo[lane] : 0.f, my_hi = mine ? C.hi[lane] : 0.f, my_mid = mine ? C.mid[lane] : 0.f;
   float my_p = (SIG && mine) ? C.p[lane] : 0.f;
-  auto classify_mine = [&]() -> int {
+  // (the whole warp runs it: lane j's candidate reaches the others by shuffles; cn <= 32)
+  auto classify = [&]() -> int {
     int cp = 0, cc = 0;
 #pragma unroll 4
     for (int j = 0; j < cn; ++j) {
-      const int f = C.e[j];
-      const float hf = C.hi[j], lf = C.lo[j];
+      const int f = __shfl_sync(0xffffffffu, my_e, j);
+      const float hf = __shfl_sync(0xffffffffu, my_hi, j), lf = __shfl_sync(0xffffffffu, my_lo, j);
       const bool other = j != lane;
       cp += other && ((hf > my_lo) || (hf == my_lo && f < my_e));
       cc += other && ((lf > my_hi) || (lf == my_hi && f < my_e));
     }
-    return (cp < k) ? ST_IN : (cc >= k ? ST_OUT : ST_UNDECIDED);
+    return !mine ? ST_OUT : (cp < k) ? ST_IN : (cc >= k ? ST_OUT : ST_UNDECIDED);
   };
-  int st = mine ? classify_mine() : ST_OUT;
+  int st = classify();
   // 5. fp64 recompute of the undecided candidates
   int n_ref = 0;
   if (refine_f64) {
@@ -584,7 +585,7 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
         ++n_ref;
       }
       __syncwarp();
-      st = mine ? classify_mine() : ST_OUT;
+      st = classify();
     }
   }
   if (__any_sync(0xffffffffu, st == ST_UNDECIDED && my_lo != my_hi)) {
