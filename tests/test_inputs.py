@@ -55,6 +55,25 @@ def test_bench_algorithmic_bytes_closed_form():
     assert b["gate_up_bytes"] == 2 * (32 * 2 * I * H + 2 * Is * H) + 2 * (T * k * H + T * H + T * k * I + T * Is)
 
 
+def test_bench_roofline_of_the_one_gemm_launch():
+    """With 16-token tiles (decode) the dominant kernel is the one launch of both GEMMs: its
+    roofline counts both GEMMs' bytes and FLOPs; the long prefill's is the gate/up GEMM's."""
+    import bench
+    peaks = dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+    d4, p16 = inputs.CONFIGS["decode_t4"], inputs.CONFIGS["prefill_t16384_skew"]
+    assert bench.gemms_in_one_launch(d4, False) and bench.gemms_in_one_launch(inputs.CONFIGS["decode_t128"], False)
+    assert not bench.gemms_in_one_launch(d4, True)  # FP8 weights: two launches
+    assert not bench.gemms_in_one_launch(p16, False) and not bench.gemms_in_one_launch(inputs.CONFIGS["prefill_t4096"], False)
+    counts = np.zeros(d4.E, np.int64)
+    counts[:32] = 1
+    alg = bench.algorithmic(d4, counts)
+    r = bench.roofline(alg, peaks, 0.16, False, "decode_t4", fused=True)
+    assert r["bound"] == "hbm" and r["algorithmic_bytes"] == alg["gate_up_bytes"] + alg["down_bytes"]
+    assert abs(r["achieved"] - (alg["gate_up_bytes"] + alg["down_bytes"]) / 0.16e-3 / 1e9) < 1e-6
+    r2 = bench.roofline(alg, peaks, 0.12, False, "decode_t4", fused=False)
+    assert r2["algorithmic_bytes"] == alg["gate_up_bytes"]
+
+
 def test_bench_traffic_ratio_follows_its_source(tmp_path, monkeypatch):
     """roofline.traffic comes from a `traffic-ratio` line of a committed ncu summary, scaled
     to the launch's algorithmic bytes, and is null once the kernel's code no longer matches
