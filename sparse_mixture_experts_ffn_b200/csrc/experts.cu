@@ -1,9 +1,11 @@
 // experts.cu -- grouped expert GEMMs of the MoE layer.
 //
-// bf16: one persistent, warp-specialised tcgen05 kernel per projection.  Weights are the
-// A operand (128 rows per tile, "swap-AB"), the tokens routed to an expert the B operand
-// (16, 128 or 256 per tile), so an expert's few tokens never pad a 128-row tile; the long
-// prefill's down GEMM runs 256-row x 256-token tiles over pairs of SMs (cta_group::2):
+// bf16: one persistent, warp-specialised tcgen05 kernel per projection (with 16-token tiles,
+// at decode, one launch for both: each down tile starts once its group's gate/up tiles have
+// stored their h rows).  Weights are the A operand (128 rows per tile, "swap-AB"), the tokens
+// routed to an expert the B operand (16, 128 or 256 per tile), so an expert's few tokens never
+// pad a 128-row tile; the long prefill's down GEMM runs 256-row x 256-token tiles over pairs of
+// SMs (cta_group::2):
 //   gate/up:  h[p, i]  = SiLU(x_p . Wg[e, i]) * (x_p . Wu[e, i])     (SiLU(gate) * up)
 //   down:     o[p, c]  = w_p * (h_p . Wd[e, c])                     (routing weight fused)
 // with fp32 accumulators in tensor memory and bf16 outputs.  The shared expert
@@ -13,8 +15,8 @@
 // E4M3 codes plus one E8M0 power-of-two scale per 128 x 128 block.  TMA brings the codes
 // (half the bytes of bf16); eight more warps, in two groups taking alternate k-blocks, turn
 // each 128 x 64 code tile into the bf16 tile the MMA reads, scale applied, in the layout
-// 128-byte-swizzled TMA would have written.  Every decoded weight is exact in bf16, so the GEMM is the bf16 GEMM of the
-// decoded weights, with bf16 tokens as before.
+// 128-byte-swizzled TMA would have written.  Every decoded weight is exact in bf16, so the
+// GEMM is the bf16 GEMM of the decoded weights, with bf16 tokens as before.
 // Sources: llm-atlas page "Step-3.5-Flash", "Champs bruts du config.json":
 // moe_intermediate_size 1280, share_expert_dim 1280, hidden_size 4096, norm_expert_weight.
 //
