@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(ScheduleArgs sa, int k, int 
   }
   if (sa.has_shared && threadIdx.x == 0) cnt[E] = sa.shared_rows;
   __syncthreads();
-  build_schedule(sa, cnt, order, warp_tot, ss);  // the tile descriptors: permute_kernel
+  build_schedule<true>(sa, cnt, order, warp_tot, ss);  // the tile descriptors: permute_kernel
 }
 
 // Placement for large batches: block b owns the assignments of tokens [256b, 256b+256);
@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(32 * kPermWarps) permute_kernel(
 }
 
 // Small batches: histogram, scans, schedule and placement in one block.
+template <bool kMany>
 __global__ void __launch_bounds__(1024) dispatch_small_kernel(
     ScheduleArgs sa, const int32_t* __restrict__ idx, const float* __restrict__ w, int k,
     int32_t* __restrict__ counts, int32_t* __restrict__ counts_user, int32_t* __restrict__ perm,
@@ -158,7 +159,8 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(
   __shared__ SmallDispatchSmem sm;
   pdl_wait();
   pdl_trigger();  // the next kernel may launch now; it waits for this one to finish
-  dispatch_small_block(sa, idx, w, k, counts, counts_user, perm, inv_perm, row_w, row_tok, perm_user, ctrl, sm);
+  dispatch_small_block<kMany>(sa, idx, w, k, counts, counts_user, perm, inv_perm, row_w, row_tok, perm_user, ctrl,
+                              sm);
 }
 
 // x_perm[pos, :] = x[row_tok[pos], :] for the rows of experts [e_lo, e_hi) (all experts,
@@ -214,8 +216,10 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t st) {
   if (P <= kSmallDispatch) {
     // tiny batches: 16 warps (shorter block barriers; the scans hold two groups a thread)
     const unsigned nthr = (P <= 64 && a.E + 2 <= 1024) ? 512 : 1024;
-    e = launch_pdl(dispatch_small_kernel, dim3(1), dim3(nthr), 0, st, sa, a.idx, a.w, a.k, a.counts,
-                   a.counts_user, a.perm, a.inv_perm, a.row_w, a.row_tok, a.perm_user, a.ctrl);
+    // more than 128 assignments: several placing warps, groups ranked without sorting
+    e = launch_pdl(P > 128 ? dispatch_small_kernel<true> : dispatch_small_kernel<false>, dim3(1), dim3(nthr), 0, st,
+                   sa, a.idx, a.w, a.k, a.counts, a.counts_user, a.perm, a.inv_perm, a.row_w, a.row_tok, a.perm_user,
+                   a.ctrl);
     if (e != cudaSuccess) return e;
     launches = 1;
   } else {

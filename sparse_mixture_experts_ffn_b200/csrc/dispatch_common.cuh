@@ -83,6 +83,7 @@ static_assert(sizeof(int) * 2 * 2049 >= sizeof(unsigned long long) * 2048, "room
 // of the reduction).  One block with 2 * blockDim.x >= G + 1 and blockDim.x / 64 a power
 // of two; cnt/order in shared memory, and the offsets and prefixes also kept in ss for the
 // descriptor writers.  Returns the number of groups with rows (they lead the order).
+template <bool kWideRank>
 static __device__ int build_schedule(const ScheduleArgs& a, int* cnt, int* order, unsigned long long* warp_tot,
                                      ScheduleSmem& ss) {
   using u64 = unsigned long long;
@@ -113,30 +114,41 @@ static __device__ int build_schedule(const ScheduleArgs& a, int* cnt, int* order
     }
   }
   // largest group first: order by (count desc, index asc), groups without rows last in
-  // index order.  Keys ~count << 32 | index rank the groups with rows.  Few of them (small
-  // batches): compacted into a list of at most 64 keys, each ranked by blockDim.x / 64
-  // threads that compare it with 64 / (blockDim.x / 64) keys each and add their counts; many:
-  // one ascending bitonic sort of every group's key over the next power of two >= G, padded
-  // with keys above every real one.
+  // index order.  Keys ~count << 32 | index rank the groups with rows.  Up to blockDim.x of
+  // them (kWideRank; else up to 64): compacted into a list, each key ranked by blockDim.x / span threads (span: the
+  // next power of two >= their number, at least 64) that compare it with a share of the
+  // others and add their counts; more: one ascending bitonic sort of every group's key over
+  // the next power of two >= G, padded with keys above every real one.
   auto key_of = [&](int g) -> u64 {
     return (static_cast<u64>(~static_cast<uint32_t>(cnt[g])) << 32) | static_cast<uint32_t>(g);
   };
-  if (nnz <= 64) {
+  if (nnz <= (kWideRank ? static_cast<int>(blockDim.x) : 64)) {
     u64* ckey = reinterpret_cast<u64*>(ss.istart_gu);  // written only after the ranking
     if (z0) ckey[nz_ex] = key_of(i0);
     if (z1) ckey[nz_ex + z0] = key_of(i1);
     if (i0 < G && !z0) order[nnz + (i0 - nz_ex)] = i0;
     if (i1 < G && !z1) order[nnz + (i1 - nz_ex - z0)] = i1;
     __syncthreads();
-    const int parts = static_cast<int>(blockDim.x >> 6), per = 64 / parts;
+    // span: a power of two >= nnz (at least 64); parts = blockDim / span threads per key
+    // (blockDim.x is a power of two), each comparing its key with ceil(nnz / parts) others
+    int span = 64;
+    while (span < nnz) span <<= 1;
+    const int parts = static_cast<int>(blockDim.x) / span, per = (nnz + parts - 1) / parts;
     const int slot = static_cast<int>(threadIdx.x) / parts, part = static_cast<int>(threadIdx.x) - slot * parts;
     int r = 0;
     u64 kg = 0;
     if (slot < nnz) {
       kg = ckey[slot];
-      for (int q = 0; q < per; ++q) {
-        const int h = part * per + q;
-        r += (h < nnz && ckey[h] < kg) ? 1 : 0;
+      if (kWideRank) {
+        const int h1 = min(nnz, (part + 1) * per);
+#pragma unroll 4
+        for (int h = part * per; h < h1; ++h) r += (ckey[h] < kg) ? 1 : 0;
+      } else {  // at most 64 keys: a fixed share of 64 / parts slots each
+        const int per64 = 64 / parts;
+        for (int q = 0; q < per64; ++q) {
+          const int h = part * per64 + q;
+          r += (h < nnz && ckey[h] < kg) ? 1 : 0;
+        }
       }
     }
     for (int o = parts >> 1; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
@@ -339,6 +351,9 @@ struct SmallDispatchSmem {
 
 // The whole dispatch of a small batch by one block (2 * blockDim.x >= G + 1): histogram,
 // counts, offsets, the tile schedule and descriptors, then the stable placement (one warp).
+// kMany (more than 128 assignments): several warps place the assignments, and up to
+// blockDim.x groups with rows are ranked without sorting.
+template <bool kMany>
 static __device__ void dispatch_small_block(const ScheduleArgs& sa, const int32_t* __restrict__ idx,
                                             const float* __restrict__ w, int k, int32_t* __restrict__ counts,
                                             int32_t* __restrict__ counts_user, int32_t* __restrict__ perm,
@@ -369,7 +384,7 @@ static __device__ void dispatch_small_block(const ScheduleArgs& sa, const int32_
   }
   if (sa.has_shared && threadIdx.x == 0) sm.cnt[E] = sa.shared_rows;
   __syncthreads();
-  const int nnz = build_schedule(sa, sm.cnt, sm.order, sm.warp_tot, sm.sched);
+  const int nnz = build_schedule<kMany>(sa, sm.cnt, sm.order, sm.warp_tot, sm.sched);
   __syncthreads();
   // few groups with rows: a warp per group slot; many: items spread evenly over the threads
   if (nnz <= 64)
@@ -379,9 +394,43 @@ static __device__ void dispatch_small_block(const ScheduleArgs& sa, const int32_
                       blockDim.x);
   for (int e = threadIdx.x; e < E; e += blockDim.x) sm.base[e] = sm.sched.off[e];
   __syncthreads();
-  if (threadIdx.x < 32)
-    place_assignments(idx, w, 0, P, k, E, sm.base, perm, inv_perm, row_w, row_tok, perm_user, true, e_first,
-                      w_first);
+  if (!kMany) {
+    if (threadIdx.x < 32)
+      place_assignments(idx, w, 0, P, k, E, sm.base, perm, inv_perm, row_w, row_tok, perm_user, true, e_first,
+                        w_first);
+    return;
+  }
+  // larger batches: W warps place consecutive ranges of the assignments, each from its own
+  // per-expert bases (the experts' offsets plus the counts of the earlier ranges), in the
+  // schedule tables' shared memory, free by now
+  constexpr int kScratch = static_cast<int>(sizeof(ScheduleSmem) / sizeof(int));
+  const int W = min(static_cast<int>(blockDim.x >> 5), min(8, kScratch / E));
+  int* wb = reinterpret_cast<int*>(&sm.sched);  // [W][E]: counts, then bases
+  const int64_t per = ((P + W - 1) / W + 31) / 32 * 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < W * E; i += blockDim.x) wb[i] = 0;
+  __syncthreads();
+  if (warp < W) {
+    const int64_t a0 = min64(warp * per, P), a1 = min64(a0 + per, P);
+    for (int64_t a = a0 + lane; a < a1; a += 32) {
+      const int e = idx[a];
+      if (e >= 0 && e < E) atomicAdd(&wb[warp * E + e], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = sm.base[e];
+    for (int q = 0; q < W; ++q) {
+      const int c = wb[q * E + e];
+      wb[q * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  if (warp < W) {
+    const int64_t a0 = min64(warp * per, P), a1 = min64(a0 + per, P);
+    place_assignments(idx, w, a0, a1, k, E, wb + warp * E, perm, inv_perm, row_w, row_tok, perm_user);
+  }
 }
 
 // The schedule arguments of a dispatch (tile shapes of both grouped GEMMs).
