@@ -1013,6 +1013,8 @@ struct RouterTcParams {
   double* scores;    // [T, E]
   // split only
   int chunks, chunk_slices;
+  int last_block_reduces;  // 1: the last block of each tile adds the partials (T <= 32); 0:
+                           // router_reduce_kernel does, after this launch
   const __nv_bfloat16* x;
   const __nv_bfloat16* Wr;
   float* part;       // [slices, T, E] fp32 slice partials
@@ -1225,11 +1227,13 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
         }
       }
       // the last block of this (m, n) tile adds the partials of every chunk (below)
-      fence_acq_rel_gpu();
-      named_bar_sync(1, 128);
-      if (warp == 2 && lane == 0) {
-        const unsigned int done = atomicAdd(p.tile_done + blockIdx.x, 1u);
-        *last_flag = (done == static_cast<unsigned int>(p.chunks - 1)) ? 1 : 0;
+      if (p.last_block_reduces) {
+        fence_acq_rel_gpu();
+        named_bar_sync(1, 128);
+        if (warp == 2 && lane == 0) {
+          const unsigned int done = atomicAdd(p.tile_done + blockIdx.x, 1u);
+          *last_flag = (done == static_cast<unsigned int>(p.chunks - 1)) ? 1 : 0;
+        }
       }
     }
   }
@@ -1298,6 +1302,45 @@ __global__ void __launch_bounds__(192, 1) router_gemm_tc_kernel(const __grid_con
   }
 }
 
+// The reduction-split router's sums for batches of 33..128 tokens, whose tiles' last blocks
+// would each have thousands of scores to add: one thread per score (the fp64 sum of its
+// slices' fp32 partials in slice order, as the last block forms it: the unsplit kernel's
+// result bit for bit) or norm bound (the fp64 sum of the chunks' sums of squares in chunk
+// order), over the whole grid.
+__global__ void __launch_bounds__(256) router_reduce_kernel(const __grid_constant__ RouterTcParams p) {
+  pdl_wait();
+  const int64_t ns = p.T * p.E, nx = p.T, nw = p.w_given ? 0 : p.E;
+  const int n_sl_all = (p.H / kTileK + kRtSliceSteps - 1) / kRtSliceSteps;
+  for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < ns + nx + nw;
+       j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (j < ns) {
+      const float* src = p.part + j;  // part[sl][t][e], j = t E + e
+      double acc = 0.0;
+      int b = 0;
+      for (; b + 16 <= n_sl_all; b += 16) {
+        float v[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) v[q] = __ldcg(src + (b + q) * ns);
+#pragma unroll
+        for (int q = 0; q < 16; ++q) acc += static_cast<double>(v[q]);
+      }
+      for (; b < n_sl_all; ++b) acc += static_cast<double>(__ldcg(src + b * ns));
+      p.scores[j] = acc;
+    } else {
+      const bool is_x = j < ns + nx;
+      const int64_t i = is_x ? j - ns : j - ns - nx;
+      const double* src = is_x ? p.xss + i : p.wss + i;
+      const int64_t st = is_x ? p.T : static_cast<int64_t>(p.E);
+      double ss = 0.0;
+      for (int z = 0; z < p.chunks; ++z) ss += __ldcg(src + z * st);
+      if (is_x)
+        p.xnorm[i] = norm_ub_from_sumsq(ss, p.Hx);
+      else
+        p.wnorm[i] = norm_ub_from_sumsq(ss, p.H);
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------------
 // host launchers
 // ---------------------------------------------------------------------------------------
@@ -1338,10 +1381,11 @@ int router_slice_len(int /*H*/) { return kRtSliceSteps * kTileK; }
 // Reduction chunks of the tensor-core router: 1 when the (m, n) tiles fill the GPU or the
 // batch is too large for one block per tile to add the partials quickly, else the fewest
 // (at most 16, at least one slice each) that bring the blocks to one per SM.
-constexpr int64_t kRtSplitMaxTokens = 32;
+constexpr int64_t kRtSplitMaxTokens = 32;        // the tiles' last blocks add the partials
+constexpr int64_t kRtSplitReduceMaxTokens = 128; // router_reduce_kernel adds them
 static_assert(kRtSplitMaxTokens + kRtExperts <= 192, "one thread per norm bound in a tile's last block");
 static int router_chunks(int64_t T, int E, int H) {
-  if (T > kRtSplitMaxTokens) return 1;
+  if (T > kRtSplitReduceMaxTokens) return 1;
   const int64_t tiles = ((T + kTileM - 1) / kTileM) * ((E + kRtExperts - 1) / kRtExperts);
   const int n_sl = (H / kTileK + kRtSliceSteps - 1) / kRtSliceSteps;
   int c = 1;
@@ -1503,6 +1547,7 @@ static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
     p.tile_done = a.group_done;
     p.xnorm = a.xnorm;
     p.wnorm = a.wnorm;
+    p.last_block_reduces = a.T <= kRtSplitMaxTokens ? 1 : 0;
   } else {
     const int64_t wrows = a.w32 ? 0 : a.E;  // split fp32 weights come with their norm bounds
     e = launch_pdl(row_norm_ub_kernel<bf16>, dim3(static_cast<unsigned>(((a.T + wrows) * 32 + 255) / 256)),
@@ -1515,6 +1560,13 @@ static cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t st) {
                       static_cast<unsigned>(chunks)),
                  dim3(192), static_cast<size_t>(kRtSmem), st, p);
   if (e != cudaSuccess) return e;
+  if (chunks > 1 && !p.last_block_reduces) {
+    const int64_t jobs = a.T * a.E + a.T + a.E;
+    e = launch_pdl(router_reduce_kernel, dim3(static_cast<unsigned>(std::min<int64_t>((jobs + 255) / 256, 148 * 4))),
+                   dim3(256), 0, st, p);
+    if (e != cudaSuccess) return e;
+    ++launches;
+  }
   const float* Wf = static_cast<const float*>(a.Wr);
   if (a.w32)  // the recomputations read the fp32 weights themselves
     e = a.sigmoid ? launch_select_epl<float, true>(a, Wf, coef, Kg, st)

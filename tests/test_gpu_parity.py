@@ -53,6 +53,9 @@ SMALL = [
     # 16-token tiles (both GEMMs in one launch) without a shared expert, the gate/up
     # reduction split: fewer items than blocks, so blocks start on down tiles and wait
     dict(T=5, H=256, E=32, top_k=4, I=256, I_shared=0),
+    # router reduction split over 4 chunks for 100 tokens: the partials added by a separate
+    # grid-wide kernel rather than by each tile's last block
+    dict(T=100, H=1024, E=96, top_k=6, I=128, I_shared=128),
     # 256-token tiles (about 350 tokens per expert: one full and one ragged tile each)
     dict(T=700, H=256, E=8, top_k=4, I=256, I_shared=128),
     # 256 x 256 tiles over pairs of SMs (widths multiples of 256): ragged token tiles, a
@@ -120,6 +123,7 @@ def test_sigmoid_router(sz, with_bias):
 FP32_ROUTER_CASES = [
     dict(T=257, H=256, E=32, top_k=4, I=128, I_shared=128),    # unsplit tensor-core scores
     dict(T=3, H=2176, E=200, top_k=8, I=128, I_shared=128),    # reduction split over blocks
+    dict(T=60, H=1024, E=96, top_k=6, I=128, I_shared=128),    # split, grid-wide reduce kernel
 ]
 
 
