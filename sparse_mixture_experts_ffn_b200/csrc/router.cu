@@ -521,6 +521,7 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
   int cn = 0;
   bool cand_r[EPL];
   float hi_r[EPL];
+  unsigned m_r[EPL];
 #pragma unroll
   for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
@@ -528,10 +529,11 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
     cand_r[i] = (e < E) && ordered(hi_r[i]) >= lk;
   }
 #pragma unroll
+  for (int i = 0; i < EPL; ++i) m_r[i] = __ballot_sync(0xffffffffu, cand_r[i]);  // independent ballots
+#pragma unroll
   for (int i = 0; i < EPL; ++i) {
     const int e = lane + 32 * i;
-    const unsigned m = __ballot_sync(0xffffffffu, cand_r[i]);
-    const int pos = cn + __popc(m & ((1u << lane) - 1u));
+    const int pos = cn + __popc(m_r[i] & ((1u << lane) - 1u));
     if (cand_r[i] && pos < 32) {
       C.e[pos] = e;
       C.lo[pos] = kf.key_lo_b(__dadd_rd(sh_r[i], -d_r[i]), b_r[i]);
@@ -539,7 +541,7 @@ __device__ __forceinline__ bool select_token(const double* __restrict__ srow, do
       C.mid[pos] = kf.key_b(sh_r[i], b_r[i]);
       if (SIG) C.p[pos] = kf.score(sh_r[i]);
     }
-    cn += __popc(m);
+    cn += __popc(m_r[i]);
   }
   if (cn > 32) return false;
   __syncwarp();
